@@ -1,0 +1,384 @@
+"""Pins for the fp64 oracle: each test checks the oracle against something other than
+itself -- hand-derived values, closed forms, brute force on tiny inputs, textbook
+special cases and invariants the pages state.  CPU only, seconds.
+
+Page titles cited: "Pruning LLMs with Thanos" (THANOS) and "Weight Pruning in Large
+Language Models: How SparseGPT, Wanda, and Semi-Structured 2:4 Sparsity ..." (BLOG).
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand_problem(seed, c=6, b=10, n=24, outlier=True):
+    rng = np.random.default_rng(seed)
+    Xt = rng.normal(size=(n, b))
+    if outlier:
+        Xt[:, rng.integers(b)] *= 7.0
+    W = rng.normal(scale=0.5, size=(c, b))
+    return W, Xt
+
+
+def _brute_gram(Xt):
+    n, b = Xt.shape
+    G = np.zeros((b, b))
+    for i in range(b):
+        for j in range(b):
+            s = 0.0
+            for t in range(n):
+                s += Xt[t, i] * Xt[t, j]
+            G[i, j] = s
+    return G
+
+
+# --------------------------------------------------------------------------- statistics
+
+def test_gram_matches_triple_loop():
+    _, Xt = _rand_problem(0, b=5, n=7)
+    assert np.allclose(oracle.gram(Xt), _brute_gram(Xt), rtol=1e-13, atol=1e-13)
+    assert np.allclose(oracle.hessian(Xt), 2.0 * _brute_gram(Xt), rtol=1e-13, atol=1e-13)
+
+
+def test_damping_is_relative_to_mean_undamped_diagonal():
+    H = np.diag([1.0, 2.0, 3.0, 6.0])
+    Hd, lam = oracle.damp_hessian(H, 0.5)
+    assert lam == pytest.approx(0.5 * 3.0)
+    assert np.allclose(np.diag(Hd), [2.5, 3.5, 4.5, 7.5])
+
+
+def test_inverse_cholesky_upper_is_upper_and_factors_inverse():
+    W, Xt = _rand_problem(1)
+    Hd, _ = oracle.damp_hessian(oracle.hessian(Xt), 0.01)
+    U = oracle.inverse_cholesky_upper(Hd)
+    assert np.allclose(np.tril(U, -1), 0.0)
+    assert np.all(np.diag(U) > 0)
+    assert np.allclose(U.T @ U @ Hd, np.eye(Hd.shape[0]), atol=1e-10)
+    # trailing principal inverses come from U's trailing block (what the factored mode relies on)
+    for j in range(Hd.shape[0]):
+        assert np.allclose(U[j:, j:].T @ U[j:, j:], np.linalg.inv(Hd[j:, j:]), rtol=1e-9, atol=1e-12)
+
+
+# --------------------------------------------------------------------------- single deletion (I1)
+
+def test_single_deletion_error_closed_form():
+    """THANOS 'Why magnitude alone misses important weights': deleting W_kq with the rest
+    frozen costs W_kq^2 ||X_q||^2; with H it is W_kq^2 H_qq."""
+    W, Xt = _rand_problem(2)
+    G = oracle.gram(Xt)
+    H = oracle.hessian(Xt)
+    c, b = W.shape
+    for k in range(c):
+        for q in range(b):
+            Wd = W.copy()
+            Wd[k, q] = 0.0
+            direct = float(np.sum(((Wd - W) @ Xt.T) ** 2))
+            closed = W[k, q] ** 2 * np.sum(Xt[:, q] ** 2)
+            assert oracle.recon_loss(W, Wd, G) == pytest.approx(closed, rel=1e-12)
+            assert direct == pytest.approx(closed, rel=1e-12)
+            d = np.zeros(b)
+            d[q] = -W[k, q]
+            assert d @ H @ d == pytest.approx(W[k, q] ** 2 * H[q, q], rel=1e-12)
+    # Wanda's score squared orders weights exactly like the deletion error
+    S = oracle.wanda_scores(W, np.diag(G))
+    assert np.allclose(S ** 2, W ** 2 * np.diag(G)[None, :], rtol=1e-12)
+
+
+# --------------------------------------------------------------------------- row decomposition (I2)
+
+def test_loss_decomposes_over_rows():
+    W, Xt = _rand_problem(3, c=8)
+    r = oracle.prune_layer(W, Xt=Xt, sparsity=0.5, block=4)
+    direct = float(np.sum(((r["W"] - W) @ Xt.T) ** 2))
+    per_row = oracle.row_losses(W, r["W"], oracle.gram(Xt))
+    assert r["loss"] == pytest.approx(direct, rel=1e-10)
+    assert per_row.sum() == pytest.approx(direct, rel=1e-10)
+    for k in range(W.shape[0]):
+        assert per_row[k] == pytest.approx(float(np.sum(((r["W"][k] - W[k]) @ Xt.T) ** 2)), rel=1e-10)
+
+
+# --------------------------------------------------------------------------- joint update (I3, I13)
+
+def _lstsq_row(w, Xt, lam, j, Q_abs):
+    """min over delta supported on [j, b) with delta_Q = -w_Q of
+    ||sqrt2 X^T delta||^2 + lam ||delta||^2, solved as a least-squares problem."""
+    n, b = Xt.shape
+    A = np.arange(j, b)
+    F = np.array([q for q in A if q not in set(Q_abs)], dtype=int)
+    M = np.vstack([math.sqrt(2.0) * Xt, math.sqrt(lam) * np.eye(b)])
+    dQ = -w[Q_abs]
+    rhs = -(M[:, Q_abs] @ dQ)
+    dF = np.linalg.lstsq(M[:, F], rhs, rcond=None)[0] if F.size else np.zeros(0)
+    out = w.copy()
+    out[Q_abs] = 0.0
+    out[F] += dF
+    return out
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_row_update_equals_constrained_least_squares(seed):
+    W, Xt = _rand_problem(10 + seed, c=3, b=9, n=20)
+    damp = 0.05
+    H = oracle.hessian(Xt)
+    Hd, lam = oracle.damp_hessian(H, damp)
+    rng = np.random.default_rng(seed)
+    for j in (0, 2, 5):
+        K = oracle.active_inverse(Hd, j)
+        for size in range(1, 4):
+            Q_rel = np.sort(rng.choice(min(4, 9 - j), size=min(size, 9 - j), replace=False))
+            w = W[0]
+            got = w.copy()
+            got[j:] = oracle.thanos_row_update(w[j:], Q_rel, K[Q_rel, :])
+            want = _lstsq_row(w, Xt, lam, j, Q_rel + j)
+            assert np.allclose(got, want, rtol=1e-9, atol=1e-11)
+            assert np.all(got[Q_rel + j] == 0.0)
+            assert np.array_equal(got[:j], w[:j])
+
+
+def test_single_block_is_optimal_over_every_mask_exhaustive():
+    """c=1, b=6, one block: for every 3-of-6 mask, the joint update reaches the least-squares
+    optimum of the damped objective, so no other choice of kept values does better."""
+    W, Xt = _rand_problem(20, c=1, b=6, n=15)
+    H = oracle.hessian(Xt)
+    Hd, lam = oracle.damp_hessian(H, 0.01)
+    K = oracle.active_inverse(Hd, 0)
+    w = W[0]
+    for Q in itertools.combinations(range(6), 3):
+        Q = np.array(Q)
+        got = oracle.thanos_row_update(w, Q, K[Q, :])
+        want = _lstsq_row(w, Xt, lam, 0, Q)
+        assert np.allclose(got, want, rtol=1e-9, atol=1e-11)
+        d = got - w
+        rng = np.random.default_rng(0)
+        for _ in range(5):       # random feasible perturbations never lower the damped loss
+            p = rng.normal(size=6) * 1e-3
+            p[Q] = 0.0
+            assert (d + p) @ Hd @ (d + p) >= d @ Hd @ d - 1e-12
+
+
+# --------------------------------------------------------------------------- hand-derived goldens
+
+def _golden_cases():
+    with open(os.path.join(GOLDEN, "obs_hand_examples.json")) as f:
+        return json.load(f)["cases"]
+
+
+@pytest.mark.parametrize("case", _golden_cases(), ids=lambda c: c["name"])
+def test_hand_derived_examples(case):
+    s = case.get("sparsity")
+    if s is None:
+        s = case["sparsity_num"] / case["sparsity_den"]
+    r = oracle.prune_layer(np.array(case["W"]), H=np.array(case["H"], float), sparsity=s,
+                           block=case["block"], damp=0.0, method=case["method"])
+    assert np.allclose(r["W"], case["W_hat"], rtol=0, atol=1e-12)
+    assert np.array_equal(r["mask"].astype(int), np.array(case["mask"]))
+    assert r["loss"] == pytest.approx(case["loss"], rel=1e-12)
+    r2 = oracle.prune_layer(np.array(case["W"]), H=np.array(case["H"], float), sparsity=s,
+                            block=case["block"], damp=0.0, method=case["method"], mode="definitional")
+    assert np.allclose(r2["W"], case["W_hat"], rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------- invariants (I4, I5)
+
+@pytest.mark.parametrize("method", ["thanos", "sparsegpt"])
+@pytest.mark.parametrize("c,b,B", [(7, 24, 8), (5, 30, 8), (9, 17, 5), (1, 12, 12)])
+def test_unstructured_budget_and_exact_zeros(method, c, b, B):
+    rng = np.random.default_rng(c * b)
+    Xt = rng.normal(size=(3 * b, b))
+    W = rng.normal(size=(c, b))
+    for s in (0.0, 0.3, 0.5, 0.9):
+        r = oracle.prune_layer(W, Xt=Xt, sparsity=s, block=B, method=method)
+        assert np.all(r["W"][r["mask"]] == 0.0)
+        if method == "thanos":
+            assert int(r["mask"].sum()) == math.floor(s * c * b)
+        else:
+            want = sum(math.floor(s * c * (min(j + B, b) - j)) for j in range(0, b, B))
+            assert int(r["mask"].sum()) == want
+
+
+@pytest.mark.parametrize("method", ["thanos", "sparsegpt"])
+@pytest.mark.parametrize("nm", [(2, 4), (4, 8), (1, 4)])
+def test_nm_groups_keep_exactly_n(method, nm):
+    n_keep, m = nm
+    rng = np.random.default_rng(5)
+    b = 32
+    Xt = rng.normal(size=(80, b))
+    W = rng.normal(size=(6, b))
+    r = oracle.prune_layer(W, Xt=Xt, pattern="nm", nm=nm, block=16, method=method)
+    groups = r["mask"].reshape(6, b // m, m)
+    assert np.all(groups.sum(axis=2) == m - n_keep)
+    assert np.all(r["W"][r["mask"]] == 0.0)
+
+
+def test_nm_ties_prune_lower_column_first():
+    S = np.array([[1.0, 1.0, 1.0, 1.0, 3.0, 2.0, 2.0, 1.0]])
+    mask, _ = oracle.nm_mask(S, 2, 4)
+    assert mask.astype(int).tolist() == [[1, 1, 0, 0, 0, 1, 0, 1]]
+
+
+def test_global_selection_tie_order():
+    S = np.array([[1.0, 0.5, 1.0],
+                  [1.0, 2.0, 1.0]])
+    # order by (score, column, row): (0.5,1,0), (1,0,0), (1,0,1), (1,2,0), (1,2,1), (2,1,1)
+    m, t_last, t_next = oracle.lowest_global(S, 0, 3)
+    assert m.astype(int).tolist() == [[1, 1, 0], [1, 0, 0]]
+    assert (t_last, t_next) == (1.0, 1.0)
+    m, _, _ = oracle.lowest_global(S, 0, 4)
+    assert m.astype(int).tolist() == [[1, 1, 1], [1, 0, 0]]
+
+
+# --------------------------------------------------------------------------- diagonal Hessian (I6)
+
+def test_orthogonal_features_reduce_to_static_wanda_selection():
+    """With X X^T diagonal no update reaches another coordinate, so the dynamic global
+    budget picks exactly the static lowest floor(s c b) Wanda scores."""
+    rng = np.random.default_rng(7)
+    c, b, n = 9, 20, 40
+    Qo, _ = np.linalg.qr(rng.normal(size=(n, b)))
+    d = rng.uniform(0.5, 3.0, size=b)
+    Xt = Qo * d[None, :]                      # columns orthogonal -> X X^T = diag(d^2)
+    W = rng.normal(size=(c, b))
+    r = oracle.prune_layer(W, Xt=Xt, sparsity=0.5, block=4)
+    score = np.abs(W) * d[None, :]
+    k = math.floor(0.5 * c * b)
+    idx = np.argsort(score.ravel(), kind="stable")[:k]
+    static = np.zeros(c * b, bool)
+    static[idx] = True
+    assert np.array_equal(r["mask"], static.reshape(c, b))
+    assert np.allclose(r["W"], np.where(r["mask"], 0.0, W), atol=1e-12)
+
+
+# --------------------------------------------------------------------------- padding (I7)
+
+def test_identity_padding_leaves_updates_unchanged():
+    """THANOS 'Making irregular row masks batchable': padded u (zeros), R (zero rows) and
+    R-hat (identity fill) give the same updates as the unpadded per-row solves."""
+    W, Xt = _rand_problem(30, c=5, b=12, n=30)
+    Hd, _ = oracle.damp_hessian(oracle.hessian(Xt), 0.01)
+    K = oracle.active_inverse(Hd, 0)
+    rng = np.random.default_rng(1)
+    Qs = [np.sort(rng.choice(6, size=s, replace=False)) for s in (0, 1, 3, 2, 5)]
+    smax = max(len(q) for q in Qs)
+    U_pad = np.zeros((5, smax))
+    R_pad = np.zeros((5, smax, 12))
+    Rh_pad = np.tile(np.eye(smax), (5, 1, 1))
+    for k, Q in enumerate(Qs):
+        s = len(Q)
+        U_pad[k, :s] = W[k, Q]
+        R_pad[k, :s] = K[Q, :]
+        Rh_pad[k, :s, :s] = K[np.ix_(Q, Q)]
+    Z = np.linalg.solve(Rh_pad, U_pad[..., None])[..., 0]
+    D_pad = -np.einsum("ks,ksa->ka", Z, R_pad)
+    for k, Q in enumerate(Qs):
+        got = oracle.thanos_row_update(W[k], Q, K[Q, :])
+        want = W[k] + D_pad[k]
+        want[Q] = 0.0
+        assert np.allclose(got, want, atol=1e-12)
+
+
+# --------------------------------------------------------------------------- sequential OBS (I8)
+
+@pytest.mark.parametrize("seed", range(3))
+def test_joint_update_equals_correctly_conditioned_sequential_obs(seed):
+    """THANOS 'The scaling problem...': sequential OBS with the inverse downdated after each
+    removal (other coordinates stay free) represents the same fixed constraint set."""
+    W, Xt = _rand_problem(40 + seed, c=1, b=10, n=25)
+    Hd, _ = oracle.damp_hessian(oracle.hessian(Xt), 0.02)
+    K = oracle.active_inverse(Hd, 0)
+    Q = np.array([1, 4, 5, 8])
+    joint = oracle.thanos_row_update(W[0], Q, K[Q, :])
+    rng = np.random.default_rng(seed)
+    for _ in range(3):
+        w = W[0].copy()
+        Kc = K.copy()
+        for q in rng.permutation(Q):
+            w = w - (w[q] / Kc[q, q]) * Kc[q, :]
+            Kc = Kc - np.outer(Kc[:, q], Kc[q, :]) / Kc[q, q]
+        w[Q] = 0.0
+        assert np.allclose(w, joint, atol=1e-10)
+
+
+# --------------------------------------------------------------------------- loss ordering (I9)
+
+def test_joint_update_is_below_every_other_update_for_the_same_mask():
+    """With one block and a fixed mask the joint update is the exact minimiser of the damped
+    objective (THANOS 'Contribution one'), so the column-sequential update and the no-update
+    (Wanda-style) result -- both feasible for the same mask -- can only be worse.  Between
+    those two there is no fixed order: each sequential step is measured from the already
+    compensated weights, not from W."""
+    W, Xt = _rand_problem(50, c=6, b=16, n=40)
+    H = oracle.hessian(Xt)
+    Hd, _ = oracle.damp_hessian(H, 0.01)
+    U = oracle.inverse_cholesky_upper(Hd)
+    r = oracle.prune_layer(W, H=H, sparsity=0.5, block=16)        # one block
+    mask = r["mask"]
+    Ws = W.copy()
+    oracle.sparsegpt_block(Ws, 0, 16, mask, U=U)
+    Wz = np.where(mask, 0.0, W)
+
+    def damped(Wx):
+        D = Wx - W
+        return np.einsum("kq,kq->k", D @ Hd, D)
+    assert np.all(damped(r["W"]) <= damped(Ws) + 1e-12)
+    assert np.all(damped(r["W"]) <= damped(Wz) + 1e-12)
+    assert np.any(damped(r["W"]) < damped(Ws) - 1e-6)
+
+
+# --------------------------------------------------------------------------- scale (I10)
+
+@pytest.mark.parametrize("method,pattern", [("thanos", "unstructured"), ("thanos", "nm"),
+                                            ("sparsegpt", "unstructured"), ("sparsegpt", "nm")])
+def test_scaling_activations_leaves_result_unchanged(method, pattern):
+    W, Xt = _rand_problem(60, c=6, b=16, n=40)
+    a = oracle.prune_layer(W, Xt=Xt, block=8, method=method, pattern=pattern)
+    b_ = oracle.prune_layer(W, Xt=3.7 * Xt, block=8, method=method, pattern=pattern)
+    assert np.array_equal(a["mask"], b_["mask"])
+    assert np.allclose(a["W"], b_["W"], rtol=1e-9, atol=1e-12)
+
+
+# --------------------------------------------------------------------------- factored form (I11)
+
+@pytest.mark.parametrize("method,pattern,B", [("thanos", "unstructured", 5), ("thanos", "nm", 8),
+                                              ("sparsegpt", "unstructured", 6), ("sparsegpt", "nm", 4)])
+def test_definitional_and_factored_modes_agree(method, pattern, B):
+    W, Xt = _rand_problem(70, c=7, b=24, n=50)
+    a = oracle.prune_layer(W, Xt=Xt, block=B, method=method, pattern=pattern, mode="factored")
+    d = oracle.prune_layer(W, Xt=Xt, block=B, method=method, pattern=pattern, mode="definitional")
+    assert np.array_equal(a["mask"], d["mask"])
+    assert np.allclose(a["W"], d["W"], rtol=1e-10, atol=1e-12)
+
+
+# --------------------------------------------------------------------------- B = 1 (I12)
+
+def test_thanos_with_unit_block_is_the_sparsegpt_column_update():
+    W, Xt = _rand_problem(80, c=5, b=12, n=30)
+    Hd, _ = oracle.damp_hessian(oracle.hessian(Xt), 0.01)
+    U = oracle.inverse_cholesky_upper(Hd)
+    mask = np.random.default_rng(0).random(W.shape) < 0.5
+    Wt = W.copy()
+    for q in range(12):
+        K_row = oracle.active_inverse(Hd, q)[:1, :]        # the single block row of inv(H_d[q:, q:])
+        for k in range(5):
+            if mask[k, q]:
+                Wt[k, q:] = oracle.thanos_row_update(Wt[k, q:], np.array([0]), K_row)
+    Ws = W.copy()
+    oracle.sparsegpt_block(Ws, 0, 12, mask, U=U)
+    Wd = W.copy()
+    oracle.sparsegpt_block(Wd, 0, 12, mask, Hd=Hd)
+    assert np.allclose(Wt, Ws, atol=1e-11)
+    assert np.allclose(Wd, Ws, atol=1e-11)
+
+
+def test_sparsegpt_uses_conditioned_diagonal():
+    W, Xt = _rand_problem(90, c=3, b=8, n=20)
+    Hd, _ = oracle.damp_hessian(oracle.hessian(Xt), 0.01)
+    U = oracle.inverse_cholesky_upper(Hd)
+    for q in range(8):
+        assert U[q, q] ** 2 == pytest.approx(oracle.conditioned_diag(Hd, q), rel=1e-10)
