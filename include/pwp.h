@@ -1,0 +1,144 @@
+/*
+ * pwp.h -- C ABI of the B200 layer-reconstruction pruning library (libpwp.so).
+ *
+ * One linear layer W (c x b, rows = outputs, columns = input features) and its
+ * calibration activations X (the pages' X is b x n with examples as columns; it
+ * is passed here token-major, [n, b], the PyTorch activation layout) are turned
+ * into a pruned and reconstructed W-hat and a pruning mask, following
+ *   "Pruning LLMs with Thanos" (sections "The layer-reconstruction lens",
+ *   "Contribution one: solve a selected set directly", "Contribution two: keep
+ *   the budget global and the execution local") and, for the column-sequential
+ *   special case, "Weight Pruning in Large Language Models ..." (llms.blog),
+ *   section "SparseGPT: Second-Order Reconstruction at Scale".
+ *
+ * Conventions for every entry point:
+ *   - All pointers named *_dev are device pointers; the caller owns every buffer.
+ *     The library allocates no device or host memory: all scratch comes from the
+ *     caller's workspace `ws` of `ws_bytes` bytes (at least 256-byte aligned).
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream)
+ *     and the call returns without synchronising.
+ *   - Argument errors are detected on the host before anything is enqueued and
+ *     returned synchronously (PWP_EINVAL, PWP_EWORKSPACE).  A CUDA launch error
+ *     returns PWP_ECUDA.
+ *   - Errors found on the device (a non-positive pivot, a wait that ran out, an
+ *     unreachable budget) are written to the caller's device-resident pwp_stats
+ *     (`status`, `status_site`); every later kernel of the same call becomes a
+ *     no-op.  The caller reads `stats_dev` after synchronising the stream.
+ *   - Calls on different streams with different workspaces are independent;
+ *     two calls that share a workspace must be ordered by the caller.
+ */
+#ifndef PWP_H
+#define PWP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PWP_OK = 0,
+    PWP_EINVAL = 1,      /* bad shape, pattern, sparsity, block or dtype */
+    PWP_ENOTSPD = 2,     /* damped Hessian not positive definite (pivot <= 0) */
+    PWP_EWORKSPACE = 3,  /* workspace missing, misaligned or too small */
+    PWP_ECUDA = 4,       /* a CUDA launch or runtime call failed */
+    PWP_ETIMEOUT = 5,    /* a bounded device-side wait gave up */
+    PWP_EBUDGET = 6      /* the unstructured target could not be reached */
+} pwp_status;
+
+typedef enum { PWP_THANOS = 0, PWP_SPARSEGPT = 1 } pwp_method;
+typedef enum { PWP_UNSTRUCTURED = 0, PWP_NM = 1 } pwp_pattern;
+typedef enum { PWP_BF16 = 0, PWP_FP32 = 1 } pwp_dtype;
+
+/* Method configuration ("Thanos - Method of Pruning LLMs", section "Usage":
+ * --prune_method, --sparsity_ratio, --sparsity_type).
+ *   method   : PWP_THANOS (joint row solves, dynamic global budget) or
+ *              PWP_SPARSEGPT (column-sequential OBS, per-block quota).
+ *   pattern  : PWP_UNSTRUCTURED, or PWP_NM with 0 < nm_n < nm_m <= 32 (keep nm_n of
+ *              every nm_m consecutive weights of a row; groups start at column 0).
+ *   sparsity : fraction of weights removed, 0 <= sparsity < 1 (ignored for PWP_NM).
+ *   block    : column block width B, 1 <= B <= 128; for PWP_NM a multiple of nm_m.
+ *   damp     : lambda = damp * mean(diag H) of the undamped H, damp >= 0. */
+typedef struct {
+    int32_t method;
+    int32_t pattern;
+    int32_t nm_n;
+    int32_t nm_m;
+    float sparsity;
+    int32_t block;
+    float damp;
+} pwp_config;
+
+/* Device-resident results of one prune call (the caller allocates it in device
+ * memory and reads it back after the stream is synchronised). */
+typedef struct {
+    int32_t status;          /* pwp_status found on the device, PWP_OK otherwise */
+    int32_t status_site;     /* index of the kernel that first set `status` */
+    int64_t pruned;          /* number of mask entries set (weights removed) */
+    int64_t target;          /* floor(sparsity*c*b) for Thanos unstructured, else the
+                                number of removals the pattern implies */
+    float lambda;            /* damping actually added to the diagonal */
+    int32_t shortfall;       /* 1 if a block wanted more removals than it had weights */
+    int32_t reread_blocks;   /* blocks whose exact threshold needed a second pass */
+    int32_t tie_blocks;      /* blocks whose threshold fell on tied scores */
+    int32_t reserved[4];
+} pwp_stats;
+
+/* Bytes of workspace pwp_prune_layer / pwp_prune_layer_x need for this
+ * configuration and shape.  Returns 0 for an invalid configuration. */
+size_t pwp_workspace_bytes(const pwp_config* cfg, int32_t c, int32_t b);
+
+/* Hessian accumulation, H (b x b fp32, row-major, full symmetric) :=
+ *   beta * H + 2 X X^T     (pages' X = b x n; here X_dev is [n, b] token-major),
+ * "Weight Pruning in Large Language Models ...", section "SparseGPT: Second-Order
+ * Reconstruction at Scale" (H = 2 X X^T; damping is added later by the prune call).
+ * Calling it repeatedly with beta = 1 streams calibration batches into one H.
+ *   X_dev   : [n, b] elements of type xtype (PWP_BF16 or PWP_FP32), row stride b.
+ *   n >= 0, 1 <= b <= 16384, beta in {0, 1}.  H_dev: b*b floats.
+ * Needs no workspace. */
+pwp_status pwp_hessian_accumulate(const void* X_dev, int32_t xtype, int64_t n, int32_t b,
+                                  float* H_dev, int32_t beta, void* stream);
+
+/* Damping and factorisation (the "Cholesky decomposition of H^-1 once per layer"
+ * of the llms.blog SparseGPT section).  On entry H_dev holds the undamped
+ * H = 2XX^T (b x b, row-major; only the upper triangle is read).  On return the
+ * upper triangle of H_dev holds U, upper triangular with (H + lambda I)^-1 = U^T U,
+ * lambda = damp * mean(diag H); the strict lower triangle is left unspecified.
+ * g_diag_dev (b floats) receives diag(H)/2 = ||X_q||^2 before damping.
+ * ws/ws_bytes: scratch of at least pwp_factor_workspace_bytes(b) bytes.
+ * stats_dev receives lambda and a PWP_ENOTSPD status on a non-positive pivot. */
+size_t pwp_factor_workspace_bytes(int32_t b);
+pwp_status pwp_damp_factor(float* H_dev, int32_t b, float damp, float* g_diag_dev,
+                           void* ws, size_t ws_bytes, pwp_stats* stats_dev, void* stream);
+
+/* Prune one layer given its undamped Hessian.
+ *   W_dev     : c x b row-major weights of type wtype (read only).
+ *   H_dev     : undamped H = 2 X X^T (b x b fp32); DESTROYED (holds U on return).
+ *   W_out_dev : c x b fp32, receives W-hat (pruned entries exactly 0.0f).
+ *   mask_dev  : c x b bytes, receives 1 where a weight was removed, else 0.
+ *   1 <= c, 1 <= b <= 16384, c*b < 2^31.
+ * Method: "Pruning LLMs with Thanos", sections "Contribution one" and
+ * "Contribution two" (PWP_THANOS); llms.blog SparseGPT section (PWP_SPARSEGPT). */
+pwp_status pwp_prune_layer(const pwp_config* cfg, const void* W_dev, int32_t wtype,
+                           int32_t c, int32_t b, float* H_dev, float* W_out_dev,
+                           uint8_t* mask_dev, void* ws, size_t ws_bytes,
+                           pwp_stats* stats_dev, void* stream);
+
+/* Same as pwp_prune_layer, but first builds H = 2 X X^T into H_dev (b x b fp32,
+ * caller-owned scratch, overwritten) from token-major activations X_dev ([n, b]). */
+pwp_status pwp_prune_layer_x(const pwp_config* cfg, const void* W_dev, int32_t wtype,
+                             int32_t c, int32_t b, const void* X_dev, int32_t xtype,
+                             int64_t n, float* H_dev, float* W_out_dev, uint8_t* mask_dev,
+                             void* ws, size_t ws_bytes, pwp_stats* stats_dev, void* stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char* pwp_status_string(int32_t status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int32_t pwp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PWP_H */

@@ -1,0 +1,256 @@
+"""Python binding of libpwp (B200 layer-reconstruction pruning).
+
+Argument marshalling only: every step of the prune runs in the CUDA kernels of
+libpwp.so, reached through its C ABI (include/pwp.h).  PyTorch provides device
+memory and the current stream.  There is no CPU fallback: if the library is
+missing, loading it raises.
+
+Names mirror the C entry points: ``hessian_accumulate``, ``damp_factor``,
+``prune_layer`` (H given or built from X), ``workspace_bytes``, plus
+``prune_layer_host`` for a call that starts and ends in host memory.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import numpy as np
+
+__all__ = [
+    "lib", "Config", "Stats", "THANOS", "SPARSEGPT", "UNSTRUCTURED", "NM", "BF16", "FP32",
+    "PwpError", "config", "workspace_bytes", "hessian_accumulate", "damp_factor", "prune_layer",
+    "prune_layer_host", "status_string", "LIB_PATH",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpwp.so")
+
+THANOS, SPARSEGPT = 0, 1
+UNSTRUCTURED, NM = 0, 1
+BF16, FP32 = 0, 1
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("method", ctypes.c_int32), ("pattern", ctypes.c_int32), ("nm_n", ctypes.c_int32),
+                ("nm_m", ctypes.c_int32), ("sparsity", ctypes.c_float), ("block", ctypes.c_int32),
+                ("damp", ctypes.c_float)]
+
+
+class Stats(ctypes.Structure):
+    _fields_ = [("status", ctypes.c_int32), ("status_site", ctypes.c_int32),
+                ("pruned", ctypes.c_int64), ("target", ctypes.c_int64), ("lam", ctypes.c_float),
+                ("shortfall", ctypes.c_int32), ("reread_blocks", ctypes.c_int32),
+                ("tie_blocks", ctypes.c_int32), ("reserved", ctypes.c_int32 * 4)]
+
+
+class PwpError(RuntimeError):
+    def __init__(self, status, where=""):
+        self.status = int(status)
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+_lib = None
+_vp, _sz, _i32, _i64, _f32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
+_SIGS = {
+    "pwp_workspace_bytes": (_sz, [ctypes.POINTER(Config), _i32, _i32]),
+    "pwp_factor_workspace_bytes": (_sz, [_i32]),
+    "pwp_hessian_accumulate": (_i32, [_vp, _i32, _i64, _i32, _vp, _i32, _vp]),
+    "pwp_damp_factor": (_i32, [_vp, _i32, _f32, _vp, _vp, _sz, _vp, _vp]),
+    "pwp_prune_layer": (_i32, [ctypes.POINTER(Config), _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _sz,
+                               _vp, _vp]),
+    "pwp_prune_layer_x": (_i32, [ctypes.POINTER(Config), _vp, _i32, _i32, _i32, _vp, _i32, _i64, _vp,
+                                 _vp, _vp, _vp, _sz, _vp, _vp]),
+    "pwp_status_string": (ctypes.c_char_p, [_i32]),
+    "pwp_version": (_i32, []),
+}
+
+
+def lib():
+    """Load libpwp.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libpwp.so not built ({LIB_PATH}); run python -m post_weight_pruning_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(s) -> str:
+    return lib().pwp_status_string(int(s)).decode()
+
+
+def _check(status, where):
+    if status != 0:
+        raise PwpError(status, where)
+
+
+def config(method="thanos", pattern="unstructured", nm=(2, 4), sparsity=0.5, block=128, damp=0.01) -> Config:
+    m = {"thanos": THANOS, "sparsegpt": SPARSEGPT}[method] if isinstance(method, str) else int(method)
+    if isinstance(pattern, str):
+        p = {"unstructured": UNSTRUCTURED, "nm": NM}[pattern]
+    else:
+        p = int(pattern)
+    n_keep, m_grp = nm if p == NM else (0, 0)
+    return Config(m, p, int(n_keep), int(m_grp), float(sparsity), int(block), float(damp))
+
+
+def workspace_bytes(cfg: Config, c: int, b: int) -> int:
+    return int(lib().pwp_workspace_bytes(ctypes.byref(cfg), int(c), int(b)))
+
+
+# ------------------------------------------------------------------- torch helpers
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_ptr(stream=None):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t):
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return FP32
+    raise TypeError(f"unsupported dtype {t.dtype}; use torch.bfloat16 or torch.float32")
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def new_stats(device="cuda"):
+    torch = _torch()
+    return torch.zeros(ctypes.sizeof(Stats), dtype=torch.uint8, device=device)
+
+
+def read_stats(stats_t) -> Stats:
+    raw = stats_t.cpu().numpy().tobytes()
+    return Stats.from_buffer_copy(raw)
+
+
+def hessian_accumulate(X, H=None, beta=0, stream=None):
+    """H := beta*H + 2 X X^T for token-major X ([n, b], bf16 or fp32 CUDA tensor)."""
+    torch = _torch()
+    _need_cuda(X)
+    n, b = X.shape
+    if H is None:
+        H = torch.empty((b, b), dtype=torch.float32, device=X.device)
+    _need_cuda(H)
+    st = lib().pwp_hessian_accumulate(_vp(X.data_ptr()), _dtype_code(X), int(n), int(b), _vp(H.data_ptr()),
+                                      int(beta), _stream_ptr(stream))
+    _check(st, "pwp_hessian_accumulate")
+    return H
+
+
+def damp_factor(H, damp=0.01, stream=None):
+    """In place: upper triangle of H becomes U with (H + lambda I)^-1 = U^T U.
+    Returns (g_diag, stats tensor)."""
+    torch = _torch()
+    _need_cuda(H)
+    b = H.shape[0]
+    g = torch.empty(b, dtype=torch.float32, device=H.device)
+    nws = int(lib().pwp_factor_workspace_bytes(int(b)))
+    ws = torch.empty(nws, dtype=torch.uint8, device=H.device)
+    stats = new_stats(H.device)
+    st = lib().pwp_damp_factor(_vp(H.data_ptr()), int(b), float(damp), _vp(g.data_ptr()), _vp(ws.data_ptr()),
+                               nws, _vp(stats.data_ptr()), _stream_ptr(stream))
+    _check(st, "pwp_damp_factor")
+    return g, stats
+
+
+@dataclass
+class Workspace:
+    ws: object
+    nbytes: int
+
+
+def make_workspace(cfg: Config, c, b, device="cuda") -> Workspace:
+    torch = _torch()
+    n = workspace_bytes(cfg, c, b)
+    if n == 0:
+        raise PwpError(1, "pwp_workspace_bytes")
+    return Workspace(torch.empty(n, dtype=torch.uint8, device=device), n)
+
+
+def prune_layer(W, *, H=None, X=None, sparsity=0.5, pattern="unstructured", nm=(2, 4), block=128,
+                damp=0.01, method="thanos", W_out=None, mask=None, workspace=None, stats=None,
+                stream=None, check=True):
+    """Prune one layer on the GPU.
+
+    W: [c, b] bf16/fp32 CUDA tensor.  Give either H (undamped 2XX^T, fp32 [b, b],
+    DESTROYED: holds U afterwards) or X (token-major [n, b] activations; an H
+    scratch is allocated unless H is also passed).  Returns (W_hat fp32, mask uint8,
+    Stats) -- with check=False the stats tensor is returned unread and nothing syncs."""
+    torch = _torch()
+    _need_cuda(W, H, X)
+    c, b = W.shape
+    cfg = config(method, pattern, nm, sparsity, block, damp)
+    if workspace is None:
+        workspace = make_workspace(cfg, c, b, W.device)
+    if W_out is None:
+        W_out = torch.empty((c, b), dtype=torch.float32, device=W.device)
+    if mask is None:
+        mask = torch.empty((c, b), dtype=torch.uint8, device=W.device)
+    if stats is None:
+        stats = new_stats(W.device)
+    L = lib()
+    if X is not None:
+        if H is None:
+            H = torch.empty((b, b), dtype=torch.float32, device=W.device)
+        st = L.pwp_prune_layer_x(ctypes.byref(cfg), _vp(W.data_ptr()), _dtype_code(W), int(c), int(b),
+                                 _vp(X.data_ptr()), _dtype_code(X), int(X.shape[0]), _vp(H.data_ptr()),
+                                 _vp(W_out.data_ptr()), _vp(mask.data_ptr()), _vp(workspace.ws.data_ptr()),
+                                 workspace.nbytes, _vp(stats.data_ptr()), _stream_ptr(stream))
+        where = "pwp_prune_layer_x"
+    else:
+        if H is None:
+            raise ValueError("give H or X")
+        st = L.pwp_prune_layer(ctypes.byref(cfg), _vp(W.data_ptr()), _dtype_code(W), int(c), int(b),
+                               _vp(H.data_ptr()), _vp(W_out.data_ptr()), _vp(mask.data_ptr()),
+                               _vp(workspace.ws.data_ptr()), workspace.nbytes, _vp(stats.data_ptr()),
+                               _stream_ptr(stream))
+        where = "pwp_prune_layer"
+    _check(st, where)
+    if not check:
+        return W_out, mask, stats
+    s = read_stats(stats)
+    if s.status != 0:
+        raise PwpError(s.status, where + " (device)")
+    return W_out, mask, s
+
+
+def prune_layer_host(W_host, X_host, *, out_W=None, out_mask=None, device="cuda", **kw):
+    """End-to-end call from host memory: copies W and X (pinned torch CPU tensors) to the
+    device, prunes, and copies W_hat and the mask back into (pinned) host tensors."""
+    torch = _torch()
+    c, b = W_host.shape
+    Wd = W_host.to(device, non_blocking=True)
+    Xd = X_host.to(device, non_blocking=True)
+    Wo, mk, stats = prune_layer(Wd, X=Xd, check=False, **kw)
+    if out_W is None:
+        out_W = torch.empty((c, b), dtype=torch.float32, pin_memory=True)
+    if out_mask is None:
+        out_mask = torch.empty((c, b), dtype=torch.uint8, pin_memory=True)
+    out_W.copy_(Wo, non_blocking=True)
+    out_mask.copy_(mk, non_blocking=True)
+    return out_W, out_mask, stats
+
+
+def from_bf16_bits(u16: np.ndarray, device="cuda"):
+    """Upload bf16 bit patterns (uint16 numpy array) as a torch.bfloat16 tensor."""
+    torch = _torch()
+    t = torch.from_numpy(np.ascontiguousarray(u16).view(np.int16))
+    return t.view(torch.bfloat16).to(device)

@@ -1,0 +1,122 @@
+// C ABI of libpwp: argument checks, workspace layout and the launch sequence.
+// The declarations and their contracts are in include/pwp.h.
+#include <cstring>
+
+#include "pwp_internal.cuh"
+
+namespace pwp {
+struct PruneBuffers;
+size_t prune_ws_layout(int c, int b, int B, PruneBuffers* pb, char* base);
+cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c, int b, float* H,
+                         float* Wout, uint8_t* mask, void* ws, pwp_stats* st, cudaStream_t s);
+cudaError_t launch_hessian_simt(const void* X, int xtype, long long n, int b, float* H, int beta,
+                                cudaStream_t s);
+cudaError_t launch_hessian_tc(const void* X, long long n, int b, float* H, int beta, cudaStream_t s,
+                              bool* used);
+}  // namespace pwp
+
+using namespace pwp;
+
+static bool valid_dtype(int32_t t) { return t == PWP_BF16 || t == PWP_FP32; }
+
+static bool valid_cfg(const pwp_config* cfg, int32_t c, int32_t b) {
+  if (!cfg) return false;
+  if (c < 1 || b < 1 || b > 16384) return false;
+  if ((long long)c * (long long)b >= (1LL << 31)) return false;
+  if (cfg->method != PWP_THANOS && cfg->method != PWP_SPARSEGPT) return false;
+  if (cfg->block < 1 || cfg->block > kMaxBlock) return false;
+  if (!(cfg->damp >= 0.f) || !(cfg->damp < 1e30f)) return false;
+  if (cfg->pattern == PWP_UNSTRUCTURED) {
+    if (!(cfg->sparsity >= 0.f && cfg->sparsity < 1.f)) return false;
+  } else if (cfg->pattern == PWP_NM) {
+    const int n = cfg->nm_n, m = cfg->nm_m;
+    if (m < 2 || m > 32 || (m & (m - 1)) != 0) return false;  // m must divide a warp
+    if (n < 1 || n >= m) return false;
+    if (b % m != 0 || cfg->block % m != 0) return false;
+  } else {
+    return false;
+  }
+  return true;
+}
+
+static bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+extern "C" {
+
+const char* pwp_status_string(int32_t status) {
+  switch (status) {
+    case PWP_OK: return "ok";
+    case PWP_EINVAL: return "invalid argument";
+    case PWP_ENOTSPD: return "damped Hessian is not positive definite";
+    case PWP_EWORKSPACE: return "workspace missing, misaligned or too small";
+    case PWP_ECUDA: return "CUDA error";
+    case PWP_ETIMEOUT: return "bounded device-side wait timed out";
+    case PWP_EBUDGET: return "sparsity target could not be met";
+    default: return "unknown status";
+  }
+}
+
+int32_t pwp_version(void) { return 100; }
+
+size_t pwp_workspace_bytes(const pwp_config* cfg, int32_t c, int32_t b) {
+  if (!valid_cfg(cfg, c, b)) return 0;
+  return prune_ws_layout(c, b, cfg->block, nullptr, nullptr);
+}
+
+size_t pwp_factor_workspace_bytes(int32_t b) {
+  if (b < 1 || b > 16384) return 0;
+  return factor_ws_bytes(b);
+}
+
+pwp_status pwp_hessian_accumulate(const void* X, int32_t xtype, int64_t n, int32_t b, float* H,
+                                  int32_t beta, void* stream) {
+  if (!H || b < 1 || b > 16384 || n < 0 || (n > 0 && !X) || !valid_dtype(xtype) ||
+      (beta != 0 && beta != 1))
+    return PWP_EINVAL;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e;
+  bool used = false;
+  if (xtype == PWP_BF16) {
+    e = launch_hessian_tc(X, n, b, H, beta, s, &used);
+    if (e != cudaSuccess) return PWP_ECUDA;
+  }
+  if (!used) e = launch_hessian_simt(X, xtype, n, b, H, beta, s);
+  return e == cudaSuccess ? PWP_OK : PWP_ECUDA;
+}
+
+pwp_status pwp_damp_factor(float* H, int32_t b, float damp, float* g_diag, void* ws, size_t ws_bytes,
+                           pwp_stats* st, void* stream) {
+  if (!H || !g_diag || !st || b < 1 || b > 16384 || !(damp >= 0.f)) return PWP_EINVAL;
+  if (!ws || !aligned(ws, 256) || ws_bytes < factor_ws_bytes(b)) return PWP_EWORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemsetAsync(st, 0, sizeof(pwp_stats), s) != cudaSuccess) return PWP_ECUDA;
+  cudaError_t e = launch_damp_factor(H, b, damp, g_diag, ws, ws_bytes, st, s);
+  return e == cudaSuccess ? PWP_OK : PWP_ECUDA;
+}
+
+pwp_status pwp_prune_layer(const pwp_config* cfg, const void* W, int32_t wtype, int32_t c, int32_t b,
+                           float* H, float* W_out, uint8_t* mask, void* ws, size_t ws_bytes,
+                           pwp_stats* st, void* stream) {
+  if (!valid_cfg(cfg, c, b) || !valid_dtype(wtype) || !W || !H || !W_out || !mask || !st)
+    return PWP_EINVAL;
+  if (!ws || !aligned(ws, 256) || ws_bytes < prune_ws_layout(c, b, cfg->block, nullptr, nullptr))
+    return PWP_EWORKSPACE;
+  cudaError_t e = launch_prune(cfg, W, wtype, c, b, H, W_out, mask, ws, st, (cudaStream_t)stream);
+  return e == cudaSuccess ? PWP_OK : PWP_ECUDA;
+}
+
+pwp_status pwp_prune_layer_x(const pwp_config* cfg, const void* W, int32_t wtype, int32_t c, int32_t b,
+                             const void* X, int32_t xtype, int64_t n, float* H, float* W_out,
+                             uint8_t* mask, void* ws, size_t ws_bytes, pwp_stats* st, void* stream) {
+  if (!valid_cfg(cfg, c, b) || !valid_dtype(wtype) || !valid_dtype(xtype) || !W || !H || !W_out ||
+      !mask || !st || n < 0 || (n > 0 && !X))
+    return PWP_EINVAL;
+  if (!ws || !aligned(ws, 256) || ws_bytes < prune_ws_layout(c, b, cfg->block, nullptr, nullptr))
+    return PWP_EWORKSPACE;
+  pwp_status ps = pwp_hessian_accumulate(X, xtype, n, b, H, 0, stream);
+  if (ps != PWP_OK) return ps;
+  cudaError_t e = launch_prune(cfg, W, wtype, c, b, H, W_out, mask, ws, st, (cudaStream_t)stream);
+  return e == cudaSuccess ? PWP_OK : PWP_ECUDA;
+}
+
+}  // extern "C"

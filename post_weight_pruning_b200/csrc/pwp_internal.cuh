@@ -1,0 +1,67 @@
+// Internal declarations shared by the CUDA translation units of libpwp.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/pwp.h"
+
+namespace pwp {
+
+constexpr int kNumSM = 148;              // B200
+constexpr int kHist1Bits = 15;           // first radix level: key bits [30:16]
+constexpr int kHist1Bins = 1 << kHist1Bits;
+constexpr int kHist2Bins = 1 << 16;      // second level: key bits [15:0]
+constexpr int kFactorNB = 64;            // panel width of the blocked factorisation
+constexpr int kMaxBlock = 128;           // largest column block B
+
+// Per-call device control block (lives at the start of the workspace).
+struct Ctl {
+  long long zstar;        // global removal target (Thanos unstructured)
+  long long pruned;       // removals so far
+  long long take;         // entries to select in the current region
+  long long count_less;   // entries with key < T
+  long long m;            // tied entries (key == T) that must also be selected
+  long long ties;         // entries with key == T in the region
+  long long pstar;        // tie cut-off: column-major position inside the block (inclusive)
+  unsigned int b1;        // top-level bin holding the threshold
+  unsigned int r1;        // rank of the threshold inside bin b1 (1-based)
+  unsigned int T;         // exact 31-bit score key of the threshold
+  int mode;               // 0: select nothing, 1: key/position rule
+  int pad[6];
+};
+
+// Where device-side failures are recorded (pwp_stats::status_site).
+enum Site : int {
+  kSiteDamp = 1, kSiteCholDiag = 2, kSiteSolve = 3, kSitePick = 4, kSiteFinal = 5,
+};
+
+__device__ __forceinline__ bool failed(const pwp_stats* st) {
+  return *((volatile const int32_t*)&st->status) != PWP_OK;
+}
+
+__device__ __forceinline__ void set_error(pwp_stats* st, int status, int site) {
+  if (atomicCAS((int*)&st->status, PWP_OK, status) == PWP_OK) st->status_site = site;
+}
+
+// Monotone key of a non-negative fp32 score: its bit pattern with the sign bit cleared
+// (a NaN of either sign stays inside the 31-bit key range the histograms cover).
+__device__ __forceinline__ unsigned int score_key(float s) { return __float_as_uint(s) & 0x7fffffffu; }
+
+// Thanos ranks by |W| * ||X_q|| (Wanda score).
+__device__ __forceinline__ float wanda_score(float w, float xnorm) { return fabsf(w) * xnorm; }
+
+// SparseGPT ranks by W^2 / [H^-1]_qq = (W / U_qq)^2.
+__device__ __forceinline__ float obs_score(float w, float uqq) {
+  float t = w / uqq;
+  return t * t;
+}
+
+// ---------------------------------------------------------------- launchers (host side)
+cudaError_t launch_hessian(const void* X, int xtype, long long n, int b, float* H, int beta,
+                           cudaStream_t s);
+cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void* ws,
+                               size_t ws_bytes, pwp_stats* st, cudaStream_t s);
+size_t factor_ws_bytes(int b);
+
+}  // namespace pwp

@@ -1,0 +1,83 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point that
+include/pwp.h declares, and rejects bad arguments on the host before launching."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import post_weight_pruning_b200 as pwp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(pwp_[a-z0-9_]+)\s*\(", src))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    L = pwp.lib()
+    names = _declared()
+    assert {"pwp_prune_layer", "pwp_prune_layer_x", "pwp_hessian_accumulate",
+            "pwp_workspace_bytes", "pwp_status_string"} <= names
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings():
+    for s in range(7):
+        assert pwp.status_string(s)
+    assert pwp.status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("kw", [
+    dict(sparsity=1.0), dict(sparsity=-0.1), dict(block=0), dict(block=129),
+    dict(pattern="nm", nm=(2, 3)), dict(pattern="nm", nm=(4, 4)), dict(pattern="nm", nm=(0, 4)),
+    dict(pattern="nm", nm=(2, 4), block=6), dict(damp=-1.0), dict(method=7),
+])
+def test_invalid_configs_have_no_workspace(kw):
+    cfg = pwp.config(**kw)
+    assert pwp.workspace_bytes(cfg, 64, 64) == 0
+
+
+def test_workspace_grows_with_shape_and_is_256_aligned():
+    cfg = pwp.config(block=128)
+    a = pwp.workspace_bytes(cfg, 128, 256)
+    b = pwp.workspace_bytes(cfg, 4096, 4096)
+    assert 0 < a < b and a % 256 == 0 and b % 256 == 0
+    assert pwp.workspace_bytes(pwp.config(pattern="nm", nm=(2, 4)), 64, 66) == 0   # b % m != 0
+
+
+def test_argument_errors_return_before_any_launch():
+    L = pwp.lib()
+    cfg = pwp.config()
+    vp = ctypes.c_void_p
+    # null pointers -> EINVAL
+    assert L.pwp_prune_layer(ctypes.byref(cfg), None, 0, 16, 16, None, None, None, None, 0, None, None) == 1
+    # too-small workspace -> EWORKSPACE (pointers are never dereferenced on the host)
+    fake = vp(1 << 20)
+    assert L.pwp_prune_layer(ctypes.byref(cfg), fake, 0, 16, 16, fake, fake, fake, fake, 10, fake, None) == 3
+    # misaligned workspace
+    n = pwp.workspace_bytes(cfg, 16, 16)
+    assert L.pwp_prune_layer(ctypes.byref(cfg), fake, 0, 16, 16, fake, fake, fake, vp((1 << 20) + 8), n,
+                             fake, None) == 3
+    # bad dtype / beta / shape
+    assert L.pwp_hessian_accumulate(fake, 7, 10, 16, fake, 0, None) == 1
+    assert L.pwp_hessian_accumulate(fake, 0, 10, 16, fake, 2, None) == 1
+    assert L.pwp_hessian_accumulate(fake, 0, 10, 0, fake, 0, None) == 1
+    assert L.pwp_damp_factor(fake, 16, 0.01, fake, None, 0, fake, None) == 3
+    assert L.pwp_prune_layer_x(ctypes.byref(cfg), fake, 0, 16, 16, fake, 0, -1, fake, fake, fake, fake, n,
+                               fake, None) == 1
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(pwp, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(pwp, "_lib", None)
+    with pytest.raises(ImportError):
+        pwp.lib()

@@ -1,0 +1,150 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the same
+seeded inputs.  Bars: masks meet every invariant bit-exactly and agree with the
+oracle's at >= 99.99% of positions, disagreeing only at near-ties of the oracle's own
+scores; W-hat within 1e-3 relative Frobenius; reconstruction loss within 1e-2."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests import _parity as P
+
+pytestmark = pytest.mark.gpu
+
+# Relative score gap under which the oracle's own choice is a near-tie.  The GPU
+# computes in fp32: scores carry the fp32 rounding of H (accumulated over n tokens),
+# of the factor and of every earlier block's update, a few 1e-6 relative.
+TIE_TOL = 2e-5
+
+
+def _torch():
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return torch
+
+
+CASES = [
+    # workload-scale fp32 layer, B = 32, every method and pattern
+    ("layer128x256_fp32", "thanos", "unstructured", (0, 0)),
+    ("layer128x256_fp32", "thanos", "nm", (2, 4)),
+    ("layer128x256_fp32", "thanos", "nm", (4, 8)),
+    ("layer128x256_fp32", "sparsegpt", "unstructured", (0, 0)),
+    ("layer128x256_fp32", "sparsegpt", "nm", (2, 4)),
+    ("layer128x256_fp32", "sparsegpt", "nm", (4, 8)),
+]
+
+
+def _check(W, dtype, gpu, orc, X, pattern, nm, block, target):
+    res = P.compare(W, dtype, gpu, orc, pattern=pattern, nm=nm, block=block, tie_tol=TIE_TOL)
+    W_hat, mask, st = gpu
+    assert res["status"] == 0
+    assert res["zeros_exact"]
+    assert res["n_mask"] == target == res["stats_pruned"]
+    if pattern == "nm":
+        n_keep, m = nm
+        g = mask.reshape(mask.shape[0], -1, m).sum(axis=2)
+        assert np.all(g == m - n_keep)
+    assert res["agree"] >= P.MASK_AGREE, res
+    assert res["n_dis_not_tie"] == 0, res
+    assert res["w_rel"] <= P.W_REL_TOL, res
+    G = 0.5 * oracle.hessian(synth.to_f64(X, dtype))
+    lg = P.loss_of(W, dtype, W_hat, G)
+    assert abs(lg - orc["loss"]) <= P.LOSS_REL_TOL * orc["loss"], (lg, orc["loss"])
+    return res
+
+
+@pytest.mark.parametrize("name,method,pattern,nm", CASES)
+def test_small_layer_matches_oracle(name, method, pattern, nm):
+    _torch()
+    wl = synth.workload(name)
+    W, X = synth.make_W(wl), synth.make_X_tokens(wl)
+    kw = dict(method=method, pattern=pattern, nm=nm, block=wl.block, sparsity=wl.sparsity, damp=wl.damp)
+    gpu = P.run_gpu(W, X, wl.dtype, **kw)
+    orc = P.run_oracle(W, X, wl.dtype, **kw)
+    _check(W, wl.dtype, gpu, orc, X, pattern, nm, wl.block, orc["pruned"])
+
+
+@pytest.mark.parametrize("c,b,n,B,dtype,method,pattern,nm,s", [
+    (37, 200, 300, 48, "fp32", "thanos", "unstructured", (0, 0), 0.37),      # ragged last block
+    (37, 200, 300, 48, "fp32", "sparsegpt", "unstructured", (0, 0), 0.37),
+    (37, 200, 300, 48, "fp32", "thanos", "nm", (4, 8), 0.5),
+    (70, 96, 160, 128, "fp32", "thanos", "unstructured", (0, 0), 0.6),       # one block wider than b
+    (3, 5, 9, 1, "fp32", "thanos", "unstructured", (0, 0), 0.5),             # B = 1
+    (3, 5, 9, 1, "fp32", "sparsegpt", "unstructured", (0, 0), 0.5),
+    (1, 64, 80, 16, "fp32", "thanos", "unstructured", (0, 0), 0.5),          # single row
+    (256, 512, 1024, 128, "bf16", "thanos", "unstructured", (0, 0), 0.5),    # bf16, several 128-blocks
+    (256, 512, 1024, 128, "bf16", "thanos", "nm", (2, 4), 0.5),
+    (256, 512, 1024, 64, "bf16", "sparsegpt", "unstructured", (0, 0), 0.5),
+])
+def test_shapes_and_edges_match_oracle(c, b, n, B, dtype, method, pattern, nm, s):
+    _torch()
+    wl = synth.custom(c, b, n, dtype=dtype, outlier_frac=0.02, outlier_scale=20.0, block=B,
+                      sparsity=s, seed=c + b)
+    W, X = synth.make_W(wl), synth.make_X_tokens(wl)
+    kw = dict(method=method, pattern=pattern, nm=nm, block=B, sparsity=s, damp=0.01)
+    gpu = P.run_gpu(W, X, dtype, **kw)
+    orc = P.run_oracle(W, X, dtype, **kw)
+    _check(W, dtype, gpu, orc, X, pattern, nm, B, orc["pruned"])
+
+
+def test_zero_sparsity_is_identity():
+    _torch()
+    wl = synth.custom(20, 48, 64, dtype="bf16", block=16)
+    W, X = synth.make_W(wl), synth.make_X_tokens(wl)
+    W_hat, mask, st = P.run_gpu(W, X, "bf16", method="thanos", pattern="unstructured", nm=(0, 0),
+                                block=16, sparsity=0.0, damp=0.01)
+    assert st.status == 0 and st.pruned == 0 and not mask.any()
+    assert np.array_equal(W_hat, synth.to_f64(W, "bf16"))
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_hessian_matches_fp64(dtype):
+    torch = _torch()
+    import post_weight_pruning_b200 as pwp
+    wl = synth.custom(8, 200, 700, dtype=dtype, outlier_frac=0.02, outlier_scale=50.0)
+    X = synth.make_X_tokens(wl)
+    _, Xt = P.torch_inputs(synth.make_W(wl), X, dtype)
+    H = pwp.hessian_accumulate(Xt)
+    H2 = H.clone()
+    pwp.hessian_accumulate(Xt, H2, beta=1)
+    torch.cuda.synchronize()
+    ref = oracle.hessian(synth.to_f64(X, dtype))
+    Hg = H.cpu().numpy().astype(np.float64)
+    scale = np.sqrt(np.outer(np.diag(ref), np.diag(ref)))
+    assert np.max(np.abs(Hg - ref) / scale) < 1e-5
+    assert np.array_equal(Hg, Hg.T)
+    assert np.allclose(H2.cpu().numpy(), 2 * H.cpu().numpy(), rtol=1e-6, atol=0)
+
+
+def test_factor_matches_fp64():
+    torch = _torch()
+    import post_weight_pruning_b200 as pwp
+    wl = synth.custom(8, 300, 900, dtype="fp32", outlier_frac=0.02, outlier_scale=20.0)
+    X64 = synth.to_f64(synth.make_X_tokens(wl), "fp32")
+    H = oracle.hessian(X64)
+    Hd, lam = oracle.damp_hessian(H, 0.01)
+    U_ref = oracle.inverse_cholesky_upper(Hd)
+    Ht = torch.from_numpy(H.astype(np.float32)).cuda()
+    g, stats = pwp.damp_factor(Ht, 0.01)
+    torch.cuda.synchronize()
+    st = pwp.read_stats(stats)
+    assert st.status == 0
+    assert st.lam == pytest.approx(lam, rel=1e-5)
+    U = np.triu(Ht.cpu().numpy().astype(np.float64))
+    assert np.linalg.norm(U - U_ref) / np.linalg.norm(U_ref) < 1e-4
+    assert np.allclose(g.cpu().numpy(), np.diag(H) / 2, rtol=1e-6)
+
+
+def test_non_spd_is_reported_not_faulted():
+    torch = _torch()
+    import post_weight_pruning_b200 as pwp
+    # rank-deficient activations and no damping: H is singular
+    Xt = torch.zeros((10, 96), dtype=torch.float32, device="cuda")
+    Xt[:, :5] = torch.randn(10, 5, device="cuda")
+    W = torch.randn(16, 96, device="cuda")
+    with pytest.raises(pwp.PwpError) as e:
+        pwp.prune_layer(W, X=Xt, damp=0.0, block=32)
+    assert e.value.status == 2
