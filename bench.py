@@ -1,0 +1,416 @@
+#!/usr/bin/env python
+"""Benchmark: one-layer Thanos prune on the LLaMA-7B-shaped q_proj workload.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mine|reference]
+
+A step is the whole hot path on one layer: H = 2XX^T from the layer's activations,
+damping + factorisation, and the block sweep (scores, exact global-budget masks,
+joint row solves, trailing updates), through the library's C ABI
+(pwp_prune_layer_x).  The workload is W 4096x4096 bf16, X 16384x4096 bf16 tokens
+(8 x 2048) with 0.5% outlier features x50, 50% unstructured sparsity, B = 128.
+
+Under torchrun every rank prunes its own copy of the layer (independent layers of a
+model; no data-path collective), so the job's throughput is the sum over ranks
+("scaling": "weak").  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "layer prune time (ms) & weights/sec, 4096×4096 @50%; % of TC/HBM roofline"
+UNIT = "weights/s"
+WORKLOAD = "q_proj4096x4096"
+K_HESSIAN, K_FACTOR, K_STREAM, K_SELECT, K_SOLVE = 0, 1, 2, 3, 4
+CLASS_NAMES = {K_HESSIAN: "hessian_xxt", K_FACTOR: "factor", K_STREAM: "stream_update_score",
+               K_SELECT: "select", K_SOLVE: "row_solve"}
+CLASS_SOURCES = {K_HESSIAN: ["hessian_tc.cu", "hessian_simt.cu"], K_FACTOR: ["factor.cu"],
+                 K_STREAM: ["prune.cu"], K_SELECT: ["prune.cu"], K_SOLVE: ["prune.cu"]}
+
+
+def _load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured",
+                "sm_max_mhz": d.get("sm_max_mhz", 1965.0)}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback", "sm_max_mhz": 1965.0}
+
+
+def _source_hash(names):
+    h = hashlib.sha256()
+    for n in names:
+        p = os.path.join(ROOT, "post_weight_pruning_b200", "csrc", n)
+        if os.path.exists(p):
+            h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def _traffic_record(cls):
+    """Per-launch DRAM bytes of a kernel class from the committed ncu summary, or None if
+    the kernel's source changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    want = _source_hash(CLASS_SOURCES[cls])
+    for line in open(p):
+        f = line.split()
+        if len(f) >= 4 and not line.startswith("#") and f[0] == CLASS_NAMES[cls] and f[1] == want \
+                and f[2] == WORKLOAD:
+            return float(f[3])
+    return None
+
+
+# ------------------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------ algorithmic work
+
+def algorithmic_work(cls, wl, per_launch_ms, mask=None):
+    """(total algorithmic units over the recorded launches, unit, bound)."""
+    c, b, n, B = wl.c, wl.b, wl.n, wl.block
+    nblk = (b + B - 1) // B
+    if cls == K_HESSIAN:
+        return float(b) * b * n * len(per_launch_ms), "flop", "tensor"
+    if cls == K_STREAM:
+        # per block t: read + write the fp32 active region, read B rows of U over it
+        total = 0.0
+        for t in range(nblk):
+            j = t * B
+            total += 8.0 * c * (b - j) + (4.0 * B * (b - j) if t > 0 else 0.0)
+        steps = max(1, len(per_launch_ms) // nblk)
+        return total * steps, "byte", "hbm"
+    if cls == K_SELECT:
+        total = sum(4.0 * c * (b - t * B) for t in range(nblk))
+        steps = max(1, len(per_launch_ms) // nblk)
+        return total * steps, "byte", "hbm"
+    if cls == K_SOLVE:
+        m = mask.reshape(c, nblk, B).sum(axis=2).astype(np.float64)   # s per row per block
+        flops = float(np.sum(m ** 3 / 3.0 + 2.0 * m ** 2 + 4.0 * m * B))
+        steps = max(1, len(per_launch_ms) // nblk)
+        return flops * steps, "flop", "alu"
+    if cls == K_FACTOR:
+        return 2.0 * b ** 3 / 3.0 * len(per_launch_ms), "flop", "alu"
+    raise ValueError(cls)
+
+
+def fp32_alu_peak_tflops(sm_mhz):
+    # 148 SMs x 128 fp32 lanes x 2 flop per FMA
+    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
+# ------------------------------------------------------------------------------ CPU oracle
+
+def cpu_oracle_sample(wl, W_store, X_store, rows):
+    import oracle
+    import synth
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count()
+    W64 = synth.to_f64(W_store[:rows], wl.dtype)
+    t0 = time.perf_counter()
+    X64 = synth.to_f64(X_store, wl.dtype)
+    r = oracle.prune_layer(W64, Xt=X64, sparsity=float(np.float32(wl.sparsity)), block=wl.block,
+                           damp=wl.damp, method="thanos", pattern="unstructured")
+    dt = time.perf_counter() - t0
+    assert r["pruned"] == r["zstar"]
+    return {"value": rows * wl.b / dt, "unit": UNIT, "cores": int(threads), "kind": "oracle",
+            "sample": (f"fp64 numpy oracle on the {wl.name} workload restricted to its first {rows} "
+                       f"output rows: full H from all {wl.n} tokens, full factor, all "
+                       f"{(wl.b + wl.block - 1) // wl.block} blocks; {dt:.1f} s for "
+                       f"{rows}x{wl.b} weights")}
+
+
+# ------------------------------------------------------------------------------ reference arm
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import synth
+    wl = synth.workload(WORKLOAD)
+    W = synth.make_W(wl)
+    X = synth.make_X_tokens(wl)
+    rows = 128
+    for _ in range(args.warmup):
+        cpu_oracle_sample(wl, W, X, rows)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        cb = cpu_oracle_sample(wl, W, X, rows)
+        times.append(time.perf_counter() - t0)
+    tot = sum(times)
+    value = rows * wl.b * args.steps / tot
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": _config(wl),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cb["cores"], "kind": "oracle",
+                         "sample": cb["sample"]},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _config(wl):
+    return {"workload": (f"{wl.name}: W {wl.c}x{wl.b} bf16 ~N(0,0.02^2), X {wl.n}x{wl.b} bf16 tokens "
+                         f"(8x2048), 0.5% outlier features x50, Thanos 50% unstructured global "
+                         f"budget, B={wl.block}, damp={wl.damp}"),
+            "c": wl.c, "b": wl.b, "n_tokens": wl.n, "block": wl.block, "sparsity": wl.sparsity,
+            "input_dtype": "bf16", "l2": "flushed between steps (256 MiB write, untimed)",
+            "parallelism": "independent layer per rank"}
+
+
+# ------------------------------------------------------------------------------ GPU arm
+
+def run_mine(args):
+    import torch
+    import torch.distributed as dist
+    import synth
+    import post_weight_pruning_b200 as pwp
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    L = pwp.lib()
+    L.pwp_kernel_launches.restype = ctypes.c_int64
+    L.pwp_profile_enable.argtypes = [ctypes.c_int32, ctypes.c_int32]
+    L.pwp_profile_read.argtypes = [ctypes.c_void_p, ctypes.c_int32]
+
+    wl = synth.workload(WORKLOAD)
+    W_store = synth.make_W(wl)
+    X_store = synth.make_X_tokens(wl)
+    Wt = pwp.from_bf16_bits(W_store, dev)
+    Xt = pwp.from_bf16_bits(X_store, dev)
+    c, b = wl.c, wl.b
+    cfg_kw = dict(method="thanos", pattern="unstructured", sparsity=wl.sparsity, block=wl.block, damp=wl.damp)
+    ws = pwp.make_workspace(pwp.config(**cfg_kw), c, b, dev)
+    H = torch.empty((b, b), dtype=torch.float32, device=dev)
+    W_out = torch.empty((c, b), dtype=torch.float32, device=dev)
+    mask = torch.empty((c, b), dtype=torch.uint8, device=dev)
+    stats = pwp.new_stats(dev)
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)   # 256 MiB > 126 MB L2
+    stream = torch.cuda.current_stream()
+
+    def step():
+        pwp.prune_layer(Wt, X=Xt, H=H, W_out=W_out, mask=mask, workspace=ws, stats=stats, check=False,
+                        **cfg_kw)
+
+    nblk = (b + wl.block - 1) // wl.block
+    launches_per_class = {K_HESSIAN: 1, K_FACTOR: 1, K_STREAM: nblk, K_SELECT: nblk, K_SOLVE: nblk}
+
+    for i in range(max(args.warmup, 1)):
+        flush.fill_(float(i))
+        step()
+    torch.cuda.synchronize()
+    st = pwp.read_stats(stats)
+    if st.status != 0 or st.pruned != st.target:
+        raise RuntimeError(f"warm-up step failed: status {st.status} pruned {st.pruned} target {st.target}")
+
+    # phase breakdown (untimed pass per kernel class) to pick the dominant kernel
+    phase_ms = {}
+    for cls in (K_HESSIAN, K_FACTOR, K_STREAM, K_SELECT, K_SOLVE):
+        L.pwp_profile_enable(cls, launches_per_class[cls])
+        flush.fill_(0.0)
+        step()
+        buf = (ctypes.c_float * launches_per_class[cls])()
+        n = L.pwp_profile_read(buf, launches_per_class[cls])
+        phase_ms[CLASS_NAMES[cls]] = float(sum(buf[:n]))
+    L.pwp_profile_enable(-1, 0)
+    dom = max((K_HESSIAN, K_FACTOR, K_STREAM, K_SELECT, K_SOLVE), key=lambda k: phase_ms[CLASS_NAMES[k]])
+
+    # timed region
+    cap = launches_per_class[dom] * args.steps
+    L.pwp_profile_enable(dom, cap)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = L.pwp_kernel_launches()
+    for i in range(args.steps):
+        flush.fill_(float(i + 1))
+        ev0[i].record(stream)
+        step()
+        ev1[i].record(stream)
+    torch.cuda.synchronize()
+    launches = L.pwp_kernel_launches() - launches0
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    step_ms = [ev0[i].elapsed_time(ev1[i]) for i in range(args.steps)]
+    total_ms = float(sum(step_ms))
+    buf = (ctypes.c_float * cap)()
+    nrec = L.pwp_profile_read(buf, cap)
+    L.pwp_profile_enable(-1, 0)
+    dom_ms = [float(x) for x in buf[:nrec]]
+    st = pwp.read_stats(stats)
+    if st.status != 0 or st.pruned != st.target:
+        raise RuntimeError(f"timed step failed: status {st.status}")
+    mask_np = mask.cpu().numpy() if dom == K_SOLVE else None
+
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+    value = world * c * b * args.steps / (max_ms / 1e3)
+
+    # end to end through the public API from pinned host buffers
+    W_host = torch.from_numpy(W_store.view(np.int16)).view(torch.bfloat16).pin_memory()
+    X_host = torch.from_numpy(X_store.view(np.int16)).view(torch.bfloat16).pin_memory()
+    out_W = torch.empty((c, b), dtype=torch.float32).pin_memory()
+    out_m = torch.empty((c, b), dtype=torch.uint8).pin_memory()
+    e2e_steps = max(1, min(args.steps, 5))
+    for i in range(2):
+        pwp.prune_layer_host(W_host, X_host, out_W=out_W, out_mask=out_m, device=dev, **cfg_kw)
+    torch.cuda.synchronize()
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+    for i in range(e2e_steps):
+        flush.fill_(float(i))
+        e0[i].record(stream)
+        pwp.prune_layer_host(W_host, X_host, out_W=out_W, out_mask=out_m, device=dev, **cfg_kw)
+        e1[i].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = float(sum(e0[i].elapsed_time(e1[i]) for i in range(e2e_steps)))
+    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = world * c * b * e2e_steps / (float(te.item()) / 1e3)
+
+    if rank == 0:
+        peaks = _load_peaks()
+        work, unit, bound = algorithmic_work(dom, wl, dom_ms, mask_np)
+        dur_s = sum(dom_ms) / 1e3
+        if unit == "byte":
+            achieved = work / dur_s / 1e9
+            peak, punit, psrc = peaks["hbm_gbs"], "GB/s", peaks["source"] + " hbm_gbs"
+        elif bound == "tensor":
+            achieved = work / dur_s / 1e12
+            peak, punit, psrc = peaks["bf16_tflops"], "TFLOP/s", peaks["source"] + " bf16_tflops (burst)"
+        else:
+            achieved = work / dur_s / 1e12
+            mhz = peaks["sm_max_mhz"]
+            peak, punit, psrc = fp32_alu_peak_tflops(mhz), "TFLOP/s", f"fp32 FMA issue rate at {mhz:.0f} MHz"
+        traffic = _traffic_record(dom)
+        roof = {"kernel": CLASS_NAMES[dom], "bound": bound, "achieved": achieved, "peak": peak, "unit": punit,
+                "frac": achieved / peak, "traffic": traffic, "peak_source": psrc,
+                "launches_timed": len(dom_ms)}
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": _config(wl),
+            "roofline": roof,
+            "phases_ms": phase_ms,
+            "gpu_launches": int(launches),
+            "e2e": {"value": e2e_value, "unit": UNIT,
+                    "h2d_bytes_per_step": int(W_host.numel() * 2 + X_host.numel() * 2),
+                    "d2h_bytes_per_step": int(out_W.numel() * 4 + out_m.numel())},
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_oracle_sample(wl, W_store, X_store, args.cpu_rows)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=256)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_mine(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -132,6 +132,25 @@ pwp_status pwp_prune_layer_x(const pwp_config* cfg, const void* W_dev, int32_t w
                              int64_t n, float* H_dev, float* W_out_dev, uint8_t* mask_dev,
                              void* ws, size_t ws_bytes, pwp_stats* stats_dev, void* stream);
 
+/* Instrumentation (no counterpart on the pages).
+ * pwp_kernel_launches: number of kernels this process has enqueued through the library.
+ * pwp_profile_enable(which, capacity): record a pair of CUDA events on the call's stream
+ *   around each launch of kernel class `which` (pwp_kernel_class), for up to `capacity`
+ *   launches; which < 0 switches recording off and frees the events.
+ * pwp_profile_read(ms, cap): waits for the recorded events, writes up to `cap` elapsed
+ *   times (milliseconds, one per launch, in launch order) and returns how many; the
+ *   record is then cleared. */
+typedef enum {
+    PWP_K_HESSIAN = 0,   /* the X X^T accumulation kernel */
+    PWP_K_FACTOR = 1,    /* the whole damping + factorisation phase */
+    PWP_K_STREAM = 2,    /* per block: trailing update + rescoring + histogram */
+    PWP_K_SELECT = 3,    /* per block: exact threshold selection */
+    PWP_K_SOLVE = 4      /* per block: per-row solves and in-block update */
+} pwp_kernel_class;
+int64_t pwp_kernel_launches(void);
+int32_t pwp_profile_enable(int32_t which, int32_t capacity);
+int32_t pwp_profile_read(float* ms_out, int32_t cap);
+
 /* Static, NUL-terminated description of a status code. */
 const char* pwp_status_string(int32_t status);
 

@@ -76,11 +76,14 @@ pwp_status pwp_hessian_accumulate(const void* X, int32_t xtype, int64_t n, int32
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e;
   bool used = false;
+  prof_begin(kKHessian, s);
   if (xtype == PWP_BF16) {
     e = launch_hessian_tc(X, n, b, H, beta, s, &used);
     if (e != cudaSuccess) return PWP_ECUDA;
   }
   if (!used) e = launch_hessian_simt(X, xtype, n, b, H, beta, s);
+  prof_end(kKHessian, s);
+  count_launches(1);
   return e == cudaSuccess ? PWP_OK : PWP_ECUDA;
 }
 

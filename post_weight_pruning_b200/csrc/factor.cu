@@ -279,24 +279,31 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
   const int np = (b + NB - 1) / NB;
   float* Vall = (float*)ws;
   float* T = Vall + (size_t)np * NB * NB;
+  long long nl = 0;
   damp_kernel<<<1, 1024, 0, s>>>(H, b, damp, g_diag, st);
+  ++nl;
   for (int p = np - 1; p >= 0; --p) {
     const int p0 = p * NB, nb = min(NB, b - p0);
     float* V = Vall + (size_t)p * NB * NB;
     chol_diag_kernel<<<1, 256, 0, s>>>(H, b, p0, nb, V, st);
+    ++nl;
     if (p0 > 0) {
+      nl += 2;
       chol_panel_kernel<<<(p0 + 7) / 8, 256, 0, s>>>(H, b, p0, nb, V, st);
       const int nT = (p0 + 63) / 64;
       chol_update_kernel<<<nT * (nT + 1) / 2, 256, 0, s>>>(H, b, p0, nb, st);
     }
   }
   put_diag_inverses_kernel<<<np, 256, 0, s>>>(H, b, Vall, st);
+  ++nl;
   for (int p = 1; p < np; ++p) {
     const int p0 = p * NB, nb = min(NB, b - p0);
     const float* V = Vall + (size_t)p * NB * NB;
     trmm_kernel<<<(p0 + 63) / 64, 256, 0, s>>>(H, b, p0, nb, T, st);
     trmm_finish_kernel<<<(p0 + 7) / 8, 256, 0, s>>>(H, b, p0, nb, T, V, st);
+    nl += 2;
   }
+  count_launches(nl);
   return cudaGetLastError();
 }
 

@@ -695,13 +695,18 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
     g_stream_grid = nsm;
     attrs = true;
   }
+  long long nl = 0;
   init_ctl_kernel<<<1, 1, 0, s>>>(pb.ctl, zstar, st, target);
   cudaMemsetAsync(pb.hist1, 0, sizeof(unsigned int) * kHist1Bins, s);
   convert_w_kernel<<<4 * g_stream_grid, 256, 0, s>>>(W, wtype, Wout, N);
+  nl += 2;
+  prof_begin(kKFactor, s);
   cudaError_t e = launch_damp_factor(H, b, cfg->damp, pb.g_diag, pb.fws, pb.fws_bytes, st, s);
+  prof_end(kKFactor, s);
   if (e != cudaSuccess) return e;
   prep_diag_kernel<<<(b + 255) / 256, 256, 0, s>>>(H, b, pb.g_diag, pb.xnorm, pb.udiag);
   block_mats_kernel<<<nblk, 256, B * (B + 1) * 4, s>>>(H, b, B, pb.Hb, pb.UJt, st);
+  nl += 2;
 
   const int solve_smem = 4 * (2 * B + B * (B + 1) / 2) * 4;
   for (int t = 0; t < nblk; ++t) {
@@ -711,28 +716,43 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
     const float* UJt_t = pb.UJt + (size_t)t * B * B;
     if (!nm && thanos) {
       // rescore the whole active region [j, b) while applying the previous block's update
+      prof_begin(kKStream, s);
       stream_kernel<kWanda><<<g_stream_grid, 256, kHist1Bins * 4, s>>>(
           Wout, c, b, j, pb.Zp, Bp, B, H, jp, pb.xnorm, b, pb.hist1, st);
+      prof_end(kKStream, s);
+      prof_begin(kKSelect, s);
       pick1_kernel<<<1, 1024, 0, s>>>(pb.ctl, pb.hist1, pb.hist2, (long long)c * (b - j), 1, 0, st);
       refine_kernel<kWanda><<<4 * g_stream_grid, 256, 0, s>>>(Wout, c, b, j, b, pb.xnorm, pb.ctl,
                                                               pb.hist2, st);
       pick2_kernel<kWanda><<<1, 1024, 0, s>>>(pb.ctl, pb.hist2, Wout, c, b, j, j1, pb.xnorm, st);
+      prof_end(kKSelect, s);
+      nl += 4;
     } else if (!nm) {
       // SparseGPT: update the active region, score only the block
+      prof_begin(kKStream, s);
       stream_kernel<kObs><<<g_stream_grid, 256, kHist1Bins * 4, s>>>(
           Wout, c, b, j, pb.Zp, Bp, B, H, jp, pb.udiag, j1, pb.hist1, st);
+      prof_end(kKStream, s);
+      prof_begin(kKSelect, s);
       long long quota = (long long)((double)cfg->sparsity * (double)c * (double)(j1 - j));
       pick1_kernel<<<1, 1024, 0, s>>>(pb.ctl, pb.hist1, pb.hist2, (long long)c * (j1 - j), 0, quota,
                                       st);
       refine_kernel<kObs><<<4 * g_stream_grid, 256, 0, s>>>(Wout, c, b, j, j1, pb.udiag, pb.ctl,
                                                             pb.hist2, st);
       pick2_kernel<kObs><<<1, 1024, 0, s>>>(pb.ctl, pb.hist2, Wout, c, b, j, j1, pb.udiag, st);
+      prof_end(kKSelect, s);
+      nl += 4;
     } else if (t > 0) {
+      prof_begin(kKStream, s);
       stream_kernel<kNoScore><<<g_stream_grid, 256, 0, s>>>(Wout, c, b, j, pb.Zp, Bp, B, H, jp,
                                                             pb.xnorm, j, pb.hist1, st);
+      prof_end(kKStream, s);
+      nl += 1;
     }
     const int rows_per_cta = thanos ? 4 : 8;
     const int grid = (c + rows_per_cta - 1) / rows_per_cta;
+    prof_begin(kKSolve, s);
+    nl += 1;
     if (thanos) {
       if (nm)
         thanos_solve_kernel<true><<<grid, 128, solve_smem, s>>>(Wout, c, b, j, B, Hb_t, UJt_t,
@@ -752,8 +772,10 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
                                                            mask, pb.Zp, cfg->nm_n, cfg->nm_m,
                                                            pb.ctl, st);
     }
+    prof_end(kKSolve, s);
   }
   finalize_kernel<<<1, 1, 0, s>>>(pb.ctl, st, (thanos && !nm) ? 1 : 0);
+  count_launches(nl + 1);
   return cudaGetLastError();
 }
 

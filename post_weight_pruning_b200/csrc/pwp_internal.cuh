@@ -57,6 +57,12 @@ __device__ __forceinline__ float obs_score(float w, float uqq) {
   return t * t;
 }
 
+// ---------------------------------------------------------------- instrumentation (host side)
+enum KernelClass { kKHessian = 0, kKFactor = 1, kKStream = 2, kKSelect = 3, kKSolve = 4 };
+void prof_begin(int which, cudaStream_t s);
+void prof_end(int which, cudaStream_t s);
+void count_launches(long long n);
+
 // ---------------------------------------------------------------- launchers (host side)
 cudaError_t launch_hessian(const void* X, int xtype, long long n, int b, float* H, int beta,
                            cudaStream_t s);
