@@ -132,6 +132,25 @@ pwp_status pwp_prune_layer_x(const pwp_config* cfg, const void* W_dev, int32_t w
                              int64_t n, float* H_dev, float* W_out_dev, uint8_t* mask_dev,
                              void* ws, size_t ws_bytes, pwp_stats* stats_dev, void* stream);
 
+/* Prune without a caller-provided workspace (the pages have no counterpart: this is a
+ * convenience of this library).  For callers that cannot allocate device memory when
+ * they call -- an operator in a runtime that hands it only its input and output
+ * buffers, or a process whose device memory belongs to a framework allocator -- the
+ * scratch comes from one static device array of PWP_NOALLOC_SCRATCH_BYTES inside the
+ * library, which every GPU that loads the library keeps until the process exits.
+ *   Arguments, results and H's destruction are exactly those of pwp_prune_layer.
+ *   Returns PWP_EWORKSPACE, without enqueuing anything, when the configuration needs
+ *   more scratch than PWP_NOALLOC_SCRATCH_BYTES (pwp_workspace_bytes tells how much).
+ *   The first call on each device looks up the array's device address (with that
+ *   device current); make that first call before capturing any stream into a graph.
+ *   Nothing is allocated or freed.  All calls share the one array: calls whose work
+ *   overlaps on the GPU (different streams, or threads without ordering) race and give
+ *   wrong results; order them. */
+#define PWP_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+pwp_status pwp_prune_layer_noalloc(const pwp_config* cfg, const void* W_dev, int32_t wtype,
+                                   int32_t c, int32_t b, float* H_dev, float* W_out_dev,
+                                   uint8_t* mask_dev, pwp_stats* stats_dev, void* stream);
+
 /* Instrumentation (no counterpart on the pages).
  * pwp_kernel_launches: number of kernels this process has enqueued through the library.
  * pwp_profile_enable(which, capacity): record a pair of CUDA events on the call's stream
