@@ -6,7 +6,7 @@
 
 namespace pwp {
 struct PruneBuffers;
-size_t prune_ws_layout(int c, int b, int B, PruneBuffers* pb, char* base);
+size_t prune_ws_layout(const pwp_config* cfg, int c, int b, PruneBuffers* pb, char* base);
 cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c, int b, float* H,
                          float* Wout, uint8_t* mask, void* ws, pwp_stats* st, cudaStream_t s);
 cudaError_t launch_hessian_simt(const void* X, int xtype, long long n, int b, float* H, int beta,
@@ -60,7 +60,7 @@ int32_t pwp_version(void) { return 100; }
 
 size_t pwp_workspace_bytes(const pwp_config* cfg, int32_t c, int32_t b) {
   if (!valid_cfg(cfg, c, b)) return 0;
-  return prune_ws_layout(c, b, cfg->block, nullptr, nullptr);
+  return prune_ws_layout(cfg, c, b, nullptr, nullptr);
 }
 
 size_t pwp_factor_workspace_bytes(int32_t b) {
@@ -102,7 +102,7 @@ pwp_status pwp_prune_layer(const pwp_config* cfg, const void* W, int32_t wtype, 
                            pwp_stats* st, void* stream) {
   if (!valid_cfg(cfg, c, b) || !valid_dtype(wtype) || !W || !H || !W_out || !mask || !st)
     return PWP_EINVAL;
-  if (!ws || !aligned(ws, 256) || ws_bytes < prune_ws_layout(c, b, cfg->block, nullptr, nullptr))
+  if (!ws || !aligned(ws, 256) || ws_bytes < prune_ws_layout(cfg, c, b, nullptr, nullptr))
     return PWP_EWORKSPACE;
   cudaError_t e = launch_prune(cfg, W, wtype, c, b, H, W_out, mask, ws, st, (cudaStream_t)stream);
   return e == cudaSuccess ? PWP_OK : PWP_ECUDA;
@@ -114,7 +114,7 @@ pwp_status pwp_prune_layer_x(const pwp_config* cfg, const void* W, int32_t wtype
   if (!valid_cfg(cfg, c, b) || !valid_dtype(wtype) || !valid_dtype(xtype) || !W || !H || !W_out ||
       !mask || !st || n < 0 || (n > 0 && !X))
     return PWP_EINVAL;
-  if (!ws || !aligned(ws, 256) || ws_bytes < prune_ws_layout(c, b, cfg->block, nullptr, nullptr))
+  if (!ws || !aligned(ws, 256) || ws_bytes < prune_ws_layout(cfg, c, b, nullptr, nullptr))
     return PWP_EWORKSPACE;
   pwp_status ps = pwp_hessian_accumulate(X, xtype, n, b, H, 0, stream);
   if (ps != PWP_OK) return ps;

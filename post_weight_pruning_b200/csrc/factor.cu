@@ -11,18 +11,20 @@
 // Route, without ever forming H^-1:  H_d = V V^T with V upper triangular (a Cholesky
 // factorisation that starts from the last column), then U = V^-1.  Because
 // H_d^-1 = V^-T V^-1 = U^T U with U upper, this is the required factor.
-// Both phases are blocked by 64-column panels and run in place on the upper
-// triangle of H:
-//   factor  (panels from the last):  diagonal block in shared memory,
-//            panel rows above it via the block's explicit triangular inverse,
-//            symmetric rank-64 update of the not-yet-factored top-left part;
-//   inverse (panels from the first): U[0:p0, P] = -U[0:p0, 0:p0] V[0:p0, P] U_PP.
+// Both phases run in place on the upper triangle of H:
+//   factor, 64-column panels from the last: rows above the panel via the diagonal
+//     block's explicit inverse, then a symmetric rank-64 update of the top-left part;
+//     the CTA that updates the next panel's diagonal block also factors and inverts it
+//     (look-ahead), so the serial chain is one kernel pair per panel;
+//   inverse, recursive doubling: with the diagonal blocks inverted, neighbouring
+//     blocks [A B; 0 D] are merged as [A^-1, -A^-1 B D^-1; 0, D^-1] level by level,
+//     each level two batched triangular-times-dense products.
 #include "pwp_internal.cuh"
 
 namespace pwp {
 namespace {
 
-constexpr int NB = kFactorNB;
+constexpr int NB = kFactorNB;  // 64
 
 __global__ void __launch_bounds__(1024) damp_kernel(float* __restrict__ H, int b, float damp,
                                                     float* __restrict__ g_diag, pwp_stats* st) {
@@ -52,68 +54,82 @@ __global__ void __launch_bounds__(1024) damp_kernel(float* __restrict__ H, int b
   for (int q = threadIdx.x; q < b; q += blockDim.x) H[(long long)q * b + q] += lam;
 }
 
-// Factor the nb x nb diagonal block at p0 (already carrying the updates of every
-// later panel): A = V_PP V_PP^T, V_PP upper.  Writes V_PP to H and its inverse
-// W_PP = V_PP^-1 (upper, zero below) to Vinv[NB][NB].
-__global__ void __launch_bounds__(256) chol_diag_kernel(float* __restrict__ H, int b, int p0, int nb,
-                                                        float* __restrict__ Vinv, pwp_stats* st) {
-  __shared__ float A[NB][NB + 1];
-  __shared__ float Wi[NB][NB + 1];
-  __shared__ int bad;
-  if (failed(st)) return;
+// Factor the nb x nb block held in A (symmetric, upper triangle valid) as A = V V^T, V
+// upper (last column first), and invert V.  256 threads.  On return A's upper triangle
+// holds V and Wi holds V^-1 (upper, zero below).  Returns false on a non-positive pivot.
+__device__ bool factor_diag_block(float (*A)[NB + 1], float (*Wi)[NB + 1], int nb, int* bad,
+                                  pwp_stats* st) {
   const int tid = threadIdx.x;
-  if (tid == 0) bad = 0;
-  for (int idx = tid; idx < nb * nb; idx += blockDim.x) {
-    int r = idx / nb, s = idx % nb;
-    if (r <= s) {
-      float v = H[(long long)(p0 + r) * b + p0 + s];
-      A[r][s] = v;
-      A[s][r] = v;
-    }
-  }
-  __syncthreads();
   for (int i = nb - 1; i >= 0; --i) {
     if (tid == 0) {
-      float d = A[i][i];
+      const float d = A[i][i];
       if (!(d > 0.f) || !isfinite(d)) {
-        bad = 1;
+        *bad = 1;
         set_error(st, PWP_ENOTSPD, kSiteCholDiag);
       } else {
         A[i][i] = sqrtf(d);
       }
     }
     __syncthreads();
-    if (bad) return;
-    const float piv = A[i][i];
-    for (int r = tid; r < i; r += blockDim.x) A[r][i] = A[r][i] / piv;
+    if (*bad) return false;
+    const float inv = 1.f / A[i][i];
+    if (tid < i) A[tid][i] *= inv;
     __syncthreads();
-    for (int idx = tid; idx < i * i; idx += blockDim.x) {
-      int r = idx / i, s = idx % i;
-      if (r <= s) A[r][s] -= A[r][i] * A[s][i];
+    // rank-1 update of the leading i x i upper triangle: thread owns column s = tid & 63,
+    // rows r = (tid >> 6) + 4k
+    {
+      const int sc = tid & 63, r0 = tid >> 6;
+      if (sc < i) {
+        const float vs = A[sc][i];
+        for (int r = r0; r <= sc; r += 4) A[r][sc] = fmaf(-A[r][i], vs, A[r][sc]);
+      }
     }
     __syncthreads();
   }
-  // inverse of the upper-triangular block, one column per thread
-  if (tid < nb) {
-    const int c = tid;
-    for (int r = c + 1; r < NB; ++r) Wi[r][c] = 0.f;
-    Wi[c][c] = 1.f / A[c][c];
-    for (int i = c - 1; i >= 0; --i) {
-      float s = 0.f;
-      for (int t = i + 1; t <= c; ++t) s = fmaf(A[i][t], Wi[t][c], s);
-      Wi[i][c] = -s / A[i][i];
-    }
+  // Wi = V^-1 (upper).  Diagonal first, then rows from the bottom: for row r, entries
+  // c > r: Wi[r][c] = -(sum_{t=r+1..c} V[r][t] Wi[t][c]) / V[r][r].  Threads own columns
+  // c (tid & 63) and split the sum four ways (tid >> 6).
+  if (tid < NB) {
+    for (int r = 0; r < NB; ++r) Wi[r][tid] = (r == tid && tid < nb) ? 1.f / A[tid][tid] : 0.f;
   }
   __syncthreads();
-  for (int idx = tid; idx < NB * NB; idx += blockDim.x) {
+  __shared__ float part[4][NB];
+  const int cc = tid & 63, qq = tid >> 6;
+  for (int r = nb - 2; r >= 0; --r) {
+    float s = 0.f;
+    if (cc > r && cc < nb)
+      for (int t = r + 1 + qq; t <= cc; t += 4) s = fmaf(A[r][t], Wi[t][cc], s);
+    part[qq][cc] = s;
+    __syncthreads();
+    if (qq == 0 && cc > r && cc < nb)
+      Wi[r][cc] = -(part[0][cc] + part[1][cc] + part[2][cc] + part[3][cc]) * Wi[r][r];
+    __syncthreads();
+  }
+  return true;
+}
+
+// Stand-alone factorisation of the diagonal block at p0 (used for the last panel).
+__global__ void __launch_bounds__(256) chol_diag_kernel(float* __restrict__ H, int b, int p0, int nb,
+                                                        float* __restrict__ Vinv, pwp_stats* st) {
+  __shared__ float A[NB][NB + 1];
+  __shared__ float Wi[NB][NB + 1];
+  __shared__ int bad;
+  if (failed(st)) return;
+  if (threadIdx.x == 0) bad = 0;
+  for (int idx = threadIdx.x; idx < nb * nb; idx += blockDim.x) {
+    int r = idx / nb, s = idx % nb;
+    if (r <= s) A[r][s] = H[(long long)(p0 + r) * b + p0 + s];
+  }
+  __syncthreads();
+  if (!factor_diag_block(A, Wi, nb, &bad, st)) return;
+  for (int idx = threadIdx.x; idx < NB * NB; idx += blockDim.x) {
     int r = idx / NB, s = idx % NB;
-    float w = (r < nb && s < nb && r <= s) ? Wi[r][s] : 0.f;
-    Vinv[idx] = w;
+    Vinv[idx] = (r < nb && s < nb && r <= s) ? Wi[r][s] : 0.f;
     if (r < nb && s < nb && r <= s) H[(long long)(p0 + r) * b + p0 + s] = A[r][s];
   }
 }
 
-// Rows above the panel: V[r, P] = A[r, P] (V_PP^T)^-1 = A[r, P] Winv^T, r < p0.
+// Rows above the panel: V[r, P] = A[r, P] (V_PP^T)^-1 = A[r, P] Wi^T, r < p0.
 __global__ void __launch_bounds__(256) chol_panel_kernel(float* __restrict__ H, int b, int p0, int nb,
                                                          const float* __restrict__ Vinv,
                                                          const pwp_stats* st) {
@@ -121,65 +137,90 @@ __global__ void __launch_bounds__(256) chol_panel_kernel(float* __restrict__ H, 
   __shared__ float rowbuf[8][NB];
   if (failed(st)) return;
   for (int idx = threadIdx.x; idx < NB * NB; idx += blockDim.x) Wi[idx / NB][idx % NB] = Vinv[idx];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.x * 8 + warp;
   __syncthreads();
-  if (r >= p0) return;
-  float* hr = H + (long long)r * b + p0;
-  for (int t = lane; t < nb; t += 32) rowbuf[warp][t] = hr[t];
-  __syncwarp();
-  for (int c = lane; c < nb; c += 32) {
-    float s = 0.f;
-    for (int t = c; t < nb; ++t) s = fmaf(rowbuf[warp][t], Wi[c][t], s);
-    hr[c] = s;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int r = blockIdx.x * 8 + warp; r < p0; r += gridDim.x * 8) {
+    float* hr = H + (long long)r * b + p0;
+    for (int t = lane; t < nb; t += 32) rowbuf[warp][t] = hr[t];
+    __syncwarp();
+    for (int c = lane; c < nb; c += 32) {
+      float s = 0.f;
+      for (int t = c; t < nb; ++t) s = fmaf(rowbuf[warp][t], Wi[c][t], s);
+      hr[c] = s;
+    }
+    __syncwarp();
   }
 }
 
-// Symmetric update of the top-left part: A[r][s] -= sum_t V[r][p0+t] V[s][p0+t],
-// r <= s < p0 (64x64 tiles on or above the diagonal).
+// Symmetric update of the top-left part: A[r][s] -= sum_t V[r][p0+t] V[s][p0+t] for
+// r <= s < p0, 128x128 tiles on or above the diagonal, 8x8 outputs per thread.  The CTA
+// whose tile holds the next panel's diagonal block [p0-NB, p0) then factors it.
 __global__ void __launch_bounds__(256) chol_update_kernel(float* __restrict__ H, int b, int p0, int nb,
-                                                          const pwp_stats* st) {
-  __shared__ float Ar[64][NB + 1];
-  __shared__ float Br[64][NB + 1];
+                                                          float* __restrict__ Vinv_next,
+                                                          pwp_stats* st) {
+  extern __shared__ __align__(16) float fsm[];
+  float (*As)[128 + 4] = reinterpret_cast<float (*)[132]>(fsm);               // [NB][132], k-major
+  float (*Bs)[128 + 4] = reinterpret_cast<float (*)[132]>(fsm + NB * 132);
+  __shared__ int bad;
   if (failed(st)) return;
-  const int nT = (p0 + 63) / 64;
+  const int nT = (p0 + 127) / 128;
   int I = 0, rem = blockIdx.x;
   while (rem >= nT - I) { rem -= nT - I; ++I; }
   const int J = I + rem;
-  const int i0 = I * 64, j0 = J * 64;
-  for (int idx = threadIdx.x; idx < 64 * NB; idx += blockDim.x) {
-    int rr = idx / NB, t = idx % NB;
+  const int i0 = I * 128, j0 = J * 128;
+  for (int idx = threadIdx.x; idx < 128 * NB; idx += blockDim.x) {
+    const int rr = idx / NB, t = idx % NB;
     float a = 0.f, c = 0.f;
     if (t < nb) {
       if (i0 + rr < p0) a = H[(long long)(i0 + rr) * b + p0 + t];
       if (j0 + rr < p0) c = H[(long long)(j0 + rr) * b + p0 + t];
     }
-    Ar[rr][t] = a;
-    Br[rr][t] = c;
+    As[t][rr] = a;
+    Bs[t][rr] = c;
   }
   __syncthreads();
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  float acc[4][4] = {};
-  for (int t = 0; t < nb; ++t) {
-    float av[4], bv[4];
+  float acc[8][8] = {};
+#pragma unroll 4
+  for (int t = 0; t < NB; ++t) {
+    const float4 a0 = *reinterpret_cast<const float4*>(&As[t][ty * 4]);
+    const float4 a1 = *reinterpret_cast<const float4*>(&As[t][64 + ty * 4]);
+    const float4 b0 = *reinterpret_cast<const float4*>(&Bs[t][tx * 4]);
+    const float4 b1 = *reinterpret_cast<const float4*>(&Bs[t][64 + tx * 4]);
+    const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-    for (int x = 0; x < 4; ++x) av[x] = Ar[ty + 16 * x][t];
+    for (int x = 0; x < 8; ++x)
 #pragma unroll
-    for (int y = 0; y < 4; ++y) bv[y] = Br[tx + 16 * y][t];
-#pragma unroll
-    for (int x = 0; x < 4; ++x)
-#pragma unroll
-      for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
+      for (int y = 0; y < 8; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
   }
 #pragma unroll
-  for (int x = 0; x < 4; ++x) {
-    int r = i0 + ty + 16 * x;
+  for (int x = 0; x < 8; ++x) {
+    const int r = i0 + (x < 4 ? ty * 4 + x : 64 + ty * 4 + x - 4);
     if (r >= p0) continue;
 #pragma unroll
-    for (int y = 0; y < 4; ++y) {
-      int s = j0 + tx + 16 * y;
+    for (int y = 0; y < 8; ++y) {
+      const int s = j0 + (y < 4 ? tx * 4 + y : 64 + tx * 4 + y - 4);
       if (s < p0 && r <= s) H[(long long)r * b + s] -= acc[x][y];
     }
+  }
+  // look-ahead: factor the next panel's diagonal block if this tile holds it
+  const int q0 = p0 - NB;
+  if (q0 < 0 || I != J || q0 < i0 || q0 >= i0 + 128) return;
+  __syncthreads();  // this CTA's own writes to H are visible to its threads
+  float (*A)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(fsm);
+  float (*Wi)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(fsm + NB * (NB + 1));
+  if (threadIdx.x == 0) bad = 0;
+  for (int idx = threadIdx.x; idx < NB * NB; idx += blockDim.x) {
+    int r = idx / NB, s = idx % NB;
+    if (r <= s) A[r][s] = H[(long long)(q0 + r) * b + q0 + s];
+  }
+  __syncthreads();
+  if (!factor_diag_block(A, Wi, NB, &bad, st)) return;
+  for (int idx = threadIdx.x; idx < NB * NB; idx += blockDim.x) {
+    int r = idx / NB, s = idx % NB;
+    Vinv_next[idx] = (r <= s) ? Wi[r][s] : 0.f;
+    if (r <= s) H[(long long)(q0 + r) * b + q0 + s] = A[r][s];
   }
 }
 
@@ -197,81 +238,97 @@ __global__ void put_diag_inverses_kernel(float* __restrict__ H, int b, const flo
   }
 }
 
-// T[r][c] = sum_{t = r}^{p0-1} U[r][t] V[t][p0 + c]  (U: already-inverted top-left
-// part, V: factor column block of panel P).  64 rows x nb columns per CTA.
-__global__ void __launch_bounds__(256) trmm_kernel(const float* __restrict__ H, int b, int p0, int nb,
-                                                   float* __restrict__ T, const pwp_stats* st) {
-  __shared__ float Us[64][33];
-  __shared__ float Ps[32][NB + 1];
+// Batched product C = alpha * A B (+ C when accumulate), one 128x128 tile per CTA
+// (8x8 per thread), K in chunks of 16.  A (M x K) and B (K x N) are read with row
+// stride lda / ldb; a_upper: A is upper triangular (A[m][k] = 0 for k < m);
+// b_upper: B is upper triangular (B[k][n] = 0 for n < k).  blockIdx.z selects the
+// batch entry, whose matrices start batch_* elements further on.
+struct TriGemm {
+  int M, N, K;
+  const float* A; long long lda, batch_a;
+  const float* B; long long ldb, batch_b;
+  float* C; long long ldc, batch_c;
+  float alpha;
+  int a_upper, b_upper;
+};
+
+__global__ void __launch_bounds__(256) trigemm_kernel(TriGemm g, const pwp_stats* st) {
+  __shared__ __align__(16) float As[16][128 + 4];
+  __shared__ __align__(16) float Bs[16][128 + 4];
   if (failed(st)) return;
-  const int i0 = blockIdx.x * 64;
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  float acc[4][4] = {};
-  for (int t0 = i0; t0 < p0; t0 += 32) {
-    for (int idx = threadIdx.x; idx < 64 * 32; idx += blockDim.x) {
-      int rr = idx / 32, kk = idx % 32;
-      int r = i0 + rr, t = t0 + kk;
-      Us[rr][kk] = (r < p0 && t < p0 && t >= r) ? H[(long long)r * b + t] : 0.f;
-    }
-    for (int idx = threadIdx.x; idx < 32 * NB; idx += blockDim.x) {
-      int kk = idx / NB, cc = idx % NB;
-      int t = t0 + kk;
-      Ps[kk][cc] = (t < p0 && cc < nb) ? H[(long long)t * b + p0 + cc] : 0.f;
+  const float* A = g.A + blockIdx.z * g.batch_a;
+  const float* B = g.B + blockIdx.z * g.batch_b;
+  float* C = g.C + blockIdx.z * g.batch_c;
+  const int m0 = blockIdx.y * 128, n0 = blockIdx.x * 128;
+  if (m0 >= g.M || n0 >= g.N) return;
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  // the triangular operand bounds the useful k range of this tile
+  int kbeg = 0, kend = g.K;
+  if (g.a_upper) kbeg = m0;                       // k >= m
+  if (g.b_upper) kend = min(kend, n0 + 128);      // k <= n
+  float acc[8][8] = {};
+  for (int k0 = kbeg; k0 < kend; k0 += 16) {
+    for (int idx = tid; idx < 16 * 128; idx += 256) {
+      // A tile: rows m0..m0+127, k0..k0+15 (k fastest -> coalesced in A's rows)
+      const int mm = idx >> 4, kk = idx & 15;
+      const int m = m0 + mm, k = k0 + kk;
+      float a = 0.f;
+      if (m < g.M && k < kend && (!g.a_upper || k >= m)) a = A[(long long)m * g.lda + k];
+      As[kk][mm] = a;
+      // B tile: k0..k0+15, n0..n0+127 (n fastest)
+      const int kb = idx >> 7, nn = idx & 127;
+      const int kq = k0 + kb, n = n0 + nn;
+      float bv = 0.f;
+      if (kq < kend && n < g.N && (!g.b_upper || n >= kq)) bv = B[(long long)kq * g.ldb + n];
+      Bs[kb][nn] = bv;
     }
     __syncthreads();
-#pragma unroll 8
-    for (int kk = 0; kk < 32; ++kk) {
-      float av[4], bv[4];
 #pragma unroll
-      for (int x = 0; x < 4; ++x) av[x] = Us[ty + 16 * x][kk];
+    for (int kk = 0; kk < 16; ++kk) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[kk][64 + ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[kk][64 + tx * 4]);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-      for (int y = 0; y < 4; ++y) bv[y] = Ps[kk][tx + 16 * y];
+      for (int x = 0; x < 8; ++x)
 #pragma unroll
-      for (int x = 0; x < 4; ++x)
-#pragma unroll
-        for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
+        for (int y = 0; y < 8; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
     }
     __syncthreads();
   }
 #pragma unroll
-  for (int x = 0; x < 4; ++x) {
-    int r = i0 + ty + 16 * x;
-    if (r >= p0) continue;
+  for (int x = 0; x < 8; ++x) {
+    const int m = m0 + (x < 4 ? ty * 4 + x : 64 + ty * 4 + x - 4);
+    if (m >= g.M) continue;
 #pragma unroll
-    for (int y = 0; y < 4; ++y) {
-      int cc = tx + 16 * y;
-      if (cc < nb) T[(long long)r * NB + cc] = acc[x][y];
+    for (int y = 0; y < 8; ++y) {
+      const int n = n0 + (y < 4 ? tx * 4 + y : 64 + tx * 4 + y - 4);
+      if (n < g.N) C[(long long)m * g.ldc + n] = g.alpha * acc[x][y];
     }
   }
 }
 
-// U[r][p0 + c] = - sum_{t <= c} T[r][t] W_PP[t][c], one row per warp.
-__global__ void __launch_bounds__(256) trmm_finish_kernel(float* __restrict__ H, int b, int p0, int nb,
-                                                          const float* __restrict__ T,
-                                                          const float* __restrict__ Vinv,
-                                                          const pwp_stats* st) {
-  __shared__ float Wi[NB][NB + 1];
-  __shared__ float rowbuf[8][NB];
-  if (failed(st)) return;
-  for (int idx = threadIdx.x; idx < NB * NB; idx += blockDim.x) Wi[idx / NB][idx % NB] = Vinv[idx];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.x * 8 + warp;
-  __syncthreads();
-  if (r >= p0) return;
-  for (int t = lane; t < nb; t += 32) rowbuf[warp][t] = T[(long long)r * NB + t];
-  __syncwarp();
-  for (int c = lane; c < nb; c += 32) {
-    float s = 0.f;
-    for (int t = 0; t <= c; ++t) s = fmaf(rowbuf[warp][t], Wi[t][c], s);
-    H[(long long)r * b + p0 + c] = -s;
-  }
+void launch_trigemm(const TriGemm& g, int batch, const pwp_stats* st, cudaStream_t s) {
+  dim3 grid((g.N + 127) / 128, (g.M + 127) / 128, batch);
+  trigemm_kernel<<<grid, 256, 0, s>>>(g, st);
 }
 
 }  // namespace
 
 size_t factor_ws_bytes(int b) {
-  size_t np = (size_t)(b + NB - 1) / NB;
-  return np * NB * NB * sizeof(float) + (size_t)b * NB * sizeof(float) + 256;
+  const size_t np = (size_t)(b + NB - 1) / NB;
+  // temporary of the doubling levels: the full pairs of a level, or its ragged pair,
+  // whichever is larger (the two run one after the other on the stream)
+  size_t tmp = 0;
+  for (size_t m = NB; m < (size_t)b; m *= 2) {
+    const size_t full = (size_t)b / (2 * m), rest = (size_t)b - full * 2 * m;
+    size_t need = full * m * m;
+    if (rest > m && m * (rest - m) > need) need = m * (rest - m);
+    if (need > tmp) tmp = need;
+  }
+  return np * NB * NB * sizeof(float) + tmp * sizeof(float) + 256;
 }
 
 cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void* ws, size_t ws_bytes,
@@ -279,29 +336,59 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
   const int np = (b + NB - 1) / NB;
   float* Vall = (float*)ws;
   float* T = Vall + (size_t)np * NB * NB;
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(chol_update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * NB * 132 * 4);
+    attr = true;
+  }
   long long nl = 0;
   damp_kernel<<<1, 1024, 0, s>>>(H, b, damp, g_diag, st);
   ++nl;
-  for (int p = np - 1; p >= 0; --p) {
+  // factor, panels from the last; the last panel's diagonal block stands alone
+  {
+    const int p = np - 1, p0 = p * NB, nb = b - p0;
+    chol_diag_kernel<<<1, 256, 0, s>>>(H, b, p0, nb, Vall + (size_t)p * NB * NB, st);
+    ++nl;
+  }
+  for (int p = np - 1; p >= 1; --p) {
     const int p0 = p * NB, nb = min(NB, b - p0);
     float* V = Vall + (size_t)p * NB * NB;
-    chol_diag_kernel<<<1, 256, 0, s>>>(H, b, p0, nb, V, st);
-    ++nl;
-    if (p0 > 0) {
-      nl += 2;
-      chol_panel_kernel<<<(p0 + 7) / 8, 256, 0, s>>>(H, b, p0, nb, V, st);
-      const int nT = (p0 + 63) / 64;
-      chol_update_kernel<<<nT * (nT + 1) / 2, 256, 0, s>>>(H, b, p0, nb, st);
-    }
+    const int pgrid = min((p0 + 7) / 8, 4 * kNumSM);
+    chol_panel_kernel<<<pgrid, 256, 0, s>>>(H, b, p0, nb, V, st);
+    const int nT = (p0 + 127) / 128;
+    chol_update_kernel<<<nT * (nT + 1) / 2, 256, 2 * NB * 132 * 4, s>>>(H, b, p0, nb,
+                                                                      Vall + (size_t)(p - 1) * NB * NB, st);
+    nl += 2;
   }
   put_diag_inverses_kernel<<<np, 256, 0, s>>>(H, b, Vall, st);
   ++nl;
-  for (int p = 1; p < np; ++p) {
-    const int p0 = p * NB, nb = min(NB, b - p0);
-    const float* V = Vall + (size_t)p * NB * NB;
-    trmm_kernel<<<(p0 + 63) / 64, 256, 0, s>>>(H, b, p0, nb, T, st);
-    trmm_finish_kernel<<<(p0 + 7) / 8, 256, 0, s>>>(H, b, p0, nb, T, V, st);
-    nl += 2;
+  // inverse by recursive doubling: merge [A B; 0 D] pairs of width m
+  for (int m = NB; m < b; m *= 2) {
+    const int full = b / (2 * m);                 // pairs with both halves of width m
+    const int rest = b - full * 2 * m;            // a ragged pair if rest > m
+    for (int pass = 0; pass < 2; ++pass) {
+      int batch, i0, m2;
+      if (pass == 0) {
+        batch = full;
+        i0 = 0;
+        m2 = m;
+      } else {
+        batch = rest > m ? 1 : 0;
+        i0 = full * 2 * m;
+        m2 = rest - m;
+      }
+      if (batch == 0) continue;
+      const long long step = (long long)2 * m * b + 2 * m;   // next pair's corner
+      // T = A^-1 B   (A^-1: m x m upper at (i0, i0); B: m x m2 at (i0, i0+m))
+      TriGemm g1{m, m2, m, H + (long long)i0 * b + i0, b, step, H + (long long)i0 * b + i0 + m, b, step,
+                 T, m2, (long long)m * m2, 1.f, 1, 0};
+      launch_trigemm(g1, batch, st, s);
+      // B = -T D^-1  (D^-1: m2 x m2 upper at (i0+m, i0+m))
+      TriGemm g2{m, m2, m2, T, m2, (long long)m * m2, H + (long long)(i0 + m) * b + i0 + m, b, step,
+                 H + (long long)i0 * b + i0 + m, b, step, -1.f, 0, 1};
+      launch_trigemm(g2, batch, st, s);
+      nl += 2;
+    }
   }
   count_launches(nl);
   return cudaGetLastError();

@@ -17,7 +17,7 @@
 
 namespace pwp {
 struct PruneBuffers;
-size_t prune_ws_layout(int c, int b, int B, PruneBuffers* pb, char* base);
+size_t prune_ws_layout(const pwp_config* cfg, int c, int b, PruneBuffers* pb, char* base);
 cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c, int b, float* H,
                          float* Wout, uint8_t* mask, void* ws, pwp_stats* st, cudaStream_t s);
 }  // namespace pwp

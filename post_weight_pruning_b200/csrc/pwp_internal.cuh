@@ -57,6 +57,36 @@ __device__ __forceinline__ float obs_score(float w, float uqq) {
   return t * t;
 }
 
+enum ScoreKind { kNoScore = 0, kWanda = 1, kObs = 2 };
+
+template <int SCORE>
+__device__ __forceinline__ unsigned int key_of(float w, float p) {
+  return SCORE == kWanda ? score_key(wanda_score(w, p)) : score_key(obs_score(w, p));
+}
+
+// Selection flag of one entry of block row k (column qq of the block).
+// Unstructured: key < T, or key == T with column-major position qq*c + k at or before
+// the tie cut-off.  N:M: rank inside the group of nm_m lanes by (key, column) below
+// nm_m - nm_n.  Every lane of the warp must call it (N:M shuffles within the group).
+template <bool NM>
+__device__ __forceinline__ bool selected(unsigned int key, bool valid, int qq, int k, int c,
+                                         const Ctl& ctl, int nm_n, int nm_m) {
+  if (NM) {
+    const int lane = threadIdx.x & 31;
+    const int base = lane & ~(nm_m - 1);
+    int rank = 0;
+    for (int o = 0; o < nm_m; ++o) {
+      unsigned int ko = __shfl_sync(0xffffffffu, key, base + o);
+      rank += (ko < key) || (ko == key && base + o < lane);
+    }
+    return valid && rank < nm_m - nm_n;
+  }
+  if (!valid || ctl.mode == 0) return false;
+  if (key < ctl.T) return true;
+  if (key == ctl.T) return (long long)qq * c + k <= ctl.pstar;
+  return false;
+}
+
 // ---------------------------------------------------------------- instrumentation (host side)
 enum KernelClass { kKHessian = 0, kKFactor = 1, kKStream = 2, kKSelect = 3, kKSolve = 4 };
 void prof_begin(int which, cudaStream_t s);
@@ -69,5 +99,21 @@ cudaError_t launch_hessian(const void* X, int xtype, long long n, int b, float* 
 cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void* ws,
                                size_t ws_bytes, pwp_stats* st, cudaStream_t s);
 size_t factor_ws_bytes(int b);
+
+// exact selection of the `take` smallest keys of a region (select.cu)
+void launch_pick1(Ctl* ctl, unsigned int* hist1, unsigned int* hist2, long long region_n,
+                  int global_budget, long long quota, pwp_stats* st, cudaStream_t s);
+void launch_refine(int score, const float* W, int c, int b, int q0, int q1, const float* sc,
+                   const Ctl* ctl, unsigned int* hist2, const pwp_stats* st, cudaStream_t s);
+void launch_pick2(int score, Ctl* ctl, const unsigned int* hist2, const float* W, int c, int b,
+                  int j, int j1, const float* sc, pwp_stats* st, cudaStream_t s);
+
+// per-row work of one block (solve.cu); returns the number of kernels launched
+int launch_thanos_solve(bool nm, const float* W, int c, int b, int j, int B, const float* Kt,
+                        const float* xnorm, Ctl* ctl, uint8_t* mask, float* Zs, int nm_n, int nm_m,
+                        int* ovf, pwp_stats* st, cudaStream_t s);
+int launch_sparsegpt_solve(bool nm, const float* W, int c, int b, int j, int B, const float* H,
+                           const float* udiag, Ctl* ctl, uint8_t* mask, float* Zs, int nm_n,
+                           int nm_m, pwp_stats* st, cudaStream_t s);
 
 }  // namespace pwp

@@ -1,0 +1,268 @@
+// Exact selection of the r lowest-scoring weights of a region.
+//
+// "Pruning LLMs with Thanos", section "Contribution two: keep the budget global and
+// the execution local", steps 1-4: the residual count r, the rescored active region,
+// and "exactly that many lowest-scoring weights" as the candidate set.  For SparseGPT
+// the region is the current block and r its quota.
+//
+// Keys are the bit patterns of the non-negative fp32 scores, so ordering keys orders
+// scores.  The r-th smallest key T is found by a two-level radix select:
+//   level 1: a histogram of key bits [30:16] (built while the scores are produced),
+//   level 2: a histogram of bits [15:0] over the entries of the level-1 bin (refine),
+// then T = (bin1 << 16) | bin2.  Among entries equal to T, the order is (column, row)
+// -- the pages do not fix one -- so when only some tied entries are taken, the cut-off
+// position inside the current block is located as well.
+#include <climits>
+
+#include "pwp_internal.cuh"
+
+namespace pwp {
+namespace {
+
+__device__ __forceinline__ long long warp_sum_ll(long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Find, in a histogram of NB bins (1024 threads), the bin holding the `rank`-th
+// (1-based) entry.  Each warp owns a contiguous range of NB/32 bins read in coalesced
+// 32-bin chunks.  Returns the bin in *bin (-1 if the histogram holds fewer entries) and
+// the number of entries in lower bins in *before.
+template <int NB>
+__device__ void find_rank(const unsigned int* __restrict__ hist, long long rank, int* bin,
+                          long long* before, long long* sh_warp, int* sh_sel, long long* sh_base) {
+  constexpr int PER_WARP = NB / 32;
+  constexpr int CHUNKS = PER_WARP / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned int* h = hist + warp * PER_WARP;
+  long long sum = 0;
+#pragma unroll 8
+  for (int ch = 0; ch < CHUNKS; ++ch) sum += h[ch * 32 + lane];
+  sum = warp_sum_ll(sum);
+  if (lane == 0) sh_warp[warp] = sum;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    long long cum = 0;
+    int sel = -1;
+    for (int w = 0; w < 32; ++w) {
+      if (rank > cum && rank <= cum + sh_warp[w]) { sel = w; break; }
+      cum += sh_warp[w];
+    }
+    *sh_sel = sel;
+    *sh_base = cum;
+  }
+  __syncthreads();
+  const int sel = *sh_sel;
+  if (sel < 0) {
+    *bin = -1;
+    *before = 0;
+    return;
+  }
+  if (warp == sel) {
+    long long cum = *sh_base;
+    const unsigned int* hs = hist + sel * PER_WARP;
+    for (int ch = 0; ch < CHUNKS; ++ch) {
+      long long v = hs[ch * 32 + lane];
+      long long tot = warp_sum_ll(v);
+      if (rank <= cum + tot) {
+        // inclusive prefix inside the chunk
+        long long x = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          long long yv = __shfl_up_sync(0xffffffffu, x, o);
+          if (lane >= o) x += yv;
+        }
+        const bool hit = (rank > cum + x - v) && (rank <= cum + x);
+        const unsigned int m = __ballot_sync(0xffffffffu, hit);
+        const int src = __ffs(m) - 1;
+        long long excl = __shfl_sync(0xffffffffu, cum + x - v, src);
+        if (lane == 0) {
+          sh_warp[0] = sel * PER_WARP + ch * 32 + src;
+          sh_warp[1] = excl;
+        }
+        break;
+      }
+      cum += tot;
+    }
+  }
+  __syncthreads();
+  *bin = (int)sh_warp[0];
+  *before = sh_warp[1];
+}
+
+__global__ void __launch_bounds__(1024) pick1_kernel(Ctl* ctl, unsigned int* __restrict__ hist1,
+                                                     unsigned int* __restrict__ hist2, long long region_n,
+                                                     int global_budget, long long quota, pwp_stats* st) {
+  __shared__ long long sh_warp[32];
+  __shared__ int sh_sel;
+  __shared__ long long sh_base, s_take;
+  if (failed(st)) return;
+  if (threadIdx.x == 0) {
+    long long r = global_budget ? ctl->zstar - ctl->pruned : quota;
+    long long take = r < region_n ? r : region_n;
+    if (take < r) st->shortfall = 1;
+    if (take < 0) take = 0;
+    ctl->take = take;
+    ctl->mode = take > 0 ? 1 : 0;
+    s_take = take;
+  }
+  __syncthreads();
+  const long long take = s_take;
+  if (take > 0) {
+    int bin;
+    long long before;
+    find_rank<kHist1Bins>(hist1, take, &bin, &before, sh_warp, &sh_sel, &sh_base);
+    if (threadIdx.x == 0) {
+      if (bin < 0) {
+        set_error(st, PWP_EBUDGET, kSitePick);
+        ctl->mode = 0;
+      } else {
+        ctl->b1 = (unsigned int)bin;
+        ctl->r1 = (unsigned int)(take - before);
+        ctl->count_less = before;
+      }
+    }
+    __syncthreads();
+  }
+  for (int i = threadIdx.x; i < kHist1Bins; i += blockDim.x) hist1[i] = 0u;
+  for (int i = threadIdx.x; i < kHist2Bins; i += blockDim.x) hist2[i] = 0u;
+}
+
+// Level-2 histogram: key bits [15:0] of the entries whose bits [30:16] equal b1.
+// One row per CTA iteration, columns across threads (coalesced).
+template <int SCORE>
+__global__ void __launch_bounds__(256) refine_kernel(const float* __restrict__ W, int c, int b, int q0,
+                                                     int q1, const float* __restrict__ sc,
+                                                     const Ctl* __restrict__ ctl,
+                                                     unsigned int* __restrict__ hist2,
+                                                     const pwp_stats* st) {
+  if (failed(st) || ctl->mode == 0) return;
+  const unsigned int b1 = ctl->b1;
+  for (int r = blockIdx.x; r < c; r += gridDim.x) {
+    const float* wr = W + (long long)r * b;
+    for (int q = q0 + threadIdx.x; q < q1; q += blockDim.x) {
+      unsigned int key = key_of<SCORE>(wr[q], __ldg(sc + q));
+      if ((key >> 16) == b1) atomicAdd(&hist2[key & 0xffffu], 1u);
+    }
+  }
+}
+
+template <int SCORE>
+__global__ void __launch_bounds__(1024) pick2_kernel(Ctl* ctl, const unsigned int* __restrict__ hist2,
+                                                     const float* __restrict__ W, int c, int b, int j,
+                                                     int j1, const float* __restrict__ sc,
+                                                     pwp_stats* st) {
+  __shared__ long long sh_warp[32];
+  __shared__ int sh_sel;
+  __shared__ long long sh_base;
+  __shared__ unsigned int colcnt[kMaxBlock];
+  __shared__ int s_qstar;
+  __shared__ long long s_need;
+  if (failed(st) || ctl->mode == 0) return;
+  const int tid = threadIdx.x;
+  const long long r1 = ctl->r1;
+  int lo;
+  long long before2;
+  find_rank<kHist2Bins>(hist2, r1, &lo, &before2, sh_warp, &sh_sel, &sh_base);
+  if (lo < 0) {
+    if (tid == 0) set_error(st, PWP_EBUDGET, kSitePick);
+    return;
+  }
+  const unsigned int T = (ctl->b1 << 16) | (unsigned int)lo;
+  const long long ties = hist2[lo];
+  const long long count_less = ctl->count_less + before2;
+  const long long m = ctl->take - count_less;  // 1 <= m <= ties
+  __syncthreads();
+  if (tid == 0) {
+    ctl->T = T;
+    ctl->ties = ties;
+    ctl->m = m;
+    ctl->count_less = count_less;
+    ctl->pstar = LLONG_MAX;
+    if (ties > 1) st->tie_blocks += 1;
+  }
+  if (m >= ties) return;  // every tied entry is taken
+  // Some but not all ties are taken: count ties per block column (rows coalesced).
+  const int nJ = j1 - j;
+  for (int i = tid; i < kMaxBlock; i += blockDim.x) colcnt[i] = 0u;
+  __syncthreads();
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int r = warp; r < c; r += 32) {
+    for (int qq = lane; qq < nJ; qq += 32) {
+      unsigned int key = key_of<SCORE>(W[(long long)r * b + j + qq], __ldg(sc + j + qq));
+      if (key == T) atomicAdd(&colcnt[qq], 1u);
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    long long cum = 0;
+    int qstar = -1;
+    for (int qq = 0; qq < nJ; ++qq) {
+      if (cum + colcnt[qq] >= m) { qstar = qq; break; }
+      cum += colcnt[qq];
+    }
+    s_qstar = qstar;
+    s_need = m - cum;  // 1-based rank of the last taken tie inside column qstar
+  }
+  __syncthreads();
+  if (s_qstar < 0) return;  // fewer than m ties inside the block: all of them are taken
+  const int q = j + s_qstar;
+  const int per = (c + 1023) / 1024;
+  long long cnt = 0;
+  for (int i = 0; i < per; ++i) {
+    int r = tid * per + i;
+    if (r < c && key_of<SCORE>(W[(long long)r * b + q], __ldg(sc + q)) == T) ++cnt;
+  }
+  // exclusive scan of cnt over the CTA
+  long long x = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    long long yv = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += yv;
+  }
+  if (lane == 31) sh_warp[warp] = x;
+  __syncthreads();
+  long long wbase = 0;
+  for (int w = 0; w < warp; ++w) wbase += sh_warp[w];
+  const long long bef = wbase + x - cnt;
+  const long long need = s_need;
+  if (bef < need && need <= bef + cnt) {
+    long long k = bef;
+    for (int i = 0; i < per; ++i) {
+      int r = tid * per + i;
+      if (r < c && key_of<SCORE>(W[(long long)r * b + q], __ldg(sc + q)) == T) {
+        if (++k == need) {
+          ctl->pstar = (long long)s_qstar * c + r;
+          break;
+        }
+      }
+    }
+  }
+}
+
+}  // namespace
+
+void launch_pick1(Ctl* ctl, unsigned int* hist1, unsigned int* hist2, long long region_n,
+                  int global_budget, long long quota, pwp_stats* st, cudaStream_t s) {
+  pick1_kernel<<<1, 1024, 0, s>>>(ctl, hist1, hist2, region_n, global_budget, quota, st);
+}
+
+void launch_refine(int score, const float* W, int c, int b, int q0, int q1, const float* sc,
+                   const Ctl* ctl, unsigned int* hist2, const pwp_stats* st, cudaStream_t s) {
+  const int grid = c < 4 * kNumSM ? c : 4 * kNumSM;
+  if (score == kWanda)
+    refine_kernel<kWanda><<<grid, 256, 0, s>>>(W, c, b, q0, q1, sc, ctl, hist2, st);
+  else
+    refine_kernel<kObs><<<grid, 256, 0, s>>>(W, c, b, q0, q1, sc, ctl, hist2, st);
+}
+
+void launch_pick2(int score, Ctl* ctl, const unsigned int* hist2, const float* W, int c, int b, int j,
+                  int j1, const float* sc, pwp_stats* st, cudaStream_t s) {
+  if (score == kWanda)
+    pick2_kernel<kWanda><<<1, 1024, 0, s>>>(ctl, hist2, W, c, b, j, j1, sc, st);
+  else
+    pick2_kernel<kObs><<<1, 1024, 0, s>>>(ctl, hist2, W, c, b, j, j1, sc, st);
+}
+
+}  // namespace pwp

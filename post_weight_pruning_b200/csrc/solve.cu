@@ -1,0 +1,322 @@
+// Per-row work of one column block: the mask, and the coefficients of the row's
+// compensating update.
+//
+// Thanos ("Pruning LLMs with Thanos", section "Contribution one: solve a selected set
+// directly"): for row k with selected set Q in block J, u = W[k, Q] and
+// R-hat = K[Q, Q] with K = inv(H_d[A, A]); z = R-hat^-1 u and the row's update is
+// delta_k = -z^T K[Q, A].  This kernel produces z (scattered into a B-wide row, zero
+// outside Q); the stream kernel then applies W[:, A] -= Z K[J, A] for all rows at once,
+// and sets W[k, Q] to exactly zero.
+//
+// SparseGPT ("Weight Pruning in Large Language Models ...", section "SparseGPT"): the
+// column-sequential sweep inside the block, e_q = W_q / U_qq on selected entries, whose
+// in-block part is replayed here row by row to get e; the stream kernel applies
+// W[:, A] -= E U[J, A].
+#include "pwp_internal.cuh"
+
+namespace pwp {
+namespace {
+
+// Packed lower-triangular storage with every row starting on a 16-byte boundary:
+// row i holds entries 0..i and is padded to a multiple of 4 floats.
+__host__ __device__ constexpr int poff(int i) {
+  return 4 * (2 * (i >> 2) * ((i >> 2) + 1) + (i & 3) * ((i >> 2) + 1));
+}
+
+template <int SCAP>
+struct SolveSmem {
+  static constexpr int kL = poff(SCAP);
+  static constexpr int kY = SCAP + 4;
+  static constexpr int kPerWarp = kL + kY + SCAP;  // floats: L, y, Qidx
+};
+
+// Cholesky R-hat = L L^T (left-looking, 4-column panels; lanes own rows) with u carried
+// as an extra row so that the factorisation also gives y = L^-1 u, then L^T z = y.
+// L holds R-hat's lower triangle on entry; y holds u.  On return y[0..s) = z.
+// Returns false on a non-positive pivot.  Whole warp, uniform control flow.
+__device__ bool chol_solve(float* __restrict__ L, float* __restrict__ y, int s, int lane) {
+  for (int jp = 0; jp < s; jp += 4) {
+    if (jp > 0) {
+      const float* p0 = L + poff(jp);
+      const float* p1 = L + poff(jp + 1);
+      const float* p2 = L + poff(jp + 2);
+      const float* p3 = L + poff(jp + 3);
+      for (int i = jp + lane; i <= s; i += 32) {
+        float* ri = (i < s) ? L + poff(i) : y;
+        float a0 = ri[jp], a1 = ri[jp + 1], a2 = ri[jp + 2], a3 = ri[jp + 3];
+#pragma unroll 2
+        for (int t = 0; t < jp; t += 4) {
+          const float4 x = *reinterpret_cast<const float4*>(ri + t);
+          const float4 q0 = *reinterpret_cast<const float4*>(p0 + t);
+          const float4 q1 = *reinterpret_cast<const float4*>(p1 + t);
+          const float4 q2 = *reinterpret_cast<const float4*>(p2 + t);
+          const float4 q3 = *reinterpret_cast<const float4*>(p3 + t);
+          a0 = fmaf(-x.x, q0.x, a0); a0 = fmaf(-x.y, q0.y, a0); a0 = fmaf(-x.z, q0.z, a0); a0 = fmaf(-x.w, q0.w, a0);
+          a1 = fmaf(-x.x, q1.x, a1); a1 = fmaf(-x.y, q1.y, a1); a1 = fmaf(-x.z, q1.z, a1); a1 = fmaf(-x.w, q1.w, a1);
+          a2 = fmaf(-x.x, q2.x, a2); a2 = fmaf(-x.y, q2.y, a2); a2 = fmaf(-x.z, q2.z, a2); a2 = fmaf(-x.w, q2.w, a2);
+          a3 = fmaf(-x.x, q3.x, a3); a3 = fmaf(-x.y, q3.y, a3); a3 = fmaf(-x.z, q3.z, a3); a3 = fmaf(-x.w, q3.w, a3);
+        }
+        ri[jp] = a0;
+        ri[jp + 1] = a1;
+        ri[jp + 2] = a2;
+        ri[jp + 3] = a3;
+      }
+      __syncwarp();
+    }
+    const int pend = min(jp + 4, s);
+    for (int a = jp; a < pend; ++a) {
+      const float d = L[poff(a) + a];
+      if (!(d > 0.f)) return false;
+      const float l = sqrtf(d);
+      const float inv = 1.f / l;
+      __syncwarp();
+      for (int i = a + 1 + lane; i <= s; i += 32) {
+        float* ri = (i < s) ? L + poff(i) : y;
+        ri[a] *= inv;
+      }
+      if (lane == 0) L[poff(a) + a] = l;
+      __syncwarp();
+      if (a + 1 < pend) {
+        for (int i = a + 1 + lane; i <= s; i += 32) {
+          float* ri = (i < s) ? L + poff(i) : y;
+          const float lia = ri[a];
+          const int cend = (i < s) ? min(pend - 1, i) : pend - 1;
+          for (int cc = a + 1; cc <= cend; ++cc) ri[cc] = fmaf(-lia, L[poff(cc) + a], ri[cc]);
+        }
+        __syncwarp();
+      }
+    }
+  }
+  for (int a = s - 1; a >= 0; --a) {
+    const float za = y[a] / L[poff(a) + a];
+    __syncwarp();
+    const float* ra = L + poff(a);
+    for (int t = lane; t < a; t += 32) y[t] = fmaf(-ra[t], za, y[t]);
+    if (lane == 0) y[a] = za;
+    __syncwarp();
+  }
+  return true;
+}
+
+// One warp per row.  Rows whose selected set exceeds SCAP are appended to the
+// overflow list ovf (ovf[0] = count, ovf[1..] = rows) for a second pass with a larger
+// SCAP; when rows_from_list is set, the rows come from that list.
+template <int SCAP, bool NM>
+__global__ void __launch_bounds__(256) thanos_solve_kernel(const float* __restrict__ W, int c, int b,
+                                                           int j, int B, const float* __restrict__ Kt,
+                                                           const float* __restrict__ xnorm,
+                                                           Ctl* __restrict__ ctlp,
+                                                           uint8_t* __restrict__ mask,
+                                                           float* __restrict__ Zs, int nm_n, int nm_m,
+                                                           int* __restrict__ ovf, int rows_from_list,
+                                                           pwp_stats* st) {
+  extern __shared__ __align__(16) float smem[];
+  if (failed(st)) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwarps = blockDim.x >> 5;
+  float* L = smem + warp * SolveSmem<SCAP>::kPerWarp;
+  float* y = L + SolveSmem<SCAP>::kL;
+  int* Qidx = reinterpret_cast<int*>(y + SolveSmem<SCAP>::kY);
+  const Ctl ctl = *ctlp;
+  const int nJ = min(B, b - j);
+  const int nrows = rows_from_list ? *((volatile int*)ovf) : c;
+  constexpr int MAXI = kMaxBlock / 32;
+  for (int idx = blockIdx.x * nwarps + warp; idx < nrows; idx += gridDim.x * nwarps) {
+    const int k = rows_from_list ? ovf[1 + idx] : idx;
+    const float* wrow = W + (long long)k * b + j;
+    float w[MAXI];
+    bool sel[MAXI];
+    int pos[MAXI];
+    int s = 0;
+#pragma unroll
+    for (int i = 0; i < MAXI; ++i) {
+      const int qq = lane + 32 * i;
+      const bool valid = qq < nJ;
+      w[i] = valid ? wrow[qq] : 0.f;
+      const unsigned int key = valid ? key_of<kWanda>(w[i], __ldg(xnorm + j + qq)) : 0xffffffffu;
+      sel[i] = (32 * i < nJ) ? selected<NM>(key, valid, qq, k, c, ctl, nm_n, nm_m) : false;
+      const unsigned int bal = __ballot_sync(0xffffffffu, sel[i]);
+      pos[i] = s + __popc(bal & ((1u << lane) - 1u));
+      s += __popc(bal);
+    }
+    if (s > SCAP) {
+      if (lane == 0) {
+        int at = atomicAdd(ovf, 1);
+        ovf[1 + at] = k;
+      }
+      continue;
+    }
+    uint8_t* mrow = mask + (long long)k * b + j;
+#pragma unroll
+    for (int i = 0; i < MAXI; ++i) {
+      const int qq = lane + 32 * i;
+      if (qq < nJ) mrow[qq] = sel[i] ? 1 : 0;
+      if (sel[i]) {
+        Qidx[pos[i]] = qq;
+        y[pos[i]] = w[i];
+      }
+    }
+    __syncwarp();
+    bool ok = true;
+    if (s > 0) {
+      // R-hat = K[Q, Q], lower triangle, gathered four rows at a time
+      constexpr int CH = (SCAP + 31) / 32;
+      for (int a0 = 0; a0 < s; a0 += 4) {
+        float v[4][CH];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int a = a0 + r;
+          const float* krow = Kt + (size_t)(a < s ? Qidx[a] : 0) * b + j;
+#pragma unroll
+          for (int ch = 0; ch < CH; ++ch) {
+            const int cc = lane + 32 * ch;
+            v[r][ch] = (a < s && cc <= a) ? __ldg(krow + Qidx[cc]) : 0.f;
+          }
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int a = a0 + r;
+#pragma unroll
+          for (int ch = 0; ch < CH; ++ch) {
+            const int cc = lane + 32 * ch;
+            if (a < s && cc <= a) L[poff(a) + cc] = v[r][ch];
+          }
+        }
+      }
+      __syncwarp();
+      ok = chol_solve(L, y, s, lane);
+      if (!ok && lane == 0) set_error(st, PWP_ENOTSPD, kSiteSolve);
+      if (lane == 0) atomicAdd((unsigned long long*)&ctlp->pruned, (unsigned long long)s);
+    }
+    float* zrow = Zs + (long long)k * B;
+#pragma unroll
+    for (int i = 0; i < MAXI; ++i) {
+      const int qq = lane + 32 * i;
+      if (qq < B) zrow[qq] = (qq < nJ && sel[i] && ok) ? y[pos[i]] : 0.f;
+    }
+    __syncwarp();
+  }
+}
+
+// SparseGPT in-block sweep, one warp per row (no shared memory): for each block column
+// q in order, e = W_q / U_qq on a selected entry (0 otherwise) and the later block
+// columns of the row drop e * U[q, .].  Writes e (the row of E) and the mask.
+template <bool NM>
+__global__ void __launch_bounds__(256) sparsegpt_solve_kernel(const float* __restrict__ W, int c, int b,
+                                                              int j, int B, const float* __restrict__ H,
+                                                              const float* __restrict__ udiag,
+                                                              Ctl* __restrict__ ctlp,
+                                                              uint8_t* __restrict__ mask,
+                                                              float* __restrict__ Zs, int nm_n, int nm_m,
+                                                              pwp_stats* st) {
+  if (failed(st)) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int k = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (k >= c) return;
+  const Ctl ctl = *ctlp;
+  const int nJ = min(B, b - j);
+  constexpr int MAXI = kMaxBlock / 32;
+  float w[MAXI], e[MAXI];
+  bool sel[MAXI];
+  const float* wrow = W + (long long)k * b + j;
+  int s = 0;
+#pragma unroll
+  for (int i = 0; i < MAXI; ++i) {
+    const int qq = lane + 32 * i;
+    const bool valid = qq < nJ;
+    w[i] = valid ? wrow[qq] : 0.f;
+    e[i] = 0.f;
+    const unsigned int key = valid ? key_of<kObs>(w[i], __ldg(udiag + j + qq)) : 0xffffffffu;
+    sel[i] = (32 * i < nJ) ? selected<NM>(key, valid, qq, k, c, ctl, nm_n, nm_m) : false;
+    s += __popc(__ballot_sync(0xffffffffu, sel[i]));
+  }
+  for (int qq = 0; qq < nJ; ++qq) {
+    const int owner = qq & 31, slot = qq >> 5;
+    float wq = 0.f;
+    bool sq = false;
+#pragma unroll
+    for (int i = 0; i < MAXI; ++i)
+      if (i == slot) { wq = w[i]; sq = sel[i]; }
+    wq = __shfl_sync(0xffffffffu, wq, owner);
+    sq = __shfl_sync(0xffffffffu, sq, owner);
+    if (!sq) continue;
+    const float ev = wq / __ldg(udiag + j + qq);
+    const float* urow = H + (long long)(j + qq) * b + j;
+#pragma unroll
+    for (int i = 0; i < MAXI; ++i) {
+      const int p = lane + 32 * i;
+      if (p > qq && p < nJ) w[i] = fmaf(-ev, urow[p], w[i]);
+      if (p == qq) e[i] = ev;
+    }
+  }
+  uint8_t* mrow = mask + (long long)k * b + j;
+  float* zrow = Zs + (long long)k * B;
+#pragma unroll
+  for (int i = 0; i < MAXI; ++i) {
+    const int qq = lane + 32 * i;
+    if (qq < nJ) mrow[qq] = sel[i] ? 1 : 0;
+    if (qq < B) zrow[qq] = e[i];
+  }
+  if (lane == 0 && s > 0) atomicAdd((unsigned long long*)&ctlp->pruned, (unsigned long long)s);
+}
+
+template <int SCAP, bool NM>
+void launch_thanos_variant(int warps, const float* W, int c, int b, int j, int B, const float* Kt,
+                           const float* xnorm, Ctl* ctl, uint8_t* mask, float* Zs, int nm_n, int nm_m,
+                           int* ovf, int from_list, pwp_stats* st, cudaStream_t s) {
+  const int smem = warps * SolveSmem<SCAP>::kPerWarp * 4;
+  static bool set = false;
+  if (!set) {
+    cudaFuncSetAttribute(thanos_solve_kernel<SCAP, NM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    set = true;
+  }
+  int grid;
+  if (from_list) {
+    grid = kNumSM;
+  } else {
+    grid = (c + warps - 1) / warps;
+  }
+  thanos_solve_kernel<SCAP, NM><<<grid, warps * 32, smem, s>>>(W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n,
+                                                              nm_m, ovf, from_list, st);
+}
+
+}  // namespace
+
+// Rows whose selected set fits 80 entries go through an 8-warp CTA with 14 KB of
+// shared memory per warp; the rare larger sets (up to 128) take a second launch with
+// 35 KB per warp.
+int launch_thanos_solve(bool nm, const float* W, int c, int b, int j, int B, const float* Kt,
+                        const float* xnorm, Ctl* ctl, uint8_t* mask, float* Zs, int nm_n, int nm_m,
+                        int* ovf, pwp_stats* st, cudaStream_t s) {
+  const int s_nm = nm ? B / nm_m * (nm_m - nm_n) : 0;
+  const bool big_only = nm ? s_nm > 80 : false;
+  if (big_only) {
+    if (nm)
+      launch_thanos_variant<128, true>(4, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, ovf, 0, st, s);
+    return 1;
+  }
+  const bool need_second = !nm && B > 80;
+  if (need_second) cudaMemsetAsync(ovf, 0, sizeof(int), s);
+  if (nm)
+    launch_thanos_variant<80, true>(8, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, ovf, 0, st, s);
+  else
+    launch_thanos_variant<80, false>(8, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, ovf, 0, st, s);
+  if (need_second) {
+    launch_thanos_variant<128, false>(4, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, ovf, 1, st, s);
+    return 2;
+  }
+  return 1;
+}
+
+int launch_sparsegpt_solve(bool nm, const float* W, int c, int b, int j, int B, const float* H,
+                           const float* udiag, Ctl* ctl, uint8_t* mask, float* Zs, int nm_n, int nm_m,
+                           pwp_stats* st, cudaStream_t s) {
+  const int grid = (c + 7) / 8;
+  if (nm)
+    sparsegpt_solve_kernel<true><<<grid, 256, 0, s>>>(W, c, b, j, B, H, udiag, ctl, mask, Zs, nm_n, nm_m, st);
+  else
+    sparsegpt_solve_kernel<false><<<grid, 256, 0, s>>>(W, c, b, j, B, H, udiag, ctl, mask, Zs, nm_n, nm_m, st);
+  return 1;
+}
+
+}  // namespace pwp

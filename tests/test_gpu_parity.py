@@ -119,10 +119,12 @@ def test_hessian_matches_fp64(dtype):
     assert np.allclose(H2.cpu().numpy(), 2 * H.cpu().numpy(), rtol=1e-6, atol=0)
 
 
-def test_factor_matches_fp64():
+@pytest.mark.parametrize("b", [300, 1000, 1536])
+def test_factor_matches_fp64(b):
+    """b = 1000: ragged last panel and a ragged pair at every doubling level of the inverse."""
     torch = _torch()
     import post_weight_pruning_b200 as pwp
-    wl = synth.custom(8, 300, 900, dtype="fp32", outlier_frac=0.02, outlier_scale=20.0)
+    wl = synth.custom(8, b, 3 * b, dtype="fp32", outlier_frac=0.02, outlier_scale=20.0)
     X64 = synth.to_f64(synth.make_X_tokens(wl), "fp32")
     H = oracle.hessian(X64)
     Hd, lam = oracle.damp_hessian(H, 0.01)
