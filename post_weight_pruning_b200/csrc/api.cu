@@ -8,11 +8,13 @@ namespace pwp {
 struct PruneBuffers;
 size_t prune_ws_layout(const pwp_config* cfg, int c, int b, PruneBuffers* pb, char* base);
 cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c, int b, float* H,
-                         float* Wout, uint8_t* mask, void* ws, pwp_stats* st, cudaStream_t s);
+                         float* Wout, uint8_t* mask, void* ws, pwp_stats* st, cudaStream_t s,
+                         bool stats_ready);
 cudaError_t launch_hessian_simt(const void* X, int xtype, long long n, int b, float* H, int beta,
                                 cudaStream_t s);
 cudaError_t launch_hessian_tc(const void* X, long long n, int b, float* H, int beta, cudaStream_t s,
-                              bool* used);
+                              bool* used, pwp_stats* st);
+cudaError_t launch_stats_init(pwp_stats* st, cudaStream_t s);
 }  // namespace pwp
 
 using namespace pwp;
@@ -68,23 +70,28 @@ size_t pwp_factor_workspace_bytes(int32_t b) {
   return factor_ws_bytes(b);
 }
 
-pwp_status pwp_hessian_accumulate(const void* X, int32_t xtype, int64_t n, int32_t b, float* H,
-                                  int32_t beta, void* stream) {
-  if (!H || b < 1 || b > 16384 || n < 0 || (n > 0 && !X) || !valid_dtype(xtype) ||
-      (beta != 0 && beta != 1))
-    return PWP_EINVAL;
-  cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e;
+// H := beta*H + 2 X X^T; device-side failures go to st when it is given.
+static pwp_status hessian_impl(const void* X, int32_t xtype, int64_t n, int32_t b, float* H, int32_t beta,
+                               pwp_stats* st, cudaStream_t s) {
+  cudaError_t e = cudaSuccess;
   bool used = false;
   prof_begin(kKHessian, s);
   if (xtype == PWP_BF16) {
-    e = launch_hessian_tc(X, n, b, H, beta, s, &used);
+    e = launch_hessian_tc(X, n, b, H, beta, s, &used, st);
     if (e != cudaSuccess) return PWP_ECUDA;
   }
   if (!used) e = launch_hessian_simt(X, xtype, n, b, H, beta, s);
   prof_end(kKHessian, s);
   count_launches(1);
   return e == cudaSuccess ? PWP_OK : PWP_ECUDA;
+}
+
+pwp_status pwp_hessian_accumulate(const void* X, int32_t xtype, int64_t n, int32_t b, float* H,
+                                  int32_t beta, void* stream) {
+  if (!H || b < 1 || b > 16384 || n < 0 || (n > 0 && !X) || !valid_dtype(xtype) ||
+      (beta != 0 && beta != 1))
+    return PWP_EINVAL;
+  return hessian_impl(X, xtype, n, b, H, beta, nullptr, (cudaStream_t)stream);
 }
 
 pwp_status pwp_damp_factor(float* H, int32_t b, float damp, float* g_diag, void* ws, size_t ws_bytes,
@@ -104,7 +111,7 @@ pwp_status pwp_prune_layer(const pwp_config* cfg, const void* W, int32_t wtype, 
     return PWP_EINVAL;
   if (!ws || !aligned(ws, 256) || ws_bytes < prune_ws_layout(cfg, c, b, nullptr, nullptr))
     return PWP_EWORKSPACE;
-  cudaError_t e = launch_prune(cfg, W, wtype, c, b, H, W_out, mask, ws, st, (cudaStream_t)stream);
+  cudaError_t e = launch_prune(cfg, W, wtype, c, b, H, W_out, mask, ws, st, (cudaStream_t)stream, false);
   return e == cudaSuccess ? PWP_OK : PWP_ECUDA;
 }
 
@@ -116,9 +123,11 @@ pwp_status pwp_prune_layer_x(const pwp_config* cfg, const void* W, int32_t wtype
     return PWP_EINVAL;
   if (!ws || !aligned(ws, 256) || ws_bytes < prune_ws_layout(cfg, c, b, nullptr, nullptr))
     return PWP_EWORKSPACE;
-  pwp_status ps = pwp_hessian_accumulate(X, xtype, n, b, H, 0, stream);
+  cudaStream_t s = (cudaStream_t)stream;
+  if (launch_stats_init(st, s) != cudaSuccess) return PWP_ECUDA;
+  pwp_status ps = hessian_impl(X, xtype, n, b, H, 0, st, s);
   if (ps != PWP_OK) return ps;
-  cudaError_t e = launch_prune(cfg, W, wtype, c, b, H, W_out, mask, ws, st, (cudaStream_t)stream);
+  cudaError_t e = launch_prune(cfg, W, wtype, c, b, H, W_out, mask, ws, st, s, true);
   return e == cudaSuccess ? PWP_OK : PWP_ECUDA;
 }
 

@@ -54,65 +54,143 @@ __global__ void __launch_bounds__(1024) damp_kernel(float* __restrict__ H, int b
   for (int q = threadIdx.x; q < b; q += blockDim.x) H[(long long)q * b + q] += lam;
 }
 
-// Factor the nb x nb block held in A (symmetric, upper triangle valid) as A = V V^T, V
-// upper (last column first), and invert V.  256 threads.  On return A's upper triangle
-// holds V and Wi holds V^-1 (upper, zero below).  Returns false on a non-positive pivot.
+// Factor the nb x nb diagonal block (nb <= 64) held in A (symmetric; the upper triangle
+// is read) as A = V V^T with V upper triangular, and invert V.  256 threads.
+// Working on the reversed matrix P = J A J (J the reversal), this is the ordinary
+// Cholesky P = L L^T from the top-left, with V = J L J and V^-1 = J L^-1 J.  Each
+// thread keeps a 4x4 cyclic sub-block of P (rows ty + 16a, columns tx + 16c) in
+// registers; every pivot step needs one barrier, with the pivot column broadcast
+// through a double-buffered shared vector.  Entries beyond nb are an identity pad.
+// On return A's upper triangle holds V and Wi holds V^-1 (upper, zero below).
+// Returns false on a non-positive pivot (recorded in st).
 __device__ bool factor_diag_block(float (*A)[NB + 1], float (*Wi)[NB + 1], int nb, int* bad,
                                   pwp_stats* st) {
-  const int tid = threadIdx.x;
-  for (int i = nb - 1; i >= 0; --i) {
-    if (tid == 0) {
-      const float d = A[i][i];
-      if (!(d > 0.f) || !isfinite(d)) {
+  __shared__ float colbuf[2][NB];
+  __shared__ float Lsh[NB][NB + 1];
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int off = NB - nb;  // P[r][s] = A[nb-1-(r-off)][...] for r, s >= off; identity before
+  float P[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int r = ty + 16 * a, s = tx + 16 * c;
+      float v;
+      if (r < off || s < off) {
+        v = (r == s) ? 1.f : 0.f;
+      } else {
+        const int ar = NB - 1 - r, as = NB - 1 - s;   // A index, in [0, nb)
+        v = ar <= as ? A[ar][as] : A[as][ar];
+      }
+      P[a][c] = v;
+    }
+  if (tid == 0) *bad = 0;
+  // Cholesky of P; pivot k = 16 kb + kk keeps the register index kb a constant
+#pragma unroll
+  for (int kb = 0; kb < 4; ++kb)
+  for (int kk = 0; kk < 16; ++kk) {
+    const int k = 16 * kb + kk;
+    float* cb = colbuf[k & 1];
+    if (tx == kk) {
+#pragma unroll
+      for (int a = 0; a < 4; ++a) cb[ty + 16 * a] = P[a][kb];
+    }
+    __syncthreads();
+    const float d = cb[k];
+    if (!(d > 0.f) || !isfinite(d)) {
+      if (tid == 0) {
         *bad = 1;
         set_error(st, PWP_ENOTSPD, kSiteCholDiag);
-      } else {
-        A[i][i] = sqrtf(d);
+      }
+      return false;
+    }
+    const float lkk = sqrtf(d);
+    const float inv_d = 1.f / d;
+    float cr[4], cs[4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) cr[a] = cb[ty + 16 * a];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) cs[c] = cb[tx + 16 * c];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int r = ty + 16 * a;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int s = tx + 16 * c;
+        if (s == k && r >= k) P[a][c] = cr[a] / lkk;                 // final column k of L
+        else if (r > k && s > k) P[a][c] = fmaf(-cr[a] * inv_d, cs[c], P[a][c]);
       }
     }
-    __syncthreads();
-    if (*bad) return false;
-    const float inv = 1.f / A[i][i];
-    if (tid < i) A[tid][i] *= inv;
-    __syncthreads();
-    // rank-1 update of the leading i x i upper triangle: thread owns column s = tid & 63,
-    // rows r = (tid >> 6) + 4k
-    {
-      const int sc = tid & 63, r0 = tid >> 6;
-      if (sc < i) {
-        const float vs = A[sc][i];
-        for (int r = r0; r <= sc; r += 4) A[r][sc] = fmaf(-A[r][i], vs, A[r][sc]);
-      }
-    }
-    __syncthreads();
   }
-  // Wi = V^-1 (upper).  Diagonal first, then rows from the bottom: for row r, entries
-  // c > r: Wi[r][c] = -(sum_{t=r+1..c} V[r][t] Wi[t][c]) / V[r][r].  Threads own columns
-  // c (tid & 63) and split the sum four ways (tid >> 6).
-  if (tid < NB) {
-    for (int r = 0; r < NB; ++r) Wi[r][tid] = (r == tid && tid < nb) ? 1.f / A[tid][tid] : 0.f;
+  // L (lower) to shared memory
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int r = ty + 16 * a, s = tx + 16 * c;
+      Lsh[r][s] = r >= s ? P[a][c] : 0.f;
+    }
+  // X = L^-1 by forward substitution on all columns at once: for k: X[k][:] /= L[k][k],
+  // then X[r][:] -= L[r][k] X[k][:] for r > k.  Thread keeps the same 4x4 sub-block.
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) P[a][c] = (ty + 16 * a == tx + 16 * c) ? 1.f : 0.f;
+  __syncthreads();
+#pragma unroll
+  for (int kb = 0; kb < 4; ++kb)
+  for (int kk = 0; kk < 16; ++kk) {
+    const int k = 16 * kb + kk;
+    float* rb = colbuf[k & 1];
+    const float lkk = Lsh[k][k];
+    if (ty == kk) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        P[kb][c] = P[kb][c] / lkk;
+        rb[tx + 16 * c] = P[kb][c];
+      }
+    }
+    __syncthreads();
+    float lr[4], xs[4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) lr[a] = Lsh[ty + 16 * a][k];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) xs[c] = rb[tx + 16 * c];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      if (ty + 16 * a > k) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) P[a][c] = fmaf(-lr[a], xs[c], P[a][c]);
+      }
+    }
   }
   __syncthreads();
-  __shared__ float part[4][NB];
-  const int cc = tid & 63, qq = tid >> 6;
-  for (int r = nb - 2; r >= 0; --r) {
-    float s = 0.f;
-    if (cc > r && cc < nb)
-      for (int t = r + 1 + qq; t <= cc; t += 4) s = fmaf(A[r][t], Wi[t][cc], s);
-    part[qq][cc] = s;
-    __syncthreads();
-    if (qq == 0 && cc > r && cc < nb)
-      Wi[r][cc] = -(part[0][cc] + part[1][cc] + part[2][cc] + part[3][cc]) * Wi[r][r];
-    __syncthreads();
-  }
+  // back to A's orientation: V[i][j] = L[NB-1-i][NB-1-j], V^-1[i][j] = X[NB-1-i][NB-1-j]
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int r = ty + 16 * a, s = tx + 16 * c;
+      if (r >= off && s >= off) {                      // inside the nb block
+        const int i = NB - 1 - r, jj = NB - 1 - s;     // the same reversal as on load
+        if (i <= jj) {
+          A[i][jj] = Lsh[r][s];
+          Wi[i][jj] = P[a][c];
+        } else {
+          Wi[i][jj] = 0.f;
+        }
+      }
+    }
+  __syncthreads();
   return true;
 }
 
 // Stand-alone factorisation of the diagonal block at p0 (used for the last panel).
 __global__ void __launch_bounds__(256) chol_diag_kernel(float* __restrict__ H, int b, int p0, int nb,
                                                         float* __restrict__ Vinv, pwp_stats* st) {
-  __shared__ float A[NB][NB + 1];
-  __shared__ float Wi[NB][NB + 1];
+  extern __shared__ __align__(16) float dsm[];   // A and Wi, 2 x NB x (NB + 1) floats
+  float (*A)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(dsm);
+  float (*Wi)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(dsm + NB * (NB + 1));
   __shared__ int bad;
   if (failed(st)) return;
   if (threadIdx.x == 0) bad = 0;
@@ -339,6 +417,8 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
   static bool attr = false;
   if (!attr) {
     cudaFuncSetAttribute(chol_update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * NB * 132 * 4);
+    // 33 KB dynamic on top of 17 KB static shared memory: above the 48 KB default
+    cudaFuncSetAttribute(chol_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * NB * (NB + 1) * 4);
     attr = true;
   }
   long long nl = 0;
@@ -347,7 +427,7 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
   // factor, panels from the last; the last panel's diagonal block stands alone
   {
     const int p = np - 1, p0 = p * NB, nb = b - p0;
-    chol_diag_kernel<<<1, 256, 0, s>>>(H, b, p0, nb, Vall + (size_t)p * NB * NB, st);
+    chol_diag_kernel<<<1, 256, 2 * NB * (NB + 1) * 4, s>>>(H, b, p0, nb, Vall + (size_t)p * NB * NB, st);
     ++nl;
   }
   for (int p = np - 1; p >= 1; --p) {

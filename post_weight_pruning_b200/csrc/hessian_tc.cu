@@ -1,10 +1,340 @@
-// Hessian accumulation on the tensor cores (bf16 activations) -- placeholder that
-// declines, so the CUDA-core path runs.
+// Hessian accumulation H = beta*H + 2 X X^T on the 5th-generation tensor cores
+// (bf16 activations, fp32 accumulation in tensor memory).
+//
+// "Weight Pruning in Large Language Models ..." (llms.blog), section "SparseGPT:
+// Second-Order Reconstruction at Scale": H = 2 X X^T.  X is token-major [n, b], so
+// H[i][j] = 2 sum_t X[t][i] X[t][j] is a product whose two operands are both stored
+// feature-contiguous ("MN-major" in the tensor-core operand terminology): A[i][t] =
+// X[t][i] and B[t][j] = X[t][j] come straight from X with no transpose.
+//
+// One CTA computes one 128 x 256 tile of H (rows i0.., columns j0..) over all n tokens:
+//   - a single thread issues TMA loads of 64-feature x 64-token boxes (128-byte
+//     swizzle) into a 4-stage ring, two boxes for A and four for B per stage;
+//   - a single thread issues tcgen05.mma (M=128, N=256, K=16, bf16 x bf16 -> fp32)
+//     into a 256-column accumulator in tensor memory, four per stage, and releases each
+//     stage with tcgen05.commit;
+//   - all four warps read the accumulator back (tcgen05.ld, 32 lanes x 32 columns at a
+//     time), scale by 2 and write both H[i][j] and its mirror H[j][i] for i <= j.
+// Only tiles that hold some i <= j are launched; entries with i > j are left to their
+// mirror, so H comes out exactly symmetric.  Every wait is bounded: a wait that runs
+// out records PWP_ETIMEOUT (or, without a status word, writes NaN into the tile).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "pwp_internal.cuh"
 
 namespace pwp {
-cudaError_t launch_hessian_tc(const void*, long long, int, float*, int, cudaStream_t, bool* used) {
-  *used = false;
-  return cudaSuccess;
+namespace {
+
+constexpr int TM = 128, TN = 256, TK = 64, STAGES = 4;
+constexpr int BOX_BYTES = 64 * TK * 2;           // one 64-feature x 64-token bf16 box
+constexpr int A_BYTES = TM * TK * 2;             // 2 boxes
+constexpr int B_BYTES = TN * TK * 2;             // 4 boxes
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;   // 48 KB
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+// kind::f16 instruction descriptor: D fp32, A and B bf16, both MN-major, N = 256, M = 128
+constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
+                           ((uint32_t)(TN >> 3) << 17) | ((uint32_t)(TM >> 4) << 24);
+constexpr long long kSpinLimit = 1ll << 26;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
 }
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+// Bounded wait for the phase of the given parity to complete.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  const uint32_t addr = smem_u32(bar);
+  for (long long i = 0; i < kSpinLimit; ++i) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred P1;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
+        "selp.b32 %0, 1, 0, P1;\n\t}"
+        : "=r"(done)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+          smem_u32(dst)),
+      "l"((uint64_t)map), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle.  For MN-major operands the
+// leading offset is the distance between 64-element MN chunks and the stride offset
+// the distance between 8-row groups along K.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // descriptor version for this architecture
+  d |= (uint64_t)2 << 61;  // SWIZZLE_128B
+  return d;
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(da), "l"(db), "r"(IDESC), "r"(acc)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Tiles (I, J) of 128 rows x 256 columns that hold some entry with row <= column,
+// enumerated column-tile by column-tile: I < 2J + 2.
+__host__ __device__ inline int tile_count(int b) {
+  const int nI = (b + TM - 1) / TM, nJ = (b + TN - 1) / TN;
+  int cnt = 0;
+  for (int J = 0; J < nJ; ++J) cnt += min(nI, 2 * J + 2);
+  return cnt;
+}
+
+__device__ inline void tile_of(int idx, int b, int& I, int& J) {
+  const int nI = (b + TM - 1) / TM;
+  J = 0;
+  while (true) {
+    const int cnt = min(nI, 2 * J + 2);
+    if (idx < cnt) break;
+    idx -= cnt;
+    ++J;
+  }
+  I = idx;
+}
+
+__global__ void __launch_bounds__(128, 1) syrk_tc_kernel(const __grid_constant__ CUtensorMap tmap, long long n,
+                                                         int b, float* __restrict__ H, int beta, pwp_stats* st) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* done = empty + STAGES;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int I, J;
+  tile_of(blockIdx.x, b, I, J);
+  const int i0 = I * TM, j0 = J * TN;
+  const int nk = (int)((n + TK - 1) / TK);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(done, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    abort_flag = 0;
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_slot)),
+                 "r"(TN)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&tmap) : "memory");
+      int issued = 0;
+      for (int kt = 0; kt < nk; ++kt) {
+        const int s = kt % STAGES;
+        if (kt >= STAGES && !mbar_wait(&empty[s], ((kt / STAGES) - 1) & 1)) {
+          abort_flag = 1;
+          break;
+        }
+        mbar_expect_tx(&full[s], STAGE_BYTES);
+        uint8_t* a = smem + s * STAGE_BYTES;
+        uint8_t* bb = a + A_BYTES;
+        const int y = kt * TK;
+        tma_load_2d(a, &tmap, &full[s], i0, y);
+        tma_load_2d(a + BOX_BYTES, &tmap, &full[s], i0 + 64, y);
+#pragma unroll
+        for (int h = 0; h < 4; ++h) tma_load_2d(bb + h * BOX_BYTES, &tmap, &full[s], j0 + 64 * h, y);
+        issued = kt + 1;
+      }
+      // on an abort, let the copies already in flight land before the CTA exits
+      if (abort_flag) {
+        for (int kt = issued - STAGES > 0 ? issued - STAGES : 0; kt < issued; ++kt)
+          mbar_wait(&full[kt % STAGES], (kt / STAGES) & 1);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t sbase = smem_u32(smem);
+      bool ok = true;
+      for (int kt = 0; kt < nk; ++kt) {
+        const int s = kt % STAGES;
+        if (!mbar_wait(&full[s], (kt / STAGES) & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_addr = sbase + s * STAGE_BYTES;
+        const uint32_t b_addr = a_addr + A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < TK / 16; ++kk) {
+          const uint64_t da = sw128_desc(a_addr + kk * 2048, BOX_BYTES, 1024);
+          const uint64_t db = sw128_desc(b_addr + kk * 2048, BOX_BYTES, 1024);
+          mma_bf16(tmem, da, db, (kt | kk) != 0 ? 1u : 0u);
+        }
+        mma_commit(&empty[s]);
+      }
+      if (ok) mma_commit(done);
+      else abort_flag = 1;
+    }
+    __syncwarp();
+  }
+
+  // epilogue: warp w owns accumulator lanes (tile rows) 32w .. 32w + 31
+  bool have = mbar_wait(done, 0);
+  __syncwarp();
+  have = __all_sync(0xffffffffu, have && !*((volatile int*)&abort_flag));
+  tc_fence_after();
+  const int r = i0 + warp * 32 + lane;
+  if (!have) {
+    if (threadIdx.x == 0) {
+      if (st) set_error(st, PWP_ETIMEOUT, 6);
+    }
+    if (!st && r < b) {
+      for (int c = j0; c < min(b, j0 + TN); ++c)
+        if (r <= c) H[(long long)r * b + c] = __int_as_float(0x7fc00000);
+    }
+  } else {
+#pragma unroll 1
+    for (int ch = 0; ch < TN / 32; ++ch) {
+      float v[32];
+      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(ch * 32), v);
+      const int c0 = j0 + ch * 32;
+      if (c0 >= b || r >= b) continue;
+      // direct row: this thread's 32 consecutive columns, 16-byte stores where whole
+      float* hr = H + (long long)r * b + c0;
+      const bool vec = ((b & 3) == 0) && (r <= c0) && (c0 + 32 <= b);
+      if (vec) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          float4 o = make_float4(2.f * v[4 * q], 2.f * v[4 * q + 1], 2.f * v[4 * q + 2], 2.f * v[4 * q + 3]);
+          if (beta) {
+            const float4 old = *reinterpret_cast<const float4*>(hr + 4 * q);
+            o.x += old.x; o.y += old.y; o.z += old.z; o.w += old.w;
+          }
+          *reinterpret_cast<float4*>(hr + 4 * q) = o;
+          v[4 * q] = o.x; v[4 * q + 1] = o.y; v[4 * q + 2] = o.z; v[4 * q + 3] = o.w;
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          const int c = c0 + k;
+          if (c < b && r <= c) {
+            const float val = beta ? hr[k] + 2.f * v[k] : 2.f * v[k];
+            hr[k] = val;
+            v[k] = val;
+          }
+        }
+      }
+      // mirror: for each column, the warp writes 32 consecutive row entries
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        const int c = c0 + k;
+        if (c < b && r < c) H[(long long)c * b + r] = v[k];
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TN) : "memory");
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+}  // namespace
+
+// Declines (used = false) when the shape does not meet the TMA rules (row stride a
+// multiple of 16 bytes, 16-byte aligned base) or there is nothing to accumulate.
+cudaError_t launch_hessian_tc(const void* X, long long n, int b, float* H, int beta, cudaStream_t s, bool* used,
+                              pwp_stats* st) {
+  *used = false;
+  if (n < 1 || b < 1 || (b % 8) != 0 || ((uintptr_t)X % 16) != 0 || n > 0x7fffffffLL) return cudaSuccess;
+  PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode();
+  if (!encode) return cudaSuccess;
+  CUtensorMap map;
+  cuuint64_t dims[2] = {(cuuint64_t)b, (cuuint64_t)n};
+  cuuint64_t strides[1] = {(cuuint64_t)b * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)TK};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult cr = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(X), dims, strides, box, estr,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) return cudaSuccess;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(syrk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  syrk_tc_kernel<<<tile_count(b), 128, SMEM_BYTES, s>>>(map, n, b, H, beta, st);
+  *used = true;
+  return cudaGetLastError();
+}
+
 }  // namespace pwp

@@ -19,7 +19,8 @@ namespace pwp {
 struct PruneBuffers;
 size_t prune_ws_layout(const pwp_config* cfg, int c, int b, PruneBuffers* pb, char* base);
 cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c, int b, float* H,
-                         float* Wout, uint8_t* mask, void* ws, pwp_stats* st, cudaStream_t s);
+                         float* Wout, uint8_t* mask, void* ws, pwp_stats* st, cudaStream_t s,
+                         bool stats_ready);
 }  // namespace pwp
 
 namespace {
@@ -63,6 +64,6 @@ extern "C" pwp_status pwp_prune_layer_noalloc(const pwp_config* cfg, const void*
   cudaStream_t s = (cudaStream_t)stream;
   // The array keeps whatever the previous call left in it; start from zeros.
   if (cudaMemsetAsync(ws, 0, need, s) != cudaSuccess) return PWP_ECUDA;
-  cudaError_t e = pwp::launch_prune(cfg, W, wtype, c, b, H, W_out, mask, ws, st, s);
+  cudaError_t e = pwp::launch_prune(cfg, W, wtype, c, b, H, W_out, mask, ws, st, s, false);
   return e == cudaSuccess ? PWP_OK : PWP_ECUDA;
 }

@@ -23,18 +23,22 @@ namespace pwp {
 
 // ------------------------------------------------------------------ setup kernels
 
-__global__ void init_ctl_kernel(Ctl* ctl, long long zstar, pwp_stats* st, long long target) {
-  ctl->zstar = zstar;
-  ctl->pruned = 0;
-  ctl->mode = 0;
+__global__ void init_stats_kernel(pwp_stats* st) {
   st->status = PWP_OK;
   st->status_site = 0;
   st->pruned = 0;
-  st->target = target;
+  st->target = 0;
   st->lambda = 0.f;
   st->shortfall = 0;
   st->reread_blocks = 0;
   st->tie_blocks = 0;
+}
+
+__global__ void init_ctl_kernel(Ctl* ctl, long long zstar, pwp_stats* st, long long target) {
+  ctl->zstar = zstar;
+  ctl->pruned = 0;
+  ctl->mode = 0;
+  st->target = target;
 }
 
 __global__ void convert_w_kernel(const void* __restrict__ W, int wtype, float* __restrict__ Wout,
@@ -273,8 +277,17 @@ static void launch_stream(float* W, int c, int b, int u0, int j, int col_end, co
                                                              r_upper_from, mask, sc, hist_end, hist1, st);
 }
 
+cudaError_t launch_stats_init(pwp_stats* st, cudaStream_t s) {
+  init_stats_kernel<<<1, 1, 0, s>>>(st);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+// stats_ready: the caller already reset *st on this stream (and may have recorded an
+// earlier device-side failure in it, which then turns this call's kernels into no-ops).
 cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c, int b, float* H,
-                         float* Wout, uint8_t* mask, void* ws, pwp_stats* st, cudaStream_t s) {
+                         float* Wout, uint8_t* mask, void* ws, pwp_stats* st, cudaStream_t s,
+                         bool stats_ready) {
   PruneBuffers pb;
   const int B = cfg->block;
   prune_ws_layout(cfg, c, b, &pb, (char*)ws);
@@ -303,6 +316,10 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
     g_nsm = nsm;
   }
   long long nl = 0;
+  if (!stats_ready) {
+    init_stats_kernel<<<1, 1, 0, s>>>(st);
+    ++nl;
+  }
   init_ctl_kernel<<<1, 1, 0, s>>>(pb.ctl, zstar, st, target);
   cudaMemsetAsync(pb.hist1, 0, sizeof(unsigned int) * kHist1Bins, s);
   convert_w_kernel<<<4 * g_nsm, 256, 0, s>>>(W, wtype, Wout, N);

@@ -100,11 +100,13 @@ def test_zero_sparsity_is_identity():
     assert np.array_equal(W_hat, synth.to_f64(W, "bf16"))
 
 
-@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
-def test_hessian_matches_fp64(dtype):
+@pytest.mark.parametrize("dtype,b,n", [("fp32", 200, 700), ("bf16", 200, 700), ("bf16", 1024, 2048),
+                                       ("bf16", 264, 130), ("bf16", 1000, 64)])
+def test_hessian_matches_fp64(dtype, b, n):
+    """bf16 runs on the tensor cores: several 128x256 tiles, ragged feature and token edges."""
     torch = _torch()
     import post_weight_pruning_b200 as pwp
-    wl = synth.custom(8, 200, 700, dtype=dtype, outlier_frac=0.02, outlier_scale=50.0)
+    wl = synth.custom(8, b, n, dtype=dtype, outlier_frac=0.02, outlier_scale=50.0)
     X = synth.make_X_tokens(wl)
     _, Xt = P.torch_inputs(synth.make_W(wl), X, dtype)
     H = pwp.hessian_accumulate(Xt)
