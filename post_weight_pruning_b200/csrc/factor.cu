@@ -104,23 +104,24 @@ __device__ bool factor_diag_block(float (*A)[NB + 1], float (*Wi)[NB + 1], int n
       }
       return false;
     }
-    const float lkk = sqrtf(d);
-    const float inv_d = 1.f / d;
-    float cr[4], cs[4];
+    const float inv_l = 1.f / sqrtf(d);
+    const float inv_d = inv_l * inv_l;
+    float lr[4], cs[4];
 #pragma unroll
-    for (int a = 0; a < 4; ++a) cr[a] = cb[ty + 16 * a];
+    for (int a = 0; a < 4; ++a) lr[a] = cb[ty + 16 * a] * inv_l;    // L[r][k]
 #pragma unroll
-    for (int c = 0; c < 4; ++c) cs[c] = cb[tx + 16 * c];
+    for (int c = 0; c < 4; ++c) cs[c] = cb[tx + 16 * c] * inv_l;    // L[s][k]
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
       const int r = ty + 16 * a;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int s = tx + 16 * c;
-        if (s == k && r >= k) P[a][c] = cr[a] / lkk;                 // final column k of L
-        else if (r > k && s > k) P[a][c] = fmaf(-cr[a] * inv_d, cs[c], P[a][c]);
+        if (s == k && r >= k) P[a][c] = lr[a];                       // final column k of L
+        else if (r > k && s > k) P[a][c] = fmaf(-lr[a], cs[c], P[a][c]);
       }
     }
+    (void)inv_d;
   }
   // L (lower) to shared memory
 #pragma unroll
@@ -142,11 +143,11 @@ __device__ bool factor_diag_block(float (*A)[NB + 1], float (*Wi)[NB + 1], int n
   for (int kk = 0; kk < 16; ++kk) {
     const int k = 16 * kb + kk;
     float* rb = colbuf[k & 1];
-    const float lkk = Lsh[k][k];
     if (ty == kk) {
+      const float ilkk = 1.f / Lsh[k][k];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        P[kb][c] = P[kb][c] / lkk;
+        P[kb][c] = P[kb][c] * ilkk;
         rb[tx + 16 * c] = P[kb][c];
       }
     }
@@ -242,7 +243,22 @@ __global__ void __launch_bounds__(256) chol_update_kernel(float* __restrict__ H,
   __shared__ int bad;
   if (failed(st)) return;
   const int nT = (p0 + 127) / 128;
-  int I = 0, rem = blockIdx.x;
+  // blockIdx 0 takes the tile holding the next panel's diagonal block, so its serial
+  // factorisation starts first and overlaps the other tiles; that tile's own slot in
+  // the upper-triangle enumeration goes to blockIdx 0's original tile.
+  const int q0 = p0 - NB;
+  int look = -1;
+  if (q0 >= 0) {
+    const int Id = q0 / 128;  // diagonal tile (Id, Id)
+    look = 0;
+    for (int i = 0; i < Id; ++i) look += nT - i;
+  }
+  int slot = blockIdx.x;
+  if (look >= 0) {
+    if (slot == 0) slot = look;
+    else if (slot == look) slot = 0;
+  }
+  int I = 0, rem = slot;
   while (rem >= nT - I) { rem -= nT - I; ++I; }
   const int J = I + rem;
   const int i0 = I * 128, j0 = J * 128;
@@ -283,7 +299,6 @@ __global__ void __launch_bounds__(256) chol_update_kernel(float* __restrict__ H,
     }
   }
   // look-ahead: factor the next panel's diagonal block if this tile holds it
-  const int q0 = p0 - NB;
   if (q0 < 0 || I != J || q0 < i0 || q0 >= i0 + 128) return;
   __syncthreads();  // this CTA's own writes to H are visible to its threads
   float (*A)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(fsm);

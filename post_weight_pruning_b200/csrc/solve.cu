@@ -33,17 +33,27 @@ struct SolveSmem {
 // Cholesky R-hat = L L^T (left-looking, 4-column panels; lanes own rows) with u carried
 // as an extra row so that the factorisation also gives y = L^-1 u, then L^T z = y.
 // L holds R-hat's lower triangle on entry; y holds u.  On return y[0..s) = z.
-// Returns false on a non-positive pivot.  Whole warp, uniform control flow.
+// Per panel [jp, jp+4): every row i >= jp (the u row included) first takes the
+// contributions of columns < jp (float4 dot products against the four panel rows),
+// the 4x4 diagonal block is factored in the registers of lanes 0..3 with shuffles,
+// and every other row finishes its four panel entries by a 4x4 forward substitution.
+// One __syncwarp per panel.  Returns false on a non-positive pivot (uniform).
+template <int SCAP>
 __device__ bool chol_solve(float* __restrict__ L, float* __restrict__ y, int s, int lane) {
+  constexpr int MAXR = (SCAP + 1 + 31) / 32;   // rows jp..s over the 32 lanes
   for (int jp = 0; jp < s; jp += 4) {
-    if (jp > 0) {
-      const float* p0 = L + poff(jp);
-      const float* p1 = L + poff(jp + 1);
-      const float* p2 = L + poff(jp + 2);
-      const float* p3 = L + poff(jp + 3);
-      for (int i = jp + lane; i <= s; i += 32) {
-        float* ri = (i < s) ? L + poff(i) : y;
-        float a0 = ri[jp], a1 = ri[jp + 1], a2 = ri[jp + 2], a3 = ri[jp + 3];
+    const float* p0 = L + poff(jp);
+    const float* p1 = L + poff(jp + 1);
+    const float* p2 = L + poff(jp + 2);
+    const float* p3 = L + poff(jp + 3);
+    float acc[MAXR][4];
+#pragma unroll
+    for (int r = 0; r < MAXR; ++r) {
+      const int i = jp + lane + 32 * r;
+      if (i <= s) {
+        const float* ri = (i < s) ? L + poff(i) : y;
+        const float4 a = *reinterpret_cast<const float4*>(ri + jp);
+        float a0 = a.x, a1 = a.y, a2 = a.z, a3 = a.w;
 #pragma unroll 2
         for (int t = 0; t < jp; t += 4) {
           const float4 x = *reinterpret_cast<const float4*>(ri + t);
@@ -56,43 +66,81 @@ __device__ bool chol_solve(float* __restrict__ L, float* __restrict__ y, int s, 
           a2 = fmaf(-x.x, q2.x, a2); a2 = fmaf(-x.y, q2.y, a2); a2 = fmaf(-x.z, q2.z, a2); a2 = fmaf(-x.w, q2.w, a2);
           a3 = fmaf(-x.x, q3.x, a3); a3 = fmaf(-x.y, q3.y, a3); a3 = fmaf(-x.z, q3.z, a3); a3 = fmaf(-x.w, q3.w, a3);
         }
-        ri[jp] = a0;
-        ri[jp + 1] = a1;
-        ri[jp + 2] = a2;
-        ri[jp + 3] = a3;
+        acc[r][0] = a0; acc[r][1] = a1; acc[r][2] = a2; acc[r][3] = a3;
+      } else {
+        acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
       }
-      __syncwarp();
     }
-    const int pend = min(jp + 4, s);
-    for (int a = jp; a < pend; ++a) {
-      const float d = L[poff(a) + a];
-      if (!(d > 0.f)) return false;
-      const float l = sqrtf(d);
-      const float inv = 1.f / l;
-      __syncwarp();
-      for (int i = a + 1 + lane; i <= s; i += 32) {
-        float* ri = (i < s) ? L + poff(i) : y;
-        ri[a] *= inv;
-      }
-      if (lane == 0) L[poff(a) + a] = l;
-      __syncwarp();
-      if (a + 1 < pend) {
-        for (int i = a + 1 + lane; i <= s; i += 32) {
-          float* ri = (i < s) ? L + poff(i) : y;
-          const float lia = ri[a];
-          const int cend = (i < s) ? min(pend - 1, i) : pend - 1;
-          for (int cc = a + 1; cc <= cend; ++cc) ri[cc] = fmaf(-lia, L[poff(cc) + a], ri[cc]);
+    const int pw = min(4, s - jp);
+    // 4x4 diagonal block: rows jp..jp+pw-1 are acc[0] of lanes 0..pw-1
+    float il[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      il[c] = 1.f;
+      if (c < pw) {
+        const float d = __shfl_sync(0xffffffffu, acc[0][c], c);
+        if (!(d > 0.f)) return false;
+        const float l = sqrtf(d);
+        il[c] = 1.f / l;
+        if (lane == c) acc[0][c] = l;
+        else if (lane > c && lane < pw) acc[0][c] *= il[c];
+#pragma unroll
+        for (int c2 = c + 1; c2 < 4; ++c2) {
+          const float lc2 = __shfl_sync(0xffffffffu, acc[0][c], c2);   // L[jp+c2][jp+c]
+          if (lane >= c2 && lane < pw) acc[0][c2] = fmaf(-acc[0][c], lc2, acc[0][c2]);
         }
-        __syncwarp();
       }
     }
-  }
-  for (int a = s - 1; a >= 0; --a) {
-    const float za = y[a] / L[poff(a) + a];
+    // the factored block, broadcast: Ld[c][c2] = L[jp+c][jp+c2], c2 <= c
+    float Ld[4][4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+      for (int c2 = 0; c2 < 4; ++c2) Ld[c][c2] = (c2 <= c) ? __shfl_sync(0xffffffffu, acc[0][c2], c) : 0.f;
+    // finish the panel entries of every row below the block and write back
+#pragma unroll
+    for (int r = 0; r < MAXR; ++r) {
+      const int i = jp + lane + 32 * r;
+      if (i > s) continue;
+      float* ri = (i < s) ? L + poff(i) : y;
+      float4 o;
+      if (i < jp + pw && i < s) {
+        o = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+      } else {
+        const float x0 = acc[r][0] * il[0];
+        const float x1 = (acc[r][1] - x0 * Ld[1][0]) * il[1];
+        const float x2 = (acc[r][2] - x0 * Ld[2][0] - x1 * Ld[2][1]) * il[2];
+        const float x3 = (acc[r][3] - x0 * Ld[3][0] - x1 * Ld[3][1] - x2 * Ld[3][2]) * il[3];
+        o = make_float4(x0, x1, x2, x3);
+      }
+      *reinterpret_cast<float4*>(ri + jp) = o;
+    }
     __syncwarp();
-    const float* ra = L + poff(a);
-    for (int t = lane; t < a; t += 32) y[t] = fmaf(-ra[t], za, y[t]);
-    if (lane == 0) y[a] = za;
+  }
+  // back substitution L^T z = y, four rows at a time from the bottom
+  for (int a0 = (s - 1) & ~3; a0 >= 0; a0 -= 4) {
+    const int pw = min(4, s - a0);
+    float z[4];
+#pragma unroll
+    for (int c = 3; c >= 0; --c) {
+      z[c] = 0.f;
+      if (c < pw) {
+        float v = y[a0 + c];
+#pragma unroll
+        for (int c2 = c + 1; c2 < 4; ++c2)
+          if (c2 < pw) v = fmaf(-L[poff(a0 + c2) + a0 + c], z[c2], v);
+        z[c] = v / L[poff(a0 + c) + a0 + c];
+      }
+    }
+    __syncwarp();
+    for (int t = lane; t < a0; t += 32) {
+      float v = y[t];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        if (c < pw) v = fmaf(-L[poff(a0 + c) + t], z[c], v);
+      y[t] = v;
+    }
+    if (lane < pw) y[a0 + lane] = z[lane];
     __syncwarp();
   }
   return true;
@@ -184,7 +232,7 @@ __global__ void __launch_bounds__(256) thanos_solve_kernel(const float* __restri
         }
       }
       __syncwarp();
-      ok = chol_solve(L, y, s, lane);
+      ok = chol_solve<SCAP>(L, y, s, lane);
       if (!ok && lane == 0) set_error(st, PWP_ENOTSPD, kSiteSolve);
       if (lane == 0) atomicAdd((unsigned long long*)&ctlp->pruned, (unsigned long long)s);
     }
