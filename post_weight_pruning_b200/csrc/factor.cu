@@ -193,7 +193,7 @@ __global__ void __launch_bounds__(256) chol_diag_kernel(float* __restrict__ H, i
   float (*A)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(dsm);
   float (*Wi)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(dsm + NB * (NB + 1));
   __shared__ int bad;
-  if (failed(st)) return;
+  if (cta_failed(st)) return;
   if (threadIdx.x == 0) bad = 0;
   for (int idx = threadIdx.x; idx < nb * nb; idx += blockDim.x) {
     int r = idx / nb, s = idx % nb;
@@ -214,7 +214,7 @@ __global__ void __launch_bounds__(256) chol_panel_kernel(float* __restrict__ H, 
                                                          const pwp_stats* st) {
   __shared__ float Wi[NB][NB + 1];
   __shared__ float rowbuf[8][NB];
-  if (failed(st)) return;
+  if (cta_failed(st)) return;
   for (int idx = threadIdx.x; idx < NB * NB; idx += blockDim.x) Wi[idx / NB][idx % NB] = Vinv[idx];
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(256) chol_update_kernel(float* __restrict__ H,
   float (*As)[128 + 4] = reinterpret_cast<float (*)[132]>(fsm);               // [NB][132], k-major
   float (*Bs)[128 + 4] = reinterpret_cast<float (*)[132]>(fsm + NB * 132);
   __shared__ int bad;
-  if (failed(st)) return;
+  if (cta_failed(st)) return;
   const int nT = (p0 + 127) / 128;
   // blockIdx 0 takes the tile holding the next panel's diagonal block, so its serial
   // factorisation starts first and overlaps the other tiles; that tile's own slot in
@@ -321,7 +321,7 @@ __global__ void __launch_bounds__(256) chol_update_kernel(float* __restrict__ H,
 // matrix has the inverses of its diagonal blocks on its block diagonal).
 __global__ void put_diag_inverses_kernel(float* __restrict__ H, int b, const float* __restrict__ Vall,
                                          const pwp_stats* st) {
-  if (failed(st)) return;
+  if (cta_failed(st)) return;
   const int p = blockIdx.x;
   const int p0 = p * NB, nb = min(NB, b - p0);
   const float* V = Vall + (size_t)p * NB * NB;
@@ -348,7 +348,7 @@ struct TriGemm {
 __global__ void __launch_bounds__(256) trigemm_kernel(TriGemm g, const pwp_stats* st) {
   __shared__ __align__(16) float As[16][128 + 4];
   __shared__ __align__(16) float Bs[16][128 + 4];
-  if (failed(st)) return;
+  if (cta_failed(st)) return;
   const float* A = g.A + blockIdx.z * g.batch_a;
   const float* B = g.B + blockIdx.z * g.batch_b;
   float* C = g.C + blockIdx.z * g.batch_c;

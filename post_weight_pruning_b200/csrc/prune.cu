@@ -70,7 +70,7 @@ __global__ void prep_diag_kernel(const float* __restrict__ H, int b, const float
 __global__ void __launch_bounds__(256) kmat_kernel(const float* __restrict__ H, int b, int B,
                                                    float* __restrict__ K_all, const pwp_stats* st) {
   extern __shared__ __align__(16) float sm[];
-  if (failed(st)) return;
+  if (cta_failed(st)) return;
   const int t = blockIdx.y;
   const int j = t * B, nJ = min(B, b - j);
   const int q0 = j + blockIdx.x * 128;
@@ -132,7 +132,7 @@ __global__ void __launch_bounds__(256) stream_kernel(float* __restrict__ W, int 
   extern __shared__ unsigned int shist[];  // kHist1Bins when SCORE != 0
   __shared__ float Zs[64][33];
   __shared__ __align__(16) float Rs[32][128];
-  if (failed(st)) return;
+  if (cta_failed(st)) return;
   const int tid = threadIdx.x;
   const int tx = tid & 15, ty = tid >> 4;
   if (SCORE != kNoScore)
@@ -229,7 +229,6 @@ struct PruneBuffers {
   float* udiag;
   float* Zs;
   float* K;
-  int* ovf;
   void* fws;
   size_t fws_bytes;
 };
@@ -255,7 +254,6 @@ size_t prune_ws_layout(const pwp_config* cfg, int c, int b, PruneBuffers* pb, ch
   t.udiag = (float*)take(sizeof(float) * b);
   t.Zs = (float*)take(sizeof(float) * (size_t)c * B);
   t.K = thanos ? (float*)take(sizeof(float) * (size_t)nblk * B * b) : nullptr;
-  t.ovf = (int*)take(sizeof(int) * ((size_t)c + 1));
   t.fws_bytes = factor_ws_bytes(b);
   t.fws = take(t.fws_bytes);
   if (pb) *pb = t;
@@ -374,7 +372,7 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
     prof_begin(kKSolve, s);
     if (thanos)
       nl += launch_thanos_solve(nm, Wout, c, b, j, B, pb.K + (size_t)t * B * b, pb.xnorm, pb.ctl, mask, pb.Zs,
-                                cfg->nm_n, cfg->nm_m, pb.ovf, st, s);
+                                cfg->nm_n, cfg->nm_m, st, s);
     else
       nl += launch_sparsegpt_solve(nm, Wout, c, b, j, B, H, pb.udiag, pb.ctl, mask, pb.Zs, cfg->nm_n,
                                    cfg->nm_m, st, s);

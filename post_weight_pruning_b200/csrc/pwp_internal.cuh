@@ -40,6 +40,24 @@ __device__ __forceinline__ bool failed(const pwp_stats* st) {
   return *((volatile const int32_t*)&st->status) != PWP_OK;
 }
 
+// The early-exit checks below must give every thread of a CTA (or of a warp, for
+// kernels that only synchronise within warps) the same answer: another CTA may record
+// an error while this one starts, and a thread that returned while its neighbours go
+// on to a barrier or a full-mask shuffle would leave them waiting forever.
+__device__ __forceinline__ bool cta_failed(const pwp_stats* st) {
+  __shared__ int f;
+  __syncthreads();
+  if (threadIdx.x == 0) f = failed(st) ? 1 : 0;
+  __syncthreads();
+  return f != 0;
+}
+
+__device__ __forceinline__ bool warp_failed(const pwp_stats* st) {
+  int f = 0;
+  if ((threadIdx.x & 31) == 0) f = failed(st) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, f, 0) != 0;
+}
+
 __device__ __forceinline__ void set_error(pwp_stats* st, int status, int site) {
   if (atomicCAS((int*)&st->status, PWP_OK, status) == PWP_OK) st->status_site = site;
 }
@@ -111,7 +129,7 @@ void launch_pick2(int score, Ctl* ctl, const unsigned int* hist2, const float* W
 // per-row work of one block (solve.cu); returns the number of kernels launched
 int launch_thanos_solve(bool nm, const float* W, int c, int b, int j, int B, const float* Kt,
                         const float* xnorm, Ctl* ctl, uint8_t* mask, float* Zs, int nm_n, int nm_m,
-                        int* ovf, pwp_stats* st, cudaStream_t s);
+                        pwp_stats* st, cudaStream_t s);
 int launch_sparsegpt_solve(bool nm, const float* W, int c, int b, int j, int B, const float* H,
                            const float* udiag, Ctl* ctl, uint8_t* mask, float* Zs, int nm_n,
                            int nm_m, pwp_stats* st, cudaStream_t s);

@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(1024) pick1_kernel(Ctl* ctl, unsigned int* __r
   __shared__ long long sh_warp[32];
   __shared__ int sh_sel;
   __shared__ long long sh_base, s_take;
-  if (failed(st)) return;
+  if (cta_failed(st)) return;
   if (threadIdx.x == 0) {
     long long r = global_budget ? ctl->zstar - ctl->pruned : quota;
     long long take = r < region_n ? r : region_n;
@@ -137,7 +137,7 @@ __global__ void __launch_bounds__(256) refine_kernel(const float* __restrict__ W
                                                      const Ctl* __restrict__ ctl,
                                                      unsigned int* __restrict__ hist2,
                                                      const pwp_stats* st) {
-  if (failed(st) || ctl->mode == 0) return;
+  if (cta_failed(st) || ctl->mode == 0) return;
   const unsigned int b1 = ctl->b1;
   for (int r = blockIdx.x; r < c; r += gridDim.x) {
     const float* wr = W + (long long)r * b;
@@ -159,7 +159,7 @@ __global__ void __launch_bounds__(1024) pick2_kernel(Ctl* ctl, const unsigned in
   __shared__ unsigned int colcnt[kMaxBlock];
   __shared__ int s_qstar;
   __shared__ long long s_need;
-  if (failed(st) || ctl->mode == 0) return;
+  if (cta_failed(st) || ctl->mode == 0) return;
   const int tid = threadIdx.x;
   const long long r1 = ctl->r1;
   int lo;

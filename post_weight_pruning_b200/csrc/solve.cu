@@ -74,12 +74,13 @@ __device__ bool chol_solve(float* __restrict__ L, float* __restrict__ y, int s, 
     const int pw = min(4, s - jp);
     // 4x4 diagonal block: rows jp..jp+pw-1 are acc[0] of lanes 0..pw-1
     float il[4];
+    bool ok = true;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       il[c] = 1.f;
       if (c < pw) {
         const float d = __shfl_sync(0xffffffffu, acc[0][c], c);
-        if (!(d > 0.f)) return false;
+        if (!(d > 0.f)) { ok = false; break; }
         const float l = sqrtf(d);
         il[c] = 1.f / l;
         if (lane == c) acc[0][c] = l;
@@ -97,6 +98,7 @@ __device__ bool chol_solve(float* __restrict__ L, float* __restrict__ y, int s, 
     for (int c = 0; c < 4; ++c)
 #pragma unroll
       for (int c2 = 0; c2 < 4; ++c2) Ld[c][c2] = (c2 <= c) ? __shfl_sync(0xffffffffu, acc[0][c2], c) : 0.f;
+    if (!ok) return false;
     // finish the panel entries of every row below the block and write back
 #pragma unroll
     for (int r = 0; r < MAXR; ++r) {
@@ -146,9 +148,7 @@ __device__ bool chol_solve(float* __restrict__ L, float* __restrict__ y, int s, 
   return true;
 }
 
-// One warp per row.  Rows whose selected set exceeds SCAP are appended to the
-// overflow list ovf (ovf[0] = count, ovf[1..] = rows) for a second pass with a larger
-// SCAP; when rows_from_list is set, the rows come from that list.
+// One warp per row; SCAP bounds the selected set (and sizes the per-warp shared memory).
 template <int SCAP, bool NM>
 __global__ void __launch_bounds__(256) thanos_solve_kernel(const float* __restrict__ W, int c, int b,
                                                            int j, int B, const float* __restrict__ Kt,
@@ -156,10 +156,9 @@ __global__ void __launch_bounds__(256) thanos_solve_kernel(const float* __restri
                                                            Ctl* __restrict__ ctlp,
                                                            uint8_t* __restrict__ mask,
                                                            float* __restrict__ Zs, int nm_n, int nm_m,
-                                                           int* __restrict__ ovf, int rows_from_list,
                                                            pwp_stats* st) {
   extern __shared__ __align__(16) float smem[];
-  if (failed(st)) return;
+  if (warp_failed(st)) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nwarps = blockDim.x >> 5;
   float* L = smem + warp * SolveSmem<SCAP>::kPerWarp;
@@ -167,10 +166,8 @@ __global__ void __launch_bounds__(256) thanos_solve_kernel(const float* __restri
   int* Qidx = reinterpret_cast<int*>(y + SolveSmem<SCAP>::kY);
   const Ctl ctl = *ctlp;
   const int nJ = min(B, b - j);
-  const int nrows = rows_from_list ? *((volatile int*)ovf) : c;
   constexpr int MAXI = kMaxBlock / 32;
-  for (int idx = blockIdx.x * nwarps + warp; idx < nrows; idx += gridDim.x * nwarps) {
-    const int k = rows_from_list ? ovf[1 + idx] : idx;
+  for (int k = blockIdx.x * nwarps + warp; k < c; k += gridDim.x * nwarps) {
     const float* wrow = W + (long long)k * b + j;
     float w[MAXI];
     bool sel[MAXI];
@@ -187,11 +184,8 @@ __global__ void __launch_bounds__(256) thanos_solve_kernel(const float* __restri
       pos[i] = s + __popc(bal & ((1u << lane) - 1u));
       s += __popc(bal);
     }
-    if (s > SCAP) {
-      if (lane == 0) {
-        int at = atomicAdd(ovf, 1);
-        ovf[1 + at] = k;
-      }
+    if (s > SCAP) {   // cannot happen: the launcher picks SCAP >= the block's largest set
+      if (lane == 0) set_error(st, PWP_EINVAL, kSiteSolve);
       continue;
     }
     uint8_t* mrow = mask + (long long)k * b + j;
@@ -257,7 +251,7 @@ __global__ void __launch_bounds__(256) sparsegpt_solve_kernel(const float* __res
                                                               uint8_t* __restrict__ mask,
                                                               float* __restrict__ Zs, int nm_n, int nm_m,
                                                               pwp_stats* st) {
-  if (failed(st)) return;
+  if (warp_failed(st)) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int k = blockIdx.x * (blockDim.x >> 5) + warp;
   if (k >= c) return;
@@ -311,47 +305,37 @@ __global__ void __launch_bounds__(256) sparsegpt_solve_kernel(const float* __res
 template <int SCAP, bool NM>
 void launch_thanos_variant(int warps, const float* W, int c, int b, int j, int B, const float* Kt,
                            const float* xnorm, Ctl* ctl, uint8_t* mask, float* Zs, int nm_n, int nm_m,
-                           int* ovf, int from_list, pwp_stats* st, cudaStream_t s) {
+                           pwp_stats* st, cudaStream_t s) {
   const int smem = warps * SolveSmem<SCAP>::kPerWarp * 4;
   static bool set = false;
   if (!set) {
     cudaFuncSetAttribute(thanos_solve_kernel<SCAP, NM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     set = true;
   }
-  int grid;
-  if (from_list) {
-    grid = kNumSM;
-  } else {
-    grid = (c + warps - 1) / warps;
-  }
+  const int grid = (c + warps - 1) / warps;
   thanos_solve_kernel<SCAP, NM><<<grid, warps * 32, smem, s>>>(W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n,
-                                                              nm_m, ovf, from_list, st);
+                                                              nm_m, st);
 }
 
 }  // namespace
 
-// Rows whose selected set fits 80 entries go through an 8-warp CTA with 14 KB of
-// shared memory per warp; the rare larger sets (up to 128) take a second launch with
-// 35 KB per warp.
+// The selected set of a row is at most B (unstructured) or exactly B (m-n)/m (N:M).
+// Sets of at most 80 go through 8-warp CTAs with 14 KB of shared memory per warp (two
+// CTAs per SM); larger possible sets use 6-warp CTAs with 35 KB per warp.
 int launch_thanos_solve(bool nm, const float* W, int c, int b, int j, int B, const float* Kt,
                         const float* xnorm, Ctl* ctl, uint8_t* mask, float* Zs, int nm_n, int nm_m,
-                        int* ovf, pwp_stats* st, cudaStream_t s) {
-  const int s_nm = nm ? B / nm_m * (nm_m - nm_n) : 0;
-  const bool big_only = nm ? s_nm > 80 : false;
-  if (big_only) {
+                        pwp_stats* st, cudaStream_t s) {
+  const int smax = nm ? B / nm_m * (nm_m - nm_n) : min(B, b - j);
+  if (smax <= 80) {
     if (nm)
-      launch_thanos_variant<128, true>(4, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, ovf, 0, st, s);
-    return 1;
-  }
-  const bool need_second = !nm && B > 80;
-  if (need_second) cudaMemsetAsync(ovf, 0, sizeof(int), s);
-  if (nm)
-    launch_thanos_variant<80, true>(8, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, ovf, 0, st, s);
-  else
-    launch_thanos_variant<80, false>(8, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, ovf, 0, st, s);
-  if (need_second) {
-    launch_thanos_variant<128, false>(4, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, ovf, 1, st, s);
-    return 2;
+      launch_thanos_variant<80, true>(8, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, st, s);
+    else
+      launch_thanos_variant<80, false>(8, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, st, s);
+  } else {
+    if (nm)
+      launch_thanos_variant<128, true>(6, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, st, s);
+    else
+      launch_thanos_variant<128, false>(6, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, st, s);
   }
   return 1;
 }

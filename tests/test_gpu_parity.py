@@ -78,6 +78,9 @@ def test_small_layer_matches_oracle(name, method, pattern, nm):
     (256, 512, 1024, 128, "bf16", "thanos", "unstructured", (0, 0), 0.5),    # bf16, several 128-blocks
     (256, 512, 1024, 128, "bf16", "thanos", "nm", (2, 4), 0.5),
     (256, 512, 1024, 64, "bf16", "sparsegpt", "unstructured", (0, 0), 0.5),
+    (64, 256, 512, 128, "fp32", "thanos", "unstructured", (0, 0), 0.8),      # rows above 80 selected
+    (48, 256, 512, 128, "fp32", "thanos", "unstructured", (0, 0), 0.93),
+    (32, 256, 512, 128, "fp32", "thanos", "nm", (1, 4), 0.5),                # 96 per row
 ])
 def test_shapes_and_edges_match_oracle(c, b, n, B, dtype, method, pattern, nm, s):
     _torch()
