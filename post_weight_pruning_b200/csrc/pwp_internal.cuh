@@ -129,7 +129,7 @@ void launch_pick2(int score, Ctl* ctl, const unsigned int* hist2, const float* W
 // per-row work of one block (solve.cu); returns the number of kernels launched
 int launch_thanos_solve(bool nm, const float* W, int c, int b, int j, int B, const float* Kt,
                         const float* xnorm, Ctl* ctl, uint8_t* mask, float* Zs, int nm_n, int nm_m,
-                        pwp_stats* st, cudaStream_t s);
+                        int* ovf, pwp_stats* st, cudaStream_t s);
 int launch_sparsegpt_solve(bool nm, const float* W, int c, int b, int j, int B, const float* H,
                            const float* udiag, Ctl* ctl, uint8_t* mask, float* Zs, int nm_n,
                            int nm_m, pwp_stats* st, cudaStream_t s);

@@ -46,29 +46,39 @@ __device__ bool chol_solve(float* __restrict__ L, float* __restrict__ y, int s, 
     const float* p1 = L + poff(jp + 1);
     const float* p2 = L + poff(jp + 2);
     const float* p3 = L + poff(jp + 3);
+    // rows i = jp + lane + 32 r (i == s is the u row): start from their current
+    // entries jp..jp+3, then subtract the contributions of columns t < jp; each panel
+    // row is loaded once per t-step and applied to all of the lane's rows
     float acc[MAXR][4];
+    const float* rp[MAXR];
 #pragma unroll
     for (int r = 0; r < MAXR; ++r) {
       const int i = jp + lane + 32 * r;
+      rp[r] = (i < s) ? L + poff(i) : y;
       if (i <= s) {
-        const float* ri = (i < s) ? L + poff(i) : y;
-        const float4 a = *reinterpret_cast<const float4*>(ri + jp);
-        float a0 = a.x, a1 = a.y, a2 = a.z, a3 = a.w;
-#pragma unroll 2
-        for (int t = 0; t < jp; t += 4) {
-          const float4 x = *reinterpret_cast<const float4*>(ri + t);
-          const float4 q0 = *reinterpret_cast<const float4*>(p0 + t);
-          const float4 q1 = *reinterpret_cast<const float4*>(p1 + t);
-          const float4 q2 = *reinterpret_cast<const float4*>(p2 + t);
-          const float4 q3 = *reinterpret_cast<const float4*>(p3 + t);
-          a0 = fmaf(-x.x, q0.x, a0); a0 = fmaf(-x.y, q0.y, a0); a0 = fmaf(-x.z, q0.z, a0); a0 = fmaf(-x.w, q0.w, a0);
-          a1 = fmaf(-x.x, q1.x, a1); a1 = fmaf(-x.y, q1.y, a1); a1 = fmaf(-x.z, q1.z, a1); a1 = fmaf(-x.w, q1.w, a1);
-          a2 = fmaf(-x.x, q2.x, a2); a2 = fmaf(-x.y, q2.y, a2); a2 = fmaf(-x.z, q2.z, a2); a2 = fmaf(-x.w, q2.w, a2);
-          a3 = fmaf(-x.x, q3.x, a3); a3 = fmaf(-x.y, q3.y, a3); a3 = fmaf(-x.z, q3.z, a3); a3 = fmaf(-x.w, q3.w, a3);
-        }
-        acc[r][0] = a0; acc[r][1] = a1; acc[r][2] = a2; acc[r][3] = a3;
+        const float4 a = *reinterpret_cast<const float4*>(rp[r] + jp);
+        acc[r][0] = a.x; acc[r][1] = a.y; acc[r][2] = a.z; acc[r][3] = a.w;
       } else {
         acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
+      }
+    }
+    const int nr = (s - jp) / 32 + 1;   // rounds holding at least one row of [jp, s]
+#pragma unroll 2
+    for (int t = 0; t < jp; t += 4) {
+      const float4 q0 = *reinterpret_cast<const float4*>(p0 + t);
+      const float4 q1 = *reinterpret_cast<const float4*>(p1 + t);
+      const float4 q2 = *reinterpret_cast<const float4*>(p2 + t);
+      const float4 q3 = *reinterpret_cast<const float4*>(p3 + t);
+#pragma unroll
+      for (int r = 0; r < MAXR; ++r) {
+        if (r < nr && jp + lane + 32 * r <= s) {
+          const float4 x = *reinterpret_cast<const float4*>(rp[r] + t);
+          float* a = acc[r];
+          a[0] = fmaf(-x.x, q0.x, a[0]); a[0] = fmaf(-x.y, q0.y, a[0]); a[0] = fmaf(-x.z, q0.z, a[0]); a[0] = fmaf(-x.w, q0.w, a[0]);
+          a[1] = fmaf(-x.x, q1.x, a[1]); a[1] = fmaf(-x.y, q1.y, a[1]); a[1] = fmaf(-x.z, q1.z, a[1]); a[1] = fmaf(-x.w, q1.w, a[1]);
+          a[2] = fmaf(-x.x, q2.x, a[2]); a[2] = fmaf(-x.y, q2.y, a[2]); a[2] = fmaf(-x.z, q2.z, a[2]); a[2] = fmaf(-x.w, q2.w, a[2]);
+          a[3] = fmaf(-x.x, q3.x, a[3]); a[3] = fmaf(-x.y, q3.y, a[3]); a[3] = fmaf(-x.z, q3.z, a[3]); a[3] = fmaf(-x.w, q3.w, a[3]);
+        }
       }
     }
     const int pw = min(4, s - jp);
@@ -149,6 +159,9 @@ __device__ bool chol_solve(float* __restrict__ L, float* __restrict__ y, int s, 
 }
 
 // One warp per row; SCAP bounds the selected set (and sizes the per-warp shared memory).
+// With an overflow list ovf (ovf[0] = count, ovf[1..] = rows): in the first pass
+// (rows_from_list = 0) a row whose set exceeds SCAP is appended to the list and left;
+// the second pass (rows_from_list = 1, larger SCAP) takes its rows from the list.
 template <int SCAP, bool NM>
 __global__ void __launch_bounds__(256) thanos_solve_kernel(const float* __restrict__ W, int c, int b,
                                                            int j, int B, const float* __restrict__ Kt,
@@ -156,6 +169,7 @@ __global__ void __launch_bounds__(256) thanos_solve_kernel(const float* __restri
                                                            Ctl* __restrict__ ctlp,
                                                            uint8_t* __restrict__ mask,
                                                            float* __restrict__ Zs, int nm_n, int nm_m,
+                                                           int* __restrict__ ovf, int rows_from_list,
                                                            pwp_stats* st) {
   extern __shared__ __align__(16) float smem[];
   if (warp_failed(st)) return;
@@ -167,7 +181,16 @@ __global__ void __launch_bounds__(256) thanos_solve_kernel(const float* __restri
   const Ctl ctl = *ctlp;
   const int nJ = min(B, b - j);
   constexpr int MAXI = kMaxBlock / 32;
-  for (int k = blockIdx.x * nwarps + warp; k < c; k += gridDim.x * nwarps) {
+  int nrows = c;
+  if (rows_from_list) {
+    nrows = *((volatile const int*)ovf);
+    if (nrows < 0 || nrows > c) {   // the list holds at most one entry per row
+      if (lane == 0) set_error(st, PWP_EINVAL, kSiteSolve);
+      return;
+    }
+  }
+  for (int idx = blockIdx.x * nwarps + warp; idx < nrows; idx += gridDim.x * nwarps) {
+    const int k = rows_from_list ? ovf[1 + idx] : idx;
     const float* wrow = W + (long long)k * b + j;
     float w[MAXI];
     bool sel[MAXI];
@@ -184,8 +207,15 @@ __global__ void __launch_bounds__(256) thanos_solve_kernel(const float* __restri
       pos[i] = s + __popc(bal & ((1u << lane) - 1u));
       s += __popc(bal);
     }
-    if (s > SCAP) {   // cannot happen: the launcher picks SCAP >= the block's largest set
-      if (lane == 0) set_error(st, PWP_EINVAL, kSiteSolve);
+    if (s > SCAP) {
+      if (lane == 0) {
+        if (ovf && !rows_from_list) {
+          const int at = atomicAdd(ovf, 1);
+          ovf[1 + at] = k;
+        } else {
+          set_error(st, PWP_EINVAL, kSiteSolve);   // no larger pass to defer to
+        }
+      }
       continue;
     }
     uint8_t* mrow = mask + (long long)k * b + j;
@@ -201,27 +231,45 @@ __global__ void __launch_bounds__(256) thanos_solve_kernel(const float* __restri
     __syncwarp();
     bool ok = true;
     if (s > 0) {
-      // R-hat = K[Q, Q], lower triangle, gathered four rows at a time
+      // R-hat = K[Q, Q], lower triangle: row a is K row q_a, loaded whole (lane l holds
+      // columns 4l..4l+3), and entry (a, cc) is picked from lane q_cc / 4 by shuffles
       constexpr int CH = (SCAP + 31) / 32;
+      int qv[CH];
+#pragma unroll
+      for (int ch = 0; ch < CH; ++ch) qv[ch] = (lane + 32 * ch < s) ? Qidx[lane + 32 * ch] : 0;
+      const bool vec = ((b & 3) == 0) && ((j & 3) == 0);
+      const int c4 = 4 * lane;
       for (int a0 = 0; a0 < s; a0 += 4) {
-        float v[4][CH];
+        // four K rows in flight, then the picks from registers
+        float4 kv[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
           const int a = a0 + r;
-          const float* krow = Kt + (size_t)(a < s ? Qidx[a] : 0) * b + j;
-#pragma unroll
-          for (int ch = 0; ch < CH; ++ch) {
-            const int cc = lane + 32 * ch;
-            v[r][ch] = (a < s && cc <= a) ? __ldg(krow + Qidx[cc]) : 0.f;
+          const float* krow = Kt + (size_t)(a < s ? Qidx[a] : Qidx[0]) * b + j;
+          if (vec && c4 + 3 < nJ) {
+            kv[r] = __ldg(reinterpret_cast<const float4*>(krow + c4));
+          } else {
+            kv[r].x = c4 < nJ ? __ldg(krow + c4) : 0.f;
+            kv[r].y = c4 + 1 < nJ ? __ldg(krow + c4 + 1) : 0.f;
+            kv[r].z = c4 + 2 < nJ ? __ldg(krow + c4 + 2) : 0.f;
+            kv[r].w = c4 + 3 < nJ ? __ldg(krow + c4 + 3) : 0.f;
           }
         }
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
           const int a = a0 + r;
+          if (a >= s) break;
 #pragma unroll
           for (int ch = 0; ch < CH; ++ch) {
+            if (32 * ch > a) break;
+            const int src = qv[ch] >> 2, comp = qv[ch] & 3;
+            const float vx = __shfl_sync(0xffffffffu, kv[r].x, src);
+            const float vy = __shfl_sync(0xffffffffu, kv[r].y, src);
+            const float vz = __shfl_sync(0xffffffffu, kv[r].z, src);
+            const float vw = __shfl_sync(0xffffffffu, kv[r].w, src);
+            const float v = comp == 0 ? vx : comp == 1 ? vy : comp == 2 ? vz : vw;
             const int cc = lane + 32 * ch;
-            if (a < s && cc <= a) L[poff(a) + cc] = v[r][ch];
+            if (cc <= a) L[poff(a) + cc] = v;
           }
         }
       }
@@ -305,39 +353,45 @@ __global__ void __launch_bounds__(256) sparsegpt_solve_kernel(const float* __res
 template <int SCAP, bool NM>
 void launch_thanos_variant(int warps, const float* W, int c, int b, int j, int B, const float* Kt,
                            const float* xnorm, Ctl* ctl, uint8_t* mask, float* Zs, int nm_n, int nm_m,
-                           pwp_stats* st, cudaStream_t s) {
+                           int* ovf, int from_list, pwp_stats* st, cudaStream_t s) {
   const int smem = warps * SolveSmem<SCAP>::kPerWarp * 4;
   static bool set = false;
   if (!set) {
     cudaFuncSetAttribute(thanos_solve_kernel<SCAP, NM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     set = true;
   }
-  const int grid = (c + warps - 1) / warps;
+  const int grid = from_list ? kNumSM : (c + warps - 1) / warps;
   thanos_solve_kernel<SCAP, NM><<<grid, warps * 32, smem, s>>>(W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n,
-                                                              nm_m, st);
+                                                              nm_m, ovf, from_list, st);
 }
 
 }  // namespace
 
-// The selected set of a row is at most B (unstructured) or exactly B (m-n)/m (N:M).
-// Sets of at most 80 go through 8-warp CTAs with 14 KB of shared memory per warp (two
-// CTAs per SM); larger possible sets use 6-warp CTAs with 35 KB per warp.
+// A row's selected set is at most min(B, block width) (unstructured) or exactly
+// B (m-n)/m (N:M).  Sets of at most 80 go through 8-warp CTAs with 14 KB of shared
+// memory per warp (two CTAs per SM).  When a block can hold larger sets, the rows that
+// actually have one are listed by that pass and solved by a second pass of 6-warp CTAs
+// with 35 KB per warp; N:M patterns with more than 80 per row use the larger CTAs
+// directly.
 int launch_thanos_solve(bool nm, const float* W, int c, int b, int j, int B, const float* Kt,
                         const float* xnorm, Ctl* ctl, uint8_t* mask, float* Zs, int nm_n, int nm_m,
-                        pwp_stats* st, cudaStream_t s) {
+                        int* ovf, pwp_stats* st, cudaStream_t s) {
   const int smax = nm ? B / nm_m * (nm_m - nm_n) : min(B, b - j);
-  if (smax <= 80) {
-    if (nm)
-      launch_thanos_variant<80, true>(8, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, st, s);
+  if (nm) {
+    if (smax <= 80)
+      launch_thanos_variant<80, true>(8, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, nullptr, 0, st, s);
     else
-      launch_thanos_variant<80, false>(8, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, st, s);
-  } else {
-    if (nm)
-      launch_thanos_variant<128, true>(6, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, st, s);
-    else
-      launch_thanos_variant<128, false>(6, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, st, s);
+      launch_thanos_variant<128, true>(6, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, nullptr, 0, st, s);
+    return 1;
   }
-  return 1;
+  if (smax <= 80) {
+    launch_thanos_variant<80, false>(8, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, nullptr, 0, st, s);
+    return 1;
+  }
+  cudaMemsetAsync(ovf, 0, sizeof(int), s);
+  launch_thanos_variant<80, false>(8, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, ovf, 0, st, s);
+  launch_thanos_variant<128, false>(6, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, ovf, 1, st, s);
+  return 2;
 }
 
 int launch_sparsegpt_solve(bool nm, const float* W, int c, int b, int j, int B, const float* H,
