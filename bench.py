@@ -38,7 +38,7 @@ K_HESSIAN, K_FACTOR, K_STREAM, K_SELECT, K_SOLVE = 0, 1, 2, 3, 4
 CLASS_NAMES = {K_HESSIAN: "hessian_xxt", K_FACTOR: "factor", K_STREAM: "stream_update_score",
                K_SELECT: "select", K_SOLVE: "row_solve"}
 CLASS_SOURCES = {K_HESSIAN: ["hessian_tc.cu", "hessian_simt.cu"], K_FACTOR: ["factor.cu"],
-                 K_STREAM: ["prune.cu"], K_SELECT: ["prune.cu"], K_SOLVE: ["prune.cu"]}
+                 K_STREAM: ["prune.cu"], K_SELECT: ["select.cu"], K_SOLVE: ["solve.cu"]}
 
 
 def _load_peaks():
@@ -157,6 +157,19 @@ def algorithmic_work(cls, wl, per_launch_ms, mask=None):
     if cls == K_FACTOR:
         return 2.0 * b ** 3 / 3.0 * len(per_launch_ms), "flop", "alu"
     raise ValueError(cls)
+
+
+def job_throughput(local_ms, world, weights_per_step, steps, device=None):
+    """Whole-job throughput (weights/s) from this rank's device time: every rank prunes
+    its own layer, so the job processes world x weights_per_step x steps weights in the
+    time of the slowest rank (max over ranks).  Returns (value, max_ms)."""
+    import torch
+    t = torch.tensor([float(local_ms)], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+    return world * weights_per_step * steps / (max_ms / 1e3), max_ms
 
 
 def fp32_alu_peak_tflops(sm_mhz):
@@ -327,11 +340,7 @@ def run_mine(args):
         raise RuntimeError(f"timed step failed: status {st.status}")
     mask_np = mask.cpu().numpy() if dom == K_SOLVE else None
 
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
-    value = world * c * b * args.steps / (max_ms / 1e3)
+    value, max_ms = job_throughput(total_ms, world, c * b, args.steps, dev)
 
     # end to end through the public API from pinned host buffers
     W_host = torch.from_numpy(W_store.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -351,10 +360,7 @@ def run_mine(args):
         e1[i].record(stream)
     torch.cuda.synchronize()
     e2e_ms = float(sum(e0[i].elapsed_time(e1[i]) for i in range(e2e_steps)))
-    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = world * c * b * e2e_steps / (float(te.item()) / 1e3)
+    e2e_value, _ = job_throughput(e2e_ms, world, c * b, e2e_steps, dev)
 
     if rank == 0:
         peaks = _load_peaks()

@@ -229,7 +229,7 @@ struct PruneBuffers {
   float* udiag;
   float* Zs;
   float* K;
-  int* ovf;
+  float* gscratch;
   void* fws;
   size_t fws_bytes;
 };
@@ -255,7 +255,8 @@ size_t prune_ws_layout(const pwp_config* cfg, int c, int b, PruneBuffers* pb, ch
   t.udiag = (float*)take(sizeof(float) * b);
   t.Zs = (float*)take(sizeof(float) * (size_t)c * B);
   t.K = thanos ? (float*)take(sizeof(float) * (size_t)nblk * B * b) : nullptr;
-  t.ovf = (int*)take(sizeof(int) * ((size_t)c + 1));
+  const size_t gbytes = thanos ? solve_scratch_bytes(B, cfg->pattern == PWP_NM, cfg->nm_n, cfg->nm_m) : 0;
+  t.gscratch = gbytes ? (float*)take(gbytes) : nullptr;
   t.fws_bytes = factor_ws_bytes(b);
   t.fws = take(t.fws_bytes);
   if (pb) *pb = t;
@@ -374,7 +375,7 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
     prof_begin(kKSolve, s);
     if (thanos)
       nl += launch_thanos_solve(nm, Wout, c, b, j, B, pb.K + (size_t)t * B * b, pb.xnorm, pb.ctl, mask, pb.Zs,
-                                cfg->nm_n, cfg->nm_m, pb.ovf, st, s);
+                                cfg->nm_n, cfg->nm_m, pb.gscratch, st, s);
     else
       nl += launch_sparsegpt_solve(nm, Wout, c, b, j, B, H, pb.udiag, pb.ctl, mask, pb.Zs, cfg->nm_n,
                                    cfg->nm_m, st, s);

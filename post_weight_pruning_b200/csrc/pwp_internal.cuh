@@ -14,6 +14,8 @@ constexpr int kHist1Bins = 1 << kHist1Bits;
 constexpr int kHist2Bins = 1 << 16;      // second level: key bits [15:0]
 constexpr int kFactorNB = 64;            // panel width of the blocked factorisation
 constexpr int kMaxBlock = 128;           // largest column block B
+constexpr int kSolveCtas = 2 * kNumSM;   // persistent grid of the row-solve kernel
+constexpr int kSolveNS = 79;             // factor rows kept in shared memory at capacity 128
 
 // Per-call device control block (lives at the start of the workspace).
 struct Ctl {
@@ -129,7 +131,8 @@ void launch_pick2(int score, Ctl* ctl, const unsigned int* hist2, const float* W
 // per-row work of one block (solve.cu); returns the number of kernels launched
 int launch_thanos_solve(bool nm, const float* W, int c, int b, int j, int B, const float* Kt,
                         const float* xnorm, Ctl* ctl, uint8_t* mask, float* Zs, int nm_n, int nm_m,
-                        int* ovf, pwp_stats* st, cudaStream_t s);
+                        float* gscratch, pwp_stats* st, cudaStream_t s);
+size_t solve_scratch_bytes(int B, bool nm, int nm_n, int nm_m);
 int launch_sparsegpt_solve(bool nm, const float* W, int c, int b, int j, int B, const float* H,
                            const float* udiag, Ctl* ctl, uint8_t* mask, float* Zs, int nm_n,
                            int nm_m, pwp_stats* st, cudaStream_t s);

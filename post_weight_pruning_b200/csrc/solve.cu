@@ -23,11 +23,22 @@ __host__ __device__ constexpr int poff(int i) {
   return 4 * (2 * (i >> 2) * ((i >> 2) + 1) + (i & 3) * ((i >> 2) + 1));
 }
 
-template <int SCAP>
+// Per warp: rows 0..NS-1 of the packed factor, the u/y vector and the selected indices in
+// shared memory; rows NS..SCAP-1 (only rows with more than NS selections reach them) in a
+// per-warp slot of global scratch.
+template <int SCAP, int NS>
 struct SolveSmem {
-  static constexpr int kL = poff(SCAP);
+  static constexpr int kL = poff(NS);
   static constexpr int kY = SCAP + 4;
   static constexpr int kPerWarp = kL + kY + SCAP;  // floats: L, y, Qidx
+  static constexpr int kGlobal = poff(SCAP) - poff(NS);   // floats of global scratch per warp
+};
+
+template <int NS>
+struct Rows {
+  float* L;   // shared, rows < NS
+  float* G;   // global, rows >= NS
+  __device__ __forceinline__ float* row(int i) const { return i < NS ? L + poff(i) : G + (poff(i) - poff(NS)); }
 };
 
 // Cholesky R-hat = L L^T (left-looking, 4-column panels; lanes own rows) with u carried
@@ -38,14 +49,14 @@ struct SolveSmem {
 // the 4x4 diagonal block is factored in the registers of lanes 0..3 with shuffles,
 // and every other row finishes its four panel entries by a 4x4 forward substitution.
 // One __syncwarp per panel.  Returns false on a non-positive pivot (uniform).
-template <int SCAP>
-__device__ bool chol_solve(float* __restrict__ L, float* __restrict__ y, int s, int lane) {
+template <int SCAP, int NS>
+__device__ bool chol_solve(const Rows<NS> R, float* __restrict__ y, int s, int lane) {
   constexpr int MAXR = (SCAP + 1 + 31) / 32;   // rows jp..s over the 32 lanes
   for (int jp = 0; jp < s; jp += 4) {
-    const float* p0 = L + poff(jp);
-    const float* p1 = L + poff(jp + 1);
-    const float* p2 = L + poff(jp + 2);
-    const float* p3 = L + poff(jp + 3);
+    const float* p0 = R.row(jp);
+    const float* p1 = R.row(jp + 1);
+    const float* p2 = R.row(jp + 2);
+    const float* p3 = R.row(jp + 3);
     // rows i = jp + lane + 32 r (i == s is the u row): start from their current
     // entries jp..jp+3, then subtract the contributions of columns t < jp; each panel
     // row is loaded once per t-step and applied to all of the lane's rows
@@ -54,7 +65,7 @@ __device__ bool chol_solve(float* __restrict__ L, float* __restrict__ y, int s, 
 #pragma unroll
     for (int r = 0; r < MAXR; ++r) {
       const int i = jp + lane + 32 * r;
-      rp[r] = (i < s) ? L + poff(i) : y;
+      rp[r] = (i < s) ? R.row(i) : y;
       if (i <= s) {
         const float4 a = *reinterpret_cast<const float4*>(rp[r] + jp);
         acc[r][0] = a.x; acc[r][1] = a.y; acc[r][2] = a.z; acc[r][3] = a.w;
@@ -114,7 +125,7 @@ __device__ bool chol_solve(float* __restrict__ L, float* __restrict__ y, int s, 
     for (int r = 0; r < MAXR; ++r) {
       const int i = jp + lane + 32 * r;
       if (i > s) continue;
-      float* ri = (i < s) ? L + poff(i) : y;
+      float* ri = (i < s) ? R.row(i) : y;
       float4 o;
       if (i < jp + pw && i < s) {
         o = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
@@ -140,8 +151,8 @@ __device__ bool chol_solve(float* __restrict__ L, float* __restrict__ y, int s, 
         float v = y[a0 + c];
 #pragma unroll
         for (int c2 = c + 1; c2 < 4; ++c2)
-          if (c2 < pw) v = fmaf(-L[poff(a0 + c2) + a0 + c], z[c2], v);
-        z[c] = v / L[poff(a0 + c) + a0 + c];
+          if (c2 < pw) v = fmaf(-R.row(a0 + c2)[a0 + c], z[c2], v);
+        z[c] = v / R.row(a0 + c)[a0 + c];
       }
     }
     __syncwarp();
@@ -149,7 +160,7 @@ __device__ bool chol_solve(float* __restrict__ L, float* __restrict__ y, int s, 
       float v = y[t];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
-        if (c < pw) v = fmaf(-L[poff(a0 + c) + t], z[c], v);
+        if (c < pw) v = fmaf(-R.row(a0 + c)[t], z[c], v);
       y[t] = v;
     }
     if (lane < pw) y[a0 + lane] = z[lane];
@@ -158,39 +169,29 @@ __device__ bool chol_solve(float* __restrict__ L, float* __restrict__ y, int s, 
   return true;
 }
 
-// One warp per row; SCAP bounds the selected set (and sizes the per-warp shared memory).
-// With an overflow list ovf (ovf[0] = count, ovf[1..] = rows): in the first pass
-// (rows_from_list = 0) a row whose set exceeds SCAP is appended to the list and left;
-// the second pass (rows_from_list = 1, larger SCAP) takes its rows from the list.
-template <int SCAP, bool NM>
+// One warp per row over a persistent grid (each warp keeps one scratch slot).  SCAP
+// bounds the selected set; rows beyond NS of a large set live in the warp's global slot.
+template <int SCAP, int NS, bool NM>
 __global__ void __launch_bounds__(256) thanos_solve_kernel(const float* __restrict__ W, int c, int b,
                                                            int j, int B, const float* __restrict__ Kt,
                                                            const float* __restrict__ xnorm,
                                                            Ctl* __restrict__ ctlp,
                                                            uint8_t* __restrict__ mask,
                                                            float* __restrict__ Zs, int nm_n, int nm_m,
-                                                           int* __restrict__ ovf, int rows_from_list,
-                                                           pwp_stats* st) {
+                                                           float* __restrict__ gscratch, pwp_stats* st) {
   extern __shared__ __align__(16) float smem[];
   if (warp_failed(st)) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nwarps = blockDim.x >> 5;
-  float* L = smem + warp * SolveSmem<SCAP>::kPerWarp;
-  float* y = L + SolveSmem<SCAP>::kL;
-  int* Qidx = reinterpret_cast<int*>(y + SolveSmem<SCAP>::kY);
+  const int slot = blockIdx.x * nwarps + warp;
+  float* L = smem + warp * SolveSmem<SCAP, NS>::kPerWarp;
+  float* y = L + SolveSmem<SCAP, NS>::kL;
+  int* Qidx = reinterpret_cast<int*>(y + SolveSmem<SCAP, NS>::kY);
+  const Rows<NS> R{L, gscratch ? gscratch + (size_t)slot * SolveSmem<SCAP, NS>::kGlobal : nullptr};
   const Ctl ctl = *ctlp;
   const int nJ = min(B, b - j);
   constexpr int MAXI = kMaxBlock / 32;
-  int nrows = c;
-  if (rows_from_list) {
-    nrows = *((volatile const int*)ovf);
-    if (nrows < 0 || nrows > c) {   // the list holds at most one entry per row
-      if (lane == 0) set_error(st, PWP_EINVAL, kSiteSolve);
-      return;
-    }
-  }
-  for (int idx = blockIdx.x * nwarps + warp; idx < nrows; idx += gridDim.x * nwarps) {
-    const int k = rows_from_list ? ovf[1 + idx] : idx;
+  for (int k = slot; k < c; k += gridDim.x * nwarps) {
     const float* wrow = W + (long long)k * b + j;
     float w[MAXI];
     bool sel[MAXI];
@@ -207,15 +208,8 @@ __global__ void __launch_bounds__(256) thanos_solve_kernel(const float* __restri
       pos[i] = s + __popc(bal & ((1u << lane) - 1u));
       s += __popc(bal);
     }
-    if (s > SCAP) {
-      if (lane == 0) {
-        if (ovf && !rows_from_list) {
-          const int at = atomicAdd(ovf, 1);
-          ovf[1 + at] = k;
-        } else {
-          set_error(st, PWP_EINVAL, kSiteSolve);   // no larger pass to defer to
-        }
-      }
+    if (s > SCAP || (s > NS && !R.G)) {   // excluded by the launcher's choice of SCAP / scratch
+      if (lane == 0) set_error(st, PWP_EINVAL, kSiteSolve);
       continue;
     }
     uint8_t* mrow = mask + (long long)k * b + j;
@@ -269,12 +263,12 @@ __global__ void __launch_bounds__(256) thanos_solve_kernel(const float* __restri
             const float vw = __shfl_sync(0xffffffffu, kv[r].w, src);
             const float v = comp == 0 ? vx : comp == 1 ? vy : comp == 2 ? vz : vw;
             const int cc = lane + 32 * ch;
-            if (cc <= a) L[poff(a) + cc] = v;
+            if (cc <= a) R.row(a)[cc] = v;
           }
         }
       }
       __syncwarp();
-      ok = chol_solve<SCAP>(L, y, s, lane);
+      ok = chol_solve<SCAP, NS>(R, y, s, lane);
       if (!ok && lane == 0) set_error(st, PWP_ENOTSPD, kSiteSolve);
       if (lane == 0) atomicAdd((unsigned long long*)&ctlp->pruned, (unsigned long long)s);
     }
@@ -350,48 +344,53 @@ __global__ void __launch_bounds__(256) sparsegpt_solve_kernel(const float* __res
   if (lane == 0 && s > 0) atomicAdd((unsigned long long*)&ctlp->pruned, (unsigned long long)s);
 }
 
-template <int SCAP, bool NM>
-void launch_thanos_variant(int warps, const float* W, int c, int b, int j, int B, const float* Kt,
-                           const float* xnorm, Ctl* ctl, uint8_t* mask, float* Zs, int nm_n, int nm_m,
-                           int* ovf, int from_list, pwp_stats* st, cudaStream_t s) {
-  const int smem = warps * SolveSmem<SCAP>::kPerWarp * 4;
+template <int SCAP, int NS, bool NM>
+void launch_thanos_variant(const float* W, int c, int b, int j, int B, const float* Kt, const float* xnorm,
+                           Ctl* ctl, uint8_t* mask, float* Zs, int nm_n, int nm_m, float* gscratch,
+                           pwp_stats* st, cudaStream_t s) {
+  constexpr int warps = 8;
+  const int smem = warps * SolveSmem<SCAP, NS>::kPerWarp * 4;
   static bool set = false;
   if (!set) {
-    cudaFuncSetAttribute(thanos_solve_kernel<SCAP, NM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaFuncSetAttribute(thanos_solve_kernel<SCAP, NS, NM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     set = true;
   }
-  const int grid = from_list ? kNumSM : (c + warps - 1) / warps;
-  thanos_solve_kernel<SCAP, NM><<<grid, warps * 32, smem, s>>>(W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n,
-                                                              nm_m, ovf, from_list, st);
+  const int grid = min((c + warps - 1) / warps, kSolveCtas);
+  thanos_solve_kernel<SCAP, NS, NM><<<grid, warps * 32, smem, s>>>(W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n,
+                                                                  nm_m, gscratch, st);
 }
 
 }  // namespace
 
+size_t solve_scratch_bytes(int B, bool nm, int nm_n, int nm_m) {
+  const int smax = nm ? B / nm_m * (nm_m - nm_n) : B;
+  if (smax <= 80) return 0;
+  return (size_t)kSolveCtas * 8 * SolveSmem<kMaxBlock, kSolveNS>::kGlobal * sizeof(float);
+}
+
 // A row's selected set is at most min(B, block width) (unstructured) or exactly
-// B (m-n)/m (N:M).  Sets of at most 80 go through 8-warp CTAs with 14 KB of shared
-// memory per warp (two CTAs per SM).  When a block can hold larger sets, the rows that
-// actually have one are listed by that pass and solved by a second pass of 6-warp CTAs
-// with 35 KB per warp; N:M patterns with more than 80 per row use the larger CTAs
-// directly.
+// B (m-n)/m (N:M).  8-warp CTAs keep up to 80 rows of each warp's factor in shared memory
+// (two CTAs per SM); when a block can hold larger sets (capacity 128, whose larger u/index
+// vectors leave room for 79 rows at two CTAs per SM), rows 79..127 of a large set go to
+// the warp's slot of global scratch.
 int launch_thanos_solve(bool nm, const float* W, int c, int b, int j, int B, const float* Kt,
                         const float* xnorm, Ctl* ctl, uint8_t* mask, float* Zs, int nm_n, int nm_m,
-                        int* ovf, pwp_stats* st, cudaStream_t s) {
+                        float* gscratch, pwp_stats* st, cudaStream_t s) {
   const int smax = nm ? B / nm_m * (nm_m - nm_n) : min(B, b - j);
-  if (nm) {
-    if (smax <= 80)
-      launch_thanos_variant<80, true>(8, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, nullptr, 0, st, s);
-    else
-      launch_thanos_variant<128, true>(6, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, nullptr, 0, st, s);
-    return 1;
-  }
   if (smax <= 80) {
-    launch_thanos_variant<80, false>(8, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, nullptr, 0, st, s);
-    return 1;
+    if (nm)
+      launch_thanos_variant<80, 80, true>(W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, nullptr, st, s);
+    else
+      launch_thanos_variant<80, 80, false>(W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, nullptr, st, s);
+  } else {
+    if (nm)
+      launch_thanos_variant<kMaxBlock, kSolveNS, true>(W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m,
+                                                       gscratch, st, s);
+    else
+      launch_thanos_variant<kMaxBlock, kSolveNS, false>(W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m,
+                                                        gscratch, st, s);
   }
-  cudaMemsetAsync(ovf, 0, sizeof(int), s);
-  launch_thanos_variant<80, false>(8, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, ovf, 0, st, s);
-  launch_thanos_variant<128, false>(6, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, ovf, 1, st, s);
-  return 2;
+  return 1;
 }
 
 int launch_sparsegpt_solve(bool nm, const float* W, int c, int b, int j, int B, const float* H,
