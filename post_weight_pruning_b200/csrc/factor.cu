@@ -429,12 +429,11 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
   const int np = (b + NB - 1) / NB;
   float* Vall = (float*)ws;
   float* T = Vall + (size_t)np * NB * NB;
-  static bool attr = false;
-  if (!attr) {
+  static std::atomic<unsigned long long> attr_done{0};
+  if (first_on_device(attr_done)) {
     cudaFuncSetAttribute(chol_update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * NB * 132 * 4);
     // 33 KB dynamic on top of 17 KB static shared memory: above the 48 KB default
     cudaFuncSetAttribute(chol_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * NB * (NB + 1) * 4);
-    attr = true;
   }
   long long nl = 0;
   damp_kernel<<<1, 1024, 0, s>>>(H, b, damp, g_diag, st);

@@ -326,11 +326,10 @@ cudaError_t launch_hessian_tc(const void* X, long long n, int b, float* H, int b
                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return cudaSuccess;
-  static bool attr = false;
-  if (!attr) {
+  static std::atomic<unsigned long long> attr_done{0};
+  if (first_on_device(attr_done)) {
     cudaError_t e = cudaFuncSetAttribute(syrk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   syrk_tc_kernel<<<tile_count(b), 128, SMEM_BYTES, s>>>(map, n, b, H, beta, st);
   *used = true;

@@ -255,7 +255,7 @@ size_t prune_ws_layout(const pwp_config* cfg, int c, int b, PruneBuffers* pb, ch
   t.udiag = (float*)take(sizeof(float) * b);
   t.Zs = (float*)take(sizeof(float) * (size_t)c * B);
   t.K = thanos ? (float*)take(sizeof(float) * (size_t)nblk * B * b) : nullptr;
-  const size_t gbytes = thanos ? solve_scratch_bytes(B, cfg->pattern == PWP_NM, cfg->nm_n, cfg->nm_m) : 0;
+  const size_t gbytes = thanos ? solve_scratch_bytes(c, B, cfg->pattern == PWP_NM, cfg->nm_n, cfg->nm_m) : 0;
   t.gscratch = gbytes ? (float*)take(gbytes) : nullptr;
   t.fws_bytes = factor_ws_bytes(b);
   t.fws = take(t.fws_bytes);
@@ -265,7 +265,8 @@ size_t prune_ws_layout(const pwp_config* cfg, int c, int b, PruneBuffers* pb, ch
 
 // ------------------------------------------------------------------ driver
 
-static int g_nsm = 0;
+static std::atomic<int> g_nsm{0};
+static std::atomic<unsigned long long> g_attr_done{0};
 
 template <int SCORE>
 static void launch_stream(float* W, int c, int b, int u0, int j, int col_end, const float* Z, int Bp, int ldz,
@@ -273,7 +274,8 @@ static void launch_stream(float* W, int c, int b, int u0, int j, int col_end, co
                           int hist_end, unsigned int* hist1, const pwp_stats* st, cudaStream_t s) {
   const int smem = SCORE != kNoScore ? kHist1Bins * 4 : 0;
   const int tiles = ((col_end - u0 + 127) / 128) * ((c + 63) / 64);
-  const int grid = tiles < g_nsm ? tiles : g_nsm;
+  const int nsm = g_nsm.load();
+  const int grid = tiles < nsm ? tiles : nsm;
   stream_kernel<SCORE><<<grid > 0 ? grid : 1, 256, smem, s>>>(W, c, b, u0, j, col_end, Z, Bp, ldz, R, ldr,
                                                              r_upper_from, mask, sc, hist_end, hist1, st);
 }
@@ -306,7 +308,7 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
     for (int t = 0; t < nblk; ++t)
       target += (long long)((double)cfg->sparsity * (double)c * (double)min(B, b - t * B));
   }
-  if (!g_nsm) {
+  if (first_on_device(g_attr_done)) {
     cudaFuncSetAttribute(stream_kernel<kWanda>, cudaFuncAttributeMaxDynamicSharedMemorySize, kHist1Bins * 4);
     cudaFuncSetAttribute(stream_kernel<kObs>, cudaFuncAttributeMaxDynamicSharedMemorySize, kHist1Bins * 4);
     cudaFuncSetAttribute(kmat_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -323,7 +325,7 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
   }
   init_ctl_kernel<<<1, 1, 0, s>>>(pb.ctl, zstar, st, target);
   cudaMemsetAsync(pb.hist1, 0, sizeof(unsigned int) * kHist1Bins, s);
-  convert_w_kernel<<<4 * g_nsm, 256, 0, s>>>(W, wtype, Wout, N);
+  convert_w_kernel<<<4 * g_nsm.load(), 256, 0, s>>>(W, wtype, Wout, N);
   nl += 2;
   prof_begin(kKFactor, s);
   cudaError_t e = launch_damp_factor(H, b, cfg->damp, pb.g_diag, pb.fws, pb.fws_bytes, st, s);

@@ -4,9 +4,21 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/pwp.h"
 
 namespace pwp {
+
+// True on the first call for the current device with this flag word.  Kernel
+// attributes (dynamic shared memory limits) are per device, so each device of a
+// multi-GPU process sets them once.  Devices past 63 always set them again (harmless).
+inline bool first_on_device(std::atomic<unsigned long long>& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return true;
+  const unsigned long long bit = 1ull << dev;
+  return (done.fetch_or(bit) & bit) == 0;
+}
 
 constexpr int kNumSM = 148;              // B200
 constexpr int kHist1Bits = 15;           // first radix level: key bits [30:16]
@@ -132,7 +144,7 @@ void launch_pick2(int score, Ctl* ctl, const unsigned int* hist2, const float* W
 int launch_thanos_solve(bool nm, const float* W, int c, int b, int j, int B, const float* Kt,
                         const float* xnorm, Ctl* ctl, uint8_t* mask, float* Zs, int nm_n, int nm_m,
                         float* gscratch, pwp_stats* st, cudaStream_t s);
-size_t solve_scratch_bytes(int B, bool nm, int nm_n, int nm_m);
+size_t solve_scratch_bytes(int c, int B, bool nm, int nm_n, int nm_m);
 int launch_sparsegpt_solve(bool nm, const float* W, int c, int b, int j, int B, const float* H,
                            const float* udiag, Ctl* ctl, uint8_t* mask, float* Zs, int nm_n,
                            int nm_m, pwp_stats* st, cudaStream_t s);

@@ -350,11 +350,9 @@ void launch_thanos_variant(const float* W, int c, int b, int j, int B, const flo
                            pwp_stats* st, cudaStream_t s) {
   constexpr int warps = 8;
   const int smem = warps * SolveSmem<SCAP, NS>::kPerWarp * 4;
-  static bool set = false;
-  if (!set) {
+  static std::atomic<unsigned long long> attr_done{0};
+  if (first_on_device(attr_done))
     cudaFuncSetAttribute(thanos_solve_kernel<SCAP, NS, NM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    set = true;
-  }
   const int grid = min((c + warps - 1) / warps, kSolveCtas);
   thanos_solve_kernel<SCAP, NS, NM><<<grid, warps * 32, smem, s>>>(W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n,
                                                                   nm_m, gscratch, st);
@@ -362,10 +360,11 @@ void launch_thanos_variant(const float* W, int c, int b, int j, int B, const flo
 
 }  // namespace
 
-size_t solve_scratch_bytes(int B, bool nm, int nm_n, int nm_m) {
+size_t solve_scratch_bytes(int c, int B, bool nm, int nm_n, int nm_m) {
   const int smax = nm ? B / nm_m * (nm_m - nm_n) : B;
   if (smax <= 80) return 0;
-  return (size_t)kSolveCtas * 8 * SolveSmem<kMaxBlock, kSolveNS>::kGlobal * sizeof(float);
+  const int grid = min((c + 7) / 8, kSolveCtas);  // the launch's grid (8 warps per CTA)
+  return (size_t)grid * 8 * SolveSmem<kMaxBlock, kSolveNS>::kGlobal * sizeof(float);
 }
 
 // A row's selected set is at most min(B, block width) (unstructured) or exactly
