@@ -18,10 +18,7 @@
 // Only tiles that hold some i <= j are launched; entries with i > j are left to their
 // mirror, so H comes out exactly symmetric.  Every wait is bounded: a wait that runs
 // out records PWP_ETIMEOUT (or, without a status word, writes NaN into the tile).
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
-#include "pwp_internal.cuh"
+#include "tc_common.cuh"
 
 namespace pwp {
 namespace {
@@ -35,58 +32,7 @@ constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 // kind::f16 instruction descriptor: D fp32, A and B bf16, both MN-major, N = 256, M = 128
 constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
                            ((uint32_t)(TN >> 3) << 17) | ((uint32_t)(TM >> 4) << 24);
-constexpr long long kSpinLimit = 1ll << 26;
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-
-// Bounded wait for the phase of the given parity to complete.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  const uint32_t addr = smem_u32(bar);
-  for (long long i = 0; i < kSpinLimit; ++i) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred P1;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
-        "selp.b32 %0, 1, 0, P1;\n\t}"
-        : "=r"(done)
-        : "r"(addr), "r"(parity)
-        : "memory");
-    if (done) return true;
-  }
-  return false;
-}
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
-          smem_u32(dst)),
-      "l"((uint64_t)map), "r"(smem_u32(bar)), "r"(x), "r"(y)
-      : "memory");
-}
-
-// Shared-memory matrix descriptor, 128-byte swizzle.  For MN-major operands the
-// leading offset is the distance between 64-element MN chunks and the stride offset
-// the distance between 8-row groups along K.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-  d |= (uint64_t)1 << 46;  // descriptor version for this architecture
-  d |= (uint64_t)2 << 61;  // SWIZZLE_128B
-  return d;
-}
+using namespace tc;
 
 __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t acc) {
   asm volatile(
@@ -95,29 +41,6 @@ __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t da, uint64_t 
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
       "l"(da), "l"(db), "r"(IDESC), "r"(acc)
       : "memory");
-}
-
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // Tiles (I, J) of 128 rows x 256 columns that hold some entry with row <= column,
@@ -167,19 +90,16 @@ __global__ void __launch_bounds__(128, 1) syrk_tc_kernel(const __grid_constant__
     abort_flag = 0;
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_slot)),
-                 "r"(TN)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    tmem_alloc(&tmem_slot, TN);
   }
-  tc_fence_before();
+  fence_before();
   __syncthreads();
-  tc_fence_after();
+  fence_after();
   const uint32_t tmem = tmem_slot;
 
   if (warp == 0) {
     if (lane == 0) {
-      asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&tmap) : "memory");
+      prefetch_map(&tmap);
       int issued = 0;
       for (int kt = 0; kt < nk; ++kt) {
         const int s = kt % STAGES;
@@ -214,7 +134,7 @@ __global__ void __launch_bounds__(128, 1) syrk_tc_kernel(const __grid_constant__
           ok = false;
           break;
         }
-        tc_fence_after();
+        fence_after();
         const uint32_t a_addr = sbase + s * STAGE_BYTES;
         const uint32_t b_addr = a_addr + A_BYTES;
 #pragma unroll
@@ -235,11 +155,11 @@ __global__ void __launch_bounds__(128, 1) syrk_tc_kernel(const __grid_constant__
   bool have = mbar_wait(done, 0);
   __syncwarp();
   have = __all_sync(0xffffffffu, have && !*((volatile int*)&abort_flag));
-  tc_fence_after();
+  fence_after();
   const int r = i0 + warp * 32 + lane;
   if (!have) {
     if (threadIdx.x == 0) {
-      if (st) set_error(st, PWP_ETIMEOUT, 6);
+      if (st) set_error(st, PWP_ETIMEOUT, kSiteHessian);
     }
     if (!st && r < b) {
       for (int c = j0; c < min(b, j0 + TN); ++c)
@@ -285,29 +205,25 @@ __global__ void __launch_bounds__(128, 1) syrk_tc_kernel(const __grid_constant__
       }
     }
   }
-  tc_fence_before();
+  fence_before();
   __syncthreads();
-  tc_fence_after();
-  if (warp == 1) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TN) : "memory");
-  }
+  fence_after();
+  if (warp == 1) tmem_free(tmem, TN);
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
+}  // namespace
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    return (PFN_cuTensorMapEncodeTiled_v12000) nullptr;
+  }();
   return fn;
 }
-
-}  // namespace
 
 // Declines (used = false) when the shape does not meet the TMA rules (row stride a
 // multiple of 16 bytes, 16-byte aligned base) or there is nothing to accumulate.
@@ -315,7 +231,7 @@ cudaError_t launch_hessian_tc(const void* X, long long n, int b, float* H, int b
                               pwp_stats* st) {
   *used = false;
   if (n < 1 || b < 1 || (b % 8) != 0 || ((uintptr_t)X % 16) != 0 || n > 0x7fffffffLL) return cudaSuccess;
-  PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode();
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (!encode) return cudaSuccess;
   CUtensorMap map;
   cuuint64_t dims[2] = {(cuuint64_t)b, (cuuint64_t)n};

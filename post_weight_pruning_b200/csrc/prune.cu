@@ -65,10 +65,15 @@ __global__ void prep_diag_kernel(const float* __restrict__ H, int b, const float
 }
 
 // K_t[p][q] = sum_{r <= p} U[j+r][j+p] U[j+r][q] for p < |J_t|, q in [j_t, b): block t's
-// rows of the active inverse.  Stored with row stride b (columns < j_t unused).
-// Grid (column tiles of 128, blocks); 128x128 outputs per CTA, 8x8 per thread.
+// rows of the active inverse.  Two forms: the in-block square K_t[:, j_t:j_t+B] in fp32
+// (K_in, B x B per block, row stride B; the square is symmetric) for the row solves, and
+// K_t transposed as TF32 head and fp32 remainder (K_hi, K_lo: b x B per block, row q
+// holds column q of K_t, rows < j_t unused) -- the K-major operand of the tensor-core
+// update.  Grid (column tiles of 128, blocks); 128x128 outputs per CTA, 8x8 per thread,
+// staged through shared memory so that every output row is written contiguously.
 __global__ void __launch_bounds__(256) kmat_kernel(const float* __restrict__ H, int b, int B,
-                                                   float* __restrict__ K_all, const pwp_stats* st) {
+                                                   float* __restrict__ K_in, float* __restrict__ K_hi,
+                                                   float* __restrict__ K_lo, const pwp_stats* st) {
   extern __shared__ __align__(16) float sm[];
   if (cta_failed(st)) return;
   const int t = blockIdx.y;
@@ -100,31 +105,54 @@ __global__ void __launch_bounds__(256) kmat_kernel(const float* __restrict__ H, 
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[x][e] = fmaf(pv[x], qv[e], acc[x][e]);
   }
-  float* Kt = K_all + (size_t)t * B * b;
+  // stage the tile transposed, T[qq][p], then write rows q with p contiguous
+  __syncthreads();
+  float* T = sm;
+  const int ldt = B + 1;
 #pragma unroll
   for (int x = 0; x < 8; ++x) {
     const int p = ty + 16 * x;
-    if (p >= nJ) continue;
+    if (p >= B) continue;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int q = q0 + tx + 16 * e;
-      if (q < b) Kt[(size_t)p * b + q] = acc[x][e];
-    }
+    for (int e = 0; e < 8; ++e) T[(tx + 16 * e) * ldt + p] = acc[x][e];
   }
+  __syncthreads();
+  float* Kin = K_in + (size_t)t * B * B;
+  float* Kh = K_hi + (size_t)t * b * B;
+  float* Kl = K_lo + (size_t)t * b * B;
+  for (int idx = threadIdx.x; idx < 128 * B; idx += blockDim.x) {
+    const int qq = idx / B, p = idx - qq * B;
+    const int q = q0 + qq;
+    if (q >= b || p >= nJ) continue;
+    const float v = T[qq * ldt + p];
+    const float h = tf32_head(v);
+    Kh[(size_t)q * B + p] = h;
+    Kl[(size_t)q * B + p] = v - h;
+    if (q < j + nJ) Kin[(size_t)(q - j) * B + p] = v;  // K_t[p][q] = K_t[q-j][j+p]
+  }
+}
+
+static int kmat_smem_bytes(int B) {
+  const int operands = B * B + B * 128, staged = 128 * (B + 1);
+  return (operands > staged ? operands : staged) * 4;
 }
 
 // ------------------------------------------------------------------ stream
 
-// Over columns [u0, col_end):  W -= Z[:, 0:Bp] * R[0:Bp, :]  (R row stride ldr; skipped
-// when Bp == 0; with r_upper_from >= 0 the entries of R left of U's diagonal count as
-// zero); entries of columns < j whose mask byte is set become exactly 0 (they
-// are the previous block's removed weights, now final); for SCORE != 0 the key bits
-// [30:16] of every entry in columns [j, hist_end) go into the level-1 histogram.
+// CUDA-core form of the update, for shapes the tensor-core kernel does not take.
+// Over columns [u0, col_end):  W -= Z[:, 0:Bp] * R[0:Bp, :]  with Z = Zhi + Zlo and
+// R = Rhi + Rlo (Rlo may be null; R row stride ldr, or stored transposed, R[k][q] at
+// R[q*ldr + k], when r_trans; skipped when Bp == 0; with r_upper_from >= 0 the entries
+// of R left of U's diagonal count as zero); entries of columns < j whose mask byte is set become exactly 0 (they
+// are the previous block's removed weights, now final); for SCORE != 0 the top key bits
+// (above kKeyLoBits) of every entry in columns [j, hist_end) go into the level-1 histogram.
 // Tiles of 64 rows x 128 columns, persistent grid-stride loop.
 template <int SCORE>
 __global__ void __launch_bounds__(256) stream_kernel(float* __restrict__ W, int c, int b, int u0, int j,
-                                                     int col_end, const float* __restrict__ Z, int Bp,
-                                                     int ldz, const float* __restrict__ R, int ldr,
+                                                     int col_end, const float* __restrict__ Z,
+                                                     const float* __restrict__ Zlo, int Bp, int ldz,
+                                                     const float* __restrict__ R,
+                                                     const float* __restrict__ Rlo, int ldr, int r_trans,
                                                      int r_upper_from, const uint8_t* __restrict__ mask,
                                                      const float* __restrict__ sc, int hist_end,
                                                      unsigned int* __restrict__ hist1,
@@ -156,7 +184,7 @@ __global__ void __launch_bounds__(256) stream_kernel(float* __restrict__ W, int 
       for (int idx = tid; idx < 64 * 32; idx += 256) {
         int rr = idx >> 5, kk = idx & 31;
         int r = r0 + rr, k = k0 + kk;
-        Zs[rr][kk] = (r < c && k < Bp) ? Z[(long long)r * ldz + k] : 0.f;
+        Zs[rr][kk] = (r < c && k < Bp) ? Z[(long long)r * ldz + k] + Zlo[(long long)r * ldz + k] : 0.f;
       }
       for (int idx = tid; idx < 32 * 128; idx += 256) {
         int kk = idx >> 7, cc = idx & 127;
@@ -164,7 +192,8 @@ __global__ void __launch_bounds__(256) stream_kernel(float* __restrict__ W, int 
         // r_upper_from >= 0: R's row k is row r_upper_from + k of the upper factor U, zero
         // left of the diagonal
         const bool in = k < Bp && q < col_end && (r_upper_from < 0 || q >= r_upper_from + k);
-        Rs[kk][cc] = in ? R[(long long)k * ldr + q] : 0.f;
+        const long long at = r_trans ? (long long)q * ldr + k : (long long)k * ldr + q;
+        Rs[kk][cc] = in ? (Rlo ? R[at] + Rlo[at] : R[at]) : 0.f;
       }
       __syncthreads();
 #pragma unroll 4
@@ -197,7 +226,7 @@ __global__ void __launch_bounds__(256) stream_kernel(float* __restrict__ W, int 
           if (Bp > 0) W[(long long)r * b + q] = v;
           if (SCORE != kNoScore && q < hist_end) {
             unsigned int key = key_of<SCORE>(v, __ldg(sc + q));
-            atomicAdd(&shist[key >> 16], 1u);
+            atomicAdd(&shist[key >> kKeyLoBits], 1u);
           }
         }
       }
@@ -209,6 +238,22 @@ __global__ void __launch_bounds__(256) stream_kernel(float* __restrict__ W, int 
       unsigned int v = shist[i];
       if (v) atomicAdd(&hist1[i], v);
     }
+  }
+}
+
+// Rows [jp, jp+Bp) of U over columns [jp, b), transposed (row q holds U[jp:jp+Bp, q],
+// row stride B) as TF32 head and fp32 remainder, zero left of U's diagonal: SparseGPT's
+// K-major operand of the tensor-core update.
+__global__ void urows_kernel(const float* __restrict__ H, int b, int B, int jp, int Bp, float* __restrict__ Rhi,
+                             float* __restrict__ Rlo, const pwp_stats* st) {
+  if (failed(st)) return;
+  const long long n = (long long)Bp * (b - jp);
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const int k = (int)(i % Bp), q = jp + (int)(i / Bp);
+    const float v = q >= jp + k ? H[(long long)(jp + k) * b + q] : 0.f;
+    const float h = tf32_head(v);
+    Rhi[(long long)q * B + k] = h;
+    Rlo[(long long)q * B + k] = v - h;
   }
 }
 
@@ -227,8 +272,12 @@ struct PruneBuffers {
   float* g_diag;
   float* xnorm;
   float* udiag;
-  float* Zs;
-  float* K;
+  float* Zs;       // 2c x B: TF32 heads of Z, then the remainders
+  float* K_in;     // Thanos: blocks x B x B, in-block inverse rows (fp32)
+  float* K_hi;     // Thanos: blocks x b x B, inverse rows transposed, TF32 head
+  float* K_lo;     //   ... and remainder
+  float* R_hi;     // SparseGPT: b x B, the current block's rows of U transposed, TF32 head
+  float* R_lo;     //   ... and remainder
   float* gscratch;
   void* fws;
   size_t fws_bytes;
@@ -253,8 +302,12 @@ size_t prune_ws_layout(const pwp_config* cfg, int c, int b, PruneBuffers* pb, ch
   t.g_diag = (float*)take(sizeof(float) * b);
   t.xnorm = (float*)take(sizeof(float) * b);
   t.udiag = (float*)take(sizeof(float) * b);
-  t.Zs = (float*)take(sizeof(float) * (size_t)c * B);
-  t.K = thanos ? (float*)take(sizeof(float) * (size_t)nblk * B * b) : nullptr;
+  t.Zs = (float*)take(sizeof(float) * 2 * (size_t)c * B);
+  t.K_in = thanos ? (float*)take(sizeof(float) * (size_t)nblk * B * B) : nullptr;
+  t.K_hi = thanos ? (float*)take(sizeof(float) * (size_t)nblk * B * b) : nullptr;
+  t.K_lo = thanos ? (float*)take(sizeof(float) * (size_t)nblk * B * b) : nullptr;
+  t.R_hi = thanos ? nullptr : (float*)take(sizeof(float) * (size_t)B * b);
+  t.R_lo = thanos ? nullptr : (float*)take(sizeof(float) * (size_t)B * b);
   const size_t gbytes = thanos ? solve_scratch_bytes(c, B, cfg->pattern == PWP_NM, cfg->nm_n, cfg->nm_m) : 0;
   t.gscratch = gbytes ? (float*)take(gbytes) : nullptr;
   t.fws_bytes = factor_ws_bytes(b);
@@ -269,15 +322,33 @@ static std::atomic<int> g_nsm{0};
 static std::atomic<unsigned long long> g_attr_done{0};
 
 template <int SCORE>
-static void launch_stream(float* W, int c, int b, int u0, int j, int col_end, const float* Z, int Bp, int ldz,
-                          const float* R, int ldr, int r_upper_from, const uint8_t* mask, const float* sc,
-                          int hist_end, unsigned int* hist1, const pwp_stats* st, cudaStream_t s) {
+static void launch_stream(float* W, int c, int b, int u0, int j, int col_end, const float* Z, const float* Zlo,
+                          int Bp, int ldz, const float* R, const float* Rlo, int ldr, int r_trans, int r_upper_from,
+                          const uint8_t* mask, const float* sc, int hist_end, unsigned int* hist1,
+                          const pwp_stats* st, cudaStream_t s) {
   const int smem = SCORE != kNoScore ? kHist1Bins * 4 : 0;
   const int tiles = ((col_end - u0 + 127) / 128) * ((c + 63) / 64);
   const int nsm = g_nsm.load();
   const int grid = tiles < nsm ? tiles : nsm;
-  stream_kernel<SCORE><<<grid > 0 ? grid : 1, 256, smem, s>>>(W, c, b, u0, j, col_end, Z, Bp, ldz, R, ldr,
-                                                             r_upper_from, mask, sc, hist_end, hist1, st);
+  stream_kernel<SCORE><<<grid > 0 ? grid : 1, 256, smem, s>>>(W, c, b, u0, j, col_end, Z, Zlo, Bp, ldz, R, Rlo,
+                                                             ldr, r_trans, r_upper_from, mask, sc, hist_end, hist1,
+                                                             st);
+}
+
+static void launch_stream_any(int score, float* W, int c, int b, int u0, int j, const float* Z, const float* Zlo,
+                              int Bp, int ldz, const float* R, const float* Rlo, int ldr, int r_trans,
+                              int r_upper_from,
+                              const uint8_t* mask, const float* sc, int hist_end, unsigned int* hist1,
+                              const pwp_stats* st, cudaStream_t s) {
+  if (score == kWanda)
+    launch_stream<kWanda>(W, c, b, u0, j, b, Z, Zlo, Bp, ldz, R, Rlo, ldr, r_trans, r_upper_from, mask, sc, hist_end,
+                          hist1, st, s);
+  else if (score == kObs)
+    launch_stream<kObs>(W, c, b, u0, j, b, Z, Zlo, Bp, ldz, R, Rlo, ldr, r_trans, r_upper_from, mask, sc, hist_end,
+                        hist1, st, s);
+  else
+    launch_stream<kNoScore>(W, c, b, u0, j, b, Z, Zlo, Bp, ldz, R, Rlo, ldr, r_trans, r_upper_from, mask, sc,
+                            hist_end, hist1, st, s);
 }
 
 cudaError_t launch_stats_init(pwp_stats* st, cudaStream_t s) {
@@ -311,8 +382,7 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
   if (first_on_device(g_attr_done)) {
     cudaFuncSetAttribute(stream_kernel<kWanda>, cudaFuncAttributeMaxDynamicSharedMemorySize, kHist1Bins * 4);
     cudaFuncSetAttribute(stream_kernel<kObs>, cudaFuncAttributeMaxDynamicSharedMemorySize, kHist1Bins * 4);
-    cudaFuncSetAttribute(kmat_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (kMaxBlock * kMaxBlock + kMaxBlock * 128) * 4);
+    cudaFuncSetAttribute(kmat_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kmat_smem_bytes(kMaxBlock));
     int dev = 0, nsm = kNumSM;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
@@ -335,35 +405,55 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
   ++nl;
   if (thanos) {
     dim3 g((b + 127) / 128, nblk);
-    kmat_kernel<<<g, 256, (B * B + B * 128) * 4, s>>>(H, b, B, pb.K, st);
+    kmat_kernel<<<g, 256, kmat_smem_bytes(B), s>>>(H, b, B, pb.K_in, pb.K_hi, pb.K_lo, st);
     ++nl;
   }
   const int score = nm ? kNoScore : (thanos ? kWanda : kObs);
   const float* sc = thanos ? pb.xnorm : pb.udiag;
+  const float* Zlo = pb.Zs + (size_t)c * B;
+  // tensor-core update: 16-byte rows for TMA (b, B multiples of 4), aligned W and mask
+  const bool tc_shape = (b % 4) == 0 && (B % 4) == 0 && ((uintptr_t)Wout % 16) == 0 && ((uintptr_t)mask % 4) == 0;
   for (int t = 0; t <= nblk; ++t) {
     const int j = t * B, j1 = min(b, j + B);
     const int jp = (t - 1) * B, Bp = t > 0 ? min(B, b - jp) : 0;
-    const float* R = nullptr;
-    if (t > 0) R = thanos ? pb.K + (size_t)(t - 1) * B * b : H + (size_t)jp * b;
     const int u0 = t > 0 ? jp : j;
-    const int rup = thanos ? -1 : jp;
-    if (t == nblk) {  // the last block's columns: apply its in-block update, zero its removals
-      prof_begin(kKStream, s);
-      launch_stream<kNoScore>(Wout, c, b, u0, b, b, pb.Zs, Bp, B, R, b, rup, mask, sc, b, pb.hist1, st, s);
-      prof_end(kKStream, s);
-      ++nl;
-      break;
-    }
-    const int hist_end = thanos ? b : j1;
+    const int jj = t == nblk ? b : j;          // the last pass only finishes the last block
+    const int pass_score = t == nblk ? kNoScore : score;
+    const int hist_end = t == nblk ? b : (thanos ? b : j1);
     prof_begin(kKStream, s);
-    if (score == kWanda)
-      launch_stream<kWanda>(Wout, c, b, u0, j, b, pb.Zs, Bp, B, R, b, rup, mask, sc, hist_end, pb.hist1, st, s);
-    else if (score == kObs)
-      launch_stream<kObs>(Wout, c, b, u0, j, b, pb.Zs, Bp, B, R, b, rup, mask, sc, hist_end, pb.hist1, st, s);
-    else if (t > 0)
-      launch_stream<kNoScore>(Wout, c, b, u0, j, b, pb.Zs, Bp, B, R, b, rup, mask, sc, j, pb.hist1, st, s);
+    if (t > 0) {
+      // W[:, jp:b] -= Z R with R = block t-1's rows of K (Thanos) or of U (SparseGPT)
+      bool done = false;
+      if (tc_shape) {
+        const float* Rh = thanos ? pb.K_hi + (size_t)(t - 1) * b * B : pb.R_hi;
+        const float* Rl = thanos ? pb.K_lo + (size_t)(t - 1) * b * B : pb.R_lo;
+        if (!thanos) {
+          const long long n = (long long)Bp * (b - jp);
+          const int grid = (int)min((n + 255) / 256, (long long)8 * g_nsm.load());
+          urows_kernel<<<grid, 256, 0, s>>>(H, b, B, jp, Bp, pb.R_hi, pb.R_lo, st);
+          ++nl;
+        }
+        cudaError_t e2 = cudaSuccess;
+        done = launch_stream_tc(pass_score, Wout, c, b, u0, jj, pb.Zs, Zlo, Bp, B, Rh, Rl, mask, sc, hist_end,
+                                pb.hist1, st, s, &e2);
+        if (e2 != cudaSuccess) return e2;
+      }
+      if (!done) {
+        // Thanos: K_t transposed (row stride B); SparseGPT: U's rows in place in H
+        const float* R = thanos ? pb.K_hi + (size_t)(t - 1) * b * B : H + (size_t)jp * b;
+        const float* Rlo = thanos ? pb.K_lo + (size_t)(t - 1) * b * B : nullptr;
+        launch_stream_any(pass_score, Wout, c, b, u0, jj, pb.Zs, Zlo, Bp, B, R, Rlo, thanos ? B : b, thanos ? 1 : 0,
+                          thanos ? -1 : jp, mask, sc, hist_end, pb.hist1, st, s);
+      }
+      ++nl;
+    } else if (score != kNoScore) {
+      // first block: nothing to apply yet, only the scores of the active region
+      launch_stream_any(score, Wout, c, b, j, j, pb.Zs, Zlo, 0, B, nullptr, nullptr, b, 0, -1, mask, sc, hist_end,
+                        pb.hist1, st, s);
+      ++nl;
+    }
     prof_end(kKStream, s);
-    if (score != kNoScore || t > 0) ++nl;
+    if (t == nblk) break;
     if (score != kNoScore) {
       const long long region = thanos ? (long long)c * (b - j) : (long long)c * (j1 - j);
       const long long quota = thanos ? 0 : (long long)((double)cfg->sparsity * (double)c * (double)(j1 - j));
@@ -376,7 +466,7 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
     }
     prof_begin(kKSolve, s);
     if (thanos)
-      nl += launch_thanos_solve(nm, Wout, c, b, j, B, pb.K + (size_t)t * B * b, pb.xnorm, pb.ctl, mask, pb.Zs,
+      nl += launch_thanos_solve(nm, Wout, c, b, j, B, pb.K_in + (size_t)t * B * B, pb.xnorm, pb.ctl, mask, pb.Zs,
                                 cfg->nm_n, cfg->nm_m, pb.gscratch, st, s);
     else
       nl += launch_sparsegpt_solve(nm, Wout, c, b, j, B, H, pb.udiag, pb.ctl, mask, pb.Zs, cfg->nm_n,

@@ -21,9 +21,10 @@ inline bool first_on_device(std::atomic<unsigned long long>& done) {
 }
 
 constexpr int kNumSM = 148;              // B200
-constexpr int kHist1Bits = 15;           // first radix level: key bits [30:16]
+constexpr int kKeyLoBits = 18;           // second radix level: key bits [17:0]
+constexpr int kHist1Bits = 31 - kKeyLoBits;  // first level: key bits [30:18] (32 KB of shared memory)
 constexpr int kHist1Bins = 1 << kHist1Bits;
-constexpr int kHist2Bins = 1 << 16;      // second level: key bits [15:0]
+constexpr int kHist2Bins = 1 << kKeyLoBits;
 constexpr int kFactorNB = 64;            // panel width of the blocked factorisation
 constexpr int kMaxBlock = 128;           // largest column block B
 constexpr int kSolveCtas = 2 * kNumSM;   // persistent grid of the row-solve kernel
@@ -47,7 +48,8 @@ struct Ctl {
 
 // Where device-side failures are recorded (pwp_stats::status_site).
 enum Site : int {
-  kSiteDamp = 1, kSiteCholDiag = 2, kSiteSolve = 3, kSitePick = 4, kSiteFinal = 5,
+  kSiteDamp = 1, kSiteCholDiag = 2, kSiteSolve = 3, kSitePick = 4, kSiteFinal = 5, kSiteHessian = 6,
+  kSiteStream = 7,
 };
 
 __device__ __forceinline__ bool failed(const pwp_stats* st) {
@@ -90,6 +92,15 @@ __device__ __forceinline__ float obs_score(float w, float uqq) {
 }
 
 enum ScoreKind { kNoScore = 0, kWanda = 1, kObs = 2 };
+
+// Head of an fp32 value in TF32 (round to nearest, ties away from zero).  With
+// lo = x - head (exact in fp32), x == head + lo; the tensor-core update multiplies
+// head*head + head*lo + lo*head, which carries fp32-level accuracy.
+__device__ __forceinline__ float tf32_head(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
 
 template <int SCORE>
 __device__ __forceinline__ unsigned int key_of(float w, float p) {
@@ -139,6 +150,15 @@ void launch_refine(int score, const float* W, int c, int b, int q0, int q1, cons
                    const Ctl* ctl, unsigned int* hist2, const pwp_stats* st, cudaStream_t s);
 void launch_pick2(int score, Ctl* ctl, const unsigned int* hist2, const float* W, int c, int b,
                   int j, int j1, const float* sc, pwp_stats* st, cudaStream_t s);
+
+// W[:, u0:b] -= Z R on the tensor cores (stream_tc.cu), fused with zeroing the previous
+// block's removals and the level-1 histogram of the scores of columns [j, hist_end).
+// Z (c x Bp, row stride ldz) and R, stored transposed (b x Bp, row stride ldz), come as
+// TF32 head and fp32 remainder arrays.  Returns false, launching nothing, when the
+// shape or alignment does not allow the tensor-core path.
+bool launch_stream_tc(int score, float* W, int c, int b, int u0, int j, const float* Zhi, const float* Zlo,
+                      int Bp, int ldz, const float* Rhi, const float* Rlo, const uint8_t* mask, const float* sc,
+                      int hist_end, unsigned int* hist1, pwp_stats* st, cudaStream_t s, cudaError_t* err);
 
 // per-row work of one block (solve.cu); returns the number of kernels launched
 int launch_thanos_solve(bool nm, const float* W, int c, int b, int j, int B, const float* Kt,

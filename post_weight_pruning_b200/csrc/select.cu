@@ -7,9 +7,9 @@
 //
 // Keys are the bit patterns of the non-negative fp32 scores, so ordering keys orders
 // scores.  The r-th smallest key T is found by a two-level radix select:
-//   level 1: a histogram of key bits [30:16] (built while the scores are produced),
-//   level 2: a histogram of bits [15:0] over the entries of the level-1 bin (refine),
-// then T = (bin1 << 16) | bin2.  Among entries equal to T, the order is (column, row)
+//   level 1: a histogram of key bits [30:18] (built while the scores are produced),
+//   level 2: a histogram of bits [17:0] over the entries of the level-1 bin (refine),
+// then T = (bin1 << 18) | bin2.  Among entries equal to T, the order is (column, row)
 // -- the pages do not fix one -- so when only some tied entries are taken, the cut-off
 // position inside the current block is located as well.
 #include <climits>
@@ -26,69 +26,75 @@ __device__ __forceinline__ long long warp_sum_ll(long long v) {
 }
 
 // Find, in a histogram of NB bins (1024 threads), the bin holding the `rank`-th
-// (1-based) entry.  Each warp owns a contiguous range of NB/32 bins read in coalesced
-// 32-bin chunks.  Returns the bin in *bin (-1 if the histogram holds fewer entries) and
-// the number of entries in lower bins in *before.
+// (1-based) entry.  While the range is wider than the CTA, each of the 32 warps sums
+// one 32nd of it (coalesced) and the range narrows to the warp slice holding the rank;
+// the last range (at most 1024 bins) is resolved by a CTA-wide prefix sum.  Returns
+// the bin in *bin (-1 if the histogram holds fewer entries) and the number of entries
+// in lower bins in *before.
 template <int NB>
 __device__ void find_rank(const unsigned int* __restrict__ hist, long long rank, int* bin,
                           long long* before, long long* sh_warp, int* sh_sel, long long* sh_base) {
-  constexpr int PER_WARP = NB / 32;
-  constexpr int CHUNKS = PER_WARP / 32;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const unsigned int* h = hist + warp * PER_WARP;
-  long long sum = 0;
-#pragma unroll 8
-  for (int ch = 0; ch < CHUNKS; ++ch) sum += h[ch * 32 + lane];
-  sum = warp_sum_ll(sum);
-  if (lane == 0) sh_warp[warp] = sum;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    long long cum = 0;
-    int sel = -1;
-    for (int w = 0; w < 32; ++w) {
-      if (rank > cum && rank <= cum + sh_warp[w]) { sel = w; break; }
-      cum += sh_warp[w];
+  static_assert(NB >= 32 && (NB & (NB - 1)) == 0, "power-of-two histogram");
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int base = 0;
+  int size = NB;
+  long long below = 0;
+  while (size > 1024) {
+    const int per = size / 32;
+    const unsigned int* h = hist + base + warp * per;
+    long long sum = 0;
+    for (int i = lane; i < per; i += 32) sum += h[i];
+    sum = warp_sum_ll(sum);
+    if (lane == 0) sh_warp[warp] = sum;
+    __syncthreads();
+    if (tid == 0) {
+      long long cum = 0;
+      int sel = -1;
+      for (int w = 0; w < 32; ++w) {
+        if (rank - below > cum && rank - below <= cum + sh_warp[w]) { sel = w; break; }
+        cum += sh_warp[w];
+      }
+      *sh_sel = sel;
+      *sh_base = cum;
     }
-    *sh_sel = sel;
-    *sh_base = cum;
+    __syncthreads();
+    const int sel = *sh_sel;
+    const long long cum = *sh_base;
+    __syncthreads();  // sh_warp / sh_sel are rewritten by the next round
+    if (sel < 0) {
+      *bin = -1;
+      *before = 0;
+      return;
+    }
+    base += sel * per;
+    below += cum;
+    size = per;
+  }
+  // last range: one bin per thread, inclusive prefix over the CTA
+  const long long v = tid < size ? (long long)hist[base + tid] : 0;
+  long long x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sh_warp[warp] = x;
+  if (tid == 0) *sh_sel = -1;
+  __syncthreads();
+  long long wbase = 0;
+  for (int w = 0; w < warp; ++w) wbase += sh_warp[w];
+  const long long incl = below + wbase + x;
+  // exactly one thread holds the rank when 1 <= rank <= total
+  if (v > 0 && rank > incl - v && rank <= incl) {
+    *sh_sel = base + tid;
+    *sh_base = incl - v;
   }
   __syncthreads();
   const int sel = *sh_sel;
-  if (sel < 0) {
-    *bin = -1;
-    *before = 0;
-    return;
-  }
-  if (warp == sel) {
-    long long cum = *sh_base;
-    const unsigned int* hs = hist + sel * PER_WARP;
-    for (int ch = 0; ch < CHUNKS; ++ch) {
-      long long v = hs[ch * 32 + lane];
-      long long tot = warp_sum_ll(v);
-      if (rank <= cum + tot) {
-        // inclusive prefix inside the chunk
-        long long x = v;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          long long yv = __shfl_up_sync(0xffffffffu, x, o);
-          if (lane >= o) x += yv;
-        }
-        const bool hit = (rank > cum + x - v) && (rank <= cum + x);
-        const unsigned int m = __ballot_sync(0xffffffffu, hit);
-        const int src = __ffs(m) - 1;
-        long long excl = __shfl_sync(0xffffffffu, cum + x - v, src);
-        if (lane == 0) {
-          sh_warp[0] = sel * PER_WARP + ch * 32 + src;
-          sh_warp[1] = excl;
-        }
-        break;
-      }
-      cum += tot;
-    }
-  }
-  __syncthreads();
-  *bin = (int)sh_warp[0];
-  *before = sh_warp[1];
+  const long long bef = *sh_base;
+  __syncthreads();  // the caller reuses the shared words
+  *bin = sel;
+  *before = sel < 0 ? 0 : bef;
 }
 
 __global__ void __launch_bounds__(1024) pick1_kernel(Ctl* ctl, unsigned int* __restrict__ hist1,
@@ -129,7 +135,7 @@ __global__ void __launch_bounds__(1024) pick1_kernel(Ctl* ctl, unsigned int* __r
   for (int i = threadIdx.x; i < kHist2Bins; i += blockDim.x) hist2[i] = 0u;
 }
 
-// Level-2 histogram: key bits [15:0] of the entries whose bits [30:16] equal b1.
+// Level-2 histogram: the low kKeyLoBits key bits of the entries whose top bits equal b1.
 // One row per CTA iteration, columns across threads (coalesced).
 template <int SCORE>
 __global__ void __launch_bounds__(256) refine_kernel(const float* __restrict__ W, int c, int b, int q0,
@@ -143,7 +149,7 @@ __global__ void __launch_bounds__(256) refine_kernel(const float* __restrict__ W
     const float* wr = W + (long long)r * b;
     for (int q = q0 + threadIdx.x; q < q1; q += blockDim.x) {
       unsigned int key = key_of<SCORE>(wr[q], __ldg(sc + q));
-      if ((key >> 16) == b1) atomicAdd(&hist2[key & 0xffffu], 1u);
+      if ((key >> kKeyLoBits) == b1) atomicAdd(&hist2[key & (unsigned int)(kHist2Bins - 1)], 1u);
     }
   }
 }
@@ -169,7 +175,7 @@ __global__ void __launch_bounds__(1024) pick2_kernel(Ctl* ctl, const unsigned in
     if (tid == 0) set_error(st, PWP_EBUDGET, kSitePick);
     return;
   }
-  const unsigned int T = (ctl->b1 << 16) | (unsigned int)lo;
+  const unsigned int T = (ctl->b1 << kKeyLoBits) | (unsigned int)lo;
   const long long ties = hist2[lo];
   const long long count_less = ctl->count_less + before2;
   const long long m = ctl->take - count_less;  // 1 <= m <= ties

@@ -6,7 +6,11 @@
 // R-hat = K[Q, Q] with K = inv(H_d[A, A]); z = R-hat^-1 u and the row's update is
 // delta_k = -z^T K[Q, A].  This kernel produces z (scattered into a B-wide row, zero
 // outside Q); the stream kernel then applies W[:, A] -= Z K[J, A] for all rows at once,
-// and sets W[k, Q] to exactly zero.
+// and sets W[k, Q] to exactly zero.  R-hat is gathered from the block's in-block inverse
+// K[J, J] (B x B, row stride B).
+//
+// Both kernels store a row of Z as a TF32 head (rows 0..c-1 of Zs) and its exact fp32
+// remainder (rows c..2c-1), the operand form of the tensor-core update.
 //
 // SparseGPT ("Weight Pruning in Large Language Models ...", section "SparseGPT"): the
 // column-sequential sweep inside the block, e_q = W_q / U_qq on selected entries, whose
@@ -231,7 +235,7 @@ __global__ void __launch_bounds__(256) thanos_solve_kernel(const float* __restri
       int qv[CH];
 #pragma unroll
       for (int ch = 0; ch < CH; ++ch) qv[ch] = (lane + 32 * ch < s) ? Qidx[lane + 32 * ch] : 0;
-      const bool vec = ((b & 3) == 0) && ((j & 3) == 0);
+      const bool vec = (B & 3) == 0;
       const int c4 = 4 * lane;
       for (int a0 = 0; a0 < s; a0 += 4) {
         // four K rows in flight, then the picks from registers
@@ -239,7 +243,7 @@ __global__ void __launch_bounds__(256) thanos_solve_kernel(const float* __restri
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
           const int a = a0 + r;
-          const float* krow = Kt + (size_t)(a < s ? Qidx[a] : Qidx[0]) * b + j;
+          const float* krow = Kt + (size_t)(a < s ? Qidx[a] : Qidx[0]) * B;
           if (vec && c4 + 3 < nJ) {
             kv[r] = __ldg(reinterpret_cast<const float4*>(krow + c4));
           } else {
@@ -273,10 +277,16 @@ __global__ void __launch_bounds__(256) thanos_solve_kernel(const float* __restri
       if (lane == 0) atomicAdd((unsigned long long*)&ctlp->pruned, (unsigned long long)s);
     }
     float* zrow = Zs + (long long)k * B;
+    float* zlo = zrow + (long long)c * B;
 #pragma unroll
     for (int i = 0; i < MAXI; ++i) {
       const int qq = lane + 32 * i;
-      if (qq < B) zrow[qq] = (qq < nJ && sel[i] && ok) ? y[pos[i]] : 0.f;
+      if (qq < B) {
+        const float z = (qq < nJ && sel[i] && ok) ? y[pos[i]] : 0.f;
+        const float h = tf32_head(z);
+        zrow[qq] = h;
+        zlo[qq] = z - h;
+      }
     }
     __syncwarp();
   }
@@ -335,11 +345,16 @@ __global__ void __launch_bounds__(256) sparsegpt_solve_kernel(const float* __res
   }
   uint8_t* mrow = mask + (long long)k * b + j;
   float* zrow = Zs + (long long)k * B;
+  float* zlo = zrow + (long long)c * B;
 #pragma unroll
   for (int i = 0; i < MAXI; ++i) {
     const int qq = lane + 32 * i;
     if (qq < nJ) mrow[qq] = sel[i] ? 1 : 0;
-    if (qq < B) zrow[qq] = e[i];
+    if (qq < B) {
+      const float h = tf32_head(e[i]);
+      zrow[qq] = h;
+      zlo[qq] = e[i] - h;
+    }
   }
   if (lane == 0 && s > 0) atomicAdd((unsigned long long*)&ctlp->pruned, (unsigned long long)s);
 }

@@ -1,0 +1,325 @@
+// The per-block compensation W[:, u0:b] -= Z R on the 5th-generation tensor cores,
+// fused with finishing the previous block's removals and rescoring the active region.
+//
+// "Pruning LLMs with Thanos", section "Contribution one: solve a selected set directly":
+// every row's update delta_k = -z_k^T K[Q, A] is a row of the product Z K_t (Z the z's
+// scattered into the block's B columns); section "Contribution two: keep the budget
+// global and the execution local", step 2: the active region is rescored on the updated
+// weights before the next candidate set is formed.  For SparseGPT ("Weight Pruning in
+// Large Language Models ...", section "SparseGPT") R is the block's rows of U.
+//
+// The product is a dense c x (b-u0) x B contraction.  It runs as TF32 MMAs with fp32
+// accumulation in tensor memory; each operand comes as a TF32 head and its fp32
+// remainder (x = head + lo), and the accumulator takes head*head + head*lo + lo*head,
+// which keeps the product at fp32-level accuracy (the dropped lo*lo term is below 2^-22
+// of it).
+//
+// Both operands are K-major: Z is c x B (row stride B) and R is stored transposed,
+// b x B (row q holds column q of R; TF32 operands stored N-major would need a different
+// shared-memory atom than the plain 128-byte swizzle).
+//
+// One persistent CTA per SM walks 128 x 128 output tiles:
+//   - warp 4 (one thread) streams 32-deep K slices of 128 rows of Z and of R^T with TMA
+//     into a 3-stage ring, 128-byte swizzle;
+//   - warp 5 (one thread) issues tcgen05.mma kind::tf32 (M 128, N 128, K 8) into one of
+//     two 128-column accumulators, so the epilogue of one tile overlaps the MMAs of the
+//     next;
+//   - warps 0-3 (one tile row per thread) load the row's 128 weights before the
+//     accumulator is ready, subtract it, set the previous block's removed weights to
+//     exactly 0, store, and histogram the score keys of columns [j, hist_end) in shared
+//     memory (flushed to the level-1 histogram once per CTA).
+// Every wait is bounded; a wait that runs out records PWP_ETIMEOUT and the other roles
+// of the CTA stop at their next wait.
+#include "tc_common.cuh"
+
+namespace pwp {
+namespace {
+
+using namespace tc;
+
+constexpr int TM = 128, TN = 128, TK = 32, STAGES = 3;
+constexpr int A_BYTES = TM * TK * 4;                     // 16 KB: 128 rows x 128 bytes
+constexpr int B_BYTES = TN * TK * 4;                     // 16 KB: 128 rows x 128 bytes
+constexpr int STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;   // heads and remainders of both
+constexpr int HIST_OFF = STAGES * STAGE_BYTES;
+constexpr int BAR_OFF = HIST_OFF + kHist1Bins * 4;
+constexpr int SMEM_BYTES = 1024 + BAR_OFF + 128;
+constexpr int kAccCols = 2 * TN;
+constexpr int kProducerWarp = 4, kMmaWarp = 5, kThreads = 192;
+// kind::tf32 instruction descriptor: D fp32, A and B tf32, both K-major, N = 128, M = 128
+constexpr uint32_t IDESC = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(TN >> 3) << 17) |
+                           ((uint32_t)(TM >> 4) << 24);
+
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+
+__device__ __forceinline__ void mma_tf32(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(da), "l"(db), "r"(IDESC), "r"(acc)
+      : "memory");
+}
+
+template <int SCORE>
+__global__ void __launch_bounds__(kThreads, 1)
+    stream_tc_kernel(const __grid_constant__ CUtensorMap mzh, const __grid_constant__ CUtensorMap mzl,
+                     const __grid_constant__ CUtensorMap mrh, const __grid_constant__ CUtensorMap mrl,
+                     float* __restrict__ W, int c, int b, int u0, int j, int Bp,
+                     const uint8_t* __restrict__ mask, const float* __restrict__ sc, int hist_end,
+                     unsigned int* __restrict__ hist1, pwp_stats* st) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  unsigned int* shist = reinterpret_cast<unsigned int*>(smem + HIST_OFF);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;   // accumulator a holds a finished tile
+  uint64_t* tempty = tfull + 2;       // accumulator a has been read out
+  uint64_t* drain = tempty + 2;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+  volatile int* abortp = &abort_flag;
+
+  if (cta_failed(st)) return;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int mt = (c + TM - 1) / TM;
+  const int ntiles = mt * ((b - u0 + TN - 1) / TN);
+  const int nkc = (Bp + TK - 1) / TK;
+
+  if (SCORE != kNoScore)
+    for (int i = tid; i < kHist1Bins; i += kThreads) shist[i] = 0u;
+  if (tid == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    mbar_init(drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    abort_flag = 0;
+  }
+  if (warp == kMmaWarp) tmem_alloc(&tmem_slot, kAccCols);
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  if (warp == kProducerWarp) {
+    if (lane == 0) {
+      prefetch_map(&mzh);
+      prefetch_map(&mzl);
+      prefetch_map(&mrh);
+      prefetch_map(&mrl);
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const int m0 = (tile % mt) * TM, n0 = u0 + (tile / mt) * TN;
+        for (int kc = 0; kc < nkc; ++kc) {
+          const int s = it % STAGES;
+          if (it >= STAGES && !mbar_wait(&empty[s], ((it / STAGES) - 1) & 1, abortp)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&full[s], STAGE_BYTES);
+          uint8_t* a = smem + s * STAGE_BYTES;
+          tma_load_2d(a, &mzh, &full[s], kc * TK, m0);
+          tma_load_2d(a + A_BYTES, &mzl, &full[s], kc * TK, m0);
+          tma_load_2d(a + 2 * A_BYTES, &mrh, &full[s], kc * TK, n0);
+          tma_load_2d(a + 2 * A_BYTES + B_BYTES, &mrl, &full[s], kc * TK, n0);
+          ++it;
+        }
+      }
+      if (!ok) {
+        *abortp = 1;
+        // the copies already issued land before the CTA leaves
+        for (int k = it - STAGES > 0 ? it - STAGES : 0; k < it; ++k) mbar_wait(&full[k % STAGES], (k / STAGES) & 1);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      const uint32_t sbase = smem_u32(smem);
+      int it = 0, tc = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tc) {
+        const int acc = tc & 1;
+        if (tc >= 2 && !mbar_wait(&tempty[acc], ((tc >> 1) - 1) & 1, abortp)) {
+          ok = false;
+          break;
+        }
+        fence_after();
+        const uint32_t d = tmem + (uint32_t)(acc * TN);
+        for (int kc = 0; kc < nkc; ++kc) {
+          const int s = it % STAGES;
+          if (!mbar_wait(&full[s], (it / STAGES) & 1, abortp)) {
+            ok = false;
+            break;
+          }
+          fence_after();
+          const uint32_t ah = sbase + s * STAGE_BYTES, al = ah + A_BYTES;
+          const uint32_t bh = ah + 2 * A_BYTES, bl = bh + B_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < TK / 8; ++kk) {
+            // K-major: a K step of 8 is 32 bytes inside each 128-byte row
+            const uint64_t dah = sw128_desc(ah + kk * 32, 16, 1024);
+            const uint64_t dal = sw128_desc(al + kk * 32, 16, 1024);
+            const uint64_t dbh = sw128_desc(bh + kk * 32, 16, 1024);
+            const uint64_t dbl = sw128_desc(bl + kk * 32, 16, 1024);
+            mma_tf32(d, dah, dbh, (kc | kk) != 0 ? 1u : 0u);
+            mma_tf32(d, dah, dbl, 1u);
+            mma_tf32(d, dal, dbh, 1u);
+          }
+          mma_commit(&empty[s]);
+          ++it;
+        }
+        if (!ok) break;
+        mma_commit(&tfull[acc]);
+      }
+      if (!ok) {
+        *abortp = 1;
+        mma_commit(drain);  // completes once every MMA issued so far has finished
+        mbar_wait(drain, 0);
+      }
+    }
+    __syncwarp();
+  } else {
+    // epilogue: warp w reads accumulator lanes 32w .. 32w+31, i.e. tile rows
+    int tc = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tc) {
+      const int acc = tc & 1;
+      const int m0 = (tile % mt) * TM, n0 = u0 + (tile / mt) * TN;
+      const int r = m0 + warp * 32 + lane;
+      const bool row_ok = r < c;
+      float* wrow = W + (long long)r * b;
+      // the row's weights are loaded while the tensor cores work (b % 4 == 0: a float4
+      // that starts inside the row ends inside it)
+      float4 wv[TN / 4];
+#pragma unroll
+      for (int i = 0; i < TN / 4; ++i) {
+        const int q = n0 + 4 * i;
+        wv[i] = (row_ok && q < b) ? *reinterpret_cast<const float4*>(wrow + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      bool have = mbar_wait(&tfull[acc], (tc >> 1) & 1, abortp);
+      have = __all_sync(0xffffffffu, have);
+      if (!have) {
+        if (lane == 0) *abortp = 1;
+        break;
+      }
+      fence_after();
+#pragma unroll
+      for (int ch = 0; ch < TN / 32; ++ch) {
+        float v[32];
+        __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the guards below
+        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(acc * TN + ch * 32), v);
+        const int q0 = n0 + ch * 32;
+        if (!row_ok || q0 >= b) continue;
+        uint32_t mb[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        if (q0 < j) {
+          const uint32_t* mr = reinterpret_cast<const uint32_t*>(mask + (long long)r * b + q0);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mb[i] = (q0 + 4 * i < b) ? mr[i] : 0u;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int q = q0 + 4 * i;
+          if (q >= b) break;
+          const float4 w4 = wv[ch * 8 + i];
+          float o[4] = {w4.x - v[4 * i], w4.y - v[4 * i + 1], w4.z - v[4 * i + 2], w4.w - v[4 * i + 3]};
+          float s4[4] = {0.f, 0.f, 0.f, 0.f};
+          if (SCORE != kNoScore && q + 3 >= j && q < hist_end) {
+            const float4 t = __ldg(reinterpret_cast<const float4*>(sc + q));
+            s4[0] = t.x; s4[1] = t.y; s4[2] = t.z; s4[3] = t.w;
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int qe = q + e;
+            if (qe < j) {
+              if ((mb[i] >> (8 * e)) & 0xffu) o[e] = 0.f;
+            } else if (SCORE != kNoScore && qe < hist_end) {
+              atomicAdd(&shist[key_of<SCORE>(o[e], s4[e]) >> kKeyLoBits], 1u);
+            }
+          }
+          *reinterpret_cast<float4*>(wrow + q) = make_float4(o[0], o[1], o[2], o[3]);
+        }
+      }
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  fence_before();
+  __syncthreads();
+  fence_after();
+  if (warp == kMmaWarp) tmem_free(tmem, kAccCols);
+  if (tid == 0 && *abortp) set_error(st, PWP_ETIMEOUT, kSiteStream);
+  if (SCORE != kNoScore) {
+    for (int i = tid; i < kHist1Bins; i += kThreads) {
+      const unsigned int v = shist[i];
+      if (v) atomicAdd(&hist1[i], v);
+    }
+  }
+}
+
+template <int SCORE>
+cudaError_t launch_variant(const CUtensorMap* maps, float* W, int c, int b, int u0, int j, int Bp,
+                           const uint8_t* mask, const float* sc, int hist_end, unsigned int* hist1, pwp_stats* st,
+                           cudaStream_t s) {
+  static std::atomic<unsigned long long> attr_done{0};
+  if (first_on_device(attr_done)) {
+    cudaError_t e = cudaFuncSetAttribute(stream_tc_kernel<SCORE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+  }
+  int dev = 0, nsm = kNumSM;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  const int ntiles = ((c + TM - 1) / TM) * ((b - u0 + TN - 1) / TN);
+  const int grid = ntiles < nsm ? ntiles : nsm;
+  stream_tc_kernel<SCORE><<<grid, kThreads, SMEM_BYTES, s>>>(maps[0], maps[1], maps[2], maps[3], W, c, b, u0, j,
+                                                             Bp, mask, sc, hist_end, hist1, st);
+  return cudaGetLastError();
+}
+
+// fp32 2-D tensor map: `inner` contiguous elements per row, `rows` rows `ld` apart,
+// boxes of box_x x box_y, 128-byte swizzle, zero fill outside.
+bool encode_f32(CUtensorMap* map, const float* base, int inner, int rows, int ld, int box_x, int box_y) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (!encode) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 4};
+  cuuint32_t box[2] = {(cuuint32_t)box_x, (cuuint32_t)box_y};
+  cuuint32_t estr[2] = {1, 1};
+  return encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool launch_stream_tc(int score, float* W, int c, int b, int u0, int j, const float* Zhi, const float* Zlo, int Bp,
+                      int ldz, const float* Rhi, const float* Rlo, const uint8_t* mask, const float* sc,
+                      int hist_end, unsigned int* hist1, pwp_stats* st, cudaStream_t s, cudaError_t* err) {
+  *err = cudaSuccess;
+  // b, u0 multiples of 4: the epilogue moves whole float4s of W and 4-byte words of mask
+  if (c < 1 || Bp < 1 || Bp > ldz || u0 >= b || (b % 4) != 0 || (ldz % 4) != 0 || (u0 % 4) != 0) return false;
+  if (((uintptr_t)W % 16) != 0 || ((uintptr_t)mask % 4) != 0) return false;
+  for (const float* p : {Zhi, Zlo, Rhi, Rlo})
+    if (((uintptr_t)p % 16) != 0) return false;
+  CUtensorMap maps[4];
+  if (!encode_f32(&maps[0], Zhi, Bp, c, ldz, TK, TM) || !encode_f32(&maps[1], Zlo, Bp, c, ldz, TK, TM) ||
+      !encode_f32(&maps[2], Rhi, Bp, b, ldz, TK, TN) || !encode_f32(&maps[3], Rlo, Bp, b, ldz, TK, TN))
+    return false;
+  if (score == kWanda)
+    *err = launch_variant<kWanda>(maps, W, c, b, u0, j, Bp, mask, sc, hist_end, hist1, st, s);
+  else if (score == kObs)
+    *err = launch_variant<kObs>(maps, W, c, b, u0, j, Bp, mask, sc, hist_end, hist1, st, s);
+  else
+    *err = launch_variant<kNoScore>(maps, W, c, b, u0, j, Bp, mask, sc, hist_end, hist1, st, s);
+  return true;
+}
+
+}  // namespace pwp
