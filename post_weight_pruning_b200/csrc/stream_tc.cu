@@ -12,24 +12,26 @@
 // accumulation in tensor memory; each operand comes as a TF32 head and its fp32
 // remainder (x = head + lo), and the accumulator takes head*head + head*lo + lo*head,
 // which keeps the product at fp32-level accuracy (the dropped lo*lo term is below 2^-22
-// of it).
+// of it).  Both operands are K-major: Z is c x B (row stride B) and R is stored
+// transposed, b x B (row q holds column q of R; TF32 operands stored N-major would need
+// a different shared-memory atom than the plain 128-byte swizzle).
 //
-// Both operands are K-major: Z is c x B (row stride B) and R is stored transposed,
-// b x B (row q holds column q of R; TF32 operands stored N-major would need a different
-// shared-memory atom than the plain 128-byte swizzle).
-//
-// One persistent CTA per SM walks 128 x 128 output tiles:
-//   - warp 4 (one thread) streams 32-deep K slices of 128 rows of Z and of R^T with TMA
-//     into a 3-stage ring, 128-byte swizzle;
-//   - warp 5 (one thread) issues tcgen05.mma kind::tf32 (M 128, N 128, K 8) into one of
+// One persistent CTA per SM walks 128 x 128 output tiles with four roles:
+//   - warp 8 (one thread) streams 32-deep K slices of 128 rows of Z and of R^T with TMA
+//     into a 2-stage ring, 128-byte swizzle;
+//   - warp 9 (one thread) issues tcgen05.mma kind::tf32 (M 128, N 128, K 8) into one of
 //     two 128-column accumulators, so the epilogue of one tile overlaps the MMAs of the
 //     next;
-//   - warps 0-3 (one tile row per thread) load the row's 128 weights before the
-//     accumulator is ready, subtract it, set the previous block's removed weights to
-//     exactly 0, store, and histogram the score keys of columns [j, hist_end) in shared
-//     memory (flushed to the level-1 histogram once per CTA).
-// Every wait is bounded; a wait that runs out records PWP_ETIMEOUT and the other roles
-// of the CTA stop at their next wait.
+//   - warp 10 (one thread) brings the tile of W into shared memory with TMA, in two
+//     64-column halves with a buffer each, so a half loads while the other is worked on;
+//   - warps 0-7 (warp w: tile rows 32(w%4).., columns 32(w/4).. of each half) read the
+//     accumulator, subtract it from W in shared memory, set the previous block's removed
+//     weights to exactly 0, histogram the score keys of columns [j, hist_end) in shared
+//     memory (flushed to the level-1 histogram once per CTA), and one thread stores the
+//     half back with TMA.
+// Every wait is bounded; a wait that runs out records PWP_ETIMEOUT, the other roles stop
+// at their next wait, and the epilogue warps take each stop decision together through a
+// reducing barrier.
 #include "tc_common.cuh"
 
 namespace pwp {
@@ -37,15 +39,19 @@ namespace {
 
 using namespace tc;
 
-constexpr int TM = 128, TN = 128, TK = 32, STAGES = 3;
+constexpr int TM = 128, TN = 128, TK = 32, STAGES = 2;
 constexpr int A_BYTES = TM * TK * 4;                     // 16 KB: 128 rows x 128 bytes
 constexpr int B_BYTES = TN * TK * 4;                     // 16 KB: 128 rows x 128 bytes
 constexpr int STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;   // heads and remainders of both
-constexpr int HIST_OFF = STAGES * STAGE_BYTES;
+constexpr int W_BOX = TM * 32 * 4;                       // 16 KB: 128 rows x 32 columns of W
+constexpr int W_HALF = 2 * W_BOX;                        // 64 columns
+constexpr int W_OFF = STAGES * STAGE_BYTES;
+constexpr int HIST_OFF = W_OFF + 2 * W_HALF;
 constexpr int BAR_OFF = HIST_OFF + kHist1Bins * 4;
 constexpr int SMEM_BYTES = 1024 + BAR_OFF + 128;
 constexpr int kAccCols = 2 * TN;
-constexpr int kProducerWarp = 4, kMmaWarp = 5, kThreads = 192;
+constexpr int kEpiWarps = 8, kProducerWarp = 8, kMmaWarp = 9, kWLoadWarp = 10, kThreads = 352;
+constexpr int kEpiBarrier = 1;
 // kind::tf32 instruction descriptor: D fp32, A and B tf32, both K-major, N = 128, M = 128
 constexpr uint32_t IDESC = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(TN >> 3) << 17) |
                            ((uint32_t)(TM >> 4) << 24);
@@ -61,21 +67,27 @@ __device__ __forceinline__ void mma_tf32(uint32_t tmem_d, uint64_t da, uint64_t 
       : "memory");
 }
 
+// Byte offset of the 16-byte unit u (columns 4u..4u+3) of row r in a 128-byte-swizzled box.
+__device__ __forceinline__ uint32_t sw_off(int r, int u) { return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4)); }
+
 template <int SCORE>
 __global__ void __launch_bounds__(kThreads, 1)
     stream_tc_kernel(const __grid_constant__ CUtensorMap mzh, const __grid_constant__ CUtensorMap mzl,
                      const __grid_constant__ CUtensorMap mrh, const __grid_constant__ CUtensorMap mrl,
-                     float* __restrict__ W, int c, int b, int u0, int j, int Bp,
+                     const __grid_constant__ CUtensorMap mw, int c, int b, int u0, int j, int Bp,
                      const uint8_t* __restrict__ mask, const float* __restrict__ sc, int hist_end,
                      unsigned int* __restrict__ hist1, pwp_stats* st) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* wbuf = smem + W_OFF;
   unsigned int* shist = reinterpret_cast<unsigned int*>(smem + HIST_OFF);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;   // accumulator a holds a finished tile
   uint64_t* tempty = tfull + 2;       // accumulator a has been read out
-  uint64_t* drain = tempty + 2;
+  uint64_t* wfull = tempty + 2;       // W half h is in shared memory
+  uint64_t* wfree = wfull + 2;        // W half h has been stored back
+  uint64_t* drain = wfree + 2;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   volatile int* abortp = &abort_flag;
@@ -95,7 +107,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);
+      mbar_init(&tempty[a], kEpiWarps);
+      mbar_init(&wfull[a], 1);
+      mbar_init(&wfree[a], 1);
     }
     mbar_init(drain, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -185,70 +199,137 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
+  } else if (warp == kWLoadWarp) {
+    if (lane == 0) {
+      prefetch_map(&mw);
+      int tc = 0, issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tc) {
+        const int m0 = (tile % mt) * TM, n0 = u0 + (tile / mt) * TN;
+        for (int h = 0; h < 2; ++h) {
+          if (tc >= 1 && !mbar_wait(&wfree[h], (tc - 1) & 1, abortp)) {
+            ok = false;
+            break;
+          }
+          uint8_t* dst = wbuf + h * W_HALF;
+          mbar_expect_tx(&wfull[h], W_HALF);
+          tma_load_2d(dst, &mw, &wfull[h], n0 + 64 * h, m0);
+          tma_load_2d(dst + W_BOX, &mw, &wfull[h], n0 + 64 * h + 32, m0);
+          ++issued;
+        }
+      }
+      if (!ok) {
+        *abortp = 1;
+        for (int k = issued - 2 > 0 ? issued - 2 : 0; k < issued; ++k) mbar_wait(&wfull[k & 1], (k >> 1) & 1);
+      }
+    }
+    __syncwarp();
   } else {
-    // epilogue: warp w reads accumulator lanes 32w .. 32w+31, i.e. tile rows
+    // epilogue: warp w reads accumulator lanes 32(w%4).. (tile rows) and, in each half,
+    // the 32 columns 32(w/4)..
+    const int quarter = warp & 3, colsel = warp >> 2;
+    const int rl = quarter * 32 + lane;  // tile row of this thread
     int tc = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tc) {
       const int acc = tc & 1;
       const int m0 = (tile % mt) * TM, n0 = u0 + (tile / mt) * TN;
-      const int r = m0 + warp * 32 + lane;
+      const int r = m0 + rl;
       const bool row_ok = r < c;
-      float* wrow = W + (long long)r * b;
-      // the row's weights are loaded while the tensor cores work (b % 4 == 0: a float4
-      // that starts inside the row ends inside it)
-      float4 wv[TN / 4];
+      bool ok = mbar_wait(&tfull[acc], (tc >> 1) & 1, abortp);
+      bool stop = false;
+      for (int h = 0; h < 2; ++h) {
+        ok = ok && mbar_wait(&wfull[h], tc & 1, abortp);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+          fence_after();
+          float v[32];
+          tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * TN + h * 64 + colsel * 32), v);
+          if (h == 1) {  // this warp is done with the accumulator
+            fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[acc]);
+          }
+          const int q0 = n0 + h * 64 + colsel * 32;
+          uint8_t* box = wbuf + h * W_HALF + colsel * W_BOX;
+          if (q0 + 32 <= j) {
+            // previous block: apply, and zero the removed weights
+            const uint32_t* mr = reinterpret_cast<const uint32_t*>(mask + (long long)r * b + q0);
 #pragma unroll
-      for (int i = 0; i < TN / 4; ++i) {
-        const int q = n0 + 4 * i;
-        wv[i] = (row_ok && q < b) ? *reinterpret_cast<const float4*>(wrow + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int u = 0; u < 8; ++u) {
+              float4* p4 = reinterpret_cast<float4*>(box + sw_off(rl, u));
+              float4 w4 = *p4;
+              const uint32_t mb = row_ok ? mr[u] : 0u;
+              w4.x = (mb & 0xffu) ? 0.f : w4.x - v[4 * u];
+              w4.y = (mb & 0xff00u) ? 0.f : w4.y - v[4 * u + 1];
+              w4.z = (mb & 0xff0000u) ? 0.f : w4.z - v[4 * u + 2];
+              w4.w = (mb & 0xff000000u) ? 0.f : w4.w - v[4 * u + 3];
+              *p4 = w4;
+            }
+          } else if (q0 >= j && q0 + 32 <= hist_end && q0 + 32 <= b) {
+            // active columns, all scored
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              float4* p4 = reinterpret_cast<float4*>(box + sw_off(rl, u));
+              float4 w4 = *p4;
+              w4.x -= v[4 * u];
+              w4.y -= v[4 * u + 1];
+              w4.z -= v[4 * u + 2];
+              w4.w -= v[4 * u + 3];
+              *p4 = w4;
+              if (SCORE != kNoScore && row_ok) {
+                const float4 s4 = __ldg(reinterpret_cast<const float4*>(sc + q0 + 4 * u));
+                atomicAdd(&shist[key_of<SCORE>(w4.x, s4.x) >> kKeyLoBits], 1u);
+                atomicAdd(&shist[key_of<SCORE>(w4.y, s4.y) >> kKeyLoBits], 1u);
+                atomicAdd(&shist[key_of<SCORE>(w4.z, s4.z) >> kKeyLoBits], 1u);
+                atomicAdd(&shist[key_of<SCORE>(w4.w, s4.w) >> kKeyLoBits], 1u);
+              }
+            }
+          } else if (q0 < b) {
+            // mixed chunk (block edge, scored-range edge or the layer's last columns)
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              float4* p4 = reinterpret_cast<float4*>(box + sw_off(rl, u));
+              float o[4];
+              {
+                const float4 w4 = *p4;
+                o[0] = w4.x - v[4 * u];
+                o[1] = w4.y - v[4 * u + 1];
+                o[2] = w4.z - v[4 * u + 2];
+                o[3] = w4.w - v[4 * u + 3];
+              }
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int q = q0 + 4 * u + e;
+                if (!row_ok || q >= b) continue;
+                if (q < j) {
+                  if (mask[(long long)r * b + q]) o[e] = 0.f;
+                } else if (SCORE != kNoScore && q < hist_end) {
+                  atomicAdd(&shist[key_of<SCORE>(o[e], __ldg(sc + q)) >> kKeyLoBits], 1u);
+                }
+              }
+              *p4 = make_float4(o[0], o[1], o[2], o[3]);
+            }
+          }
+          fence_proxy_async_smem();
+        }
+        stop = barrier_or(kEpiBarrier, kEpiWarps * 32, !ok || *abortp);
+        if (stop) break;
+        if (tid == 0) {
+          // the whole half goes back; rows and columns outside W are not written
+          const uint8_t* src = wbuf + h * W_HALF;
+          tma_store_2d(&mw, src, n0 + 64 * h, m0);
+          tma_store_2d(&mw, src + W_BOX, n0 + 64 * h + 32, m0);
+          bulk_commit();
+          bulk_wait_read0();
+          mbar_arrive(&wfree[h]);
+        }
       }
-      bool have = mbar_wait(&tfull[acc], (tc >> 1) & 1, abortp);
-      have = __all_sync(0xffffffffu, have);
-      if (!have) {
+      if (stop) {
         if (lane == 0) *abortp = 1;
         break;
       }
-      fence_after();
-#pragma unroll
-      for (int ch = 0; ch < TN / 32; ++ch) {
-        float v[32];
-        __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the guards below
-        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(acc * TN + ch * 32), v);
-        const int q0 = n0 + ch * 32;
-        if (!row_ok || q0 >= b) continue;
-        uint32_t mb[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-        if (q0 < j) {
-          const uint32_t* mr = reinterpret_cast<const uint32_t*>(mask + (long long)r * b + q0);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) mb[i] = (q0 + 4 * i < b) ? mr[i] : 0u;
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int q = q0 + 4 * i;
-          if (q >= b) break;
-          const float4 w4 = wv[ch * 8 + i];
-          float o[4] = {w4.x - v[4 * i], w4.y - v[4 * i + 1], w4.z - v[4 * i + 2], w4.w - v[4 * i + 3]};
-          float s4[4] = {0.f, 0.f, 0.f, 0.f};
-          if (SCORE != kNoScore && q + 3 >= j && q < hist_end) {
-            const float4 t = __ldg(reinterpret_cast<const float4*>(sc + q));
-            s4[0] = t.x; s4[1] = t.y; s4[2] = t.z; s4[3] = t.w;
-          }
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int qe = q + e;
-            if (qe < j) {
-              if ((mb[i] >> (8 * e)) & 0xffu) o[e] = 0.f;
-            } else if (SCORE != kNoScore && qe < hist_end) {
-              atomicAdd(&shist[key_of<SCORE>(o[e], s4[e]) >> kKeyLoBits], 1u);
-            }
-          }
-          *reinterpret_cast<float4*>(wrow + q) = make_float4(o[0], o[1], o[2], o[3]);
-        }
-      }
-      fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
     }
+    if (tid == 0) bulk_wait0();
   }
 
   fence_before();
@@ -265,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int SCORE>
-cudaError_t launch_variant(const CUtensorMap* maps, float* W, int c, int b, int u0, int j, int Bp,
+cudaError_t launch_variant(const CUtensorMap* maps, int c, int b, int u0, int j, int Bp,
                            const uint8_t* mask, const float* sc, int hist_end, unsigned int* hist1, pwp_stats* st,
                            cudaStream_t s) {
   static std::atomic<unsigned long long> attr_done{0};
@@ -279,8 +360,8 @@ cudaError_t launch_variant(const CUtensorMap* maps, float* W, int c, int b, int 
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   const int ntiles = ((c + TM - 1) / TM) * ((b - u0 + TN - 1) / TN);
   const int grid = ntiles < nsm ? ntiles : nsm;
-  stream_tc_kernel<SCORE><<<grid, kThreads, SMEM_BYTES, s>>>(maps[0], maps[1], maps[2], maps[3], W, c, b, u0, j,
-                                                             Bp, mask, sc, hist_end, hist1, st);
+  stream_tc_kernel<SCORE><<<grid, kThreads, SMEM_BYTES, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4], c, b, u0,
+                                                             j, Bp, mask, sc, hist_end, hist1, st);
   return cudaGetLastError();
 }
 
@@ -309,16 +390,17 @@ bool launch_stream_tc(int score, float* W, int c, int b, int u0, int j, const fl
   if (((uintptr_t)W % 16) != 0 || ((uintptr_t)mask % 4) != 0) return false;
   for (const float* p : {Zhi, Zlo, Rhi, Rlo})
     if (((uintptr_t)p % 16) != 0) return false;
-  CUtensorMap maps[4];
+  CUtensorMap maps[5];
   if (!encode_f32(&maps[0], Zhi, Bp, c, ldz, TK, TM) || !encode_f32(&maps[1], Zlo, Bp, c, ldz, TK, TM) ||
-      !encode_f32(&maps[2], Rhi, Bp, b, ldz, TK, TN) || !encode_f32(&maps[3], Rlo, Bp, b, ldz, TK, TN))
+      !encode_f32(&maps[2], Rhi, Bp, b, ldz, TK, TN) || !encode_f32(&maps[3], Rlo, Bp, b, ldz, TK, TN) ||
+      !encode_f32(&maps[4], W, b, c, b, 32, TM))
     return false;
   if (score == kWanda)
-    *err = launch_variant<kWanda>(maps, W, c, b, u0, j, Bp, mask, sc, hist_end, hist1, st, s);
+    *err = launch_variant<kWanda>(maps, c, b, u0, j, Bp, mask, sc, hist_end, hist1, st, s);
   else if (score == kObs)
-    *err = launch_variant<kObs>(maps, W, c, b, u0, j, Bp, mask, sc, hist_end, hist1, st, s);
+    *err = launch_variant<kObs>(maps, c, b, u0, j, Bp, mask, sc, hist_end, hist1, st, s);
   else
-    *err = launch_variant<kNoScore>(maps, W, c, b, u0, j, Bp, mask, sc, hist_end, hist1, st, s);
+    *err = launch_variant<kNoScore>(maps, c, b, u0, j, Bp, mask, sc, hist_end, hist1, st, s);
   return true;
 }
 
