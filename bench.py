@@ -387,6 +387,7 @@ def run_mine(args):
             "config": _config(wl),
             "roofline": roof,
             "phases_ms": phase_ms,
+            "select_stats": {"blocks": nblk, "reread_blocks": int(st.reread_blocks), "tie_blocks": int(st.tie_blocks)},
             "gpu_launches": int(launches),
             "e2e": {"value": e2e_value, "unit": UNIT,
                     "h2d_bytes_per_step": int(W_host.numel() * 2 + X_host.numel() * 2),

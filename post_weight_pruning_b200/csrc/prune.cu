@@ -38,6 +38,11 @@ __global__ void init_ctl_kernel(Ctl* ctl, long long zstar, pwp_stats* st, long l
   ctl->zstar = zstar;
   ctl->pruned = 0;
   ctl->mode = 0;
+  ctl->b1 = 0;
+  ctl->b1_valid = 0;
+  ctl->l2_ready = 0;
+  ctl->dirty_pred = 0;
+  ctl->dirty_reread = 0;
   st->target = target;
 }
 
@@ -156,7 +161,8 @@ __global__ void __launch_bounds__(256) stream_kernel(float* __restrict__ W, int 
                                                      int r_upper_from, const uint8_t* __restrict__ mask,
                                                      const float* __restrict__ sc, int hist_end,
                                                      unsigned int* __restrict__ hist1,
-                                                     const pwp_stats* st) {
+                                                     const Ctl* __restrict__ ctl, unsigned int* __restrict__ h2,
+                                                     unsigned int* __restrict__ h2s, const pwp_stats* st) {
   extern __shared__ unsigned int shist[];  // kHist1Bins when SCORE != 0
   __shared__ float Zs[64][33];
   __shared__ __align__(16) float Rs[32][128];
@@ -167,6 +173,8 @@ __global__ void __launch_bounds__(256) stream_kernel(float* __restrict__ W, int 
     for (int i = tid; i < kHist1Bins; i += blockDim.x) shist[i] = 0u;
   const int ncols = col_end - u0;
   const int tiles_c = (ncols + 127) / 128, tiles_r = (c + 63) / 64;
+  // level-1 bin of the previous block's threshold: its level-2 histogram is built here
+  const unsigned int pred = (SCORE != kNoScore && ctl->b1_valid) ? ctl->b1 : 0xffffffffu;
   const long long ntiles = (long long)tiles_c * tiles_r;
   __syncthreads();
   for (long long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
@@ -227,6 +235,7 @@ __global__ void __launch_bounds__(256) stream_kernel(float* __restrict__ W, int 
           if (SCORE != kNoScore && q < hist_end) {
             unsigned int key = key_of<SCORE>(v, __ldg(sc + q));
             atomicAdd(&shist[key >> kKeyLoBits], 1u);
+            count_level2(key, pred, h2, h2s);
           }
         }
       }
@@ -268,7 +277,7 @@ __global__ void finalize_kernel(const Ctl* ctl, pwp_stats* st, int check_budget)
 struct PruneBuffers {
   Ctl* ctl;
   unsigned int* hist1;
-  unsigned int* hist2;
+  Level2 l2;
   float* g_diag;
   float* xnorm;
   float* udiag;
@@ -298,7 +307,11 @@ size_t prune_ws_layout(const pwp_config* cfg, int c, int b, PruneBuffers* pb, ch
   PruneBuffers t;
   t.ctl = (Ctl*)take(sizeof(Ctl));
   t.hist1 = (unsigned int*)take(sizeof(unsigned int) * kHist1Bins);
-  t.hist2 = (unsigned int*)take(sizeof(unsigned int) * kHist2Bins);
+  // the four level-2 arrays are contiguous, so one memset clears them
+  t.l2.pred = (unsigned int*)take(sizeof(unsigned int) * (2 * kHist2Bins + 2 * kHist2SumBins));
+  t.l2.pred_sum = t.l2.pred ? t.l2.pred + kHist2Bins : nullptr;
+  t.l2.reread = t.l2.pred ? t.l2.pred_sum + kHist2SumBins : nullptr;
+  t.l2.reread_sum = t.l2.pred ? t.l2.reread + kHist2Bins : nullptr;
   t.g_diag = (float*)take(sizeof(float) * b);
   t.xnorm = (float*)take(sizeof(float) * b);
   t.udiag = (float*)take(sizeof(float) * b);
@@ -324,31 +337,30 @@ static std::atomic<unsigned long long> g_attr_done{0};
 template <int SCORE>
 static void launch_stream(float* W, int c, int b, int u0, int j, int col_end, const float* Z, const float* Zlo,
                           int Bp, int ldz, const float* R, const float* Rlo, int ldr, int r_trans, int r_upper_from,
-                          const uint8_t* mask, const float* sc, int hist_end, unsigned int* hist1,
-                          const pwp_stats* st, cudaStream_t s) {
+                          const uint8_t* mask, const float* sc, int hist_end, unsigned int* hist1, const Ctl* ctl,
+                          Level2 l2, const pwp_stats* st, cudaStream_t s) {
   const int smem = SCORE != kNoScore ? kHist1Bins * 4 : 0;
   const int tiles = ((col_end - u0 + 127) / 128) * ((c + 63) / 64);
   const int nsm = g_nsm.load();
   const int grid = tiles < nsm ? tiles : nsm;
   stream_kernel<SCORE><<<grid > 0 ? grid : 1, 256, smem, s>>>(W, c, b, u0, j, col_end, Z, Zlo, Bp, ldz, R, Rlo,
                                                              ldr, r_trans, r_upper_from, mask, sc, hist_end, hist1,
-                                                             st);
+                                                             ctl, l2.pred, l2.pred_sum, st);
 }
 
 static void launch_stream_any(int score, float* W, int c, int b, int u0, int j, const float* Z, const float* Zlo,
                               int Bp, int ldz, const float* R, const float* Rlo, int ldr, int r_trans,
-                              int r_upper_from,
-                              const uint8_t* mask, const float* sc, int hist_end, unsigned int* hist1,
-                              const pwp_stats* st, cudaStream_t s) {
+                              int r_upper_from, const uint8_t* mask, const float* sc, int hist_end,
+                              unsigned int* hist1, const Ctl* ctl, Level2 l2, const pwp_stats* st, cudaStream_t s) {
   if (score == kWanda)
     launch_stream<kWanda>(W, c, b, u0, j, b, Z, Zlo, Bp, ldz, R, Rlo, ldr, r_trans, r_upper_from, mask, sc, hist_end,
-                          hist1, st, s);
+                          hist1, ctl, l2, st, s);
   else if (score == kObs)
     launch_stream<kObs>(W, c, b, u0, j, b, Z, Zlo, Bp, ldz, R, Rlo, ldr, r_trans, r_upper_from, mask, sc, hist_end,
-                        hist1, st, s);
+                        hist1, ctl, l2, st, s);
   else
     launch_stream<kNoScore>(W, c, b, u0, j, b, Z, Zlo, Bp, ldz, R, Rlo, ldr, r_trans, r_upper_from, mask, sc,
-                            hist_end, hist1, st, s);
+                            hist_end, hist1, ctl, l2, st, s);
 }
 
 cudaError_t launch_stats_init(pwp_stats* st, cudaStream_t s) {
@@ -395,6 +407,7 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
   }
   init_ctl_kernel<<<1, 1, 0, s>>>(pb.ctl, zstar, st, target);
   cudaMemsetAsync(pb.hist1, 0, sizeof(unsigned int) * kHist1Bins, s);
+  cudaMemsetAsync(pb.l2.pred, 0, sizeof(unsigned int) * (2 * kHist2Bins + 2 * kHist2SumBins), s);
   convert_w_kernel<<<4 * g_nsm.load(), 256, 0, s>>>(W, wtype, Wout, N);
   nl += 2;
   prof_begin(kKFactor, s);
@@ -435,7 +448,7 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
         }
         cudaError_t e2 = cudaSuccess;
         done = launch_stream_tc(pass_score, Wout, c, b, u0, jj, pb.Zs, Zlo, Bp, B, Rh, Rl, mask, sc, hist_end,
-                                pb.hist1, st, s, &e2);
+                                pb.hist1, pb.ctl, pb.l2, st, s, &e2);
         if (e2 != cudaSuccess) return e2;
       }
       if (!done) {
@@ -443,13 +456,13 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
         const float* R = thanos ? pb.K_hi + (size_t)(t - 1) * b * B : H + (size_t)jp * b;
         const float* Rlo = thanos ? pb.K_lo + (size_t)(t - 1) * b * B : nullptr;
         launch_stream_any(pass_score, Wout, c, b, u0, jj, pb.Zs, Zlo, Bp, B, R, Rlo, thanos ? B : b, thanos ? 1 : 0,
-                          thanos ? -1 : jp, mask, sc, hist_end, pb.hist1, st, s);
+                          thanos ? -1 : jp, mask, sc, hist_end, pb.hist1, pb.ctl, pb.l2, st, s);
       }
       ++nl;
     } else if (score != kNoScore) {
       // first block: nothing to apply yet, only the scores of the active region
       launch_stream_any(score, Wout, c, b, j, j, pb.Zs, Zlo, 0, B, nullptr, nullptr, b, 0, -1, mask, sc, hist_end,
-                        pb.hist1, st, s);
+                        pb.hist1, pb.ctl, pb.l2, st, s);
       ++nl;
     }
     prof_end(kKStream, s);
@@ -458,11 +471,12 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
       const long long region = thanos ? (long long)c * (b - j) : (long long)c * (j1 - j);
       const long long quota = thanos ? 0 : (long long)((double)cfg->sparsity * (double)c * (double)(j1 - j));
       prof_begin(kKSelect, s);
-      launch_pick1(pb.ctl, pb.hist1, pb.hist2, region, thanos ? 1 : 0, quota, st, s);
-      launch_refine(score, Wout, c, b, j, thanos ? b : j1, sc, pb.ctl, pb.hist2, st, s);
-      launch_pick2(score, pb.ctl, pb.hist2, Wout, c, b, j, j1, sc, st, s);
+      launch_pick1(pb.ctl, pb.hist1, region, thanos ? 1 : 0, quota, st, s);
+      launch_refine(score, Wout, c, b, j, thanos ? b : j1, sc, pb.ctl, pb.l2, st, s);
+      launch_pick2(score, pb.ctl, pb.l2, Wout, c, b, j, j1, sc, st, s);
+      launch_clear_level2(pb.ctl, pb.l2, s);
       prof_end(kKSelect, s);
-      nl += 3;
+      nl += 4;
     }
     prof_begin(kKSolve, s);
     if (thanos)

@@ -25,6 +25,8 @@ constexpr int kKeyLoBits = 18;           // second radix level: key bits [17:0]
 constexpr int kHist1Bits = 31 - kKeyLoBits;  // first level: key bits [30:18] (32 KB of shared memory)
 constexpr int kHist1Bins = 1 << kHist1Bits;
 constexpr int kHist2Bins = 1 << kKeyLoBits;
+constexpr int kHist2SumShift = 9;        // level-2 summary: 512 bins of 512 level-2 bins
+constexpr int kHist2SumBins = kHist2Bins >> kHist2SumShift;
 constexpr int kFactorNB = 64;            // panel width of the blocked factorisation
 constexpr int kMaxBlock = 128;           // largest column block B
 constexpr int kSolveCtas = 2 * kNumSM;   // persistent grid of the row-solve kernel
@@ -43,7 +45,12 @@ struct Ctl {
   unsigned int r1;        // rank of the threshold inside bin b1 (1-based)
   unsigned int T;         // exact 31-bit score key of the threshold
   int mode;               // 0: select nothing, 1: key/position rule
-  int pad[6];
+  int b1_valid;           // b1 holds the previous block's level-1 bin: the scoring pass
+                          // histograms the low key bits of that bin as it goes
+  int l2_ready;           // this block's bin is the predicted one: no re-read needed
+  int dirty_pred;         // the predicted level-2 histogram holds counts to clear
+  int dirty_reread;       // the re-read level-2 histogram holds counts to clear
+  int pad[2];
 };
 
 // Where device-side failures are recorded (pwp_stats::status_site).
@@ -107,6 +114,17 @@ __device__ __forceinline__ unsigned int key_of(float w, float p) {
   return SCORE == kWanda ? score_key(wanda_score(w, p)) : score_key(obs_score(w, p));
 }
 
+// Level-2 histogram entry of a key whose level-1 bin is the predicted one (pred is
+// 0xffffffff when there is no prediction): the exact count plus its 512-bin summary.
+__device__ __forceinline__ void count_level2(unsigned int key, unsigned int pred, unsigned int* __restrict__ h2,
+                                             unsigned int* __restrict__ h2s) {
+  if ((key >> kKeyLoBits) == pred) {
+    const unsigned int lo = key & (unsigned int)(kHist2Bins - 1);
+    atomicAdd(&h2[lo], 1u);
+    atomicAdd(&h2s[lo >> kHist2SumShift], 1u);
+  }
+}
+
 // Selection flag of one entry of block row k (column qq of the block).
 // Unstructured: key < T, or key == T with column-major position qq*c + k at or before
 // the tie cut-off.  N:M: rank inside the group of nm_m lanes by (key, column) below
@@ -143,13 +161,23 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
                                size_t ws_bytes, pwp_stats* st, cudaStream_t s);
 size_t factor_ws_bytes(int b);
 
+// Level-2 histograms of one block: `pred` is filled by the scoring pass for the predicted
+// level-1 bin, `reread` by the re-read when the prediction missed; each with its summary.
+struct Level2 {
+  unsigned int* pred;
+  unsigned int* pred_sum;
+  unsigned int* reread;
+  unsigned int* reread_sum;
+};
+
 // exact selection of the `take` smallest keys of a region (select.cu)
-void launch_pick1(Ctl* ctl, unsigned int* hist1, unsigned int* hist2, long long region_n,
-                  int global_budget, long long quota, pwp_stats* st, cudaStream_t s);
+void launch_pick1(Ctl* ctl, unsigned int* hist1, long long region_n, int global_budget, long long quota,
+                  pwp_stats* st, cudaStream_t s);
 void launch_refine(int score, const float* W, int c, int b, int q0, int q1, const float* sc,
-                   const Ctl* ctl, unsigned int* hist2, const pwp_stats* st, cudaStream_t s);
-void launch_pick2(int score, Ctl* ctl, const unsigned int* hist2, const float* W, int c, int b,
-                  int j, int j1, const float* sc, pwp_stats* st, cudaStream_t s);
+                   const Ctl* ctl, Level2 l2, const pwp_stats* st, cudaStream_t s);
+void launch_pick2(int score, Ctl* ctl, Level2 l2, const float* W, int c, int b, int j, int j1, const float* sc,
+                  pwp_stats* st, cudaStream_t s);
+void launch_clear_level2(const Ctl* ctl, Level2 l2, cudaStream_t s);
 
 // W[:, u0:b] -= Z R on the tensor cores (stream_tc.cu), fused with zeroing the previous
 // block's removals and the level-1 histogram of the scores of columns [j, hist_end).
@@ -158,7 +186,8 @@ void launch_pick2(int score, Ctl* ctl, const unsigned int* hist2, const float* W
 // shape or alignment does not allow the tensor-core path.
 bool launch_stream_tc(int score, float* W, int c, int b, int u0, int j, const float* Zhi, const float* Zlo,
                       int Bp, int ldz, const float* Rhi, const float* Rlo, const uint8_t* mask, const float* sc,
-                      int hist_end, unsigned int* hist1, pwp_stats* st, cudaStream_t s, cudaError_t* err);
+                      int hist_end, unsigned int* hist1, const Ctl* ctl, Level2 l2, pwp_stats* st,
+                      cudaStream_t s, cudaError_t* err);
 
 // per-row work of one block (solve.cu); returns the number of kernels launched
 int launch_thanos_solve(bool nm, const float* W, int c, int b, int j, int B, const float* Kt,

@@ -8,8 +8,10 @@
 // Keys are the bit patterns of the non-negative fp32 scores, so ordering keys orders
 // scores.  The r-th smallest key T is found by a two-level radix select:
 //   level 1: a histogram of key bits [30:18] (built while the scores are produced),
-//   level 2: a histogram of bits [17:0] over the entries of the level-1 bin (refine),
-// then T = (bin1 << 18) | bin2.  Among entries equal to T, the order is (column, row)
+//   level 2: a histogram of bits [17:0] over the entries of the level-1 bin,
+// then T = (bin1 << 18) | bin2.  The threshold's level-1 bin rarely moves from one block
+// to the next, so the scoring pass also builds the level-2 histogram of the previous
+// block's bin; only when this block's bin differs is the region read again (refine).  Among entries equal to T, the order is (column, row)
 // -- the pages do not fix one -- so when only some tied entries are taken, the cut-off
 // position inside the current block is located as well.
 #include <climits>
@@ -97,8 +99,7 @@ __device__ void find_rank(const unsigned int* __restrict__ hist, long long rank,
   *before = sel < 0 ? 0 : bef;
 }
 
-__global__ void __launch_bounds__(1024) pick1_kernel(Ctl* ctl, unsigned int* __restrict__ hist1,
-                                                     unsigned int* __restrict__ hist2, long long region_n,
+__global__ void __launch_bounds__(1024) pick1_kernel(Ctl* ctl, unsigned int* __restrict__ hist1, long long region_n,
                                                      int global_budget, long long quota, pwp_stats* st) {
   __shared__ long long sh_warp[32];
   __shared__ int sh_sel;
@@ -111,6 +112,9 @@ __global__ void __launch_bounds__(1024) pick1_kernel(Ctl* ctl, unsigned int* __r
     if (take < 0) take = 0;
     ctl->take = take;
     ctl->mode = take > 0 ? 1 : 0;
+    ctl->l2_ready = 0;
+    ctl->dirty_pred = ctl->b1_valid;  // the scoring pass counted into the predicted histogram
+    ctl->dirty_reread = 0;
     s_take = take;
   }
   __syncthreads();
@@ -124,7 +128,12 @@ __global__ void __launch_bounds__(1024) pick1_kernel(Ctl* ctl, unsigned int* __r
         set_error(st, PWP_EBUDGET, kSitePick);
         ctl->mode = 0;
       } else {
+        const bool hit = ctl->b1_valid && ctl->b1 == (unsigned int)bin;
+        ctl->l2_ready = hit ? 1 : 0;
+        ctl->dirty_reread = hit ? 0 : 1;
+        if (!hit) st->reread_blocks += 1;
         ctl->b1 = (unsigned int)bin;
+        ctl->b1_valid = 1;
         ctl->r1 = (unsigned int)(take - before);
         ctl->count_less = before;
       }
@@ -132,32 +141,28 @@ __global__ void __launch_bounds__(1024) pick1_kernel(Ctl* ctl, unsigned int* __r
     __syncthreads();
   }
   for (int i = threadIdx.x; i < kHist1Bins; i += blockDim.x) hist1[i] = 0u;
-  for (int i = threadIdx.x; i < kHist2Bins; i += blockDim.x) hist2[i] = 0u;
 }
 
-// Level-2 histogram: the low kKeyLoBits key bits of the entries whose top bits equal b1.
-// One row per CTA iteration, columns across threads (coalesced).
+// Level-2 histogram (re-read): the low kKeyLoBits key bits of the entries whose top
+// bits equal b1, when the scoring pass predicted another bin.  One row per CTA
+// iteration, columns across threads (coalesced).
 template <int SCORE>
 __global__ void __launch_bounds__(256) refine_kernel(const float* __restrict__ W, int c, int b, int q0,
                                                      int q1, const float* __restrict__ sc,
-                                                     const Ctl* __restrict__ ctl,
-                                                     unsigned int* __restrict__ hist2,
-                                                     const pwp_stats* st) {
-  if (cta_failed(st) || ctl->mode == 0) return;
+                                                     const Ctl* __restrict__ ctl, unsigned int* __restrict__ h2,
+                                                     unsigned int* __restrict__ h2s, const pwp_stats* st) {
+  if (cta_failed(st) || ctl->mode == 0 || ctl->l2_ready) return;
   const unsigned int b1 = ctl->b1;
   for (int r = blockIdx.x; r < c; r += gridDim.x) {
     const float* wr = W + (long long)r * b;
-    for (int q = q0 + threadIdx.x; q < q1; q += blockDim.x) {
-      unsigned int key = key_of<SCORE>(wr[q], __ldg(sc + q));
-      if ((key >> kKeyLoBits) == b1) atomicAdd(&hist2[key & (unsigned int)(kHist2Bins - 1)], 1u);
-    }
+    for (int q = q0 + threadIdx.x; q < q1; q += blockDim.x)
+      count_level2(key_of<SCORE>(wr[q], __ldg(sc + q)), b1, h2, h2s);
   }
 }
 
 template <int SCORE>
-__global__ void __launch_bounds__(1024) pick2_kernel(Ctl* ctl, const unsigned int* __restrict__ hist2,
-                                                     const float* __restrict__ W, int c, int b, int j,
-                                                     int j1, const float* __restrict__ sc,
+__global__ void __launch_bounds__(1024) pick2_kernel(Ctl* ctl, Level2 l2, const float* __restrict__ W, int c,
+                                                     int b, int j, int j1, const float* __restrict__ sc,
                                                      pwp_stats* st) {
   __shared__ long long sh_warp[32];
   __shared__ int sh_sel;
@@ -168,15 +173,25 @@ __global__ void __launch_bounds__(1024) pick2_kernel(Ctl* ctl, const unsigned in
   if (cta_failed(st) || ctl->mode == 0) return;
   const int tid = threadIdx.x;
   const long long r1 = ctl->r1;
-  int lo;
-  long long before2;
-  find_rank<kHist2Bins>(hist2, r1, &lo, &before2, sh_warp, &sh_sel, &sh_base);
-  if (lo < 0) {
+  const unsigned int* h2 = ctl->l2_ready ? l2.pred : l2.reread;
+  const unsigned int* h2s = ctl->l2_ready ? l2.pred_sum : l2.reread_sum;
+  // summary bin first, then the 512 level-2 bins under it
+  int sb;
+  long long before_s;
+  find_rank<kHist2SumBins>(h2s, r1, &sb, &before_s, sh_warp, &sh_sel, &sh_base);
+  int sub = -1;
+  long long before_sub = 0;
+  if (sb >= 0)
+    find_rank<(1 << kHist2SumShift)>(h2 + ((size_t)sb << kHist2SumShift), r1 - before_s, &sub, &before_sub,
+                                     sh_warp, &sh_sel, &sh_base);
+  if (sb < 0 || sub < 0) {
     if (tid == 0) set_error(st, PWP_EBUDGET, kSitePick);
     return;
   }
+  const int lo = (sb << kHist2SumShift) + sub;
+  const long long before2 = before_s + before_sub;
   const unsigned int T = (ctl->b1 << kKeyLoBits) | (unsigned int)lo;
-  const long long ties = hist2[lo];
+  const long long ties = h2[lo];
   const long long count_less = ctl->count_less + before2;
   const long long m = ctl->take - count_less;  // 1 <= m <= ties
   __syncthreads();
@@ -247,28 +262,50 @@ __global__ void __launch_bounds__(1024) pick2_kernel(Ctl* ctl, const unsigned in
   }
 }
 
+// Zero the level-2 histograms this block wrote, ready for the next block.
+__global__ void clear_level2_kernel(const Ctl* __restrict__ ctl, Level2 l2) {
+  const bool a = ctl->dirty_pred != 0, r = ctl->dirty_reread != 0;
+  if (!a && !r) return;
+  const int stride = gridDim.x * blockDim.x;
+  uint4* pa = reinterpret_cast<uint4*>(l2.pred);
+  uint4* pr = reinterpret_cast<uint4*>(l2.reread);
+  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < kHist2Bins / 4; i += stride) {
+    if (a) pa[i] = z;
+    if (r) pr[i] = z;
+  }
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < kHist2SumBins; i += stride) {
+    if (a) l2.pred_sum[i] = 0u;
+    if (r) l2.reread_sum[i] = 0u;
+  }
+}
+
 }  // namespace
 
-void launch_pick1(Ctl* ctl, unsigned int* hist1, unsigned int* hist2, long long region_n,
-                  int global_budget, long long quota, pwp_stats* st, cudaStream_t s) {
-  pick1_kernel<<<1, 1024, 0, s>>>(ctl, hist1, hist2, region_n, global_budget, quota, st);
+void launch_pick1(Ctl* ctl, unsigned int* hist1, long long region_n, int global_budget, long long quota,
+                  pwp_stats* st, cudaStream_t s) {
+  pick1_kernel<<<1, 1024, 0, s>>>(ctl, hist1, region_n, global_budget, quota, st);
 }
 
 void launch_refine(int score, const float* W, int c, int b, int q0, int q1, const float* sc,
-                   const Ctl* ctl, unsigned int* hist2, const pwp_stats* st, cudaStream_t s) {
+                   const Ctl* ctl, Level2 l2, const pwp_stats* st, cudaStream_t s) {
   const int grid = c < 4 * kNumSM ? c : 4 * kNumSM;
   if (score == kWanda)
-    refine_kernel<kWanda><<<grid, 256, 0, s>>>(W, c, b, q0, q1, sc, ctl, hist2, st);
+    refine_kernel<kWanda><<<grid, 256, 0, s>>>(W, c, b, q0, q1, sc, ctl, l2.reread, l2.reread_sum, st);
   else
-    refine_kernel<kObs><<<grid, 256, 0, s>>>(W, c, b, q0, q1, sc, ctl, hist2, st);
+    refine_kernel<kObs><<<grid, 256, 0, s>>>(W, c, b, q0, q1, sc, ctl, l2.reread, l2.reread_sum, st);
 }
 
-void launch_pick2(int score, Ctl* ctl, const unsigned int* hist2, const float* W, int c, int b, int j,
-                  int j1, const float* sc, pwp_stats* st, cudaStream_t s) {
+void launch_pick2(int score, Ctl* ctl, Level2 l2, const float* W, int c, int b, int j, int j1, const float* sc,
+                  pwp_stats* st, cudaStream_t s) {
   if (score == kWanda)
-    pick2_kernel<kWanda><<<1, 1024, 0, s>>>(ctl, hist2, W, c, b, j, j1, sc, st);
+    pick2_kernel<kWanda><<<1, 1024, 0, s>>>(ctl, l2, W, c, b, j, j1, sc, st);
   else
-    pick2_kernel<kObs><<<1, 1024, 0, s>>>(ctl, hist2, W, c, b, j, j1, sc, st);
+    pick2_kernel<kObs><<<1, 1024, 0, s>>>(ctl, l2, W, c, b, j, j1, sc, st);
+}
+
+void launch_clear_level2(const Ctl* ctl, Level2 l2, cudaStream_t s) {
+  clear_level2_kernel<<<kNumSM, 256, 0, s>>>(ctl, l2);
 }
 
 }  // namespace pwp

@@ -76,7 +76,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __grid_constant__ CUtensorMap mrh, const __grid_constant__ CUtensorMap mrl,
                      const __grid_constant__ CUtensorMap mw, int c, int b, int u0, int j, int Bp,
                      const uint8_t* __restrict__ mask, const float* __restrict__ sc, int hist_end,
-                     unsigned int* __restrict__ hist1, pwp_stats* st) {
+                     unsigned int* __restrict__ hist1, const Ctl* __restrict__ ctl, unsigned int* __restrict__ h2,
+                     unsigned int* __restrict__ h2s, pwp_stats* st) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* wbuf = smem + W_OFF;
@@ -97,6 +98,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int mt = (c + TM - 1) / TM;
   const int ntiles = mt * ((b - u0 + TN - 1) / TN);
   const int nkc = (Bp + TK - 1) / TK;
+  // level-1 bin of the previous block's threshold: its level-2 histogram is built here
+  const unsigned int pred = (SCORE != kNoScore && ctl->b1_valid) ? ctl->b1 : 0xffffffffu;
 
   if (SCORE != kNoScore)
     for (int i = tid; i < kHist1Bins; i += kThreads) shist[i] = 0u;
@@ -278,10 +281,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               *p4 = w4;
               if (SCORE != kNoScore && row_ok) {
                 const float4 s4 = __ldg(reinterpret_cast<const float4*>(sc + q0 + 4 * u));
-                atomicAdd(&shist[key_of<SCORE>(w4.x, s4.x) >> kKeyLoBits], 1u);
-                atomicAdd(&shist[key_of<SCORE>(w4.y, s4.y) >> kKeyLoBits], 1u);
-                atomicAdd(&shist[key_of<SCORE>(w4.z, s4.z) >> kKeyLoBits], 1u);
-                atomicAdd(&shist[key_of<SCORE>(w4.w, s4.w) >> kKeyLoBits], 1u);
+                const unsigned int k0 = key_of<SCORE>(w4.x, s4.x), k1 = key_of<SCORE>(w4.y, s4.y);
+                const unsigned int k2 = key_of<SCORE>(w4.z, s4.z), k3 = key_of<SCORE>(w4.w, s4.w);
+                atomicAdd(&shist[k0 >> kKeyLoBits], 1u);
+                atomicAdd(&shist[k1 >> kKeyLoBits], 1u);
+                atomicAdd(&shist[k2 >> kKeyLoBits], 1u);
+                atomicAdd(&shist[k3 >> kKeyLoBits], 1u);
+                count_level2(k0, pred, h2, h2s);
+                count_level2(k1, pred, h2, h2s);
+                count_level2(k2, pred, h2, h2s);
+                count_level2(k3, pred, h2, h2s);
               }
             }
           } else if (q0 < b) {
@@ -304,7 +313,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (q < j) {
                   if (mask[(long long)r * b + q]) o[e] = 0.f;
                 } else if (SCORE != kNoScore && q < hist_end) {
-                  atomicAdd(&shist[key_of<SCORE>(o[e], __ldg(sc + q)) >> kKeyLoBits], 1u);
+                  const unsigned int key = key_of<SCORE>(o[e], __ldg(sc + q));
+                  atomicAdd(&shist[key >> kKeyLoBits], 1u);
+                  count_level2(key, pred, h2, h2s);
                 }
               }
               *p4 = make_float4(o[0], o[1], o[2], o[3]);
@@ -347,8 +358,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int SCORE>
 cudaError_t launch_variant(const CUtensorMap* maps, int c, int b, int u0, int j, int Bp,
-                           const uint8_t* mask, const float* sc, int hist_end, unsigned int* hist1, pwp_stats* st,
-                           cudaStream_t s) {
+                           const uint8_t* mask, const float* sc, int hist_end, unsigned int* hist1, const Ctl* ctl,
+                           Level2 l2, pwp_stats* st, cudaStream_t s) {
   static std::atomic<unsigned long long> attr_done{0};
   if (first_on_device(attr_done)) {
     cudaError_t e = cudaFuncSetAttribute(stream_tc_kernel<SCORE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -361,7 +372,8 @@ cudaError_t launch_variant(const CUtensorMap* maps, int c, int b, int u0, int j,
   const int ntiles = ((c + TM - 1) / TM) * ((b - u0 + TN - 1) / TN);
   const int grid = ntiles < nsm ? ntiles : nsm;
   stream_tc_kernel<SCORE><<<grid, kThreads, SMEM_BYTES, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4], c, b, u0,
-                                                             j, Bp, mask, sc, hist_end, hist1, st);
+                                                             j, Bp, mask, sc, hist_end, hist1, ctl, l2.pred,
+                                                             l2.pred_sum, st);
   return cudaGetLastError();
 }
 
@@ -383,7 +395,8 @@ bool encode_f32(CUtensorMap* map, const float* base, int inner, int rows, int ld
 
 bool launch_stream_tc(int score, float* W, int c, int b, int u0, int j, const float* Zhi, const float* Zlo, int Bp,
                       int ldz, const float* Rhi, const float* Rlo, const uint8_t* mask, const float* sc,
-                      int hist_end, unsigned int* hist1, pwp_stats* st, cudaStream_t s, cudaError_t* err) {
+                      int hist_end, unsigned int* hist1, const Ctl* ctl, Level2 l2, pwp_stats* st, cudaStream_t s,
+                      cudaError_t* err) {
   *err = cudaSuccess;
   // b, u0 multiples of 4: the epilogue moves whole float4s of W and 4-byte words of mask
   if (c < 1 || Bp < 1 || Bp > ldz || u0 >= b || (b % 4) != 0 || (ldz % 4) != 0 || (u0 % 4) != 0) return false;
@@ -396,11 +409,11 @@ bool launch_stream_tc(int score, float* W, int c, int b, int u0, int j, const fl
       !encode_f32(&maps[4], W, b, c, b, 32, TM))
     return false;
   if (score == kWanda)
-    *err = launch_variant<kWanda>(maps, c, b, u0, j, Bp, mask, sc, hist_end, hist1, st, s);
+    *err = launch_variant<kWanda>(maps, c, b, u0, j, Bp, mask, sc, hist_end, hist1, ctl, l2, st, s);
   else if (score == kObs)
-    *err = launch_variant<kObs>(maps, c, b, u0, j, Bp, mask, sc, hist_end, hist1, st, s);
+    *err = launch_variant<kObs>(maps, c, b, u0, j, Bp, mask, sc, hist_end, hist1, ctl, l2, st, s);
   else
-    *err = launch_variant<kNoScore>(maps, c, b, u0, j, Bp, mask, sc, hist_end, hist1, st, s);
+    *err = launch_variant<kNoScore>(maps, c, b, u0, j, Bp, mask, sc, hist_end, hist1, ctl, l2, st, s);
   return true;
 }
 
