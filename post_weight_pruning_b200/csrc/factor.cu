@@ -57,19 +57,23 @@ __global__ void __launch_bounds__(1024) damp_kernel(float* __restrict__ H, int b
 // Factor the nb x nb diagonal block (nb <= 64) held in A (symmetric; the upper triangle
 // is read) as A = V V^T with V upper triangular, and invert V.  256 threads.
 // Working on the reversed matrix P = J A J (J the reversal), this is the ordinary
-// Cholesky P = L L^T from the top-left, with V = J L J and V^-1 = J L^-1 J.  Each
-// thread keeps a 4x4 cyclic sub-block of P (rows ty + 16a, columns tx + 16c) in
-// registers; every pivot step needs one barrier, with the pivot column broadcast
-// through a double-buffered shared vector.  Entries beyond nb are an identity pad.
+// Cholesky P = L L^T from the top-left, with V = J L J and V^-1 = J L^-1 J.  One
+// right-looking sweep produces both L and X = L^-1: at pivot k, column k of L is the
+// pivot column scaled by 1/sqrt(P_kk); row k of X (which already holds every earlier
+// pivot's elimination) is final once scaled the same way, and is then eliminated from
+// the rows below it, as the trailing part of P is.  Each thread keeps a 4x4 cyclic
+// sub-block of P and of X (rows ty + 16a, columns tx + 16c) in registers; a pivot step
+// needs one barrier, with the pivot column of P and pivot row of X broadcast through
+// double-buffered shared vectors.  Entries beyond nb are an identity pad.
 // On return A's upper triangle holds V and Wi holds V^-1 (upper, zero below).
 // Returns false on a non-positive pivot (recorded in st).
 __device__ bool factor_diag_block(float (*A)[NB + 1], float (*Wi)[NB + 1], int nb, int* bad,
                                   pwp_stats* st) {
   __shared__ float colbuf[2][NB];
-  __shared__ float Lsh[NB][NB + 1];
+  __shared__ float rowbuf[2][NB];
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   const int off = NB - nb;  // P[r][s] = A[nb-1-(r-off)][...] for r, s >= off; identity before
-  float P[4][4];
+  float P[4][4], X[4][4];
 #pragma unroll
   for (int a = 0; a < 4; ++a)
 #pragma unroll
@@ -83,89 +87,59 @@ __device__ bool factor_diag_block(float (*A)[NB + 1], float (*Wi)[NB + 1], int n
         v = ar <= as ? A[ar][as] : A[as][ar];
       }
       P[a][c] = v;
+      X[a][c] = (r == s) ? 1.f : 0.f;
     }
   if (tid == 0) *bad = 0;
-  // Cholesky of P; pivot k = 16 kb + kk keeps the register index kb a constant
+  // pivot k = 16 kb + kk keeps the register index kb a constant
 #pragma unroll
   for (int kb = 0; kb < 4; ++kb)
   for (int kk = 0; kk < 16; ++kk) {
     const int k = 16 * kb + kk;
     float* cb = colbuf[k & 1];
+    float* rb = rowbuf[k & 1];
     if (tx == kk) {
 #pragma unroll
       for (int a = 0; a < 4; ++a) cb[ty + 16 * a] = P[a][kb];
     }
+    if (ty == kk) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) rb[tx + 16 * c] = X[kb][c];
+    }
     __syncthreads();
     const float d = cb[k];
-    if (!(d > 0.f) || !isfinite(d)) {
+    if (!(d > 0.f) || !isfinite(d)) {   // the same value for every thread
       if (tid == 0) {
         *bad = 1;
         set_error(st, PWP_ENOTSPD, kSiteCholDiag);
       }
       return false;
     }
-    const float inv_l = 1.f / sqrtf(d);
-    const float inv_d = inv_l * inv_l;
-    float lr[4], cs[4];
+    const float inv_l = rsqrtf(d);
+    float lr[4], cs[4], xk[4];
 #pragma unroll
     for (int a = 0; a < 4; ++a) lr[a] = cb[ty + 16 * a] * inv_l;    // L[r][k]
 #pragma unroll
-    for (int c = 0; c < 4; ++c) cs[c] = cb[tx + 16 * c] * inv_l;    // L[s][k]
+    for (int c = 0; c < 4; ++c) {
+      cs[c] = cb[tx + 16 * c] * inv_l;                              // L[s][k]
+      xk[c] = rb[tx + 16 * c] * inv_l;                              // X[k][s], final
+    }
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
       const int r = ty + 16 * a;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int s = tx + 16 * c;
-        if (s == k && r >= k) P[a][c] = lr[a];                       // final column k of L
-        else if (r > k && s > k) P[a][c] = fmaf(-lr[a], cs[c], P[a][c]);
-      }
-    }
-    (void)inv_d;
-  }
-  // L (lower) to shared memory
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int r = ty + 16 * a, s = tx + 16 * c;
-      Lsh[r][s] = r >= s ? P[a][c] : 0.f;
-    }
-  // X = L^-1 by forward substitution on all columns at once: for k: X[k][:] /= L[k][k],
-  // then X[r][:] -= L[r][k] X[k][:] for r > k.  Thread keeps the same 4x4 sub-block.
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) P[a][c] = (ty + 16 * a == tx + 16 * c) ? 1.f : 0.f;
-  __syncthreads();
-#pragma unroll
-  for (int kb = 0; kb < 4; ++kb)
-  for (int kk = 0; kk < 16; ++kk) {
-    const int k = 16 * kb + kk;
-    float* rb = colbuf[k & 1];
-    if (ty == kk) {
-      const float ilkk = 1.f / Lsh[k][k];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        P[kb][c] = P[kb][c] * ilkk;
-        rb[tx + 16 * c] = P[kb][c];
-      }
-    }
-    __syncthreads();
-    float lr[4], xs[4];
-#pragma unroll
-    for (int a = 0; a < 4; ++a) lr[a] = Lsh[ty + 16 * a][k];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) xs[c] = rb[tx + 16 * c];
-#pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      if (ty + 16 * a > k) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) P[a][c] = fmaf(-lr[a], xs[c], P[a][c]);
+        if (s == k) {
+          if (r >= k) P[a][c] = lr[a];                              // column k of L
+        } else if (r > k && s > k) {
+          P[a][c] = fmaf(-lr[a], cs[c], P[a][c]);
+        }
+        if (r == k) X[a][c] = xk[c];
+        else if (r > k) X[a][c] = fmaf(-lr[a], xk[c], X[a][c]);
       }
     }
   }
-  __syncthreads();
+  __syncthreads();  // every thread is done reading A
   // back to A's orientation: V[i][j] = L[NB-1-i][NB-1-j], V^-1[i][j] = X[NB-1-i][NB-1-j]
 #pragma unroll
   for (int a = 0; a < 4; ++a)
@@ -175,8 +149,8 @@ __device__ bool factor_diag_block(float (*A)[NB + 1], float (*Wi)[NB + 1], int n
       if (r >= off && s >= off) {                      // inside the nb block
         const int i = NB - 1 - r, jj = NB - 1 - s;     // the same reversal as on load
         if (i <= jj) {
-          A[i][jj] = Lsh[r][s];
-          Wi[i][jj] = P[a][c];
+          A[i][jj] = P[a][c];
+          Wi[i][jj] = X[a][c];
         } else {
           Wi[i][jj] = 0.f;
         }
