@@ -123,19 +123,27 @@ __device__ bool factor_diag_block(float (*A)[NB + 1], float (*Wi)[NB + 1], int n
       cs[c] = cb[tx + 16 * c] * inv_l;                              // L[s][k]
       xk[c] = rb[tx + 16 * c] * inv_l;                              // X[k][s], final
     }
+    // r = ty + 16a and k = 16kb + kk with a, kb compile-time: r > k is decided at
+    // compile time except in register row a == kb (likewise for columns)
+    const bool ty_gt = ty > kk, ty_eq = ty == kk, tx_gt = tx > kk, tx_eq = tx == kk;
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
-      const int r = ty + 16 * a;
+      if (a < kb) continue;                                         // rows above the pivot
+      const bool r_gt = a > kb || ty_gt, r_eq = a == kb && ty_eq;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const int s = tx + 16 * c;
-        if (s == k) {
-          if (r >= k) P[a][c] = lr[a];                              // column k of L
-        } else if (r > k && s > k) {
-          P[a][c] = fmaf(-lr[a], cs[c], P[a][c]);
+        if (c >= kb) {                                              // P: columns >= k
+          const bool s_eq = c == kb && tx_eq, s_gt = c > kb || tx_gt;
+          if (s_eq) {
+            if (r_gt || r_eq) P[a][c] = lr[a];                      // column k of L
+          } else if (r_gt && s_gt) {
+            P[a][c] = fmaf(-lr[a], cs[c], P[a][c]);
+          }
         }
-        if (r == k) X[a][c] = xk[c];
-        else if (r > k) X[a][c] = fmaf(-lr[a], xk[c], X[a][c]);
+        if (c <= kb) {                                              // X row k is zero right of k
+          if (r_eq) X[a][c] = xk[c];
+          else if (r_gt) X[a][c] = fmaf(-lr[a], xk[c], X[a][c]);
+        }
       }
     }
   }
@@ -182,25 +190,33 @@ __global__ void __launch_bounds__(256) chol_diag_kernel(float* __restrict__ H, i
   }
 }
 
-// Rows above the panel: V[r, P] = A[r, P] (V_PP^T)^-1 = A[r, P] Wi^T, r < p0.
+// Rows above the panel: V[r, P] = A[r, P] (V_PP^T)^-1 = A[r, P] Wi^T, r < p0.  One warp
+// per row over a grid of one CTA per SM (the 64x64 inverse is staged once per CTA);
+// lane l produces columns l and l + 32.
 __global__ void __launch_bounds__(256) chol_panel_kernel(float* __restrict__ H, int b, int p0, int nb,
                                                          const float* __restrict__ Vinv,
                                                          const pwp_stats* st) {
-  __shared__ float Wi[NB][NB + 1];
+  __shared__ float WiT[NB][NB + 1];  // WiT[t][c] = Wi[c][t]
   __shared__ float rowbuf[8][NB];
   if (cta_failed(st)) return;
-  for (int idx = threadIdx.x; idx < NB * NB; idx += blockDim.x) Wi[idx / NB][idx % NB] = Vinv[idx];
+  for (int idx = threadIdx.x; idx < NB * NB; idx += blockDim.x) WiT[idx % NB][idx / NB] = Vinv[idx];
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int r = blockIdx.x * 8 + warp; r < p0; r += gridDim.x * 8) {
     float* hr = H + (long long)r * b + p0;
-    for (int t = lane; t < nb; t += 32) rowbuf[warp][t] = hr[t];
+    rowbuf[warp][lane] = lane < nb ? hr[lane] : 0.f;
+    rowbuf[warp][lane + 32] = lane + 32 < nb ? hr[lane + 32] : 0.f;
     __syncwarp();
-    for (int c = lane; c < nb; c += 32) {
-      float s = 0.f;
-      for (int t = c; t < nb; ++t) s = fmaf(rowbuf[warp][t], Wi[c][t], s);
-      hr[c] = s;
+    // Wi is upper triangular: Wi[c][t] = 0 for t < c
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll 8
+    for (int t = 0; t < NB; ++t) {
+      const float x = rowbuf[warp][t];
+      s0 = fmaf(x, WiT[t][lane], s0);
+      s1 = fmaf(x, WiT[t][lane + 32], s1);
     }
+    if (lane < nb) hr[lane] = s0;
+    if (lane + 32 < nb) hr[lane + 32] = s1;
     __syncwarp();
   }
 }
@@ -421,7 +437,7 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
   for (int p = np - 1; p >= 1; --p) {
     const int p0 = p * NB, nb = min(NB, b - p0);
     float* V = Vall + (size_t)p * NB * NB;
-    const int pgrid = min((p0 + 7) / 8, 4 * kNumSM);
+    const int pgrid = min((p0 + 7) / 8, kNumSM);
     chol_panel_kernel<<<pgrid, 256, 0, s>>>(H, b, p0, nb, V, st);
     const int nT = (p0 + 127) / 128;
     chol_update_kernel<<<nT * (nT + 1) / 2, 256, 2 * NB * 132 * 4, s>>>(H, b, p0, nb,
