@@ -52,9 +52,10 @@ struct Rows {
 // contributions of columns < jp (float4 dot products against the four panel rows),
 // the 4x4 diagonal block is factored in the registers of lanes 0..3 with shuffles,
 // and every other row finishes its four panel entries by a 4x4 forward substitution.
-// One __syncwarp per panel.  Returns false on a non-positive pivot (uniform).
+// One __syncwarp per panel.  The reciprocal of every diagonal entry goes to idg for the
+// back substitution.  Returns false on a non-positive pivot (uniform).
 template <int SCAP, int NS>
-__device__ bool chol_solve(const Rows<NS> R, float* __restrict__ y, int s, int lane) {
+__device__ bool chol_solve(const Rows<NS> R, float* __restrict__ y, float* __restrict__ idg, int s, int lane) {
   constexpr int MAXR = (SCAP + 1 + 31) / 32;   // rows jp..s over the 32 lanes
   for (int jp = 0; jp < s; jp += 4) {
     const float* p0 = R.row(jp);
@@ -106,8 +107,9 @@ __device__ bool chol_solve(const Rows<NS> R, float* __restrict__ y, int s, int l
       if (c < pw) {
         const float d = __shfl_sync(0xffffffffu, acc[0][c], c);
         if (!(d > 0.f)) { ok = false; break; }
-        const float l = sqrtf(d);
-        il[c] = 1.f / l;
+        il[c] = rsqrtf(d);
+        const float l = d * il[c];
+        if (lane == 0) idg[jp + c] = il[c];
         if (lane == c) acc[0][c] = l;
         else if (lane > c && lane < pw) acc[0][c] *= il[c];
 #pragma unroll
@@ -144,9 +146,13 @@ __device__ bool chol_solve(const Rows<NS> R, float* __restrict__ y, int s, int l
     }
     __syncwarp();
   }
-  // back substitution L^T z = y, four rows at a time from the bottom
+  // back substitution L^T z = y, four rows at a time from the bottom: the 4x4 corner
+  // is solved redundantly by every lane, then the rows above drop its contribution
   for (int a0 = (s - 1) & ~3; a0 >= 0; a0 -= 4) {
     const int pw = min(4, s - a0);
+    const float* rr[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) rr[c] = R.row(a0 + (c < pw ? c : pw - 1));
     float z[4];
 #pragma unroll
     for (int c = 3; c >= 0; --c) {
@@ -155,8 +161,8 @@ __device__ bool chol_solve(const Rows<NS> R, float* __restrict__ y, int s, int l
         float v = y[a0 + c];
 #pragma unroll
         for (int c2 = c + 1; c2 < 4; ++c2)
-          if (c2 < pw) v = fmaf(-R.row(a0 + c2)[a0 + c], z[c2], v);
-        z[c] = v / R.row(a0 + c)[a0 + c];
+          if (c2 < pw) v = fmaf(-rr[c2][a0 + c], z[c2], v);
+        z[c] = v * idg[a0 + c];
       }
     }
     __syncwarp();
@@ -164,7 +170,7 @@ __device__ bool chol_solve(const Rows<NS> R, float* __restrict__ y, int s, int l
       float v = y[t];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
-        if (c < pw) v = fmaf(-R.row(a0 + c)[t], z[c], v);
+        if (c < pw) v = fmaf(-rr[c][t], z[c], v);
       y[t] = v;
     }
     if (lane < pw) y[a0 + lane] = z[lane];
@@ -272,7 +278,8 @@ __global__ void __launch_bounds__(256) thanos_solve_kernel(const float* __restri
         }
       }
       __syncwarp();
-      ok = chol_solve<SCAP, NS>(R, y, s, lane);
+      __syncwarp();  // the selected indices are spent: their slots hold 1 / L_ii from here on
+      ok = chol_solve<SCAP, NS>(R, y, reinterpret_cast<float*>(Qidx), s, lane);
       if (!ok && lane == 0) set_error(st, PWP_ENOTSPD, kSiteSolve);
       if (lane == 0) atomicAdd((unsigned long long*)&ctlp->pruned, (unsigned long long)s);
     }
