@@ -45,104 +45,100 @@ struct Rows {
   __device__ __forceinline__ float* row(int i) const { return i < NS ? L + poff(i) : G + (poff(i) - poff(NS)); }
 };
 
-// Cholesky R-hat = L L^T (left-looking, 4-column panels; lanes own rows) with u carried
+// Cholesky R-hat = L L^T (left-looking, 8-column panels; lanes own rows) with u carried
 // as an extra row so that the factorisation also gives y = L^-1 u, then L^T z = y.
 // L holds R-hat's lower triangle on entry; y holds u.  On return y[0..s) = z.
-// Per panel [jp, jp+4): every row i >= jp (the u row included) first takes the
-// contributions of columns < jp (float4 dot products against the four panel rows),
-// the 4x4 diagonal block is factored in the registers of lanes 0..3 with shuffles,
-// and every other row finishes its four panel entries by a 4x4 forward substitution.
-// One __syncwarp per panel.  The reciprocal of every diagonal entry goes to idg for the
-// back substitution.  Returns false on a non-positive pivot (uniform).
+// Per panel [jp, jp+8), the rows i in [jp, s] (s: the u row) go over the lanes in rounds
+// of 32: each takes the contributions of columns < jp (float4 dot products against the
+// eight panel rows), then in the first round the 8x8 diagonal block, held by lanes
+// 0..7, is factored with shuffles; every other row finishes its eight panel entries by
+// forward substitution.  A packed row i holds columns up to 4*(i/4)+3, so rows jp..jp+3
+// of a panel touch only its first four columns.  One __syncwarp per panel.  The
+// reciprocal of every diagonal entry goes to idg for the back substitution.  Returns
+// false on a non-positive pivot (uniform).
 template <int SCAP, int NS>
 __device__ bool chol_solve(const Rows<NS> R, float* __restrict__ y, float* __restrict__ idg, int s, int lane) {
-  constexpr int MAXR = (SCAP + 1 + 31) / 32;   // rows jp..s over the 32 lanes
-  for (int jp = 0; jp < s; jp += 4) {
-    const float* p0 = R.row(jp);
-    const float* p1 = R.row(jp + 1);
-    const float* p2 = R.row(jp + 2);
-    const float* p3 = R.row(jp + 3);
-    // rows i = jp + lane + 32 r (i == s is the u row): start from their current
-    // entries jp..jp+3, then subtract the contributions of columns t < jp; each panel
-    // row is loaded once per t-step and applied to all of the lane's rows
-    float acc[MAXR][4];
-    const float* rp[MAXR];
+  for (int jp = 0; jp < s; jp += 8) {
+    const int pw = min(8, s - jp);
+    const float* pr[8];
 #pragma unroll
-    for (int r = 0; r < MAXR; ++r) {
-      const int i = jp + lane + 32 * r;
-      rp[r] = (i < s) ? R.row(i) : y;
-      if (i <= s) {
-        const float4 a = *reinterpret_cast<const float4*>(rp[r] + jp);
-        acc[r][0] = a.x; acc[r][1] = a.y; acc[r][2] = a.z; acc[r][3] = a.w;
-      } else {
-        acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
-      }
-    }
-    const int nr = (s - jp) / 32 + 1;   // rounds holding at least one row of [jp, s]
-#pragma unroll 2
-    for (int t = 0; t < jp; t += 4) {
-      const float4 q0 = *reinterpret_cast<const float4*>(p0 + t);
-      const float4 q1 = *reinterpret_cast<const float4*>(p1 + t);
-      const float4 q2 = *reinterpret_cast<const float4*>(p2 + t);
-      const float4 q3 = *reinterpret_cast<const float4*>(p3 + t);
+    for (int c = 0; c < 8; ++c) pr[c] = R.row(jp + (c < pw ? c : 0));   // padding rows: any valid row
+    const int nr = (s - jp + 1 + 31) >> 5;
+    float Ld[8][8];
+    float il[8];
 #pragma unroll
-      for (int r = 0; r < MAXR; ++r) {
-        if (r < nr && jp + lane + 32 * r <= s) {
-          const float4 x = *reinterpret_cast<const float4*>(rp[r] + t);
-          float* a = acc[r];
-          a[0] = fmaf(-x.x, q0.x, a[0]); a[0] = fmaf(-x.y, q0.y, a[0]); a[0] = fmaf(-x.z, q0.z, a[0]); a[0] = fmaf(-x.w, q0.w, a[0]);
-          a[1] = fmaf(-x.x, q1.x, a[1]); a[1] = fmaf(-x.y, q1.y, a[1]); a[1] = fmaf(-x.z, q1.z, a[1]); a[1] = fmaf(-x.w, q1.w, a[1]);
-          a[2] = fmaf(-x.x, q2.x, a[2]); a[2] = fmaf(-x.y, q2.y, a[2]); a[2] = fmaf(-x.z, q2.z, a[2]); a[2] = fmaf(-x.w, q2.w, a[2]);
-          a[3] = fmaf(-x.x, q3.x, a[3]); a[3] = fmaf(-x.y, q3.y, a[3]); a[3] = fmaf(-x.z, q3.z, a[3]); a[3] = fmaf(-x.w, q3.w, a[3]);
-        }
-      }
-    }
-    const int pw = min(4, s - jp);
-    // 4x4 diagonal block: rows jp..jp+pw-1 are acc[0] of lanes 0..pw-1
-    float il[4];
-    bool ok = true;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < 8; ++c) {
       il[c] = 1.f;
-      if (c < pw) {
-        const float d = __shfl_sync(0xffffffffu, acc[0][c], c);
-        if (!(d > 0.f)) { ok = false; break; }
-        il[c] = rsqrtf(d);
-        const float l = d * il[c];
-        if (lane == 0) idg[jp + c] = il[c];
-        if (lane == c) acc[0][c] = l;
-        else if (lane > c && lane < pw) acc[0][c] *= il[c];
 #pragma unroll
-        for (int c2 = c + 1; c2 < 4; ++c2) {
-          const float lc2 = __shfl_sync(0xffffffffu, acc[0][c], c2);   // L[jp+c2][jp+c]
-          if (lane >= c2 && lane < pw) acc[0][c2] = fmaf(-acc[0][c], lc2, acc[0][c2]);
+      for (int c2 = 0; c2 < 8; ++c2) Ld[c][c2] = 0.f;
+    }
+    for (int r = 0; r < nr; ++r) {
+      const int i = jp + lane + 32 * r;
+      float* ri = (i < s) ? R.row(i) : y;
+      const bool two = (i >= jp + 4) || (i >= s);   // the row holds panel columns jp+4..
+      float acc[8];
+      {
+        const float4 a = *reinterpret_cast<const float4*>(ri + jp);
+        acc[0] = a.x; acc[1] = a.y; acc[2] = a.z; acc[3] = a.w;
+        float4 bq = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (two) bq = *reinterpret_cast<const float4*>(ri + jp + 4);
+        acc[4] = bq.x; acc[5] = bq.y; acc[6] = bq.z; acc[7] = bq.w;
+      }
+#pragma unroll 2
+      for (int t = 0; t < jp; t += 4) {
+        const float4 x = *reinterpret_cast<const float4*>(ri + t);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const float4 q = *reinterpret_cast<const float4*>(pr[c] + t);
+          float v = acc[c];
+          v = fmaf(-x.x, q.x, v);
+          v = fmaf(-x.y, q.y, v);
+          v = fmaf(-x.z, q.z, v);
+          v = fmaf(-x.w, q.w, v);
+          acc[c] = v;
         }
       }
-    }
-    // the factored block, broadcast: Ld[c][c2] = L[jp+c][jp+c2], c2 <= c
-    float Ld[4][4];
+      if (r == 0) {
+        // the 8x8 diagonal block: rows jp..jp+pw-1 are acc of lanes 0..pw-1
+        bool ok = true;
 #pragma unroll
-    for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < 8; ++c) {
+          if (c < pw) {
+            const float d = __shfl_sync(0xffffffffu, acc[c], c);
+            if (!(d > 0.f)) { ok = false; break; }
+            il[c] = rsqrtf(d);
+            if (lane == c) acc[c] = d * il[c];
+            else if (lane > c && lane < pw) acc[c] *= il[c];
+            if (lane == 0) idg[jp + c] = il[c];
 #pragma unroll
-      for (int c2 = 0; c2 < 4; ++c2) Ld[c][c2] = (c2 <= c) ? __shfl_sync(0xffffffffu, acc[0][c2], c) : 0.f;
-    if (!ok) return false;
-    // finish the panel entries of every row below the block and write back
+            for (int c2 = c + 1; c2 < 8; ++c2) {
+              const float lc2 = __shfl_sync(0xffffffffu, acc[c], c2);   // L[jp+c2][jp+c]
+              if (lane >= c2 && lane < pw) acc[c2] = fmaf(-acc[c], lc2, acc[c2]);
+            }
+          }
+        }
+        if (!ok) return false;
 #pragma unroll
-    for (int r = 0; r < MAXR; ++r) {
-      const int i = jp + lane + 32 * r;
-      if (i > s) continue;
-      float* ri = (i < s) ? R.row(i) : y;
-      float4 o;
-      if (i < jp + pw && i < s) {
-        o = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
-      } else {
-        const float x0 = acc[r][0] * il[0];
-        const float x1 = (acc[r][1] - x0 * Ld[1][0]) * il[1];
-        const float x2 = (acc[r][2] - x0 * Ld[2][0] - x1 * Ld[2][1]) * il[2];
-        const float x3 = (acc[r][3] - x0 * Ld[3][0] - x1 * Ld[3][1] - x2 * Ld[3][2]) * il[3];
-        o = make_float4(x0, x1, x2, x3);
+        for (int c = 0; c < 8; ++c)
+#pragma unroll
+          for (int c2 = 0; c2 <= c; ++c2) Ld[c][c2] = __shfl_sync(0xffffffffu, acc[c2], c);
       }
-      *reinterpret_cast<float4*>(ri + jp) = o;
+      if (i > s) continue;
+      if (i < jp + pw && i < s) {
+        *reinterpret_cast<float4*>(ri + jp) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        if (two) *reinterpret_cast<float4*>(ri + jp + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+      } else {
+        float x[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          float v = acc[c];
+#pragma unroll
+          for (int c2 = 0; c2 < c; ++c2) v = fmaf(-x[c2], Ld[c][c2], v);
+          x[c] = v * il[c];
+        }
+        *reinterpret_cast<float4*>(ri + jp) = make_float4(x[0], x[1], x[2], x[3]);
+        *reinterpret_cast<float4*>(ri + jp + 4) = make_float4(x[4], x[5], x[6], x[7]);
+      }
     }
     __syncwarp();
   }
