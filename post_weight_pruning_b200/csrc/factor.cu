@@ -192,9 +192,12 @@ __global__ void __launch_bounds__(256) chol_diag_kernel(float* __restrict__ H, i
 
 // Rows above the panel: V[r, P] = A[r, P] (V_PP^T)^-1 = A[r, P] Wi^T, r < p0.  One warp
 // per row over a grid of one CTA per SM (the 64x64 inverse is staged once per CTA);
-// lane l produces columns l and l + 32.
+// lane l produces columns l and l + 32.  With vs_hi set, the rows also go to vs_hi /
+// vs_lo (row stride NB) as TF32 head and fp32 remainder: the operand of the tensor-core
+// trailing update.
 __global__ void __launch_bounds__(256) chol_panel_kernel(float* __restrict__ H, int b, int p0, int nb,
                                                          const float* __restrict__ Vinv,
+                                                         float* __restrict__ vs_hi, float* __restrict__ vs_lo,
                                                          const pwp_stats* st) {
   __shared__ float WiT[NB][NB + 1];  // WiT[t][c] = Wi[c][t]
   __shared__ float rowbuf[8][NB];
@@ -217,6 +220,13 @@ __global__ void __launch_bounds__(256) chol_panel_kernel(float* __restrict__ H, 
     }
     if (lane < nb) hr[lane] = s0;
     if (lane + 32 < nb) hr[lane + 32] = s1;
+    if (vs_hi) {
+      const float h0 = tf32_head(s0), h1 = tf32_head(s1);
+      vs_hi[(size_t)r * NB + lane] = h0;
+      vs_lo[(size_t)r * NB + lane] = s0 - h0;
+      vs_hi[(size_t)r * NB + lane + 32] = h1;
+      vs_lo[(size_t)r * NB + lane + 32] = s1 - h1;
+    }
     __syncwarp();
   }
 }
@@ -400,10 +410,9 @@ void launch_trigemm(const TriGemm& g, int batch, const pwp_stats* st, cudaStream
 
 }  // namespace
 
-size_t factor_ws_bytes(int b) {
-  const size_t np = (size_t)(b + NB - 1) / NB;
-  // temporary of the doubling levels: the full pairs of a level, or its ragged pair,
-  // whichever is larger (the two run one after the other on the stream)
+// Floats of the doubling levels' temporary: the full pairs of a level, or its ragged
+// pair, whichever is larger (the two run one after the other on the stream).
+static size_t doubling_tmp_floats(int b) {
   size_t tmp = 0;
   for (size_t m = NB; m < (size_t)b; m *= 2) {
     const size_t full = (size_t)b / (2 * m), rest = (size_t)b - full * 2 * m;
@@ -411,7 +420,14 @@ size_t factor_ws_bytes(int b) {
     if (rest > m && m * (rest - m) > need) need = m * (rest - m);
     if (need > tmp) tmp = need;
   }
-  return np * NB * NB * sizeof(float) + tmp * sizeof(float) + 256;
+  return tmp;
+}
+
+// Diagonal-block inverses, the doubling temporary, and the current panel's rows as TF32
+// head and remainder (2 x b x NB), the last 256-byte aligned.
+size_t factor_ws_bytes(int b) {
+  const size_t np = (size_t)(b + NB - 1) / NB;
+  return (np * NB * NB + doubling_tmp_floats(b) + 2 * (size_t)b * NB) * sizeof(float) + 512;
 }
 
 cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void* ws, size_t ws_bytes,
@@ -419,6 +435,9 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
   const int np = (b + NB - 1) / NB;
   float* Vall = (float*)ws;
   float* T = Vall + (size_t)np * NB * NB;
+  float* vs_hi = reinterpret_cast<float*>(
+      (reinterpret_cast<uintptr_t>(T + doubling_tmp_floats(b)) + 255) & ~(uintptr_t)255);
+  float* vs_lo = vs_hi + (size_t)b * NB;
   static std::atomic<unsigned long long> attr_done{0};
   if (first_on_device(attr_done)) {
     cudaFuncSetAttribute(chol_update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * NB * 132 * 4);
@@ -438,11 +457,22 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
     const int p0 = p * NB, nb = min(NB, b - p0);
     float* V = Vall + (size_t)p * NB * NB;
     const int pgrid = min((p0 + 7) / 8, kNumSM);
-    chol_panel_kernel<<<pgrid, 256, 0, s>>>(H, b, p0, nb, V, st);
-    const int nT = (p0 + 127) / 128;
-    chol_update_kernel<<<nT * (nT + 1) / 2, 256, 2 * NB * 132 * 4, s>>>(H, b, p0, nb,
-                                                                      Vall + (size_t)(p - 1) * NB * NB, st);
-    nl += 2;
+    chol_panel_kernel<<<pgrid, 256, 0, s>>>(H, b, p0, nb, V, vs_hi, vs_lo, st);
+    // H[0:p0, 0:p0] -= V[0:p0, P] V[0:p0, P]^T on the tensor cores (tiles on or above the
+    // diagonal), then the next panel's diagonal block on its own; the CUDA-core kernel
+    // (which also factors that block) when the tensor-core path is not available
+    cudaError_t e2 = cudaSuccess;
+    const bool tc = launch_stream_tc(kNoScore, H, p0, p0, b, 0, 0, vs_hi, vs_lo, nb, NB, vs_hi, vs_lo, nullptr,
+                                     nullptr, 0, nullptr, nullptr, Level2{}, st, s, &e2, true);
+    if (e2 != cudaSuccess) return e2;
+    if (tc) {
+      chol_diag_kernel<<<1, 256, 2 * NB * (NB + 1) * 4, s>>>(H, b, p0 - NB, NB, Vall + (size_t)(p - 1) * NB * NB, st);
+    } else {
+      const int nT = (p0 + 127) / 128;
+      chol_update_kernel<<<nT * (nT + 1) / 2, 256, 2 * NB * 132 * 4, s>>>(H, b, p0, nb,
+                                                                        Vall + (size_t)(p - 1) * NB * NB, st);
+    }
+    nl += 3;
   }
   put_diag_inverses_kernel<<<np, 256, 0, s>>>(H, b, Vall, st);
   ++nl;

@@ -447,7 +447,7 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
           ++nl;
         }
         cudaError_t e2 = cudaSuccess;
-        done = launch_stream_tc(pass_score, Wout, c, b, u0, jj, pb.Zs, Zlo, Bp, B, Rh, Rl, mask, sc, hist_end,
+        done = launch_stream_tc(pass_score, Wout, c, b, b, u0, jj, pb.Zs, Zlo, Bp, B, Rh, Rl, mask, sc, hist_end,
                                 pb.hist1, pb.ctl, pb.l2, st, s, &e2);
         if (e2 != cudaSuccess) return e2;
       }

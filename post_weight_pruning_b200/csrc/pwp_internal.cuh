@@ -181,13 +181,15 @@ void launch_clear_level2(const Ctl* ctl, Level2 l2, cudaStream_t s);
 
 // W[:, u0:b] -= Z R on the tensor cores (stream_tc.cu), fused with zeroing the previous
 // block's removals and the level-1 histogram of the scores of columns [j, hist_end).
-// Z (c x Bp, row stride ldz) and R, stored transposed (b x Bp, row stride ldz), come as
-// TF32 head and fp32 remainder arrays.  Returns false, launching nothing, when the
-// shape or alignment does not allow the tensor-core path.
-bool launch_stream_tc(int score, float* W, int c, int b, int u0, int j, const float* Zhi, const float* Zlo,
+// W is c x b with row stride ldw (mask: row stride b); with `upper` (c == b, u0 == 0)
+// only the 128x128 tiles on or above the diagonal are visited.  Z (c x Bp, row stride ldz) and R,
+// stored transposed (b x Bp, row stride ldz), come as TF32 head and fp32 remainder
+// arrays.  Returns false, launching nothing, when the shape or alignment does not allow
+// the tensor-core path.
+bool launch_stream_tc(int score, float* W, int c, int b, int ldw, int u0, int j, const float* Zhi, const float* Zlo,
                       int Bp, int ldz, const float* Rhi, const float* Rlo, const uint8_t* mask, const float* sc,
                       int hist_end, unsigned int* hist1, const Ctl* ctl, Level2 l2, pwp_stats* st,
-                      cudaStream_t s, cudaError_t* err);
+                      cudaStream_t s, cudaError_t* err, bool upper = false);
 
 // per-row work of one block (solve.cu); returns the number of kernels launched
 int launch_thanos_solve(bool nm, const float* W, int c, int b, int j, int B, const float* Kt,

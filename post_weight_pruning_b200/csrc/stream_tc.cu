@@ -67,6 +67,21 @@ __device__ __forceinline__ void mma_tf32(uint32_t tmem_d, uint64_t da, uint64_t 
       : "memory");
 }
 
+// Origin of tile `tile` of the walk: every (m, n) tile, m fastest, or with `upper` (a
+// square W, u0 = 0) only the tiles with m <= n, column by column.
+__device__ __forceinline__ void tile_origin(int tile, int mt, int u0, int upper, int& m0, int& n0) {
+  if (!upper) {
+    m0 = (tile % mt) * TM;
+    n0 = u0 + (tile / mt) * TN;
+    return;
+  }
+  int n = (int)((sqrtf(8.f * (float)tile + 1.f) - 1.f) * 0.5f);
+  while ((n + 1) * (n + 2) / 2 <= tile) ++n;
+  while (n > 0 && n * (n + 1) / 2 > tile) --n;
+  m0 = (tile - n * (n + 1) / 2) * TM;
+  n0 = n * TN;
+}
+
 // Byte offset of the 16-byte unit u (columns 4u..4u+3) of row r in a 128-byte-swizzled box.
 __device__ __forceinline__ uint32_t sw_off(int r, int u) { return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4)); }
 
@@ -74,7 +89,7 @@ template <int SCORE>
 __global__ void __launch_bounds__(kThreads, 1)
     stream_tc_kernel(const __grid_constant__ CUtensorMap mzh, const __grid_constant__ CUtensorMap mzl,
                      const __grid_constant__ CUtensorMap mrh, const __grid_constant__ CUtensorMap mrl,
-                     const __grid_constant__ CUtensorMap mw, int c, int b, int u0, int j, int Bp,
+                     const __grid_constant__ CUtensorMap mw, int c, int b, int u0, int j, int Bp, int upper,
                      const uint8_t* __restrict__ mask, const float* __restrict__ sc, int hist_end,
                      unsigned int* __restrict__ hist1, const Ctl* __restrict__ ctl, unsigned int* __restrict__ h2,
                      unsigned int* __restrict__ h2s, pwp_stats* st) {
@@ -96,7 +111,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (cta_failed(st)) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int mt = (c + TM - 1) / TM;
-  const int ntiles = mt * ((b - u0 + TN - 1) / TN);
+  const int ntiles = upper ? mt * (mt + 1) / 2 : mt * ((b - u0 + TN - 1) / TN);
   const int nkc = (Bp + TK - 1) / TK;
   // level-1 bin of the previous block's threshold: its level-2 histogram is built here
   const unsigned int pred = (SCORE != kNoScore && ctl->b1_valid) ? ctl->b1 : 0xffffffffu;
@@ -133,7 +148,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-        const int m0 = (tile % mt) * TM, n0 = u0 + (tile / mt) * TN;
+        int m0, n0;
+        tile_origin(tile, mt, u0, upper, m0, n0);
         for (int kc = 0; kc < nkc; ++kc) {
           const int s = it % STAGES;
           if (it >= STAGES && !mbar_wait(&empty[s], ((it / STAGES) - 1) & 1, abortp)) {
@@ -208,7 +224,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int tc = 0, issued = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tc) {
-        const int m0 = (tile % mt) * TM, n0 = u0 + (tile / mt) * TN;
+        int m0, n0;
+        tile_origin(tile, mt, u0, upper, m0, n0);
         for (int h = 0; h < 2; ++h) {
           if (tc >= 1 && !mbar_wait(&wfree[h], (tc - 1) & 1, abortp)) {
             ok = false;
@@ -235,7 +252,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int tc = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tc) {
       const int acc = tc & 1;
-      const int m0 = (tile % mt) * TM, n0 = u0 + (tile / mt) * TN;
+      int m0, n0;
+        tile_origin(tile, mt, u0, upper, m0, n0);
       const int r = m0 + rl;
       const bool row_ok = r < c;
       bool ok = mbar_wait(&tfull[acc], (tc >> 1) & 1, abortp);
@@ -357,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int SCORE>
-cudaError_t launch_variant(const CUtensorMap* maps, int c, int b, int u0, int j, int Bp,
+cudaError_t launch_variant(const CUtensorMap* maps, int c, int b, int u0, int j, int Bp, int upper,
                            const uint8_t* mask, const float* sc, int hist_end, unsigned int* hist1, const Ctl* ctl,
                            Level2 l2, pwp_stats* st, cudaStream_t s) {
   static std::atomic<unsigned long long> attr_done{0};
@@ -369,10 +387,11 @@ cudaError_t launch_variant(const CUtensorMap* maps, int c, int b, int u0, int j,
   int dev = 0, nsm = kNumSM;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  const int ntiles = ((c + TM - 1) / TM) * ((b - u0 + TN - 1) / TN);
+  const int mt = (c + TM - 1) / TM;
+  const int ntiles = upper ? mt * (mt + 1) / 2 : mt * ((b - u0 + TN - 1) / TN);
   const int grid = ntiles < nsm ? ntiles : nsm;
   stream_tc_kernel<SCORE><<<grid, kThreads, SMEM_BYTES, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4], c, b, u0,
-                                                             j, Bp, mask, sc, hist_end, hist1, ctl, l2.pred,
+                                                             j, Bp, upper, mask, sc, hist_end, hist1, ctl, l2.pred,
                                                              l2.pred_sum, st);
   return cudaGetLastError();
 }
@@ -393,27 +412,30 @@ bool encode_f32(CUtensorMap* map, const float* base, int inner, int rows, int ld
 
 }  // namespace
 
-bool launch_stream_tc(int score, float* W, int c, int b, int u0, int j, const float* Zhi, const float* Zlo, int Bp,
-                      int ldz, const float* Rhi, const float* Rlo, const uint8_t* mask, const float* sc,
+bool launch_stream_tc(int score, float* W, int c, int b, int ldw, int u0, int j, const float* Zhi, const float* Zlo,
+                      int Bp, int ldz, const float* Rhi, const float* Rlo, const uint8_t* mask, const float* sc,
                       int hist_end, unsigned int* hist1, const Ctl* ctl, Level2 l2, pwp_stats* st, cudaStream_t s,
-                      cudaError_t* err) {
+                      cudaError_t* err, bool upper) {
   *err = cudaSuccess;
+  if (upper && (c != b || u0 != 0)) return false;
   // b, u0 multiples of 4: the epilogue moves whole float4s of W and 4-byte words of mask
-  if (c < 1 || Bp < 1 || Bp > ldz || u0 >= b || (b % 4) != 0 || (ldz % 4) != 0 || (u0 % 4) != 0) return false;
+  if (c < 1 || Bp < 1 || Bp > ldz || u0 >= b || (b % 4) != 0 || (ldw % 4) != 0 || ldw < b || (ldz % 4) != 0 ||
+      (u0 % 4) != 0)
+    return false;
   if (((uintptr_t)W % 16) != 0 || ((uintptr_t)mask % 4) != 0) return false;
   for (const float* p : {Zhi, Zlo, Rhi, Rlo})
     if (((uintptr_t)p % 16) != 0) return false;
   CUtensorMap maps[5];
   if (!encode_f32(&maps[0], Zhi, Bp, c, ldz, TK, TM) || !encode_f32(&maps[1], Zlo, Bp, c, ldz, TK, TM) ||
       !encode_f32(&maps[2], Rhi, Bp, b, ldz, TK, TN) || !encode_f32(&maps[3], Rlo, Bp, b, ldz, TK, TN) ||
-      !encode_f32(&maps[4], W, b, c, b, 32, TM))
+      !encode_f32(&maps[4], W, b, c, ldw, 32, TM))
     return false;
   if (score == kWanda)
-    *err = launch_variant<kWanda>(maps, c, b, u0, j, Bp, mask, sc, hist_end, hist1, ctl, l2, st, s);
+    *err = launch_variant<kWanda>(maps, c, b, u0, j, Bp, upper ? 1 : 0, mask, sc, hist_end, hist1, ctl, l2, st, s);
   else if (score == kObs)
-    *err = launch_variant<kObs>(maps, c, b, u0, j, Bp, mask, sc, hist_end, hist1, ctl, l2, st, s);
+    *err = launch_variant<kObs>(maps, c, b, u0, j, Bp, upper ? 1 : 0, mask, sc, hist_end, hist1, ctl, l2, st, s);
   else
-    *err = launch_variant<kNoScore>(maps, c, b, u0, j, Bp, mask, sc, hist_end, hist1, ctl, l2, st, s);
+    *err = launch_variant<kNoScore>(maps, c, b, u0, j, Bp, upper ? 1 : 0, mask, sc, hist_end, hist1, ctl, l2, st, s);
   return true;
 }
 
