@@ -345,9 +345,63 @@ struct TriGemm {
   int a_upper, b_upper;
 };
 
-__global__ void __launch_bounds__(256) trigemm_kernel(TriGemm g, const pwp_stats* st) {
-  __shared__ __align__(16) float As[16][128 + 4];
-  __shared__ __align__(16) float Bs[16][128 + 4];
+// Operand chunk of one 16-deep K step, held in registers between the global loads and the
+// shared-memory stores: A rows m0 + (tid >> 2) + 64 h, columns k0 + 4 (tid & 3) ..;
+// B rows k0 + (tid >> 5) + 8 h, columns n0 + 4 (tid & 31) ...
+struct TriChunk {
+  float4 a[2], b[2];
+};
+
+// vec: every row start and column origin is 16-byte aligned, so whole float4s are read
+// and the masks applied afterwards; otherwise element by element.
+__device__ __forceinline__ void trigemm_load(const TriGemm& g, const float* A, const float* B, int m0, int n0,
+                                             int k0, int kend, bool vec, TriChunk& ch) {
+  const int tid = threadIdx.x;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int m = m0 + (tid >> 2) + 64 * h, k = k0 + 4 * (tid & 3);
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
+    if (m < g.M) {
+      const float* src = A + (long long)m * g.lda + k;
+      if (vec && k + 3 < kend) {
+        const float4 t = *reinterpret_cast<const float4*>(src);
+        v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[e] = k + e < kend ? src[e] : 0.f;
+      }
+      if (g.a_upper) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[e] = k + e >= m ? v[e] : 0.f;   // A[m][k] = 0 for k < m
+      }
+    }
+    ch.a[h] = make_float4(v[0], v[1], v[2], v[3]);
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int k = k0 + (tid >> 5) + 8 * h, n = n0 + 4 * (tid & 31);
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
+    if (k < kend) {
+      const float* src = B + (long long)k * g.ldb + n;
+      if (vec && n + 3 < g.N) {
+        const float4 t = *reinterpret_cast<const float4*>(src);
+        v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[e] = n + e < g.N ? src[e] : 0.f;
+      }
+      if (g.b_upper) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[e] = n + e >= k ? v[e] : 0.f;   // B[k][n] = 0 for n < k
+      }
+    }
+    ch.b[h] = make_float4(v[0], v[1], v[2], v[3]);
+  }
+}
+
+__global__ void __launch_bounds__(256) trigemm_kernel(TriGemm g, int vec, const pwp_stats* st) {
+  __shared__ __align__(16) float As[2][16][128 + 4];
+  __shared__ __align__(16) float Bs[2][16][128 + 4];
   if (cta_failed(st)) return;
   const float* A = g.A + blockIdx.z * g.batch_a;
   const float* B = g.B + blockIdx.z * g.batch_b;
@@ -360,28 +414,29 @@ __global__ void __launch_bounds__(256) trigemm_kernel(TriGemm g, const pwp_stats
   if (g.a_upper) kbeg = m0;                       // k >= m
   if (g.b_upper) kend = min(kend, n0 + 128);      // k <= n
   float acc[8][8] = {};
+  TriChunk ch;
+  int buf = 0;
+  if (kbeg < kend) trigemm_load(g, A, B, m0, n0, kbeg, kend, vec != 0, ch);
   for (int k0 = kbeg; k0 < kend; k0 += 16) {
-    for (int idx = tid; idx < 16 * 128; idx += 256) {
-      // A tile: rows m0..m0+127, k0..k0+15 (k fastest -> coalesced in A's rows)
-      const int mm = idx >> 4, kk = idx & 15;
-      const int m = m0 + mm, k = k0 + kk;
-      float a = 0.f;
-      if (m < g.M && k < kend && (!g.a_upper || k >= m)) a = A[(long long)m * g.lda + k];
-      As[kk][mm] = a;
-      // B tile: k0..k0+15, n0..n0+127 (n fastest)
-      const int kb = idx >> 7, nn = idx & 127;
-      const int kq = k0 + kb, n = n0 + nn;
-      float bv = 0.f;
-      if (kq < kend && n < g.N && (!g.b_upper || n >= kq)) bv = B[(long long)kq * g.ldb + n];
-      Bs[kb][nn] = bv;
+    // stage the chunk in registers, fetch the next one, then compute on the stage
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int mm = (tid >> 2) + 64 * h, kk = 4 * (tid & 3);
+      As[buf][kk][mm] = ch.a[h].x;
+      As[buf][kk + 1][mm] = ch.a[h].y;
+      As[buf][kk + 2][mm] = ch.a[h].z;
+      As[buf][kk + 3][mm] = ch.a[h].w;
+      const int kb = (tid >> 5) + 8 * h, nn = 4 * (tid & 31);
+      *reinterpret_cast<float4*>(&Bs[buf][kb][nn]) = ch.b[h];
     }
     __syncthreads();
+    if (k0 + 16 < kend) trigemm_load(g, A, B, m0, n0, k0 + 16, kend, vec != 0, ch);
 #pragma unroll
     for (int kk = 0; kk < 16; ++kk) {
-      const float4 a0 = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
-      const float4 a1 = *reinterpret_cast<const float4*>(&As[kk][64 + ty * 4]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[kk][64 + tx * 4]);
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][64 + ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][kk][64 + tx * 4]);
       const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
       const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
@@ -389,23 +444,40 @@ __global__ void __launch_bounds__(256) trigemm_kernel(TriGemm g, const pwp_stats
 #pragma unroll
         for (int y = 0; y < 8; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
     }
-    __syncthreads();
+    buf ^= 1;  // the next chunk goes to the other stage: one barrier per chunk suffices
   }
 #pragma unroll
   for (int x = 0; x < 8; ++x) {
     const int m = m0 + (x < 4 ? ty * 4 + x : 64 + ty * 4 + x - 4);
     if (m >= g.M) continue;
+    float* crow = C + (long long)m * g.ldc;
+    const int na = n0 + tx * 4, nb2 = n0 + 64 + tx * 4;
+    if (vec && na + 3 < g.N) {
+      *reinterpret_cast<float4*>(crow + na) =
+          make_float4(g.alpha * acc[x][0], g.alpha * acc[x][1], g.alpha * acc[x][2], g.alpha * acc[x][3]);
+    } else {
 #pragma unroll
-    for (int y = 0; y < 8; ++y) {
-      const int n = n0 + (y < 4 ? tx * 4 + y : 64 + tx * 4 + y - 4);
-      if (n < g.N) C[(long long)m * g.ldc + n] = g.alpha * acc[x][y];
+      for (int y = 0; y < 4; ++y)
+        if (na + y < g.N) crow[na + y] = g.alpha * acc[x][y];
+    }
+    if (vec && nb2 + 3 < g.N) {
+      *reinterpret_cast<float4*>(crow + nb2) =
+          make_float4(g.alpha * acc[x][4], g.alpha * acc[x][5], g.alpha * acc[x][6], g.alpha * acc[x][7]);
+    } else {
+#pragma unroll
+      for (int y = 4; y < 8; ++y)
+        if (nb2 + y - 4 < g.N) crow[nb2 + y - 4] = g.alpha * acc[x][y];
     }
   }
 }
 
 void launch_trigemm(const TriGemm& g, int batch, const pwp_stats* st, cudaStream_t s) {
   dim3 grid((g.N + 127) / 128, (g.M + 127) / 128, batch);
-  trigemm_kernel<<<grid, 256, 0, s>>>(g, st);
+  // float4 access needs 16-byte aligned rows and batch entries
+  const bool vec = ((uintptr_t)g.A % 16) == 0 && ((uintptr_t)g.B % 16) == 0 && ((uintptr_t)g.C % 16) == 0 &&
+                   (g.lda % 4) == 0 && (g.ldb % 4) == 0 && (g.ldc % 4) == 0 && (g.batch_a % 4) == 0 &&
+                   (g.batch_b % 4) == 0 && (g.batch_c % 4) == 0;
+  trigemm_kernel<<<grid, 256, 0, s>>>(g, vec ? 1 : 0, st);
 }
 
 }  // namespace
