@@ -38,7 +38,7 @@ K_HESSIAN, K_FACTOR, K_STREAM, K_SELECT, K_SOLVE = 0, 1, 2, 3, 4
 CLASS_NAMES = {K_HESSIAN: "hessian_xxt", K_FACTOR: "factor", K_STREAM: "stream_update_score",
                K_SELECT: "select", K_SOLVE: "row_solve"}
 CLASS_SOURCES = {K_HESSIAN: ["hessian_tc.cu", "hessian_simt.cu"], K_FACTOR: ["factor.cu"],
-                 K_STREAM: ["prune.cu"], K_SELECT: ["select.cu"], K_SOLVE: ["solve.cu"]}
+                 K_STREAM: ["stream_tc.cu", "prune.cu"], K_SELECT: ["select.cu"], K_SOLVE: ["solve.cu"]}
 
 
 def _load_peaks():

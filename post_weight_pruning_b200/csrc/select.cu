@@ -209,11 +209,36 @@ __global__ void __launch_bounds__(1024) pick2_kernel(Ctl* ctl, Level2 l2, const 
   for (int i = tid; i < kMaxBlock; i += blockDim.x) colcnt[i] = 0u;
   __syncthreads();
   const int warp = tid >> 5, lane = tid & 31;
-  for (int r = warp; r < c; r += 32) {
-    for (int qq = lane; qq < nJ; qq += 32) {
-      unsigned int key = key_of<SCORE>(W[(long long)r * b + j + qq], __ldg(sc + j + qq));
-      if (key == T) atomicAdd(&colcnt[qq], 1u);
+  {
+    // lane counts block columns lane + 32e in registers; four rows' loads in flight
+    constexpr int E = kMaxBlock / 32;
+    unsigned int cnt[E];
+    float scv[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      cnt[e] = 0u;
+      scv[e] = lane + 32 * e < nJ ? __ldg(sc + j + lane + 32 * e) : 0.f;
     }
+    for (int r0 = warp; r0 < c; r0 += 32 * 4) {
+      float v[4][E];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int r = r0 + 32 * u;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int qq = lane + 32 * e;
+          v[u][e] = (r < c && qq < nJ) ? W[(long long)r * b + j + qq] : 0.f;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+          if (r0 + 32 * u < c && lane + 32 * e < nJ && key_of<SCORE>(v[u][e], scv[e]) == T) ++cnt[e];
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+      if (cnt[e]) atomicAdd(&colcnt[lane + 32 * e], cnt[e]);
   }
   __syncthreads();
   if (tid == 0) {
