@@ -307,11 +307,12 @@ size_t prune_ws_layout(const pwp_config* cfg, int c, int b, PruneBuffers* pb, ch
   PruneBuffers t;
   t.ctl = (Ctl*)take(sizeof(Ctl));
   t.hist1 = (unsigned int*)take(sizeof(unsigned int) * kHist1Bins);
-  // the four level-2 arrays are contiguous, so one memset clears them
-  t.l2.pred = (unsigned int*)take(sizeof(unsigned int) * (2 * kHist2Bins + 2 * kHist2SumBins));
+  // the level-2 arrays and the tie counts are contiguous, so one memset clears them
+  t.l2.pred = (unsigned int*)take(sizeof(unsigned int) * (2 * kHist2Bins + 2 * kHist2SumBins + kMaxBlock));
   t.l2.pred_sum = t.l2.pred ? t.l2.pred + kHist2Bins : nullptr;
   t.l2.reread = t.l2.pred ? t.l2.pred_sum + kHist2SumBins : nullptr;
   t.l2.reread_sum = t.l2.pred ? t.l2.reread + kHist2Bins : nullptr;
+  t.l2.tie_count = t.l2.pred ? t.l2.reread_sum + kHist2SumBins : nullptr;
   t.g_diag = (float*)take(sizeof(float) * b);
   t.xnorm = (float*)take(sizeof(float) * b);
   t.udiag = (float*)take(sizeof(float) * b);
@@ -407,7 +408,7 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
   }
   init_ctl_kernel<<<1, 1, 0, s>>>(pb.ctl, zstar, st, target);
   cudaMemsetAsync(pb.hist1, 0, sizeof(unsigned int) * kHist1Bins, s);
-  cudaMemsetAsync(pb.l2.pred, 0, sizeof(unsigned int) * (2 * kHist2Bins + 2 * kHist2SumBins), s);
+  cudaMemsetAsync(pb.l2.pred, 0, sizeof(unsigned int) * (2 * kHist2Bins + 2 * kHist2SumBins + kMaxBlock), s);
   convert_w_kernel<<<4 * g_nsm.load(), 256, 0, s>>>(W, wtype, Wout, N);
   nl += 2;
   prof_begin(kKFactor, s);
@@ -474,9 +475,10 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
       launch_pick1(pb.ctl, pb.hist1, region, thanos ? 1 : 0, quota, st, s);
       launch_refine(score, Wout, c, b, j, thanos ? b : j1, sc, pb.ctl, pb.l2, st, s);
       launch_pick2(score, pb.ctl, pb.l2, Wout, c, b, j, j1, sc, st, s);
-      launch_clear_level2(pb.ctl, pb.l2, s);
+      launch_clear_level2(score, pb.ctl, pb.l2, Wout, c, b, j, j1, sc, s);
+      launch_tie_pick(score, pb.ctl, pb.l2, Wout, c, b, j, j1, sc, st, s);
       prof_end(kKSelect, s);
-      nl += 4;
+      nl += 5;
     }
     prof_begin(kKSolve, s);
     if (thanos)

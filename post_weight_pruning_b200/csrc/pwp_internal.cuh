@@ -50,7 +50,8 @@ struct Ctl {
   int l2_ready;           // this block's bin is the predicted one: no re-read needed
   int dirty_pred;         // the predicted level-2 histogram holds counts to clear
   int dirty_reread;       // the re-read level-2 histogram holds counts to clear
-  int pad[2];
+  int tie_scan;           // some but not all entries tied at T are taken: locate the cut-off
+  int pad[1];
 };
 
 // Where device-side failures are recorded (pwp_stats::status_site).
@@ -168,6 +169,7 @@ struct Level2 {
   unsigned int* pred_sum;
   unsigned int* reread;
   unsigned int* reread_sum;
+  unsigned int* tie_count;   // kMaxBlock per-column counts of entries tied at T
 };
 
 // exact selection of the `take` smallest keys of a region (select.cu)
@@ -177,7 +179,12 @@ void launch_refine(int score, const float* W, int c, int b, int q0, int q1, cons
                    const Ctl* ctl, Level2 l2, const pwp_stats* st, cudaStream_t s);
 void launch_pick2(int score, Ctl* ctl, Level2 l2, const float* W, int c, int b, int j, int j1, const float* sc,
                   pwp_stats* st, cudaStream_t s);
-void launch_clear_level2(const Ctl* ctl, Level2 l2, cudaStream_t s);
+// After pick2: clear the level-2 histograms the block wrote and, when only some tied
+// entries are taken, count the ties per block column (grid-wide); then find the cut-off.
+void launch_clear_level2(int score, const Ctl* ctl, Level2 l2, const float* W, int c, int b, int j, int j1,
+                         const float* sc, cudaStream_t s);
+void launch_tie_pick(int score, Ctl* ctl, Level2 l2, const float* W, int c, int b, int j, int j1, const float* sc,
+                     pwp_stats* st, cudaStream_t s);
 
 // W[:, u0:b] -= Z R on the tensor cores (stream_tc.cu), fused with zeroing the previous
 // block's removals and the level-1 histogram of the scores of columns [j, hist_end).

@@ -115,6 +115,7 @@ __global__ void __launch_bounds__(1024) pick1_kernel(Ctl* ctl, unsigned int* __r
     ctl->l2_ready = 0;
     ctl->dirty_pred = ctl->b1_valid;  // the scoring pass counted into the predicted histogram
     ctl->dirty_reread = 0;
+    ctl->tie_scan = 0;
     s_take = take;
   }
   __syncthreads();
@@ -167,9 +168,6 @@ __global__ void __launch_bounds__(1024) pick2_kernel(Ctl* ctl, Level2 l2, const 
   __shared__ long long sh_warp[32];
   __shared__ int sh_sel;
   __shared__ long long sh_base;
-  __shared__ unsigned int colcnt[kMaxBlock];
-  __shared__ int s_qstar;
-  __shared__ long long s_need;
   if (cta_failed(st) || ctl->mode == 0) return;
   const int tid = threadIdx.x;
   const long long r1 = ctl->r1;
@@ -203,68 +201,100 @@ __global__ void __launch_bounds__(1024) pick2_kernel(Ctl* ctl, Level2 l2, const 
     ctl->pstar = LLONG_MAX;
     if (ties > 1) st->tie_blocks += 1;
   }
-  if (m >= ties) return;  // every tied entry is taken
-  // Some but not all ties are taken: count ties per block column (rows coalesced).
-  const int nJ = j1 - j;
-  for (int i = tid; i < kMaxBlock; i += blockDim.x) colcnt[i] = 0u;
-  __syncthreads();
-  const int warp = tid >> 5, lane = tid & 31;
-  {
-    // lane counts block columns lane + 32e in registers; four rows' loads in flight
-    constexpr int E = kMaxBlock / 32;
-    unsigned int cnt[E];
-    float scv[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      cnt[e] = 0u;
-      scv[e] = lane + 32 * e < nJ ? __ldg(sc + j + lane + 32 * e) : 0.f;
+  // some but not all tied entries are taken: the grid-wide count and the cut-off search follow
+  if (tid == 0) ctl->tie_scan = m < ties ? 1 : 0;
+}
+
+// Zero the level-2 histograms this block wrote, ready for the next block; and, when only
+// some of the entries tied at T are taken, count the block's tied entries per column
+// (rows over the grid's warps, lane l counting columns l + 32e in registers).
+template <int SCORE>
+__global__ void __launch_bounds__(256) clear_level2_kernel(const Ctl* __restrict__ ctl, Level2 l2,
+                                                           const float* __restrict__ W, int c, int b, int j, int j1,
+                                                           const float* __restrict__ sc) {
+  const bool a = ctl->dirty_pred != 0, r = ctl->dirty_reread != 0;
+  const int gtid = blockIdx.x * blockDim.x + threadIdx.x, stride = gridDim.x * blockDim.x;
+  if (a || r) {
+    uint4* pa = reinterpret_cast<uint4*>(l2.pred);
+    uint4* pr = reinterpret_cast<uint4*>(l2.reread);
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = gtid; i < kHist2Bins / 4; i += stride) {
+      if (a) pa[i] = z;
+      if (r) pr[i] = z;
     }
-    for (int r0 = warp; r0 < c; r0 += 32 * 4) {
-      float v[4][E];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int r = r0 + 32 * u;
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-          const int qq = lane + 32 * e;
-          v[u][e] = (r < c && qq < nJ) ? W[(long long)r * b + j + qq] : 0.f;
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int e = 0; e < E; ++e)
-          if (r0 + 32 * u < c && lane + 32 * e < nJ && key_of<SCORE>(v[u][e], scv[e]) == T) ++cnt[e];
+    for (int i = gtid; i < kHist2SumBins; i += stride) {
+      if (a) l2.pred_sum[i] = 0u;
+      if (r) l2.reread_sum[i] = 0u;
     }
+  }
+  if (ctl->mode == 0 || !ctl->tie_scan) return;
+  const unsigned int T = ctl->T;
+  const int nJ = j1 - j, lane = threadIdx.x & 31;
+  const int gwarp = gtid >> 5, nwarps = stride >> 5;
+  constexpr int E = kMaxBlock / 32;
+  unsigned int cnt[E];
+  float scv[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    cnt[e] = 0u;
+    scv[e] = lane + 32 * e < nJ ? __ldg(sc + j + lane + 32 * e) : 0.f;
+  }
+  for (int row = gwarp; row < c; row += nwarps) {
+    const float* wr = W + (long long)row * b + j;
+    float v[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) v[e] = lane + 32 * e < nJ ? wr[lane + 32 * e] : 0.f;
 #pragma unroll
     for (int e = 0; e < E; ++e)
-      if (cnt[e]) atomicAdd(&colcnt[lane + 32 * e], cnt[e]);
+      if (lane + 32 * e < nJ && key_of<SCORE>(v[e], scv[e]) == T) ++cnt[e];
   }
-  __syncthreads();
+#pragma unroll
+  for (int e = 0; e < E; ++e)
+    if (cnt[e]) atomicAdd(&l2.tie_count[lane + 32 * e], cnt[e]);
+}
+
+// The cut-off among the tied entries: with m of them taken in (column, row) order, the
+// column holding the m-th, then its row (one CTA scans that column); the per-column
+// counts are zeroed for the next block.
+template <int SCORE>
+__global__ void __launch_bounds__(1024) tie_pick_kernel(Ctl* ctl, Level2 l2, const float* __restrict__ W, int c,
+                                                        int b, int j, int j1, const float* __restrict__ sc,
+                                                        pwp_stats* st) {
+  __shared__ long long sh_warp[32];
+  __shared__ int s_qstar;
+  __shared__ long long s_need;
+  if (cta_failed(st) || ctl->mode == 0 || !ctl->tie_scan) return;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nJ = j1 - j;
+  const unsigned int T = ctl->T;
+  const long long m = ctl->m;
   if (tid == 0) {
     long long cum = 0;
     int qstar = -1;
     for (int qq = 0; qq < nJ; ++qq) {
-      if (cum + colcnt[qq] >= m) { qstar = qq; break; }
-      cum += colcnt[qq];
+      const long long cq = l2.tie_count[qq];
+      if (cum + cq >= m) { qstar = qq; break; }
+      cum += cq;
     }
     s_qstar = qstar;
     s_need = m - cum;  // 1-based rank of the last taken tie inside column qstar
   }
   __syncthreads();
+  for (int i = tid; i < kMaxBlock; i += blockDim.x) l2.tie_count[i] = 0u;
   if (s_qstar < 0) return;  // fewer than m ties inside the block: all of them are taken
   const int q = j + s_qstar;
+  const float scq = __ldg(sc + q);
   const int per = (c + 1023) / 1024;
   long long cnt = 0;
   for (int i = 0; i < per; ++i) {
-    int r = tid * per + i;
-    if (r < c && key_of<SCORE>(W[(long long)r * b + q], __ldg(sc + q)) == T) ++cnt;
+    const int r = tid * per + i;
+    if (r < c && key_of<SCORE>(W[(long long)r * b + q], scq) == T) ++cnt;
   }
   // exclusive scan of cnt over the CTA
   long long x = cnt;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    long long yv = __shfl_up_sync(0xffffffffu, x, o);
+    const long long yv = __shfl_up_sync(0xffffffffu, x, o);
     if (lane >= o) x += yv;
   }
   if (lane == 31) sh_warp[warp] = x;
@@ -276,32 +306,14 @@ __global__ void __launch_bounds__(1024) pick2_kernel(Ctl* ctl, Level2 l2, const 
   if (bef < need && need <= bef + cnt) {
     long long k = bef;
     for (int i = 0; i < per; ++i) {
-      int r = tid * per + i;
-      if (r < c && key_of<SCORE>(W[(long long)r * b + q], __ldg(sc + q)) == T) {
+      const int r = tid * per + i;
+      if (r < c && key_of<SCORE>(W[(long long)r * b + q], scq) == T) {
         if (++k == need) {
           ctl->pstar = (long long)s_qstar * c + r;
           break;
         }
       }
     }
-  }
-}
-
-// Zero the level-2 histograms this block wrote, ready for the next block.
-__global__ void clear_level2_kernel(const Ctl* __restrict__ ctl, Level2 l2) {
-  const bool a = ctl->dirty_pred != 0, r = ctl->dirty_reread != 0;
-  if (!a && !r) return;
-  const int stride = gridDim.x * blockDim.x;
-  uint4* pa = reinterpret_cast<uint4*>(l2.pred);
-  uint4* pr = reinterpret_cast<uint4*>(l2.reread);
-  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < kHist2Bins / 4; i += stride) {
-    if (a) pa[i] = z;
-    if (r) pr[i] = z;
-  }
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < kHist2SumBins; i += stride) {
-    if (a) l2.pred_sum[i] = 0u;
-    if (r) l2.reread_sum[i] = 0u;
   }
 }
 
@@ -329,8 +341,20 @@ void launch_pick2(int score, Ctl* ctl, Level2 l2, const float* W, int c, int b, 
     pick2_kernel<kObs><<<1, 1024, 0, s>>>(ctl, l2, W, c, b, j, j1, sc, st);
 }
 
-void launch_clear_level2(const Ctl* ctl, Level2 l2, cudaStream_t s) {
-  clear_level2_kernel<<<kNumSM, 256, 0, s>>>(ctl, l2);
+void launch_clear_level2(int score, const Ctl* ctl, Level2 l2, const float* W, int c, int b, int j, int j1,
+                         const float* sc, cudaStream_t s) {
+  if (score == kWanda)
+    clear_level2_kernel<kWanda><<<kNumSM, 256, 0, s>>>(ctl, l2, W, c, b, j, j1, sc);
+  else
+    clear_level2_kernel<kObs><<<kNumSM, 256, 0, s>>>(ctl, l2, W, c, b, j, j1, sc);
+}
+
+void launch_tie_pick(int score, Ctl* ctl, Level2 l2, const float* W, int c, int b, int j, int j1, const float* sc,
+                     pwp_stats* st, cudaStream_t s) {
+  if (score == kWanda)
+    tie_pick_kernel<kWanda><<<1, 1024, 0, s>>>(ctl, l2, W, c, b, j, j1, sc, st);
+  else
+    tie_pick_kernel<kObs><<<1, 1024, 0, s>>>(ctl, l2, W, c, b, j, j1, sc, st);
 }
 
 }  // namespace pwp

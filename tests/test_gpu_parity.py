@@ -155,3 +155,27 @@ def test_non_spd_is_reported_not_faulted():
     with pytest.raises(pwp.PwpError) as e:
         pwp.prune_layer(W, X=Xt, damp=0.0, block=32)
     assert e.value.status == 2
+
+
+def test_exact_ties_follow_column_row_order():
+    """Weights on a 1/64 grid and +-1 activations give every feature the same norm, so the
+    first block's scores tie in large groups; at 33% the global budget takes 452 of the 949
+    entries of the first block tied at the threshold (checked against the oracle when this
+    case was built).  The pages fix no order among equal scores; both sides take ties in
+    (column, row) order, so the first block's mask must match the oracle's exactly."""
+    _torch()
+    wl = synth.custom(64, 256, 512, dtype="fp32", block=32, sparsity=0.33, seed=7)
+    W = (np.round(synth.make_W(wl).astype(np.float64) * 64.0) / 64.0).astype(np.float32)
+    rng = np.random.default_rng(7)
+    X = rng.choice(np.array([-1.0, 1.0], dtype=np.float32), size=(512, 256))
+    kw = dict(method="thanos", pattern="unstructured", nm=(0, 0), block=32, sparsity=0.33, damp=0.01)
+    gpu = P.run_gpu(W, X, "fp32", **kw)
+    orc = P.run_oracle(W, X, "fp32", **kw)
+    W_hat, mask, st = gpu
+    s0 = np.abs(W[:, :32].astype(np.float64))
+    thr = s0[orc["mask"][:, :32]].max()
+    tied = s0 == thr
+    assert 0 < (tied & orc["mask"][:, :32]).sum() < tied.sum()   # a partial tie group
+    assert st.tie_blocks >= 1
+    assert np.array_equal(mask[:, :32], orc["mask"][:, :32])
+    _check(W, "fp32", gpu, orc, X, "unstructured", (0, 0), 32, orc["pruned"])
