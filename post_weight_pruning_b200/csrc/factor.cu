@@ -62,15 +62,15 @@ __global__ void __launch_bounds__(1024) damp_kernel(float* __restrict__ H, int b
 // pivot column scaled by 1/sqrt(P_kk); row k of X (which already holds every earlier
 // pivot's elimination) is final once scaled the same way, and is then eliminated from
 // the rows below it, as the trailing part of P is.  Each thread keeps a 4x4 cyclic
-// sub-block of P and of X (rows ty + 16a, columns tx + 16c) in registers; a pivot step
-// needs one barrier, with the pivot column of P and pivot row of X broadcast through
+// sub-block of P and of X (rows ty + 16a, columns tx + 16c) in registers; pivots go two
+// per barrier, with the two pivot columns of P and pivot rows of X broadcast through
 // double-buffered shared vectors.  Entries beyond nb are an identity pad.
 // On return A's upper triangle holds V and Wi holds V^-1 (upper, zero below).
 // Returns false on a non-positive pivot (recorded in st).
 __device__ bool factor_diag_block(float (*A)[NB + 1], float (*Wi)[NB + 1], int nb, int* bad,
                                   pwp_stats* st) {
-  __shared__ float colbuf[2][NB];
-  __shared__ float rowbuf[2][NB];
+  __shared__ float colbuf[2][2][NB];
+  __shared__ float rowbuf[2][2][NB];
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   const int off = NB - nb;  // P[r][s] = A[nb-1-(r-off)][...] for r, s >= off; identity before
   float P[4][4], X[4][4];
@@ -90,59 +90,86 @@ __device__ bool factor_diag_block(float (*A)[NB + 1], float (*Wi)[NB + 1], int n
       X[a][c] = (r == s) ? 1.f : 0.f;
     }
   if (tid == 0) *bad = 0;
-  // pivot k = 16 kb + kk keeps the register index kb a constant
+  // two pivots k, k+1 per barrier (k = 16 kb + kk, kk even, so both sit in register block
+  // kb, a compile-time index): columns k and k+1 of P and rows k and k+1 of X are
+  // broadcast as they stand, and every thread rebuilds column k+1 and row k+1 after
+  // pivot k from them
 #pragma unroll
   for (int kb = 0; kb < 4; ++kb)
-  for (int kk = 0; kk < 16; ++kk) {
+  for (int kk = 0; kk < 16; kk += 2) {
     const int k = 16 * kb + kk;
-    float* cb = colbuf[k & 1];
-    float* rb = rowbuf[k & 1];
+    const int par = (k >> 1) & 1;
+    float* cb0 = colbuf[par][0];
+    float* cb1 = colbuf[par][1];
+    float* rb0 = rowbuf[par][0];
+    float* rb1 = rowbuf[par][1];
     if (tx == kk) {
 #pragma unroll
-      for (int a = 0; a < 4; ++a) cb[ty + 16 * a] = P[a][kb];
+      for (int a = 0; a < 4; ++a) cb0[ty + 16 * a] = P[a][kb];
+    }
+    if (tx == kk + 1) {
+#pragma unroll
+      for (int a = 0; a < 4; ++a) cb1[ty + 16 * a] = P[a][kb];
     }
     if (ty == kk) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) rb[tx + 16 * c] = X[kb][c];
+      for (int c = 0; c < 4; ++c) rb0[tx + 16 * c] = X[kb][c];
+    }
+    if (ty == kk + 1) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) rb1[tx + 16 * c] = X[kb][c];
     }
     __syncthreads();
-    const float d = cb[k];
-    if (!(d > 0.f) || !isfinite(d)) {   // the same value for every thread
+    const float d0 = cb0[k];
+    const float il0 = rsqrtf(d0);
+    const float l10 = cb0[k + 1] * il0;                 // L[k+1][k]
+    const float d1 = cb1[k + 1] - l10 * l10;            // pivot k+1 after pivot k
+    if (!(d0 > 0.f) || !isfinite(d0) || !(d1 > 0.f) || !isfinite(d1)) {   // uniform
       if (tid == 0) {
         *bad = 1;
         set_error(st, PWP_ENOTSPD, kSiteCholDiag);
       }
       return false;
     }
-    const float inv_l = rsqrtf(d);
-    float lr[4], cs[4], xk[4];
-#pragma unroll
-    for (int a = 0; a < 4; ++a) lr[a] = cb[ty + 16 * a] * inv_l;    // L[r][k]
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      cs[c] = cb[tx + 16 * c] * inv_l;                              // L[s][k]
-      xk[c] = rb[tx + 16 * c] * inv_l;                              // X[k][s], final
-    }
-    // r = ty + 16a and k = 16kb + kk with a, kb compile-time: r > k is decided at
-    // compile time except in register row a == kb (likewise for columns)
-    const bool ty_gt = ty > kk, ty_eq = ty == kk, tx_gt = tx > kk, tx_eq = tx == kk;
+    const float il1 = rsqrtf(d1);
+    float lr0[4], lr1[4], cs0[4], cs1[4], x0[4], x1[4];
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
-      if (a < kb) continue;                                         // rows above the pivot
-      const bool r_gt = a > kb || ty_gt, r_eq = a == kb && ty_eq;
+      lr0[a] = cb0[ty + 16 * a] * il0;                                // L[r][k]
+      lr1[a] = fmaf(-lr0[a], l10, cb1[ty + 16 * a]) * il1;            // L[r][k+1]
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      cs0[c] = cb0[tx + 16 * c] * il0;                                // L[s][k]
+      cs1[c] = fmaf(-cs0[c], l10, cb1[tx + 16 * c]) * il1;            // L[s][k+1]
+      x0[c] = rb0[tx + 16 * c] * il0;                                 // X[k][s], final
+      x1[c] = fmaf(-l10, x0[c], rb1[tx + 16 * c]) * il1;              // X[k+1][s], final
+    }
+    // r = ty + 16a, s = tx + 16c: relations to k and k+1 are compile-time except in
+    // register block kb
+    const bool ty_gt0 = ty > kk, ty_eq0 = ty == kk, ty_gt1 = ty > kk + 1, ty_eq1 = ty == kk + 1;
+    const bool tx_eq0 = tx == kk, tx_eq1 = tx == kk + 1, tx_gt1 = tx > kk + 1;
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      if (a < kb) continue;                                         // rows above both pivots
+      const bool r_ge0 = a > kb || ty_gt0 || ty_eq0, r_ge1 = a > kb || ty_gt1 || ty_eq1;
+      const bool r_gt1 = a > kb || ty_gt1, r_eq0 = a == kb && ty_eq0, r_eq1 = a == kb && ty_eq1;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         if (c >= kb) {                                              // P: columns >= k
-          const bool s_eq = c == kb && tx_eq, s_gt = c > kb || tx_gt;
-          if (s_eq) {
-            if (r_gt || r_eq) P[a][c] = lr[a];                      // column k of L
-          } else if (r_gt && s_gt) {
-            P[a][c] = fmaf(-lr[a], cs[c], P[a][c]);
+          const bool s_eq0 = c == kb && tx_eq0, s_eq1 = c == kb && tx_eq1, s_gt1 = c > kb || tx_gt1;
+          if (s_eq0) {
+            if (r_ge0) P[a][c] = lr0[a];                            // column k of L
+          } else if (s_eq1) {
+            if (r_ge1) P[a][c] = lr1[a];                            // column k+1 of L
+          } else if (r_gt1 && s_gt1) {
+            P[a][c] = fmaf(-lr1[a], cs1[c], fmaf(-lr0[a], cs0[c], P[a][c]));
           }
         }
-        if (c <= kb) {                                              // X row k is zero right of k
-          if (r_eq) X[a][c] = xk[c];
-          else if (r_gt) X[a][c] = fmaf(-lr[a], xk[c], X[a][c]);
+        if (c <= kb) {                                              // X rows k, k+1 are zero right of k+1
+          if (r_eq0) X[a][c] = x0[c];
+          else if (r_eq1) X[a][c] = x1[c];
+          else if (r_gt1) X[a][c] = fmaf(-lr1[a], x1[c], fmaf(-lr0[a], x0[c], X[a][c]));
         }
       }
     }
