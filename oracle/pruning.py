@@ -22,6 +22,9 @@ Sources (web pages, cited by title and section):
   Sparsity".
 * [README] "Thanos - Method of Pruning LLMs" -- section "Usage" (methods
   thanos / sparsegpt, sparsity types unstructured / 2:4 / 4:8).
+* [BLOG] also for the no-update baselines: "Wanda: Pruning by Weights and
+  Activations" (per-row thresholds, no weight update) and "The Failure of
+  Magnitude Pruning in Large Transformers" (rank by |W_ij|).
 
 Everything is fp64.  Library primitives used as single steps: matrix product,
 ``numpy.linalg.inv``, ``numpy.linalg.cholesky``, ``numpy.linalg.solve``,
@@ -41,6 +44,7 @@ __all__ = [
     "gram", "hessian", "damp_hessian", "inverse_cholesky_upper", "active_inverse",
     "conditioned_diag", "wanda_scores", "obs_scores", "lowest_global", "nm_mask",
     "thanos_row_update", "sparsegpt_block", "prune_layer", "recon_loss", "row_losses",
+    "row_quota_mask", "prune_no_update",
 ]
 
 
@@ -343,3 +347,61 @@ def prune_layer(W, *, Xt=None, H=None, sparsity=0.5, pattern="unstructured", nm=
         "g_diag": g_diag, "blocks": blocks, "dscore": dscore, "nm_gap": nm_gap,
         "zstar": zstar, "pruned": pruned, "shortfall": shortfall,
     }
+
+
+# ----------------------------------------------------------------------------- no-update baselines
+
+def row_quota_mask(S: np.ndarray, count: int) -> np.ndarray:
+    """Per output row, remove the ``count`` lowest scores; among equal scores the lower
+    column goes first.  [BLOG] "Wanda: Pruning by Weights and Activations" (the pruning
+    threshold is set independently for each output row, and the lowest s% of the row's
+    scores are zeroed)."""
+    c, b = S.shape
+    mask = np.zeros((c, b), dtype=bool)
+    if count <= 0:
+        return mask
+    cols = np.arange(b)
+    for k in range(c):
+        order = np.lexsort((cols, S[k]))      # by score, then by column
+        mask[k, order[:count]] = True
+    return mask
+
+
+def prune_no_update(W, *, Xt=None, H=None, sparsity=0.5, pattern="unstructured", nm=(2, 4),
+                    method="wanda"):
+    """Wanda or magnitude pruning of one layer: a score per weight, a per-row mask, and no
+    compensation -- kept weights are returned unchanged, removed ones are exactly 0.
+
+    method "wanda": S_kq = |W_kq| * ||X_q||_2 with ||X_q||^2 = G_qq = (X X^T)_qq, taken
+      from Xt ([n, b]) or from an undamped H = 2 X X^T as H_qq / 2.  [BLOG] "Wanda:
+      Pruning by Weights and Activations".
+    method "magnitude": S_kq = |W_kq|.  [BLOG] "The Failure of Magnitude Pruning in Large
+      Transformers"; [THANOS] "Why magnitude alone misses important weights".  The pages
+      do not say whether its quota is per row or per layer; the per-row quota of Wanda
+      is used.
+    pattern "unstructured": floor(sparsity * b) removed per row; "nm": in every aligned
+      group of m consecutive weights of a row, the m - n lowest removed (nm_mask).
+    Returns a dict with W (fp64), mask, pruned, target and the scores S."""
+    W = np.asarray(W, dtype=np.float64)
+    c, b = W.shape
+    if method == "wanda":
+        if Xt is not None:
+            g = np.einsum("tq,tq->q", np.asarray(Xt, dtype=np.float64), np.asarray(Xt, dtype=np.float64))
+        else:
+            g = 0.5 * np.diag(np.asarray(H, dtype=np.float64))
+        S = wanda_scores(W, g)
+    elif method == "magnitude":
+        S = np.abs(W)
+    else:
+        raise ValueError(method)
+    if pattern == "unstructured":
+        count = int(np.floor(float(sparsity) * b))
+        mask = row_quota_mask(S, count)
+        target = c * count
+    else:
+        n, m = nm
+        mask, _ = nm_mask(S, n, m)
+        target = c * (b // m) * (m - n)
+    What = np.where(mask, 0.0, W)
+    return {"W": What, "mask": mask, "pruned": int(mask.sum()), "target": target, "S": S}
+

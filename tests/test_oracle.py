@@ -382,3 +382,68 @@ def test_sparsegpt_uses_conditioned_diagonal():
     U = oracle.inverse_cholesky_upper(Hd)
     for q in range(8):
         assert U[q, q] ** 2 == pytest.approx(oracle.conditioned_diag(Hd, q), rel=1e-10)
+
+
+# ----------------------------------------------------------------------------- no-update baselines
+
+def test_row_quota_mask_is_the_per_row_order_statistic():
+    """Properties that fix the mask: exactly `count` per row; every removed score <= every
+    kept score of its row; at the boundary value the removed ties sit left of the kept."""
+    rng = np.random.default_rng(11)
+    S = rng.integers(0, 6, size=(40, 37)).astype(np.float64)   # many exact ties
+    for count in (0, 1, 9, 18, 36, 37):
+        M = oracle.row_quota_mask(S, count)
+        assert np.all(M.sum(axis=1) == count)
+        for k in range(S.shape[0]):
+            rem, kep = S[k, M[k]], S[k, ~M[k]]
+            if rem.size and kep.size:
+                assert rem.max() <= kep.min()
+                v = rem.max()
+                if v == kep.min():
+                    assert np.flatnonzero(M[k] & (S[k] == v)).max() < np.flatnonzero(~M[k] & (S[k] == v)).min()
+
+
+def test_no_update_hand_example():
+    g = json.load(open(os.path.join(GOLDEN, "no_update_hand_example.json")))
+    W = np.array(g["W"])
+    Xt = np.array(g["Xt"], dtype=np.float64)
+    for method in ("wanda", "magnitude"):
+        want = np.array(g[method + "_mask"])
+        r = oracle.prune_no_update(W, Xt=Xt, sparsity=g["sparsity"], method=method)
+        assert np.array_equal(r["mask"], want)
+        r = oracle.prune_no_update(W, Xt=Xt, pattern="nm", nm=(2, 4), method=method)
+        assert np.array_equal(r["mask"], want)
+        # H = 2 X X^T gives the same norms
+        r = oracle.prune_no_update(W, H=oracle.hessian(Xt), sparsity=g["sparsity"], method=method)
+        assert np.array_equal(r["mask"], want)
+
+
+def test_no_update_leaves_kept_weights_and_zeroes_removed():
+    rng = np.random.default_rng(12)
+    W = rng.normal(0, 0.02, size=(16, 64))
+    Xt = rng.normal(size=(100, 64))
+    r = oracle.prune_no_update(W, Xt=Xt, sparsity=0.6, method="wanda")
+    assert np.all(r["W"][r["mask"]] == 0.0)
+    assert np.array_equal(r["W"][~r["mask"]], W[~r["mask"]])
+    assert r["pruned"] == r["target"] == 16 * int(np.floor(0.6 * 64))
+
+
+def test_wanda_with_equal_feature_norms_is_magnitude():
+    """With every ||X_q|| equal the Wanda score is |W| times a constant, so the masks of the
+    two methods coincide (the special case in which activations carry no information)."""
+    rng = np.random.default_rng(13)
+    W = rng.normal(0, 0.02, size=(24, 96))
+    Xt = rng.choice([-1.0, 1.0], size=(50, 96))
+    for pattern, nm in (("unstructured", (0, 0)), ("nm", (2, 4)), ("nm", (4, 8))):
+        a = oracle.prune_no_update(W, Xt=Xt, sparsity=0.5, pattern=pattern, nm=nm, method="wanda")
+        b = oracle.prune_no_update(W, Xt=Xt, sparsity=0.5, pattern=pattern, nm=nm, method="magnitude")
+        assert np.array_equal(a["mask"], b["mask"])
+
+
+def test_wanda_scale_of_activations_does_not_change_the_mask():
+    rng = np.random.default_rng(14)
+    W = rng.normal(0, 0.02, size=(8, 40))
+    Xt = rng.normal(size=(30, 40))
+    a = oracle.prune_no_update(W, Xt=Xt, sparsity=0.3, method="wanda")
+    b = oracle.prune_no_update(W, Xt=7.0 * Xt, sparsity=0.3, method="wanda")
+    assert np.array_equal(a["mask"], b["mask"])
