@@ -34,11 +34,13 @@ sys.path.insert(0, ROOT)
 METRIC = "layer prune time (ms) & weights/sec, 4096×4096 @50%; % of TC/HBM roofline"
 UNIT = "weights/s"
 WORKLOAD = "q_proj4096x4096"
-K_HESSIAN, K_FACTOR, K_STREAM, K_SELECT, K_SOLVE = 0, 1, 2, 3, 4
+K_HESSIAN, K_FACTOR, K_STREAM, K_SELECT, K_SOLVE, K_ROWPRUNE, K_COLNORM = 0, 1, 2, 3, 4, 5, 6
 CLASS_NAMES = {K_HESSIAN: "hessian_xxt", K_FACTOR: "factor", K_STREAM: "stream_update_score",
-               K_SELECT: "select", K_SOLVE: "row_solve"}
+               K_SELECT: "select", K_SOLVE: "row_solve", K_ROWPRUNE: "row_prune", K_COLNORM: "col_norm"}
 CLASS_SOURCES = {K_HESSIAN: ["hessian_tc.cu", "hessian_simt.cu"], K_FACTOR: ["factor.cu"],
-                 K_STREAM: ["stream_tc.cu", "prune.cu"], K_SELECT: ["select.cu"], K_SOLVE: ["solve.cu"]}
+                 K_STREAM: ["stream_tc.cu", "prune.cu"], K_SELECT: ["select.cu"], K_SOLVE: ["solve.cu"],
+                 K_ROWPRUNE: ["rowprune.cu"], K_COLNORM: ["rowprune.cu"]}
+SECOND_ORDER = ("thanos", "sparsegpt")
 
 
 def _load_peaks():
@@ -131,10 +133,16 @@ class ClockSampler:
 
 # ------------------------------------------------------------------------------ algorithmic work
 
-def algorithmic_work(cls, wl, per_launch_ms, mask=None):
+def algorithmic_work(cls, wl, per_launch_ms, mask=None, method="thanos"):
     """(total algorithmic units over the recorded launches, unit, bound)."""
     c, b, n, B = wl.c, wl.b, wl.n, wl.block
     nblk = (b + B - 1) // B
+    if cls == K_ROWPRUNE:
+        # read W (bf16), write W-hat (fp32) and the mask, read the column norms (Wanda)
+        per = c * b * (2.0 + 4.0 + 1.0) + (4.0 * b if method == "wanda" else 0.0)
+        return per * len(per_launch_ms), "byte", "hbm"
+    if cls == K_COLNORM:
+        return 2.0 * n * b * len(per_launch_ms), "byte", "hbm"   # read X (bf16) once
     if cls == K_HESSIAN:
         return float(b) * b * n * len(per_launch_ms), "flop", "tensor"
     if cls == K_STREAM:
@@ -179,7 +187,7 @@ def fp32_alu_peak_tflops(sm_mhz):
 
 # ------------------------------------------------------------------------------ CPU oracle
 
-def cpu_oracle_sample(wl, W_store, X_store, rows):
+def cpu_oracle_sample(wl, W_store, X_store, rows, method="thanos"):
     import oracle
     import synth
     try:
@@ -190,15 +198,19 @@ def cpu_oracle_sample(wl, W_store, X_store, rows):
     W64 = synth.to_f64(W_store[:rows], wl.dtype)
     t0 = time.perf_counter()
     X64 = synth.to_f64(X_store, wl.dtype)
-    r = oracle.prune_layer(W64, Xt=X64, sparsity=float(np.float32(wl.sparsity)), block=wl.block,
-                           damp=wl.damp, method="thanos", pattern="unstructured")
+    s32 = float(np.float32(wl.sparsity))
+    if method in SECOND_ORDER:
+        r = oracle.prune_layer(W64, Xt=X64, sparsity=s32, block=wl.block, damp=wl.damp, method=method,
+                               pattern="unstructured")
+        what = f"full H from all {wl.n} tokens, full factor, all {(wl.b + wl.block - 1) // wl.block} blocks"
+    else:
+        r = oracle.prune_no_update(W64, Xt=X64, sparsity=s32, method=method)
+        what = f"norms from all {wl.n} tokens" if method == "wanda" else "no activations"
     dt = time.perf_counter() - t0
-    assert r["pruned"] == r["zstar"]
+    assert r["pruned"] == r.get("zstar", r.get("target"))
     return {"value": rows * wl.b / dt, "unit": UNIT, "cores": int(threads), "kind": "oracle",
-            "sample": (f"fp64 numpy oracle on the {wl.name} workload restricted to its first {rows} "
-                       f"output rows: full H from all {wl.n} tokens, full factor, all "
-                       f"{(wl.b + wl.block - 1) // wl.block} blocks; {dt:.1f} s for "
-                       f"{rows}x{wl.b} weights")}
+            "sample": (f"fp64 numpy oracle ({method}) on the {wl.name} workload restricted to its first "
+                       f"{rows} output rows: {what}; {dt:.1f} s for {rows}x{wl.b} weights")}
 
 
 # ------------------------------------------------------------------------------ reference arm
@@ -213,11 +225,11 @@ def run_reference(args):
     X = synth.make_X_tokens(wl)
     rows = 128
     for _ in range(args.warmup):
-        cpu_oracle_sample(wl, W, X, rows)
+        cpu_oracle_sample(wl, W, X, rows, args.method)
     times = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        cb = cpu_oracle_sample(wl, W, X, rows)
+        cb = cpu_oracle_sample(wl, W, X, rows, args.method)
         times.append(time.perf_counter() - t0)
     tot = sum(times)
     value = rows * wl.b * args.steps / tot
@@ -225,7 +237,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": _config(wl),
+        "data": "synthetic", "config": _config(wl, args.method),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cb["cores"], "kind": "oracle",
                          "sample": cb["sample"]},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -234,10 +246,14 @@ def run_reference(args):
     return 0
 
 
-def _config(wl):
+def _config(wl, method="thanos"):
+    how = {"thanos": f"Thanos 50% unstructured global budget, B={wl.block}, damp={wl.damp}",
+           "sparsegpt": f"SparseGPT 50% unstructured per-block quota, B={wl.block}, damp={wl.damp}",
+           "wanda": "Wanda 50% per-row quota, no weight update",
+           "magnitude": "magnitude 50% per-row quota, no weight update"}[method]
     return {"workload": (f"{wl.name}: W {wl.c}x{wl.b} bf16 ~N(0,0.02^2), X {wl.n}x{wl.b} bf16 tokens "
-                         f"(8x2048), 0.5% outlier features x50, Thanos 50% unstructured global "
-                         f"budget, B={wl.block}, damp={wl.damp}"),
+                         f"(8x2048), 0.5% outlier features x50, {how}"),
+            "method": method,
             "c": wl.c, "b": wl.b, "n_tokens": wl.n, "block": wl.block, "sparsity": wl.sparsity,
             "input_dtype": "bf16", "l2": "flushed between steps (256 MiB write, untimed)",
             "parallelism": "independent layer per rank"}
@@ -271,9 +287,10 @@ def run_mine(args):
     Wt = pwp.from_bf16_bits(W_store, dev)
     Xt = pwp.from_bf16_bits(X_store, dev)
     c, b = wl.c, wl.b
-    cfg_kw = dict(method="thanos", pattern="unstructured", sparsity=wl.sparsity, block=wl.block, damp=wl.damp)
+    method = args.method
+    cfg_kw = dict(method=method, pattern="unstructured", sparsity=wl.sparsity, block=wl.block, damp=wl.damp)
     ws = pwp.make_workspace(pwp.config(**cfg_kw), c, b, dev)
-    H = torch.empty((b, b), dtype=torch.float32, device=dev)
+    H = torch.empty((b, b), dtype=torch.float32, device=dev) if method in SECOND_ORDER else None
     W_out = torch.empty((c, b), dtype=torch.float32, device=dev)
     mask = torch.empty((c, b), dtype=torch.uint8, device=dev)
     stats = pwp.new_stats(dev)
@@ -285,7 +302,12 @@ def run_mine(args):
                         **cfg_kw)
 
     nblk = (b + wl.block - 1) // wl.block
-    launches_per_class = {K_HESSIAN: 1, K_FACTOR: 1, K_STREAM: nblk, K_SELECT: nblk, K_SOLVE: nblk}
+    launches_per_class = {K_HESSIAN: 1, K_FACTOR: 1, K_STREAM: nblk, K_SELECT: nblk, K_SOLVE: nblk,
+                          K_ROWPRUNE: 1, K_COLNORM: 1}
+    if method in SECOND_ORDER:
+        classes = (K_HESSIAN, K_FACTOR, K_STREAM, K_SELECT, K_SOLVE)
+    else:
+        classes = (K_COLNORM, K_ROWPRUNE) if method == "wanda" else (K_ROWPRUNE,)
 
     for i in range(max(args.warmup, 1)):
         flush.fill_(float(i))
@@ -297,7 +319,7 @@ def run_mine(args):
 
     # phase breakdown (untimed pass per kernel class) to pick the dominant kernel
     phase_ms = {}
-    for cls in (K_HESSIAN, K_FACTOR, K_STREAM, K_SELECT, K_SOLVE):
+    for cls in classes:
         L.pwp_profile_enable(cls, launches_per_class[cls])
         flush.fill_(0.0)
         step()
@@ -305,7 +327,7 @@ def run_mine(args):
         n = L.pwp_profile_read(buf, launches_per_class[cls])
         phase_ms[CLASS_NAMES[cls]] = float(sum(buf[:n]))
     L.pwp_profile_enable(-1, 0)
-    dom = max((K_HESSIAN, K_FACTOR, K_STREAM, K_SELECT, K_SOLVE), key=lambda k: phase_ms[CLASS_NAMES[k]])
+    dom = max(classes, key=lambda k: phase_ms[CLASS_NAMES[k]])
 
     # timed region
     cap = launches_per_class[dom] * args.steps
@@ -364,7 +386,7 @@ def run_mine(args):
 
     if rank == 0:
         peaks = _load_peaks()
-        work, unit, bound = algorithmic_work(dom, wl, dom_ms, mask_np)
+        work, unit, bound = algorithmic_work(dom, wl, dom_ms, mask_np, method)
         dur_s = sum(dom_ms) / 1e3
         if unit == "byte":
             achieved = work / dur_s / 1e9
@@ -384,18 +406,20 @@ def run_mine(args):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": _config(wl),
+            "config": _config(wl, method),
             "roofline": roof,
             "phases_ms": phase_ms,
-            "select_stats": {"blocks": nblk, "reread_blocks": int(st.reread_blocks), "tie_blocks": int(st.tie_blocks)},
             "gpu_launches": int(launches),
             "e2e": {"value": e2e_value, "unit": UNIT,
                     "h2d_bytes_per_step": int(W_host.numel() * 2 + X_host.numel() * 2),
                     "d2h_bytes_per_step": int(out_W.numel() * 4 + out_m.numel())},
             "clocks": clocks,
         }
+        if method in SECOND_ORDER:
+            line["select_stats"] = {"blocks": nblk, "reread_blocks": int(st.reread_blocks),
+                                    "tie_blocks": int(st.tie_blocks)}
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_oracle_sample(wl, W_store, X_store, args.cpu_rows)
+            line["cpu_baseline"] = cpu_oracle_sample(wl, W_store, X_store, args.cpu_rows, method)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -411,6 +435,8 @@ def main():
     ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=256)
+    ap.add_argument("--method", default="thanos", choices=["thanos", "sparsegpt", "wanda", "magnitude"],
+                    help="pruning method timed on the q_proj workload (default: thanos, the headline)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -47,18 +47,25 @@ typedef enum {
     PWP_EBUDGET = 6      /* the unstructured target could not be reached */
 } pwp_status;
 
-typedef enum { PWP_THANOS = 0, PWP_SPARSEGPT = 1 } pwp_method;
+typedef enum { PWP_THANOS = 0, PWP_SPARSEGPT = 1, PWP_WANDA = 2, PWP_MAGNITUDE = 3 } pwp_method;
 typedef enum { PWP_UNSTRUCTURED = 0, PWP_NM = 1 } pwp_pattern;
 typedef enum { PWP_BF16 = 0, PWP_FP32 = 1 } pwp_dtype;
 
 /* Method configuration ("Thanos - Method of Pruning LLMs", section "Usage":
  * --prune_method, --sparsity_ratio, --sparsity_type).
  *   method   : PWP_THANOS (joint row solves, dynamic global budget) or
- *              PWP_SPARSEGPT (column-sequential OBS, per-block quota).
+ *              PWP_SPARSEGPT (column-sequential OBS, per-block quota), or one of the
+ *              no-update baselines of the llms.blog page: PWP_WANDA (score
+ *              |W_kq| * ||X_q||, section "Wanda: Pruning by Weights and Activations")
+ *              and PWP_MAGNITUDE (score |W_kq|, section "The Failure of Magnitude
+ *              Pruning in Large Transformers"); both remove floor(sparsity * b) weights
+ *              of every row (ties: lower column first), or the nm_m - nm_n lowest of
+ *              every group, and change no other weight; block and damp are ignored.
  *   pattern  : PWP_UNSTRUCTURED, or PWP_NM with 0 < nm_n < nm_m <= 32 (keep nm_n of
  *              every nm_m consecutive weights of a row; groups start at column 0).
  *   sparsity : fraction of weights removed, 0 <= sparsity < 1 (ignored for PWP_NM).
- *   block    : column block width B, 1 <= B <= 128; for PWP_NM a multiple of nm_m.
+ *   block    : column block width B, 1 <= B <= 128; for PWP_NM a multiple of nm_m
+ *              (Thanos and SparseGPT only).
  *   damp     : lambda = damp * mean(diag H) of the undamped H, damp >= 0. */
 typedef struct {
     int32_t method;
@@ -114,7 +121,10 @@ pwp_status pwp_damp_factor(float* H_dev, int32_t b, float damp, float* g_diag_de
 
 /* Prune one layer given its undamped Hessian.
  *   W_dev     : c x b row-major weights of type wtype (read only).
- *   H_dev     : undamped H = 2 X X^T (b x b fp32); DESTROYED (holds U on return).
+ *   H_dev     : undamped H = 2 X X^T (b x b fp32); DESTROYED (holds U on return) by
+ *               PWP_THANOS and PWP_SPARSEGPT; PWP_WANDA reads only its diagonal
+ *               (||X_q||^2 = H_qq / 2) and leaves it unchanged; PWP_MAGNITUDE does not
+ *               use it (it may be NULL).
  *   W_out_dev : c x b fp32, receives W-hat (pruned entries exactly 0.0f).
  *   mask_dev  : c x b bytes, receives 1 where a weight was removed, else 0.
  *   1 <= c, 1 <= b <= 16384, c*b < 2^31.
@@ -126,7 +136,9 @@ pwp_status pwp_prune_layer(const pwp_config* cfg, const void* W_dev, int32_t wty
                            pwp_stats* stats_dev, void* stream);
 
 /* Same as pwp_prune_layer, but first builds H = 2 X X^T into H_dev (b x b fp32,
- * caller-owned scratch, overwritten) from token-major activations X_dev ([n, b]). */
+ * caller-owned scratch, overwritten) from token-major activations X_dev ([n, b]).
+ * PWP_WANDA takes ||X_q|| straight from X (fp64 sums) and PWP_MAGNITUDE ignores X; for
+ * these two H_dev is not used and may be NULL. */
 pwp_status pwp_prune_layer_x(const pwp_config* cfg, const void* W_dev, int32_t wtype,
                              int32_t c, int32_t b, const void* X_dev, int32_t xtype,
                              int64_t n, float* H_dev, float* W_out_dev, uint8_t* mask_dev,
@@ -164,7 +176,9 @@ typedef enum {
     PWP_K_FACTOR = 1,    /* the whole damping + factorisation phase */
     PWP_K_STREAM = 2,    /* per block: trailing update + rescoring + histogram */
     PWP_K_SELECT = 3,    /* per block: exact threshold selection */
-    PWP_K_SOLVE = 4      /* per block: per-row solves and in-block update */
+    PWP_K_SOLVE = 4,     /* per block: per-row solves and in-block update */
+    PWP_K_ROWPRUNE = 5,  /* Wanda / magnitude: the per-row (or per-group) selection */
+    PWP_K_COLNORM = 6    /* Wanda from X: the column norms of X */
 } pwp_kernel_class;
 int64_t pwp_kernel_launches(void);
 int32_t pwp_profile_enable(int32_t which, int32_t capacity);

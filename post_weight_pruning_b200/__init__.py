@@ -18,14 +18,15 @@ from dataclasses import dataclass
 import numpy as np
 
 __all__ = [
-    "lib", "Config", "Stats", "THANOS", "SPARSEGPT", "UNSTRUCTURED", "NM", "BF16", "FP32",
+    "lib", "Config", "Stats", "THANOS", "SPARSEGPT", "WANDA", "MAGNITUDE", "UNSTRUCTURED", "NM", "BF16", "FP32",
     "PwpError", "config", "workspace_bytes", "hessian_accumulate", "damp_factor", "prune_layer",
     "prune_layer_host", "status_string", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpwp.so")
 
-THANOS, SPARSEGPT = 0, 1
+THANOS, SPARSEGPT, WANDA, MAGNITUDE = 0, 1, 2, 3
+METHODS = {"thanos": THANOS, "sparsegpt": SPARSEGPT, "wanda": WANDA, "magnitude": MAGNITUDE}
 UNSTRUCTURED, NM = 0, 1
 BF16, FP32 = 0, 1
 
@@ -90,7 +91,7 @@ def _check(status, where):
 
 
 def config(method="thanos", pattern="unstructured", nm=(2, 4), sparsity=0.5, block=128, damp=0.01) -> Config:
-    m = {"thanos": THANOS, "sparsegpt": SPARSEGPT}[method] if isinstance(method, str) else int(method)
+    m = METHODS[method] if isinstance(method, str) else int(method)
     if isinstance(pattern, str):
         p = {"unstructured": UNSTRUCTURED, "nm": NM}[pattern]
     else:
@@ -191,9 +192,11 @@ def prune_layer(W, *, H=None, X=None, sparsity=0.5, pattern="unstructured", nm=(
     """Prune one layer on the GPU.
 
     W: [c, b] bf16/fp32 CUDA tensor.  Give either H (undamped 2XX^T, fp32 [b, b],
-    DESTROYED: holds U afterwards) or X (token-major [n, b] activations; an H
-    scratch is allocated unless H is also passed).  Returns (W_hat fp32, mask uint8,
-    Stats) -- with check=False the stats tensor is returned unread and nothing syncs."""
+    DESTROYED by thanos/sparsegpt: holds U afterwards; wanda reads its diagonal) or X
+    (token-major [n, b] activations; for thanos/sparsegpt an H scratch is allocated
+    unless H is also passed).  method "magnitude" needs neither.  Returns (W_hat fp32,
+    mask uint8, Stats) -- with check=False the stats tensor is returned unread and
+    nothing syncs."""
     torch = _torch()
     _need_cuda(W, H, X)
     c, b = W.shape
@@ -207,19 +210,22 @@ def prune_layer(W, *, H=None, X=None, sparsity=0.5, pattern="unstructured", nm=(
     if stats is None:
         stats = new_stats(W.device)
     L = lib()
+    no_update = cfg.method in (WANDA, MAGNITUDE)
     if X is not None:
-        if H is None:
+        if H is None and not no_update:
             H = torch.empty((b, b), dtype=torch.float32, device=W.device)
         st = L.pwp_prune_layer_x(ctypes.byref(cfg), _vp(W.data_ptr()), _dtype_code(W), int(c), int(b),
-                                 _vp(X.data_ptr()), _dtype_code(X), int(X.shape[0]), _vp(H.data_ptr()),
+                                 _vp(X.data_ptr()), _dtype_code(X), int(X.shape[0]),
+                                 _vp(H.data_ptr() if H is not None else 0),
                                  _vp(W_out.data_ptr()), _vp(mask.data_ptr()), _vp(workspace.ws.data_ptr()),
                                  workspace.nbytes, _vp(stats.data_ptr()), _stream_ptr(stream))
         where = "pwp_prune_layer_x"
     else:
-        if H is None:
+        if H is None and cfg.method != MAGNITUDE:
             raise ValueError("give H or X")
         st = L.pwp_prune_layer(ctypes.byref(cfg), _vp(W.data_ptr()), _dtype_code(W), int(c), int(b),
-                               _vp(H.data_ptr()), _vp(W_out.data_ptr()), _vp(mask.data_ptr()),
+                               _vp(H.data_ptr() if H is not None else 0), _vp(W_out.data_ptr()),
+                               _vp(mask.data_ptr()),
                                _vp(workspace.ws.data_ptr()), workspace.nbytes, _vp(stats.data_ptr()),
                                _stream_ptr(stream))
         where = "pwp_prune_layer"

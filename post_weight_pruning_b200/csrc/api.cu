@@ -25,16 +25,17 @@ static bool valid_cfg(const pwp_config* cfg, int32_t c, int32_t b) {
   if (!cfg) return false;
   if (c < 1 || b < 1 || b > 16384) return false;
   if ((long long)c * (long long)b >= (1LL << 31)) return false;
-  if (cfg->method != PWP_THANOS && cfg->method != PWP_SPARSEGPT) return false;
-  if (cfg->block < 1 || cfg->block > kMaxBlock) return false;
-  if (!(cfg->damp >= 0.f) || !(cfg->damp < 1e30f)) return false;
+  if (cfg->method < PWP_THANOS || cfg->method > PWP_MAGNITUDE) return false;
+  const bool second_order = cfg->method == PWP_THANOS || cfg->method == PWP_SPARSEGPT;
+  if (second_order && (cfg->block < 1 || cfg->block > kMaxBlock)) return false;
+  if (second_order && !(cfg->damp >= 0.f && cfg->damp < 1e30f)) return false;
   if (cfg->pattern == PWP_UNSTRUCTURED) {
     if (!(cfg->sparsity >= 0.f && cfg->sparsity < 1.f)) return false;
   } else if (cfg->pattern == PWP_NM) {
     const int n = cfg->nm_n, m = cfg->nm_m;
     if (m < 2 || m > 32 || (m & (m - 1)) != 0) return false;  // m must divide a warp
     if (n < 1 || n >= m) return false;
-    if (b % m != 0 || cfg->block % m != 0) return false;
+    if (b % m != 0 || (second_order && cfg->block % m != 0)) return false;
   } else {
     return false;
   }
@@ -107,8 +108,8 @@ pwp_status pwp_damp_factor(float* H, int32_t b, float damp, float* g_diag, void*
 pwp_status pwp_prune_layer(const pwp_config* cfg, const void* W, int32_t wtype, int32_t c, int32_t b,
                            float* H, float* W_out, uint8_t* mask, void* ws, size_t ws_bytes,
                            pwp_stats* st, void* stream) {
-  if (!valid_cfg(cfg, c, b) || !valid_dtype(wtype) || !W || !H || !W_out || !mask || !st)
-    return PWP_EINVAL;
+  if (!valid_cfg(cfg, c, b) || !valid_dtype(wtype) || !W || !W_out || !mask || !st) return PWP_EINVAL;
+  if (!H && cfg->method != PWP_MAGNITUDE) return PWP_EINVAL;
   if (!ws || !aligned(ws, 256) || ws_bytes < prune_ws_layout(cfg, c, b, nullptr, nullptr))
     return PWP_EWORKSPACE;
   cudaError_t e = launch_prune(cfg, W, wtype, c, b, H, W_out, mask, ws, st, (cudaStream_t)stream, false);
@@ -118,12 +119,17 @@ pwp_status pwp_prune_layer(const pwp_config* cfg, const void* W, int32_t wtype, 
 pwp_status pwp_prune_layer_x(const pwp_config* cfg, const void* W, int32_t wtype, int32_t c, int32_t b,
                              const void* X, int32_t xtype, int64_t n, float* H, float* W_out,
                              uint8_t* mask, void* ws, size_t ws_bytes, pwp_stats* st, void* stream) {
-  if (!valid_cfg(cfg, c, b) || !valid_dtype(wtype) || !valid_dtype(xtype) || !W || !H || !W_out ||
-      !mask || !st || n < 0 || (n > 0 && !X))
+  const bool no_update = valid_cfg(cfg, c, b) && (cfg->method == PWP_WANDA || cfg->method == PWP_MAGNITUDE);
+  if (!valid_cfg(cfg, c, b) || !valid_dtype(wtype) || !valid_dtype(xtype) || !W || (!H && !no_update) ||
+      !W_out || !mask || !st || n < 0 || (n > 0 && !X))
     return PWP_EINVAL;
   if (!ws || !aligned(ws, 256) || ws_bytes < prune_ws_layout(cfg, c, b, nullptr, nullptr))
     return PWP_EWORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;
+  if (no_update) {
+    cudaError_t e = launch_no_update(cfg, W, wtype, c, b, nullptr, X, xtype, n, W_out, mask, ws, st, false, s);
+    return e == cudaSuccess ? PWP_OK : PWP_ECUDA;
+  }
   if (launch_stats_init(st, s) != cudaSuccess) return PWP_ECUDA;
   pwp_status ps = hessian_impl(X, xtype, n, b, H, 0, st, s);
   if (ps != PWP_OK) return ps;

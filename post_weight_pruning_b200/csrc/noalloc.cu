@@ -56,7 +56,8 @@ extern "C" pwp_status pwp_prune_layer_noalloc(const pwp_config* cfg, const void*
                                               uint8_t* mask, pwp_stats* st, void* stream) {
   // same argument contract as pwp_prune_layer
   size_t need = pwp_workspace_bytes(cfg, c, b);
-  if (need == 0 || (wtype != PWP_BF16 && wtype != PWP_FP32) || !W || !H || !W_out || !mask || !st)
+  if (need == 0 || (wtype != PWP_BF16 && wtype != PWP_FP32) || !W || (!H && cfg->method != PWP_MAGNITUDE) ||
+      !W_out || !mask || !st)
     return PWP_EINVAL;
   if (need > (size_t)PWP_NOALLOC_SCRATCH_BYTES) return PWP_EWORKSPACE;
   void* ws = nullptr;

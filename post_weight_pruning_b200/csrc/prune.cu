@@ -295,6 +295,7 @@ struct PruneBuffers {
 static size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
 
 size_t prune_ws_layout(const pwp_config* cfg, int c, int b, PruneBuffers* pb, char* base) {
+  if (cfg->method == PWP_WANDA || cfg->method == PWP_MAGNITUDE) return no_update_ws_bytes(b);
   const int B = cfg->block;
   const int nblk = (b + B - 1) / B;
   const bool thanos = cfg->method == PWP_THANOS;
@@ -375,6 +376,9 @@ cudaError_t launch_stats_init(pwp_stats* st, cudaStream_t s) {
 cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c, int b, float* H,
                          float* Wout, uint8_t* mask, void* ws, pwp_stats* st, cudaStream_t s,
                          bool stats_ready) {
+  if (cfg->method == PWP_WANDA || cfg->method == PWP_MAGNITUDE)
+    return launch_no_update(cfg, W, wtype, c, b, cfg->method == PWP_WANDA ? H : nullptr, nullptr, 0, 0, Wout,
+                            mask, ws, st, stats_ready, s);
   PruneBuffers pb;
   const int B = cfg->block;
   prune_ws_layout(cfg, c, b, &pb, (char*)ws);

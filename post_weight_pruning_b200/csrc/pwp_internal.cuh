@@ -150,7 +150,8 @@ __device__ __forceinline__ bool selected(unsigned int key, bool valid, int qq, i
 }
 
 // ---------------------------------------------------------------- instrumentation (host side)
-enum KernelClass { kKHessian = 0, kKFactor = 1, kKStream = 2, kKSelect = 3, kKSolve = 4 };
+enum KernelClass { kKHessian = 0, kKFactor = 1, kKStream = 2, kKSelect = 3, kKSolve = 4, kKRowPrune = 5,
+                   kKColNorm = 6 };
 void prof_begin(int which, cudaStream_t s);
 void prof_end(int which, cudaStream_t s);
 void count_launches(long long n);
@@ -197,6 +198,13 @@ bool launch_stream_tc(int score, float* W, int c, int b, int ldw, int u0, int j,
                       int Bp, int ldz, const float* Rhi, const float* Rlo, const uint8_t* mask, const float* sc,
                       int hist_end, unsigned int* hist1, const Ctl* ctl, Level2 l2, pwp_stats* st,
                       cudaStream_t s, cudaError_t* err, bool upper = false);
+
+// Wanda / magnitude: per-row quota or N:M groups, no weight update (rowprune.cu).  H
+// (its diagonal) or X ([n, b]) gives ||X_q|| for Wanda.
+size_t no_update_ws_bytes(int b);
+cudaError_t launch_no_update(const pwp_config* cfg, const void* W, int wtype, int c, int b, const float* H,
+                             const void* X, int xtype, long long n, float* Wout, uint8_t* mask, void* ws,
+                             pwp_stats* st, bool stats_ready, cudaStream_t s);
 
 // per-row work of one block (solve.cu); returns the number of kernels launched
 int launch_thanos_solve(bool nm, const float* W, int c, int b, int j, int B, const float* Kt,

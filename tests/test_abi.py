@@ -81,3 +81,26 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(pwp, "_lib", None)
     with pytest.raises(ImportError):
         pwp.lib()
+
+
+def test_no_update_methods_validation():
+    """Wanda and magnitude ignore block and damp, still check the pattern, and take H only
+    where they need it (magnitude never; Wanda through pwp_prune_layer)."""
+    L = pwp.lib()
+    vp = ctypes.c_void_p
+    fake = vp(1 << 20)
+    for method in ("wanda", "magnitude"):
+        cfg = pwp.config(method=method, block=1000, damp=-1.0)          # ignored fields
+        n = pwp.workspace_bytes(cfg, 16, 64)
+        assert n > 0 and n % 256 == 0
+        assert pwp.workspace_bytes(pwp.config(method=method, pattern="nm", nm=(2, 4)), 16, 66) == 0
+        assert pwp.workspace_bytes(pwp.config(method=method, sparsity=1.0), 16, 64) == 0
+        # too-small workspace still wins over everything after the argument checks
+        assert L.pwp_prune_layer(ctypes.byref(cfg), fake, 0, 16, 64, fake, fake, fake, fake, 10, fake, None) == 3
+    # Wanda through pwp_prune_layer needs H; magnitude does not (it fails on the workspace)
+    cfg = pwp.config(method="wanda")
+    assert L.pwp_prune_layer(ctypes.byref(cfg), fake, 0, 16, 64, None, fake, fake, fake, 10, fake, None) == 1
+    cfg = pwp.config(method="magnitude")
+    assert L.pwp_prune_layer(ctypes.byref(cfg), fake, 0, 16, 64, None, fake, fake, fake, 10, fake, None) == 3
+    bad = pwp.config(method=4)
+    assert pwp.workspace_bytes(bad, 16, 64) == 0
