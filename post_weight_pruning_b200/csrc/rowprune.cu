@@ -265,7 +265,13 @@ cudaError_t launch_no_update(const pwp_config* cfg, const void* W, int wtype, in
     static std::atomic<unsigned long long> attr_done{0};
     if (first_on_device(attr_done))
       cudaFuncSetAttribute(row_quota_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * 16384 * 4);
-    const int grid = c < 2 * nsm ? c : 2 * nsm;
+    // as many resident CTAs as shared memory allows: the radix passes are latency-bound
+    int per_sm = 2;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, row_quota_kernel, kRowThreads, smem) != cudaSuccess ||
+        per_sm < 1)
+      per_sm = 1;
+    const long long cap = (long long)per_sm * nsm;
+    const int grid = (int)(c < cap ? c : cap);
     row_quota_kernel<<<grid, kRowThreads, smem, s>>>(W, wtype, c, b, wanda ? xnorm : nullptr, quota, Wout, mask,
                                                      st);
   }
