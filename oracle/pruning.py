@@ -44,7 +44,7 @@ __all__ = [
     "gram", "hessian", "damp_hessian", "inverse_cholesky_upper", "active_inverse",
     "conditioned_diag", "wanda_scores", "obs_scores", "lowest_global", "nm_mask",
     "thanos_row_update", "sparsegpt_block", "prune_layer", "recon_loss", "row_losses",
-    "row_quota_mask", "prune_no_update",
+    "row_quota_mask", "prune_no_update", "bf16_bits_rne", "pack_24",
 ]
 
 
@@ -404,4 +404,41 @@ def prune_no_update(W, *, Xt=None, H=None, sparsity=0.5, pattern="unstructured",
         target = c * (b // m) * (m - n)
     What = np.where(mask, 0.0, W)
     return {"W": What, "mask": mask, "pruned": int(mask.sum()), "target": target, "S": S}
+
+
+# ----------------------------------------------------------------------------- 2:4 storage
+
+def bf16_bits_rne(x: np.ndarray) -> np.ndarray:
+    """bfloat16 bit patterns of fp32 values, rounded to nearest with ties to even (the
+    upper 16 bits of the fp32 pattern after adding 0x7fff plus the kept half's lowest
+    bit).  Finite inputs only."""
+    u = np.asarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    return ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+def pack_24(What: np.ndarray, mask: np.ndarray):
+    """Compressed 2:4 storage of a pruned layer: in every aligned group of four weights of
+    a row exactly two are kept; store those two values at 16-bit precision (bfloat16, in
+    column order) and their 2-bit positions in the group.  [BLOG] "N:M Semi-Structured
+    Sparsity (2:4 Pattern)": only the 2 non-zero values and 2-bit index metadata are
+    stored.  The pages do not give the metadata layout the tensor cores read; here each
+    group's positions form one 4-bit field idx0 | idx1 << 2 (idx0 < idx1), eight groups per
+    32-bit word, the first group in the lowest bits, words row-major (ceil(b/32) per row).
+    Returns (values: uint16 c x b/2, meta: uint32 c x ceil(b/32))."""
+    What = np.asarray(What, dtype=np.float32)
+    mask = np.asarray(mask, dtype=bool)
+    c, b = What.shape
+    assert b % 4 == 0
+    groups = b // 4
+    values = np.zeros((c, 2 * groups), dtype=np.uint16)
+    meta = np.zeros((c, (groups + 7) // 8), dtype=np.uint32)
+    bits = bf16_bits_rne(What)
+    for k in range(c):
+        for g in range(groups):
+            kept = [e for e in range(4) if not mask[k, 4 * g + e]]
+            assert len(kept) == 2, (k, g)
+            values[k, 2 * g] = bits[k, 4 * g + kept[0]]
+            values[k, 2 * g + 1] = bits[k, 4 * g + kept[1]]
+            meta[k, g // 8] |= np.uint32((kept[0] | (kept[1] << 2)) << (4 * (g % 8)))
+    return values, meta
 

@@ -447,3 +447,37 @@ def test_wanda_scale_of_activations_does_not_change_the_mask():
     a = oracle.prune_no_update(W, Xt=Xt, sparsity=0.3, method="wanda")
     b = oracle.prune_no_update(W, Xt=7.0 * Xt, sparsity=0.3, method="wanda")
     assert np.array_equal(a["mask"], b["mask"])
+
+
+# ----------------------------------------------------------------------------- 2:4 storage
+
+def test_pack24_hand_example():
+    g = json.load(open(os.path.join(GOLDEN, "pack24_hand_example.json")))
+    v, m = oracle.pack_24(np.array(g["What"], dtype=np.float32), np.array(g["mask"]))
+    assert v.tolist() == g["values"] and m.tolist() == g["meta"]
+
+
+def test_bf16_rne_known_patterns():
+    x = np.array([1.0, -2.0, 0.5, 3.0, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -9, 65504.0, 0.0], dtype=np.float32)
+    # 1 + 2^-8 is halfway between 1 and 1 + 2^-7: ties to even -> 1.0; 1 + 3*2^-9 rounds up
+    assert oracle.bf16_bits_rne(x).tolist() == [0x3F80, 0xC000, 0x3F00, 0x4040, 0x3F80, 0x3F81, 0x4780, 0x0000]
+
+
+def test_pack24_roundtrip_restores_the_rounded_layer():
+    """Unpacking by the stated layout gives back W-hat rounded to bfloat16 with the
+    removed weights zero, for a 2:4 mask from the oracle itself."""
+    rng = np.random.default_rng(15)
+    W = rng.normal(0, 0.02, size=(12, 72))
+    r = oracle.prune_no_update(W, pattern="nm", nm=(2, 4), method="magnitude")
+    What = r["W"].astype(np.float32)
+    v, m = oracle.pack_24(What, r["mask"])
+    c, b = What.shape
+    back = np.zeros((c, b), dtype=np.float32)
+    for k in range(c):
+        for g in range(b // 4):
+            field = (int(m[k, g // 8]) >> (4 * (g % 8))) & 0xF
+            for slot, pos in enumerate((field & 3, field >> 2)):
+                back[k, 4 * g + pos] = (np.uint32(v[k, 2 * g + slot]) << np.uint32(16)).view(np.float32)
+    want = (oracle.bf16_bits_rne(What).astype(np.uint32) << 16).view(np.float32)
+    want[r["mask"]] = 0.0
+    assert np.array_equal(back, want)
