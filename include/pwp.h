@@ -144,6 +144,25 @@ pwp_status pwp_prune_layer_x(const pwp_config* cfg, const void* W_dev, int32_t w
                              int64_t n, float* H_dev, float* W_out_dev, uint8_t* mask_dev,
                              void* ws, size_t ws_bytes, pwp_stats* stats_dev, void* stream);
 
+/* Compressed 2:4 storage of a pruned layer ("Weight Pruning in Large Language Models
+ * ...", llms.blog, section "N:M Semi-Structured Sparsity (2:4 Pattern)": only the two
+ * kept values of every aligned group of four, at 16-bit precision, and 2-bit index
+ * metadata are stored).  The pages do not give the metadata layout sparse tensor cores
+ * read; this one is plain and row-major:
+ *   W_hat_dev : c x b fp32 (e.g. pwp_prune_layer's W_out), 16-byte aligned;
+ *   mask_dev  : c x b bytes, 1 = removed, 4-byte aligned; every aligned group of four
+ *               must keep exactly two entries (mask 0);
+ *   values_dev: c x b/2 uint16, the kept values as bfloat16 bit patterns (round to
+ *               nearest even), in column order within each group;
+ *   meta_dev  : c x ceil(b/32) uint32; group g of a row is the 4-bit field
+ *               idx0 | idx1 << 2 (positions 0..3 of its kept entries, idx0 < idx1) at
+ *               bits 4(g%8).. of word g/8 of the row;
+ *   1 <= c, 4 <= b <= 16384, b % 4 == 0, c*b < 2^31.
+ * stats_dev is cleared first; a group that does not keep exactly two entries sets status
+ * PWP_EINVAL (its field then reads positions 0 and 1). */
+pwp_status pwp_pack_24(const float* W_hat_dev, const uint8_t* mask_dev, int32_t c, int32_t b,
+                       uint16_t* values_dev, uint32_t* meta_dev, pwp_stats* stats_dev, void* stream);
+
 /* Prune without a caller-provided workspace (the pages have no counterpart: this is a
  * convenience of this library).  For callers that cannot allocate device memory when
  * they call -- an operator in a runtime that hands it only its input and output

@@ -61,6 +61,7 @@ _SIGS = {
                                _vp, _vp]),
     "pwp_prune_layer_x": (_i32, [ctypes.POINTER(Config), _vp, _i32, _i32, _i32, _vp, _i32, _i64, _vp,
                                  _vp, _vp, _vp, _sz, _vp, _vp]),
+    "pwp_pack_24": (_i32, [_vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp]),
     "pwp_status_string": (ctypes.c_char_p, [_i32]),
     "pwp_version": (_i32, []),
 }
@@ -236,6 +237,28 @@ def prune_layer(W, *, H=None, X=None, sparsity=0.5, pattern="unstructured", nm=(
     if s.status != 0:
         raise PwpError(s.status, where + " (device)")
     return W_out, mask, s
+
+
+def pack_24(W_hat, mask, *, stream=None, check=True):
+    """Compressed 2:4 storage of a pruned layer (pwp_pack_24).  W_hat: fp32 [c, b] and
+    mask: uint8 [c, b] CUDA tensors with exactly two kept entries in every aligned group
+    of four.  Returns (values: int16 [c, b/2] holding bfloat16 bit patterns, meta: int32
+    [c, ceil(b/32)] holding the 4-bit position fields, Stats or the unread stats tensor)."""
+    torch = _torch()
+    _need_cuda(W_hat, mask)
+    c, b = W_hat.shape
+    values = torch.empty((c, b // 2), dtype=torch.int16, device=W_hat.device)
+    meta = torch.empty((c, (b // 4 + 7) // 8), dtype=torch.int32, device=W_hat.device)
+    stats = new_stats(W_hat.device)
+    st = lib().pwp_pack_24(_vp(W_hat.data_ptr()), _vp(mask.data_ptr()), int(c), int(b), _vp(values.data_ptr()),
+                           _vp(meta.data_ptr()), _vp(stats.data_ptr()), _stream_ptr(stream))
+    _check(st, "pwp_pack_24")
+    if not check:
+        return values, meta, stats
+    s = read_stats(stats)
+    if s.status != 0:
+        raise PwpError(s.status, "pwp_pack_24 (device)")
+    return values, meta, s
 
 
 def prune_layer_host(W_host, X_host, *, out_W=None, out_mask=None, device="cuda", **kw):

@@ -137,4 +137,15 @@ pwp_status pwp_prune_layer_x(const pwp_config* cfg, const void* W, int32_t wtype
   return e == cudaSuccess ? PWP_OK : PWP_ECUDA;
 }
 
+pwp_status pwp_pack_24(const float* W_hat, const uint8_t* mask, int32_t c, int32_t b, uint16_t* values,
+                       uint32_t* meta, pwp_stats* st, void* stream) {
+  if (!W_hat || !mask || !values || !meta || !st || c < 1 || b < 4 || b > 16384 || (b % 4) != 0 ||
+      (long long)c * (long long)b >= (1LL << 31) || !aligned(W_hat, 16) || !aligned(mask, 4))
+    return PWP_EINVAL;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemsetAsync(st, 0, sizeof(pwp_stats), s) != cudaSuccess) return PWP_ECUDA;
+  cudaError_t e = launch_pack24(W_hat, mask, c, b, values, meta, st, s);
+  return e == cudaSuccess ? PWP_OK : PWP_ECUDA;
+}
+
 }  // extern "C"

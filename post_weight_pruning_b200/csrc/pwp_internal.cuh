@@ -57,7 +57,7 @@ struct Ctl {
 // Where device-side failures are recorded (pwp_stats::status_site).
 enum Site : int {
   kSiteDamp = 1, kSiteCholDiag = 2, kSiteSolve = 3, kSitePick = 4, kSiteFinal = 5, kSiteHessian = 6,
-  kSiteStream = 7,
+  kSiteStream = 7, kSitePack = 8,
 };
 
 __device__ __forceinline__ bool failed(const pwp_stats* st) {
@@ -205,6 +205,10 @@ size_t no_update_ws_bytes(int b);
 cudaError_t launch_no_update(const pwp_config* cfg, const void* W, int wtype, int c, int b, const float* H,
                              const void* X, int xtype, long long n, float* Wout, uint8_t* mask, void* ws,
                              pwp_stats* st, bool stats_ready, cudaStream_t s);
+
+// compressed 2:4 storage (pack24.cu)
+cudaError_t launch_pack24(const float* What, const uint8_t* mask, int c, int b, uint16_t* values, uint32_t* meta,
+                          pwp_stats* st, cudaStream_t s);
 
 // per-row work of one block (solve.cu); returns the number of kernels launched
 int launch_thanos_solve(bool nm, const float* W, int c, int b, int j, int B, const float* Kt,

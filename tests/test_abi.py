@@ -104,3 +104,14 @@ def test_no_update_methods_validation():
     assert L.pwp_prune_layer(ctypes.byref(cfg), fake, 0, 16, 64, None, fake, fake, fake, 10, fake, None) == 3
     bad = pwp.config(method=4)
     assert pwp.workspace_bytes(bad, 16, 64) == 0
+
+
+def test_pack24_argument_errors():
+    L = pwp.lib()
+    vp = ctypes.c_void_p
+    fake = vp(1 << 20)
+    assert L.pwp_pack_24(None, fake, 4, 8, fake, fake, fake, None) == 1
+    assert L.pwp_pack_24(fake, fake, 4, 6, fake, fake, fake, None) == 1            # b % 4 != 0
+    assert L.pwp_pack_24(fake, fake, 0, 8, fake, fake, fake, None) == 1            # c < 1
+    assert L.pwp_pack_24(vp((1 << 20) + 4), fake, 4, 8, fake, fake, fake, None) == 1   # W-hat not 16-byte aligned
+    assert L.pwp_pack_24(fake, vp((1 << 20) + 2), 4, 8, fake, fake, fake, None) == 1   # mask not 4-byte aligned
