@@ -1,0 +1,46 @@
+"""Host arithmetic of bench.py's roofline object: the algorithmic work of each kernel class
+for a small workload, against values worked out by hand from the stated definitions."""
+import numpy as np
+
+import bench
+import synth
+
+
+def _wl():
+    return synth.custom(8, 20, 12, dtype="fp32", block=8, sparsity=0.5)   # c=8, b=20, n=12, B=8
+
+
+def test_stream_bytes():
+    # blocks j = 0, 8, 16: 8c(b-j) = 64*20, 64*12, 64*4; K rows 4*B*(b-j) for t > 0: 32*12, 32*4
+    want = 64 * (20 + 12 + 4) + 32 * (12 + 4)
+    work, unit, bound = bench.algorithmic_work(bench.K_STREAM, _wl(), [1.0, 1.0, 1.0])
+    assert (work, unit, bound) == (want, "byte", "hbm")
+
+
+def test_select_and_hessian_and_factor():
+    wl = _wl()
+    assert bench.algorithmic_work(bench.K_SELECT, wl, [1.0] * 3) == (4 * 8 * (20 + 12 + 4), "byte", "hbm")
+    assert bench.algorithmic_work(bench.K_HESSIAN, wl, [1.0]) == (20 * 20 * 12, "flop", "tensor")
+    assert bench.algorithmic_work(bench.K_FACTOR, wl, [1.0]) == (2 * 20 ** 3 / 3, "flop", "alu")
+
+
+def test_solve_flops_from_the_mask():
+    """s = the selected count of a row in a block; per row and block s^3/3 + 2 s^2 + 4 s B."""
+    wl = synth.custom(8, 24, 12, dtype="fp32", block=8, sparsity=0.5)    # three whole blocks
+    mask = np.zeros((8, 24), dtype=np.uint8)
+    mask[0, 0:3] = 1          # row 0, block 0: s = 3
+    mask[1, 8:10] = 1         # row 1, block 1: s = 2
+    want = (27 / 3 + 2 * 9 + 4 * 3 * 8) + (8 / 3 + 2 * 4 + 4 * 2 * 8)
+    work, unit, bound = bench.algorithmic_work(bench.K_SOLVE, wl, [1.0] * 3, mask)
+    assert np.isclose(work, want) and unit == "flop" and bound == "alu"
+
+
+def test_no_update_bytes():
+    wl = _wl()
+    assert bench.algorithmic_work(bench.K_ROWPRUNE, wl, [1.0], method="wanda") == (8 * 20 * 7 + 4 * 20, "byte", "hbm")
+    assert bench.algorithmic_work(bench.K_ROWPRUNE, wl, [1.0, 1.0], method="magnitude") == (2 * 8 * 20 * 7, "byte", "hbm")
+    assert bench.algorithmic_work(bench.K_COLNORM, wl, [1.0]) == (2 * 12 * 20, "byte", "hbm")
+
+
+def test_alu_peak_formula():
+    assert np.isclose(bench.fp32_alu_peak_tflops(1965.0), 148 * 128 * 2 * 1965e6 / 1e12)
