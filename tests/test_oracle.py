@@ -481,3 +481,21 @@ def test_pack24_roundtrip_restores_the_rounded_layer():
     want = (oracle.bf16_bits_rne(What).astype(np.uint32) << 16).view(np.float32)
     want[r["mask"]] = 0.0
     assert np.array_equal(back, want)
+
+
+def test_block0_expectation_matches_the_full_oracle():
+    """The full-size check's first-block expectation (scores of the untouched W, the global
+    candidate set or the N:M groups) equals block 0 of a complete oracle prune."""
+    from tests import _fullsize
+    import synth
+    for pattern, nm in (("unstructured", (0, 0)), ("nm", (2, 4)), ("nm", (4, 8))):
+        wl = synth.custom(48, 96, 160, dtype="bf16", outlier_frac=0.02, outlier_scale=20.0, block=32,
+                          sparsity=0.5, seed=31)
+        W, X = synth.make_W(wl), synth.make_X_tokens(wl)
+        W64, X64 = synth.to_f64(W, "bf16"), synth.to_f64(X, "bf16")
+        full = oracle.prune_layer(W64, Xt=X64, sparsity=float(np.float32(0.5)), pattern=pattern, nm=nm, block=32,
+                                  damp=0.01, method="thanos")
+        g = _fullsize.column_norms_sq(X, "bf16", chunk=50)
+        m0, decided = _fullsize.block0_expected(W64, g, pattern=pattern, nm=nm, sparsity=0.5, block=32, tol=0.0)
+        assert np.array_equal(m0, full["mask"][:, :32])
+        assert decided.shape == m0.shape
