@@ -9,12 +9,18 @@
  *   "Contribution one: solve a selected set directly", "Contribution two: keep
  *   the budget global and the execution local") and, for the column-sequential
  *   special case, "Weight Pruning in Large Language Models ..." (llms.blog),
- *   section "SparseGPT: Second-Order Reconstruction at Scale".
+ *   section "SparseGPT: Second-Order Reconstruction at Scale".  The same page's
+ *   sections "Wanda: Pruning by Weights and Activations", "The Failure of Magnitude
+ *   Pruning in Large Transformers" and "N:M Semi-Structured Sparsity (2:4 Pattern)"
+ *   define the no-update methods (PWP_WANDA, PWP_MAGNITUDE) and the compressed 2:4
+ *   storage (pwp_pack_24).
  *
  * Conventions for every entry point:
  *   - All pointers named *_dev are device pointers; the caller owns every buffer.
- *     The library allocates no device or host memory: all scratch comes from the
- *     caller's workspace `ws` of `ws_bytes` bytes (at least 256-byte aligned).
+ *     The library allocates no device memory: all scratch comes from the caller's
+ *     workspace `ws` of `ws_bytes` bytes (at least 256-byte aligned), or, for
+ *     pwp_prune_layer_noalloc, from one static array inside the library.  Only the
+ *     optional event timing (pwp_profile_enable) creates CUDA events.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream)
  *     and the call returns without synchronising.
  *   - Argument errors are detected on the host before anything is enqueued and

@@ -59,7 +59,7 @@ const char* pwp_status_string(int32_t status) {
   }
 }
 
-int32_t pwp_version(void) { return 100; }
+int32_t pwp_version(void) { return 200; }
 
 size_t pwp_workspace_bytes(const pwp_config* cfg, int32_t c, int32_t b) {
   if (!valid_cfg(cfg, c, b)) return 0;
