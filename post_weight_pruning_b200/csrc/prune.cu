@@ -478,7 +478,7 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
       prof_begin(kKSelect, s);
       launch_pick1(pb.ctl, pb.hist1, region, thanos ? 1 : 0, quota, st, s);
       launch_refine(score, Wout, c, b, j, thanos ? b : j1, sc, pb.ctl, pb.l2, st, s);
-      launch_pick2(score, pb.ctl, pb.l2, Wout, c, b, j, j1, sc, st, s);
+      launch_pick2(pb.ctl, pb.l2, st, s);
       launch_clear_level2(score, pb.ctl, pb.l2, Wout, c, b, j, j1, sc, s);
       launch_tie_pick(score, pb.ctl, pb.l2, Wout, c, b, j, j1, sc, st, s);
       prof_end(kKSelect, s);

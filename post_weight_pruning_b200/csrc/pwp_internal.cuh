@@ -178,8 +178,7 @@ void launch_pick1(Ctl* ctl, unsigned int* hist1, long long region_n, int global_
                   pwp_stats* st, cudaStream_t s);
 void launch_refine(int score, const float* W, int c, int b, int q0, int q1, const float* sc,
                    const Ctl* ctl, Level2 l2, const pwp_stats* st, cudaStream_t s);
-void launch_pick2(int score, Ctl* ctl, Level2 l2, const float* W, int c, int b, int j, int j1, const float* sc,
-                  pwp_stats* st, cudaStream_t s);
+void launch_pick2(Ctl* ctl, Level2 l2, pwp_stats* st, cudaStream_t s);
 // After pick2: clear the level-2 histograms the block wrote and, when only some tied
 // entries are taken, count the ties per block column (grid-wide); then find the cut-off.
 void launch_clear_level2(int score, const Ctl* ctl, Level2 l2, const float* W, int c, int b, int j, int j1,

@@ -161,10 +161,7 @@ __global__ void __launch_bounds__(256) refine_kernel(const float* __restrict__ W
   }
 }
 
-template <int SCORE>
-__global__ void __launch_bounds__(1024) pick2_kernel(Ctl* ctl, Level2 l2, const float* __restrict__ W, int c,
-                                                     int b, int j, int j1, const float* __restrict__ sc,
-                                                     pwp_stats* st) {
+__global__ void __launch_bounds__(1024) pick2_kernel(Ctl* ctl, Level2 l2, pwp_stats* st) {
   __shared__ long long sh_warp[32];
   __shared__ int sh_sel;
   __shared__ long long sh_base;
@@ -333,12 +330,8 @@ void launch_refine(int score, const float* W, int c, int b, int q0, int q1, cons
     refine_kernel<kObs><<<grid, 256, 0, s>>>(W, c, b, q0, q1, sc, ctl, l2.reread, l2.reread_sum, st);
 }
 
-void launch_pick2(int score, Ctl* ctl, Level2 l2, const float* W, int c, int b, int j, int j1, const float* sc,
-                  pwp_stats* st, cudaStream_t s) {
-  if (score == kWanda)
-    pick2_kernel<kWanda><<<1, 1024, 0, s>>>(ctl, l2, W, c, b, j, j1, sc, st);
-  else
-    pick2_kernel<kObs><<<1, 1024, 0, s>>>(ctl, l2, W, c, b, j, j1, sc, st);
+void launch_pick2(Ctl* ctl, Level2 l2, pwp_stats* st, cudaStream_t s) {
+  pick2_kernel<<<1, 1024, 0, s>>>(ctl, l2, st);
 }
 
 void launch_clear_level2(int score, const Ctl* ctl, Level2 l2, const float* W, int c, int b, int j, int j1,

@@ -81,6 +81,8 @@ def test_small_layer_matches_oracle(name, method, pattern, nm):
     (64, 256, 512, 128, "fp32", "thanos", "unstructured", (0, 0), 0.8),      # rows above 80 selected
     (48, 256, 512, 128, "fp32", "thanos", "unstructured", (0, 0), 0.93),
     (32, 256, 512, 128, "fp32", "thanos", "nm", (1, 4), 0.5),                # 96 per row
+    (24, 150, 200, 32, "fp32", "thanos", "unstructured", (0, 0), 0.5),       # b % 4 != 0: CUDA-core update
+    (24, 150, 200, 32, "fp32", "sparsegpt", "unstructured", (0, 0), 0.5),    #   and factor fallbacks
 ])
 def test_shapes_and_edges_match_oracle(c, b, n, B, dtype, method, pattern, nm, s):
     _torch()
