@@ -13,9 +13,11 @@
 // H_d^-1 = V^-T V^-1 = U^T U with U upper, this is the required factor.
 // Both phases run in place on the upper triangle of H:
 //   factor, 64-column panels from the last: rows above the panel via the diagonal
-//     block's explicit inverse, then a symmetric rank-64 update of the top-left part;
-//     the CTA that updates the next panel's diagonal block also factors and inverts it
-//     (look-ahead), so the serial chain is one kernel pair per panel;
+//     block's explicit inverse, then a symmetric rank-64 update of the top-left part
+//     on the tensor cores (the 3xTF32 update kernel, tiles on or above the diagonal),
+//     then the next panel's diagonal block, factored and inverted by one CTA; where TMA
+//     cannot take the shape, a CUDA-core update whose CTA holding the next diagonal
+//     block also factors and inverts it (look-ahead);
 //   inverse, recursive doubling: with the diagonal blocks inverted, neighbouring
 //     blocks [A B; 0 D] are merged as [A^-1, -A^-1 B D^-1; 0, D^-1] level by level,
 //     each level two batched triangular-times-dense products.
