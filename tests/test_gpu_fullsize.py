@@ -12,7 +12,7 @@ import synth
 from tests import _fullsize as F
 from tests import _parity as P
 
-pytestmark = pytest.mark.gpu
+pytestmark = [pytest.mark.gpu, pytest.mark.fullsize]
 
 TIE_TOL = 2e-5
 
