@@ -128,9 +128,27 @@ def _dtype_code(t):
 
 
 def _need_cuda(*ts):
+    dev = None
     for t in ts:
-        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+        if t is None:
+            continue
+        if not t.is_cuda or not t.is_contiguous():
             raise ValueError("tensors must be contiguous CUDA tensors")
+        if dev is not None and t.device != dev:
+            raise ValueError(f"tensors on different devices ({dev}, {t.device})")
+        dev = t.device
+
+
+def _expect(t, name, shape, dtypes):
+    """The kernels see only a pointer and the sizes passed beside it, so a tensor whose
+    shape or element type differs from them would be read or written out of bounds:
+    reject it here."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected one of {[str(d) for d in dtypes]}")
 
 
 def new_stats(device="cuda"):
@@ -146,11 +164,14 @@ def read_stats(stats_t) -> Stats:
 def hessian_accumulate(X, H=None, beta=0, stream=None):
     """H := beta*H + 2 X X^T for token-major X ([n, b], bf16 or fp32 CUDA tensor)."""
     torch = _torch()
-    _need_cuda(X)
+    if X.dim() != 2:
+        raise ValueError(f"X: expected [n, b], got shape {tuple(X.shape)}")
     n, b = X.shape
+    _expect(X, "X", (n, b), (torch.bfloat16, torch.float32))
+    _expect(H, "H", (b, b), (torch.float32,))
+    _need_cuda(X, H)
     if H is None:
         H = torch.empty((b, b), dtype=torch.float32, device=X.device)
-    _need_cuda(H)
     st = lib().pwp_hessian_accumulate(_vp(X.data_ptr()), _dtype_code(X), int(n), int(b), _vp(H.data_ptr()),
                                       int(beta), _stream_ptr(stream))
     _check(st, "pwp_hessian_accumulate")
@@ -161,8 +182,9 @@ def damp_factor(H, damp=0.01, stream=None):
     """In place: upper triangle of H becomes U with (H + lambda I)^-1 = U^T U.
     Returns (g_diag, stats tensor)."""
     torch = _torch()
-    _need_cuda(H)
     b = H.shape[0]
+    _expect(H, "H", (b, b), (torch.float32,))
+    _need_cuda(H)
     g = torch.empty(b, dtype=torch.float32, device=H.device)
     nws = int(lib().pwp_factor_workspace_bytes(int(b)))
     ws = torch.empty(nws, dtype=torch.uint8, device=H.device)
@@ -199,8 +221,22 @@ def prune_layer(W, *, H=None, X=None, sparsity=0.5, pattern="unstructured", nm=(
     mask uint8, Stats) -- with check=False the stats tensor is returned unread and
     nothing syncs."""
     torch = _torch()
-    _need_cuda(W, H, X)
+    if W.dim() != 2:
+        raise ValueError(f"W: expected [c, b], got shape {tuple(W.shape)}")
     c, b = W.shape
+    _expect(W, "W", (c, b), (torch.bfloat16, torch.float32))
+    _expect(H, "H", (b, b), (torch.float32,))
+    if X is not None:
+        if X.dim() != 2:
+            raise ValueError(f"X: expected [n, b], got shape {tuple(X.shape)}")
+        _expect(X, "X", (X.shape[0], b), (torch.bfloat16, torch.float32))
+    _expect(W_out, "W_out", (c, b), (torch.float32,))
+    _expect(mask, "mask", (c, b), (torch.uint8,))
+    _expect(stats, "stats", (ctypes.sizeof(Stats),), (torch.uint8,))
+    if workspace is not None and workspace.nbytes > workspace.ws.numel() * workspace.ws.element_size():
+        raise ValueError(f"workspace: {workspace.nbytes} bytes claimed, tensor holds "
+                         f"{workspace.ws.numel() * workspace.ws.element_size()}")
+    _need_cuda(W, H, X, W_out, mask, stats, workspace.ws if workspace is not None else None)
     cfg = config(method, pattern, nm, sparsity, block, damp)
     if workspace is None:
         workspace = make_workspace(cfg, c, b, W.device)
@@ -245,8 +281,12 @@ def pack_24(W_hat, mask, *, stream=None, check=True):
     of four.  Returns (values: int16 [c, b/2] holding bfloat16 bit patterns, meta: int32
     [c, ceil(b/32)] holding the 4-bit position fields, Stats or the unread stats tensor)."""
     torch = _torch()
-    _need_cuda(W_hat, mask)
+    if W_hat.dim() != 2:
+        raise ValueError(f"W_hat: expected [c, b], got shape {tuple(W_hat.shape)}")
     c, b = W_hat.shape
+    _expect(W_hat, "W_hat", (c, b), (torch.float32,))
+    _expect(mask, "mask", (c, b), (torch.uint8,))
+    _need_cuda(W_hat, mask)
     values = torch.empty((c, b // 2), dtype=torch.int16, device=W_hat.device)
     meta = torch.empty((c, (b // 4 + 7) // 8), dtype=torch.int32, device=W_hat.device)
     stats = new_stats(W_hat.device)
