@@ -1,0 +1,111 @@
+"""One layer on several GPUs: token-sharded H and row-sharded prunes.
+
+One process per GPU; torch.distributed (NCCL between GPUs) carries the one exchange.
+Both shardings are exact by the structure of the problem:
+
+* Tokens.  H = 2 X X^T is a sum over calibration tokens ("Pruning LLMs with Thanos",
+  "The layer-reconstruction lens"; the weight-pruning blog page, "SparseGPT:
+  Second-Order Reconstruction at Scale"), so rank r builds 2 X_r X_r^T from its own
+  token shard on the tensor cores and one all-reduce (sum) leaves H on every rank.
+* Rows.  The reconstruction loss is a sum of independent per-row terms (same section of
+  the Thanos page).  With H on every rank, each rank factors it and prunes its own slice
+  of W's rows, which reproduces the rows of a one-GPU prune on that H wherever nothing
+  couples rows: N:M patterns (every group lies inside one row) and the per-row quotas
+  of Wanda and magnitude.  The unstructured global budget of Thanos and SparseGPT ties
+  every row to each block's threshold ("Contribution two: keep the budget global and the
+  execution local"); sharding it needs the block's selection histograms reduced across
+  ranks inside the sweep, which is not done here, so that case is refused.
+
+Without an initialised process group every function acts as a single rank.
+"""
+from __future__ import annotations
+
+from . import MAGNITUDE, METHODS, NM, WANDA, hessian_accumulate, prune_layer
+
+__all__ = ["token_range", "row_range", "rows_independent", "allreduce_hessian", "hessian_sharded",
+           "prune_rows", "gather_rows"]
+
+
+def _dist():
+    import torch.distributed as dist
+    return dist
+
+
+def _world(group=None):
+    dist = _dist()
+    if not (dist.is_available() and dist.is_initialized()):
+        return 1, 0
+    return dist.get_world_size(group), dist.get_rank(group)
+
+
+def _split(total: int, world: int, rank: int):
+    if world < 1 or not 0 <= rank < world or total < 0:
+        raise ValueError(f"bad split: total={total} world={world} rank={rank}")
+    base, extra = divmod(total, world)
+    lo = rank * base + min(rank, extra)
+    return lo, lo + base + (1 if rank < extra else 0)
+
+
+def token_range(n: int, world: int, rank: int):
+    """[t0, t1): this rank's calibration tokens; shards differ in size by at most one."""
+    return _split(n, world, rank)
+
+
+def row_range(c: int, world: int, rank: int):
+    """[r0, r1): this rank's rows of W; shards differ in size by at most one."""
+    return _split(c, world, rank)
+
+
+def rows_independent(method="thanos", pattern="unstructured") -> bool:
+    """True where a prune of a row slice gives exactly those rows of the whole-layer prune."""
+    m = METHODS[method] if isinstance(method, str) else int(method)
+    p = ({"unstructured": 0, "nm": NM}[pattern] if isinstance(pattern, str) else int(pattern))
+    return p == NM or m in (WANDA, MAGNITUDE)
+
+
+def allreduce_hessian(H, group=None):
+    """In place: every rank's partial 2 X_r X_r^T becomes the sum over ranks."""
+    world, _ = _world(group)
+    if world > 1:
+        dist = _dist()
+        dist.all_reduce(H, op=dist.ReduceOp.SUM, group=group)
+    return H
+
+
+def hessian_sharded(X_local, group=None, stream=None):
+    """H = 2 X X^T over the tokens of all ranks: this rank's token shard X_local ([n_r, b],
+    bf16/fp32 CUDA tensor) on the tensor cores, then one all-reduce.  Every rank must pass
+    the same b; a rank may hold no tokens (n_r = 0)."""
+    H = hessian_accumulate(X_local, stream=stream)
+    return allreduce_hessian(H, group)
+
+
+def prune_rows(W_local, H, *, method="thanos", pattern="nm", group=None, **kw):
+    """Prune this rank's rows W_local ([c_r, b]) against the whole layer's H (destroyed
+    as in ``prune_layer``).  Only where ``rows_independent(method, pattern)``; returns
+    ``prune_layer``'s (W_hat, mask, stats) for the local rows."""
+    if not rows_independent(method, pattern):
+        raise NotImplementedError(
+            "unstructured Thanos/SparseGPT couples all rows through each block's global threshold; "
+            "row sharding it needs the selection histograms reduced across ranks inside the sweep")
+    if H is None and (METHODS[method] if isinstance(method, str) else int(method)) != MAGNITUDE:
+        raise ValueError("give the layer's H (hessian_sharded)")
+    return prune_layer(W_local, H=H, method=method, pattern=pattern, **kw)
+
+
+def gather_rows(local, c: int, group=None):
+    """Concatenate every rank's row slice (as cut by ``row_range``) into the [c, ...]
+    tensor on every rank."""
+    import torch
+    world, rank = _world(group)
+    r0, r1 = row_range(c, world, rank)
+    if local.shape[0] != r1 - r0:
+        raise ValueError(f"rank {rank} holds {local.shape[0]} rows, row_range gives {r1 - r0}")
+    if world == 1:
+        return local
+    rows = -(-c // world)                      # the largest shard
+    padded = torch.zeros((rows,) + tuple(local.shape[1:]), dtype=local.dtype, device=local.device)
+    padded[: r1 - r0].copy_(local)
+    parts = [torch.empty_like(padded) for _ in range(world)]
+    _dist().all_gather(parts, padded, group=group)
+    return torch.cat([p[: row_range(c, world, r)[1] - row_range(c, world, r)[0]] for r, p in enumerate(parts)])

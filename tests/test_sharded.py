@@ -1,0 +1,133 @@
+"""Host logic of the multi-GPU layer prune (CPU): the token and row splits, the
+all-reduce of per-rank Hessians and the row gather over gloo ranks (world size 2), and,
+on the oracle, the property that makes row sharding exact -- for N:M patterns and the
+per-row quotas of Wanda and magnitude a prune of a row slice gives exactly those rows of
+the whole-layer prune, while the unstructured global budget couples the rows."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import oracle
+import synth
+from post_weight_pruning_b200 import sharded
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+@pytest.mark.parametrize("total,world", [(0, 1), (7, 2), (16384, 3), (5, 8), (11008, 8)])
+def test_splits_partition_and_balance(total, world):
+    for split in (sharded.token_range, sharded.row_range):
+        ranges = [split(total, world, r) for r in range(world)]
+        assert ranges[0][0] == 0 and ranges[-1][1] == total
+        assert all(a[1] == b[0] for a, b in zip(ranges, ranges[1:]))
+        sizes = [hi - lo for lo, hi in ranges]
+        assert min(sizes) >= 0 and max(sizes) - min(sizes) <= 1
+
+
+def test_split_rejects_bad_rank():
+    with pytest.raises(ValueError):
+        sharded.row_range(10, 2, 2)
+
+
+@pytest.mark.parametrize("method,pattern,want", [
+    ("thanos", "nm", True), ("sparsegpt", "nm", True), ("wanda", "unstructured", True),
+    ("magnitude", "unstructured", True), ("thanos", "unstructured", False), ("sparsegpt", "unstructured", False),
+])
+def test_rows_independent(method, pattern, want):
+    assert sharded.rows_independent(method, pattern) is want
+
+
+def test_prune_rows_refuses_the_global_budget():
+    W = torch.zeros(8, 16)
+    with pytest.raises(NotImplementedError):
+        sharded.prune_rows(W, torch.zeros(16, 16), method="thanos", pattern="unstructured")
+
+
+def _layer(c=24, b=64, n=256, seed=5):
+    wl = synth.custom(c, b, n, dtype="fp32", outlier_frac=0.05, outlier_scale=10.0, seed=seed)
+    W = synth.to_f64(synth.make_W(wl), "fp32")
+    Xt = synth.to_f64(synth.make_X_tokens(wl), "fp32")
+    return W, Xt
+
+
+@pytest.mark.parametrize("method,pattern,nm", [
+    ("thanos", "nm", (2, 4)), ("thanos", "nm", (4, 8)), ("sparsegpt", "nm", (2, 4)),
+])
+def test_oracle_row_slices_reproduce_the_layer_nm(method, pattern, nm):
+    W, Xt = _layer()
+    H = oracle.hessian(Xt)
+    full = oracle.prune_layer(W, H=H, method=method, pattern=pattern, nm=nm, block=16)
+    for world in (2, 3):
+        for r in range(world):
+            r0, r1 = sharded.row_range(W.shape[0], world, r)
+            part = oracle.prune_layer(W[r0:r1], H=H, method=method, pattern=pattern, nm=nm, block=16)
+            assert np.array_equal(part["mask"], full["mask"][r0:r1])
+            np.testing.assert_allclose(part["W"], full["W"][r0:r1], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("method,pattern", [("wanda", "unstructured"), ("magnitude", "unstructured"),
+                                            ("wanda", "nm")])
+def test_oracle_row_slices_reproduce_the_layer_no_update(method, pattern):
+    W, Xt = _layer(c=21)
+    full = oracle.prune_no_update(W, Xt=Xt, method=method, pattern=pattern, sparsity=0.4)
+    for r in range(3):
+        r0, r1 = sharded.row_range(W.shape[0], 3, r)
+        part = oracle.prune_no_update(W[r0:r1], Xt=Xt, method=method, pattern=pattern, sparsity=0.4)
+        assert np.array_equal(part["mask"], full["mask"][r0:r1])
+        assert np.array_equal(part["W"], full["W"][r0:r1])
+
+
+def test_oracle_unstructured_budget_couples_rows():
+    # rows of very different scale: the global budget takes most removals from the small
+    # rows, a per-slice budget cannot
+    W, Xt = _layer(c=24)
+    W[:12] *= 10.0
+    H = oracle.hessian(Xt)
+    full = oracle.prune_layer(W, H=H, method="thanos", sparsity=0.5, block=16)
+    part = oracle.prune_layer(W[:12], H=H, method="thanos", sparsity=0.5, block=16)
+    assert full["mask"][:12].sum() < part["mask"].sum()
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        W, Xt = _layer(c=7, n=250)
+        t0, t1 = sharded.token_range(Xt.shape[0], world, rank)
+        H = torch.from_numpy(oracle.hessian(Xt[t0:t1]))       # this rank's 2 X_r X_r^T
+        sharded.allreduce_hessian(H)
+        r0, r1 = sharded.row_range(W.shape[0], world, rank)
+        G = sharded.gather_rows(torch.from_numpy(W[r0:r1]).contiguous(), W.shape[0])
+        out[rank] = (H.numpy(), G.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_reduce_h_and_gather_rows():
+    world = 2
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_worker, args=(world, _free_port(), out), nprocs=world, start_method="spawn")
+    W, Xt = _layer(c=7, n=250)
+    H_ref = oracle.hessian(Xt)
+    for r in range(world):
+        H, G = out[r]
+        np.testing.assert_allclose(H, H_ref, rtol=1e-12, atol=1e-12 * np.abs(H_ref).max())
+        assert np.array_equal(G, W)
+    assert np.array_equal(out[0][0], out[1][0])
+
+
+def test_single_rank_without_process_group():
+    W = torch.arange(12.0).reshape(4, 3)
+    assert sharded.gather_rows(W, 4) is W
+    H = torch.ones(3, 3)
+    assert sharded.allreduce_hessian(H) is H
