@@ -41,6 +41,12 @@ CLASS_SOURCES = {K_HESSIAN: ["hessian_tc.cu", "hessian_simt.cu"], K_FACTOR: ["fa
                  K_STREAM: ["stream_tc.cu", "prune.cu"], K_SELECT: ["select.cu"], K_SOLVE: ["solve.cu"],
                  K_ROWPRUNE: ["rowprune.cu"], K_COLNORM: ["rowprune.cu"]}
 SECOND_ORDER = ("thanos", "sparsegpt")
+# The only prune times the source pages give: whole models on other hardware, context only.
+PAGES_CONTEXT = {
+    "sparsegpt": "about 4 h to prune a 175B-parameter model to 50% unstructured on one A100 (whole model)",
+    "wanda": "under 10 min for a 70B-parameter model on one GPU (whole model, no reconstruction)",
+    "thanos": "no prune time reported",
+}
 
 
 def _load_peaks():
@@ -414,6 +420,7 @@ def run_mine(args):
                     "h2d_bytes_per_step": int(W_host.numel() * 2 + X_host.numel() * 2),
                     "d2h_bytes_per_step": int(out_W.numel() * 4 + out_m.numel())},
             "clocks": clocks,
+            "context_from_pages": PAGES_CONTEXT,
         }
         if method in SECOND_ORDER:
             line["select_stats"] = {"blocks": nblk, "reread_blocks": int(st.reread_blocks),

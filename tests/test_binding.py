@@ -62,3 +62,96 @@ def test_pack_24_refuses_mismatched_buffers():
         pwp.pack_24(torch.zeros(4, 8), torch.zeros(4, 4, dtype=torch.uint8))
     with pytest.raises(TypeError):
         pwp.pack_24(torch.zeros(4, 8), torch.zeros(4, 8, dtype=torch.bool))
+
+
+class _FakeLib:
+    """Stands in for libpwp.so so that the marshalling runs on the CPU: records the
+    arguments of each entry point and reports success."""
+
+    def __init__(self, ws_bytes=4096):
+        self.ws_bytes = ws_bytes
+        self.calls = {}
+
+    def pwp_workspace_bytes(self, cfg, c, b):
+        return self.ws_bytes
+
+    def _record(name):
+        def f(self, *a):
+            self.calls[name] = a
+            return 0
+        return f
+
+    pwp_prune_layer = _record("pwp_prune_layer")
+    pwp_prune_layer_x = _record("pwp_prune_layer_x")
+    pwp_pack_24 = _record("pwp_pack_24")
+    pwp_hessian_accumulate = _record("pwp_hessian_accumulate")
+
+
+@pytest.fixture
+def fake(monkeypatch):
+    import ctypes
+    f = _FakeLib()
+    monkeypatch.setattr(pwp, "lib", lambda: f)
+    monkeypatch.setattr(pwp, "_need_cuda", lambda *ts: None)
+    monkeypatch.setattr(pwp, "_stream_ptr", lambda stream=None: ctypes.c_void_p(0))
+    return f
+
+
+def _ptr(v):
+    return v.value if hasattr(v, "value") else v
+
+
+def test_prune_layer_x_marshalling(fake):
+    c, b, n = 6, 32, 40
+    W = torch.zeros(c, b, dtype=torch.bfloat16)
+    X = torch.zeros(n, b, dtype=torch.float32)
+    W_hat, mask, st = pwp.prune_layer(W, X=X, method="thanos", pattern="nm", nm=(2, 4), block=16, damp=0.05)
+    a = fake.calls["pwp_prune_layer_x"]
+    cfg = a[0]._obj
+    assert (cfg.method, cfg.pattern, cfg.nm_n, cfg.nm_m, cfg.block) == (pwp.THANOS, pwp.NM, 2, 4, 16)
+    assert cfg.damp == pytest.approx(0.05)
+    assert _ptr(a[1]) == W.data_ptr() and a[2] == pwp.BF16 and (a[3], a[4]) == (c, b)
+    assert _ptr(a[5]) == X.data_ptr() and a[6] == pwp.FP32 and a[7] == n
+    assert _ptr(a[8]) not in (None, 0)                      # an H scratch was allocated
+    assert _ptr(a[9]) == W_hat.data_ptr() and _ptr(a[10]) == mask.data_ptr()
+    assert a[12] == fake.ws_bytes
+    assert W_hat.shape == (c, b) and W_hat.dtype == torch.float32
+    assert mask.shape == (c, b) and mask.dtype == torch.uint8
+    assert st.status == 0
+
+
+def test_prune_layer_no_update_passes_no_h(fake):
+    W = torch.zeros(4, 16, dtype=torch.float32)
+    X = torch.zeros(8, 16, dtype=torch.bfloat16)
+    pwp.prune_layer(W, X=X, method="wanda", sparsity=0.25)
+    a = fake.calls["pwp_prune_layer_x"]
+    assert a[0]._obj.method == pwp.WANDA
+    assert _ptr(a[8]) in (None, 0)
+    pwp.prune_layer(W, method="magnitude", check=False)
+    a = fake.calls["pwp_prune_layer"]
+    assert a[0]._obj.method == pwp.MAGNITUDE and _ptr(a[5]) in (None, 0)
+
+
+def test_prune_layer_with_h_and_caller_buffers(fake):
+    c, b = 5, 24
+    W = torch.zeros(c, b)
+    H = torch.zeros(b, b)
+    W_out = torch.zeros(c, b)
+    mask = torch.zeros(c, b, dtype=torch.uint8)
+    ws = pwp.Workspace(torch.zeros(4096, dtype=torch.uint8), 4096)
+    stats = pwp.new_stats("cpu")
+    r = pwp.prune_layer(W, H=H, W_out=W_out, mask=mask, workspace=ws, stats=stats, check=False)
+    assert r[0] is W_out and r[1] is mask and r[2] is stats
+    a = fake.calls["pwp_prune_layer"]
+    assert _ptr(a[5]) == H.data_ptr() and _ptr(a[8]) == ws.ws.data_ptr() and a[9] == 4096
+    assert _ptr(a[10]) == stats.data_ptr()
+
+
+def test_pack_24_marshalling(fake):
+    c, b = 3, 100
+    values, meta, st = pwp.pack_24(torch.zeros(c, b), torch.zeros(c, b, dtype=torch.uint8))
+    a = fake.calls["pwp_pack_24"]
+    assert (a[2], a[3]) == (c, b)
+    assert values.shape == (c, b // 2) and values.dtype == torch.int16
+    assert meta.shape == (c, 4) and meta.dtype == torch.int32        # ceil(25 groups / 8)
+    assert _ptr(a[4]) == values.data_ptr() and _ptr(a[5]) == meta.data_ptr()
