@@ -32,7 +32,7 @@ def test_token_shards_sum_to_the_layer_hessian():
         Hs += sharded.hessian_sharded(Xt[t0:t1].contiguous())   # no process group: one rank's share
     torch.cuda.synchronize()
     d = torch.sqrt(torch.diagonal(H))
-    assert float(((Hs - H).abs() / torch.outer(d, d)).max()) < 1e-5
+    assert float(((Hs - H).abs() / torch.outer(d, d)).max()) < 3e-5     # each side within 1e-5 of fp64
 
 
 @pytest.mark.parametrize("method,pattern,nm,sparsity", [
