@@ -499,3 +499,18 @@ def test_block0_expectation_matches_the_full_oracle():
         m0, decided = _fullsize.block0_expected(W64, g, pattern=pattern, nm=nm, sparsity=0.5, block=32, tol=0.0)
         assert np.array_equal(m0, full["mask"][:, :32])
         assert decided.shape == m0.shape
+
+
+def test_dead_features_go_first_and_undamped_singular_h_is_refused():
+    """A feature that is zero on every token has G_qq = 0, so its weights score 0 and the
+    global budget takes all of them first; the damping keeps H_d positive definite.  With
+    damp 0 the same H is singular and the factor refuses it."""
+    rng = np.random.default_rng(8)
+    Xt = rng.normal(size=(64, 16))
+    Xt[:, [3, 7]] = 0.0
+    W = rng.normal(0, 0.02, size=(8, 16))
+    r = oracle.prune_layer(W, Xt=Xt, sparsity=0.5, block=16, damp=0.01)
+    assert r["mask"][:, [3, 7]].all()
+    assert r["pruned"] == 64
+    with pytest.raises(np.linalg.LinAlgError):
+        oracle.prune_layer(W, Xt=Xt, sparsity=0.5, block=16, damp=0.0)
