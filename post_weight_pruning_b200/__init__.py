@@ -20,7 +20,7 @@ import numpy as np
 __all__ = [
     "lib", "Config", "Stats", "THANOS", "SPARSEGPT", "WANDA", "MAGNITUDE", "UNSTRUCTURED", "NM", "BF16", "FP32",
     "PwpError", "config", "workspace_bytes", "hessian_accumulate", "damp_factor", "prune_layer",
-    "prune_layer_host", "status_string", "LIB_PATH",
+    "prune_layer_host", "prune_block", "pack_24", "status_string", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpwp.so")
@@ -273,6 +273,44 @@ def prune_layer(W, *, H=None, X=None, sparsity=0.5, pattern="unstructured", nm=(
     if s.status != 0:
         raise PwpError(s.status, where + " (device)")
     return W_out, mask, s
+
+
+def prune_block(weights, activations, feeds, *, stream=None, check=True, **cfg):
+    """Prune the linear layers of one transformer block.  Thanos / SparseGPT: one H per
+    distinct input, built once on the tensor cores and shared by every layer that reads
+    that input (q, k and v read the attention input; gate and up the MLP input).  Wanda /
+    magnitude: no H.
+
+    weights: {layer: W [c, b]}; activations: {input: X [n, b]} (token-major);
+    feeds: {layer: input}; cfg: as for ``prune_layer`` (method, pattern, sparsity, ...).
+    Returns {layer: (W_hat, mask, Stats)} (the unread stats tensor with check=False)."""
+    torch = _torch()
+    for layer, W in weights.items():
+        if layer not in feeds or feeds[layer] not in activations:
+            raise ValueError(f"layer {layer!r}: no input given")
+        if W.dim() != 2 or activations[feeds[layer]].shape[-1] != W.shape[1]:
+            raise ValueError(f"layer {layer!r}: W {tuple(W.shape)} does not match its input "
+                             f"{tuple(activations[feeds[layer]].shape)}")
+    method = cfg.get("method", "thanos")
+    m = METHODS[method] if isinstance(method, str) else int(method)
+    out = {}
+    for inp, X in activations.items():
+        users = [layer for layer in weights if feeds[layer] == inp]
+        if not users:
+            continue
+        if m in (WANDA, MAGNITUDE):
+            # no Hessian: Wanda takes the feature norms straight from X
+            for layer in users:
+                out[layer] = prune_layer(weights[layer], X=X, stream=stream, check=check, **cfg)
+            continue
+        H = hessian_accumulate(X, stream=stream)
+        for i, layer in enumerate(users):
+            # the prune overwrites its H with the factor: every reader of the input but
+            # the last gets a copy
+            Hl = H if i == len(users) - 1 else H.clone()
+            out[layer] = prune_layer(weights[layer], H=Hl, stream=stream, check=check, **cfg)
+        del H
+    return out
 
 
 def pack_24(W_hat, mask, *, stream=None, check=True):

@@ -5,8 +5,9 @@ holds none of the pruning arithmetic, so both the CUDA path and the fp64
 oracle can consume the same bytes without sharing any of the method.
 
 Every draw is addressable: row ``k`` of ``W`` comes from
-``default_rng([seed, 0, k])`` and feature row ``i`` of the activations of input
-``a`` (the pages' ``X`` is ``b x n`` with examples as columns, "Pruning LLMs
+``default_rng([seed, 0, k])`` (layer ``l > 0`` of a decoder block:
+``default_rng([seed, 100 + l, k])``) and feature row ``i`` of the activations of
+input ``a`` (the pages' ``X`` is ``b x n`` with examples as columns, "Pruning LLMs
 with Thanos", section "The layer-reconstruction lens") comes from
 ``default_rng([seed, 1 + a, i])``, so any subset of rows can be regenerated
 without drawing the rest.  Outlier features are chosen by
@@ -19,12 +20,14 @@ here fewer Gaussian or Laplace sequences stand in for that dataset).
 from __future__ import annotations
 
 import dataclasses
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 
 __all__ = [
     "Workload", "WORKLOADS", "workload", "make_W", "make_X_features",
     "make_X_tokens", "f64_to_bf16_bits", "bf16_bits_to_f64", "bf16_bits_to_f32",
-    "custom",
+    "custom", "decoder_block", "BLOCK_INPUTS", "BLOCK_LAYERS",
 ]
 
 
@@ -45,6 +48,7 @@ class Workload:
     damp: float = 0.01
     seed: int = 0
     input_id: int = 0      # which activation stream feeds this layer
+    w_id: int = 0          # which weight stream (layers of one decoder block differ)
 
 
 WORKLOADS = {
@@ -63,8 +67,36 @@ WORKLOADS = {
 }
 
 
+# One LLaMA-7B-shaped decoder block, 128 x 2048 calibration tokens: four activation
+# inputs (q, k, v read the attention input; gate and up the MLP input) and seven layers,
+# all at 50% unstructured with the global budget, B = 128.
+BLOCK_TOKENS = 128 * 2048
+BLOCK_INPUTS = {          # name: (b, distribution, outlier fraction, outlier scale, input id)
+    "attn_in": (4096, "gaussian", 0.005, 50.0, 1),
+    "o_in": (4096, "gaussian", 0.005, 50.0, 2),
+    "mlp_in": (4096, "gaussian", 0.005, 50.0, 3),
+    "down_in": (11008, "laplace", 0.0, 1.0, 4),
+}
+BLOCK_LAYERS = [          # (name, input, c); the layer's index is its weight stream
+    ("q_proj", "attn_in", 4096), ("k_proj", "attn_in", 4096), ("v_proj", "attn_in", 4096),
+    ("o_proj", "o_in", 4096), ("gate_proj", "mlp_in", 11008), ("up_proj", "mlp_in", 11008),
+    ("down_proj", "down_in", 4096),
+]
+
+
 def workload(name: str) -> Workload:
     return WORKLOADS[name]
+
+
+def decoder_block(n: int = BLOCK_TOKENS):
+    """{layer name: (input name, Workload)} of the decoder block; layers that read the
+    same input have identical activation parameters, so make_X_tokens gives one X."""
+    out = {}
+    for l, (name, inp, c) in enumerate(BLOCK_LAYERS):
+        b, dist, frac, scale, a = BLOCK_INPUTS[inp]
+        out[name] = (inp, Workload(f"block_{name}", c, b, n, "bf16", dist, frac, scale, "unstructured",
+                                   (0, 0), 0.5, 128, 0.01, 0, a, l))
+    return out
 
 
 def custom(c, b, n, dtype="fp32", x_dist="gaussian", outlier_frac=0.0, outlier_scale=1.0,
@@ -117,8 +149,9 @@ def make_W(wl: Workload, rows=None) -> np.ndarray:
     rows = range(wl.c) if rows is None else rows
     rows = list(rows)
     out = np.empty((len(rows), wl.b), dtype=np.float64)
+    stream = 0 if wl.w_id == 0 else 100 + wl.w_id
     for i, k in enumerate(rows):
-        out[i] = np.random.default_rng([wl.seed, 0, int(k)]).normal(0.0, 0.02, wl.b)
+        out[i] = np.random.default_rng([wl.seed, stream, int(k)]).normal(0.0, 0.02, wl.b)
     return _store(out, wl.dtype)
 
 
@@ -155,13 +188,23 @@ def make_X_features(wl: Workload, features=None) -> np.ndarray:
     return _store(out, wl.dtype)
 
 
-def make_X_tokens(wl: Workload, chunk: int = 512) -> np.ndarray:
-    """Token-major activations [n, b] (PyTorch activation layout), storage dtype."""
+def make_X_tokens(wl: Workload, chunk: int = 512, threads: int = 1) -> np.ndarray:
+    """Token-major activations [n, b] (PyTorch activation layout), storage dtype.  With
+    threads > 1 feature chunks are drawn concurrently (each feature row has its own
+    generator, so the result is the same)."""
     dt = np.float32 if wl.dtype == "fp32" else np.uint16
     out = np.empty((wl.n, wl.b), dtype=dt)
-    for f0 in range(0, wl.b, chunk):
-        f1 = min(wl.b, f0 + chunk)
+
+    def fill(f0, f1):
         out[:, f0:f1] = make_X_features(wl, range(f0, f1)).T
+
+    if threads <= 1:
+        for f0 in range(0, wl.b, chunk):
+            fill(f0, min(wl.b, f0 + chunk))
+        return out
+    step = 64
+    with ThreadPoolExecutor(threads) as ex:
+        list(ex.map(lambda f0: fill(f0, min(wl.b, f0 + step)), range(0, wl.b, step)))
     return out
 
 

@@ -71,6 +71,7 @@ class _FakeLib:
     def __init__(self, ws_bytes=4096):
         self.ws_bytes = ws_bytes
         self.calls = {}
+        self.log = []
 
     def pwp_workspace_bytes(self, cfg, c, b):
         return self.ws_bytes
@@ -78,6 +79,7 @@ class _FakeLib:
     def _record(name):
         def f(self, *a):
             self.calls[name] = a
+            self.log.append((name, a))
             return 0
         return f
 
@@ -155,3 +157,38 @@ def test_pack_24_marshalling(fake):
     assert values.shape == (c, b // 2) and values.dtype == torch.int16
     assert meta.shape == (c, 4) and meta.dtype == torch.int32        # ceil(25 groups / 8)
     assert _ptr(a[4]) == values.data_ptr() and _ptr(a[5]) == meta.data_ptr()
+
+
+def test_prune_block_builds_one_h_per_input(fake):
+    b1, b2, n = 16, 24, 32
+    weights = {"q": torch.zeros(8, b1), "k": torch.zeros(4, b1), "o": torch.zeros(6, b1),
+               "down": torch.zeros(5, b2)}
+    acts = {"attn_in": torch.zeros(n, b1, dtype=torch.bfloat16), "o_in": torch.zeros(n, b1),
+            "down_in": torch.zeros(n, b2, dtype=torch.bfloat16)}
+    feeds = {"q": "attn_in", "k": "attn_in", "o": "o_in", "down": "down_in"}
+    out = pwp.prune_block(weights, acts, feeds, method="thanos", sparsity=0.5, block=8)
+    assert set(out) == set(weights)
+    hess = [a for name, a in fake.log if name == "pwp_hessian_accumulate"]
+    prunes = [a for name, a in fake.log if name == "pwp_prune_layer"]
+    assert [_ptr(a[0]) for a in hess] == [acts[k].data_ptr() for k in ("attn_in", "o_in", "down_in")]
+    assert [(a[3], a[4]) for a in prunes] == [(8, b1), (4, b1), (6, b1), (5, b2)]
+    h_ptr = [_ptr(a[4]) for a in hess]                  # where each H was built
+    # q gets a copy of the attention input's H, k (its last reader) the H itself
+    assert _ptr(prunes[0][5]) != h_ptr[0] and _ptr(prunes[1][5]) == h_ptr[0]
+    assert _ptr(prunes[2][5]) == h_ptr[1] and _ptr(prunes[3][5]) == h_ptr[2]
+
+
+def test_prune_block_wanda_needs_no_h(fake):
+    weights = {"gate": torch.zeros(8, 16), "up": torch.zeros(8, 16)}
+    acts = {"mlp_in": torch.zeros(32, 16, dtype=torch.bfloat16)}
+    pwp.prune_block(weights, acts, {"gate": "mlp_in", "up": "mlp_in"}, method="wanda")
+    assert not [1 for name, _ in fake.log if name == "pwp_hessian_accumulate"]
+    xs = [a for name, a in fake.log if name == "pwp_prune_layer_x"]
+    assert len(xs) == 2 and all(_ptr(a[5]) == acts["mlp_in"].data_ptr() for a in xs)
+
+
+def test_prune_block_checks_its_wiring(fake):
+    with pytest.raises(ValueError, match="no input"):
+        pwp.prune_block({"q": torch.zeros(4, 16)}, {"attn_in": torch.zeros(8, 16)}, {})
+    with pytest.raises(ValueError, match="does not match"):
+        pwp.prune_block({"q": torch.zeros(4, 16)}, {"a": torch.zeros(8, 12)}, {"q": "a"})
