@@ -284,7 +284,6 @@ def prune_block(weights, activations, feeds, *, stream=None, check=True, **cfg):
     weights: {layer: W [c, b]}; activations: {input: X [n, b]} (token-major);
     feeds: {layer: input}; cfg: as for ``prune_layer`` (method, pattern, sparsity, ...).
     Returns {layer: (W_hat, mask, Stats)} (the unread stats tensor with check=False)."""
-    torch = _torch()
     for layer, W in weights.items():
         if layer not in feeds or feeds[layer] not in activations:
             raise ValueError(f"layer {layer!r}: no input given")
