@@ -77,7 +77,11 @@ def hessian_sharded(X_local, group=None, stream=None):
     bf16/fp32 CUDA tensor) on the tensor cores, then one all-reduce.  Every rank must pass
     the same b; a rank may hold no tokens (n_r = 0)."""
     H = hessian_accumulate(X_local, stream=stream)
-    return allreduce_hessian(H, group)
+    if stream is None:
+        return allreduce_hessian(H, group)
+    import torch
+    with torch.cuda.stream(stream):            # the collective waits for the H build on this stream
+        return allreduce_hessian(H, group)
 
 
 def prune_rows(W_local, H, *, method="thanos", pattern="nm", group=None, **kw):
