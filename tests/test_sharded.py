@@ -131,3 +131,80 @@ def test_single_rank_without_process_group():
     assert sharded.gather_rows(W, 4) is W
     H = torch.ones(3, 3)
     assert sharded.allreduce_hessian(H) is H
+
+
+# --------------------------------------------------------------------------------------
+# The exchange the unstructured global budget needs under row sharding (not built on the
+# GPU): per block, every rank histograms its own keys, the histograms are summed across
+# ranks, and the per-column counts of keys equal to the threshold are gathered so that
+# every rank knows how many tied entries precede its own in (column, row) order.  Checked
+# here with the selection's two radix levels (13 + 18 bits of the fp32 key) and gloo ranks:
+# the union of the ranks' masks must be the oracle's lowest-r selection.
+
+LO_BITS = 18
+
+
+def _find_bin(hist, rank_1based):
+    """(bin holding the rank-th smallest key, number of keys in lower bins)."""
+    cum = np.cumsum(hist, dtype=np.int64)
+    b = int(np.searchsorted(cum, rank_1based))
+    return b, int(cum[b - 1]) if b > 0 else 0
+
+
+def _sharded_select(S_local, r, world):
+    """This rank's part of the lowest-r selection over all ranks' rows (rank order = row
+    order), with the exchanges a row-sharded GPU sweep would make."""
+    keys = S_local.astype(np.float32).view(np.uint32)
+    h1 = torch.from_numpy(np.bincount((keys >> LO_BITS).ravel(), minlength=1 << (31 - LO_BITS)).astype(np.int64))
+    dist.all_reduce(h1)                                              # exchange 1: level-1 counts
+    b1, below1 = _find_bin(h1.numpy(), r)
+    in_b1 = (keys >> LO_BITS) == b1
+    h2 = torch.from_numpy(np.bincount((keys[in_b1] & ((1 << LO_BITS) - 1)).ravel(),
+                                      minlength=1 << LO_BITS).astype(np.int64))
+    dist.all_reduce(h2)                                              # exchange 2: level-2 counts
+    b2, below2 = _find_bin(h2.numpy(), r - below1)
+    T = np.uint32((b1 << LO_BITS) | b2)
+    need = r - below1 - below2                                       # tied entries to take
+    tied = keys == T
+    t_local = torch.from_numpy(tied.sum(axis=0).astype(np.int64))   # per column
+    gathered = [torch.zeros_like(t_local) for _ in range(world)]
+    dist.all_gather(gathered, t_local)                               # exchange 3: tie counts
+    t_all = torch.stack(gathered).numpy()                            # [world, columns]
+    me = dist.get_rank()
+    before = np.concatenate([[0], np.cumsum(t_all.sum(axis=0))[:-1]]) + t_all[:me].sum(axis=0)
+    take = np.clip(need - before, 0, t_all[me])                      # this rank's ties per column
+    mask = keys < T
+    for q in np.flatnonzero(take):
+        rows = np.flatnonzero(tied[:, q])[: take[q]]
+        mask[rows, q] = True
+    return mask
+
+
+def _select_worker(rank, world, port, S32, r, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        r0, r1 = sharded.row_range(S32.shape[0], world, rank)
+        out[rank] = _sharded_select(S32[r0:r1], r, world)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,ties", [(2, False), (3, True)])
+def test_global_budget_exchange_reproduces_the_global_selection(world, ties):
+    rng = np.random.default_rng(40 + world)
+    W = rng.normal(0, 0.02, size=(29, 48))
+    if ties:
+        W = np.round(W * 64) / 64                  # large groups of equal scores
+    g = rng.uniform(0.5, 2.0, size=48) if not ties else np.ones(48)
+    S32 = oracle.wanda_scores(W, g).astype(np.float32)
+    r = int(0.45 * S32.size)
+    want, t_last, _ = oracle.lowest_global(S32.astype(np.float64), 0, r)
+    if ties:
+        assert (S32 == np.float32(t_last)).sum() > 10            # the boundary really is tied
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_select_worker, args=(world, _free_port(), S32, r, out), nprocs=world, start_method="spawn")
+    got = np.concatenate([out[k] for k in range(world)])
+    assert got.sum() == r
+    assert np.array_equal(got, want)
