@@ -1,5 +1,8 @@
-"""Host arithmetic of bench.py's roofline object: the algorithmic work of each kernel class
-for a small workload, against values worked out by hand from the stated definitions."""
+"""Host side of bench.py: the roofline object's algorithmic work of each kernel class for a
+small workload, against values worked out by hand from the stated definitions, and the
+reference arm's contract line."""
+import os
+
 import numpy as np
 
 import bench
@@ -44,3 +47,26 @@ def test_no_update_bytes():
 
 def test_alu_peak_formula():
     assert np.isclose(bench.fp32_alu_peak_tflops(1965.0), 148 * 128 * 2 * 1965e6 / 1e12)
+
+
+def test_reference_arm_prints_the_contract_line():
+    """The reference arm (the fp64 oracle on the host cores) runs without a GPU: its one
+    JSON line carries the keys of the benchmark contract."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "3"],
+                         cwd=root, capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "weights/s" and d["value"] > 0
+    assert (d["n_gpus"], d["steps"], d["warmup"]) == (1, 1, 3)
+    assert d["higher_is_better"] is True and d["vs_baseline"] is None and d["data"] == "synthetic"
+    assert d["config"]["workload"].startswith("q_proj4096x4096")
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": "weights/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert abs(d["ms_per_step"] - 4096 * 128 / d["value"] * 1e3) < 1e-6 * d["ms_per_step"]
