@@ -8,7 +8,7 @@ import pytest
 import synth
 from tests import _parity as P
 
-pytestmark = pytest.mark.gpu
+pytestmark = [pytest.mark.gpu, pytest.mark.integration]
 
 
 def _torch():

@@ -10,7 +10,7 @@ import pytest
 import synth
 from tests import _parity as P
 
-pytestmark = pytest.mark.gpu
+pytestmark = [pytest.mark.gpu, pytest.mark.integration]
 
 GUARD = 4096                       # guard elements on each side (a multiple of 256 bytes)
 F32_FILL = 0x7FC0DEAD              # a NaN pattern no kernel writes

@@ -6,9 +6,8 @@ It takes its scratch from one static device array inside the library.  Here it i
 called through the C ABI twice in a row on the same inputs -- the second call finds
 the first call's leftovers in that shared array -- and both results must match the
 regular workspace entry point, pwp_prune_layer, within the parity tolerances the
-other GPU tests use.  The file name sorts after the other small-case files, so a run
-that stops at the first failure has already run them (only the benchmark-sized cases,
-ordered last of all, come after it)."""
+other GPU tests use.  The file name sorts after the other plain parity files, so a run
+that stops at the first failure has already run them."""
 import ctypes
 
 import numpy as np
