@@ -34,7 +34,7 @@ def test_full_size_workload(name):
     torch = _torch()
     import post_weight_pruning_b200 as pwp
     wl = synth.workload(name)
-    W, X = synth.make_W(wl), synth.make_X_tokens(wl)
+    W, X = synth.make_W(wl), synth.make_X_tokens(wl, threads=max(1, min(16, os.cpu_count() or 1)))
     Wt, Xt = P.torch_inputs(W, X, wl.dtype)
     g = F.column_norms_sq(X, wl.dtype)
 
