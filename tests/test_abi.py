@@ -115,3 +115,16 @@ def test_pack24_argument_errors():
     assert L.pwp_pack_24(fake, fake, 0, 8, fake, fake, fake, None) == 1            # c < 1
     assert L.pwp_pack_24(vp((1 << 20) + 4), fake, 4, 8, fake, fake, fake, None) == 1   # W-hat not 16-byte aligned
     assert L.pwp_pack_24(fake, vp((1 << 20) + 2), 4, 8, fake, fake, fake, None) == 1   # mask not 4-byte aligned
+
+
+@pytest.mark.parametrize("c,b,B,method,mib", [
+    (4096, 4096, 128, "thanos", 201.8), (4096, 4096, 128, "sparsegpt", 29.1), (4096, 4096, 128, "wanda", 1.0),
+    (4096, 4096, 128, "magnitude", 1.0), (256, 512, 128, "thanos", 10.2), (1024, 1024, 64, "thanos", 12.5),
+    (1024, 1024, 128, "thanos", 33.5),
+])
+def test_workspace_sizes_match_the_documented_figures(c, b, B, method, mib):
+    import post_weight_pruning_b200 as pwp
+    n = pwp.workspace_bytes(pwp.config(method=method, block=B), c, b)
+    assert round(n / 2**20, 1) == mib
+    # the no-workspace entry point takes every shape whose workspace fits its 16 MiB array
+    assert (n <= 16 * 2**20) == (mib <= 16.0)
