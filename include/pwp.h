@@ -180,6 +180,8 @@ pwp_status pwp_pack_24(const float* W_hat_dev, const uint8_t* mask_dev, int32_t 
  *   more scratch than PWP_NOALLOC_SCRATCH_BYTES (pwp_workspace_bytes tells how much).
  *   The first call on each device looks up the array's device address (with that
  *   device current); make that first call before capturing any stream into a graph.
+ *   After cudaDeviceReset the next call looks the address up again (the lookup is
+ *   keyed by the context), so it must again come before any capture.
  *   Nothing is allocated or freed.  All calls share the one array: calls whose work
  *   overlaps on the GPU (different streams, or threads without ordering) race and give
  *   wrong results; order them. */
@@ -206,6 +208,15 @@ typedef enum {
     PWP_K_COLNORM = 6    /* Wanda from X: the column norms of X */
 } pwp_kernel_class;
 int64_t pwp_kernel_launches(void);
+/* pwp_set_wait_limit(polls): every bounded device-side wait of the tensor-core kernels
+ *   (an mbarrier wait between the copy, MMA and epilogue roles of one CTA) gives up after
+ *   this many polls and the call reports PWP_ETIMEOUT in stats (status_site names the
+ *   kernel).  Applies to kernels enqueued after the call; polls < 0 restores the default
+ *   (2^26); 0 makes every such wait give up at once, which lets a test drive the timeout
+ *   paths without any fault.  Copies and MMAs already in flight are always waited for
+ *   with the default limit before a CTA leaves.  Returns the previous limit.  Process-wide,
+ *   not tied to a stream: set it only while no other thread enqueues library work. */
+int64_t pwp_set_wait_limit(int64_t polls);
 int32_t pwp_profile_enable(int32_t which, int32_t capacity);
 int32_t pwp_profile_read(float* ms_out, int32_t cap);
 

@@ -234,14 +234,19 @@ def recon_loss(W: np.ndarray, What: np.ndarray, G: np.ndarray) -> float:
 # ----------------------------------------------------------------------------- the layer
 
 def prune_layer(W, *, Xt=None, H=None, sparsity=0.5, pattern="unstructured", nm=(2, 4),
-                block=128, damp=0.01, method="thanos", mode="factored", rows=None):
+                block=128, damp=0.01, method="thanos", mode="factored", rows=None, fixed_mask=None):
     """Prune one linear layer.
 
     W: c x b weights (any float dtype, widened exactly to fp64).  Xt: [n, b]
     token-major activations, or H: the undamped 2XX^T (b x b).  ``rows``: optional
     subset of rows of W to process -- valid only where rows do not interact (N:M
     patterns and the per-row work of a fixed mask); the unstructured global budget
-    couples all rows and needs every row.
+    couples all rows and needs every row.  ``fixed_mask``: optional c x b boolean mask
+    (for the processed rows) used as every block's selection instead of choosing one
+    (Thanos only).  Once the masks are given the rows do not interact -- the loss is a sum
+    of per-row terms ([THANOS] "The layer-reconstruction lens") and each row's update
+    depends only on its own selected set ([THANOS] "Contribution one") -- so any subset of
+    rows of a layer pruned elsewhere can be replayed exactly, also under the global budget.
 
     Thanos (method="thanos"), per block J = [j, j+B) with active region A = [j, b):
       1. K = inv(H_d[A, A]) (mode "definitional") or K[J, A] = U[J,J]^T U[J,A] with
@@ -277,8 +282,13 @@ def prune_layer(W, *, Xt=None, H=None, sparsity=0.5, pattern="unstructured", nm=
     if not unstructured:
         n_keep, m_grp = nm
         assert b % m_grp == 0 and B % m_grp == 0
-    if unstructured and method == "thanos" and rows is not None:
+    if unstructured and method == "thanos" and rows is not None and fixed_mask is None:
         raise ValueError("the global budget couples rows; a row subset is not defined")
+    if fixed_mask is not None:
+        if method != "thanos":
+            raise ValueError("fixed_mask replays Thanos row updates only")
+        fixed_mask = np.asarray(fixed_mask, dtype=bool)
+        assert fixed_mask.shape == (c, b)
 
     What = W0.copy()
     mask = np.zeros((c, b), dtype=bool)
@@ -298,7 +308,10 @@ def prune_layer(W, *, Xt=None, H=None, sparsity=0.5, pattern="unstructured", nm=
                 K_JA = U[j:j1, j:j1].T @ U[j:j1, j:]
             else:
                 K_JA = active_inverse(Hd, j)[:nJ, :]
-            if unstructured:
+            if fixed_mask is not None:
+                M = fixed_mask[:, j:j1]
+                dscore[:, j:j1] = wanda_scores(What[:, j:j1], g_diag[j:j1])
+            elif unstructured:
                 S = wanda_scores(What[:, j:], g_diag[j:])
                 r = zstar - pruned
                 take = min(r, c * (b - j))

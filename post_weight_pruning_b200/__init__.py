@@ -20,7 +20,7 @@ import numpy as np
 __all__ = [
     "lib", "Config", "Stats", "THANOS", "SPARSEGPT", "WANDA", "MAGNITUDE", "UNSTRUCTURED", "NM", "BF16", "FP32",
     "PwpError", "config", "workspace_bytes", "hessian_accumulate", "damp_factor", "prune_layer",
-    "prune_layer_host", "prune_block", "pack_24", "status_string", "LIB_PATH",
+    "prune_layer_host", "prune_block", "pack_24", "status_string", "set_wait_limit", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpwp.so")
@@ -63,6 +63,7 @@ _SIGS = {
                                  _vp, _vp, _vp, _sz, _vp, _vp]),
     "pwp_pack_24": (_i32, [_vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp]),
     "pwp_status_string": (ctypes.c_char_p, [_i32]),
+    "pwp_set_wait_limit": (_i64, [_i64]),
     "pwp_version": (_i32, []),
 }
 
@@ -84,6 +85,12 @@ def lib():
 
 def status_string(s) -> str:
     return lib().pwp_status_string(int(s)).decode()
+
+
+def set_wait_limit(polls: int) -> int:
+    """Polls every bounded device-side wait of the tensor-core kernels makes before it
+    gives up with PWP_ETIMEOUT (negative: the default, 2^26).  Returns the previous limit."""
+    return int(lib().pwp_set_wait_limit(int(polls)))
 
 
 def _check(status, where):

@@ -11,6 +11,8 @@
 // array is part of the loaded module, so every GPU on which the library is used holds
 // PWP_NOALLOC_SCRATCH_BYTES of it until the process exits.  No call here allocates or
 // frees memory; the kernels are the same ones pwp_prune_layer launches.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "pwp_internal.cuh"
@@ -30,20 +32,50 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[PWP_NOALLOC_SCR
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_scratch_addr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};   // id of the context the address belongs to
+
+// Unique id of the calling thread's current context (0 if there is none yet, or if the
+// driver does not provide the calls).  Ids are never reused within a process, so a
+// context created after cudaDeviceReset differs.  The two driver calls are reached through
+// the runtime's entry-point lookup, so the library does not link the driver library.
+unsigned long long current_context_id() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static const GetCurrent get_current = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    return (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess) ? reinterpret_cast<GetCurrent>(p) : (GetCurrent) nullptr;
+  }();
+  static const GetId get_id = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    return (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess) ? reinterpret_cast<GetId>(p) : (GetId) nullptr;
+  }();
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 // The host-side name g_noalloc_scratch is only a stand-in for the symbol, not a device
-// address: the device address is looked up once per device, with that device current.
+// address: the device address is looked up with the device current, once per device and
+// context (again after a device reset, whose new context reloads the module).
 cudaError_t scratch_for_current_device(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_addr[dev]) {
+  const unsigned long long id = current_context_id();
+  if (!g_scratch_addr[dev] || id == 0 || id != g_scratch_ctx[dev]) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);   // also creates the context if needed
     if (e != cudaSuccess) return e;
     g_scratch_addr[dev] = p;
+    g_scratch_ctx[dev] = current_context_id();
   }
   *out = g_scratch_addr[dev];
   return cudaSuccess;

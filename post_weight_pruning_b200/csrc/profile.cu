@@ -7,8 +7,11 @@
 namespace pwp {
 
 std::atomic<long long> g_launches{0};
+constexpr long long kDefaultWaitLimit = 1ll << 26;
+std::atomic<long long> g_wait_limit{kDefaultWaitLimit};
 
 void count_launches(long long n) { g_launches += n; }
+long long wait_limit() { return g_wait_limit.load(); }
 
 namespace {
 struct Prof {
@@ -37,6 +40,10 @@ using namespace pwp;
 extern "C" {
 
 int64_t pwp_kernel_launches(void) { return g_launches.load(); }
+
+int64_t pwp_set_wait_limit(int64_t polls) {
+  return g_wait_limit.exchange(polls < 0 ? kDefaultWaitLimit : (long long)polls);
+}
 
 int32_t pwp_profile_enable(int32_t which, int32_t capacity) {
   for (auto e : g_prof.ev0) cudaEventDestroy(e);

@@ -397,12 +397,20 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
       target += (long long)((double)cfg->sparsity * (double)c * (double)min(B, b - t * B));
   }
   if (first_on_device(g_attr_done)) {
-    cudaFuncSetAttribute(stream_kernel<kWanda>, cudaFuncAttributeMaxDynamicSharedMemorySize, kHist1Bins * 4);
-    cudaFuncSetAttribute(stream_kernel<kObs>, cudaFuncAttributeMaxDynamicSharedMemorySize, kHist1Bins * 4);
-    cudaFuncSetAttribute(kmat_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kmat_smem_bytes(kMaxBlock));
+    cudaError_t e0 = cudaFuncSetAttribute(stream_kernel<kWanda>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          kHist1Bins * 4);
+    if (e0 == cudaSuccess)
+      e0 = cudaFuncSetAttribute(stream_kernel<kObs>, cudaFuncAttributeMaxDynamicSharedMemorySize, kHist1Bins * 4);
+    if (e0 == cudaSuccess)
+      e0 = cudaFuncSetAttribute(kmat_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kmat_smem_bytes(kMaxBlock));
     int dev = 0, nsm = kNumSM;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    if (e0 == cudaSuccess) e0 = cudaGetDevice(&dev);
+    if (e0 == cudaSuccess) e0 = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    if (e0 != cudaSuccess) {
+      g_attr_done.fetch_and(~(1ull << (dev & 63)));   // try again on the next call
+      return e0;
+    }
     g_nsm = nsm;
   }
   long long nl = 0;
@@ -411,8 +419,10 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
     ++nl;
   }
   init_ctl_kernel<<<1, 1, 0, s>>>(pb.ctl, zstar, st, target);
-  cudaMemsetAsync(pb.hist1, 0, sizeof(unsigned int) * kHist1Bins, s);
-  cudaMemsetAsync(pb.l2.pred, 0, sizeof(unsigned int) * (2 * kHist2Bins + 2 * kHist2SumBins + kMaxBlock), s);
+  cudaError_t em = cudaMemsetAsync(pb.hist1, 0, sizeof(unsigned int) * kHist1Bins, s);
+  if (em == cudaSuccess)
+    em = cudaMemsetAsync(pb.l2.pred, 0, sizeof(unsigned int) * (2 * kHist2Bins + 2 * kHist2SumBins + kMaxBlock), s);
+  if (em != cudaSuccess) return em;
   convert_w_kernel<<<4 * g_nsm.load(), 256, 0, s>>>(W, wtype, Wout, N);
   nl += 2;
   prof_begin(kKFactor, s);

@@ -155,6 +155,8 @@ enum KernelClass { kKHessian = 0, kKFactor = 1, kKStream = 2, kKSelect = 3, kKSo
 void prof_begin(int which, cudaStream_t s);
 void prof_end(int which, cudaStream_t s);
 void count_launches(long long n);
+// Polls every ordinary bounded device-side wait makes before giving up (pwp_set_wait_limit).
+long long wait_limit();
 
 // ---------------------------------------------------------------- launchers (host side)
 cudaError_t launch_hessian(const void* X, int xtype, long long n, int b, float* H, int beta,

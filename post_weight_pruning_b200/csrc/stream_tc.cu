@@ -31,7 +31,8 @@
 //     half back with TMA.
 // Every wait is bounded; a wait that runs out records PWP_ETIMEOUT, the other roles stop
 // at their next wait, and the epilogue warps take each stop decision together through a
-// reducing barrier.
+// reducing barrier.  Copies and MMAs already in flight are always waited for before the
+// CTA leaves.
 #include "tc_common.cuh"
 
 namespace pwp {
@@ -92,7 +93,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __grid_constant__ CUtensorMap mw, int c, int b, int u0, int j, int Bp, int upper,
                      const uint8_t* __restrict__ mask, const float* __restrict__ sc, int hist_end,
                      unsigned int* __restrict__ hist1, const Ctl* __restrict__ ctl, unsigned int* __restrict__ h2,
-                     unsigned int* __restrict__ h2s, pwp_stats* st) {
+                     unsigned int* __restrict__ h2s, pwp_stats* st, long long spin) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* wbuf = smem + W_OFF;
@@ -152,7 +153,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tile_origin(tile, mt, u0, upper, m0, n0);
         for (int kc = 0; kc < nkc; ++kc) {
           const int s = it % STAGES;
-          if (it >= STAGES && !mbar_wait(&empty[s], ((it / STAGES) - 1) & 1, abortp)) {
+          if (it >= STAGES && !mbar_wait(&empty[s], ((it / STAGES) - 1) & 1, abortp, spin)) {
             ok = false;
             break;
           }
@@ -165,11 +166,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++it;
         }
       }
-      if (!ok) {
-        *abortp = 1;
-        // the copies already issued land before the CTA leaves
-        for (int k = it - STAGES > 0 ? it - STAGES : 0; k < it; ++k) mbar_wait(&full[k % STAGES], (k / STAGES) & 1);
-      }
+      if (!ok) *abortp = 1;
+      // every copy issued lands before the CTA leaves (already true unless a role gave up)
+      for (int k = it - STAGES > 0 ? it - STAGES : 0; k < it; ++k)
+        mbar_wait(&full[k % STAGES], (k / STAGES) & 1, kDrainLimit);
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
@@ -179,7 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tc) {
         const int acc = tc & 1;
-        if (tc >= 2 && !mbar_wait(&tempty[acc], ((tc >> 1) - 1) & 1, abortp)) {
+        if (tc >= 2 && !mbar_wait(&tempty[acc], ((tc >> 1) - 1) & 1, abortp, spin)) {
           ok = false;
           break;
         }
@@ -187,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d = tmem + (uint32_t)(acc * TN);
         for (int kc = 0; kc < nkc; ++kc) {
           const int s = it % STAGES;
-          if (!mbar_wait(&full[s], (it / STAGES) & 1, abortp)) {
+          if (!mbar_wait(&full[s], (it / STAGES) & 1, abortp, spin)) {
             ok = false;
             break;
           }
@@ -211,11 +211,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         mma_commit(&tfull[acc]);
       }
-      if (!ok) {
-        *abortp = 1;
-        mma_commit(drain);  // completes once every MMA issued so far has finished
-        mbar_wait(drain, 0);
-      }
+      if (!ok) *abortp = 1;
+      mma_commit(drain);  // completes once every MMA issued so far has finished
+      mbar_wait(drain, 0, kDrainLimit);
     }
     __syncwarp();
   } else if (warp == kWLoadWarp) {
@@ -227,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int m0, n0;
         tile_origin(tile, mt, u0, upper, m0, n0);
         for (int h = 0; h < 2; ++h) {
-          if (tc >= 1 && !mbar_wait(&wfree[h], (tc - 1) & 1, abortp)) {
+          if (tc >= 1 && !mbar_wait(&wfree[h], (tc - 1) & 1, abortp, spin)) {
             ok = false;
             break;
           }
@@ -238,10 +236,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++issued;
         }
       }
-      if (!ok) {
-        *abortp = 1;
-        for (int k = issued - 2 > 0 ? issued - 2 : 0; k < issued; ++k) mbar_wait(&wfull[k & 1], (k >> 1) & 1);
-      }
+      if (!ok) *abortp = 1;
+      // the last loads of W land before the CTA leaves, whether or not they were used
+      for (int k = issued - 2 > 0 ? issued - 2 : 0; k < issued; ++k)
+        mbar_wait(&wfull[k & 1], (k >> 1) & 1, kDrainLimit);
     }
     __syncwarp();
   } else {
@@ -256,10 +254,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tile_origin(tile, mt, u0, upper, m0, n0);
       const int r = m0 + rl;
       const bool row_ok = r < c;
-      bool ok = mbar_wait(&tfull[acc], (tc >> 1) & 1, abortp);
+      bool ok = mbar_wait(&tfull[acc], (tc >> 1) & 1, abortp, spin);
       bool stop = false;
       for (int h = 0; h < 2; ++h) {
-        ok = ok && mbar_wait(&wfull[h], tc & 1, abortp);
+        ok = ok && mbar_wait(&wfull[h], tc & 1, abortp, spin);
         ok = __all_sync(0xffffffffu, ok);
         if (ok) {
           fence_after();
@@ -392,7 +390,7 @@ cudaError_t launch_variant(const CUtensorMap* maps, int c, int b, int u0, int j,
   const int grid = ntiles < nsm ? ntiles : nsm;
   stream_tc_kernel<SCORE><<<grid, kThreads, SMEM_BYTES, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4], c, b, u0,
                                                              j, Bp, upper, mask, sc, hist_end, hist1, ctl, l2.pred,
-                                                             l2.pred_sum, st);
+                                                             l2.pred_sum, st, wait_limit());
   return cudaGetLastError();
 }
 

@@ -10,8 +10,13 @@
 namespace pwp {
 namespace tc {
 
-// Upper bound on the polls of one mbarrier wait; a wait that runs out reports failure.
-constexpr long long kSpinLimit = 1ll << 26;
+// Polls of one mbarrier wait before it gives up.  The ordinary waits of a kernel take
+// their limit from a launch parameter (pwp_set_wait_limit; kDefaultSpinLimit unless a
+// caller changed it); the waits that only let copies or MMAs already in flight finish
+// before a CTA leaves always use kDrainLimit, so that a shortened limit can never let a
+// CTA exit with asynchronous work still writing its shared or tensor memory.
+constexpr long long kDefaultSpinLimit = 1ll << 26;
+constexpr long long kDrainLimit = 1ll << 26;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -43,15 +48,16 @@ __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase of the given parity to complete.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (long long i = 0; i < kSpinLimit; ++i)
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit) {
+  for (long long i = 0; i < limit; ++i)
     if (mbar_try(bar, parity)) return true;
   return false;
 }
 
 // Bounded wait that also gives up as soon as another role of the CTA raised *abort.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort) {
-  for (long long i = 0; i < kSpinLimit; ++i) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort,
+                                          long long limit) {
+  for (long long i = 0; i < limit; ++i) {
     if (mbar_try(bar, parity)) return true;
     if ((i & 63) == 63 && *abort) return false;
   }

@@ -47,6 +47,7 @@ def compare(W_store, dtype, gpu, orc, *, pattern, nm, block, tie_tol):
     c, b = Wo.shape
     dis = np.argwhere(mask != Mo)
     tie_ok = np.zeros(len(dis), dtype=bool)
+    gaps = np.zeros(len(dis))
     if pattern == "unstructured":
         thr = {}
         for blk in orc["blocks"]:
@@ -54,15 +55,18 @@ def compare(W_store, dtype, gpu, orc, *, pattern, nm, block, tie_tol):
         for i, (k, q) in enumerate(dis):
             j = (q // block) * block
             t = thr[j]
-            tie_ok[i] = abs(orc["dscore"][k, q] - t) <= tie_tol * max(abs(t), 1e-300)
+            gaps[i] = abs(orc["dscore"][k, q] - t) / max(abs(t), 1e-300)
+            tie_ok[i] = gaps[i] <= tie_tol
     else:
         m = nm[1]
         for i, (k, q) in enumerate(dis):
-            tie_ok[i] = orc["nm_gap"][k, q // m] <= tie_tol
+            gaps[i] = orc["nm_gap"][k, q // m]
+            tie_ok[i] = gaps[i] <= tie_tol
     res = {
         "agree": 1.0 - len(dis) / (c * b),
         "n_dis": int(len(dis)),
         "n_dis_not_tie": int((~tie_ok).sum()),
+        "dis_gaps": sorted(gaps.tolist())[-8:],       # the largest relative score gaps that flipped
         "w_rel": float(np.linalg.norm(W_hat - Wo) / np.linalg.norm(Wo)),
         "zeros_exact": bool(np.all(W_hat[mask] == 0.0)),
         "n_mask": int(mask.sum()),

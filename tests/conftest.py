@@ -18,7 +18,10 @@ def pytest_collection_modifyitems(session, config, items):
     # Plain parity cases first, then the checks built on them, then the benchmark-sized
     # cases (the longest, and the largest allocations): a run stopped at the first failure
     # has still reported everything before it.
+    # The no-workspace entry point's test file (test_zz_*) goes after everything else.
     def rank(it):
+        if os.path.basename(str(it.fspath)).startswith("test_zz_"):
+            return 3
         if it.get_closest_marker("fullsize") is not None:
             return 2
         return 1 if it.get_closest_marker("integration") is not None else 0

@@ -128,3 +128,12 @@ def test_workspace_sizes_match_the_documented_figures(c, b, B, method, mib):
     assert round(n / 2**20, 1) == mib
     # the no-workspace entry point takes every shape whose workspace fits its 16 MiB array
     assert (n <= 16 * 2**20) == (mib <= 16.0)
+
+
+def test_wait_limit_setter_returns_the_previous_limit_and_restores_the_default():
+    default = 1 << 26
+    assert pwp.set_wait_limit(-1) == default          # untouched so far in this process
+    assert pwp.set_wait_limit(0) == default
+    assert pwp.set_wait_limit(12345) == 0
+    assert pwp.set_wait_limit(-5) == 12345
+    assert pwp.set_wait_limit(-1) == default

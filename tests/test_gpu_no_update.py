@@ -12,7 +12,8 @@ from tests import _parity as P
 
 pytestmark = pytest.mark.gpu
 
-TIE_TOL = 2e-5
+# score ties within 1e-6 relative: the stated bar for mask disagreements
+TIE_TOL = 1e-6
 
 
 def _torch():

@@ -514,3 +514,48 @@ def test_dead_features_go_first_and_undamped_singular_h_is_refused():
     assert r["pruned"] == 64
     with pytest.raises(np.linalg.LinAlgError):
         oracle.prune_layer(W, Xt=Xt, sparsity=0.5, block=16, damp=0.0)
+
+
+# --------------------------------------------------------------------------- fixed-mask replay
+
+def test_fixed_mask_replay_equals_sequential_least_squares():
+    """Replaying a given mask over three blocks equals, block after block, the brute-force
+    constrained least squares on [sqrt(2) X^T; sqrt(lambda) I] over that block's active
+    region with the block's selected weights forced to 0 and earlier columns frozen."""
+    W, Xt = _rand_problem(41, c=2, b=12, n=30)
+    damp = 0.03
+    B = 4
+    H = oracle.hessian(Xt)
+    _, lam = oracle.damp_hessian(H, damp)
+    mask = np.zeros((2, 12), dtype=bool)
+    mask[0, [1, 2, 5, 9, 10]] = True
+    mask[1, [0, 7, 11]] = True
+    r = oracle.prune_layer(W, H=H, block=B, damp=damp, fixed_mask=mask)
+    for k in range(2):
+        w = W[k].copy()
+        for j in range(0, 12, B):
+            Q = np.flatnonzero(mask[k, j:j + B]) + j
+            if Q.size:
+                w = _lstsq_row(w, Xt, lam, j, Q)
+        assert np.allclose(r["W"][k], w, rtol=1e-9, atol=1e-11)
+    assert np.array_equal(r["mask"], mask)
+
+
+@pytest.mark.parametrize("pattern,nm", [("unstructured", (0, 0)), ("nm", (2, 4))])
+def test_fixed_mask_replay_reproduces_full_runs_on_row_subsets(pattern, nm):
+    """With the full run's own mask given, every row -- and any subset of rows, also under
+    the global budget that couples them through the selection -- comes out as in the full
+    run, in both the factored and the definitional mode."""
+    rng = np.random.default_rng(17)
+    Xt = rng.normal(size=(60, 24))
+    Xt[:, 5] *= 9.0
+    W = rng.normal(0, 0.02, size=(10, 24))
+    for mode in ("factored", "definitional"):
+        full = oracle.prune_layer(W, Xt=Xt, sparsity=0.5, pattern=pattern, nm=nm, block=8, mode=mode)
+        again = oracle.prune_layer(W, Xt=Xt, block=8, mode=mode, fixed_mask=full["mask"])
+        assert np.allclose(again["W"], full["W"], rtol=1e-12, atol=1e-15)
+        rows = np.array([1, 4, 8])
+        sub = oracle.prune_layer(W, Xt=Xt, block=8, mode=mode, rows=rows, fixed_mask=full["mask"][rows])
+        assert np.allclose(sub["W"], full["W"][rows], rtol=1e-12, atol=1e-15)
+        assert np.isclose(sub["loss"], float(np.sum(oracle.row_losses(W[rows], full["W"][rows],
+                                                                         0.5 * oracle.hessian(Xt)))))
