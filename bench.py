@@ -19,6 +19,7 @@ import argparse
 import ctypes
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -164,13 +165,67 @@ def algorithmic_work(cls, wl, per_launch_ms, mask=None, method="thanos"):
         steps = max(1, len(per_launch_ms) // nblk)
         return total * steps, "byte", "hbm"
     if cls == K_SOLVE:
-        m = mask.reshape(c, nblk, B).sum(axis=2).astype(np.float64)   # s per row per block
-        flops = float(np.sum(m ** 3 / 3.0 + 2.0 * m ** 2 + 4.0 * m * B))
+        flops = solve_flops(wl, mask)
         steps = max(1, len(per_launch_ms) // nblk)
         return flops * steps, "flop", "alu"
     if cls == K_FACTOR:
         return 2.0 * b ** 3 / 3.0 * len(per_launch_ms), "flop", "alu"
     raise ValueError(cls)
+
+
+def solve_flops(wl, mask):
+    """Per-row solve arithmetic of one layer: sum over rows and blocks of s^3/3 + 2 s^2 (the
+    Cholesky of the s x s system and its two triangular solves), s = the row's removals in
+    the block."""
+    c, b, B = wl.c, wl.b, wl.block
+    nblk = (b + B - 1) // B
+    pad = nblk * B - b
+    m = np.pad(np.asarray(mask, dtype=np.uint8), ((0, 0), (0, pad))) if pad else np.asarray(mask, dtype=np.uint8)
+    s = m.reshape(c, nblk, B).sum(axis=2).astype(np.float64)
+    return float(np.sum(s ** 3 / 3.0 + 2.0 * s ** 2))
+
+
+def block_phase_bytes(wl):
+    """Algorithmic HBM bytes of the block prune phase: the fp32 active region read and
+    written once per block, the block's rows of the inverse over it, and W (bf16) in plus
+    W-hat (fp32) and the mask out."""
+    c, b, B = wl.c, wl.b, wl.block
+    act = sum(b - j for j in range(0, b, B))
+    return 8.0 * c * act + 4.0 * B * sum(b - j for j in range(B, b, B)) + 7.0 * c * b
+
+
+def phase_rooflines(wl, phase_ms, mask, peaks):
+    """Roofline fraction of each phase from its CUDA-event time and its algorithmic work."""
+    c, b, n, B = wl.c, wl.b, wl.n, wl.block
+    mhz = peaks["sm_max_mhz"]
+    alu = fp32_alu_peak_tflops(mhz)
+    tf32 = peaks["bf16_tflops"] * 1.1 / 2.25          # nominal tf32 : bf16 dense ratio
+    out = {}
+
+    def put(name, ms, work, unit, bound, peak, note):
+        if ms is None or ms <= 0:
+            return
+        per_s = work / (ms / 1e3)
+        ach = per_s / (1e9 if unit == "GB/s" else 1e12)
+        out[name] = {"ms": ms, "bound": bound, "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak,
+                     "work": note}
+    h = phase_ms.get("hessian_xxt")
+    put("hessian_xxt", h, float(b) * b * n, "TFLOP/s", "tensor", peaks["bf16_tflops"],
+        "b^2 n flops (symmetric half of 2 b^2 n), bf16 operands")
+    put("factor", phase_ms.get("factor"), 2.0 * b ** 3 / 3.0, "TFLOP/s", "alu", alu, "2 b^3 / 3 flops")
+    st = phase_ms.get("stream_update_score")
+    upd_flops = sum(2.0 * c * min(B, b - j) * (b - j) for j in range(0, b, B))
+    stream_bytes = sum(8.0 * c * (b - j) + (4.0 * B * (b - j) if j > 0 else 0.0) for j in range(0, b, B))
+    put("trailing_update_tensor", st, upd_flops, "TFLOP/s", "tensor", tf32,
+        "2 c B (b - j) flops per block (3xTF32 on the tensor cores; peak = measured bf16 x 1.1/2.25)")
+    put("stream_update_score", st, stream_bytes, "GB/s", "hbm", peaks["hbm_gbs"],
+        "8 c (b - j) + 4 B (b - j) bytes per block")
+    put("row_solve", phase_ms.get("row_solve"), solve_flops(wl, mask), "TFLOP/s", "alu", alu,
+        "sum of s^3/3 + 2 s^2 over rows and blocks")
+    blk = sum(phase_ms.get(k, 0.0) for k in ("stream_update_score", "select", "row_solve"))
+    put("block_phase", blk, block_phase_bytes(wl), "GB/s", "hbm", peaks["hbm_gbs"],
+        "8 c sum(b - j) + 4 B sum(b - j) + 7 c b bytes; time = update + select + solves")
+    return out
 
 
 def job_throughput(local_ms, world, weights_per_step, steps, device=None):
@@ -193,30 +248,65 @@ def fp32_alu_peak_tflops(sm_mhz):
 
 # ------------------------------------------------------------------------------ CPU oracle
 
-def cpu_oracle_sample(wl, W_store, X_store, rows, method="thanos"):
-    import oracle
-    import synth
+def _oracle_threads():
     try:
         from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+        return int(max([i.get("num_threads", 1) for i in threadpool_info()] or [1]))
     except Exception:
-        threads = os.cpu_count()
-    W64 = synth.to_f64(W_store[:rows], wl.dtype)
+        return int(os.cpu_count() or 1)
+
+
+def cpu_oracle_full(wl, W_store, X_store, method="thanos"):
+    """The fp64 oracle on the whole benchmarked layer, timed once: the same problem the GPU
+    solves (the global budget couples every row, so no row subset is the same problem)."""
+    import oracle
+    import synth
+    W64 = synth.to_f64(W_store, wl.dtype)
     t0 = time.perf_counter()
     X64 = synth.to_f64(X_store, wl.dtype)
     s32 = float(np.float32(wl.sparsity))
     if method in SECOND_ORDER:
         r = oracle.prune_layer(W64, Xt=X64, sparsity=s32, block=wl.block, damp=wl.damp, method=method,
                                pattern="unstructured")
-        what = f"full H from all {wl.n} tokens, full factor, all {(wl.b + wl.block - 1) // wl.block} blocks"
+        what = f"H from all {wl.n} tokens, the factor, all {(wl.b + wl.block - 1) // wl.block} blocks"
     else:
         r = oracle.prune_no_update(W64, Xt=X64, sparsity=s32, method=method)
         what = f"norms from all {wl.n} tokens" if method == "wanda" else "no activations"
     dt = time.perf_counter() - t0
     assert r["pruned"] == r.get("zstar", r.get("target"))
-    return {"value": rows * wl.b / dt, "unit": UNIT, "cores": int(threads), "kind": "oracle",
-            "sample": (f"fp64 numpy oracle ({method}) on the {wl.name} workload restricted to its first "
-                       f"{rows} output rows: {what}; {dt:.1f} s for {rows}x{wl.b} weights")}
+    return {"value": wl.c * wl.b / dt, "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
+            "sample": (f"fp64 numpy oracle ({method}) on the whole {wl.name} layer ({wl.c}x{wl.b} weights): "
+                       f"{what}; one run, {dt:.1f} s")}
+
+
+def cpu_oracle_row_sample(wl, W_store, X64, rows, method="thanos"):
+    """A bounded sample of the same layer for the reference arm: the block sweep of the
+    first `rows` rows (their own budget at the layer's sparsity) with the layer's H and
+    factor, whose time is counted at rows/c because the whole layer shares them.  Returns
+    (counted seconds, description)."""
+    import oracle
+    import synth
+    W64 = synth.to_f64(W_store[:rows], wl.dtype)
+    s32 = float(np.float32(wl.sparsity))
+    if method not in SECOND_ORDER:
+        t0 = time.perf_counter()
+        oracle.prune_no_update(W64, Xt=X64, sparsity=s32, method=method)
+        dt = time.perf_counter() - t0
+        return dt, f"{rows} rows of the {wl.name} layer ({method}, norms from all {wl.n} tokens)"
+    t0 = time.perf_counter()
+    H = oracle.hessian(X64)
+    t1 = time.perf_counter()
+    Hd, _ = oracle.damp_hessian(H, wl.damp)
+    oracle.inverse_cholesky_upper(Hd)
+    t2 = time.perf_counter()
+    oracle.prune_layer(W64, H=H, sparsity=s32, block=wl.block, damp=wl.damp, method=method, pattern="unstructured")
+    t3 = time.perf_counter()
+    fixed = (t1 - t0) + (t2 - t1)            # H and the factor: once per layer
+    sweep = (t3 - t2) - (t2 - t1)            # prune_layer repeats the factor: take it out
+    counted = fixed * rows / wl.c + max(sweep, 0.0)
+    return counted, (f"{rows} of {wl.c} rows of the {wl.name} layer: the {method} sweep of those rows "
+                     f"(global budget at s={wl.sparsity} on the rows) plus {rows}/{wl.c} of the layer's H "
+                     f"({wl.n} tokens) and factor time")
 
 
 # ------------------------------------------------------------------------------ reference arm
@@ -229,23 +319,24 @@ def run_reference(args):
     wl = synth.workload(WORKLOAD)
     W = synth.make_W(wl)
     X = synth.make_X_tokens(wl)
-    rows = 128
+    X64 = synth.to_f64(X, wl.dtype)
+    rows = args.cpu_rows
     for _ in range(args.warmup):
-        cpu_oracle_sample(wl, W, X, rows, args.method)
-    times = []
+        cpu_oracle_row_sample(wl, W, X64, rows, args.method)
+    counted = []
+    what = ""
     for _ in range(args.steps):
-        t0 = time.perf_counter()
-        cb = cpu_oracle_sample(wl, W, X, rows, args.method)
-        times.append(time.perf_counter() - t0)
-    tot = sum(times)
+        dt, what = cpu_oracle_row_sample(wl, W, X64, rows, args.method)
+        counted.append(dt)
+    tot = sum(counted)
     value = rows * wl.b * args.steps / tot
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": _config(wl, args.method),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cb["cores"], "kind": "oracle",
-                         "sample": cb["sample"]},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
+                         "sample": what},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -425,13 +516,148 @@ def run_mine(args):
         if method in SECOND_ORDER:
             line["select_stats"] = {"blocks": nblk, "reread_blocks": int(st.reread_blocks),
                                     "tie_blocks": int(st.tie_blocks)}
+        if method in SECOND_ORDER:
+            if mask_np is None:
+                mask_np = mask.cpu().numpy()
+            line["phases"] = phase_rooflines(wl, phase_ms, mask_np, peaks)
+        if world == 1 and not args.no_extra_workloads and method == "thanos":
+            line["workloads"] = time_other_workloads(dev, args)
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_oracle_sample(wl, W_store, X_store, args.cpu_rows, method)
+            line["cpu_baseline"] = cpu_oracle_full(wl, W_store, X_store, method)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def _time_calls(fn, steps, warmup=1):
+    """Device time (ms) of fn() per call on the current stream, after warm-up; the L2 is
+    flushed before every call (the inputs of these workloads exceed it anyway)."""
+    import torch
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    ms = []
+    for i in range(steps):
+        flush.fill_(float(i))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    del flush
+    return ms
+
+
+def _device_block_inputs(dev, seed=0):
+    """The decoder block's activations drawn on the device (torch generator, seed 0) with the
+    host generator's distributions: Gaussian with 0.5% of features x50 (attention, o and MLP
+    inputs), Laplace(0, 1/sqrt 2) with 30% of entries x1e-2 (down_proj input); 128 x 2048
+    tokens each.  Only the timing uses these; the parity tests draw on the host."""
+    import torch
+    import synth
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    acts = {}
+    for inp, (b, dist, frac, scale, _) in synth.BLOCK_INPUTS.items():
+        n = synth.BLOCK_TOKENS
+        X = torch.empty((n, b), dtype=torch.bfloat16, device=dev)
+        cols = None
+        if frac > 0:
+            k = int(round(frac * b))
+            cols = torch.randperm(b, generator=g, device=dev)[:k]
+        for r0 in range(0, n, 16384):
+            r1 = min(n, r0 + 16384)
+            if dist == "gaussian":
+                x = torch.randn((r1 - r0, b), generator=g, device=dev)
+            else:
+                u = torch.rand((r1 - r0, b), generator=g, device=dev) - 0.5
+                x = -torch.sign(u) * torch.log1p(-2.0 * u.abs()) / math.sqrt(2.0)
+                near = torch.rand((r1 - r0, b), generator=g, device=dev) < 0.3
+                x = torch.where(near, x * 1e-2, x)
+            if cols is not None:
+                x[:, cols] *= scale
+            X[r0:r1] = x.to(torch.bfloat16)
+        acts[inp] = X
+    weights = {}
+    for l, (name, inp, c) in enumerate(synth.BLOCK_LAYERS):
+        b = synth.BLOCK_INPUTS[inp][0]
+        weights[name] = (torch.randn((c, b), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    feeds = {name: inp for name, inp, _ in synth.BLOCK_LAYERS}
+    return weights, acts, feeds
+
+
+def time_other_workloads(dev, args):
+    """Prune time of the other benchmark workloads on this GPU (CUDA events, L2 flushed):
+    the 11008x4096 layer at 2:4 and the 4096x11008 layer at 4:8 (32768 tokens; H build +
+    factor + sweep, with each phase's time) and the seven-layer decoder block (128 x 2048
+    tokens; four H builds and seven prunes through prune_block)."""
+    import torch
+    import synth
+    import post_weight_pruning_b200 as pwp
+    L = pwp.lib()
+    out = {}
+    threads = max(1, min(32, os.cpu_count() or 1))
+    for name in ("up_proj11008x4096_2of4", "down_proj4096x11008_4of8"):
+        wl = synth.workload(name)
+        W_store, X_store = synth.make_W(wl), synth.make_X_tokens(wl, threads=threads)
+        Wt, Xt = pwp.from_bf16_bits(W_store, dev), pwp.from_bf16_bits(X_store, dev)
+        del X_store
+        kw = dict(method="thanos", pattern="nm", nm=wl.nm, sparsity=wl.sparsity, block=wl.block, damp=wl.damp)
+        ws = pwp.make_workspace(pwp.config(**kw), wl.c, wl.b, dev)
+        H = torch.empty((wl.b, wl.b), dtype=torch.float32, device=dev)
+        W_out = torch.empty((wl.c, wl.b), dtype=torch.float32, device=dev)
+        mask = torch.empty((wl.c, wl.b), dtype=torch.uint8, device=dev)
+        stats = pwp.new_stats(dev)
+
+        def call():
+            pwp.prune_layer(Wt, X=Xt, H=H, W_out=W_out, mask=mask, workspace=ws, stats=stats, check=False, **kw)
+        ms = _time_calls(call, steps=3)
+        nblk = (wl.b + wl.block - 1) // wl.block
+        per_class = {K_HESSIAN: 1, K_FACTOR: 1, K_STREAM: nblk, K_SELECT: nblk, K_SOLVE: nblk}
+        phases = {}
+        for cls, cnt in per_class.items():
+            L.pwp_profile_enable(cls, cnt)
+            call()
+            buf = (ctypes.c_float * cnt)()
+            n = L.pwp_profile_read(buf, cnt)
+            phases[CLASS_NAMES[cls]] = float(sum(buf[:n]))
+        L.pwp_profile_enable(-1, 0)
+        st = pwp.read_stats(stats)
+        if st.status != 0 or st.pruned != st.target:
+            raise RuntimeError(f"{name}: status {st.status}")
+        t = statistics.median(ms)
+        out[name] = {"ms": t, "weights_per_s": wl.c * wl.b / (t / 1e3), "steps": len(ms),
+                     "config": f"W {wl.c}x{wl.b} bf16, X {wl.n}x{wl.b} bf16 ({wl.x_dist}), Thanos "
+                               f"{wl.nm[0]}:{wl.nm[1]}, B={wl.block}, damp={wl.damp}",
+                     "phases_ms": phases}
+        del Wt, Xt, ws, H, W_out, mask
+        torch.cuda.empty_cache()
+
+    weights, acts, feeds = _device_block_inputs(dev)
+    res = {}
+
+    def block():
+        res.update(pwp.prune_block(weights, acts, feeds, method="thanos", pattern="unstructured", sparsity=0.5,
+                                   block=128, damp=0.01, check=False))
+    ms = _time_calls(block, steps=2)
+    for layer, (_, _, st_t) in res.items():
+        st = pwp.read_stats(st_t)
+        if st.status != 0 or st.pruned != st.target:
+            raise RuntimeError(f"decoder block {layer}: status {st.status}")
+    total = sum(int(w.numel()) for w in weights.values())
+    t = statistics.median(ms)
+    out["decoder_block"] = {"ms": t, "weights_per_s": total / (t / 1e3), "steps": len(ms),
+                            "config": ("q,k,v,o 4096x4096; gate,up 11008x4096; down 4096x11008 bf16; 128x2048 "
+                                       "tokens per input drawn on the device; Thanos 50% unstructured global budget "
+                                       "per layer, B=128; one H per input (4 builds), 7 prunes")}
+    del weights, acts, res
+    torch.cuda.empty_cache()
+    return out
 
 
 def main():
@@ -441,7 +667,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-rows", type=int, default=256)
+    ap.add_argument("--cpu-rows", type=int, default=256,
+                    help="rows of the reference arm's per-step sample")
+    ap.add_argument("--no-extra-workloads", action="store_true",
+                    help="skip the timing of the 2:4, 4:8 and decoder-block workloads")
     ap.add_argument("--method", default="thanos", choices=["thanos", "sparsegpt", "wanda", "magnitude"],
                     help="pruning method timed on the q_proj workload (default: thanos, the headline)")
     args = ap.parse_args()

@@ -243,7 +243,9 @@ def prune_layer(W, *, Xt=None, H=None, sparsity=0.5, pattern="unstructured", nm=
     patterns and the per-row work of a fixed mask); the unstructured global budget
     couples all rows and needs every row.  ``fixed_mask``: optional c x b boolean mask
     (for the processed rows) used as every block's selection instead of choosing one
-    (Thanos only).  Once the masks are given the rows do not interact -- the loss is a sum
+    (Thanos only; for the global budget over all rows, each block also records in
+    ``blocks`` the selection the budget loop would have made on the replayed state --
+    ``chosen``, with its residual count and thresholds).  Once the masks are given the rows do not interact -- the loss is a sum
     of per-row terms ([THANOS] "The layer-reconstruction lens") and each row's update
     depends only on its own selected set ([THANOS] "Contribution one") -- so any subset of
     rows of a layer pruned elsewhere can be replayed exactly, also under the global budget.
@@ -311,6 +313,13 @@ def prune_layer(W, *, Xt=None, H=None, sparsity=0.5, pattern="unstructured", nm=
             if fixed_mask is not None:
                 M = fixed_mask[:, j:j1]
                 dscore[:, j:j1] = wanda_scores(What[:, j:j1], g_diag[j:j1])
+                if unstructured and rows is None:
+                    # what step 3 of the budget loop would choose on this (replayed) state,
+                    # with the residual count left by the given mask's earlier blocks
+                    S = wanda_scores(What[:, j:], g_diag[j:])
+                    r = zstar - pruned
+                    chosen, t_last, t_next = lowest_global(S, j, min(max(r, 0), c * (b - j)))
+                    info.update(r=r, chosen=chosen[:, :nJ], t_last=t_last, t_next=t_next)
             elif unstructured:
                 S = wanda_scores(What[:, j:], g_diag[j:])
                 r = zstar - pruned

@@ -27,117 +27,172 @@ __host__ __device__ constexpr int poff(int i) {
   return 4 * (2 * (i >> 2) * ((i >> 2) + 1) + (i & 3) * ((i >> 2) + 1));
 }
 
-// Per warp: rows 0..NS-1 of the packed factor, the u/y vector and the selected indices in
-// shared memory; rows NS..SCAP-1 (only rows with more than NS selections reach them) in a
-// per-warp slot of global scratch.
-template <int SCAP, int NS>
-struct SolveSmem {
-  static constexpr int kL = poff(NS);
-  static constexpr int kY = SCAP + 4;
-  static constexpr int kPerWarp = kL + kY + SCAP;  // floats: L, y, Qidx
-  static constexpr int kGlobal = poff(SCAP) - poff(NS);   // floats of global scratch per warp
-};
+// Per warp: rows 0..kNS-1 of the packed factor, the u/y/z vector, the selected indices
+// (reused for the pivots' reciprocals) and the staged 8x8 diagonal block, in shared
+// memory; rows kNS..kCap-1 (only rows with more than kNS selections reach them) in a
+// per-warp slot of global scratch, which stays in L2.
+constexpr int kCap = kMaxBlock;      // largest selected set of a row
+constexpr int kNS = kSolveNS;        // factor rows kept in shared memory
+constexpr int kL = poff(kNS);
+constexpr int kY = kCap + 8;
+constexpr int kPerWarp = kL + kY + kCap + 64;        // floats: L, y, Qidx, D
+constexpr int kGlobalPerWarp = poff(kCap) - poff(kNS);
+constexpr int kSolveWarps = 8;
+static_assert(kL % 4 == 0 && kY % 4 == 0 && kCap % 4 == 0, "16-byte aligned regions");
 
-template <int NS>
+// Rows of the packed factor.  SMALL: every row lives in shared memory (s <= kNS), so all
+// pointers stay shared-memory pointers; otherwise rows from kNS on are in global scratch.
+template <bool SMALL>
 struct Rows {
-  float* L;   // shared, rows < NS
-  float* G;   // global, rows >= NS
-  __device__ __forceinline__ float* row(int i) const { return i < NS ? L + poff(i) : G + (poff(i) - poff(NS)); }
+  float* L;   // shared, rows < kNS
+  float* G;   // global, rows >= kNS
+  __device__ __forceinline__ float* row(int i) const {
+    if (SMALL) return L + poff(i);
+    return i < kNS ? L + poff(i) : G + (poff(i) - poff(kNS));
+  }
 };
 
-// Cholesky R-hat = L L^T (left-looking, 8-column panels; lanes own rows) with u carried
-// as an extra row so that the factorisation also gives y = L^-1 u, then L^T z = y.
-// L holds R-hat's lower triangle on entry; y holds u.  On return y[0..s) = z.
-// Per panel [jp, jp+8), the rows i in [jp, s] (s: the u row) go over the lanes in rounds
-// of 32: each takes the contributions of columns < jp (float4 dot products against the
-// eight panel rows), then in the first round the 8x8 diagonal block, held by lanes
-// 0..7, is factored with shuffles; every other row finishes its eight panel entries by
-// forward substitution.  A packed row i holds columns up to 4*(i/4)+3, so rows jp..jp+3
-// of a panel touch only its first four columns.  One __syncwarp per panel.  The
-// reciprocal of every diagonal entry goes to idg for the back substitution.  Returns
-// false on a non-positive pivot (uniform).
-template <int SCAP, int NS>
-__device__ bool chol_solve(const Rows<NS> R, float* __restrict__ y, float* __restrict__ idg, int s, int lane) {
+__device__ __forceinline__ float dot4(float4 a, float4 b, float acc) {
+  acc = fmaf(-a.x, b.x, acc);
+  acc = fmaf(-a.y, b.y, acc);
+  acc = fmaf(-a.z, b.z, acc);
+  return fmaf(-a.w, b.w, acc);
+}
+
+// acc[q][c] -= sum_{t < jp} row_q[t] * prow_c[t] for the NQ row slots of one pass.
+template <int NQ>
+__device__ __forceinline__ void panel_gemm(float (&acc)[2][8], const float* const (&rp)[2],
+                                           const float* const (&pr)[8], int jp) {
+#pragma unroll 1
+  for (int t = 0; t < jp; t += 4) {
+    float4 x[NQ];
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) x[q] = *reinterpret_cast<const float4*>(rp[q] + t);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const float4 p = *reinterpret_cast<const float4*>(pr[c] + t);
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) acc[q][c] = dot4(x[q], p, acc[q][c]);
+    }
+  }
+}
+
+// Cholesky R-hat = L L^T of the s x s gathered matrix (its lower triangle in R on entry,
+// L on return), left-looking over 8-column panels, with u carried as an extra row s so
+// that the same sweep gives y = L^-1 u; then the back substitution L^T z = y.  On return
+// y[0..s) = z.  Per panel [jp, jp+8) the rows i in [jp, s] go over the lanes, two rows per
+// lane and pass (lane l: rows jp+l+64p and jp+l+64p+32): each takes the contributions of
+// the columns before jp (float4 dot products with the eight panel rows, which every lane
+// reads as broadcasts), the panel's 8x8 diagonal block is staged in D and factored by every
+// lane alike (no shuffles; the pivots are uniform across the warp), and each row finishes
+// its eight panel entries by forward substitution.  A packed row i holds columns up to
+// 4*(i/4)+3, so rows jp..jp+3 of a panel store only its first four columns; columns beyond
+// i inside a row's padding are never read.  Reciprocal pivots go to idg for the back
+// substitution.  Returns false on a non-positive pivot (uniform).
+template <bool SMALL>
+__device__ bool chol_solve(const Rows<SMALL> R, float* __restrict__ y, float* __restrict__ idg,
+                           float* __restrict__ D, int s, int lane) {
   for (int jp = 0; jp < s; jp += 8) {
     const int pw = min(8, s - jp);
     const float* pr[8];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) pr[c] = R.row(jp + (c < pw ? c : 0));   // padding rows: any valid row
-    const int nr = (s - jp + 1 + 31) >> 5;
-    float Ld[8][8];
-    float il[8];
+    for (int c = 0; c < 8; ++c) pr[c] = R.row(jp + (c < pw ? c : 0));   // padding columns: any valid row
+    for (int pass = 0; jp + 64 * pass <= s; ++pass) {
+      const bool two = jp + 64 * pass + 32 <= s;   // uniform: some lane has a second row
+      int ii[2];
+      const float* rp[2];
+      float acc[2][8];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      il[c] = 1.f;
-#pragma unroll
-      for (int c2 = 0; c2 < 8; ++c2) Ld[c][c2] = 0.f;
-    }
-    for (int r = 0; r < nr; ++r) {
-      const int i = jp + lane + 32 * r;
-      float* ri = (i < s) ? R.row(i) : y;
-      const bool two = (i >= jp + 4) || (i >= s);   // the row holds panel columns jp+4..
-      float acc[8];
-      {
-        const float4 a = *reinterpret_cast<const float4*>(ri + jp);
-        acc[0] = a.x; acc[1] = a.y; acc[2] = a.z; acc[3] = a.w;
+      for (int q = 0; q < 2; ++q) {
+        const int i = jp + lane + 64 * pass + 32 * q;
+        ii[q] = i;
+        float* r = i < s ? R.row(i) : y;           // row s is the u row; rows past it are idle
+        rp[q] = r;
+        const bool hi = i >= jp + 4 || i >= s;     // the row's storage holds panel columns jp+4..
+        const float4 a = *reinterpret_cast<const float4*>(r + jp);
         float4 bq = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (two) bq = *reinterpret_cast<const float4*>(ri + jp + 4);
-        acc[4] = bq.x; acc[5] = bq.y; acc[6] = bq.z; acc[7] = bq.w;
+        if (hi) bq = *reinterpret_cast<const float4*>(r + jp + 4);
+        acc[q][0] = a.x; acc[q][1] = a.y; acc[q][2] = a.z; acc[q][3] = a.w;
+        acc[q][4] = bq.x; acc[q][5] = bq.y; acc[q][6] = bq.z; acc[q][7] = bq.w;
       }
-#pragma unroll 2
-      for (int t = 0; t < jp; t += 4) {
-        const float4 x = *reinterpret_cast<const float4*>(ri + t);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const float4 q = *reinterpret_cast<const float4*>(pr[c] + t);
-          float v = acc[c];
-          v = fmaf(-x.x, q.x, v);
-          v = fmaf(-x.y, q.y, v);
-          v = fmaf(-x.z, q.z, v);
-          v = fmaf(-x.w, q.w, v);
-          acc[c] = v;
+      if (two) panel_gemm<2>(acc, rp, pr, jp);
+      else panel_gemm<1>(acc, rp, pr, jp);
+      if (pass == 0) {
+        // the diagonal block: rows jp..jp+pw-1 are slot 0 of lanes 0..pw-1
+        __syncwarp();
+        if (lane < pw) {
+          *reinterpret_cast<float4*>(D + 8 * lane) = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
+          *reinterpret_cast<float4*>(D + 8 * lane + 4) = make_float4(acc[0][4], acc[0][5], acc[0][6], acc[0][7]);
         }
-      }
-      if (r == 0) {
-        // the 8x8 diagonal block: rows jp..jp+pw-1 are acc of lanes 0..pw-1
+        __syncwarp();
+        // factored in place: Ld's lower triangle becomes the block's L (its diagonal is
+        // not used: the reciprocal pivots il stand in for it)
+        float Ld[8][8];
+        float il[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const float4 lo = *reinterpret_cast<const float4*>(D + 8 * r);
+          const float4 hi = *reinterpret_cast<const float4*>(D + 8 * r + 4);
+          const float v[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+          for (int c = 0; c <= r; ++c) Ld[r][c] = v[c];
+        }
         bool ok = true;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
+          il[c] = 1.f;
           if (c < pw) {
-            const float d = __shfl_sync(0xffffffffu, acc[c], c);
-            if (!(d > 0.f)) { ok = false; break; }
+            const float d = Ld[c][c];
+            ok = ok && (d > 0.f);
             il[c] = rsqrtf(d);
-            if (lane == c) acc[c] = d * il[c];
-            else if (lane > c && lane < pw) acc[c] *= il[c];
-            if (lane == 0) idg[jp + c] = il[c];
 #pragma unroll
-            for (int c2 = c + 1; c2 < 8; ++c2) {
-              const float lc2 = __shfl_sync(0xffffffffu, acc[c], c2);   // L[jp+c2][jp+c]
-              if (lane >= c2 && lane < pw) acc[c2] = fmaf(-acc[c], lc2, acc[c2]);
-            }
+            for (int r = c + 1; r < 8; ++r) Ld[r][c] *= il[c];
+#pragma unroll
+            for (int r = c + 1; r < 8; ++r)
+#pragma unroll
+              for (int c2 = c + 1; c2 <= r; ++c2) Ld[r][c2] = fmaf(-Ld[r][c], Ld[c2][c], Ld[r][c2]);
           }
         }
-        if (!ok) return false;
+        if (!ok) return false;   // the same pivots in every lane
+        // back to D for the forward substitutions: L's strict lower triangle, and the
+        // reciprocal pivots on the diagonal (every lane holds the same values)
+        __syncwarp();
+        if (lane == 0) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
+          for (int r = 0; r < 8; ++r) {
+            float v[8];
 #pragma unroll
-          for (int c2 = 0; c2 <= c; ++c2) Ld[c][c2] = __shfl_sync(0xffffffffu, acc[c2], c);
+            for (int c = 0; c < 8; ++c) v[c] = c < r ? Ld[r][c] : (c == r ? il[r] : 0.f);
+            *reinterpret_cast<float4*>(D + 8 * r) = make_float4(v[0], v[1], v[2], v[3]);
+            *reinterpret_cast<float4*>(D + 8 * r + 4) = make_float4(v[4], v[5], v[6], v[7]);
+          }
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            if (c < pw) idg[jp + c] = il[c];
+        }
+        __syncwarp();
       }
-      if (i > s) continue;
-      if (i < jp + pw && i < s) {
-        *reinterpret_cast<float4*>(ri + jp) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        if (two) *reinterpret_cast<float4*>(ri + jp + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
-      } else {
+      // forward substitution of each row's panel entries; for a diagonal row i = jp + r
+      // this gives L[i][jp..i] with the pivot's square root at column i
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        if (q == 1 && !two) break;
+        const int i = ii[q];
+        if (i > s) continue;
         float x[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          float v = acc[c];
+          const float4 lo = *reinterpret_cast<const float4*>(D + 8 * c);
+          const float4 hi = *reinterpret_cast<const float4*>(D + 8 * c + 4);
+          const float l[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+          float v = acc[q][c];
 #pragma unroll
-          for (int c2 = 0; c2 < c; ++c2) v = fmaf(-x[c2], Ld[c][c2], v);
-          x[c] = v * il[c];
+          for (int c2 = 0; c2 < c; ++c2) v = fmaf(-x[c2], l[c2], v);
+          x[c] = v * l[c];
         }
-        *reinterpret_cast<float4*>(ri + jp) = make_float4(x[0], x[1], x[2], x[3]);
-        *reinterpret_cast<float4*>(ri + jp + 4) = make_float4(x[4], x[5], x[6], x[7]);
+        float* r = const_cast<float*>(rp[q]);
+        *reinterpret_cast<float4*>(r + jp) = make_float4(x[0], x[1], x[2], x[3]);
+        if (i >= jp + 4 || i >= s) *reinterpret_cast<float4*>(r + jp + 4) = make_float4(x[4], x[5], x[6], x[7]);
       }
     }
     __syncwarp();
@@ -175,117 +230,136 @@ __device__ bool chol_solve(const Rows<NS> R, float* __restrict__ y, float* __res
   return true;
 }
 
-// One warp per row over a persistent grid (each warp keeps one scratch slot).  SCAP
-// bounds the selected set; rows beyond NS of a large set live in the warp's global slot.
-template <int SCAP, int NS, bool NM>
-__global__ void __launch_bounds__(256) thanos_solve_kernel(const float* __restrict__ W, int c, int b,
-                                                           int j, int B, const float* __restrict__ Kt,
-                                                           const float* __restrict__ xnorm,
-                                                           Ctl* __restrict__ ctlp,
-                                                           uint8_t* __restrict__ mask,
-                                                           float* __restrict__ Zs, int nm_n, int nm_m,
-                                                           float* __restrict__ gscratch, pwp_stats* st) {
+// R-hat = K[Q, Q], lower triangle, into the packed rows: row a is K row q_a, loaded whole
+// (lane l holds columns 4l..4l+3), and entry (a, cc) is picked from lane q_cc / 4 by
+// shuffles.
+template <bool SMALL>
+__device__ void gather_rhat(const Rows<SMALL> R, const float* __restrict__ Kt, const int* __restrict__ Qidx, int s,
+                            int B, int nJ, int lane) {
+  constexpr int CH = (kCap + 31) / 32;
+  int qv[CH];
+#pragma unroll
+  for (int ch = 0; ch < CH; ++ch) qv[ch] = (lane + 32 * ch < s) ? Qidx[lane + 32 * ch] : 0;
+  const bool vec = (B & 3) == 0;
+  const int c4 = 4 * lane;
+  for (int a0 = 0; a0 < s; a0 += 4) {
+    float4 kv[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int a = a0 + r;
+      const float* krow = Kt + (size_t)(a < s ? Qidx[a] : Qidx[0]) * B;
+      if (vec && c4 + 3 < nJ) {
+        kv[r] = __ldg(reinterpret_cast<const float4*>(krow + c4));
+      } else {
+        kv[r].x = c4 < nJ ? __ldg(krow + c4) : 0.f;
+        kv[r].y = c4 + 1 < nJ ? __ldg(krow + c4 + 1) : 0.f;
+        kv[r].z = c4 + 2 < nJ ? __ldg(krow + c4 + 2) : 0.f;
+        kv[r].w = c4 + 3 < nJ ? __ldg(krow + c4 + 3) : 0.f;
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int a = a0 + r;
+      if (a >= s) break;
+      float* row = R.row(a);
+#pragma unroll
+      for (int ch = 0; ch < CH; ++ch) {
+        if (32 * ch > a) break;
+        const int src = qv[ch] >> 2, comp = qv[ch] & 3;
+        const float vx = __shfl_sync(0xffffffffu, kv[r].x, src);
+        const float vy = __shfl_sync(0xffffffffu, kv[r].y, src);
+        const float vz = __shfl_sync(0xffffffffu, kv[r].z, src);
+        const float vw = __shfl_sync(0xffffffffu, kv[r].w, src);
+        const float v = comp == 0 ? vx : comp == 1 ? vy : comp == 2 ? vz : vw;
+        const int cc = lane + 32 * ch;
+        if (cc <= a) row[cc] = v;
+      }
+    }
+  }
+  __syncwarp();
+}
+
+// One warp per row over a persistent grid (each warp keeps one shared-memory slab and one
+// global scratch slot).  A row whose selected set fits the shared rows takes the
+// shared-memory-only path; a larger one (rows past kNS in the warp's global slot) the
+// general path.
+template <bool NM>
+__global__ void __launch_bounds__(kSolveWarps * 32, 2) thanos_solve_kernel(const float* __restrict__ W, int c,
+                                                                          int b, int j, int B,
+                                                                          const float* __restrict__ Kt,
+                                                                          const float* __restrict__ xnorm,
+                                                                          Ctl* __restrict__ ctlp,
+                                                                          uint8_t* __restrict__ mask,
+                                                                          float* __restrict__ Zs, int nm_n, int nm_m,
+                                                                          float* __restrict__ gscratch,
+                                                                          pwp_stats* st) {
   extern __shared__ __align__(16) float smem[];
   if (warp_failed(st)) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nwarps = blockDim.x >> 5;
   const int slot = blockIdx.x * nwarps + warp;
-  float* L = smem + warp * SolveSmem<SCAP, NS>::kPerWarp;
-  float* y = L + SolveSmem<SCAP, NS>::kL;
-  int* Qidx = reinterpret_cast<int*>(y + SolveSmem<SCAP, NS>::kY);
-  const Rows<NS> R{L, gscratch ? gscratch + (size_t)slot * SolveSmem<SCAP, NS>::kGlobal : nullptr};
+  float* L = smem + warp * kPerWarp;
+  float* y = L + kL;
+  int* Qidx = reinterpret_cast<int*>(y + kY);
+  float* D = reinterpret_cast<float*>(Qidx + kCap);
+  float* G = gscratch ? gscratch + (size_t)slot * kGlobalPerWarp : nullptr;
   const Ctl ctl = *ctlp;
   const int nJ = min(B, b - j);
   constexpr int MAXI = kMaxBlock / 32;
   for (int k = slot; k < c; k += gridDim.x * nwarps) {
     const float* wrow = W + (long long)k * b + j;
-    float w[MAXI];
-    bool sel[MAXI];
-    int pos[MAXI];
+    uint8_t* mrow = mask + (long long)k * b + j;
+    // the selection: mask bytes, the selected indices and u = W[k, Q]; the warp keeps only
+    // the count (the positions are recounted from the mask bytes for the output)
     int s = 0;
 #pragma unroll
     for (int i = 0; i < MAXI; ++i) {
       const int qq = lane + 32 * i;
       const bool valid = qq < nJ;
-      w[i] = valid ? wrow[qq] : 0.f;
-      const unsigned int key = valid ? key_of<kWanda>(w[i], __ldg(xnorm + j + qq)) : 0xffffffffu;
-      sel[i] = (32 * i < nJ) ? selected<NM>(key, valid, qq, k, c, ctl, nm_n, nm_m) : false;
-      const unsigned int bal = __ballot_sync(0xffffffffu, sel[i]);
-      pos[i] = s + __popc(bal & ((1u << lane) - 1u));
+      const float w = valid ? wrow[qq] : 0.f;
+      const unsigned int key = valid ? key_of<kWanda>(w, __ldg(xnorm + j + qq)) : 0xffffffffu;
+      const bool sel = (32 * i < nJ) ? selected<NM>(key, valid, qq, k, c, ctl, nm_n, nm_m) : false;
+      const unsigned int bal = __ballot_sync(0xffffffffu, sel);
+      const int pos = s + __popc(bal & ((1u << lane) - 1u));
       s += __popc(bal);
+      if (valid) mrow[qq] = sel ? 1 : 0;
+      if (sel && pos < kCap) {
+        Qidx[pos] = qq;
+        y[pos] = w;
+      }
     }
-    if (s > SCAP || (s > NS && !R.G)) {   // excluded by the launcher's choice of SCAP / scratch
+    if (s > kNS && !G) {   // excluded by the launcher's choice of scratch
       if (lane == 0) set_error(st, PWP_EINVAL, kSiteSolve);
       continue;
-    }
-    uint8_t* mrow = mask + (long long)k * b + j;
-#pragma unroll
-    for (int i = 0; i < MAXI; ++i) {
-      const int qq = lane + 32 * i;
-      if (qq < nJ) mrow[qq] = sel[i] ? 1 : 0;
-      if (sel[i]) {
-        Qidx[pos[i]] = qq;
-        y[pos[i]] = w[i];
-      }
     }
     __syncwarp();
     bool ok = true;
     if (s > 0) {
-      // R-hat = K[Q, Q], lower triangle: row a is K row q_a, loaded whole (lane l holds
-      // columns 4l..4l+3), and entry (a, cc) is picked from lane q_cc / 4 by shuffles
-      constexpr int CH = (SCAP + 31) / 32;
-      int qv[CH];
-#pragma unroll
-      for (int ch = 0; ch < CH; ++ch) qv[ch] = (lane + 32 * ch < s) ? Qidx[lane + 32 * ch] : 0;
-      const bool vec = (B & 3) == 0;
-      const int c4 = 4 * lane;
-      for (int a0 = 0; a0 < s; a0 += 4) {
-        // four K rows in flight, then the picks from registers
-        float4 kv[4];
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int a = a0 + r;
-          const float* krow = Kt + (size_t)(a < s ? Qidx[a] : Qidx[0]) * B;
-          if (vec && c4 + 3 < nJ) {
-            kv[r] = __ldg(reinterpret_cast<const float4*>(krow + c4));
-          } else {
-            kv[r].x = c4 < nJ ? __ldg(krow + c4) : 0.f;
-            kv[r].y = c4 + 1 < nJ ? __ldg(krow + c4 + 1) : 0.f;
-            kv[r].z = c4 + 2 < nJ ? __ldg(krow + c4 + 2) : 0.f;
-            kv[r].w = c4 + 3 < nJ ? __ldg(krow + c4 + 3) : 0.f;
-          }
-        }
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int a = a0 + r;
-          if (a >= s) break;
-#pragma unroll
-          for (int ch = 0; ch < CH; ++ch) {
-            if (32 * ch > a) break;
-            const int src = qv[ch] >> 2, comp = qv[ch] & 3;
-            const float vx = __shfl_sync(0xffffffffu, kv[r].x, src);
-            const float vy = __shfl_sync(0xffffffffu, kv[r].y, src);
-            const float vz = __shfl_sync(0xffffffffu, kv[r].z, src);
-            const float vw = __shfl_sync(0xffffffffu, kv[r].w, src);
-            const float v = comp == 0 ? vx : comp == 1 ? vy : comp == 2 ? vz : vw;
-            const int cc = lane + 32 * ch;
-            if (cc <= a) R.row(a)[cc] = v;
-          }
-        }
+      // after the gather the selected indices are spent: their slots hold 1 / L_ii
+      if (s <= kNS) {
+        const Rows<true> R{L, nullptr};
+        gather_rhat<true>(R, Kt, Qidx, s, B, nJ, lane);
+        ok = chol_solve<true>(R, y, reinterpret_cast<float*>(Qidx), D, s, lane);
+      } else {
+        const Rows<false> R{L, G};
+        gather_rhat<false>(R, Kt, Qidx, s, B, nJ, lane);
+        ok = chol_solve<false>(R, y, reinterpret_cast<float*>(Qidx), D, s, lane);
       }
-      __syncwarp();
-      __syncwarp();  // the selected indices are spent: their slots hold 1 / L_ii from here on
-      ok = chol_solve<SCAP, NS>(R, y, reinterpret_cast<float*>(Qidx), s, lane);
       if (!ok && lane == 0) set_error(st, PWP_ENOTSPD, kSiteSolve);
       if (lane == 0) atomicAdd((unsigned long long*)&ctlp->pruned, (unsigned long long)s);
     }
     float* zrow = Zs + (long long)k * B;
     float* zlo = zrow + (long long)c * B;
+    int before = 0;
 #pragma unroll
     for (int i = 0; i < MAXI; ++i) {
       const int qq = lane + 32 * i;
+      const bool sel = qq < nJ && mrow[qq] != 0;   // this lane's own byte, written above
+      const unsigned int bal = __ballot_sync(0xffffffffu, sel);
+      const int pos = before + __popc(bal & ((1u << lane) - 1u));
+      before += __popc(bal);
       if (qq < B) {
-        const float z = (qq < nJ && sel[i] && ok) ? y[pos[i]] : 0.f;
+        const float z = (sel && ok) ? y[pos] : 0.f;
         const float h = tf32_head(z);
         zrow[qq] = h;
         zlo[qq] = z - h;
@@ -362,51 +436,41 @@ __global__ void __launch_bounds__(256) sparsegpt_solve_kernel(const float* __res
   if (lane == 0 && s > 0) atomicAdd((unsigned long long*)&ctlp->pruned, (unsigned long long)s);
 }
 
-template <int SCAP, int NS, bool NM>
+template <bool NM>
 void launch_thanos_variant(const float* W, int c, int b, int j, int B, const float* Kt, const float* xnorm,
                            Ctl* ctl, uint8_t* mask, float* Zs, int nm_n, int nm_m, float* gscratch,
                            pwp_stats* st, cudaStream_t s) {
-  constexpr int warps = 8;
-  const int smem = warps * SolveSmem<SCAP, NS>::kPerWarp * 4;
+  const int smem = kSolveWarps * kPerWarp * 4;
   static std::atomic<unsigned long long> attr_done{0};
   if (first_on_device(attr_done))
-    cudaFuncSetAttribute(thanos_solve_kernel<SCAP, NS, NM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  const int grid = min((c + warps - 1) / warps, kSolveCtas);
-  thanos_solve_kernel<SCAP, NS, NM><<<grid, warps * 32, smem, s>>>(W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n,
-                                                                  nm_m, gscratch, st);
+    cudaFuncSetAttribute(thanos_solve_kernel<NM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const int grid = min((c + kSolveWarps - 1) / kSolveWarps, kSolveCtas);
+  thanos_solve_kernel<NM><<<grid, kSolveWarps * 32, smem, s>>>(W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m,
+                                                               gscratch, st);
 }
 
 }  // namespace
 
+// Global scratch of the row solves: one slot per resident warp for factor rows past the
+// shared ones, needed only when a row can select more than kNS weights of a block.
 size_t solve_scratch_bytes(int c, int B, bool nm, int nm_n, int nm_m) {
   const int smax = nm ? B / nm_m * (nm_m - nm_n) : B;
-  if (smax <= 80) return 0;
-  const int grid = min((c + 7) / 8, kSolveCtas);  // the launch's grid (8 warps per CTA)
-  return (size_t)grid * 8 * SolveSmem<kMaxBlock, kSolveNS>::kGlobal * sizeof(float);
+  if (smax <= kNS) return 0;
+  const int grid = min((c + kSolveWarps - 1) / kSolveWarps, kSolveCtas);  // the launch's grid
+  return (size_t)grid * kSolveWarps * kGlobalPerWarp * sizeof(float);
 }
 
 // A row's selected set is at most min(B, block width) (unstructured) or exactly
-// B (m-n)/m (N:M).  8-warp CTAs keep up to 80 rows of each warp's factor in shared memory
-// (two CTAs per SM); when a block can hold larger sets (capacity 128, whose larger u/index
-// vectors leave room for 79 rows at two CTAs per SM), rows 79..127 of a large set go to
-// the warp's slot of global scratch.
+// B (m-n)/m (N:M).  8-warp CTAs, two per SM, keep kNS rows of each warp's factor in
+// shared memory; rows past them (rows with larger sets) go to the warp's slot of global
+// scratch.
 int launch_thanos_solve(bool nm, const float* W, int c, int b, int j, int B, const float* Kt,
                         const float* xnorm, Ctl* ctl, uint8_t* mask, float* Zs, int nm_n, int nm_m,
                         float* gscratch, pwp_stats* st, cudaStream_t s) {
-  const int smax = nm ? B / nm_m * (nm_m - nm_n) : min(B, b - j);
-  if (smax <= 80) {
-    if (nm)
-      launch_thanos_variant<80, 80, true>(W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, nullptr, st, s);
-    else
-      launch_thanos_variant<80, 80, false>(W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, nullptr, st, s);
-  } else {
-    if (nm)
-      launch_thanos_variant<kMaxBlock, kSolveNS, true>(W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m,
-                                                       gscratch, st, s);
-    else
-      launch_thanos_variant<kMaxBlock, kSolveNS, false>(W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m,
-                                                        gscratch, st, s);
-  }
+  if (nm)
+    launch_thanos_variant<true>(W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, gscratch, st, s);
+  else
+    launch_thanos_variant<false>(W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, gscratch, st, s);
   return 1;
 }
 

@@ -67,6 +67,11 @@ def compare(W_store, dtype, gpu, orc, *, pattern, nm, block, tie_tol):
         "n_dis": int(len(dis)),
         "n_dis_not_tie": int((~tie_ok).sum()),
         "dis_gaps": sorted(gaps.tolist())[-8:],       # the largest relative score gaps that flipped
+        # rows whose first (lowest-column) disagreement is not a tie: a later one in a row
+        # follows from that row's earlier flip
+        "rows_first_not_tie": int(sum(1 for k in np.unique(dis[:, 0]) if
+                                      not tie_ok[np.flatnonzero(dis[:, 0] == k)[np.argmin(dis[dis[:, 0] == k, 1])]]))
+        if len(dis) else 0,
         "w_rel": float(np.linalg.norm(W_hat - Wo) / np.linalg.norm(Wo)),
         "zeros_exact": bool(np.all(W_hat[mask] == 0.0)),
         "n_mask": int(mask.sum()),

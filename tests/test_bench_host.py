@@ -28,12 +28,13 @@ def test_select_and_hessian_and_factor():
 
 
 def test_solve_flops_from_the_mask():
-    """s = the selected count of a row in a block; per row and block s^3/3 + 2 s^2 + 4 s B."""
+    """s = the selected count of a row in a block; per row and block s^3/3 + 2 s^2 (the
+    Cholesky and the two triangular solves)."""
     wl = synth.custom(8, 24, 12, dtype="fp32", block=8, sparsity=0.5)    # three whole blocks
     mask = np.zeros((8, 24), dtype=np.uint8)
     mask[0, 0:3] = 1          # row 0, block 0: s = 3
     mask[1, 8:10] = 1         # row 1, block 1: s = 2
-    want = (27 / 3 + 2 * 9 + 4 * 3 * 8) + (8 / 3 + 2 * 4 + 4 * 2 * 8)
+    want = (27 / 3 + 2 * 9) + (8 / 3 + 2 * 4)
     work, unit, bound = bench.algorithmic_work(bench.K_SOLVE, wl, [1.0] * 3, mask)
     assert np.isclose(work, want) and unit == "flop" and bound == "alu"
 
@@ -56,8 +57,8 @@ def test_reference_arm_prints_the_contract_line():
     import subprocess
     import sys
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "3"],
-                         cwd=root, capture_output=True, text=True, timeout=600)
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "3",
+                          "--cpu-rows", "64"], cwd=root, capture_output=True, text=True, timeout=600)
     assert out.returncode == 0, out.stderr[-2000:]
     lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
     assert len(lines) == 1
@@ -69,7 +70,8 @@ def test_reference_arm_prints_the_contract_line():
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "weights/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
-    assert abs(d["ms_per_step"] - 4096 * 128 / d["value"] * 1e3) < 1e-6 * d["ms_per_step"]
+    assert abs(d["ms_per_step"] - 4096 * 64 / d["value"] * 1e3) < 1e-6 * d["ms_per_step"]
+    assert "64 of 4096 rows" in cb["sample"]
 
 
 def test_reference_arm_other_ranks_exit_quietly():
@@ -80,3 +82,25 @@ def test_reference_arm_other_ranks_exit_quietly():
     out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--gpus", "2"], cwd=root, env=env,
                          capture_output=True, text=True, timeout=120)
     assert out.returncode == 0 and out.stdout.strip() == ""
+
+
+def test_block_phase_bytes_and_phase_fractions():
+    """Block phase bytes: 8 c sum(b - j) + 4 B sum over blocks after the first of (b - j) +
+    7 c b; each phase's fraction is its work over its time over its peak."""
+    wl = _wl()                                   # c=8, b=20, B=8: j = 0, 8, 16
+    want = 8 * 8 * (20 + 12 + 4) + 4 * 8 * (12 + 4) + 7 * 8 * 20
+    assert bench.block_phase_bytes(wl) == want
+    peaks = {"hbm_gbs": 1000.0, "bf16_tflops": 2250.0, "sm_max_mhz": 1000.0}
+    mask = np.zeros((8, 20), dtype=np.uint8)
+    mask[:, :4] = 1                              # s = 4 in block 0 for every row
+    ph = bench.phase_rooflines(wl, {"hessian_xxt": 1.0, "factor": 2.0, "stream_update_score": 1.0,
+                                    "select": 0.5, "row_solve": 0.5}, mask, peaks)
+    assert np.isclose(ph["hessian_xxt"]["achieved"], 20 * 20 * 12 / 1e-3 / 1e12)
+    assert np.isclose(ph["hessian_xxt"]["frac"], ph["hessian_xxt"]["achieved"] / 2250.0)
+    assert np.isclose(ph["row_solve"]["achieved"], 8 * (64 / 3 + 32) / 0.5e-3 / 1e12)
+    assert np.isclose(ph["block_phase"]["ms"], 2.0)
+    assert np.isclose(ph["block_phase"]["achieved"], want / 2e-3 / 1e9)
+    # trailing update: block t's 2 c |J_t| (b - j_t) flops, applied by the next pass (the
+    # last block's by the final pass): j = 0, 8 with |J| = 8, and j = 16 with |J| = 4
+    assert np.isclose(ph["trailing_update_tensor"]["achieved"], 2 * 8 * (8 * 20 + 8 * 12 + 4 * 4) / 1e-3 / 1e12)
+    assert np.isclose(ph["trailing_update_tensor"]["peak"], 2250.0 * 1.1 / 2.25)

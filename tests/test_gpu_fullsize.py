@@ -105,10 +105,27 @@ def test_q_proj_whole_layer_matches_the_oracle():
     orc = oracle.prune_layer(W64, H=H64, sparsity=float(np.float32(wl.sparsity)), block=wl.block, damp=wl.damp)
     res = P.compare(W, wl.dtype, (W_hat, mask, st), orc, pattern="unstructured", nm=(0, 0), block=wl.block,
                     tie_tol=TIE_TOL)
-    assert res["agree"] >= P.MASK_AGREE and res["n_dis_not_tie"] == 0, res
+    assert res["agree"] >= P.MASK_AGREE, res
     assert res["w_rel"] <= P.W_REL_TOL, res
     lg = oracle.recon_loss(W64, W_hat, 0.5 * H64)
     assert abs(lg - orc["loss"]) <= P.LOSS_REL_TOL * orc["loss"], (lg, orc["loss"])
+    # Disagreements only at ties, judged on the GPU's own trajectory: once a row takes a
+    # different weight at a tie, its later weights (and the residual budget) legitimately
+    # differ from the independent run's.  The oracle replays the GPU's mask in fp64 and, at
+    # every block, applies the selection rule to that state; the GPU's block mask may
+    # differ from it only within TIE_TOL of the block's threshold.
+    rep = oracle.prune_layer(W64, H=H64, sparsity=float(np.float32(wl.sparsity)), block=wl.block, damp=wl.damp,
+                             fixed_mask=mask)
+    assert float(np.linalg.norm(W_hat - rep["W"]) / np.linalg.norm(rep["W"])) <= P.W_REL_TOL
+    worst, n_off = 0.0, 0
+    for blk in rep["blocks"]:
+        j = blk["j"]
+        t = blk["t_last"]
+        for k, q in np.argwhere(mask[:, j:j + wl.block] != blk["chosen"]):
+            gap = abs(rep["dscore"][k, j + q] - t) / max(abs(t), 1e-300)
+            worst = max(worst, gap)
+            n_off += 1
+    assert worst <= TIE_TOL, (n_off, worst, res)
 
 
 @pytest.mark.parametrize("name", ["up_proj11008x4096_2of4", "down_proj4096x11008_4of8"])

@@ -559,3 +559,24 @@ def test_fixed_mask_replay_reproduces_full_runs_on_row_subsets(pattern, nm):
         assert np.allclose(sub["W"], full["W"][rows], rtol=1e-12, atol=1e-15)
         assert np.isclose(sub["loss"], float(np.sum(oracle.row_losses(W[rows], full["W"][rows],
                                                                          0.5 * oracle.hessian(Xt)))))
+
+
+def test_fixed_mask_replay_records_the_selection_of_the_replayed_state():
+    """Replaying the full run's own mask, every block's recorded choice is the mask itself;
+    with one block-0 decision flipped, block 0's recorded choice shows the flip (and only
+    that), since the choice is made before the block's update."""
+    rng = np.random.default_rng(23)
+    Xt = rng.normal(size=(50, 20))
+    W = rng.normal(0, 0.02, size=(9, 20))
+    full = oracle.prune_layer(W, Xt=Xt, sparsity=0.5, block=5)
+    again = oracle.prune_layer(W, Xt=Xt, sparsity=0.5, block=5, fixed_mask=full["mask"])
+    for blk in again["blocks"]:
+        j = blk["j"]
+        assert np.array_equal(blk["chosen"], full["mask"][:, j:j + 5])
+        assert blk["r"] == full["zstar"] - int(full["mask"][:, :j].sum())
+    flipped = full["mask"].copy()
+    k, q = np.argwhere(flipped[:, :5])[0]
+    flipped[k, q] = False
+    other = oracle.prune_layer(W, Xt=Xt, sparsity=0.5, block=5, fixed_mask=flipped)
+    diff = np.argwhere(other["blocks"][0]["chosen"] != flipped[:, :5])
+    assert diff.tolist() == [[k, q]]
