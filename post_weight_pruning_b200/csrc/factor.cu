@@ -30,6 +30,7 @@ constexpr int NB = kFactorNB;  // 64
 
 __global__ void __launch_bounds__(1024) damp_kernel(float* __restrict__ H, int b, float damp,
                                                     float* __restrict__ g_diag, pwp_stats* st) {
+  pdl_enter();
   __shared__ double red[32];
   __shared__ float lam_s;
   double s = 0.0;
@@ -200,6 +201,7 @@ __device__ bool factor_diag_block(float (*A)[NB + 1], float (*Wi)[NB + 1], int n
 // Stand-alone factorisation of the diagonal block at p0 (used for the last panel).
 __global__ void __launch_bounds__(256) chol_diag_kernel(float* __restrict__ H, int b, int p0, int nb,
                                                         float* __restrict__ Vinv, pwp_stats* st) {
+  pdl_enter();
   extern __shared__ __align__(16) float dsm[];   // A and Wi, 2 x NB x (NB + 1) floats
   float (*A)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(dsm);
   float (*Wi)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(dsm + NB * (NB + 1));
@@ -228,6 +230,7 @@ __global__ void __launch_bounds__(256) chol_panel_kernel(float* __restrict__ H, 
                                                          const float* __restrict__ Vinv,
                                                          float* __restrict__ vs_hi, float* __restrict__ vs_lo,
                                                          const pwp_stats* st) {
+  pdl_enter();
   __shared__ float WiT[NB][NB + 1];  // WiT[t][c] = Wi[c][t]
   __shared__ float rowbuf[8][NB];
   if (cta_failed(st)) return;
@@ -266,6 +269,7 @@ __global__ void __launch_bounds__(256) chol_panel_kernel(float* __restrict__ H, 
 __global__ void __launch_bounds__(256) chol_update_kernel(float* __restrict__ H, int b, int p0, int nb,
                                                           float* __restrict__ Vinv_next,
                                                           pwp_stats* st) {
+  pdl_enter();
   extern __shared__ __align__(16) float fsm[];
   float (*As)[128 + 4] = reinterpret_cast<float (*)[132]>(fsm);               // [NB][132], k-major
   float (*Bs)[128 + 4] = reinterpret_cast<float (*)[132]>(fsm + NB * 132);
@@ -350,6 +354,7 @@ __global__ void __launch_bounds__(256) chol_update_kernel(float* __restrict__ H,
 // matrix has the inverses of its diagonal blocks on its block diagonal).
 __global__ void put_diag_inverses_kernel(float* __restrict__ H, int b, const float* __restrict__ Vall,
                                          const pwp_stats* st) {
+  pdl_enter();
   if (cta_failed(st)) return;
   const int p = blockIdx.x;
   const int p0 = p * NB, nb = min(NB, b - p0);
@@ -429,6 +434,7 @@ __device__ __forceinline__ void trigemm_load(const TriGemm& g, const float* A, c
 }
 
 __global__ void __launch_bounds__(256) trigemm_kernel(TriGemm g, int vec, const pwp_stats* st) {
+  pdl_enter();
   __shared__ __align__(16) float As[2][16][128 + 4];
   __shared__ __align__(16) float Bs[2][16][128 + 4];
   if (cta_failed(st)) return;
@@ -506,7 +512,7 @@ void launch_trigemm(const TriGemm& g, int batch, const pwp_stats* st, cudaStream
   const bool vec = ((uintptr_t)g.A % 16) == 0 && ((uintptr_t)g.B % 16) == 0 && ((uintptr_t)g.C % 16) == 0 &&
                    (g.lda % 4) == 0 && (g.ldb % 4) == 0 && (g.ldc % 4) == 0 && (g.batch_a % 4) == 0 &&
                    (g.batch_b % 4) == 0 && (g.batch_c % 4) == 0;
-  trigemm_kernel<<<grid, 256, 0, s>>>(g, vec ? 1 : 0, st);
+  launch_pdl(trigemm_kernel, dim3(grid), dim3(256), 0, s, g, vec ? 1 : 0, st);
 }
 
 }  // namespace
@@ -546,19 +552,19 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
     cudaFuncSetAttribute(chol_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * NB * (NB + 1) * 4);
   }
   long long nl = 0;
-  damp_kernel<<<1, 1024, 0, s>>>(H, b, damp, g_diag, st);
+  launch_pdl(damp_kernel, dim3(1), dim3(1024), 0, s, H, b, damp, g_diag, st);
   ++nl;
   // factor, panels from the last; the last panel's diagonal block stands alone
   {
     const int p = np - 1, p0 = p * NB, nb = b - p0;
-    chol_diag_kernel<<<1, 256, 2 * NB * (NB + 1) * 4, s>>>(H, b, p0, nb, Vall + (size_t)p * NB * NB, st);
+    launch_pdl(chol_diag_kernel, dim3(1), dim3(256), 2 * NB * (NB + 1) * 4, s, H, b, p0, nb, Vall + (size_t)p * NB * NB, st);
     ++nl;
   }
   for (int p = np - 1; p >= 1; --p) {
     const int p0 = p * NB, nb = min(NB, b - p0);
     float* V = Vall + (size_t)p * NB * NB;
     const int pgrid = min((p0 + 7) / 8, kNumSM);
-    chol_panel_kernel<<<pgrid, 256, 0, s>>>(H, b, p0, nb, V, vs_hi, vs_lo, st);
+    launch_pdl(chol_panel_kernel, dim3(pgrid), dim3(256), 0, s, H, b, p0, nb, V, vs_hi, vs_lo, st);
     // H[0:p0, 0:p0] -= V[0:p0, P] V[0:p0, P]^T on the tensor cores (tiles on or above the
     // diagonal), then the next panel's diagonal block on its own; the CUDA-core kernel
     // (which also factors that block) when the tensor-core path is not available
@@ -567,15 +573,15 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
                                      nullptr, 0, nullptr, nullptr, Level2{}, st, s, &e2, true);
     if (e2 != cudaSuccess) return e2;
     if (tc) {
-      chol_diag_kernel<<<1, 256, 2 * NB * (NB + 1) * 4, s>>>(H, b, p0 - NB, NB, Vall + (size_t)(p - 1) * NB * NB, st);
+      launch_pdl(chol_diag_kernel, dim3(1), dim3(256), 2 * NB * (NB + 1) * 4, s, H, b, p0 - NB, NB, Vall + (size_t)(p - 1) * NB * NB, st);
     } else {
       const int nT = (p0 + 127) / 128;
-      chol_update_kernel<<<nT * (nT + 1) / 2, 256, 2 * NB * 132 * 4, s>>>(H, b, p0, nb,
+      launch_pdl(chol_update_kernel, dim3(nT * (nT + 1) / 2), dim3(256), 2 * NB * 132 * 4, s, H, b, p0, nb,
                                                                         Vall + (size_t)(p - 1) * NB * NB, st);
     }
     nl += 3;
   }
-  put_diag_inverses_kernel<<<np, 256, 0, s>>>(H, b, Vall, st);
+  launch_pdl(put_diag_inverses_kernel, dim3(np), dim3(256), 0, s, H, b, Vall, st);
   ++nl;
   // inverse by recursive doubling: merge [A B; 0 D] pairs of width m
   for (int m = NB; m < b; m *= 2) {

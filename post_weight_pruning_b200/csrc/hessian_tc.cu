@@ -77,6 +77,7 @@ __device__ inline void tile_of(int idx, int b, int& I, int& J) {
 __global__ void __launch_bounds__(kThreads, 1) syrk_tc_kernel(const __grid_constant__ CUtensorMap tmap, long long n,
                                                               int b, float* __restrict__ H, int beta, pwp_stats* st,
                                                               long long spin) {
+  pdl_enter();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
@@ -302,7 +303,7 @@ cudaError_t launch_hessian_tc(const void* X, long long n, int b, float* H, int b
     cudaError_t e = cudaFuncSetAttribute(syrk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
   }
-  syrk_tc_kernel<<<tile_count(b), kThreads, SMEM_BYTES, s>>>(map, n, b, H, beta, st, wait_limit());
+  launch_pdl(syrk_tc_kernel, dim3(tile_count(b)), dim3(kThreads), SMEM_BYTES, s, map, n, b, H, beta, st, wait_limit());
   *used = true;
   return cudaGetLastError();
 }

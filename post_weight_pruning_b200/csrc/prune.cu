@@ -35,6 +35,7 @@ __global__ void init_stats_kernel(pwp_stats* st) {
 }
 
 __global__ void init_ctl_kernel(Ctl* ctl, long long zstar, pwp_stats* st, long long target) {
+  pdl_enter();
   ctl->zstar = zstar;
   ctl->pruned = 0;
   ctl->mode = 0;
@@ -48,6 +49,7 @@ __global__ void init_ctl_kernel(Ctl* ctl, long long zstar, pwp_stats* st, long l
 
 __global__ void convert_w_kernel(const void* __restrict__ W, int wtype, float* __restrict__ Wout,
                                  long long N) {
+  pdl_enter();
   long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
   long long stride = (long long)gridDim.x * blockDim.x;
   if (wtype == PWP_FP32) {
@@ -62,6 +64,7 @@ __global__ void convert_w_kernel(const void* __restrict__ W, int wtype, float* _
 // ||X_q|| = sqrt(G_qq) for the Wanda score, U_qq for the OBS score.
 __global__ void prep_diag_kernel(const float* __restrict__ H, int b, const float* __restrict__ g_diag,
                                  float* __restrict__ xnorm, float* __restrict__ udiag) {
+  pdl_enter();
   int q = blockIdx.x * blockDim.x + threadIdx.x;
   if (q < b) {
     xnorm[q] = sqrtf(g_diag[q]);
@@ -79,6 +82,7 @@ __global__ void prep_diag_kernel(const float* __restrict__ H, int b, const float
 __global__ void __launch_bounds__(256) kmat_kernel(const float* __restrict__ H, int b, int B,
                                                    float* __restrict__ K_in, float* __restrict__ K_hi,
                                                    float* __restrict__ K_lo, const pwp_stats* st) {
+  pdl_enter();
   extern __shared__ __align__(16) float sm[];
   if (cta_failed(st)) return;
   const int t = blockIdx.y;
@@ -163,6 +167,7 @@ __global__ void __launch_bounds__(256) stream_kernel(float* __restrict__ W, int 
                                                      unsigned int* __restrict__ hist1,
                                                      const Ctl* __restrict__ ctl, unsigned int* __restrict__ h2,
                                                      unsigned int* __restrict__ h2s, const pwp_stats* st) {
+  pdl_enter();
   extern __shared__ unsigned int shist[];  // kHist1Bins when SCORE != 0
   __shared__ float Zs[64][33];
   __shared__ __align__(16) float Rs[32][128];
@@ -255,6 +260,7 @@ __global__ void __launch_bounds__(256) stream_kernel(float* __restrict__ W, int 
 // K-major operand of the tensor-core update.
 __global__ void urows_kernel(const float* __restrict__ H, int b, int B, int jp, int Bp, float* __restrict__ Rhi,
                              float* __restrict__ Rlo, const pwp_stats* st) {
+  pdl_enter();
   if (failed(st)) return;
   const long long n = (long long)Bp * (b - jp);
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
@@ -267,6 +273,7 @@ __global__ void urows_kernel(const float* __restrict__ H, int b, int B, int jp, 
 }
 
 __global__ void finalize_kernel(const Ctl* ctl, pwp_stats* st, int check_budget) {
+  pdl_enter();
   st->pruned = ctl->pruned;
   if (st->status == PWP_OK && check_budget && ctl->pruned != ctl->zstar)
     set_error(st, PWP_EBUDGET, kSiteFinal);
@@ -345,7 +352,7 @@ static void launch_stream(float* W, int c, int b, int u0, int j, int col_end, co
   const int tiles = ((col_end - u0 + 127) / 128) * ((c + 63) / 64);
   const int nsm = g_nsm.load();
   const int grid = tiles < nsm ? tiles : nsm;
-  stream_kernel<SCORE><<<grid > 0 ? grid : 1, 256, smem, s>>>(W, c, b, u0, j, col_end, Z, Zlo, Bp, ldz, R, Rlo,
+  launch_pdl(stream_kernel<SCORE>, dim3(grid > 0 ? grid : 1), dim3(256), smem, s, W, c, b, u0, j, col_end, Z, Zlo, Bp, ldz, R, Rlo,
                                                              ldr, r_trans, r_upper_from, mask, sc, hist_end, hist1,
                                                              ctl, l2.pred, l2.pred_sum, st);
 }
@@ -418,22 +425,22 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
     init_stats_kernel<<<1, 1, 0, s>>>(st);
     ++nl;
   }
-  init_ctl_kernel<<<1, 1, 0, s>>>(pb.ctl, zstar, st, target);
+  launch_pdl(init_ctl_kernel, dim3(1), dim3(1), 0, s, pb.ctl, zstar, st, target);
   cudaError_t em = cudaMemsetAsync(pb.hist1, 0, sizeof(unsigned int) * kHist1Bins, s);
   if (em == cudaSuccess)
     em = cudaMemsetAsync(pb.l2.pred, 0, sizeof(unsigned int) * (2 * kHist2Bins + 2 * kHist2SumBins + kMaxBlock), s);
   if (em != cudaSuccess) return em;
-  convert_w_kernel<<<4 * g_nsm.load(), 256, 0, s>>>(W, wtype, Wout, N);
+  launch_pdl(convert_w_kernel, dim3(4 * g_nsm.load()), dim3(256), 0, s, W, wtype, Wout, N);
   nl += 2;
   prof_begin(kKFactor, s);
   cudaError_t e = launch_damp_factor(H, b, cfg->damp, pb.g_diag, pb.fws, pb.fws_bytes, st, s);
   prof_end(kKFactor, s);
   if (e != cudaSuccess) return e;
-  prep_diag_kernel<<<(b + 255) / 256, 256, 0, s>>>(H, b, pb.g_diag, pb.xnorm, pb.udiag);
+  launch_pdl(prep_diag_kernel, dim3((b + 255) / 256), dim3(256), 0, s, H, b, pb.g_diag, pb.xnorm, pb.udiag);
   ++nl;
   if (thanos) {
     dim3 g((b + 127) / 128, nblk);
-    kmat_kernel<<<g, 256, kmat_smem_bytes(B), s>>>(H, b, B, pb.K_in, pb.K_hi, pb.K_lo, st);
+    launch_pdl(kmat_kernel, dim3(g), dim3(256), kmat_smem_bytes(B), s, H, b, B, pb.K_in, pb.K_hi, pb.K_lo, st);
     ++nl;
   }
   const int score = nm ? kNoScore : (thanos ? kWanda : kObs);
@@ -458,7 +465,7 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
         if (!thanos) {
           const long long n = (long long)Bp * (b - jp);
           const int grid = (int)min((n + 255) / 256, (long long)8 * g_nsm.load());
-          urows_kernel<<<grid, 256, 0, s>>>(H, b, B, jp, Bp, pb.R_hi, pb.R_lo, st);
+          launch_pdl(urows_kernel, dim3(grid), dim3(256), 0, s, H, b, B, jp, Bp, pb.R_hi, pb.R_lo, st);
           ++nl;
         }
         cudaError_t e2 = cudaSuccess;
@@ -503,7 +510,7 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
                                    cfg->nm_m, st, s);
     prof_end(kKSolve, s);
   }
-  finalize_kernel<<<1, 1, 0, s>>>(pb.ctl, st, (thanos && !nm) ? 1 : 0);
+  launch_pdl(finalize_kernel, dim3(1), dim3(1), 0, s, pb.ctl, st, (thanos && !nm) ? 1 : 0);
   count_launches(nl + 1);
   return cudaGetLastError();
 }

@@ -20,6 +20,36 @@ inline bool first_on_device(std::atomic<unsigned long long>& done) {
   return (done.fetch_or(bit) & bit) == 0;
 }
 
+// Programmatic dependent launch.  Kernels of the prune's dependent chains are launched
+// with programmatic stream serialisation, so a kernel's CTAs may be scheduled while its
+// predecessor's last CTAs still run.  Every such kernel therefore starts with pdl_wait()
+// (griddepcontrol.wait: the predecessor grid has completed and its writes are visible)
+// before it reads anything, and lets its own dependents be scheduled at once
+// (pdl_release).  Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_enter() {
+  pdl_wait();
+  pdl_release();
+}
+
+// Launch with programmatic stream serialisation (the kernel must begin with pdl_enter()).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 constexpr int kNumSM = 148;              // B200
 constexpr int kKeyLoBits = 18;           // second radix level: key bits [17:0]
 constexpr int kHist1Bits = 31 - kKeyLoBits;  // first level: key bits [30:18] (32 KB of shared memory)

@@ -101,6 +101,7 @@ __device__ void find_rank(const unsigned int* __restrict__ hist, long long rank,
 
 __global__ void __launch_bounds__(1024) pick1_kernel(Ctl* ctl, unsigned int* __restrict__ hist1, long long region_n,
                                                      int global_budget, long long quota, pwp_stats* st) {
+  pdl_enter();
   __shared__ long long sh_warp[32];
   __shared__ int sh_sel;
   __shared__ long long sh_base, s_take;
@@ -152,6 +153,7 @@ __global__ void __launch_bounds__(256) refine_kernel(const float* __restrict__ W
                                                      int q1, const float* __restrict__ sc,
                                                      const Ctl* __restrict__ ctl, unsigned int* __restrict__ h2,
                                                      unsigned int* __restrict__ h2s, const pwp_stats* st) {
+  pdl_enter();
   if (cta_failed(st) || ctl->mode == 0 || ctl->l2_ready) return;
   const unsigned int b1 = ctl->b1;
   for (int r = blockIdx.x; r < c; r += gridDim.x) {
@@ -162,6 +164,7 @@ __global__ void __launch_bounds__(256) refine_kernel(const float* __restrict__ W
 }
 
 __global__ void __launch_bounds__(1024) pick2_kernel(Ctl* ctl, Level2 l2, pwp_stats* st) {
+  pdl_enter();
   __shared__ long long sh_warp[32];
   __shared__ int sh_sel;
   __shared__ long long sh_base;
@@ -209,6 +212,7 @@ template <int SCORE>
 __global__ void __launch_bounds__(256) clear_level2_kernel(const Ctl* __restrict__ ctl, Level2 l2,
                                                            const float* __restrict__ W, int c, int b, int j, int j1,
                                                            const float* __restrict__ sc) {
+  pdl_enter();
   const bool a = ctl->dirty_pred != 0, r = ctl->dirty_reread != 0;
   const int gtid = blockIdx.x * blockDim.x + threadIdx.x, stride = gridDim.x * blockDim.x;
   if (a || r) {
@@ -257,6 +261,7 @@ template <int SCORE>
 __global__ void __launch_bounds__(1024) tie_pick_kernel(Ctl* ctl, Level2 l2, const float* __restrict__ W, int c,
                                                         int b, int j, int j1, const float* __restrict__ sc,
                                                         pwp_stats* st) {
+  pdl_enter();
   __shared__ long long sh_warp[32];
   __shared__ int s_qstar;
   __shared__ long long s_need;
@@ -318,36 +323,36 @@ __global__ void __launch_bounds__(1024) tie_pick_kernel(Ctl* ctl, Level2 l2, con
 
 void launch_pick1(Ctl* ctl, unsigned int* hist1, long long region_n, int global_budget, long long quota,
                   pwp_stats* st, cudaStream_t s) {
-  pick1_kernel<<<1, 1024, 0, s>>>(ctl, hist1, region_n, global_budget, quota, st);
+  launch_pdl(pick1_kernel, dim3(1), dim3(1024), 0, s, ctl, hist1, region_n, global_budget, quota, st);
 }
 
 void launch_refine(int score, const float* W, int c, int b, int q0, int q1, const float* sc,
                    const Ctl* ctl, Level2 l2, const pwp_stats* st, cudaStream_t s) {
   const int grid = c < 4 * kNumSM ? c : 4 * kNumSM;
   if (score == kWanda)
-    refine_kernel<kWanda><<<grid, 256, 0, s>>>(W, c, b, q0, q1, sc, ctl, l2.reread, l2.reread_sum, st);
+    launch_pdl(refine_kernel<kWanda>, dim3(grid), dim3(256), 0, s, W, c, b, q0, q1, sc, ctl, l2.reread, l2.reread_sum, st);
   else
-    refine_kernel<kObs><<<grid, 256, 0, s>>>(W, c, b, q0, q1, sc, ctl, l2.reread, l2.reread_sum, st);
+    launch_pdl(refine_kernel<kObs>, dim3(grid), dim3(256), 0, s, W, c, b, q0, q1, sc, ctl, l2.reread, l2.reread_sum, st);
 }
 
 void launch_pick2(Ctl* ctl, Level2 l2, pwp_stats* st, cudaStream_t s) {
-  pick2_kernel<<<1, 1024, 0, s>>>(ctl, l2, st);
+  launch_pdl(pick2_kernel, dim3(1), dim3(1024), 0, s, ctl, l2, st);
 }
 
 void launch_clear_level2(int score, const Ctl* ctl, Level2 l2, const float* W, int c, int b, int j, int j1,
                          const float* sc, cudaStream_t s) {
   if (score == kWanda)
-    clear_level2_kernel<kWanda><<<kNumSM, 256, 0, s>>>(ctl, l2, W, c, b, j, j1, sc);
+    launch_pdl(clear_level2_kernel<kWanda>, dim3(kNumSM), dim3(256), 0, s, ctl, l2, W, c, b, j, j1, sc);
   else
-    clear_level2_kernel<kObs><<<kNumSM, 256, 0, s>>>(ctl, l2, W, c, b, j, j1, sc);
+    launch_pdl(clear_level2_kernel<kObs>, dim3(kNumSM), dim3(256), 0, s, ctl, l2, W, c, b, j, j1, sc);
 }
 
 void launch_tie_pick(int score, Ctl* ctl, Level2 l2, const float* W, int c, int b, int j, int j1, const float* sc,
                      pwp_stats* st, cudaStream_t s) {
   if (score == kWanda)
-    tie_pick_kernel<kWanda><<<1, 1024, 0, s>>>(ctl, l2, W, c, b, j, j1, sc, st);
+    launch_pdl(tie_pick_kernel<kWanda>, dim3(1), dim3(1024), 0, s, ctl, l2, W, c, b, j, j1, sc, st);
   else
-    tie_pick_kernel<kObs><<<1, 1024, 0, s>>>(ctl, l2, W, c, b, j, j1, sc, st);
+    launch_pdl(tie_pick_kernel<kObs>, dim3(1), dim3(1024), 0, s, ctl, l2, W, c, b, j, j1, sc, st);
 }
 
 }  // namespace pwp

@@ -293,6 +293,7 @@ __global__ void __launch_bounds__(kSolveWarps * 32, 2) thanos_solve_kernel(const
                                                                           float* __restrict__ Zs, int nm_n, int nm_m,
                                                                           float* __restrict__ gscratch,
                                                                           pwp_stats* st) {
+  pdl_enter();
   extern __shared__ __align__(16) float smem[];
   if (warp_failed(st)) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -380,6 +381,7 @@ __global__ void __launch_bounds__(256) sparsegpt_solve_kernel(const float* __res
                                                               uint8_t* __restrict__ mask,
                                                               float* __restrict__ Zs, int nm_n, int nm_m,
                                                               pwp_stats* st) {
+  pdl_enter();
   if (warp_failed(st)) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int k = blockIdx.x * (blockDim.x >> 5) + warp;
@@ -445,7 +447,7 @@ void launch_thanos_variant(const float* W, int c, int b, int j, int B, const flo
   if (first_on_device(attr_done))
     cudaFuncSetAttribute(thanos_solve_kernel<NM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   const int grid = min((c + kSolveWarps - 1) / kSolveWarps, kSolveCtas);
-  thanos_solve_kernel<NM><<<grid, kSolveWarps * 32, smem, s>>>(W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m,
+  launch_pdl(thanos_solve_kernel<NM>, dim3(grid), dim3(kSolveWarps * 32), smem, s, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m,
                                                                gscratch, st);
 }
 
@@ -479,9 +481,9 @@ int launch_sparsegpt_solve(bool nm, const float* W, int c, int b, int j, int B, 
                            pwp_stats* st, cudaStream_t s) {
   const int grid = (c + 7) / 8;
   if (nm)
-    sparsegpt_solve_kernel<true><<<grid, 256, 0, s>>>(W, c, b, j, B, H, udiag, ctl, mask, Zs, nm_n, nm_m, st);
+    launch_pdl(sparsegpt_solve_kernel<true>, dim3(grid), dim3(256), 0, s, W, c, b, j, B, H, udiag, ctl, mask, Zs, nm_n, nm_m, st);
   else
-    sparsegpt_solve_kernel<false><<<grid, 256, 0, s>>>(W, c, b, j, B, H, udiag, ctl, mask, Zs, nm_n, nm_m, st);
+    launch_pdl(sparsegpt_solve_kernel<false>, dim3(grid), dim3(256), 0, s, W, c, b, j, B, H, udiag, ctl, mask, Zs, nm_n, nm_m, st);
   return 1;
 }
 

@@ -94,6 +94,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const uint8_t* __restrict__ mask, const float* __restrict__ sc, int hist_end,
                      unsigned int* __restrict__ hist1, const Ctl* __restrict__ ctl, unsigned int* __restrict__ h2,
                      unsigned int* __restrict__ h2s, pwp_stats* st, long long spin) {
+  pdl_enter();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* wbuf = smem + W_OFF;
@@ -388,7 +389,7 @@ cudaError_t launch_variant(const CUtensorMap* maps, int c, int b, int u0, int j,
   const int mt = (c + TM - 1) / TM;
   const int ntiles = upper ? mt * (mt + 1) / 2 : mt * ((b - u0 + TN - 1) / TN);
   const int grid = ntiles < nsm ? ntiles : nsm;
-  stream_tc_kernel<SCORE><<<grid, kThreads, SMEM_BYTES, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4], c, b, u0,
+  launch_pdl(stream_tc_kernel<SCORE>, dim3(grid), dim3(kThreads), SMEM_BYTES, s, maps[0], maps[1], maps[2], maps[3], maps[4], c, b, u0,
                                                              j, Bp, upper, mask, sc, hist_end, hist1, ctl, l2.pred,
                                                              l2.pred_sum, st, wait_limit());
   return cudaGetLastError();
