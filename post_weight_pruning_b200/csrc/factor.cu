@@ -21,7 +21,7 @@
 //   inverse, recursive doubling: with the diagonal blocks inverted, neighbouring
 //     blocks [A B; 0 D] are merged as [A^-1, -A^-1 B D^-1; 0, D^-1] level by level,
 //     each level two batched triangular-times-dense products.
-#include "pwp_internal.cuh"
+#include "tc_common.cuh"
 
 namespace pwp {
 namespace {
@@ -506,6 +506,56 @@ __global__ void __launch_bounds__(256) trigemm_kernel(TriGemm g, int vec, const 
   }
 }
 
+// Operands of the tensor-core levels of the doubling inverse, as TF32 head and fp32
+// remainder (the form the 3xTF32 update kernel takes, both K-major).
+// split: dst[r][k] = sign * src[r][k] for r < rows, k < cols; with tri, entries left of
+// the upper triangle (k + koff < r, k counted from the chunk's first column koff) are 0.
+__global__ void __launch_bounds__(256) split_kernel(const float* __restrict__ src, long long lds, int rows, int cols,
+                                                    int tri, int koff, float sign, float* __restrict__ hi,
+                                                    float* __restrict__ lo, int ldd, const pwp_stats* st) {
+  pdl_enter();
+  if (failed(st)) return;
+  const long long n = (long long)rows * cols;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)(i / cols), k = (int)(i - (long long)r * cols);
+    float v = src[(long long)r * lds + k];
+    if (tri && k + koff < r) v = 0.f;
+    v *= sign;
+    const float h = tf32_head(v);
+    hi[(long long)r * ldd + k] = h;
+    lo[(long long)r * ldd + k] = v - h;
+  }
+}
+
+// Transposed split: dst[q][k] = src[k][q] for k < krows, q < ncols, through 32x32 shared
+// tiles (both sides coalesced); with tri, src is upper triangular from the chunk's first row
+// koff on: entries with q < k + koff are 0.
+__global__ void __launch_bounds__(256) tsplit_kernel(const float* __restrict__ src, long long lds, int krows,
+                                                     int ncols, int tri, int koff, float* __restrict__ hi,
+                                                     float* __restrict__ lo, int ldd, const pwp_stats* st) {
+  pdl_enter();
+  __shared__ float tile[32][33];
+  if (failed(st)) return;
+  const int k0 = blockIdx.y * 32, q0 = blockIdx.x * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8
+  for (int r = ty; r < 32; r += 8) {
+    const int k = k0 + r, q = q0 + tx;
+    float v = (k < krows && q < ncols) ? src[(long long)k * lds + q] : 0.f;
+    if (tri && q < k + koff) v = 0.f;
+    tile[r][tx] = v;
+  }
+  __syncthreads();
+  for (int r = ty; r < 32; r += 8) {
+    const int q = q0 + r, k = k0 + tx;
+    if (q < ncols && k < krows) {
+      const float v = tile[tx][r];
+      const float h = tf32_head(v);
+      hi[(long long)q * ldd + k] = h;
+      lo[(long long)q * ldd + k] = v - h;
+    }
+  }
+}
+
 void launch_trigemm(const TriGemm& g, int batch, const pwp_stats* st, cudaStream_t s) {
   dim3 grid((g.N + 127) / 128, (g.M + 127) / 128, batch);
   // float4 access needs 16-byte aligned rows and batch entries
@@ -530,11 +580,92 @@ static size_t doubling_tmp_floats(int b) {
   return tmp;
 }
 
-// Diagonal-block inverses, the doubling temporary, and the current panel's rows as TF32
-// head and remainder (2 x b x NB), the last 256-byte aligned.
+// Doubling levels at least this wide run on the tensor cores (3xTF32), their products in
+// K chunks of at most kTcChunk; narrower levels stay on the CUDA cores, where the batch of
+// small products is latency-bound anyway.
+constexpr int kTcLevel = 1024, kTcChunk = 2048;
+
+// The pairs [A B; 0 D] of a doubling level of width m: (first index, width of D).
+template <typename F>
+static void for_each_pair(int b, int m, F f) {
+  const int full = b / (2 * m), rest = b - full * 2 * m;
+  for (int p = 0; p < full; ++p) f(p * 2 * m, m);
+  if (rest > m) f(full * 2 * m, rest - m);
+}
+
+// Floats of the tensor-core levels' scratch: T (m x m2) and the operand chunks (heads and
+// remainders, m x KC and m2 x KC), for the largest pair.
+static size_t tc_levels_floats(int b) {
+  size_t need = 0;
+  for (int m = kTcLevel; m < b; m *= 2)
+    for_each_pair(b, m, [&](int, int m2) {
+      const size_t kc = (size_t)min(kTcChunk, max(m, m2));
+      const size_t f = (size_t)m * m2 + 2 * (size_t)m * kc + 2 * (size_t)m2 * kc + 64;
+      if (f > need) need = f;
+    });
+  return need;
+}
+
+// Diagonal-block inverses, the doubling temporary, the current panel's rows as TF32 head
+// and remainder (2 x b x NB), the last 256-byte aligned, then the tensor-core levels' scratch.
 size_t factor_ws_bytes(int b) {
   const size_t np = (size_t)(b + NB - 1) / NB;
-  return (np * NB * NB + doubling_tmp_floats(b) + 2 * (size_t)b * NB) * sizeof(float) + 512;
+  return (np * NB * NB + doubling_tmp_floats(b) + 2 * (size_t)b * NB + tc_levels_floats(b)) * sizeof(float) + 1024;
+}
+
+// One pair [A B; 0 D] of a doubling level on the tensor cores: T = A^-1 B, then
+// B := -T D^-1, both as W -= Z R on the 3xTF32 update kernel, over K chunks of at most
+// kTcChunk (chunk [k0, k1) of A^-1's columns touches only its rows < k1; chunk [k0, k1) of
+// D^-1's rows only columns >= k0).  A^-1, B and D^-1 sit in H (row stride b) at (i0, i0),
+// (i0, i0+m) and (i0+m, i0+m); the inverses are upper triangular and H's storage left of
+// their diagonals is stale, so the operand copies zero it.
+static cudaError_t tc_pair(float* H, int b, int i0, int m, int m2, float* tcw, pwp_stats* st, cudaStream_t s,
+                           long long* nl) {
+  auto al = [](size_t f) { return (f + 63) & ~(size_t)63; };
+  const int KC = min(kTcChunk, max(m, m2));
+  float* Tm = tcw;
+  float* Zh = Tm + al((size_t)m * m2);
+  float* Zl = Zh + al((size_t)m * KC);
+  float* Rh = Zl + al((size_t)m * KC);
+  float* Rl = Rh + al((size_t)m2 * KC);
+  float* Ainv = H + (long long)i0 * b + i0;
+  float* Bm = Ainv + m;
+  float* Dinv = H + (long long)(i0 + m) * b + i0 + m;
+  auto split = [&](const float* src, long long lds, int rows, int cols, int tri, int koff, float sign) {
+    const long long n = (long long)rows * cols;
+    const int grid = (int)min((n + 255) / 256, (long long)8 * kNumSM);
+    launch_pdl(split_kernel, dim3(grid), dim3(256), 0, s, src, lds, rows, cols, tri, koff, sign, Zh, Zl, KC,
+               (const pwp_stats*)st);
+  };
+  auto tsplit = [&](const float* src, long long lds, int krows, int ncols, int tri, int koff) {
+    launch_pdl(tsplit_kernel, dim3((ncols + 31) / 32, (krows + 31) / 32), dim3(256), 0, s, src, lds, krows, ncols,
+               tri, koff, Rh, Rl, KC, (const pwp_stats*)st);
+  };
+  cudaError_t e = cudaMemsetAsync(Tm, 0, sizeof(float) * (size_t)m * m2, s);
+  if (e != cudaSuccess) return e;
+  for (int k0 = 0; k0 < m; k0 += KC) {
+    const int kc = min(KC, m - k0), rows = min(m, k0 + kc);
+    split(Ainv + k0, b, rows, kc, 1, k0, -1.f);                     // Z = -A^-1[:, k0:k1]
+    tsplit(Bm + (long long)k0 * b, b, kc, m2, 0, 0);                // R^T = B[k0:k1, :]^T
+    if (!launch_stream_tc(kNoScore, Tm, rows, m2, m2, 0, 0, Zh, Zl, kc, KC, Rh, Rl, nullptr, nullptr, m2, nullptr,
+                          nullptr, Level2{}, st, s, &e))
+      return e != cudaSuccess ? e : cudaErrorNotSupported;
+    if (e != cudaSuccess) return e;
+    *nl += 3;
+  }
+  e = cudaMemset2DAsync(Bm, sizeof(float) * (size_t)b, 0, sizeof(float) * (size_t)m2, m, s);
+  if (e != cudaSuccess) return e;
+  for (int k0 = 0; k0 < m2; k0 += KC) {
+    const int kc = min(KC, m2 - k0);
+    split(Tm + k0, m2, m, kc, 0, 0, 1.f);                           // Z = T[:, k0:k1]
+    tsplit(Dinv + (long long)k0 * b, b, kc, m2, 1, k0);             // R^T = D^-1[k0:k1, :]^T
+    if (!launch_stream_tc(kNoScore, Bm, m, m2, b, k0, 0, Zh, Zl, kc, KC, Rh, Rl, nullptr, nullptr, m2, nullptr,
+                          nullptr, Level2{}, st, s, &e))
+      return e != cudaSuccess ? e : cudaErrorNotSupported;
+    if (e != cudaSuccess) return e;
+    *nl += 3;
+  }
+  return cudaSuccess;
 }
 
 cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void* ws, size_t ws_bytes,
@@ -545,6 +676,7 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
   float* vs_hi = reinterpret_cast<float*>(
       (reinterpret_cast<uintptr_t>(T + doubling_tmp_floats(b)) + 255) & ~(uintptr_t)255);
   float* vs_lo = vs_hi + (size_t)b * NB;
+  float* tcw = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(vs_lo + (size_t)b * NB) + 255) & ~(uintptr_t)255);
   static std::atomic<unsigned long long> attr_done{0};
   if (first_on_device(attr_done)) {
     cudaFuncSetAttribute(chol_update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * NB * 132 * 4);
@@ -570,7 +702,7 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
     // (which also factors that block) when the tensor-core path is not available
     cudaError_t e2 = cudaSuccess;
     const bool tc = launch_stream_tc(kNoScore, H, p0, p0, b, 0, 0, vs_hi, vs_lo, nb, NB, vs_hi, vs_lo, nullptr,
-                                     nullptr, 0, nullptr, nullptr, Level2{}, st, s, &e2, true);
+                                     nullptr, p0, nullptr, nullptr, Level2{}, st, s, &e2, true);
     if (e2 != cudaSuccess) return e2;
     if (tc) {
       launch_pdl(chol_diag_kernel, dim3(1), dim3(256), 2 * NB * (NB + 1) * 4, s, H, b, p0 - NB, NB, Vall + (size_t)(p - 1) * NB * NB, st);
@@ -584,7 +716,28 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
   launch_pdl(put_diag_inverses_kernel, dim3(np), dim3(256), 0, s, H, b, Vall, st);
   ++nl;
   // inverse by recursive doubling: merge [A B; 0 D] pairs of width m
+  const bool tc_levels = (b % 4) == 0 && tensor_map_encoder() != nullptr;
   for (int m = NB; m < b; m *= 2) {
+    if (m >= kTcLevel && tc_levels) {
+      cudaError_t ep = cudaSuccess;
+      for_each_pair(b, m, [&](int i0, int m2) {
+        if (ep != cudaSuccess) return;
+        if ((m2 % 4) == 0) {
+          ep = tc_pair(H, b, i0, m, m2, tcw, st, s, &nl);
+        } else {
+          const long long step = (long long)2 * m * b + 2 * m;
+          TriGemm g1{m, m2, m, H + (long long)i0 * b + i0, b, step, H + (long long)i0 * b + i0 + m, b, step,
+                     T, m2, (long long)m * m2, 1.f, 1, 0};
+          launch_trigemm(g1, 1, st, s);
+          TriGemm g2{m, m2, m2, T, m2, (long long)m * m2, H + (long long)(i0 + m) * b + i0 + m, b, step,
+                     H + (long long)i0 * b + i0 + m, b, step, -1.f, 0, 1};
+          launch_trigemm(g2, 1, st, s);
+          nl += 2;
+        }
+      });
+      if (ep != cudaSuccess) return ep;
+      continue;
+    }
     const int full = b / (2 * m);                 // pairs with both halves of width m
     const int rest = b - full * 2 * m;            // a ragged pair if rest > m
     for (int pass = 0; pass < 2; ++pass) {
