@@ -600,7 +600,7 @@ static size_t tc_levels_floats(int b) {
   for (int m = kTcLevel; m < b; m *= 2)
     for_each_pair(b, m, [&](int, int m2) {
       const size_t kc = (size_t)min(kTcChunk, max(m, m2));
-      const size_t f = (size_t)m * m2 + 2 * (size_t)m * kc + 2 * (size_t)m2 * kc + 64;
+      const size_t f = (size_t)m * m2 + 2 * (size_t)m * kc + 2 * (size_t)m2 * kc + 5 * 64;   // + rounding of 5 regions
       if (f > need) need = f;
     });
   return need;
