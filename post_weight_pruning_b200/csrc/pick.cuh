@@ -1,0 +1,317 @@
+// Exact selection of the r lowest-scoring weights of a region, as device functions run by
+// 256 threads of one CTA (the last CTA of a grid-wide pass, found with an atomic ticket).
+//
+// "Pruning LLMs with Thanos", section "Contribution two: keep the budget global and the
+// execution local", steps 1-4: the residual count r, the rescored active region, and
+// exactly that many lowest-scoring weights as the candidate set.  For SparseGPT the region
+// is the current block and r its quota.
+//
+// Keys are the bit patterns of the non-negative fp32 scores, so ordering keys orders
+// scores.  The r-th smallest key T comes from a two-level radix select: a histogram of key
+// bits [30:18] (level 1, built while the scores are produced) and one of bits [17:0] over
+// the entries of the level-1 bin (level 2).  The threshold's level-1 bin rarely moves from
+// one block to the next, so the scoring pass also builds the level-2 histogram of the
+// previous block's bin; only when this block's bin differs is the region read again.  Among
+// entries equal to T the order is (column, row) -- the pages fix none -- so when only some
+// tied entries are taken, the cut-off position inside the current block is located too.
+#pragma once
+
+#include <climits>
+
+#include "pwp_internal.cuh"
+
+namespace pwp {
+namespace pick {
+
+constexpr int kThreads = 256, kWarps = kThreads / 32;
+
+struct Shared {
+  long long warp[kWarps];
+  long long base;
+  long long take;
+  long long need;
+  int sel;
+  int last;
+};
+
+__device__ __forceinline__ long long warp_sum_ll(long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Named barrier over the kThreads participating threads.
+__device__ __forceinline__ void sync(int bar) { asm volatile("bar.sync %0, %1;" ::"r"(bar), "r"(kThreads) : "memory"); }
+
+// The bin of a histogram of NB bins holding the rank-th (1-based) entry, by threads
+// 0..kThreads-1: while the range is wider than the thread count, each warp sums one
+// kWarps-th of it (coalesced) and the range narrows to the slice holding the rank; the last
+// range is resolved by a prefix sum, one bin per thread.  *bin = -1 when the histogram holds
+// fewer entries; *before = the entries in lower bins.
+template <int NB>
+__device__ void find_rank(const unsigned int* __restrict__ hist, long long rank, int* bin, long long* before,
+                          Shared& sh, int bar, int tid) {
+  static_assert(NB >= kThreads && (NB & (NB - 1)) == 0, "power-of-two histogram");
+  const int lane = tid & 31, warp = tid >> 5;
+  int base = 0, size = NB;
+  long long below = 0;
+  while (size > kThreads) {
+    const int per = size / kWarps;
+    const unsigned int* h = hist + base + warp * per;
+    long long sum = 0;
+    for (int i = lane; i < per; i += 32) sum += h[i];
+    sum = warp_sum_ll(sum);
+    if (lane == 0) sh.warp[warp] = sum;
+    sync(bar);
+    if (tid == 0) {
+      long long cum = 0;
+      int sel = -1;
+      for (int w = 0; w < kWarps; ++w) {
+        if (rank - below > cum && rank - below <= cum + sh.warp[w]) { sel = w; break; }
+        cum += sh.warp[w];
+      }
+      sh.sel = sel;
+      sh.base = cum;
+    }
+    sync(bar);
+    const int sel = sh.sel;
+    const long long cum = sh.base;
+    sync(bar);   // the shared words are rewritten next
+    if (sel < 0) {
+      *bin = -1;
+      *before = 0;
+      return;
+    }
+    base += sel * per;
+    below += cum;
+    size = per;
+  }
+  const long long v = tid < size ? (long long)hist[base + tid] : 0;
+  long long x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sh.warp[warp] = x;
+  if (tid == 0) sh.sel = -1;
+  sync(bar);
+  long long wbase = 0;
+  for (int w = 0; w < warp; ++w) wbase += sh.warp[w];
+  const long long incl = below + wbase + x;
+  if (v > 0 && rank > incl - v && rank <= incl) {   // exactly one thread when 1 <= rank <= total
+    sh.sel = base + tid;
+    sh.base = incl - v;
+  }
+  sync(bar);
+  const int sel = sh.sel;
+  const long long bef = sh.base;
+  sync(bar);
+  *bin = sel;
+  *before = sel < 0 ? 0 : bef;
+}
+
+// Step 1 of the budget loop and the level-1 bin: take = min(r, region) with r the residual
+// global count (Thanos) or the block quota (SparseGPT); the bin of the take-th key; whether
+// the scoring pass predicted it (then the level-2 histogram is ready).  Clears the level-1
+// histogram for the next pass.
+__device__ inline void level1(Ctl* ctl, unsigned int* __restrict__ hist1, long long region_n, int global_budget,
+                              long long quota, pwp_stats* st, Shared& sh, int bar, int tid) {
+  if (tid == 0) {
+    const long long r = global_budget ? ctl->zstar - ctl->pruned : quota;
+    long long take = r < region_n ? r : region_n;
+    if (take < r) st->shortfall = 1;
+    if (take < 0) take = 0;
+    ctl->take = take;
+    ctl->mode = take > 0 ? 1 : 0;
+    ctl->l2_ready = 0;
+    ctl->dirty_pred = ctl->b1_valid;   // the scoring pass counted into the predicted histogram
+    ctl->dirty_reread = 0;
+    ctl->tie_scan = 0;
+    sh.take = take;
+  }
+  sync(bar);
+  const long long take = sh.take;
+  if (take > 0) {
+    int bin;
+    long long before;
+    find_rank<kHist1Bins>(hist1, take, &bin, &before, sh, bar, tid);
+    if (tid == 0) {
+      if (bin < 0) {
+        set_error(st, PWP_EBUDGET, kSitePick);
+        ctl->mode = 0;
+      } else {
+        const bool hit = ctl->b1_valid && ctl->b1 == (unsigned int)bin;
+        ctl->l2_ready = hit ? 1 : 0;
+        ctl->dirty_reread = hit ? 0 : 1;
+        if (!hit) st->reread_blocks += 1;
+        ctl->b1 = (unsigned int)bin;
+        ctl->b1_valid = 1;
+        ctl->r1 = (unsigned int)(take - before);
+        ctl->count_less = before;
+      }
+    }
+  }
+  sync(bar);
+  for (int i = tid; i < kHist1Bins; i += kThreads) hist1[i] = 0u;
+}
+
+// The exact key T from the level-2 histogram of the chosen level-1 bin (the predicted one
+// when it held, else the re-read one), the number m of entries tied at T that are taken,
+// and whether the cut-off among the ties has to be located.
+__device__ inline void level2(Ctl* ctl, Level2 l2, pwp_stats* st, Shared& sh, int bar, int tid) {
+  const long long r1 = ctl->r1;
+  const unsigned int* h2 = ctl->l2_ready ? l2.pred : l2.reread;
+  const unsigned int* h2s = ctl->l2_ready ? l2.pred_sum : l2.reread_sum;
+  int sb;
+  long long before_s;
+  find_rank<kHist2SumBins>(h2s, r1, &sb, &before_s, sh, bar, tid);
+  int sub = -1;
+  long long before_sub = 0;
+  if (sb >= 0)
+    find_rank<(1 << kHist2SumShift)>(h2 + ((size_t)sb << kHist2SumShift), r1 - before_s, &sub, &before_sub, sh,
+                                     bar, tid);
+  if (sb < 0 || sub < 0) {
+    if (tid == 0) {
+      set_error(st, PWP_EBUDGET, kSitePick);
+      ctl->mode = 0;
+    }
+    sync(bar);
+    return;
+  }
+  if (tid == 0) {
+    const int lo = (sb << kHist2SumShift) + sub;
+    const long long ties = h2[lo];
+    const long long count_less = ctl->count_less + before_s + before_sub;
+    const long long m = ctl->take - count_less;   // 1 <= m <= ties
+    ctl->T = (ctl->b1 << kKeyLoBits) | (unsigned int)lo;
+    ctl->ties = ties;
+    ctl->m = m;
+    ctl->count_less = count_less;
+    ctl->pstar = LLONG_MAX;
+    if (ties > 1) st->tie_blocks += 1;
+    ctl->tie_scan = m < ties ? 1 : 0;   // some but not all tied entries are taken
+  }
+  sync(bar);
+}
+
+// Counts, per block column, of the block's entries whose key equals T, over the rows
+// [r_begin, r_end) with stride r_step, added to tie_count (lane l: columns l + 32e).
+template <int SCORE>
+__device__ inline void count_ties(const Ctl* ctl, Level2 l2, const float* __restrict__ W, int b, int j, int j1,
+                                  const float* __restrict__ sc, int r_begin, int r_end, int r_step) {
+  const unsigned int T = ctl->T;
+  const int nJ = j1 - j, lane = threadIdx.x & 31;
+  constexpr int E = kMaxBlock / 32;
+  unsigned int cnt[E];
+  float scv[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    cnt[e] = 0u;
+    scv[e] = lane + 32 * e < nJ ? __ldg(sc + j + lane + 32 * e) : 0.f;
+  }
+  for (int row = r_begin; row < r_end; row += r_step) {
+    const float* wr = W + (long long)row * b + j;
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+      if (lane + 32 * e < nJ && key_of<SCORE>(wr[lane + 32 * e], scv[e]) == T) ++cnt[e];
+  }
+#pragma unroll
+  for (int e = 0; e < E; ++e)
+    if (cnt[e]) atomicAdd(&l2.tie_count[lane + 32 * e], cnt[e]);
+}
+
+// The cut-off among the tied entries: with m of them taken in (column, row) order, the
+// column holding the m-th, then its row (the threads scan that column); the per-column
+// counts are zeroed for the next block.
+template <int SCORE>
+__device__ inline void tie_cutoff(Ctl* ctl, Level2 l2, const float* __restrict__ W, int c, int b, int j, int j1,
+                                  const float* __restrict__ sc, Shared& sh, int bar, int tid) {
+  const int lane = tid & 31, warp = tid >> 5;
+  const int nJ = j1 - j;
+  const unsigned int T = ctl->T;
+  const long long m = ctl->m;
+  if (tid == 0) {
+    long long cum = 0;
+    int qstar = -1;
+    for (int qq = 0; qq < nJ; ++qq) {
+      const long long cq = l2.tie_count[qq];
+      if (cum + cq >= m) { qstar = qq; break; }
+      cum += cq;
+    }
+    sh.sel = qstar;
+    sh.need = m - cum;   // 1-based rank of the last taken tie inside column qstar
+  }
+  sync(bar);
+  const int qstar = sh.sel;
+  const long long need = sh.need;
+  sync(bar);
+  for (int i = tid; i < kMaxBlock; i += kThreads) l2.tie_count[i] = 0u;
+  if (qstar < 0) return;   // fewer than m ties inside the block: all of them are taken
+  const int q = j + qstar;
+  const float scq = __ldg(sc + q);
+  const int per = (c + kThreads - 1) / kThreads;
+  long long cnt = 0;
+  for (int i = 0; i < per; ++i) {
+    const int r = tid * per + i;
+    if (r < c && key_of<SCORE>(W[(long long)r * b + q], scq) == T) ++cnt;
+  }
+  long long x = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long yv = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += yv;
+  }
+  if (lane == 31) sh.warp[warp] = x;
+  sync(bar);
+  long long wbase = 0;
+  for (int w = 0; w < warp; ++w) wbase += sh.warp[w];
+  const long long bef = wbase + x - cnt;
+  if (bef < need && need <= bef + cnt) {
+    long long k = bef;
+    for (int i = 0; i < per; ++i) {
+      const int r = tid * per + i;
+      if (r < c && key_of<SCORE>(W[(long long)r * b + q], scq) == T) {
+        if (++k == need) {
+          ctl->pstar = (long long)qstar * c + r;
+          break;
+        }
+      }
+    }
+  }
+  sync(bar);
+}
+
+// True in exactly one CTA of the grid: the last to arrive, once every CTA's earlier global
+// writes (histogram counts) are visible to it.  Called by all threads of the CTA after its
+// last global write; the counter is reset for its next use.
+__device__ inline bool last_cta(unsigned int* ticket, Shared& sh) {
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const unsigned int t = atomicAdd(ticket, 1u);
+    sh.last = (t == gridDim.x - 1) ? 1 : 0;
+    if (sh.last) *ticket = 0u;
+  }
+  __syncthreads();
+  if (sh.last) __threadfence();
+  return sh.last != 0;
+}
+
+// After a scoring pass (all CTAs have added their level-1 counts): the last CTA takes the
+// level-1 bin and, when the predicted level-2 histogram holds, the exact threshold.
+__device__ inline void after_scoring(Ctl* ctl, unsigned int* hist1, Level2 l2, long long region_n,
+                                     int global_budget, long long quota, pwp_stats* st, Shared& sh) {
+  if (!last_cta(&ctl->ticket, sh)) return;
+  const int tid = threadIdx.x;
+  if (tid >= kThreads) return;
+  if (failed(st)) {
+    for (int i = tid; i < kHist1Bins; i += kThreads) hist1[i] = 0u;
+    return;
+  }
+  level1(ctl, hist1, region_n, global_budget, quota, st, sh, 1, tid);
+  if (ctl->mode != 0 && ctl->l2_ready) level2(ctl, l2, st, sh, 1, tid);
+}
+
+}  // namespace pick
+}  // namespace pwp

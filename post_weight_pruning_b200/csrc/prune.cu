@@ -17,7 +17,7 @@
 // the rows' z scattered into B columns.  SparseGPT's sweep has the same shape with the
 // rows of U in place of K_t.  That product is applied by the stream kernel of the next
 // block, fused with rescoring the next active region and building its histogram.
-#include "pwp_internal.cuh"
+#include "pick.cuh"
 
 namespace pwp {
 
@@ -44,6 +44,8 @@ __global__ void init_ctl_kernel(Ctl* ctl, long long zstar, pwp_stats* st, long l
   ctl->l2_ready = 0;
   ctl->dirty_pred = 0;
   ctl->dirty_reread = 0;
+  ctl->tie_scan = 0;
+  ctl->ticket = 0u;
   st->target = target;
 }
 
@@ -164,10 +166,12 @@ __global__ void __launch_bounds__(256) stream_kernel(float* __restrict__ W, int 
                                                      const float* __restrict__ Rlo, int ldr, int r_trans,
                                                      int r_upper_from, const uint8_t* __restrict__ mask,
                                                      const float* __restrict__ sc, int hist_end,
-                                                     unsigned int* __restrict__ hist1,
-                                                     const Ctl* __restrict__ ctl, unsigned int* __restrict__ h2,
-                                                     unsigned int* __restrict__ h2s, const pwp_stats* st) {
+                                                     unsigned int* __restrict__ hist1, Ctl* __restrict__ ctl,
+                                                     Level2 l2, PickArgs pk, pwp_stats* st) {
   pdl_enter();
+  unsigned int* __restrict__ h2 = l2.pred;
+  unsigned int* __restrict__ h2s = l2.pred_sum;
+  __shared__ pick::Shared psh;
   extern __shared__ unsigned int shist[];  // kHist1Bins when SCORE != 0
   __shared__ float Zs[64][33];
   __shared__ __align__(16) float Rs[32][128];
@@ -252,6 +256,8 @@ __global__ void __launch_bounds__(256) stream_kernel(float* __restrict__ W, int 
       unsigned int v = shist[i];
       if (v) atomicAdd(&hist1[i], v);
     }
+    // the last CTA to finish takes the block's level-1 bin (and threshold, when predicted)
+    if (pk.enabled) pick::after_scoring(ctl, hist1, l2, pk.region_n, pk.global_budget, pk.quota, st, psh);
   }
 }
 
@@ -346,30 +352,31 @@ static std::atomic<unsigned long long> g_attr_done{0};
 template <int SCORE>
 static void launch_stream(float* W, int c, int b, int u0, int j, int col_end, const float* Z, const float* Zlo,
                           int Bp, int ldz, const float* R, const float* Rlo, int ldr, int r_trans, int r_upper_from,
-                          const uint8_t* mask, const float* sc, int hist_end, unsigned int* hist1, const Ctl* ctl,
-                          Level2 l2, const pwp_stats* st, cudaStream_t s) {
+                          const uint8_t* mask, const float* sc, int hist_end, unsigned int* hist1, Ctl* ctl,
+                          Level2 l2, PickArgs pk, pwp_stats* st, cudaStream_t s) {
   const int smem = SCORE != kNoScore ? kHist1Bins * 4 : 0;
   const int tiles = ((col_end - u0 + 127) / 128) * ((c + 63) / 64);
   const int nsm = g_nsm.load();
   const int grid = tiles < nsm ? tiles : nsm;
   launch_pdl(stream_kernel<SCORE>, dim3(grid > 0 ? grid : 1), dim3(256), smem, s, W, c, b, u0, j, col_end, Z, Zlo, Bp, ldz, R, Rlo,
                                                              ldr, r_trans, r_upper_from, mask, sc, hist_end, hist1,
-                                                             ctl, l2.pred, l2.pred_sum, st);
+                                                             ctl, l2, pk, st);
 }
 
 static void launch_stream_any(int score, float* W, int c, int b, int u0, int j, const float* Z, const float* Zlo,
                               int Bp, int ldz, const float* R, const float* Rlo, int ldr, int r_trans,
                               int r_upper_from, const uint8_t* mask, const float* sc, int hist_end,
-                              unsigned int* hist1, const Ctl* ctl, Level2 l2, const pwp_stats* st, cudaStream_t s) {
+                              unsigned int* hist1, Ctl* ctl, Level2 l2, PickArgs pk, pwp_stats* st,
+                              cudaStream_t s) {
   if (score == kWanda)
     launch_stream<kWanda>(W, c, b, u0, j, b, Z, Zlo, Bp, ldz, R, Rlo, ldr, r_trans, r_upper_from, mask, sc, hist_end,
-                          hist1, ctl, l2, st, s);
+                          hist1, ctl, l2, pk, st, s);
   else if (score == kObs)
     launch_stream<kObs>(W, c, b, u0, j, b, Z, Zlo, Bp, ldz, R, Rlo, ldr, r_trans, r_upper_from, mask, sc, hist_end,
-                        hist1, ctl, l2, st, s);
+                        hist1, ctl, l2, pk, st, s);
   else
     launch_stream<kNoScore>(W, c, b, u0, j, b, Z, Zlo, Bp, ldz, R, Rlo, ldr, r_trans, r_upper_from, mask, sc,
-                            hist_end, hist1, ctl, l2, st, s);
+                            hist_end, hist1, ctl, l2, pk, st, s);
 }
 
 cudaError_t launch_stats_init(pwp_stats* st, cudaStream_t s) {
@@ -455,6 +462,15 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
     const int jj = t == nblk ? b : j;          // the last pass only finishes the last block
     const int pass_score = t == nblk ? kNoScore : score;
     const int hist_end = t == nblk ? b : (thanos ? b : j1);
+    // block t's selection: the scoring pass's last CTA takes the level-1 bin (and the
+    // threshold, when predicted); select_finish does the rest
+    PickArgs pk{};
+    if (pass_score != kNoScore) {
+      pk.region_n = thanos ? (long long)c * (b - j) : (long long)c * (j1 - j);
+      pk.quota = thanos ? 0 : (long long)((double)cfg->sparsity * (double)c * (double)(j1 - j));
+      pk.global_budget = thanos ? 1 : 0;
+      pk.enabled = 1;
+    }
     prof_begin(kKStream, s);
     if (t > 0) {
       // W[:, jp:b] -= Z R with R = block t-1's rows of K (Thanos) or of U (SparseGPT)
@@ -470,7 +486,7 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
         }
         cudaError_t e2 = cudaSuccess;
         done = launch_stream_tc(pass_score, Wout, c, b, b, u0, jj, pb.Zs, Zlo, Bp, B, Rh, Rl, mask, sc, hist_end,
-                                pb.hist1, pb.ctl, pb.l2, st, s, &e2);
+                                pb.hist1, pb.ctl, pb.l2, st, s, &e2, false, pk);
         if (e2 != cudaSuccess) return e2;
       }
       if (!done) {
@@ -478,28 +494,22 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
         const float* R = thanos ? pb.K_hi + (size_t)(t - 1) * b * B : H + (size_t)jp * b;
         const float* Rlo = thanos ? pb.K_lo + (size_t)(t - 1) * b * B : nullptr;
         launch_stream_any(pass_score, Wout, c, b, u0, jj, pb.Zs, Zlo, Bp, B, R, Rlo, thanos ? B : b, thanos ? 1 : 0,
-                          thanos ? -1 : jp, mask, sc, hist_end, pb.hist1, pb.ctl, pb.l2, st, s);
+                          thanos ? -1 : jp, mask, sc, hist_end, pb.hist1, pb.ctl, pb.l2, pk, st, s);
       }
       ++nl;
     } else if (score != kNoScore) {
       // first block: nothing to apply yet, only the scores of the active region
       launch_stream_any(score, Wout, c, b, j, j, pb.Zs, Zlo, 0, B, nullptr, nullptr, b, 0, -1, mask, sc, hist_end,
-                        pb.hist1, pb.ctl, pb.l2, st, s);
+                        pb.hist1, pb.ctl, pb.l2, pk, st, s);
       ++nl;
     }
     prof_end(kKStream, s);
     if (t == nblk) break;
     if (score != kNoScore) {
-      const long long region = thanos ? (long long)c * (b - j) : (long long)c * (j1 - j);
-      const long long quota = thanos ? 0 : (long long)((double)cfg->sparsity * (double)c * (double)(j1 - j));
       prof_begin(kKSelect, s);
-      launch_pick1(pb.ctl, pb.hist1, region, thanos ? 1 : 0, quota, st, s);
-      launch_refine(score, Wout, c, b, j, thanos ? b : j1, sc, pb.ctl, pb.l2, st, s);
-      launch_pick2(pb.ctl, pb.l2, st, s);
-      launch_clear_level2(score, pb.ctl, pb.l2, Wout, c, b, j, j1, sc, s);
-      launch_tie_pick(score, pb.ctl, pb.l2, Wout, c, b, j, j1, sc, st, s);
+      launch_select_finish(score, pb.ctl, pb.l2, Wout, c, b, j, j1, thanos ? b : j1, sc, st, s);
       prof_end(kKSelect, s);
-      nl += 5;
+      ++nl;
     }
     prof_begin(kKSolve, s);
     if (thanos)

@@ -81,7 +81,7 @@ struct Ctl {
   int dirty_pred;         // the predicted level-2 histogram holds counts to clear
   int dirty_reread;       // the re-read level-2 histogram holds counts to clear
   int tie_scan;           // some but not all entries tied at T are taken: locate the cut-off
-  int pad[1];
+  unsigned int ticket;    // arrivals of a grid's CTAs; the last one finishes the selection
 };
 
 // Where device-side failures are recorded (pwp_stats::status_site).
@@ -205,18 +205,20 @@ struct Level2 {
   unsigned int* tie_count;   // kMaxBlock per-column counts of entries tied at T
 };
 
-// exact selection of the `take` smallest keys of a region (select.cu)
-void launch_pick1(Ctl* ctl, unsigned int* hist1, long long region_n, int global_budget, long long quota,
-                  pwp_stats* st, cudaStream_t s);
-void launch_refine(int score, const float* W, int c, int b, int q0, int q1, const float* sc,
-                   const Ctl* ctl, Level2 l2, const pwp_stats* st, cudaStream_t s);
-void launch_pick2(Ctl* ctl, Level2 l2, pwp_stats* st, cudaStream_t s);
-// After pick2: clear the level-2 histograms the block wrote and, when only some tied
-// entries are taken, count the ties per block column (grid-wide); then find the cut-off.
-void launch_clear_level2(int score, const Ctl* ctl, Level2 l2, const float* W, int c, int b, int j, int j1,
-                         const float* sc, cudaStream_t s);
-void launch_tie_pick(int score, Ctl* ctl, Level2 l2, const float* W, int c, int b, int j, int j1, const float* sc,
-                     pwp_stats* st, cudaStream_t s);
+// Selection arguments of the scoring pass that precedes a block's selection: the region's
+// entry count and the budget (the residual global count, or the block quota); the pass's
+// last CTA takes the level-1 bin and, when predicted, the exact threshold (pick.cuh).
+struct PickArgs {
+  long long region_n;
+  long long quota;
+  int global_budget;
+  int enabled;
+};
+
+// The rest of the exact selection of a block (select.cu): the re-read when the level-1 bin
+// was not predicted, the cut-off among tied entries, and clearing the level-2 histograms.
+void launch_select_finish(int score, Ctl* ctl, Level2 l2, const float* W, int c, int b, int j, int j1, int q1,
+                          const float* sc, pwp_stats* st, cudaStream_t s);
 
 // W[:, u0:b] -= Z R on the tensor cores (stream_tc.cu), fused with zeroing the previous
 // block's removals and the level-1 histogram of the scores of columns [j, hist_end).
@@ -227,8 +229,8 @@ void launch_tie_pick(int score, Ctl* ctl, Level2 l2, const float* W, int c, int 
 // the tensor-core path.
 bool launch_stream_tc(int score, float* W, int c, int b, int ldw, int u0, int j, const float* Zhi, const float* Zlo,
                       int Bp, int ldz, const float* Rhi, const float* Rlo, const uint8_t* mask, const float* sc,
-                      int hist_end, unsigned int* hist1, const Ctl* ctl, Level2 l2, pwp_stats* st,
-                      cudaStream_t s, cudaError_t* err, bool upper = false);
+                      int hist_end, unsigned int* hist1, Ctl* ctl, Level2 l2, pwp_stats* st,
+                      cudaStream_t s, cudaError_t* err, bool upper = false, PickArgs pick = PickArgs{});
 
 // Wanda / magnitude: per-row quota or N:M groups, no weight update (rowprune.cu).  H
 // (its diagonal) or X ([n, b]) gives ||X_q|| for Wanda.

@@ -33,6 +33,7 @@
 // at their next wait, and the epilogue warps take each stop decision together through a
 // reducing barrier.  Copies and MMAs already in flight are always waited for before the
 // CTA leaves.
+#include "pick.cuh"
 #include "tc_common.cuh"
 
 namespace pwp {
@@ -92,8 +93,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __grid_constant__ CUtensorMap mrh, const __grid_constant__ CUtensorMap mrl,
                      const __grid_constant__ CUtensorMap mw, int c, int b, int u0, int j, int Bp, int upper,
                      const uint8_t* __restrict__ mask, const float* __restrict__ sc, int hist_end,
-                     unsigned int* __restrict__ hist1, const Ctl* __restrict__ ctl, unsigned int* __restrict__ h2,
-                     unsigned int* __restrict__ h2s, pwp_stats* st, long long spin) {
+                     unsigned int* __restrict__ hist1, Ctl* __restrict__ ctl, Level2 l2, PickArgs pk,
+                     pwp_stats* st, long long spin) {
+  unsigned int* __restrict__ h2 = l2.pred;
+  unsigned int* __restrict__ h2s = l2.pred_sum;
+  __shared__ pick::Shared psh;
   pdl_enter();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -370,13 +374,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const unsigned int v = shist[i];
       if (v) atomicAdd(&hist1[i], v);
     }
+    // the last CTA to finish takes the block's level-1 bin (and threshold, when predicted)
+    if (pk.enabled) pick::after_scoring(ctl, hist1, l2, pk.region_n, pk.global_budget, pk.quota, st, psh);
   }
 }
 
 template <int SCORE>
 cudaError_t launch_variant(const CUtensorMap* maps, int c, int b, int u0, int j, int Bp, int upper,
-                           const uint8_t* mask, const float* sc, int hist_end, unsigned int* hist1, const Ctl* ctl,
-                           Level2 l2, pwp_stats* st, cudaStream_t s) {
+                           const uint8_t* mask, const float* sc, int hist_end, unsigned int* hist1, Ctl* ctl,
+                           Level2 l2, PickArgs pk, pwp_stats* st, cudaStream_t s) {
   static std::atomic<unsigned long long> attr_done{0};
   if (first_on_device(attr_done)) {
     cudaError_t e = cudaFuncSetAttribute(stream_tc_kernel<SCORE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -389,9 +395,8 @@ cudaError_t launch_variant(const CUtensorMap* maps, int c, int b, int u0, int j,
   const int mt = (c + TM - 1) / TM;
   const int ntiles = upper ? mt * (mt + 1) / 2 : mt * ((b - u0 + TN - 1) / TN);
   const int grid = ntiles < nsm ? ntiles : nsm;
-  launch_pdl(stream_tc_kernel<SCORE>, dim3(grid), dim3(kThreads), SMEM_BYTES, s, maps[0], maps[1], maps[2], maps[3], maps[4], c, b, u0,
-                                                             j, Bp, upper, mask, sc, hist_end, hist1, ctl, l2.pred,
-                                                             l2.pred_sum, st, wait_limit());
+  launch_pdl(stream_tc_kernel<SCORE>, dim3(grid), dim3(kThreads), SMEM_BYTES, s, maps[0], maps[1], maps[2], maps[3],
+             maps[4], c, b, u0, j, Bp, upper, mask, sc, hist_end, hist1, ctl, l2, pk, st, wait_limit());
   return cudaGetLastError();
 }
 
@@ -413,8 +418,8 @@ bool encode_f32(CUtensorMap* map, const float* base, int inner, int rows, int ld
 
 bool launch_stream_tc(int score, float* W, int c, int b, int ldw, int u0, int j, const float* Zhi, const float* Zlo,
                       int Bp, int ldz, const float* Rhi, const float* Rlo, const uint8_t* mask, const float* sc,
-                      int hist_end, unsigned int* hist1, const Ctl* ctl, Level2 l2, pwp_stats* st, cudaStream_t s,
-                      cudaError_t* err, bool upper) {
+                      int hist_end, unsigned int* hist1, Ctl* ctl, Level2 l2, pwp_stats* st, cudaStream_t s,
+                      cudaError_t* err, bool upper, PickArgs pk) {
   *err = cudaSuccess;
   if (upper && (c != b || u0 != 0)) return false;
   // b, u0 multiples of 4: the epilogue moves whole float4s of W and 4-byte words of mask
@@ -430,11 +435,11 @@ bool launch_stream_tc(int score, float* W, int c, int b, int ldw, int u0, int j,
       !encode_f32(&maps[4], W, b, c, ldw, 32, TM))
     return false;
   if (score == kWanda)
-    *err = launch_variant<kWanda>(maps, c, b, u0, j, Bp, upper ? 1 : 0, mask, sc, hist_end, hist1, ctl, l2, st, s);
+    *err = launch_variant<kWanda>(maps, c, b, u0, j, Bp, upper ? 1 : 0, mask, sc, hist_end, hist1, ctl, l2, pk, st, s);
   else if (score == kObs)
-    *err = launch_variant<kObs>(maps, c, b, u0, j, Bp, upper ? 1 : 0, mask, sc, hist_end, hist1, ctl, l2, st, s);
+    *err = launch_variant<kObs>(maps, c, b, u0, j, Bp, upper ? 1 : 0, mask, sc, hist_end, hist1, ctl, l2, pk, st, s);
   else
-    *err = launch_variant<kNoScore>(maps, c, b, u0, j, Bp, upper ? 1 : 0, mask, sc, hist_end, hist1, ctl, l2, st, s);
+    *err = launch_variant<kNoScore>(maps, c, b, u0, j, Bp, upper ? 1 : 0, mask, sc, hist_end, hist1, ctl, l2, pk, st, s);
   return true;
 }
 
