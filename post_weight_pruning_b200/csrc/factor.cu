@@ -59,142 +59,172 @@ __global__ void __launch_bounds__(1024) damp_kernel(float* __restrict__ H, int b
 
 // Factor the nb x nb diagonal block (nb <= 64) held in A (symmetric; the upper triangle
 // is read) as A = V V^T with V upper triangular, and invert V.  256 threads.
-// Working on the reversed matrix P = J A J (J the reversal), this is the ordinary
-// Cholesky P = L L^T from the top-left, with V = J L J and V^-1 = J L^-1 J.  One
-// right-looking sweep produces both L and X = L^-1: at pivot k, column k of L is the
-// pivot column scaled by 1/sqrt(P_kk); row k of X (which already holds every earlier
-// pivot's elimination) is final once scaled the same way, and is then eliminated from
-// the rows below it, as the trailing part of P is.  Each thread keeps a 4x4 cyclic
-// sub-block of P and of X (rows ty + 16a, columns tx + 16c) in registers; pivots go two
-// per barrier, with the two pivot columns of P and pivot rows of X broadcast through
-// double-buffered shared vectors.  Entries beyond nb are an identity pad.
-// On return A's upper triangle holds V and Wi holds V^-1 (upper, zero below).
-// Returns false on a non-positive pivot (recorded in st).
-__device__ bool factor_diag_block(float (*A)[NB + 1], float (*Wi)[NB + 1], int nb, int* bad,
-                                  pwp_stats* st) {
-  __shared__ float colbuf[2][2][NB];
-  __shared__ float rowbuf[2][2][NB];
-  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  const int off = NB - nb;  // P[r][s] = A[nb-1-(r-off)][...] for r, s >= off; identity before
-  float P[4][4], X[4][4];
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int r = ty + 16 * a, s = tx + 16 * c;
-      float v;
-      if (r < off || s < off) {
-        v = (r == s) ? 1.f : 0.f;
-      } else {
-        const int ar = NB - 1 - r, as = NB - 1 - s;   // A index, in [0, nb)
-        v = ar <= as ? A[ar][as] : A[as][ar];
-      }
-      P[a][c] = v;
-      X[a][c] = (r == s) ? 1.f : 0.f;
-    }
+// Working on the reversed matrix P = J A J (J the reversal; P[r][s] = A[63-r][63-s], so
+// P's lower triangle is A's upper one and the work happens in place), this is the
+// ordinary Cholesky P = L L^T from the top-left, with V = J L J and V^-1 = J L^-1 J.
+// Blocked by 16: for each block column k, one warp factors the 16x16 diagonal block and
+// inverts it in registers (lane l holds row l of both; pivots and rows travel by
+// shuffles), then all threads form the panel L_ik = P_ik X_kk^T (X = L^-1) below it and
+// the trailing update P_ij -= L_ik L_jk^T; finally the off-diagonal blocks of X follow,
+// X_ik = -X_ii sum_{k <= t < i} L_it X_tk, by growing distance from the diagonal.  Rows
+// and columns beyond nb are an identity pad.  On return A's upper triangle holds V and Wi
+// holds V^-1 (upper, zero below).  Returns false on a non-positive pivot (recorded in st).
+__device__ bool factor_diag_block(float (*A)[NB + 1], float (*Wi)[NB + 1], int nb, int* bad, pwp_stats* st) {
+  constexpr int BS = 16, NBK = NB / BS;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  auto P = [&](int r, int c) -> float& { return A[NB - 1 - r][NB - 1 - c]; };
+  auto X = [&](int r, int c) -> float& { return Wi[NB - 1 - r][NB - 1 - c]; };
+  // identity pad beyond nb (A indices >= nb) and X = 0
+  for (int idx = tid; idx < NB * NB; idx += blockDim.x) {
+    const int i = idx / NB, jc = idx % NB;
+    if (i <= jc && jc >= nb) A[i][jc] = (i == jc) ? 1.f : 0.f;
+    Wi[i][jc] = 0.f;
+  }
   if (tid == 0) *bad = 0;
-  // two pivots k, k+1 per barrier (k = 16 kb + kk, kk even, so both sit in register block
-  // kb, a compile-time index): columns k and k+1 of P and rows k and k+1 of X are
-  // broadcast as they stand, and every thread rebuilds column k+1 and row k+1 after
-  // pivot k from them
+  __syncthreads();
+  for (int kb = 0; kb < NBK; ++kb) {
+    const int k0 = BS * kb;
+    if (warp == 0) {
+      // 16x16 diagonal block: lane l (< 16) holds row l of the block and of its inverse
+      const int l = lane & (BS - 1);
+      const bool act = lane < BS;
+      float d[BS], x[BS];
 #pragma unroll
-  for (int kb = 0; kb < 4; ++kb)
-  for (int kk = 0; kk < 16; kk += 2) {
-    const int k = 16 * kb + kk;
-    const int par = (k >> 1) & 1;
-    float* cb0 = colbuf[par][0];
-    float* cb1 = colbuf[par][1];
-    float* rb0 = rowbuf[par][0];
-    float* rb1 = rowbuf[par][1];
-    if (tx == kk) {
+      for (int c = 0; c < BS; ++c) {
+        d[c] = (act && c <= l) ? P(k0 + l, k0 + c) : 0.f;
+        x[c] = (c == l) ? 1.f : 0.f;
+      }
+      bool ok = true;
 #pragma unroll
-      for (int a = 0; a < 4; ++a) cb0[ty + 16 * a] = P[a][kb];
-    }
-    if (tx == kk + 1) {
+      for (int c = 0; c < BS; ++c) {
+        const float piv = __shfl_sync(0xffffffffu, d[c], c);
+        ok = ok && (piv > 0.f) && isfinite(piv);
+        const float il = rsqrtf(piv);
+        if (l == c) {
+          d[c] = piv * il;
 #pragma unroll
-      for (int a = 0; a < 4; ++a) cb1[ty + 16 * a] = P[a][kb];
-    }
-    if (ty == kk) {
+          for (int t = 0; t <= c; ++t) x[t] *= il;
+        } else if (l > c) {
+          d[c] *= il;
+        }
 #pragma unroll
-      for (int c = 0; c < 4; ++c) rb0[tx + 16 * c] = X[kb][c];
-    }
-    if (ty == kk + 1) {
+        for (int c2 = c + 1; c2 < BS; ++c2) {
+          const float lc2 = __shfl_sync(0xffffffffu, d[c], c2);   // L[c2][c]
+          if (l > c) d[c2] = fmaf(-d[c], lc2, d[c2]);
+        }
 #pragma unroll
-      for (int c = 0; c < 4; ++c) rb1[tx + 16 * c] = X[kb][c];
+        for (int t = 0; t <= c; ++t) {
+          const float xc = __shfl_sync(0xffffffffu, x[t], c);     // X[c][t], final
+          if (l > c) x[t] = fmaf(-d[c], xc, x[t]);
+        }
+      }
+      if (act) {
+#pragma unroll
+        for (int c = 0; c < BS; ++c)
+          if (c <= l) {
+            P(k0 + l, k0 + c) = d[c];
+            X(k0 + l, k0 + c) = x[c];
+          }
+      }
+      if (!ok && lane == 0) *bad = 1;
     }
     __syncthreads();
-    const float d0 = cb0[k];
-    const float il0 = rsqrtf(d0);
-    const float l10 = cb0[k + 1] * il0;                 // L[k+1][k]
-    const float d1 = cb1[k + 1] - l10 * l10;            // pivot k+1 after pivot k
-    if (!(d0 > 0.f) || !isfinite(d0) || !(d1 > 0.f) || !isfinite(d1)) {   // uniform
-      if (tid == 0) {
-        *bad = 1;
-        set_error(st, PWP_ENOTSPD, kSiteCholDiag);
-      }
+    if (*bad) {
+      if (tid == 0) set_error(st, PWP_ENOTSPD, kSiteCholDiag);
       return false;
     }
-    const float il1 = rsqrtf(d1);
-    float lr0[4], lr1[4], cs0[4], cs1[4], x0[4], x1[4];
+    // panel below the block: L_ik = P_ik X_kk^T, i > kb
+    const int nbelow = NBK - 1 - kb;
+    float lv[NBK - 1];
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      lr0[a] = cb0[ty + 16 * a] * il0;                                // L[r][k]
-      lr1[a] = fmaf(-lr0[a], l10, cb1[ty + 16 * a]) * il1;            // L[r][k+1]
-    }
+    for (int m = 0; m < NBK - 1; ++m) {
+      lv[m] = 0.f;
+      const int e = tid + blockDim.x * m;
+      if (m < nbelow && e < nbelow * BS * BS) {
+        const int ib = kb + 1 + e / (BS * BS), r = (e / BS) % BS, c = e % BS;
+        float v = 0.f;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      cs0[c] = cb0[tx + 16 * c] * il0;                                // L[s][k]
-      cs1[c] = fmaf(-cs0[c], l10, cb1[tx + 16 * c]) * il1;            // L[s][k+1]
-      x0[c] = rb0[tx + 16 * c] * il0;                                 // X[k][s], final
-      x1[c] = fmaf(-l10, x0[c], rb1[tx + 16 * c]) * il1;              // X[k+1][s], final
-    }
-    // r = ty + 16a, s = tx + 16c: relations to k and k+1 are compile-time except in
-    // register block kb
-    const bool ty_gt0 = ty > kk, ty_eq0 = ty == kk, ty_gt1 = ty > kk + 1, ty_eq1 = ty == kk + 1;
-    const bool tx_eq0 = tx == kk, tx_eq1 = tx == kk + 1, tx_gt1 = tx > kk + 1;
-#pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      if (a < kb) continue;                                         // rows above both pivots
-      const bool r_ge0 = a > kb || ty_gt0 || ty_eq0, r_ge1 = a > kb || ty_gt1 || ty_eq1;
-      const bool r_gt1 = a > kb || ty_gt1, r_eq0 = a == kb && ty_eq0, r_eq1 = a == kb && ty_eq1;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        if (c >= kb) {                                              // P: columns >= k
-          const bool s_eq0 = c == kb && tx_eq0, s_eq1 = c == kb && tx_eq1, s_gt1 = c > kb || tx_gt1;
-          if (s_eq0) {
-            if (r_ge0) P[a][c] = lr0[a];                            // column k of L
-          } else if (s_eq1) {
-            if (r_ge1) P[a][c] = lr1[a];                            // column k+1 of L
-          } else if (r_gt1 && s_gt1) {
-            P[a][c] = fmaf(-lr1[a], cs1[c], fmaf(-lr0[a], cs0[c], P[a][c]));
-          }
-        }
-        if (c <= kb) {                                              // X rows k, k+1 are zero right of k+1
-          if (r_eq0) X[a][c] = x0[c];
-          else if (r_eq1) X[a][c] = x1[c];
-          else if (r_gt1) X[a][c] = fmaf(-lr1[a], x1[c], fmaf(-lr0[a], x0[c], X[a][c]));
-        }
+        for (int t = 0; t < BS; ++t) v = fmaf(P(BS * ib + r, k0 + t), X(k0 + c, k0 + t), v);
+        lv[m] = v;
       }
     }
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < NBK - 1; ++m) {
+      const int e = tid + blockDim.x * m;
+      if (m < nbelow && e < nbelow * BS * BS) {
+        const int ib = kb + 1 + e / (BS * BS), r = (e / BS) % BS, c = e % BS;
+        P(BS * ib + r, k0 + c) = lv[m];
+      }
+    }
+    __syncthreads();
+    // trailing update of the blocks (i, j), kb < j <= i
+    const int nt = nbelow * (nbelow + 1) / 2;
+    for (int e = tid; e < nt * BS * BS; e += blockDim.x) {
+      int blk = e / (BS * BS);
+      const int r = (e / BS) % BS, c = e % BS;
+      int i = kb + 1, jb = kb + 1;
+      while (blk > i - (kb + 1)) { blk -= i - kb; ++i; }   // blocks of row i: j = kb+1 .. i
+      jb = kb + 1 + blk;
+      float v = P(BS * i + r, BS * jb + c);
+#pragma unroll
+      for (int t = 0; t < BS; ++t) v = fmaf(-P(BS * i + r, k0 + t), P(BS * jb + c, k0 + t), v);
+      P(BS * i + r, BS * jb + c) = v;
+    }
+    __syncthreads();
   }
-  __syncthreads();  // every thread is done reading A
-  // back to A's orientation: V[i][j] = L[NB-1-i][NB-1-j], V^-1[i][j] = X[NB-1-i][NB-1-j]
+  // off-diagonal blocks of X = L^-1, by distance dd from the diagonal (each block's sum is
+  // staged in the block itself, still zero, before the product with X_ii)
+  for (int dd = 1; dd < NBK; ++dd) {
+    const int nbk = NBK - dd;   // blocks (k + dd, k), k = 0 .. nbk-1
+    float tv[NBK - 1];
+    // tmp(k) = sum_{t = k}^{k+dd-1} L_{k+dd, t} X_{t, k}
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+    for (int m = 0; m < NBK - 1; ++m) {
+      tv[m] = 0.f;
+      const int e = tid + blockDim.x * m;
+      if (m < nbk && e < nbk * BS * BS) {
+        const int kk = e / (BS * BS), r = (e / BS) % BS, c = e % BS, ib = kk + dd;
+        float v = 0.f;
+        for (int tb = kk; tb < ib; ++tb)
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int r = ty + 16 * a, s = tx + 16 * c;
-      if (r >= off && s >= off) {                      // inside the nb block
-        const int i = NB - 1 - r, jj = NB - 1 - s;     // the same reversal as on load
-        if (i <= jj) {
-          A[i][jj] = P[a][c];
-          Wi[i][jj] = X[a][c];
-        } else {
-          Wi[i][jj] = 0.f;
-        }
+          for (int u = 0; u < BS; ++u) v = fmaf(P(BS * ib + r, BS * tb + u), X(BS * tb + u, BS * kk + c), v);
+        tv[m] = v;
       }
     }
-  __syncthreads();
+    // stage tmp in the (still zero) X block itself, then X_ik = -X_ii tmp
+#pragma unroll
+    for (int m = 0; m < NBK - 1; ++m) {
+      const int e = tid + blockDim.x * m;
+      if (m < nbk && e < nbk * BS * BS) {
+        const int kk = e / (BS * BS), r = (e / BS) % BS, c = e % BS, ib = kk + dd;
+        X(BS * ib + r, BS * kk + c) = tv[m];
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < NBK - 1; ++m) {
+      tv[m] = 0.f;
+      const int e = tid + blockDim.x * m;
+      if (m < nbk && e < nbk * BS * BS) {
+        const int kk = e / (BS * BS), r = (e / BS) % BS, c = e % BS, ib = kk + dd;
+        float v = 0.f;
+#pragma unroll
+        for (int u = 0; u < BS; ++u) v = fmaf(X(BS * ib + r, BS * ib + u), X(BS * ib + u, BS * kk + c), v);
+        tv[m] = -v;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < NBK - 1; ++m) {
+      const int e = tid + blockDim.x * m;
+      if (m < nbk && e < nbk * BS * BS) {
+        const int kk = e / (BS * BS), r = (e / BS) % BS, c = e % BS, ib = kk + dd;
+        X(BS * ib + r, BS * kk + c) = tv[m];
+      }
+    }
+    __syncthreads();
+  }
   return true;
 }
 
