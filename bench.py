@@ -575,7 +575,9 @@ def _device_block_inputs(dev, seed=0):
             if dist == "gaussian":
                 x = torch.randn((r1 - r0, b), generator=g, device=dev)
             else:
-                u = torch.rand((r1 - r0, b), generator=g, device=dev) - 0.5
+                # u uniform on the open interval (-1/2, 1/2): rand can return 0, and
+                # u = -1/2 would give log1p(-1) = -inf
+                u = torch.rand((r1 - r0, b), generator=g, device=dev).clamp_(1e-7, 1.0 - 1e-7) - 0.5
                 x = -torch.sign(u) * torch.log1p(-2.0 * u.abs()) / math.sqrt(2.0)
                 near = torch.rand((r1 - r0, b), generator=g, device=dev) < 0.3
                 x = torch.where(near, x * 1e-2, x)

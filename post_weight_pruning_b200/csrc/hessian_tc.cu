@@ -16,8 +16,8 @@
 //     H[i][j] and its mirror H[j][i] for i <= j, scaled by 2.
 // The tensor core's accumulation into tensor memory does not round to nearest: a long
 // chain of additions of positive terms (the diagonal of H is a sum of squares) drifts
-// low in proportion to the chain's length.  So no accumulator takes more than SPAN
-// tokens: the MMAs of each span of SPAN tokens start a fresh accumulator, alternating
+// low in proportion to the chain's length.  So no accumulator takes more than 512
+// tokens: the MMAs of each span of 512 tokens start a fresh accumulator, alternating
 // between two 256-column halves of tensor memory, and while the MMAs fill one half the
 // epilogue warps add the other, finished half into their running sums (each thread
 // holds 128 entries of one tile row) with ordinary round-to-nearest fp32 additions.
@@ -31,7 +31,7 @@ namespace pwp {
 namespace {
 
 constexpr int TM = 128, TN = 256, TK = 64, STAGES = 4;
-constexpr int SPAN_KT = 4;                       // k-tiles (of TK tokens) per accumulator span
+constexpr int SPAN_KT = 8;                       // k-tiles (of TK tokens) per accumulator span
 constexpr int BOX_BYTES = 64 * TK * 2;           // one 64-feature x 64-token bf16 box
 constexpr int A_BYTES = TM * TK * 2;             // 2 boxes
 constexpr int B_BYTES = TN * TK * 2;             // 4 boxes
