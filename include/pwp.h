@@ -72,7 +72,16 @@ typedef enum { PWP_BF16 = 0, PWP_FP32 = 1 } pwp_dtype;
  *   sparsity : fraction of weights removed, 0 <= sparsity < 1 (ignored for PWP_NM).
  *   block    : column block width B, 1 <= B <= 128; for PWP_NM a multiple of nm_m
  *              (Thanos and SparseGPT only).
- *   damp     : lambda = damp * mean(diag H) of the undamped H, damp >= 0. */
+ *   damp     : lambda = damp * mean(diag H) of the undamped H, damp >= 0.
+ *   alpha    : fraction of rows kept dense as outliers, 0 <= alpha < 1 (Thanos and
+ *              SparseGPT; 0 for the others).  "Pruning LLMs with Thanos", section
+ *              "Thanos versus SparseGPT on LLaMA-3 8B": alpha = 0.1 keeps 10% of the rows,
+ *              so 2:4 and 4:8 prune 45% of the layer instead of 50%.  The page does not say
+ *              which rows; here the floor(alpha * c) rows with the largest
+ *              sum_q W_kq^2 ||X_q||^2 (ties: lower row first) are returned unchanged (mask 0)
+ *              and the other rows are pruned as a layer of their own with this
+ *              configuration (the unstructured budget is floor(sparsity * rows * b) of their
+ *              weights). */
 typedef struct {
     int32_t method;
     int32_t pattern;
@@ -81,6 +90,7 @@ typedef struct {
     float sparsity;
     int32_t block;
     float damp;
+    float alpha;
 } pwp_config;
 
 /* Device-resident results of one prune call (the caller allocates it in device

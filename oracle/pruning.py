@@ -44,7 +44,7 @@ __all__ = [
     "gram", "hessian", "damp_hessian", "inverse_cholesky_upper", "active_inverse",
     "conditioned_diag", "wanda_scores", "obs_scores", "lowest_global", "nm_mask",
     "thanos_row_update", "sparsegpt_block", "prune_layer", "recon_loss", "row_losses",
-    "row_quota_mask", "prune_no_update", "bf16_bits_rne", "pack_24",
+    "row_quota_mask", "prune_no_update", "bf16_bits_rne", "pack_24", "outlier_rows", "prune_layer_alpha",
 ]
 
 
@@ -464,3 +464,46 @@ def pack_24(What: np.ndarray, mask: np.ndarray):
             meta[k, g // 8] |= np.uint32((kept[0] | (kept[1] << 2)) << (4 * (g % 8)))
     return values, meta
 
+
+
+# ----------------------------------------------------------------------------- outlier rows (alpha)
+
+def outlier_rows(W, g_diag, alpha):
+    """The rows kept dense by the alpha variant: floor(alpha * c) rows of W with the largest
+    sum over q of (W_kq * ||X_q||)^2 = W_kq^2 G_qq (ties: the lower row first).
+
+    [THANOS] "Thanos versus SparseGPT on LLaMA-3 8B": the alpha = 0.1 variant keeps 10% of
+    the rows as outliers, which lowers the total N:M sparsity from 50% to 45%.  The page does
+    not say how the rows are chosen; the reading here ranks a row by the squared norm of its
+    activation-aware scores (the scores of [BLOG] "Wanda..." that Thanos rescores with,
+    [THANOS] "Contribution two").  Returns a boolean array over rows."""
+    W = np.asarray(W, dtype=np.float64)
+    c = W.shape[0]
+    n_out = int(math.floor(float(alpha) * c))
+    score = (W ** 2) @ np.asarray(g_diag, dtype=np.float64)
+    order = np.lexsort((np.arange(c), -score))      # by score descending, then row ascending
+    out = np.zeros(c, dtype=bool)
+    out[order[:n_out]] = True
+    return out
+
+
+def prune_layer_alpha(W, *, Xt=None, H=None, alpha=0.0, **kw):
+    """The alpha variant of ``prune_layer``: the outlier rows (``outlier_rows``) keep their
+    weights, and the other rows are pruned as a layer of their own with the same
+    configuration (for the unstructured global budget: floor(sparsity * rows * b) of their
+    weights).  Returns ``prune_layer``'s dict for the whole layer (W, mask, loss, pruned,
+    zstar) plus "outliers" and "inner", the pruned rows' own result."""
+    W0 = np.array(W, dtype=np.float64)
+    if H is None:
+        H = hessian(Xt)
+    H = np.asarray(H, dtype=np.float64)
+    g = 0.5 * np.diag(H)
+    out = outlier_rows(W0, g, alpha)
+    keep = ~out
+    inner = prune_layer(W0[keep], H=H, **kw)
+    What = W0.copy()
+    What[keep] = inner["W"]
+    mask = np.zeros(W0.shape, dtype=bool)
+    mask[keep] = inner["mask"]
+    return {"W": What, "mask": mask, "loss": recon_loss(W0, What, 0.5 * H), "outliers": out, "inner": inner,
+            "pruned": inner["pruned"], "zstar": inner["zstar"]}

@@ -34,7 +34,7 @@ BF16, FP32 = 0, 1
 class Config(ctypes.Structure):
     _fields_ = [("method", ctypes.c_int32), ("pattern", ctypes.c_int32), ("nm_n", ctypes.c_int32),
                 ("nm_m", ctypes.c_int32), ("sparsity", ctypes.c_float), ("block", ctypes.c_int32),
-                ("damp", ctypes.c_float)]
+                ("damp", ctypes.c_float), ("alpha", ctypes.c_float)]
 
 
 class Stats(ctypes.Structure):
@@ -98,14 +98,15 @@ def _check(status, where):
         raise PwpError(status, where)
 
 
-def config(method="thanos", pattern="unstructured", nm=(2, 4), sparsity=0.5, block=128, damp=0.01) -> Config:
+def config(method="thanos", pattern="unstructured", nm=(2, 4), sparsity=0.5, block=128, damp=0.01,
+           alpha=0.0) -> Config:
     m = METHODS[method] if isinstance(method, str) else int(method)
     if isinstance(pattern, str):
         p = {"unstructured": UNSTRUCTURED, "nm": NM}[pattern]
     else:
         p = int(pattern)
     n_keep, m_grp = nm if p == NM else (0, 0)
-    return Config(m, p, int(n_keep), int(m_grp), float(sparsity), int(block), float(damp))
+    return Config(m, p, int(n_keep), int(m_grp), float(sparsity), int(block), float(damp), float(alpha))
 
 
 def workspace_bytes(cfg: Config, c: int, b: int) -> int:
@@ -217,7 +218,7 @@ def make_workspace(cfg: Config, c, b, device="cuda") -> Workspace:
 
 
 def prune_layer(W, *, H=None, X=None, sparsity=0.5, pattern="unstructured", nm=(2, 4), block=128,
-                damp=0.01, method="thanos", W_out=None, mask=None, workspace=None, stats=None,
+                damp=0.01, method="thanos", alpha=0.0, W_out=None, mask=None, workspace=None, stats=None,
                 stream=None, check=True):
     """Prune one layer on the GPU.
 
@@ -244,7 +245,7 @@ def prune_layer(W, *, H=None, X=None, sparsity=0.5, pattern="unstructured", nm=(
         raise ValueError(f"workspace: {workspace.nbytes} bytes claimed, tensor holds "
                          f"{workspace.ws.numel() * workspace.ws.element_size()}")
     _need_cuda(W, H, X, W_out, mask, stats, workspace.ws if workspace is not None else None)
-    cfg = config(method, pattern, nm, sparsity, block, damp)
+    cfg = config(method, pattern, nm, sparsity, block, damp, alpha)
     if workspace is None:
         workspace = make_workspace(cfg, c, b, W.device)
     if W_out is None:

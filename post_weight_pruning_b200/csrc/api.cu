@@ -29,6 +29,7 @@ static bool valid_cfg(const pwp_config* cfg, int32_t c, int32_t b) {
   const bool second_order = cfg->method == PWP_THANOS || cfg->method == PWP_SPARSEGPT;
   if (second_order && (cfg->block < 1 || cfg->block > kMaxBlock)) return false;
   if (second_order && !(cfg->damp >= 0.f && cfg->damp < 1e30f)) return false;
+  if (!(cfg->alpha >= 0.f && cfg->alpha < 1.f) || (!second_order && cfg->alpha != 0.f)) return false;
   if (cfg->pattern == PWP_UNSTRUCTURED) {
     if (!(cfg->sparsity >= 0.f && cfg->sparsity < 1.f)) return false;
   } else if (cfg->pattern == PWP_NM) {

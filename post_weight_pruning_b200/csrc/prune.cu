@@ -309,6 +309,13 @@ static size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
 
 size_t prune_ws_layout(const pwp_config* cfg, int c, int b, PruneBuffers* pb, char* base) {
   if (cfg->method == PWP_WANDA || cfg->method == PWP_MAGNITUDE) return no_update_ws_bytes(b);
+  const int n_out = alpha_rows(cfg, c);
+  if (n_out > 0) {
+    // the compact prune of the kept rows comes first (launch_prune lays it out itself)
+    pwp_config ic = *cfg;
+    ic.alpha = 0.f;
+    return alpha_ws_bytes(prune_ws_layout(&ic, c - n_out, b, nullptr, nullptr), c, b, n_out);
+  }
   const int B = cfg->block;
   const int nblk = (b + B - 1) / B;
   const bool thanos = cfg->method == PWP_THANOS;
@@ -393,6 +400,14 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
   if (cfg->method == PWP_WANDA || cfg->method == PWP_MAGNITUDE)
     return launch_no_update(cfg, W, wtype, c, b, cfg->method == PWP_WANDA ? H : nullptr, nullptr, 0, 0, Wout,
                             mask, ws, st, stats_ready, s);
+  const int n_out = alpha_rows(cfg, c);
+  if (n_out > 0) {
+    pwp_config ic = *cfg;
+    ic.alpha = 0.f;
+    const size_t inner = prune_ws_layout(&ic, c - n_out, b, nullptr, nullptr);
+    return launch_prune_alpha(cfg, W, wtype, c, b, H, Wout, mask, ws, inner, st, s, stats_ready, n_out,
+                              &launch_prune);
+  }
   PruneBuffers pb;
   const int B = cfg->block;
   prune_ws_layout(cfg, c, b, &pb, (char*)ws);

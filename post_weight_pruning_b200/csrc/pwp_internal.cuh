@@ -239,6 +239,15 @@ cudaError_t launch_no_update(const pwp_config* cfg, const void* W, int wtype, in
                              const void* X, int xtype, long long n, float* Wout, uint8_t* mask, void* ws,
                              pwp_stats* st, bool stats_ready, cudaStream_t s);
 
+// the alpha variant (alpha.cu): outlier rows kept dense, the others pruned compactly
+int alpha_rows(const pwp_config* cfg, int c);
+size_t alpha_ws_bytes(size_t inner, int c, int b, int n_out);
+cudaError_t launch_prune_alpha(const pwp_config* cfg, const void* W, int wtype, int c, int b, float* H, float* Wout,
+                               uint8_t* mask, void* ws, size_t inner_bytes, pwp_stats* st, cudaStream_t s,
+                               bool stats_ready, int n_out,
+                               cudaError_t (*inner_prune)(const pwp_config*, const void*, int, int, int, float*,
+                                                          float*, uint8_t*, void*, pwp_stats*, cudaStream_t, bool));
+
 // compressed 2:4 storage (pack24.cu)
 cudaError_t launch_pack24(const float* What, const uint8_t* mask, int c, int b, uint16_t* values, uint32_t* meta,
                           pwp_stats* st, cudaStream_t s);

@@ -39,7 +39,8 @@ def test_status_strings():
 @pytest.mark.parametrize("kw", [
     dict(sparsity=1.0), dict(sparsity=-0.1), dict(block=0), dict(block=129),
     dict(pattern="nm", nm=(2, 3)), dict(pattern="nm", nm=(4, 4)), dict(pattern="nm", nm=(0, 4)),
-    dict(pattern="nm", nm=(2, 4), block=6), dict(damp=-1.0), dict(method=7),
+    dict(pattern="nm", nm=(2, 4), block=6), dict(damp=-1.0), dict(method=7), dict(alpha=1.0), dict(alpha=-0.1),
+    dict(method="wanda", alpha=0.1),
 ])
 def test_invalid_configs_have_no_workspace(kw):
     cfg = pwp.config(**kw)
@@ -137,3 +138,14 @@ def test_wait_limit_setter_returns_the_previous_limit_and_restores_the_default()
     assert pwp.set_wait_limit(12345) == 0
     assert pwp.set_wait_limit(-5) == 12345
     assert pwp.set_wait_limit(-1) == default
+
+
+def test_alpha_workspace_holds_the_compact_layer():
+    """With alpha > 0 the workspace holds the prune of the c - floor(alpha c) kept rows plus
+    their compact copy (fp32 weights and mask) and the per-row scores, flags and positions."""
+    base = pwp.workspace_bytes(pwp.config(block=32), 36, 64)
+    got = pwp.workspace_bytes(pwp.config(block=32, alpha=0.1), 40, 64)   # floor(4.0) = 4 outlier rows
+    al = lambda x: (x + 255) // 256 * 256
+    assert got == al(base) + al(36 * 64 * 4) + al(36 * 64) + al(40 * 8) + 2 * al(40 * 4)
+    # alpha too small to keep a row: the plain workspace
+    assert pwp.workspace_bytes(pwp.config(block=32, alpha=0.01), 40, 64) == pwp.workspace_bytes(pwp.config(block=32), 40, 64)

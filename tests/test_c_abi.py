@@ -16,11 +16,11 @@ PROGRAM = r"""
 #include "pwp.h"
 
 int main(void) {
-    pwp_config cfg = {PWP_THANOS, PWP_UNSTRUCTURED, 0, 0, 0.5f, 128, 0.01f};
+    pwp_config cfg = {PWP_THANOS, PWP_UNSTRUCTURED, 0, 0, 0.5f, 128, 0.01f, 0.0f};
     size_t ws = pwp_workspace_bytes(&cfg, 4096, 4096);
-    pwp_config nm = {PWP_THANOS, PWP_NM, 2, 4, 0.0f, 128, 0.01f};
-    pwp_config bad = {PWP_THANOS, PWP_NM, 3, 6, 0.0f, 128, 0.01f};       /* m not a power of two */
-    pwp_config wanda = {PWP_WANDA, PWP_UNSTRUCTURED, 0, 0, 0.5f, 0, 0.0f}; /* block ignored */
+    pwp_config nm = {PWP_THANOS, PWP_NM, 2, 4, 0.0f, 128, 0.01f, 0.0f};
+    pwp_config bad = {PWP_THANOS, PWP_NM, 3, 6, 0.0f, 128, 0.01f, 0.0f};       /* m not a power of two */
+    pwp_config wanda = {PWP_WANDA, PWP_UNSTRUCTURED, 0, 0, 0.5f, 0, 0.0f, 0.0f}; /* block ignored */
     char W[16];
     printf("version %d\n", (int)pwp_version());
     printf("ws %zu\n", ws);
@@ -33,6 +33,7 @@ int main(void) {
                                                     (uint8_t*)W, NULL, 0, (pwp_stats*)W, NULL));
     printf("status %s\n", pwp_status_string(PWP_ENOTSPD));
     printf("stats %zu\n", sizeof(pwp_stats));
+    printf("config %zu\n", sizeof(pwp_config));
     return 0;
 }
 """
@@ -67,3 +68,4 @@ def test_header_is_plain_c_and_host_calls_work(program):
     assert int(program["eworkspace"]) == 3
     assert program["status"] == "damped Hessian is not positive definite"
     assert int(program["stats"]) == ctypes.sizeof(pwp.Stats)
+    assert int(program["config"]) == ctypes.sizeof(pwp.Config)

@@ -580,3 +580,42 @@ def test_fixed_mask_replay_records_the_selection_of_the_replayed_state():
     other = oracle.prune_layer(W, Xt=Xt, sparsity=0.5, block=5, fixed_mask=flipped)
     diff = np.argwhere(other["blocks"][0]["chosen"] != flipped[:, :5])
     assert diff.tolist() == [[k, q]]
+
+
+# --------------------------------------------------------------------------- outlier rows (alpha)
+
+def test_alpha_keeps_floor_alpha_c_rows_dense_and_gives_the_stated_total_sparsity():
+    """alpha = 0.1 keeps 10% of the rows dense; with 2:4 and 4:8 on the other rows the total
+    sparsity is 45% instead of 50% ("Thanos versus SparseGPT on LLaMA-3 8B")."""
+    rng = np.random.default_rng(61)
+    c, b = 40, 16
+    Xt = rng.normal(size=(48, b))
+    W = rng.normal(0, 0.02, size=(c, b))
+    for nm in ((2, 4), (4, 8)):
+        r = oracle.prune_layer_alpha(W, Xt=Xt, alpha=0.1, pattern="nm", nm=nm, block=8)
+        assert int(r["outliers"].sum()) == 4
+        assert np.array_equal(r["W"][r["outliers"]], W[r["outliers"]])
+        assert not r["mask"][r["outliers"]].any()
+        assert r["mask"].sum() / r["mask"].size == pytest.approx(0.45)
+    r = oracle.prune_layer_alpha(W, Xt=Xt, alpha=0.1, sparsity=0.5, block=8)
+    assert int(r["mask"].sum()) == math.floor(0.5 * 36 * b) == r["zstar"]
+
+
+def test_alpha_outlier_rows_are_the_largest_activation_weighted_rows():
+    """The dense rows are those with the largest sum of (W_kq ||X_q||)^2, by brute force over
+    the rows (ties between equal rows: the lower row first); alpha = 0 changes nothing."""
+    rng = np.random.default_rng(62)
+    c, b = 23, 10
+    Xt = rng.normal(size=(30, b)) * rng.uniform(0.2, 3.0, size=b)
+    W = rng.normal(size=(c, b))
+    W[7] = W[3]                                  # an exact tie between two rows
+    g = np.einsum("tq,tq->q", Xt, Xt)
+    out = oracle.outlier_rows(W, g, 0.2)         # floor(4.6) = 4 rows
+    score = [sum((W[k, q] * math.sqrt(g[q])) ** 2 for q in range(b)) for k in range(c)]
+    ranked = sorted(range(c), key=lambda k: (-score[k], k))
+    assert sorted(np.flatnonzero(out).tolist()) == sorted(ranked[:4])
+    tied = oracle.outlier_rows(W[[3, 7]], g, 0.5)
+    assert tied.tolist() == [True, False]
+    plain = oracle.prune_layer(W, Xt=Xt, sparsity=0.5, block=5)
+    zero = oracle.prune_layer_alpha(W, Xt=Xt, alpha=0.0, sparsity=0.5, block=5)
+    assert np.array_equal(zero["W"], plain["W"]) and np.array_equal(zero["mask"], plain["mask"])
