@@ -160,6 +160,61 @@ pwp_status pwp_prune_layer_x(const pwp_config* cfg, const void* W_dev, int32_t w
                              int64_t n, float* H_dev, float* W_out_dev, uint8_t* mask_dev,
                              void* ws, size_t ws_bytes, pwp_stats* stats_dev, void* stream);
 
+/* Stepwise sweep: one layer's rows sharded over ranks (one process per GPU), pruned with the
+ * unstructured budget counted over all ranks' rows ("Pruning LLMs with Thanos", section
+ * "Contribution two: keep the budget global and the execution local": the budget couples
+ * rows only through each block's threshold; section "The layer-reconstruction lens": the
+ * rest of the work is per row).  The caller drives the block loop of pwp_prune_layer and,
+ * between the steps, combines three buffers over ranks (pwp_sweep_buffers):
+ *   for t = 0 .. nblk-1 (nblk = ceil(b / block)):
+ *     SCORE(t)       block t-1's update and block t's scores (level-1 histogram, and the
+ *                    level-2 one of the predicted bin); this rank's removal count appended
+ *     -> sum `level1` over ranks (uint32, in place)
+ *     PICK_BIN(t)    the level-1 bin of the residual budget's last key
+ *     REREAD(t)      this rank's level-2 counts when the bin was not predicted
+ *     -> sum `level2` over ranks
+ *     PICK_KEY(t)    the exact threshold and the number of tied entries taken
+ *     COUNT_TIES(t)  this rank's tied entries per block column
+ *     -> gather `ties` from every rank into ties_all (world x 128 uint32, rank order)
+ *     CUT_TIES(t)    this rank's share of the ties, in (column, row) order with lower ranks'
+ *                    rows first
+ *     SOLVE(t)       the masks and joint solves of this rank's rows
+ *   then FINISH (the last update; stats_dev->pruned = this rank's removals, no budget
+ *   check).  SETUP comes first (stats, W-hat, the factor of H, the inverse rows).
+ * All ranks must pass the same cfg, b, c_total and H (the layer's whole undamped 2XX^T,
+ * destroyed as by pwp_prune_layer).  Thanos and SparseGPT, pattern PWP_UNSTRUCTURED,
+ * alpha 0 (other patterns need no exchange: prune row slices with pwp_prune_layer);
+ * c_total * b < 2^31.  With world = 1 the steps reproduce pwp_prune_layer exactly.  The
+ * workspace is pwp_workspace_bytes(cfg, c, b); the same one for every step of a sweep. */
+typedef enum {
+    PWP_SWEEP_SETUP = 0, PWP_SWEEP_SCORE = 1, PWP_SWEEP_PICK_BIN = 2, PWP_SWEEP_REREAD = 3,
+    PWP_SWEEP_PICK_KEY = 4, PWP_SWEEP_COUNT_TIES = 5, PWP_SWEEP_CUT_TIES = 6, PWP_SWEEP_SOLVE = 7,
+    PWP_SWEEP_FINISH = 8
+} pwp_sweep_step_kind;
+typedef struct {
+    const pwp_config* cfg;
+    const void* W_dev;          /* this rank's rows: c x b, wtype */
+    int32_t wtype;
+    int32_t c;                  /* this rank's rows */
+    int32_t b;
+    int64_t c_total;            /* every rank's rows: the budget counts these */
+    float* H_dev;
+    float* W_out_dev;           /* c x b fp32 */
+    uint8_t* mask_dev;          /* c x b */
+    void* ws;
+    size_t ws_bytes;
+    pwp_stats* stats_dev;
+    const uint32_t* ties_all_dev;   /* world x 128, for PWP_SWEEP_CUT_TIES */
+    int32_t world;
+    int32_t rank;
+    void* stream;
+} pwp_sweep;
+pwp_status pwp_sweep_step(const pwp_sweep* sweep, int32_t step, int32_t t);
+/* Device addresses (inside ws) and lengths (uint32 words) of the buffers exchanged between
+ * steps: level1 (summed), level2 (summed), ties (this rank's, to gather). */
+pwp_status pwp_sweep_buffers(const pwp_sweep* sweep, uint32_t** level1, int64_t* n_level1, uint32_t** level2,
+                             int64_t* n_level2, uint32_t** ties, int64_t* n_ties);
+
 /* Compressed 2:4 storage of a pruned layer ("Weight Pruning in Large Language Models
  * ...", llms.blog, section "N:M Semi-Structured Sparsity (2:4 Pattern)": only the two
  * kept values of every aligned group of four, at 16-bit precision, and 2-bit index

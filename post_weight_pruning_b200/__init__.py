@@ -20,7 +20,7 @@ import numpy as np
 __all__ = [
     "lib", "Config", "Stats", "THANOS", "SPARSEGPT", "WANDA", "MAGNITUDE", "UNSTRUCTURED", "NM", "BF16", "FP32",
     "PwpError", "config", "workspace_bytes", "hessian_accumulate", "damp_factor", "prune_layer",
-    "prune_layer_host", "prune_block", "pack_24", "status_string", "set_wait_limit", "LIB_PATH",
+    "prune_layer_host", "prune_block", "pack_24", "status_string", "set_wait_limit", "Sweep", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpwp.so")
@@ -44,6 +44,14 @@ class Stats(ctypes.Structure):
                 ("tie_blocks", ctypes.c_int32), ("reserved", ctypes.c_int32 * 4)]
 
 
+class SweepArgs(ctypes.Structure):
+    _fields_ = [("cfg", ctypes.POINTER(Config)), ("W", ctypes.c_void_p), ("wtype", ctypes.c_int32),
+                ("c", ctypes.c_int32), ("b", ctypes.c_int32), ("c_total", ctypes.c_int64), ("H", ctypes.c_void_p),
+                ("W_out", ctypes.c_void_p), ("mask", ctypes.c_void_p), ("ws", ctypes.c_void_p),
+                ("ws_bytes", ctypes.c_size_t), ("stats", ctypes.c_void_p), ("ties_all", ctypes.c_void_p),
+                ("world", ctypes.c_int32), ("rank", ctypes.c_int32), ("stream", ctypes.c_void_p)]
+
+
 class PwpError(RuntimeError):
     def __init__(self, status, where=""):
         self.status = int(status)
@@ -63,6 +71,10 @@ _SIGS = {
                                  _vp, _vp, _vp, _sz, _vp, _vp]),
     "pwp_pack_24": (_i32, [_vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp]),
     "pwp_status_string": (ctypes.c_char_p, [_i32]),
+    "pwp_sweep_step": (_i32, [ctypes.POINTER(SweepArgs), _i32, _i32]),
+    "pwp_sweep_buffers": (_i32, [ctypes.POINTER(SweepArgs), ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(_i64),
+                                 ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(_i64),
+                                 ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(_i64)]),
     "pwp_set_wait_limit": (_i64, [_i64]),
     "pwp_version": (_i32, []),
 }
@@ -318,6 +330,66 @@ def prune_block(weights, activations, feeds, *, stream=None, check=True, **cfg):
             out[layer] = prune_layer(weights[layer], H=Hl, stream=stream, check=check, **cfg)
         del H
     return out
+
+
+class Sweep:
+    """One rank's rows of a layer pruned with the unstructured budget counted over every
+    rank's rows, step by step (pwp_sweep_step): ``sharded.global_sweep`` drives the block
+    loop and combines ``level1`` and ``level2`` (summed) and ``ties`` (gathered into
+    ``ties_all``) over ranks between the steps.
+
+    W_local: [c, b] bf16/fp32 CUDA tensor (this rank's rows, in rank order), H: the layer's
+    undamped fp32 [b, b] H (the same on every rank; destroyed), c_total: every rank's rows."""
+    STEPS = {"setup": 0, "score": 1, "pick_bin": 2, "reread": 3, "pick_key": 4, "count_ties": 5, "cut_ties": 6,
+             "solve": 7, "finish": 8}
+
+    def __init__(self, W_local, H, c_total, world=1, rank=0, *, method="thanos", sparsity=0.5, block=128,
+                 damp=0.01, stream=None):
+        torch = _torch()
+        if W_local.dim() != 2:
+            raise ValueError(f"W: expected [c, b], got shape {tuple(W_local.shape)}")
+        c, b = W_local.shape
+        _expect(W_local, "W", (c, b), (torch.bfloat16, torch.float32))
+        _expect(H, "H", (b, b), (torch.float32,))
+        _need_cuda(W_local, H)
+        self.cfg = config(method, "unstructured", (0, 0), sparsity, block, damp)
+        self.c, self.b, self.world, self.rank = int(c), int(b), int(world), int(rank)
+        self.nblk = (b + int(block) - 1) // int(block)
+        dev = W_local.device
+        self.W, self.H = W_local, H
+        self.W_out = torch.empty((c, b), dtype=torch.float32, device=dev)
+        self.mask = torch.empty((c, b), dtype=torch.uint8, device=dev)
+        self.ws = make_workspace(self.cfg, c, b, dev)
+        self.stats = new_stats(dev)
+        self.ties_all = torch.zeros((world, 128), dtype=torch.int32, device=dev)
+        self.stream = stream
+        self.args = SweepArgs(ctypes.pointer(self.cfg), W_local.data_ptr(), _dtype_code(W_local), c, b, int(c_total),
+                              H.data_ptr(), self.W_out.data_ptr(), self.mask.data_ptr(), self.ws.ws.data_ptr(),
+                              self.ws.nbytes, self.stats.data_ptr(), self.ties_all.data_ptr(), self.world, self.rank,
+                              _stream_ptr(stream).value)
+        p = [ctypes.c_void_p() for _ in range(3)]
+        n = [_i64() for _ in range(3)]
+        _check(lib().pwp_sweep_buffers(ctypes.byref(self.args), ctypes.byref(p[0]), ctypes.byref(n[0]),
+                                       ctypes.byref(p[1]), ctypes.byref(n[1]), ctypes.byref(p[2]), ctypes.byref(n[2])),
+               "pwp_sweep_buffers")
+        base = self.ws.ws.data_ptr()
+
+        def view(ptr, count):
+            off = ptr.value - base
+            return self.ws.ws[off: off + 4 * count.value].view(torch.int32)
+        self.level1, self.level2, self.ties = view(p[0], n[0]), view(p[1], n[1]), view(p[2], n[2])
+
+    def step(self, name, t=0):
+        _check(lib().pwp_sweep_step(ctypes.byref(self.args), self.STEPS[name], int(t)), f"pwp_sweep_step({name})")
+
+    def result(self, check=True):
+        """(W_hat fp32 [c, b], mask uint8 [c, b], Stats of this rank: pruned = its removals)."""
+        if not check:
+            return self.W_out, self.mask, self.stats
+        s = read_stats(self.stats)
+        if s.status != 0:
+            raise PwpError(s.status, "pwp_sweep_step (device)")
+        return self.W_out, self.mask, s
 
 
 def pack_24(W_hat, mask, *, stream=None, check=True):

@@ -15,6 +15,11 @@ cudaError_t launch_hessian_simt(const void* X, int xtype, long long n, int b, fl
 cudaError_t launch_hessian_tc(const void* X, long long n, int b, float* H, int beta, cudaStream_t s,
                               bool* used, pwp_stats* st);
 cudaError_t launch_stats_init(pwp_stats* st, cudaStream_t s);
+cudaError_t sweep_step(const pwp_config* cfg, const void* W, int wtype, int c, int b, long long c_budget, float* H,
+                       float* Wout, uint8_t* mask, void* ws, pwp_stats* st, const unsigned int* ties_all, int world,
+                       int rank, cudaStream_t s, int step, int t);
+void sweep_buffers(const pwp_config* cfg, int c, int b, void* ws, unsigned int** level1, long long* n1,
+                   unsigned int** level2, long long* n2, unsigned int** ties, long long* nt);
 }  // namespace pwp
 
 using namespace pwp;
@@ -147,6 +152,51 @@ pwp_status pwp_pack_24(const float* W_hat, const uint8_t* mask, int32_t c, int32
   if (cudaMemsetAsync(st, 0, sizeof(pwp_stats), s) != cudaSuccess) return PWP_ECUDA;
   cudaError_t e = launch_pack24(W_hat, mask, c, b, values, meta, st, s);
   return e == cudaSuccess ? PWP_OK : PWP_ECUDA;
+}
+
+// The stepwise sweep: argument checks shared by both calls.
+static pwp_status sweep_check(const pwp_sweep* a) {
+  if (!a || !valid_cfg(a->cfg, a->c, a->b) || !valid_dtype(a->wtype)) return PWP_EINVAL;
+  const pwp_config* cfg = a->cfg;
+  if ((cfg->method != PWP_THANOS && cfg->method != PWP_SPARSEGPT) || cfg->pattern != PWP_UNSTRUCTURED ||
+      cfg->alpha != 0.f)
+    return PWP_EINVAL;
+  if (a->c_total < a->c || a->c_total * (long long)a->b >= (1LL << 31) || a->world < 1 || a->rank < 0 ||
+      a->rank >= a->world)
+    return PWP_EINVAL;
+  if (!a->ws || !aligned(a->ws, 256) || a->ws_bytes < prune_ws_layout(cfg, a->c, a->b, nullptr, nullptr))
+    return PWP_EWORKSPACE;
+  return PWP_OK;
+}
+
+pwp_status pwp_sweep_step(const pwp_sweep* a, int32_t step, int32_t t) {
+  pwp_status ps = sweep_check(a);
+  if (ps != PWP_OK) return ps;
+  if (!a->W_dev || !a->H_dev || !a->W_out_dev || !a->mask_dev || !a->stats_dev) return PWP_EINVAL;
+  const int nblk = (a->b + a->cfg->block - 1) / a->cfg->block;
+  if (step < PWP_SWEEP_SETUP || step > PWP_SWEEP_FINISH) return PWP_EINVAL;
+  if (step != PWP_SWEEP_SETUP && step != PWP_SWEEP_FINISH && (t < 0 || t >= nblk)) return PWP_EINVAL;
+  if (step == PWP_SWEEP_CUT_TIES && !a->ties_all_dev) return PWP_EINVAL;
+  cudaError_t e = sweep_step(a->cfg, a->W_dev, a->wtype, a->c, a->b, a->c_total, a->H_dev, a->W_out_dev, a->mask_dev,
+                             a->ws, a->stats_dev, a->ties_all_dev, a->world, a->rank, (cudaStream_t)a->stream, step, t);
+  return e == cudaSuccess ? PWP_OK : PWP_ECUDA;
+}
+
+pwp_status pwp_sweep_buffers(const pwp_sweep* a, uint32_t** level1, int64_t* n_level1, uint32_t** level2,
+                             int64_t* n_level2, uint32_t** ties, int64_t* n_ties) {
+  pwp_status ps = sweep_check(a);
+  if (ps != PWP_OK) return ps;
+  if (!level1 || !n_level1 || !level2 || !n_level2 || !ties || !n_ties) return PWP_EINVAL;
+  long long n1, n2, nt;
+  unsigned int *p1, *p2, *pt;
+  sweep_buffers(a->cfg, a->c, a->b, a->ws, &p1, &n1, &p2, &n2, &pt, &nt);
+  *level1 = p1;
+  *n_level1 = n1;
+  *level2 = p2;
+  *n_level2 = n2;
+  *ties = pt;
+  *n_ties = nt;
+  return PWP_OK;
 }
 
 }  // extern "C"

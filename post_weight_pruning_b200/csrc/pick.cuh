@@ -115,10 +115,11 @@ __device__ void find_rank(const unsigned int* __restrict__ hist, long long rank,
 // global count (Thanos) or the block quota (SparseGPT); the bin of the take-th key; whether
 // the scoring pass predicted it (then the level-2 histogram is ready).  Clears the level-1
 // histogram for the next pass.
+// (pruned: the removals so far over every row the budget counts; -1 for this call's own.)
 __device__ inline void level1(Ctl* ctl, unsigned int* __restrict__ hist1, long long region_n, int global_budget,
-                              long long quota, pwp_stats* st, Shared& sh, int bar, int tid) {
+                              long long quota, pwp_stats* st, Shared& sh, int bar, int tid, long long pruned = -1) {
   if (tid == 0) {
-    const long long r = global_budget ? ctl->zstar - ctl->pruned : quota;
+    const long long r = global_budget ? ctl->zstar - (pruned >= 0 ? pruned : ctl->pruned) : quota;
     long long take = r < region_n ? r : region_n;
     if (take < r) st->shortfall = 1;
     if (take < 0) take = 0;

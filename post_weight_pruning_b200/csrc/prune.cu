@@ -327,7 +327,7 @@ size_t prune_ws_layout(const pwp_config* cfg, int c, int b, PruneBuffers* pb, ch
   };
   PruneBuffers t;
   t.ctl = (Ctl*)take(sizeof(Ctl));
-  t.hist1 = (unsigned int*)take(sizeof(unsigned int) * kHist1Bins);
+  t.hist1 = (unsigned int*)take(sizeof(unsigned int) * (kHist1Bins + 4));   // + a sweep's removal count
   // the level-2 arrays and the tie counts are contiguous, so one memset clears them
   t.l2.pred = (unsigned int*)take(sizeof(unsigned int) * (2 * kHist2Bins + 2 * kHist2SumBins + kMaxBlock));
   t.l2.pred_sum = t.l2.pred ? t.l2.pred + kHist2Bins : nullptr;
@@ -392,39 +392,44 @@ cudaError_t launch_stats_init(pwp_stats* st, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-// stats_ready: the caller already reset *st on this stream (and may have recorded an
-// earlier device-side failure in it, which then turns this call's kernels into no-ops).
-cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c, int b, float* H,
-                         float* Wout, uint8_t* mask, void* ws, pwp_stats* st, cudaStream_t s,
-                         bool stats_ready) {
-  if (cfg->method == PWP_WANDA || cfg->method == PWP_MAGNITUDE)
-    return launch_no_update(cfg, W, wtype, c, b, cfg->method == PWP_WANDA ? H : nullptr, nullptr, 0, 0, Wout,
-                            mask, ws, st, stats_ready, s);
-  const int n_out = alpha_rows(cfg, c);
-  if (n_out > 0) {
-    pwp_config ic = *cfg;
-    ic.alpha = 0.f;
-    const size_t inner = prune_ws_layout(&ic, c - n_out, b, nullptr, nullptr);
-    return launch_prune_alpha(cfg, W, wtype, c, b, H, Wout, mask, ws, inner, st, s, stats_ready, n_out,
-                              &launch_prune);
-  }
+// One prune's host-side state: the configuration, sizes, buffers and derived flags.
+struct PruneRun {
+  const pwp_config* cfg;
+  int c, b, B, nblk;
+  long long c_budget;   // rows the selection budget counts (c, or all ranks' rows for a sweep)
+  bool thanos, nm, tc_shape;
+  int score;
+  float* H;
+  float* Wout;
+  uint8_t* mask;
   PruneBuffers pb;
-  const int B = cfg->block;
-  prune_ws_layout(cfg, c, b, &pb, (char*)ws);
-  const bool thanos = cfg->method == PWP_THANOS;
-  const bool nm = cfg->pattern == PWP_NM;
-  const long long N = (long long)c * b;
-  const long long zstar = (long long)((double)cfg->sparsity * (double)N);
-  const int nblk = (b + B - 1) / B;
-  long long target = 0;
-  if (nm) {
-    target = N / cfg->nm_m * (cfg->nm_m - cfg->nm_n);
-  } else if (thanos) {
-    target = zstar;
-  } else {
-    for (int t = 0; t < nblk; ++t)
-      target += (long long)((double)cfg->sparsity * (double)c * (double)min(B, b - t * B));
-  }
+  const float* sc;
+  const float* Zlo;
+  pwp_stats* st;
+  cudaStream_t s;
+};
+
+static cudaError_t prune_init(PruneRun& R, const pwp_config* cfg, int c, int b, long long c_budget, float* H,
+                              float* Wout, uint8_t* mask, void* ws, pwp_stats* st, cudaStream_t s) {
+  R.cfg = cfg;
+  R.c = c;
+  R.b = b;
+  R.B = cfg->block;
+  R.nblk = (b + R.B - 1) / R.B;
+  R.c_budget = c_budget;
+  R.thanos = cfg->method == PWP_THANOS;
+  R.nm = cfg->pattern == PWP_NM;
+  R.score = R.nm ? kNoScore : (R.thanos ? kWanda : kObs);
+  R.H = H;
+  R.Wout = Wout;
+  R.mask = mask;
+  R.st = st;
+  R.s = s;
+  prune_ws_layout(cfg, c, b, &R.pb, (char*)ws);
+  R.sc = R.thanos ? R.pb.xnorm : R.pb.udiag;
+  R.Zlo = R.pb.Zs + (size_t)c * R.B;
+  // tensor-core update: 16-byte rows for TMA (b, B multiples of 4), aligned W and mask
+  R.tc_shape = (b % 4) == 0 && (R.B % 4) == 0 && ((uintptr_t)Wout % 16) == 0 && ((uintptr_t)mask % 4) == 0;
   if (first_on_device(g_attr_done)) {
     cudaError_t e0 = cudaFuncSetAttribute(stream_kernel<kWanda>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           kHist1Bins * 4);
@@ -442,102 +447,246 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
     }
     g_nsm = nsm;
   }
-  long long nl = 0;
-  if (!stats_ready) {
-    init_stats_kernel<<<1, 1, 0, s>>>(st);
-    ++nl;
+  return cudaSuccess;
+}
+
+// Removal target and budget of the layer (over c_budget rows).
+static void prune_targets(const PruneRun& R, long long* zstar, long long* target) {
+  const long long N = R.c_budget * R.b;
+  *zstar = (long long)((double)R.cfg->sparsity * (double)N);
+  if (R.nm) {
+    *target = (long long)R.c * R.b / R.cfg->nm_m * (R.cfg->nm_m - R.cfg->nm_n);
+  } else if (R.thanos) {
+    *target = *zstar;
+  } else {
+    *target = 0;
+    for (int t = 0; t < R.nblk; ++t)
+      *target += (long long)((double)R.cfg->sparsity * (double)R.c_budget * (double)min(R.B, R.b - t * R.B));
   }
-  launch_pdl(init_ctl_kernel, dim3(1), dim3(1), 0, s, pb.ctl, zstar, st, target);
-  cudaError_t em = cudaMemsetAsync(pb.hist1, 0, sizeof(unsigned int) * kHist1Bins, s);
+}
+
+// Stats and control block, W-hat from W, the damped factor, the score scales and, for
+// Thanos, every block's rows of the active inverse.
+static cudaError_t prune_setup(PruneRun& R, const void* W, int wtype, bool stats_ready, long long* nl) {
+  long long zstar, target;
+  prune_targets(R, &zstar, &target);
+  cudaStream_t s = R.s;
+  if (!stats_ready) {
+    init_stats_kernel<<<1, 1, 0, s>>>(R.st);
+    ++*nl;
+  }
+  launch_pdl(init_ctl_kernel, dim3(1), dim3(1), 0, s, R.pb.ctl, zstar, R.st, target);
+  cudaError_t em = cudaMemsetAsync(R.pb.hist1, 0, sizeof(unsigned int) * (kHist1Bins + 4), s);
   if (em == cudaSuccess)
-    em = cudaMemsetAsync(pb.l2.pred, 0, sizeof(unsigned int) * (2 * kHist2Bins + 2 * kHist2SumBins + kMaxBlock), s);
+    em = cudaMemsetAsync(R.pb.l2.pred, 0, sizeof(unsigned int) * (2 * kHist2Bins + 2 * kHist2SumBins + kMaxBlock),
+                         s);
   if (em != cudaSuccess) return em;
-  launch_pdl(convert_w_kernel, dim3(4 * g_nsm.load()), dim3(256), 0, s, W, wtype, Wout, N);
-  nl += 2;
+  launch_pdl(convert_w_kernel, dim3(4 * g_nsm.load()), dim3(256), 0, s, W, wtype, R.Wout, (long long)R.c * R.b);
+  *nl += 2;
   prof_begin(kKFactor, s);
-  cudaError_t e = launch_damp_factor(H, b, cfg->damp, pb.g_diag, pb.fws, pb.fws_bytes, st, s);
+  cudaError_t e = launch_damp_factor(R.H, R.b, R.cfg->damp, R.pb.g_diag, R.pb.fws, R.pb.fws_bytes, R.st, s);
   prof_end(kKFactor, s);
   if (e != cudaSuccess) return e;
-  launch_pdl(prep_diag_kernel, dim3((b + 255) / 256), dim3(256), 0, s, H, b, pb.g_diag, pb.xnorm, pb.udiag);
-  ++nl;
-  if (thanos) {
-    dim3 g((b + 127) / 128, nblk);
-    launch_pdl(kmat_kernel, dim3(g), dim3(256), kmat_smem_bytes(B), s, H, b, B, pb.K_in, pb.K_hi, pb.K_lo, st);
-    ++nl;
+  launch_pdl(prep_diag_kernel, dim3((R.b + 255) / 256), dim3(256), 0, s, (const float*)R.H, R.b,
+             (const float*)R.pb.g_diag, R.pb.xnorm, R.pb.udiag);
+  ++*nl;
+  if (R.thanos) {
+    dim3 g((R.b + 127) / 128, R.nblk);
+    launch_pdl(kmat_kernel, dim3(g), dim3(256), kmat_smem_bytes(R.B), s, (const float*)R.H, R.b, R.B, R.pb.K_in,
+               R.pb.K_hi, R.pb.K_lo, (const pwp_stats*)R.st);
+    ++*nl;
   }
-  const int score = nm ? kNoScore : (thanos ? kWanda : kObs);
-  const float* sc = thanos ? pb.xnorm : pb.udiag;
-  const float* Zlo = pb.Zs + (size_t)c * B;
-  // tensor-core update: 16-byte rows for TMA (b, B multiples of 4), aligned W and mask
-  const bool tc_shape = (b % 4) == 0 && (B % 4) == 0 && ((uintptr_t)Wout % 16) == 0 && ((uintptr_t)mask % 4) == 0;
-  for (int t = 0; t <= nblk; ++t) {
-    const int j = t * B, j1 = min(b, j + B);
-    const int jp = (t - 1) * B, Bp = t > 0 ? min(B, b - jp) : 0;
-    const int u0 = t > 0 ? jp : j;
-    const int jj = t == nblk ? b : j;          // the last pass only finishes the last block
-    const int pass_score = t == nblk ? kNoScore : score;
-    const int hist_end = t == nblk ? b : (thanos ? b : j1);
+  return cudaGetLastError();
+}
+
+// Block t's selection arguments (t < nblk, scored patterns): the region's entry count and
+// the budget, both over all c_budget rows.
+static PickArgs pick_args(const PruneRun& R, int t, bool fused) {
+  PickArgs pk{};
+  if (R.score == kNoScore || t >= R.nblk) return pk;
+  const int j = t * R.B, j1 = min(R.b, j + R.B);
+  pk.region_n = R.thanos ? R.c_budget * (R.b - j) : R.c_budget * (j1 - j);
+  pk.quota = R.thanos ? 0 : (long long)((double)R.cfg->sparsity * (double)R.c_budget * (double)(j1 - j));
+  pk.global_budget = R.thanos ? 1 : 0;
+  pk.enabled = fused ? 1 : 0;
+  return pk;
+}
+
+// Pass t: apply block t-1's update to the active columns (t > 0) while scoring block t's
+// region into the level-1 histogram (t < nblk); t = nblk only finishes the last block.
+static cudaError_t prune_pass(PruneRun& R, int t, PickArgs pk, long long* nl) {
+  const int b = R.b, B = R.B, c = R.c;
+  const int j = t * B, j1 = min(b, j + B);
+  const int jp = (t - 1) * B, Bp = t > 0 ? min(B, b - jp) : 0;
+  const int u0 = t > 0 ? jp : j;
+  const int jj = t == R.nblk ? b : j;
+  const int pass_score = t == R.nblk ? kNoScore : R.score;
+  const int hist_end = t == R.nblk ? b : (R.thanos ? b : j1);
+  PruneBuffers& pb = R.pb;
+  cudaStream_t s = R.s;
+  prof_begin(kKStream, s);
+  if (t > 0) {
+    // W[:, jp:b] -= Z R with R = block t-1's rows of K (Thanos) or of U (SparseGPT)
+    bool done = false;
+    if (R.tc_shape) {
+      const float* Rh = R.thanos ? pb.K_hi + (size_t)(t - 1) * b * B : pb.R_hi;
+      const float* Rl = R.thanos ? pb.K_lo + (size_t)(t - 1) * b * B : pb.R_lo;
+      if (!R.thanos) {
+        const long long n = (long long)Bp * (b - jp);
+        const int grid = (int)min((n + 255) / 256, (long long)8 * g_nsm.load());
+        launch_pdl(urows_kernel, dim3(grid), dim3(256), 0, s, (const float*)R.H, b, B, jp, Bp, pb.R_hi, pb.R_lo,
+                   (const pwp_stats*)R.st);
+        ++*nl;
+      }
+      cudaError_t e2 = cudaSuccess;
+      done = launch_stream_tc(pass_score, R.Wout, c, b, b, u0, jj, pb.Zs, R.Zlo, Bp, B, Rh, Rl, R.mask, R.sc,
+                              hist_end, pb.hist1, pb.ctl, pb.l2, R.st, s, &e2, false, pk);
+      if (e2 != cudaSuccess) return e2;
+    }
+    if (!done) {
+      // Thanos: K_t transposed (row stride B); SparseGPT: U's rows in place in H
+      const float* Rm = R.thanos ? pb.K_hi + (size_t)(t - 1) * b * B : R.H + (size_t)jp * b;
+      const float* Rlo = R.thanos ? pb.K_lo + (size_t)(t - 1) * b * B : nullptr;
+      launch_stream_any(pass_score, R.Wout, c, b, u0, jj, pb.Zs, R.Zlo, Bp, B, Rm, Rlo, R.thanos ? B : b,
+                        R.thanos ? 1 : 0, R.thanos ? -1 : jp, R.mask, R.sc, hist_end, pb.hist1, pb.ctl, pb.l2, pk,
+                        R.st, s);
+    }
+    ++*nl;
+  } else if (R.score != kNoScore) {
+    // first block: nothing to apply yet, only the scores of the active region
+    launch_stream_any(R.score, R.Wout, c, b, j, j, pb.Zs, R.Zlo, 0, B, nullptr, nullptr, b, 0, -1, R.mask, R.sc,
+                      hist_end, pb.hist1, pb.ctl, pb.l2, pk, R.st, s);
+    ++*nl;
+  }
+  prof_end(kKStream, s);
+  return cudaSuccess;
+}
+
+// Block t's per-row work: the masks, the joint solves (Thanos) or the column sweep
+// (SparseGPT), and the rows' coefficients for the next pass.
+static void prune_solve(PruneRun& R, int t, long long* nl) {
+  const int j = t * R.B;
+  prof_begin(kKSolve, R.s);
+  if (R.thanos)
+    *nl += launch_thanos_solve(R.nm, R.Wout, R.c, R.b, j, R.B, R.pb.K_in + (size_t)t * R.B * R.B, R.pb.xnorm,
+                               R.pb.ctl, R.mask, R.pb.Zs, R.cfg->nm_n, R.cfg->nm_m, R.pb.gscratch, R.st, R.s);
+  else
+    *nl += launch_sparsegpt_solve(R.nm, R.Wout, R.c, R.b, j, R.B, R.H, R.pb.udiag, R.pb.ctl, R.mask, R.pb.Zs,
+                                  R.cfg->nm_n, R.cfg->nm_m, R.st, R.s);
+  prof_end(kKSolve, R.s);
+}
+
+// stats_ready: the caller already reset *st on this stream (and may have recorded an
+// earlier device-side failure in it, which then turns this call's kernels into no-ops).
+cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c, int b, float* H,
+                         float* Wout, uint8_t* mask, void* ws, pwp_stats* st, cudaStream_t s,
+                         bool stats_ready) {
+  if (cfg->method == PWP_WANDA || cfg->method == PWP_MAGNITUDE)
+    return launch_no_update(cfg, W, wtype, c, b, cfg->method == PWP_WANDA ? H : nullptr, nullptr, 0, 0, Wout,
+                            mask, ws, st, stats_ready, s);
+  const int n_out = alpha_rows(cfg, c);
+  if (n_out > 0) {
+    pwp_config ic = *cfg;
+    ic.alpha = 0.f;
+    const size_t inner = prune_ws_layout(&ic, c - n_out, b, nullptr, nullptr);
+    return launch_prune_alpha(cfg, W, wtype, c, b, H, Wout, mask, ws, inner, st, s, stats_ready, n_out,
+                              &launch_prune);
+  }
+  PruneRun R;
+  cudaError_t e = prune_init(R, cfg, c, b, c, H, Wout, mask, ws, st, s);
+  if (e != cudaSuccess) return e;
+  long long nl = 0;
+  e = prune_setup(R, W, wtype, stats_ready, &nl);
+  if (e != cudaSuccess) return e;
+  for (int t = 0; t <= R.nblk; ++t) {
     // block t's selection: the scoring pass's last CTA takes the level-1 bin (and the
     // threshold, when predicted); select_finish does the rest
-    PickArgs pk{};
-    if (pass_score != kNoScore) {
-      pk.region_n = thanos ? (long long)c * (b - j) : (long long)c * (j1 - j);
-      pk.quota = thanos ? 0 : (long long)((double)cfg->sparsity * (double)c * (double)(j1 - j));
-      pk.global_budget = thanos ? 1 : 0;
-      pk.enabled = 1;
-    }
-    prof_begin(kKStream, s);
-    if (t > 0) {
-      // W[:, jp:b] -= Z R with R = block t-1's rows of K (Thanos) or of U (SparseGPT)
-      bool done = false;
-      if (tc_shape) {
-        const float* Rh = thanos ? pb.K_hi + (size_t)(t - 1) * b * B : pb.R_hi;
-        const float* Rl = thanos ? pb.K_lo + (size_t)(t - 1) * b * B : pb.R_lo;
-        if (!thanos) {
-          const long long n = (long long)Bp * (b - jp);
-          const int grid = (int)min((n + 255) / 256, (long long)8 * g_nsm.load());
-          launch_pdl(urows_kernel, dim3(grid), dim3(256), 0, s, H, b, B, jp, Bp, pb.R_hi, pb.R_lo, st);
-          ++nl;
-        }
-        cudaError_t e2 = cudaSuccess;
-        done = launch_stream_tc(pass_score, Wout, c, b, b, u0, jj, pb.Zs, Zlo, Bp, B, Rh, Rl, mask, sc, hist_end,
-                                pb.hist1, pb.ctl, pb.l2, st, s, &e2, false, pk);
-        if (e2 != cudaSuccess) return e2;
-      }
-      if (!done) {
-        // Thanos: K_t transposed (row stride B); SparseGPT: U's rows in place in H
-        const float* R = thanos ? pb.K_hi + (size_t)(t - 1) * b * B : H + (size_t)jp * b;
-        const float* Rlo = thanos ? pb.K_lo + (size_t)(t - 1) * b * B : nullptr;
-        launch_stream_any(pass_score, Wout, c, b, u0, jj, pb.Zs, Zlo, Bp, B, R, Rlo, thanos ? B : b, thanos ? 1 : 0,
-                          thanos ? -1 : jp, mask, sc, hist_end, pb.hist1, pb.ctl, pb.l2, pk, st, s);
-      }
-      ++nl;
-    } else if (score != kNoScore) {
-      // first block: nothing to apply yet, only the scores of the active region
-      launch_stream_any(score, Wout, c, b, j, j, pb.Zs, Zlo, 0, B, nullptr, nullptr, b, 0, -1, mask, sc, hist_end,
-                        pb.hist1, pb.ctl, pb.l2, pk, st, s);
-      ++nl;
-    }
-    prof_end(kKStream, s);
-    if (t == nblk) break;
-    if (score != kNoScore) {
+    e = prune_pass(R, t, pick_args(R, t, true), &nl);
+    if (e != cudaSuccess) return e;
+    if (t == R.nblk) break;
+    if (R.score != kNoScore) {
+      const int j = t * R.B, j1 = min(b, j + R.B);
       prof_begin(kKSelect, s);
-      launch_select_finish(score, pb.ctl, pb.l2, Wout, c, b, j, j1, thanos ? b : j1, sc, st, s);
+      launch_select_finish(R.score, R.pb.ctl, R.pb.l2, Wout, c, b, j, j1, R.thanos ? b : j1, R.sc, st, s);
       prof_end(kKSelect, s);
       ++nl;
     }
-    prof_begin(kKSolve, s);
-    if (thanos)
-      nl += launch_thanos_solve(nm, Wout, c, b, j, B, pb.K_in + (size_t)t * B * B, pb.xnorm, pb.ctl, mask, pb.Zs,
-                                cfg->nm_n, cfg->nm_m, pb.gscratch, st, s);
-    else
-      nl += launch_sparsegpt_solve(nm, Wout, c, b, j, B, H, pb.udiag, pb.ctl, mask, pb.Zs, cfg->nm_n,
-                                   cfg->nm_m, st, s);
-    prof_end(kKSolve, s);
+    prune_solve(R, t, &nl);
   }
-  launch_pdl(finalize_kernel, dim3(1), dim3(1), 0, s, pb.ctl, st, (thanos && !nm) ? 1 : 0);
+  launch_pdl(finalize_kernel, dim3(1), dim3(1), 0, s, (const Ctl*)R.pb.ctl, st, (R.thanos && !R.nm) ? 1 : 0);
   count_launches(nl + 1);
   return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- the stepwise sweep
+// The block loop of launch_prune taken apart, for rows sharded over ranks with the
+// unstructured budget counted over every rank's rows (c_budget): the caller sums the
+// level-1 histogram (with each rank's removal count), the level-2 histograms and gathers
+// the tie counts over ranks between the steps (pwp_sweep_step in include/pwp.h).
+cudaError_t sweep_step(const pwp_config* cfg, const void* W, int wtype, int c, int b, long long c_budget, float* H,
+                       float* Wout, uint8_t* mask, void* ws, pwp_stats* st, const unsigned int* ties_all, int world,
+                       int rank, cudaStream_t s, int step, int t) {
+  PruneRun R;
+  cudaError_t e = prune_init(R, cfg, c, b, c_budget, H, Wout, mask, ws, st, s);
+  if (e != cudaSuccess) return e;
+  long long nl = 0;
+  const int j = t * R.B, j1 = min(b, j + R.B), q1 = R.thanos ? b : j1;
+  switch (step) {
+    case PWP_SWEEP_SETUP:
+      e = prune_setup(R, W, wtype, false, &nl);
+      break;
+    case PWP_SWEEP_SCORE:
+      e = prune_pass(R, t, pick_args(R, t, false), &nl);
+      if (e == cudaSuccess && t < R.nblk) {
+        launch_sweep_select(0, R.score, R.pb.ctl, R.pb.hist1, R.pb.l2, PickArgs{}, Wout, c, b, j, j1, q1, R.sc,
+                            nullptr, world, rank, st, s);
+        ++nl;
+      }
+      break;
+    case PWP_SWEEP_PICK_BIN:
+    case PWP_SWEEP_REREAD:
+    case PWP_SWEEP_PICK_KEY:
+    case PWP_SWEEP_COUNT_TIES:
+    case PWP_SWEEP_CUT_TIES: {
+      const int k = step == PWP_SWEEP_PICK_BIN ? 1 : step == PWP_SWEEP_REREAD ? 2 : step == PWP_SWEEP_PICK_KEY ? 3
+                    : step == PWP_SWEEP_COUNT_TIES ? 4 : 5;
+      prof_begin(kKSelect, s);
+      launch_sweep_select(k, R.score, R.pb.ctl, R.pb.hist1, R.pb.l2, pick_args(R, t, false), Wout, c, b, j, j1, q1,
+                          R.sc, ties_all, world, rank, st, s);
+      prof_end(kKSelect, s);
+      ++nl;
+      break;
+    }
+    case PWP_SWEEP_SOLVE:
+      launch_sweep_select(6, R.score, R.pb.ctl, R.pb.hist1, R.pb.l2, PickArgs{}, Wout, c, b, j, j1, q1, R.sc,
+                          nullptr, world, rank, st, s);
+      prune_solve(R, t, &nl);
+      ++nl;
+      break;
+    case PWP_SWEEP_FINISH:
+      e = prune_pass(R, R.nblk, PickArgs{}, &nl);
+      launch_pdl(finalize_kernel, dim3(1), dim3(1), 0, s, (const Ctl*)R.pb.ctl, st, 0);
+      ++nl;
+      break;
+    default:
+      return cudaErrorInvalidValue;
+  }
+  count_launches(nl);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+// Device addresses of the buffers the caller exchanges between ranks.
+void sweep_buffers(const pwp_config* cfg, int c, int b, void* ws, unsigned int** level1, long long* n1,
+                   unsigned int** level2, long long* n2, unsigned int** ties, long long* nt) {
+  PruneBuffers pb;
+  prune_ws_layout(cfg, c, b, &pb, (char*)ws);
+  *level1 = pb.hist1;
+  *n1 = kHist1Bins + 1;                          // + this rank's removal count
+  *level2 = pb.l2.pred;
+  *n2 = 2 * ((long long)kHist2Bins + kHist2SumBins);   // predicted and re-read, with their summaries
+  *ties = pb.l2.tie_count;
+  *nt = kMaxBlock;
 }
 
 }  // namespace pwp

@@ -219,6 +219,9 @@ struct PickArgs {
 // was not predicted, the cut-off among tied entries, and clearing the level-2 histograms.
 void launch_select_finish(int score, Ctl* ctl, Level2 l2, const float* W, int c, int b, int j, int j1, int q1,
                           const float* sc, pwp_stats* st, cudaStream_t s);
+void launch_sweep_select(int step, int score, Ctl* ctl, unsigned int* hist1, Level2 l2, PickArgs pk, const float* W,
+                         int c, int b, int j, int j1, int q1, const float* sc, const unsigned int* ties_all, int world,
+                         int rank, pwp_stats* st, cudaStream_t s);
 
 // W[:, u0:b] -= Z R on the tensor cores (stream_tc.cu), fused with zeroing the previous
 // block's removals and the level-1 histogram of the scores of columns [j, hist_end).

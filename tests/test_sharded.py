@@ -46,9 +46,9 @@ def test_rows_independent(method, pattern, want):
     assert sharded.rows_independent(method, pattern) is want
 
 
-def test_prune_rows_refuses_the_global_budget():
+def test_prune_rows_sends_the_global_budget_to_the_sweep():
     W = torch.zeros(8, 16)
-    with pytest.raises(NotImplementedError):
+    with pytest.raises(ValueError, match="prune_rows_global"):
         sharded.prune_rows(W, torch.zeros(16, 16), method="thanos", pattern="unstructured")
 
 
@@ -208,3 +208,89 @@ def test_global_budget_exchange_reproduces_the_global_selection(world, ties):
     got = np.concatenate([out[k] for k in range(world)])
     assert got.sum() == r
     assert np.array_equal(got, want)
+
+
+# ----------------------------------------------------------------------------- the stepwise sweep
+
+def _sweep_worker(rank, world, port, W, H, out, kw):
+    from tests._sweep_standin import NumpySweep
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        r0, r1 = sharded.row_range(W.shape[0], world, rank)
+        sw = NumpySweep(W[r0:r1], H, W.shape[0], world, rank, **kw)
+        sharded.global_sweep([sw], sharded.TorchComm())
+        out[rank] = (sw.W, sw.mask, sw.pruned)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,ties", [(2, False), (3, True)])
+def test_global_sweep_over_gloo_ranks_reproduces_the_whole_layer(world, ties):
+    """The real host loop (sharded.global_sweep with its torch.distributed collectives) over
+    gloo ranks, each holding a row slice of one layer under the global budget: the ranks'
+    masks and weights together are the oracle's whole-layer prune.  With ties, the first
+    block's threshold falls inside large groups of equal scores spread over the ranks."""
+    rng = np.random.default_rng(70 + world)
+    c, b, n = 29, 32, 96
+    if ties:
+        W = np.round(rng.normal(0, 0.02, size=(c, b)) * 64) / 64
+        Xt = rng.choice([-1.0, 1.0], size=(n, b))              # every feature the same norm
+    else:
+        W = rng.normal(0, 0.02, size=(c, b))
+        Xt = rng.normal(size=(n, b)) * rng.uniform(0.5, 2.0, size=b)
+    H = oracle.hessian(Xt)
+    kw = dict(sparsity=0.5, block=8, damp=0.01)
+    want = oracle.prune_layer(W, H=H, **kw)
+    if ties:
+        S0 = oracle.wanda_scores(W, np.diag(H) / 2)
+        assert (S0 == want["blocks"][0]["t_last"]).sum() > 10     # the boundary really is tied
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_sweep_worker, args=(world, _free_port(), W, H, out, kw), nprocs=world, start_method="spawn")
+    got_W = np.concatenate([out[r][0] for r in range(world)])
+    got_m = np.concatenate([out[r][1] for r in range(world)])
+    assert sum(out[r][2] for r in range(world)) == want["zstar"]
+    assert np.array_equal(got_m, want["mask"])
+    assert np.allclose(got_W, want["W"], rtol=1e-9, atol=1e-12)
+
+
+def test_global_sweep_drops_the_cross_rank_tie_order_and_fails():
+    """A plant in the stand-in, not the library: if a rank ignored the lower ranks' tied
+    entries (rank 0's cut-off used by every rank), the union would take too many ties."""
+    from tests._sweep_standin import NumpySweep
+
+    class Careless(NumpySweep):
+        def _cut_ties(self, t):
+            keep = self.rank
+            self.rank = 0
+            self.ties_all.numpy()[:] = 0
+            self.ties_all.numpy()[0, :] = self.ties.numpy()
+            super()._cut_ties(t)
+            self.rank = keep
+
+    rng = np.random.default_rng(72)
+    W = np.round(rng.normal(0, 0.02, size=(20, 16)) * 64) / 64
+    Xt = rng.choice([-1.0, 1.0], size=(48, 16))
+    H = oracle.hessian(Xt)
+    sweeps = [Careless(W[r0:r1], H, 20, 2, r, sparsity=0.5, block=8)
+              for r, (r0, r1) in enumerate(sharded.row_range(20, 2, r) for r in range(2))]
+    sharded.global_sweep(sweeps, sharded.LocalComm())
+    want = oracle.prune_layer(W, H=H, sparsity=0.5, block=8)
+    got = np.concatenate([sw.mask for sw in sweeps])
+    assert not np.array_equal(got, want["mask"])
+
+
+def test_local_comm_emulates_ranks_in_one_process():
+    """The in-process communicator on the CPU stand-in reproduces the whole layer too."""
+    from tests._sweep_standin import NumpySweep
+    rng = np.random.default_rng(73)
+    W = rng.normal(0, 0.02, size=(21, 24))
+    Xt = rng.normal(size=(60, 24))
+    H = oracle.hessian(Xt)
+    sweeps = [NumpySweep(W[r0:r1], H, 21, 3, r, sparsity=0.4, block=8)
+              for r, (r0, r1) in enumerate(sharded.row_range(21, 3, r) for r in range(3))]
+    sharded.global_sweep(sweeps, sharded.LocalComm())
+    want = oracle.prune_layer(W, H=H, sparsity=0.4, block=8)
+    assert np.array_equal(np.concatenate([sw.mask for sw in sweeps]), want["mask"])
+    assert np.allclose(np.concatenate([sw.W for sw in sweeps]), want["W"], rtol=1e-9, atol=1e-12)
