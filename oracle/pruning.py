@@ -31,6 +31,11 @@ Everything is fp64.  Library primitives used as single steps: matrix product,
 ``numpy.partition`` / ``numpy.lexsort`` / ``numpy.argsort``.  There is no
 blocking, fusion or reordering beyond what the pages' algorithm states.
 
+Parity status: every function is pinned by the tests in tests/test_oracle.py, except that
+the rule by which ``outlier_rows`` chooses its rows is a reading of a page that does not
+state it -- parity unpinned for that rule (its count, tie order and the resulting sparsity
+are pinned).
+
 Notation follows [THANOS]: W is c x b (rows = outputs, columns = input
 features), X is b x n with calibration examples as columns.  Activations are
 passed token-major, ``Xt = X^T`` with shape [n, b].
