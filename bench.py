@@ -520,10 +520,18 @@ def run_mine(args):
             if mask_np is None:
                 mask_np = mask.cpu().numpy()
             line["phases"] = phase_rooflines(wl, phase_ms, mask_np, peaks)
+        # the other workloads and the CPU baseline are reported beside the headline; a
+        # failure in either is recorded in the line instead of losing it
         if world == 1 and not args.no_extra_workloads and method == "thanos":
-            line["workloads"] = time_other_workloads(dev, args)
+            try:
+                line["workloads"] = time_other_workloads(dev, args)
+            except Exception as exc:   # noqa: BLE001
+                line["workloads"] = {"error": f"{type(exc).__name__}: {exc}"}
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_oracle_full(wl, W_store, X_store, method)
+            try:
+                line["cpu_baseline"] = cpu_oracle_full(wl, W_store, X_store, method)
+            except Exception as exc:   # noqa: BLE001
+                line["cpu_baseline"] = {"error": f"{type(exc).__name__}: {exc}"}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
