@@ -79,74 +79,103 @@ __global__ void prep_diag_kernel(const float* __restrict__ H, int b, const float
 // (K_in, B x B per block, row stride B; the square is symmetric) for the row solves, and
 // K_t transposed as TF32 head and fp32 remainder (K_hi, K_lo: b x B per block, row q
 // holds column q of K_t, rows < j_t unused) -- the K-major operand of the tensor-core
-// update.  Grid (column tiles of 128, blocks); 128x128 outputs per CTA, 8x8 per thread,
-// staged through shared memory so that every output row is written contiguously.
+// update.  Grid (column tiles of 128, blocks); 128 (p) x 128 (q) outputs per CTA, 8x8 per
+// thread; the sum over r runs in chunks of 16 rows of U, double-buffered in shared memory
+// (both operands are rows of U, read as float4; U's stale lower triangle is zeroed as it is
+// loaded), and the tile is staged transposed, 64 columns at a time, so that every output
+// row is written contiguously.
+constexpr int kKmatChunk = 16;
 __global__ void __launch_bounds__(256) kmat_kernel(const float* __restrict__ H, int b, int B,
                                                    float* __restrict__ K_in, float* __restrict__ K_hi,
                                                    float* __restrict__ K_lo, const pwp_stats* st) {
   pdl_enter();
-  extern __shared__ __align__(16) float sm[];
+  __shared__ __align__(16) float sm[2 * 2 * kKmatChunk * 132];   // operands, then the staged tile
+  float (*As)[kKmatChunk][132] = reinterpret_cast<float (*)[kKmatChunk][132]>(sm);
+  float (*Bs)[kKmatChunk][132] = reinterpret_cast<float (*)[kKmatChunk][132]>(sm + 2 * kKmatChunk * 132);
   if (cta_failed(st)) return;
   const int t = blockIdx.y;
   const int j = t * B, nJ = min(B, b - j);
   const int q0 = j + blockIdx.x * 128;
   if (q0 >= b) return;
-  float* Ujj = sm;                 // [B][B]  Ujj[r][p] = U[j+r][j+p] (upper, zero below)
-  float* Ut = sm + B * B;          // [B][128] Ut[r][qq] = U[j+r][q0+qq]
-  for (int idx = threadIdx.x; idx < B * B; idx += blockDim.x) {
-    int r = idx / B, p = idx % B;
-    Ujj[idx] = (r < nJ && p < nJ && r <= p) ? H[(long long)(j + r) * b + j + p] : 0.f;
-  }
-  for (int idx = threadIdx.x; idx < B * 128; idx += blockDim.x) {
-    int r = idx >> 7, qq = idx & 127;
-    // U is upper triangular: entries left of its diagonal are zero (H's storage there is stale)
-    Ut[idx] = (r < nJ && q0 + qq < b && q0 + qq >= j + r) ? H[(long long)(j + r) * b + q0 + qq] : 0.f;
-  }
-  __syncthreads();
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  // loader: row r0 + (tid >> 5) + 8h of the chunk, columns 4 (tid & 31) .. + 3
+  auto load = [&](int r0, float4 (&a)[2], float4 (&c)[2]) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int r = r0 + (tid >> 5) + 8 * h, col = 4 * (tid & 31);
+      float va[4] = {0.f, 0.f, 0.f, 0.f}, vb[4] = {0.f, 0.f, 0.f, 0.f};
+      if (r < nJ) {
+        const float* urow = H + (long long)(j + r) * b;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int p = col + e, q = q0 + col + e;
+          va[e] = (p < nJ && p >= r) ? urow[j + p] : 0.f;     // U[j+r][j+p], upper
+          vb[e] = (q < b && q >= j + r) ? urow[q] : 0.f;      // U[j+r][q], upper
+        }
+      }
+      a[h] = make_float4(va[0], va[1], va[2], va[3]);
+      c[h] = make_float4(vb[0], vb[1], vb[2], vb[3]);
+    }
+  };
   float acc[8][8] = {};
-  for (int r = 0; r < nJ; ++r) {
-    float pv[8], qv[8];
+  float4 ra[2], rb[2];
+  int buf = 0;
+  load(0, ra, rb);
+  for (int r0 = 0; r0 < nJ; r0 += kKmatChunk) {
 #pragma unroll
-    for (int x = 0; x < 8; ++x) pv[x] = (ty + 16 * x < B) ? Ujj[r * B + ty + 16 * x] : 0.f;
+    for (int h = 0; h < 2; ++h) {
+      const int rr = (tid >> 5) + 8 * h, col = 4 * (tid & 31);
+      *reinterpret_cast<float4*>(&As[buf][rr][col]) = ra[h];
+      *reinterpret_cast<float4*>(&Bs[buf][rr][col]) = rb[h];
+    }
+    __syncthreads();
+    if (r0 + kKmatChunk < nJ) load(r0 + kKmatChunk, ra, rb);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) qv[e] = Ut[r * 128 + tx + 16 * e];
+    for (int rr = 0; rr < kKmatChunk; ++rr) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][rr][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][rr][64 + ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][rr][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][rr][64 + tx * 4]);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-    for (int x = 0; x < 8; ++x)
+      for (int x = 0; x < 8; ++x)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[x][e] = fmaf(pv[x], qv[e], acc[x][e]);
+        for (int y = 0; y < 8; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
+    }
+    buf ^= 1;   // the next chunk goes to the other stage: one barrier per chunk suffices
   }
-  // stage the tile transposed, T[qq][p], then write rows q with p contiguous
-  __syncthreads();
-  float* T = sm;
-  const int ldt = B + 1;
-#pragma unroll
-  for (int x = 0; x < 8; ++x) {
-    const int p = ty + 16 * x;
-    if (p >= B) continue;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) T[(tx + 16 * e) * ldt + p] = acc[x][e];
-  }
-  __syncthreads();
+  // acc[x][y] = K_t[p][q] with p = (x < 4 ? 4ty + x : 64 + 4ty + x - 4), q = q0 + (same with tx, y)
   float* Kin = K_in + (size_t)t * B * B;
   float* Kh = K_hi + (size_t)t * b * B;
   float* Kl = K_lo + (size_t)t * b * B;
-  for (int idx = threadIdx.x; idx < 128 * B; idx += blockDim.x) {
-    const int qq = idx / B, p = idx - qq * B;
-    const int q = q0 + qq;
-    if (q >= b || p >= nJ) continue;
-    const float v = T[qq * ldt + p];
-    const float h = tf32_head(v);
-    Kh[(size_t)q * B + p] = h;
-    Kl[(size_t)q * B + p] = v - h;
-    if (q < j + nJ) Kin[(size_t)(q - j) * B + p] = v;  // K_t[p][q] = K_t[q-j][j+p]
+  float (*T)[129] = reinterpret_cast<float (*)[129]>(sm);   // 64 q rows x 128 p
+  for (int half = 0; half < 2; ++half) {
+    __syncthreads();   // the operands (or the previous half) are no longer read
+#pragma unroll
+    for (int y = 0; y < 8; ++y) {
+      const int qq = y < 4 ? tx * 4 + y : 64 + tx * 4 + y - 4;
+      if ((qq >> 6) != half) continue;
+#pragma unroll
+      for (int x = 0; x < 8; ++x) {
+        const int p = x < 4 ? ty * 4 + x : 64 + ty * 4 + x - 4;
+        T[qq & 63][p] = acc[x][y];
+      }
+    }
+    __syncthreads();
+    for (int idx = tid; idx < 64 * B; idx += blockDim.x) {
+      const int qq = idx / B, p = idx - qq * B;
+      const int q = q0 + half * 64 + qq;
+      if (q >= b || p >= nJ) continue;
+      const float v = T[qq][p];
+      const float h = tf32_head(v);
+      Kh[(size_t)q * B + p] = h;
+      Kl[(size_t)q * B + p] = v - h;
+      if (q < j + nJ) Kin[(size_t)(q - j) * B + p] = v;  // K_t[p][q] = K_t[q-j][j+p]
+    }
   }
 }
 
-static int kmat_smem_bytes(int B) {
-  const int operands = B * B + B * 128, staged = 128 * (B + 1);
-  return (operands > staged ? operands : staged) * 4;
-}
 
 // ------------------------------------------------------------------ stream
 
@@ -435,9 +464,6 @@ static cudaError_t prune_init(PruneRun& R, const pwp_config* cfg, int c, int b, 
                                           kHist1Bins * 4);
     if (e0 == cudaSuccess)
       e0 = cudaFuncSetAttribute(stream_kernel<kObs>, cudaFuncAttributeMaxDynamicSharedMemorySize, kHist1Bins * 4);
-    if (e0 == cudaSuccess)
-      e0 = cudaFuncSetAttribute(kmat_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                kmat_smem_bytes(kMaxBlock));
     int dev = 0, nsm = kNumSM;
     if (e0 == cudaSuccess) e0 = cudaGetDevice(&dev);
     if (e0 == cudaSuccess) e0 = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
@@ -492,7 +518,7 @@ static cudaError_t prune_setup(PruneRun& R, const void* W, int wtype, bool stats
   ++*nl;
   if (R.thanos) {
     dim3 g((R.b + 127) / 128, R.nblk);
-    launch_pdl(kmat_kernel, dim3(g), dim3(256), kmat_smem_bytes(R.B), s, (const float*)R.H, R.b, R.B, R.pb.K_in,
+    launch_pdl(kmat_kernel, dim3(g), dim3(256), 0, s, (const float*)R.H, R.b, R.B, R.pb.K_in,
                R.pb.K_hi, R.pb.K_lo, (const pwp_stats*)R.st);
     ++*nl;
   }
