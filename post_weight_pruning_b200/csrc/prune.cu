@@ -85,7 +85,7 @@ __global__ void prep_diag_kernel(const float* __restrict__ H, int b, const float
 // loaded), and the tile is staged transposed, 64 columns at a time, so that every output
 // row is written contiguously.
 constexpr int kKmatChunk = 16;
-__global__ void __launch_bounds__(256) kmat_kernel(const float* __restrict__ H, int b, int B,
+__global__ void __launch_bounds__(256, 2) kmat_kernel(const float* __restrict__ H, int b, int B,
                                                    float* __restrict__ K_in, float* __restrict__ K_hi,
                                                    float* __restrict__ K_lo, const pwp_stats* st) {
   pdl_enter();
