@@ -1,5 +1,7 @@
 // Launch counting and optional per-kernel-class CUDA-event timing.
 #include <atomic>
+#include <cstdio>
+#include <cstdlib>
 #include <vector>
 
 #include "pwp_internal.cuh"
@@ -11,6 +13,28 @@ constexpr long long kDefaultWaitLimit = 1ll << 26;
 std::atomic<long long> g_wait_limit{kDefaultWaitLimit};
 
 void count_launches(long long n) { g_launches += n; }
+
+bool trace_launches() {
+  static const bool on = [] {
+    const char* v = std::getenv("PWP_TRACE");
+    return v != nullptr && v[0] != '\0' && v[0] != '0';
+  }();
+  return on;
+}
+
+void trace_launch(const void* kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t s, cudaError_t launched) {
+  const char* name = nullptr;
+  if (cudaFuncGetName(&name, kernel) != cudaSuccess || name == nullptr) name = "?";
+  std::fprintf(stderr, "pwp launch %s grid (%u,%u,%u) block %u smem %zu: %s\n", name, grid.x, grid.y, grid.z,
+               block.x, smem, cudaGetErrorString(launched));
+  std::fflush(stderr);
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(s, &cap);
+  if (launched != cudaSuccess || cap != cudaStreamCaptureStatusNone) return;
+  const cudaError_t e = cudaStreamSynchronize(s);
+  std::fprintf(stderr, "pwp   done %s: %s\n", name, cudaGetErrorString(e));
+  std::fflush(stderr);
+}
 long long wait_limit() { return g_wait_limit.load(); }
 
 namespace {

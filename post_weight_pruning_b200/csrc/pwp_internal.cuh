@@ -33,10 +33,9 @@ __device__ __forceinline__ void pdl_enter() {
   pdl_release();
 }
 
-// Launch with programmatic stream serialisation (the kernel must begin with pdl_enter()).
 template <typename... KArgs, typename... Args>
-inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                              Args... args) {
+inline cudaError_t launch_pdl_plain(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                    Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -48,6 +47,25 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+// Launch tracing for diagnosis (PWP_TRACE=1 in the environment, read once): every launch
+// through launch_pdl prints the kernel's name and shape to stderr, then waits for the
+// stream (unless it is being captured) and prints how the kernel ended, so the last line
+// names a kernel that does not finish.  Off by default; profile.cu.
+bool trace_launches();
+void trace_launch(const void* kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t s, cudaError_t launched);
+
+// Launch with programmatic stream serialisation (the kernel must begin with pdl_enter()).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+  if (trace_launches()) {
+    const cudaError_t e = launch_pdl_plain(kernel, grid, block, smem, s, args...);
+    trace_launch(reinterpret_cast<const void*>(kernel), grid, block, smem, s, e);
+    return e;
+  }
+  return launch_pdl_plain(kernel, grid, block, smem, s, args...);
 }
 
 constexpr int kNumSM = 148;              // B200

@@ -14,9 +14,13 @@ namespace tc {
 // their limit from a launch parameter (pwp_set_wait_limit; kDefaultSpinLimit unless a
 // caller changed it); the waits that only let copies or MMAs already in flight finish
 // before a CTA leaves always use kDrainLimit, so that a shortened limit can never let a
-// CTA exit with asynchronous work still writing its shared or tensor memory.
+// CTA exit with asynchronous work still writing its shared or tensor memory.  Every wait
+// also gives up after kWaitNs of wall-clock time (the global timer), however many polls
+// that took: a poll of a phase that is not complete may suspend the thread for a while,
+// so a poll count alone does not bound the time.  A legitimate wait lasts microseconds.
 constexpr long long kDefaultSpinLimit = 1ll << 26;
 constexpr long long kDrainLimit = 1ll << 26;
+constexpr unsigned long long kWaitNs = 2000000000ull;   // 2 s
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -47,19 +51,32 @@ __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
   return done != 0;
 }
 
-// Bounded wait for the phase of the given parity to complete.
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait for the phase of the given parity to complete: at most `limit` polls and
+// kWaitNs of time.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit) {
-  for (long long i = 0; i < limit; ++i)
+  if (limit > 0 && mbar_try(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (long long i = 1; i < limit; ++i) {
     if (mbar_try(bar, parity)) return true;
+    if ((i & 15) == 0 && global_ns() - t0 > kWaitNs) return false;
+  }
   return false;
 }
 
 // Bounded wait that also gives up as soon as another role of the CTA raised *abort.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort,
                                           long long limit) {
-  for (long long i = 0; i < limit; ++i) {
+  if (limit > 0 && mbar_try(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (long long i = 1; i < limit; ++i) {
     if (mbar_try(bar, parity)) return true;
-    if ((i & 63) == 63 && *abort) return false;
+    if ((i & 15) == 0 && (*abort || global_ns() - t0 > kWaitNs)) return false;
   }
   return false;
 }
