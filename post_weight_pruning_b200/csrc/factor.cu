@@ -295,8 +295,9 @@ __global__ void __launch_bounds__(256) chol_panel_kernel(float* __restrict__ H, 
 
 // Symmetric update of the top-left part: A[r][s] -= sum_t V[r][p0+t] V[s][p0+t] for
 // r <= s < p0, 128x128 tiles on or above the diagonal, 8x8 outputs per thread.  The CTA
-// whose tile holds the next panel's diagonal block [p0-NB, p0) then factors it.
-__global__ void __launch_bounds__(256) chol_update_kernel(float* __restrict__ H, int b, int p0, int nb,
+// whose tile holds the next panel's diagonal block [p0-NB, p0) then factors it (reading
+// back entries of H its other threads wrote: H is not __restrict__).
+__global__ void __launch_bounds__(256) chol_update_kernel(float* H, int b, int p0, int nb,
                                                           float* __restrict__ Vinv_next,
                                                           pwp_stats* st) {
   pdl_enter();

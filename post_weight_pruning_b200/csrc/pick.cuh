@@ -14,6 +14,13 @@
 // previous block's bin; only when this block's bin differs is the region read again.  Among
 // entries equal to T the order is (column, row) -- the pages fix none -- so when only some
 // tied entries are taken, the cut-off position inside the current block is located too.
+//
+// One thread takes each decision and records it in the control block for later kernels;
+// the CTA's other threads get it through shared memory (Shared), never by re-reading the
+// control block, and the kernels that call these functions take their control-block and
+// histogram pointers without __restrict__: a value written by one thread of a kernel and
+// read by another through global memory must not be cached by the compiler across the
+// barrier in between.
 #pragma once
 
 #include <climits>
@@ -32,6 +39,13 @@ struct Shared {
   long long need;
   int sel;
   int last;
+  // the decisions of the block's selection, for every thread of the CTA
+  int mode;        // something is removed
+  int ready;       // the predicted level-2 histogram holds the chosen bin
+  int tie_scan;    // the cut-off among tied entries has to be located
+  unsigned int T;  // the threshold key
+  long long r1;    // rank of the take-th key inside the chosen level-1 bin
+  long long m;     // entries tied at T that are taken
 };
 
 __device__ __forceinline__ long long warp_sum_ll(long long v) {
@@ -116,7 +130,8 @@ __device__ void find_rank(const unsigned int* __restrict__ hist, long long rank,
 // the scoring pass predicted it (then the level-2 histogram is ready).  Clears the level-1
 // histogram for the next pass.
 // (pruned: the removals so far over every row the budget counts; -1 for this call's own.)
-__device__ inline void level1(Ctl* ctl, unsigned int* __restrict__ hist1, long long region_n, int global_budget,
+// On return sh.mode, sh.ready and sh.r1 hold the outcome for every thread.
+__device__ inline void level1(Ctl* ctl, unsigned int* hist1, long long region_n, int global_budget,
                               long long quota, pwp_stats* st, Shared& sh, int bar, int tid, long long pruned = -1) {
   if (tid == 0) {
     const long long r = global_budget ? ctl->zstar - (pruned >= 0 ? pruned : ctl->pruned) : quota;
@@ -130,6 +145,10 @@ __device__ inline void level1(Ctl* ctl, unsigned int* __restrict__ hist1, long l
     ctl->dirty_reread = 0;
     ctl->tie_scan = 0;
     sh.take = take;
+    sh.mode = take > 0 ? 1 : 0;
+    sh.ready = 0;
+    sh.tie_scan = 0;
+    sh.r1 = 0;
   }
   sync(bar);
   const long long take = sh.take;
@@ -141,6 +160,7 @@ __device__ inline void level1(Ctl* ctl, unsigned int* __restrict__ hist1, long l
       if (bin < 0) {
         set_error(st, PWP_EBUDGET, kSitePick);
         ctl->mode = 0;
+        sh.mode = 0;
       } else {
         const bool hit = ctl->b1_valid && ctl->b1 == (unsigned int)bin;
         ctl->l2_ready = hit ? 1 : 0;
@@ -150,6 +170,8 @@ __device__ inline void level1(Ctl* ctl, unsigned int* __restrict__ hist1, long l
         ctl->b1_valid = 1;
         ctl->r1 = (unsigned int)(take - before);
         ctl->count_less = before;
+        sh.ready = hit ? 1 : 0;
+        sh.r1 = take - before;
       }
     }
   }
@@ -158,12 +180,14 @@ __device__ inline void level1(Ctl* ctl, unsigned int* __restrict__ hist1, long l
 }
 
 // The exact key T from the level-2 histogram of the chosen level-1 bin (the predicted one
-// when it held, else the re-read one), the number m of entries tied at T that are taken,
-// and whether the cut-off among the ties has to be located.
-__device__ inline void level2(Ctl* ctl, Level2 l2, pwp_stats* st, Shared& sh, int bar, int tid) {
-  const long long r1 = ctl->r1;
-  const unsigned int* h2 = ctl->l2_ready ? l2.pred : l2.reread;
-  const unsigned int* h2s = ctl->l2_ready ? l2.pred_sum : l2.reread_sum;
+// when `ready`, else the re-read one), the number m of entries tied at T that are taken,
+// and whether the cut-off among the ties has to be located.  r1: the rank inside the bin
+// (level1's sh.r1, or the control block's when level1 ran in an earlier kernel).  On
+// return sh.mode, sh.T, sh.m and sh.tie_scan hold the outcome for every thread.
+__device__ inline void level2(Ctl* ctl, Level2 l2, long long r1, int ready, pwp_stats* st, Shared& sh, int bar,
+                              int tid) {
+  const unsigned int* h2 = ready ? l2.pred : l2.reread;
+  const unsigned int* h2s = ready ? l2.pred_sum : l2.reread_sum;
   int sb;
   long long before_s;
   find_rank<kHist2SumBins>(h2s, r1, &sb, &before_s, sh, bar, tid);
@@ -176,6 +200,8 @@ __device__ inline void level2(Ctl* ctl, Level2 l2, pwp_stats* st, Shared& sh, in
     if (tid == 0) {
       set_error(st, PWP_EBUDGET, kSitePick);
       ctl->mode = 0;
+      sh.mode = 0;
+      sh.tie_scan = 0;
     }
     sync(bar);
     return;
@@ -185,13 +211,19 @@ __device__ inline void level2(Ctl* ctl, Level2 l2, pwp_stats* st, Shared& sh, in
     const long long ties = h2[lo];
     const long long count_less = ctl->count_less + before_s + before_sub;
     const long long m = ctl->take - count_less;   // 1 <= m <= ties
-    ctl->T = (ctl->b1 << kKeyLoBits) | (unsigned int)lo;
+    const unsigned int T = (ctl->b1 << kKeyLoBits) | (unsigned int)lo;
+    const int tie_scan = m < ties ? 1 : 0;        // some but not all tied entries are taken
+    ctl->T = T;
     ctl->ties = ties;
     ctl->m = m;
     ctl->count_less = count_less;
     ctl->pstar = LLONG_MAX;
     if (ties > 1) st->tie_blocks += 1;
-    ctl->tie_scan = m < ties ? 1 : 0;   // some but not all tied entries are taken
+    ctl->tie_scan = tie_scan;
+    sh.mode = 1;
+    sh.T = T;
+    sh.m = m;
+    sh.tie_scan = tie_scan;
   }
   sync(bar);
 }
@@ -199,9 +231,8 @@ __device__ inline void level2(Ctl* ctl, Level2 l2, pwp_stats* st, Shared& sh, in
 // Counts, per block column, of the block's entries whose key equals T, over the rows
 // [r_begin, r_end) with stride r_step, added to tie_count (lane l: columns l + 32e).
 template <int SCORE>
-__device__ inline void count_ties(const Ctl* ctl, Level2 l2, const float* __restrict__ W, int b, int j, int j1,
+__device__ inline void count_ties(unsigned int T, Level2 l2, const float* W, int b, int j, int j1,
                                   const float* __restrict__ sc, int r_begin, int r_end, int r_step) {
-  const unsigned int T = ctl->T;
   const int nJ = j1 - j, lane = threadIdx.x & 31;
   constexpr int E = kMaxBlock / 32;
   unsigned int cnt[E];
@@ -226,12 +257,10 @@ __device__ inline void count_ties(const Ctl* ctl, Level2 l2, const float* __rest
 // column holding the m-th, then its row (the threads scan that column); the per-column
 // counts are zeroed for the next block.
 template <int SCORE>
-__device__ inline void tie_cutoff(Ctl* ctl, Level2 l2, const float* __restrict__ W, int c, int b, int j, int j1,
-                                  const float* __restrict__ sc, Shared& sh, int bar, int tid) {
+__device__ inline void tie_cutoff(Ctl* ctl, unsigned int T, long long m, Level2 l2, const float* W, int c, int b,
+                                  int j, int j1, const float* __restrict__ sc, Shared& sh, int bar, int tid) {
   const int lane = tid & 31, warp = tid >> 5;
   const int nJ = j1 - j;
-  const unsigned int T = ctl->T;
-  const long long m = ctl->m;
   if (tid == 0) {
     long long cum = 0;
     int qstar = -1;
@@ -311,7 +340,7 @@ __device__ inline void after_scoring(Ctl* ctl, unsigned int* hist1, Level2 l2, l
     return;
   }
   level1(ctl, hist1, region_n, global_budget, quota, st, sh, 1, tid);
-  if (ctl->mode != 0 && ctl->l2_ready) level2(ctl, l2, st, sh, 1, tid);
+  if (sh.mode != 0 && sh.ready) level2(ctl, l2, sh.r1, 1, st, sh, 1, tid);
 }
 
 }  // namespace pick

@@ -195,11 +195,11 @@ __global__ void __launch_bounds__(256) stream_kernel(float* __restrict__ W, int 
                                                      const float* __restrict__ Rlo, int ldr, int r_trans,
                                                      int r_upper_from, const uint8_t* __restrict__ mask,
                                                      const float* __restrict__ sc, int hist_end,
-                                                     unsigned int* __restrict__ hist1, Ctl* __restrict__ ctl,
+                                                     unsigned int* hist1, Ctl* ctl,
                                                      Level2 l2, PickArgs pk, pwp_stats* st) {
   pdl_enter();
-  unsigned int* __restrict__ h2 = l2.pred;
-  unsigned int* __restrict__ h2s = l2.pred_sum;
+  unsigned int* h2 = l2.pred;
+  unsigned int* h2s = l2.pred_sum;
   __shared__ pick::Shared psh;
   extern __shared__ unsigned int shist[];  // kHist1Bins when SCORE != 0
   __shared__ float Zs[64][33];

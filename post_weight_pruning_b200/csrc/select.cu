@@ -19,8 +19,10 @@ __device__ __forceinline__ void zero_words(unsigned int* p, int n, int first, in
   for (int i = first; i < n / 4; i += stride) p4[i] = z;
 }
 
+// ctl without __restrict__: the last CTA's threads share decisions taken by one of them
+// (through shared memory; see pick.cuh).
 template <int SCORE>
-__global__ void __launch_bounds__(pick::kThreads) select_finish_kernel(Ctl* __restrict__ ctl, Level2 l2,
+__global__ void __launch_bounds__(pick::kThreads) select_finish_kernel(Ctl* ctl, Level2 l2,
                                                                       const float* __restrict__ W, int c, int b,
                                                                       int j, int j1, int q1,
                                                                       const float* __restrict__ sc, pwp_stats* st) {
@@ -29,23 +31,27 @@ __global__ void __launch_bounds__(pick::kThreads) select_finish_kernel(Ctl* __re
   if (cta_failed(st)) return;
   const int tid = threadIdx.x;
   const int gtid = blockIdx.x * blockDim.x + tid, stride = gridDim.x * blockDim.x;
+  // the outcome of the scoring pass's last CTA (an earlier kernel)
   const int mode = ctl->mode, ready = ctl->l2_ready, tie_scan = ctl->tie_scan;
   const bool dirty_pred = ctl->dirty_pred != 0;
   if (mode != 0 && !ready) {
     // the level-2 histogram of bin b1 over the region: rows over CTAs, columns over threads
     const unsigned int b1 = ctl->b1;
+    const long long r1 = ctl->r1;
     for (int r = blockIdx.x; r < c; r += gridDim.x) {
       const float* wr = W + (long long)r * b;
       for (int q = j + tid; q < q1; q += blockDim.x)
         count_level2(key_of<SCORE>(wr[q], __ldg(sc + q)), b1, l2.reread, l2.reread_sum);
     }
     if (!pick::last_cta(&ctl->ticket, sh)) return;
-    pick::level2(ctl, l2, st, sh, 1, tid);
-    if (ctl->mode != 0 && ctl->tie_scan) {
-      pick::count_ties<SCORE>(ctl, l2, W, b, j, j1, sc, tid >> 5, c, pick::kWarps);
+    pick::level2(ctl, l2, r1, 0, st, sh, 1, tid);
+    if (sh.mode != 0 && sh.tie_scan) {
+      const unsigned int T = sh.T;
+      const long long m = sh.m;
+      pick::count_ties<SCORE>(T, l2, W, b, j, j1, sc, tid >> 5, c, pick::kWarps);
       __threadfence_block();
       pick::sync(1);
-      pick::tie_cutoff<SCORE>(ctl, l2, W, c, b, j, j1, sc, sh, 1, tid);
+      pick::tie_cutoff<SCORE>(ctl, T, m, l2, W, c, b, j, j1, sc, sh, 1, tid);
     }
     // this CTA alone clears what the block counted into
     if (dirty_pred) {
@@ -62,10 +68,12 @@ __global__ void __launch_bounds__(pick::kThreads) select_finish_kernel(Ctl* __re
     zero_words(l2.pred_sum, kHist2SumBins, gtid, stride);
   }
   if (mode != 0 && tie_scan) {
+    const unsigned int T = ctl->T;
+    const long long m = ctl->m;
     const int gwarp = gtid >> 5, nwarps = stride >> 5;
-    pick::count_ties<SCORE>(ctl, l2, W, b, j, j1, sc, gwarp, c, nwarps);
+    pick::count_ties<SCORE>(T, l2, W, b, j, j1, sc, gwarp, c, nwarps);
     if (!pick::last_cta(&ctl->ticket, sh)) return;
-    pick::tie_cutoff<SCORE>(ctl, l2, W, c, b, j, j1, sc, sh, 1, tid);
+    pick::tie_cutoff<SCORE>(ctl, T, m, l2, W, c, b, j, j1, sc, sh, 1, tid);
   }
 }
 
@@ -81,7 +89,7 @@ __global__ void publish_count_kernel(const Ctl* __restrict__ ctl, unsigned int* 
   hist1[kHist1Bins] = (unsigned int)ctl->pruned;
 }
 
-__global__ void __launch_bounds__(pick::kThreads) pick_bin_kernel(Ctl* ctl, unsigned int* __restrict__ hist1,
+__global__ void __launch_bounds__(pick::kThreads) pick_bin_kernel(Ctl* ctl, unsigned int* hist1,
                                                                   PickArgs pk, pwp_stats* st) {
   pdl_enter();
   __shared__ pick::Shared sh;
@@ -110,7 +118,7 @@ __global__ void __launch_bounds__(pick::kThreads) pick_key_kernel(Ctl* ctl, Leve
   pdl_enter();
   __shared__ pick::Shared sh;
   if (cta_failed(st) || ctl->mode == 0) return;
-  pick::level2(ctl, l2, st, sh, 1, threadIdx.x);
+  pick::level2(ctl, l2, (long long)ctl->r1, ctl->l2_ready, st, sh, 1, threadIdx.x);
 }
 
 template <int SCORE>
@@ -120,7 +128,7 @@ __global__ void __launch_bounds__(256) count_ties_kernel(const Ctl* __restrict__
   pdl_enter();
   if (cta_failed(st) || ctl->mode == 0 || !ctl->tie_scan) return;
   const int gtid = blockIdx.x * blockDim.x + threadIdx.x, stride = gridDim.x * blockDim.x;
-  pick::count_ties<SCORE>(ctl, l2, W, b, j, j1, sc, gtid >> 5, c, stride >> 5);
+  pick::count_ties<SCORE>(ctl->T, l2, W, b, j, j1, sc, gtid >> 5, c, stride >> 5);
 }
 
 // The cut-off among tied entries when the rows are spread over ranks: (column, row) order

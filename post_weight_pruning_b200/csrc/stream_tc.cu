@@ -93,10 +93,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __grid_constant__ CUtensorMap mrh, const __grid_constant__ CUtensorMap mrl,
                      const __grid_constant__ CUtensorMap mw, int c, int b, int u0, int j, int Bp, int upper,
                      const uint8_t* __restrict__ mask, const float* __restrict__ sc, int hist_end,
-                     unsigned int* __restrict__ hist1, Ctl* __restrict__ ctl, Level2 l2, PickArgs pk,
+                     unsigned int* hist1, Ctl* ctl, Level2 l2, PickArgs pk,
                      pwp_stats* st, long long spin) {
-  unsigned int* __restrict__ h2 = l2.pred;
-  unsigned int* __restrict__ h2s = l2.pred_sum;
+  unsigned int* h2 = l2.pred;
+  unsigned int* h2s = l2.pred_sum;
   __shared__ pick::Shared psh;
   pdl_enter();
   extern __shared__ uint8_t smem_raw[];
