@@ -250,7 +250,8 @@ def prune_layer(W, *, Xt=None, H=None, sparsity=0.5, pattern="unstructured", nm=
     (for the processed rows) used as every block's selection instead of choosing one
     (Thanos only; for the global budget over all rows, each block also records in
     ``blocks`` the selection the budget loop would have made on the replayed state --
-    ``chosen``, with its residual count and thresholds).  Once the masks are given the rows do not interact -- the loss is a sum
+    ``chosen``, with its residual count and thresholds; for N:M, the groups' ``chosen``
+    removals and their ``nm_gap`` on the replayed state).  Once the masks are given the rows do not interact -- the loss is a sum
     of per-row terms ([THANOS] "The layer-reconstruction lens") and each row's update
     depends only on its own selected set ([THANOS] "Contribution one") -- so any subset of
     rows of a layer pruned elsewhere can be replayed exactly, also under the global budget.
@@ -318,6 +319,10 @@ def prune_layer(W, *, Xt=None, H=None, sparsity=0.5, pattern="unstructured", nm=
             if fixed_mask is not None:
                 M = fixed_mask[:, j:j1]
                 dscore[:, j:j1] = wanda_scores(What[:, j:j1], g_diag[j:j1])
+                if not unstructured:
+                    # the groups the N:M rule would remove on this (replayed) state
+                    chosen, gaps = nm_mask(dscore[:, j:j1], n_keep, m_grp)
+                    info.update(chosen=chosen, nm_gap=gaps)
                 if unstructured and rows is None:
                     # what step 3 of the budget loop would choose on this (replayed) state,
                     # with the residual count left by the given mask's earlier blocks

@@ -9,10 +9,15 @@ independent of the GPU:
   - the unstructured layers too large for a full oracle run: the GPU's own mask replayed
     row by row on a seeded subset (exact: once the masks are fixed, rows do not interact),
     plus the first block's selection, which depends only on W and the column norms.
-Bars: every invariant bit-exact; masks agree at >= 99.99% and differ only where the
-oracle's own score sits within 1e-6 (relative) of its selection boundary; W-hat within
-1e-3 relative Frobenius; reconstruction loss within 1e-2; the factor U within 1e-4 of the
-fp64 U; H within 1e-5 of fp64 (2e-5 over 262144 tokens), relative to sqrt(H_ii H_jj)."""
+Bars: every invariant bit-exact; masks agree at >= 99.99% with the independent oracle run
+and reconstruction loss within 1e-2 of it; ties judged on the GPU's own trajectory -- the
+oracle replays the GPU's masks in fp64 and, block by block, applies the selection rule to
+the replayed state: the GPU's block masks may differ from that choice only where the
+score sits within 1e-6 (relative) of the boundary, and W-hat is within 1e-3 relative
+Frobenius of the replay (once a row has taken a different weight at a near-tie, its later
+weights legitimately differ from the independent run's, so W-hat is not compared with
+that run); the factor U within 1e-4 of the fp64 U; H within 1e-5 of fp64 (2e-5 over
+262144 tokens), relative to sqrt(H_ii H_jj)."""
 import functools
 import os
 
@@ -106,7 +111,6 @@ def test_q_proj_whole_layer_matches_the_oracle():
     res = P.compare(W, wl.dtype, (W_hat, mask, st), orc, pattern="unstructured", nm=(0, 0), block=wl.block,
                     tie_tol=TIE_TOL)
     assert res["agree"] >= P.MASK_AGREE, res
-    assert res["w_rel"] <= P.W_REL_TOL, res
     lg = oracle.recon_loss(W64, W_hat, 0.5 * H64)
     assert abs(lg - orc["loss"]) <= P.LOSS_REL_TOL * orc["loss"], (lg, orc["loss"])
     # Disagreements only at ties, judged on the GPU's own trajectory: once a row takes a
@@ -142,8 +146,22 @@ def test_nm_layer_row_subset_matches_the_oracle(name):
     W64 = synth.to_f64(W, wl.dtype)
     orc = oracle.prune_layer(W64, H=H64, pattern="nm", nm=wl.nm, block=wl.block, damp=wl.damp, rows=rows)
     res = F.compare_rows(W64[rows], W_hat[rows], mask[rows], orc, 0.5 * H64, nm=wl.nm, tie_tol=TIE_TOL)
-    assert res["zeros_exact"] and res["agree"] >= P.MASK_AGREE and res["n_dis_not_tie"] == 0, res
-    assert res["w_rel"] <= P.W_REL_TOL and res["loss_rel"] <= P.LOSS_REL_TOL, res
+    assert res["zeros_exact"] and res["agree"] >= P.MASK_AGREE and res["loss_rel"] <= P.LOSS_REL_TOL, res
+    # ties judged on the GPU's own trajectory: the oracle replays the GPU's masks of those
+    # rows; every block's GPU groups may differ from the N:M rule on the replayed state only
+    # at near-ties, and W-hat follows the replay
+    rep = oracle.prune_layer(W64, H=H64, pattern="nm", nm=wl.nm, block=wl.block, damp=wl.damp, rows=rows,
+                             fixed_mask=mask[rows])
+    assert float(np.linalg.norm(W_hat[rows] - rep["W"]) / np.linalg.norm(rep["W"])) <= P.W_REL_TOL, res
+    m = wl.nm[1]
+    worst, n_off = 0.0, 0
+    for blk in rep["blocks"]:
+        j = blk["j"]
+        chosen = blk["chosen"]
+        for k, q in np.argwhere(mask[rows][:, j:j + chosen.shape[1]] != chosen):
+            worst = max(worst, float(blk["nm_gap"][k, q // m]))
+            n_off += 1
+    assert worst <= TIE_TOL, (n_off, worst, res)
 
 
 def test_down_proj_unstructured_rows_replay_the_oracle():

@@ -582,6 +582,28 @@ def test_fixed_mask_replay_records_the_selection_of_the_replayed_state():
     assert diff.tolist() == [[k, q]]
 
 
+def test_fixed_mask_replay_records_the_nm_choice_of_the_replayed_state():
+    """N:M: replaying the full run's own mask, every block's recorded choice is the mask
+    itself with the run's own group gaps; with one group of block 0 changed, block 0's
+    recorded choice is still the rule's (the choice precedes the block's update), so it
+    differs from the replayed mask exactly in that group."""
+    rng = np.random.default_rng(29)
+    Xt = rng.normal(size=(40, 16))
+    W = rng.normal(0, 0.02, size=(6, 16))
+    full = oracle.prune_layer(W, Xt=Xt, pattern="nm", nm=(2, 4), block=8)
+    again = oracle.prune_layer(W, Xt=Xt, pattern="nm", nm=(2, 4), block=8, fixed_mask=full["mask"])
+    for blk in again["blocks"]:
+        j = blk["j"]
+        assert np.array_equal(blk["chosen"], full["mask"][:, j:j + 8])
+        assert np.allclose(blk["nm_gap"], full["nm_gap"][:, j // 4: j // 4 + 2])
+    changed = full["mask"].copy()
+    k = 3
+    changed[k, 0:4] = ~changed[k, 0:4]          # the other two of the group's four
+    other = oracle.prune_layer(W, Xt=Xt, pattern="nm", nm=(2, 4), block=8, fixed_mask=changed)
+    diff = np.argwhere(other["blocks"][0]["chosen"] != changed[:, :8])
+    assert sorted(diff.tolist()) == [[k, q] for q in range(4)]
+
+
 # --------------------------------------------------------------------------- outlier rows (alpha)
 
 def test_alpha_keeps_floor_alpha_c_rows_dense_and_gives_the_stated_total_sparsity():
