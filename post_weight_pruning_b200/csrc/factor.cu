@@ -57,20 +57,84 @@ __global__ void __launch_bounds__(1024) damp_kernel(float* __restrict__ H, int b
   for (int q = threadIdx.x; q < b; q += blockDim.x) H[(long long)q * b + q] += lam;
 }
 
+// Pivot K of the one-warp factorisation below (K a template parameter, so that every
+// register index is a compile-time constant).  Lane k: L[k][k] and row k of X made final;
+// lanes below: L[lane][K], then the elimination of column K of L and row K of X.
+template <int K>
+__device__ __forceinline__ void chol_inv_step(float (&p)[32], float (&x)[32], int lane, bool& ok) {
+  constexpr unsigned kAll = 0xffffffffu;
+  const float piv = __shfl_sync(kAll, p[K], K);
+  ok = ok && (piv > 0.f) && isfinite(piv);
+  const float il = rsqrtf(piv);
+  p[K] = lane == K ? piv * il : (lane > K ? p[K] * il : p[K]);
+  const float xs = lane == K ? il : 1.f;
+#pragma unroll
+  for (int t = 0; t <= K; ++t) x[t] *= xs;
+#pragma unroll
+  for (int j = K + 1; j < 32; ++j) {
+    const float ljk = __shfl_sync(kAll, p[K], j);          // L[j][K]
+    if (lane >= j) p[j] = fmaf(-p[K], ljk, p[j]);
+  }
+#pragma unroll
+  for (int t = 0; t <= K; ++t) {
+    const float xkt = __shfl_sync(kAll, x[t], K);          // X[K][t], final
+    if (lane > K) x[t] = fmaf(-p[K], xkt, x[t]);
+  }
+}
+
+template <int K>
+struct CholInvSteps {
+  static __device__ __forceinline__ void run(float (&p)[32], float (&x)[32], int lane, bool& ok) {
+    chol_inv_step<K>(p, x, lane, ok);
+    CholInvSteps<K + 1>::run(p, x, lane, ok);
+  }
+};
+template <>
+struct CholInvSteps<32> {
+  static __device__ __forceinline__ void run(float (&)[32], float (&)[32], int, bool&) {}
+};
+
+// One warp factors and inverts a 32 x 32 diagonal block of P (below): P[b0.., b0..] =
+// L L^T with L lower, X = L^-1.  Lane i holds row i of both in registers; pivots and rows
+// travel by shuffles.  At pivot k, row k of X (which already carries every earlier
+// pivot's elimination) becomes final once divided by L[k][k], and is eliminated from the
+// rows below it together with column k of L.  Writes L and X (lower) back to P and X.
+// Returns false on a non-positive pivot (the same on every lane).
+template <typename FP, typename FX>
+__device__ __forceinline__ bool warp_chol_inv32(FP P, FX X, int b0, int lane) {
+  float p[32], x[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    p[j] = j <= lane ? P(b0 + lane, b0 + j) : 0.f;
+    x[j] = j == lane ? 1.f : 0.f;
+  }
+  bool ok = true;
+  CholInvSteps<0>::run(p, x, lane, ok);
+#pragma unroll
+  for (int j = 0; j < 32; ++j)
+    if (j <= lane) {
+      P(b0 + lane, b0 + j) = p[j];
+      X(b0 + lane, b0 + j) = x[j];
+    }
+  return ok;
+}
+
 // Factor the nb x nb diagonal block (nb <= 64) held in A (symmetric; the upper triangle
 // is read) as A = V V^T with V upper triangular, and invert V.  256 threads.
 // Working on the reversed matrix P = J A J (J the reversal; P[r][s] = A[63-r][63-s], so
 // P's lower triangle is A's upper one and the work happens in place), this is the
-// ordinary Cholesky P = L L^T from the top-left, with V = J L J and V^-1 = J L^-1 J.
-// Blocked by 16: for each block column k, one warp factors the 16x16 diagonal block and
-// inverts it in registers (lane l holds row l of both; pivots and rows travel by
-// shuffles), then all threads form the panel L_ik = P_ik X_kk^T (X = L^-1) below it and
-// the trailing update P_ij -= L_ik L_jk^T; finally the off-diagonal blocks of X follow,
-// X_ik = -X_ii sum_{k <= t < i} L_it X_tk, by growing distance from the diagonal.  Rows
-// and columns beyond nb are an identity pad.  On return A's upper triangle holds V and Wi
-// holds V^-1 (upper, zero below).  Returns false on a non-positive pivot (recorded in st).
+// ordinary Cholesky P = L L^T from the top-left, with V = J L J and V^-1 = J X J for
+// X = L^-1.  In 32 x 32 blocks:
+//   L11 L11^T = P11, X11 = L11^-1            (warp 0);
+//   L21 = P21 X11^T, then S = P22 - L21 L21^T  (all threads);
+//   L22 L22^T = S, X22 = L22^-1               (warp 0), while the other warps form
+//                                              T = L21 X11 in X21's place;
+//   X21 = -X22 T                              (all threads).
+// Rows and columns beyond nb (A indices >= nb) are an identity pad.  On return A's upper
+// triangle holds V and Wi holds V^-1 (upper, zero below).  Returns false on a
+// non-positive pivot (recorded in st).
 __device__ bool factor_diag_block(float (*A)[NB + 1], float (*Wi)[NB + 1], int nb, int* bad, pwp_stats* st) {
-  constexpr int BS = 16, NBK = NB / BS;
+  constexpr int H2 = NB / 2;   // 32
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   auto P = [&](int r, int c) -> float& { return A[NB - 1 - r][NB - 1 - c]; };
   auto X = [&](int r, int c) -> float& { return Wi[NB - 1 - r][NB - 1 - c]; };
@@ -82,149 +146,73 @@ __device__ bool factor_diag_block(float (*A)[NB + 1], float (*Wi)[NB + 1], int n
   }
   if (tid == 0) *bad = 0;
   __syncthreads();
-  for (int kb = 0; kb < NBK; ++kb) {
-    const int k0 = BS * kb;
-    if (warp == 0) {
-      // 16x16 diagonal block: lane l (< 16) holds row l of the block and of its inverse
-      const int l = lane & (BS - 1);
-      const bool act = lane < BS;
-      float d[BS], x[BS];
-#pragma unroll
-      for (int c = 0; c < BS; ++c) {
-        d[c] = (act && c <= l) ? P(k0 + l, k0 + c) : 0.f;
-        x[c] = (c == l) ? 1.f : 0.f;
-      }
-      bool ok = true;
-#pragma unroll
-      for (int c = 0; c < BS; ++c) {
-        const float piv = __shfl_sync(0xffffffffu, d[c], c);
-        ok = ok && (piv > 0.f) && isfinite(piv);
-        const float il = rsqrtf(piv);
-        if (l == c) {
-          d[c] = piv * il;
-#pragma unroll
-          for (int t = 0; t <= c; ++t) x[t] *= il;
-        } else if (l > c) {
-          d[c] *= il;
-        }
-#pragma unroll
-        for (int c2 = c + 1; c2 < BS; ++c2) {
-          const float lc2 = __shfl_sync(0xffffffffu, d[c], c2);   // L[c2][c]
-          if (l > c) d[c2] = fmaf(-d[c], lc2, d[c2]);
-        }
-#pragma unroll
-        for (int t = 0; t <= c; ++t) {
-          const float xc = __shfl_sync(0xffffffffu, x[t], c);     // X[c][t], final
-          if (l > c) x[t] = fmaf(-d[c], xc, x[t]);
-        }
-      }
-      if (act) {
-#pragma unroll
-        for (int c = 0; c < BS; ++c)
-          if (c <= l) {
-            P(k0 + l, k0 + c) = d[c];
-            X(k0 + l, k0 + c) = x[c];
-          }
-      }
-      if (!ok && lane == 0) *bad = 1;
-    }
-    __syncthreads();
-    if (*bad) {
-      if (tid == 0) set_error(st, PWP_ENOTSPD, kSiteCholDiag);
-      return false;
-    }
-    // panel below the block: L_ik = P_ik X_kk^T, i > kb
-    const int nbelow = NBK - 1 - kb;
-    float lv[NBK - 1];
-#pragma unroll
-    for (int m = 0; m < NBK - 1; ++m) {
-      lv[m] = 0.f;
-      const int e = tid + blockDim.x * m;
-      if (m < nbelow && e < nbelow * BS * BS) {
-        const int ib = kb + 1 + e / (BS * BS), r = (e / BS) % BS, c = e % BS;
-        float v = 0.f;
-#pragma unroll
-        for (int t = 0; t < BS; ++t) v = fmaf(P(BS * ib + r, k0 + t), X(k0 + c, k0 + t), v);
-        lv[m] = v;
-      }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int m = 0; m < NBK - 1; ++m) {
-      const int e = tid + blockDim.x * m;
-      if (m < nbelow && e < nbelow * BS * BS) {
-        const int ib = kb + 1 + e / (BS * BS), r = (e / BS) % BS, c = e % BS;
-        P(BS * ib + r, k0 + c) = lv[m];
-      }
-    }
-    __syncthreads();
-    // trailing update of the blocks (i, j), kb < j <= i
-    const int nt = nbelow * (nbelow + 1) / 2;
-    for (int e = tid; e < nt * BS * BS; e += blockDim.x) {
-      int blk = e / (BS * BS);
-      const int r = (e / BS) % BS, c = e % BS;
-      int i = kb + 1, jb = kb + 1;
-      while (blk > i - (kb + 1)) { blk -= i - kb; ++i; }   // blocks of row i: j = kb+1 .. i
-      jb = kb + 1 + blk;
-      float v = P(BS * i + r, BS * jb + c);
-#pragma unroll
-      for (int t = 0; t < BS; ++t) v = fmaf(-P(BS * i + r, k0 + t), P(BS * jb + c, k0 + t), v);
-      P(BS * i + r, BS * jb + c) = v;
-    }
-    __syncthreads();
+  if (warp == 0) {
+    const bool ok = warp_chol_inv32(P, X, 0, lane);
+    if (!ok && lane == 0) *bad = 1;
   }
-  // off-diagonal blocks of X = L^-1, by distance dd from the diagonal (each block's sum is
-  // staged in the block itself, still zero, before the product with X_ii)
-  for (int dd = 1; dd < NBK; ++dd) {
-    const int nbk = NBK - dd;   // blocks (k + dd, k), k = 0 .. nbk-1
-    float tv[NBK - 1];
-    // tmp(k) = sum_{t = k}^{k+dd-1} L_{k+dd, t} X_{t, k}
-#pragma unroll
-    for (int m = 0; m < NBK - 1; ++m) {
-      tv[m] = 0.f;
-      const int e = tid + blockDim.x * m;
-      if (m < nbk && e < nbk * BS * BS) {
-        const int kk = e / (BS * BS), r = (e / BS) % BS, c = e % BS, ib = kk + dd;
-        float v = 0.f;
-        for (int tb = kk; tb < ib; ++tb)
-#pragma unroll
-          for (int u = 0; u < BS; ++u) v = fmaf(P(BS * ib + r, BS * tb + u), X(BS * tb + u, BS * kk + c), v);
-        tv[m] = v;
-      }
-    }
-    // stage tmp in the (still zero) X block itself, then X_ik = -X_ii tmp
-#pragma unroll
-    for (int m = 0; m < NBK - 1; ++m) {
-      const int e = tid + blockDim.x * m;
-      if (m < nbk && e < nbk * BS * BS) {
-        const int kk = e / (BS * BS), r = (e / BS) % BS, c = e % BS, ib = kk + dd;
-        X(BS * ib + r, BS * kk + c) = tv[m];
-      }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int m = 0; m < NBK - 1; ++m) {
-      tv[m] = 0.f;
-      const int e = tid + blockDim.x * m;
-      if (m < nbk && e < nbk * BS * BS) {
-        const int kk = e / (BS * BS), r = (e / BS) % BS, c = e % BS, ib = kk + dd;
-        float v = 0.f;
-#pragma unroll
-        for (int u = 0; u < BS; ++u) v = fmaf(X(BS * ib + r, BS * ib + u), X(BS * ib + u, BS * kk + c), v);
-        tv[m] = -v;
-      }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int m = 0; m < NBK - 1; ++m) {
-      const int e = tid + blockDim.x * m;
-      if (m < nbk && e < nbk * BS * BS) {
-        const int kk = e / (BS * BS), r = (e / BS) % BS, c = e % BS, ib = kk + dd;
-        X(BS * ib + r, BS * kk + c) = tv[m];
-      }
-    }
-    __syncthreads();
+  __syncthreads();
+  if (*bad) {
+    if (tid == 0) set_error(st, PWP_ENOTSPD, kSiteCholDiag);
+    return false;
   }
+  // L21 = P21 X11^T (X11 is zero above its diagonal): lane -> column j, warp -> rows
+  const int j = lane;
+  float v[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const int i = H2 + warp + 8 * m;
+    float acc = 0.f;
+#pragma unroll 8
+    for (int t = 0; t < H2; ++t) acc = fmaf(P(i, t), X(j, t), acc);
+    v[m] = acc;
+  }
+  __syncthreads();   // P21 is read above and overwritten below
+#pragma unroll
+  for (int m = 0; m < 4; ++m) P(H2 + warp + 8 * m, j) = v[m];
+  __syncthreads();
+  // S = P22 - L21 L21^T on and below the diagonal, in place
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const int i = H2 + warp + 8 * m, jj = H2 + lane;
+    if (jj <= i) {
+      float acc = P(i, jj);
+#pragma unroll 8
+      for (int t = 0; t < H2; ++t) acc = fmaf(-P(i, t), P(jj, t), acc);
+      P(i, jj) = acc;
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const bool ok = warp_chol_inv32(P, X, H2, lane);
+    if (!ok && lane == 0) *bad = 1;
+  } else {
+    // T = L21 X11 (X11 is zero above its diagonal) into X21's place
+    for (int e = tid - 32; e < H2 * H2; e += blockDim.x - 32) {
+      const int i = H2 + (e >> 5), jt = e & 31;
+      float acc = 0.f;
+#pragma unroll 8
+      for (int t = 0; t < H2; ++t) acc = fmaf(P(i, t), X(t, jt), acc);
+      X(i, jt) = acc;
+    }
+  }
+  __syncthreads();
+  if (*bad) {
+    if (tid == 0) set_error(st, PWP_ENOTSPD, kSiteCholDiag);
+    return false;
+  }
+  // X21 = -X22 T (X22 is zero above its diagonal)
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const int i = H2 + warp + 8 * m;
+    float acc = 0.f;
+#pragma unroll 8
+    for (int t = H2; t < NB; ++t) acc = fmaf(X(i, t), X(t, j), acc);
+    v[m] = -acc;
+  }
+  __syncthreads();   // T is read above and overwritten below
+#pragma unroll
+  for (int m = 0; m < 4; ++m) X(H2 + warp + 8 * m, j) = v[m];
+  __syncthreads();
   return true;
 }
 
