@@ -13,7 +13,7 @@ Bars: every invariant bit-exact; masks agree at >= 99.99% with the independent o
 and reconstruction loss within 1e-2 of it; ties judged on the GPU's own trajectory -- the
 oracle replays the GPU's masks in fp64 and, block by block, applies the selection rule to
 the replayed state: the GPU's block masks may differ from that choice only where the
-score sits within 1e-6 (relative) of the boundary, and W-hat is within 1e-3 relative
+score sits within TIE_TOL = 1e-5 (relative; derived below) of the boundary, and W-hat is within 1e-3 relative
 Frobenius of the replay (once a row has taken a different weight at a near-tie, its later
 weights legitimately differ from the independent run's, so W-hat is not compared with
 that run); the factor U within 1e-4 of the fp64 U; H within 1e-5 of fp64 (2e-5 over
@@ -31,7 +31,14 @@ from tests import _parity as P
 
 pytestmark = [pytest.mark.gpu, pytest.mark.fullsize]
 
-TIE_TOL = 1e-6
+# Near-tie bar at full size, from the arithmetic of the update: a 3xTF32 product is exact to
+# about 2^-20 relative (the TF32 truncation of the remainders and the dropped remainder x
+# remainder term), so each block's update of a weight carries ~1e-6 of the update's size,
+# and the 32 (b = 4096) to 86 (b = 11008) updates an entry receives before its column is
+# decided add up like a random walk to sqrt(T) x 1e-6 = 6e-6 .. 9e-6 of the weight.  A
+# decision whose score sits within 1e-5 (relative) of the boundary can flip on that
+# rounding alone.  (The small parity cases, with at most a few blocks, keep 1e-6.)
+TIE_TOL = 1e-5
 U_REL_TOL = 1e-4
 H_TOL = 1e-5
 H_TOL_LONG = 2e-5
