@@ -57,65 +57,35 @@ __global__ void __launch_bounds__(1024) damp_kernel(float* __restrict__ H, int b
   for (int q = threadIdx.x; q < b; q += blockDim.x) H[(long long)q * b + q] += lam;
 }
 
-// Pivot K of the one-warp factorisation below (K a template parameter, so that every
-// register index is a compile-time constant).  Lane k: L[k][k] and row k of X made final;
-// lanes below: L[lane][K], then the elimination of column K of L and row K of X.
-template <int K>
-__device__ __forceinline__ void chol_inv_step(float (&p)[32], float (&x)[32], int lane, bool& ok) {
-  constexpr unsigned kAll = 0xffffffffu;
-  const float piv = __shfl_sync(kAll, p[K], K);
-  ok = ok && (piv > 0.f) && isfinite(piv);
-  const float il = rsqrtf(piv);
-  p[K] = lane == K ? piv * il : (lane > K ? p[K] * il : p[K]);
-  const float xs = lane == K ? il : 1.f;
-#pragma unroll
-  for (int t = 0; t <= K; ++t) x[t] *= xs;
-#pragma unroll
-  for (int j = K + 1; j < 32; ++j) {
-    const float ljk = __shfl_sync(kAll, p[K], j);          // L[j][K]
-    if (lane >= j) p[j] = fmaf(-p[K], ljk, p[j]);
-  }
-#pragma unroll
-  for (int t = 0; t <= K; ++t) {
-    const float xkt = __shfl_sync(kAll, x[t], K);          // X[K][t], final
-    if (lane > K) x[t] = fmaf(-p[K], xkt, x[t]);
-  }
-}
-
-template <int K>
-struct CholInvSteps {
-  static __device__ __forceinline__ void run(float (&p)[32], float (&x)[32], int lane, bool& ok) {
-    chol_inv_step<K>(p, x, lane, ok);
-    CholInvSteps<K + 1>::run(p, x, lane, ok);
-  }
-};
-template <>
-struct CholInvSteps<32> {
-  static __device__ __forceinline__ void run(float (&)[32], float (&)[32], int, bool&) {}
-};
-
-// One warp factors and inverts a 32 x 32 diagonal block of P (below): P[b0.., b0..] =
-// L L^T with L lower, X = L^-1.  Lane i holds row i of both in registers; pivots and rows
-// travel by shuffles.  At pivot k, row k of X (which already carries every earlier
-// pivot's elimination) becomes final once divided by L[k][k], and is eliminated from the
-// rows below it together with column k of L.  Writes L and X (lower) back to P and X.
-// Returns false on a non-positive pivot (the same on every lane).
-template <typename FP, typename FX>
-__device__ __forceinline__ bool warp_chol_inv32(FP P, FX X, int b0, int lane) {
-  float p[32], x[32];
-#pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    p[j] = j <= lane ? P(b0 + lane, b0 + j) : 0.f;
-    x[j] = j == lane ? 1.f : 0.f;
-  }
+// Cholesky and inverse of an 8 x 8 SPD block in registers (lower triangles; compile-time
+// indices throughout): L L^T = D, X = L^-1.  False on a non-positive pivot.
+__device__ __forceinline__ bool chol_inv8(float (&L)[8][8], float (&X)[8][8]) {
   bool ok = true;
-  CholInvSteps<0>::run(p, x, lane, ok);
+  float il[8];
 #pragma unroll
-  for (int j = 0; j < 32; ++j)
-    if (j <= lane) {
-      P(b0 + lane, b0 + j) = p[j];
-      X(b0 + lane, b0 + j) = x[j];
+  for (int c = 0; c < 8; ++c) {
+    const float piv = L[c][c];
+    ok = ok && (piv > 0.f) && isfinite(piv);
+    il[c] = rsqrtf(piv);
+    L[c][c] = piv * il[c];
+#pragma unroll
+    for (int r = c + 1; r < 8; ++r) L[r][c] *= il[c];
+#pragma unroll
+    for (int r = c + 1; r < 8; ++r)
+#pragma unroll
+      for (int c2 = c + 1; c2 <= r; ++c2) L[r][c2] = fmaf(-L[r][c], L[c2][c], L[r][c2]);
+  }
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    X[r][r] = il[r];
+#pragma unroll
+    for (int c = 0; c < r; ++c) {
+      float acc = 0.f;
+#pragma unroll
+      for (int t = c; t < r; ++t) acc = fmaf(L[r][t], X[t][c], acc);
+      X[r][c] = -il[r] * acc;
     }
+  }
   return ok;
 }
 
@@ -124,18 +94,20 @@ __device__ __forceinline__ bool warp_chol_inv32(FP P, FX X, int b0, int lane) {
 // Working on the reversed matrix P = J A J (J the reversal; P[r][s] = A[63-r][63-s], so
 // P's lower triangle is A's upper one and the work happens in place), this is the
 // ordinary Cholesky P = L L^T from the top-left, with V = J L J and V^-1 = J X J for
-// X = L^-1.  In 32 x 32 blocks:
-//   L11 L11^T = P11, X11 = L11^-1            (warp 0);
-//   L21 = P21 X11^T, then S = P22 - L21 L21^T  (all threads);
-//   L22 L22^T = S, X22 = L22^-1               (warp 0), while the other warps form
-//                                              T = L21 X11 in X21's place;
-//   X21 = -X22 T                              (all threads).
+// X = L^-1.  Right-looking in 8-column steps, every step two barriers apart:
+//   the step's 8 x 8 diagonal block is factored and inverted in registers (Ld, Xd) by
+//   each of the first 64 threads alike; thread r < 56 - k0 forms row k0+8+r of the panel,
+//   L[i, blk] = P[i, blk] Xd^T; thread t < k0 brings column t of the block's rows of X up
+//   to date, X[blk, t] := Xd X[blk, t] (those rows already carry the earlier steps'
+//   eliminations; their own columns become Xd);
+//   then all threads update the trailing part, P[i][j] -= L[i, blk] L[j, blk], and
+//   eliminate the block's rows from X's rows below it, X[i][t] -= L[i, blk] X[blk, t].
 // Rows and columns beyond nb (A indices >= nb) are an identity pad.  On return A's upper
 // triangle holds V and Wi holds V^-1 (upper, zero below).  Returns false on a
 // non-positive pivot (recorded in st).
 __device__ bool factor_diag_block(float (*A)[NB + 1], float (*Wi)[NB + 1], int nb, int* bad, pwp_stats* st) {
-  constexpr int H2 = NB / 2;   // 32
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  constexpr int BS = 8, NBK = NB / BS;
+  const int tid = threadIdx.x;
   auto P = [&](int r, int c) -> float& { return A[NB - 1 - r][NB - 1 - c]; };
   auto X = [&](int r, int c) -> float& { return Wi[NB - 1 - r][NB - 1 - c]; };
   // identity pad beyond nb (A indices >= nb) and X = 0
@@ -146,73 +118,83 @@ __device__ bool factor_diag_block(float (*A)[NB + 1], float (*Wi)[NB + 1], int n
   }
   if (tid == 0) *bad = 0;
   __syncthreads();
-  if (warp == 0) {
-    const bool ok = warp_chol_inv32(P, X, 0, lane);
-    if (!ok && lane == 0) *bad = 1;
-  }
-  __syncthreads();
-  if (*bad) {
-    if (tid == 0) set_error(st, PWP_ENOTSPD, kSiteCholDiag);
-    return false;
-  }
-  // L21 = P21 X11^T (X11 is zero above its diagonal): lane -> column j, warp -> rows
-  const int j = lane;
-  float v[4];
+#pragma unroll 1
+  for (int kb = 0; kb < NBK; ++kb) {
+    const int k0 = BS * kb, r0 = k0 + BS, rest = NB - r0;
+    if (tid < 64) {
+      float Ld[8][8], Xd[8][8];
 #pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    const int i = H2 + warp + 8 * m;
-    float acc = 0.f;
-#pragma unroll 8
-    for (int t = 0; t < H2; ++t) acc = fmaf(P(i, t), X(j, t), acc);
-    v[m] = acc;
-  }
-  __syncthreads();   // P21 is read above and overwritten below
+      for (int r = 0; r < 8; ++r)
 #pragma unroll
-  for (int m = 0; m < 4; ++m) P(H2 + warp + 8 * m, j) = v[m];
-  __syncthreads();
-  // S = P22 - L21 L21^T on and below the diagonal, in place
+        for (int c = 0; c < 8; ++c) {
+          Ld[r][c] = c <= r ? P(k0 + r, k0 + c) : 0.f;
+          Xd[r][c] = 0.f;
+        }
+      const bool ok = chol_inv8(Ld, Xd);
+      if (!ok && tid == 0) *bad = 1;
+      if (tid < rest) {                      // panel row k0 + 8 + tid
+        const int i = r0 + tid;
+        float pr[8];
 #pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    const int i = H2 + warp + 8 * m, jj = H2 + lane;
-    if (jj <= i) {
-      float acc = P(i, jj);
-#pragma unroll 8
-      for (int t = 0; t < H2; ++t) acc = fmaf(-P(i, t), P(jj, t), acc);
-      P(i, jj) = acc;
+        for (int c = 0; c < 8; ++c) pr[c] = P(i, k0 + c);
+#pragma unroll
+        for (int a = 0; a < 8; ++a) {
+          float acc = 0.f;
+#pragma unroll
+          for (int c = 0; c <= a; ++c) acc = fmaf(pr[c], Xd[a][c], acc);
+          P(i, k0 + a) = acc;
+        }
+      }
+      if (tid < k0) {                        // column tid of the block's rows of X
+        float xo[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) xo[c] = X(k0 + c, tid);
+#pragma unroll
+        for (int a = 0; a < 8; ++a) {
+          float acc = 0.f;
+#pragma unroll
+          for (int c = 0; c <= a; ++c) acc = fmaf(Xd[a][c], xo[c], acc);
+          X(k0 + a, tid) = acc;
+        }
+      }
+      if (tid == 63) {                       // the block itself
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+#pragma unroll
+          for (int c = 0; c <= r; ++c) {
+            P(k0 + r, k0 + c) = Ld[r][c];
+            X(k0 + r, k0 + c) = Xd[r][c];
+          }
+      }
     }
-  }
-  __syncthreads();
-  if (warp == 0) {
-    const bool ok = warp_chol_inv32(P, X, H2, lane);
-    if (!ok && lane == 0) *bad = 1;
-  } else {
-    // T = L21 X11 (X11 is zero above its diagonal) into X21's place
-    for (int e = tid - 32; e < H2 * H2; e += blockDim.x - 32) {
-      const int i = H2 + (e >> 5), jt = e & 31;
-      float acc = 0.f;
-#pragma unroll 8
-      for (int t = 0; t < H2; ++t) acc = fmaf(P(i, t), X(t, jt), acc);
-      X(i, jt) = acc;
+    __syncthreads();
+    if (*bad) {
+      if (tid == 0) set_error(st, PWP_ENOTSPD, kSiteCholDiag);
+      return false;
     }
-  }
-  __syncthreads();
-  if (*bad) {
-    if (tid == 0) set_error(st, PWP_ENOTSPD, kSiteCholDiag);
-    return false;
-  }
-  // X21 = -X22 T (X22 is zero above its diagonal)
+    // trailing update of P (lower triangle of the rest x rest part) and elimination of
+    // the block's rows from the rows of X below it (columns < k0 + 8)
+    const int nP = rest * (rest + 1) / 2, nX = rest * r0;
+    for (int e = tid; e < nP + nX; e += blockDim.x) {
+      if (e < nP) {
+        int ii = (int)((sqrtf(8.f * (float)e + 1.f) - 1.f) * 0.5f);
+        if ((ii + 1) * (ii + 2) / 2 <= e) ++ii;
+        if (ii * (ii + 1) / 2 > e) --ii;
+        const int i = r0 + ii, j = r0 + (e - ii * (ii + 1) / 2);
+        float acc = P(i, j);
 #pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    const int i = H2 + warp + 8 * m;
-    float acc = 0.f;
-#pragma unroll 8
-    for (int t = H2; t < NB; ++t) acc = fmaf(X(i, t), X(t, j), acc);
-    v[m] = -acc;
-  }
-  __syncthreads();   // T is read above and overwritten below
+        for (int c = 0; c < 8; ++c) acc = fmaf(-P(i, k0 + c), P(j, k0 + c), acc);
+        P(i, j) = acc;
+      } else {
+        const int e2 = e - nP, i = r0 + e2 / r0, t = e2 % r0;
+        float acc = X(i, t);
 #pragma unroll
-  for (int m = 0; m < 4; ++m) X(H2 + warp + 8 * m, j) = v[m];
-  __syncthreads();
+        for (int c = 0; c < 8; ++c) acc = fmaf(-P(i, k0 + c), X(k0 + c, t), acc);
+        X(i, t) = acc;
+      }
+    }
+    __syncthreads();
+  }
   return true;
 }
 

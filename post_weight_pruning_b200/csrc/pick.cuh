@@ -261,18 +261,27 @@ __device__ inline void tie_cutoff(Ctl* ctl, unsigned int T, long long m, Level2 
                                   int j, int j1, const float* __restrict__ sc, Shared& sh, int bar, int tid) {
   const int lane = tid & 31, warp = tid >> 5;
   const int nJ = j1 - j;
-  if (tid == 0) {
-    long long cum = 0;
-    int qstar = -1;
-    for (int qq = 0; qq < nJ; ++qq) {
-      const long long cq = l2.tie_count[qq];
-      if (cum + cq >= m) { qstar = qq; break; }
-      cum += cq;
+  {
+    // the column holding the m-th tied entry, by a prefix sum of the per-column counts
+    // (one column per thread; the first column whose running count reaches m)
+    const long long cq = tid < nJ ? (long long)l2.tie_count[tid] : 0;
+    long long x = cq;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long yv = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += yv;
     }
-    sh.sel = qstar;
-    sh.need = m - cum;   // 1-based rank of the last taken tie inside column qstar
+    if (lane == 31) sh.warp[warp] = x;
+    if (tid == 0) sh.sel = -1;   // no such column: fewer than m ties inside the block
+    sync(bar);
+    long long incl = x;
+    for (int w = 0; w < warp; ++w) incl += sh.warp[w];
+    if (cq > 0 && incl >= m && incl - cq < m) {
+      sh.sel = tid;
+      sh.need = m - (incl - cq);   // 1-based rank of the last taken tie inside that column
+    }
+    sync(bar);
   }
-  sync(bar);
   const int qstar = sh.sel;
   const long long need = sh.need;
   sync(bar);

@@ -595,9 +595,9 @@ static void prune_solve(PruneRun& R, int t, long long* nl) {
   prof_begin(kKSolve, R.s);
   if (R.thanos)
     *nl += launch_thanos_solve(R.nm, R.Wout, R.c, R.b, j, R.B, R.pb.K_in + (size_t)t * R.B * R.B, R.pb.xnorm,
-                               R.pb.ctl, R.mask, R.pb.Zs, R.cfg->nm_n, R.cfg->nm_m, R.pb.gscratch, R.st, R.s);
+                               R.pb.ctl, R.pb.l2, R.mask, R.pb.Zs, R.cfg->nm_n, R.cfg->nm_m, R.pb.gscratch, R.st, R.s);
   else
-    *nl += launch_sparsegpt_solve(R.nm, R.Wout, R.c, R.b, j, R.B, R.H, R.pb.udiag, R.pb.ctl, R.mask, R.pb.Zs,
+    *nl += launch_sparsegpt_solve(R.nm, R.Wout, R.c, R.b, j, R.B, R.H, R.pb.udiag, R.pb.ctl, R.pb.l2, R.mask, R.pb.Zs,
                                   R.cfg->nm_n, R.cfg->nm_m, R.st, R.s);
   prof_end(kKSolve, R.s);
 }
@@ -683,11 +683,8 @@ cudaError_t sweep_step(const pwp_config* cfg, const void* W, int wtype, int c, i
       ++nl;
       break;
     }
-    case PWP_SWEEP_SOLVE:
-      launch_sweep_select(6, R.score, R.pb.ctl, R.pb.hist1, R.pb.l2, PickArgs{}, Wout, c, b, j, j1, q1, R.sc,
-                          nullptr, world, rank, st, s);
+    case PWP_SWEEP_SOLVE:   // (also clears the block's level-2 histograms)
       prune_solve(R, t, &nl);
-      ++nl;
       break;
     case PWP_SWEEP_FINISH:
       e = prune_pass(R, R.nblk, PickArgs{}, &nl);

@@ -223,6 +223,21 @@ struct Level2 {
   unsigned int* tie_count;   // kMaxBlock per-column counts of entries tied at T
 };
 
+// The level-2 histograms a block's selection counted into (the control block's dirty
+// flags, set when the level-1 bin is taken), cleared for the next block by the grid of the
+// kernel that follows the selection (the row solve): thread gtid of stride.
+__device__ __forceinline__ void clear_used_level2(const Ctl& ctl, Level2 l2, int gtid, int stride) {
+  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+  if (ctl.dirty_pred) {
+    for (int i = gtid; i < kHist2Bins / 4; i += stride) reinterpret_cast<uint4*>(l2.pred)[i] = z;
+    for (int i = gtid; i < kHist2SumBins / 4; i += stride) reinterpret_cast<uint4*>(l2.pred_sum)[i] = z;
+  }
+  if (ctl.dirty_reread) {
+    for (int i = gtid; i < kHist2Bins / 4; i += stride) reinterpret_cast<uint4*>(l2.reread)[i] = z;
+    for (int i = gtid; i < kHist2SumBins / 4; i += stride) reinterpret_cast<uint4*>(l2.reread_sum)[i] = z;
+  }
+}
+
 // Selection arguments of the scoring pass that precedes a block's selection: the region's
 // entry count and the budget (the residual global count, or the block quota); the pass's
 // last CTA takes the level-1 bin and, when predicted, the exact threshold (pick.cuh).
@@ -274,12 +289,13 @@ cudaError_t launch_pack24(const float* What, const uint8_t* mask, int c, int b, 
                           pwp_stats* st, cudaStream_t s);
 
 // per-row work of one block (solve.cu); returns the number of kernels launched
+// (both also clear the level-2 histograms the block's selection used)
 int launch_thanos_solve(bool nm, const float* W, int c, int b, int j, int B, const float* Kt,
-                        const float* xnorm, Ctl* ctl, uint8_t* mask, float* Zs, int nm_n, int nm_m,
+                        const float* xnorm, Ctl* ctl, Level2 l2, uint8_t* mask, float* Zs, int nm_n, int nm_m,
                         float* gscratch, pwp_stats* st, cudaStream_t s);
 size_t solve_scratch_bytes(int c, int B, bool nm, int nm_n, int nm_m);
 int launch_sparsegpt_solve(bool nm, const float* W, int c, int b, int j, int B, const float* H,
-                           const float* udiag, Ctl* ctl, uint8_t* mask, float* Zs, int nm_n,
+                           const float* udiag, Ctl* ctl, Level2 l2, uint8_t* mask, float* Zs, int nm_n,
                            int nm_m, pwp_stats* st, cudaStream_t s);
 
 }  // namespace pwp

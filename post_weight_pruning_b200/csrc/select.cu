@@ -1,23 +1,18 @@
 // The part of a block's exact selection that follows the scoring pass (pick.cuh has the
 // selection itself and its page citations).  The scoring pass's last CTA has already taken
 // the level-1 bin of the r-th smallest key and, when the pass predicted that bin, the
-// exact threshold T.  One grid-wide kernel does the rest:
+// exact threshold T.  One grid-wide kernel does the rest, when there is any:
 //   - when the bin was not predicted (rare): re-read the region for the level-2 histogram
 //     of the chosen bin; the last CTA to finish takes T, and, if only some entries tied at
 //     T are taken, counts the block's ties per column and finds the cut-off itself;
 //   - otherwise, when only some tied entries are taken: count the block's ties per column
 //     over the grid; the last CTA finds the (column, row) cut-off;
-//   - and clears the level-2 histograms the block used, ready for the next block.
+//   - otherwise it has nothing to do.
+// The level-2 histograms the block used are cleared by the row solve that follows.
 #include "pick.cuh"
 
 namespace pwp {
 namespace {
-
-__device__ __forceinline__ void zero_words(unsigned int* p, int n, int first, int stride) {
-  uint4* p4 = reinterpret_cast<uint4*>(p);
-  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-  for (int i = first; i < n / 4; i += stride) p4[i] = z;
-}
 
 // ctl without __restrict__: the last CTA's threads share decisions taken by one of them
 // (through shared memory; see pick.cuh).
@@ -33,8 +28,8 @@ __global__ void __launch_bounds__(pick::kThreads) select_finish_kernel(Ctl* ctl,
   const int gtid = blockIdx.x * blockDim.x + tid, stride = gridDim.x * blockDim.x;
   // the outcome of the scoring pass's last CTA (an earlier kernel)
   const int mode = ctl->mode, ready = ctl->l2_ready, tie_scan = ctl->tie_scan;
-  const bool dirty_pred = ctl->dirty_pred != 0;
-  if (mode != 0 && !ready) {
+  if (mode == 0 || (ready && !tie_scan)) return;
+  if (!ready) {
     // the level-2 histogram of bin b1 over the region: rows over CTAs, columns over threads
     const unsigned int b1 = ctl->b1;
     const long long r1 = ctl->r1;
@@ -53,28 +48,15 @@ __global__ void __launch_bounds__(pick::kThreads) select_finish_kernel(Ctl* ctl,
       pick::sync(1);
       pick::tie_cutoff<SCORE>(ctl, T, m, l2, W, c, b, j, j1, sc, sh, 1, tid);
     }
-    // this CTA alone clears what the block counted into
-    if (dirty_pred) {
-      zero_words(l2.pred, kHist2Bins, tid, blockDim.x);
-      zero_words(l2.pred_sum, kHist2SumBins, tid, blockDim.x);
-    }
-    zero_words(l2.reread, kHist2Bins, tid, blockDim.x);
-    zero_words(l2.reread_sum, kHist2SumBins, tid, blockDim.x);
     return;
   }
-  // the predicted level-2 histogram was consumed by the scoring pass's last CTA
-  if (dirty_pred) {
-    zero_words(l2.pred, kHist2Bins, gtid, stride);
-    zero_words(l2.pred_sum, kHist2SumBins, gtid, stride);
-  }
-  if (mode != 0 && tie_scan) {
-    const unsigned int T = ctl->T;
-    const long long m = ctl->m;
-    const int gwarp = gtid >> 5, nwarps = stride >> 5;
-    pick::count_ties<SCORE>(T, l2, W, b, j, j1, sc, gwarp, c, nwarps);
-    if (!pick::last_cta(&ctl->ticket, sh)) return;
-    pick::tie_cutoff<SCORE>(ctl, T, m, l2, W, c, b, j, j1, sc, sh, 1, tid);
-  }
+  // predicted, with a partial tie group at T
+  const unsigned int T = ctl->T;
+  const long long m = ctl->m;
+  const int gwarp = gtid >> 5, nwarps = stride >> 5;
+  pick::count_ties<SCORE>(T, l2, W, b, j, j1, sc, gwarp, c, nwarps);
+  if (!pick::last_cta(&ctl->ticket, sh)) return;
+  pick::tie_cutoff<SCORE>(ctl, T, m, l2, W, c, b, j, j1, sc, sh, 1, tid);
 }
 
 // ---------------------------------------------------------------- the stepwise sweep
@@ -216,21 +198,6 @@ __global__ void __launch_bounds__(pick::kThreads) cut_ties_kernel(Ctl* ctl, Leve
   if (tid == 0) ctl->pstar = s_pstar;
 }
 
-__global__ void __launch_bounds__(256) clear_level2_kernel(const Ctl* __restrict__ ctl, Level2 l2,
-                                                           const pwp_stats* st) {
-  pdl_enter();
-  if (failed(st)) return;
-  const int gtid = blockIdx.x * blockDim.x + threadIdx.x, stride = gridDim.x * blockDim.x;
-  if (ctl->dirty_pred) {
-    zero_words(l2.pred, kHist2Bins, gtid, stride);
-    zero_words(l2.pred_sum, kHist2SumBins, gtid, stride);
-  }
-  if (ctl->dirty_reread) {
-    zero_words(l2.reread, kHist2Bins, gtid, stride);
-    zero_words(l2.reread_sum, kHist2SumBins, gtid, stride);
-  }
-}
-
 }  // namespace
 
 void launch_select_finish(int score, Ctl* ctl, Level2 l2, const float* W, int c, int b, int j, int j1, int q1,
@@ -285,9 +252,6 @@ void launch_sweep_select(int step, int score, Ctl* ctl, unsigned int* hist1, Lev
       else
         launch_pdl(cut_ties_kernel<kObs>, dim3(1), dim3(pick::kThreads), 0, s, ctl, l2, W, c, b, j, j1, sc,
                    ties_all, world, rank, st);
-      break;
-    case 6:   // clear the level-2 histograms the block used
-      launch_pdl(clear_level2_kernel, dim3(kNumSM), dim3(256), 0, s, (const Ctl*)ctl, l2, (const pwp_stats*)st);
       break;
     default:
       break;

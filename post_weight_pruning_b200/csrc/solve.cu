@@ -288,7 +288,7 @@ __global__ void __launch_bounds__(kSolveWarps * 32, 2) thanos_solve_kernel(const
                                                                           int b, int j, int B,
                                                                           const float* __restrict__ Kt,
                                                                           const float* __restrict__ xnorm,
-                                                                          Ctl* __restrict__ ctlp,
+                                                                          Ctl* __restrict__ ctlp, Level2 l2,
                                                                           uint8_t* __restrict__ mask,
                                                                           float* __restrict__ Zs, int nm_n, int nm_m,
                                                                           float* __restrict__ gscratch,
@@ -305,6 +305,7 @@ __global__ void __launch_bounds__(kSolveWarps * 32, 2) thanos_solve_kernel(const
   float* D = reinterpret_cast<float*>(Qidx + kCap);
   float* G = gscratch ? gscratch + (size_t)slot * kGlobalPerWarp : nullptr;
   const Ctl ctl = *ctlp;
+  clear_used_level2(ctl, l2, blockIdx.x * blockDim.x + threadIdx.x, gridDim.x * blockDim.x);
   const int nJ = min(B, b - j);
   constexpr int MAXI = kMaxBlock / 32;
   for (int k = slot; k < c; k += gridDim.x * nwarps) {
@@ -377,7 +378,7 @@ template <bool NM>
 __global__ void __launch_bounds__(256) sparsegpt_solve_kernel(const float* __restrict__ W, int c, int b,
                                                               int j, int B, const float* __restrict__ H,
                                                               const float* __restrict__ udiag,
-                                                              Ctl* __restrict__ ctlp,
+                                                              Ctl* __restrict__ ctlp, Level2 l2,
                                                               uint8_t* __restrict__ mask,
                                                               float* __restrict__ Zs, int nm_n, int nm_m,
                                                               pwp_stats* st) {
@@ -385,8 +386,9 @@ __global__ void __launch_bounds__(256) sparsegpt_solve_kernel(const float* __res
   if (warp_failed(st)) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int k = blockIdx.x * (blockDim.x >> 5) + warp;
-  if (k >= c) return;
   const Ctl ctl = *ctlp;
+  clear_used_level2(ctl, l2, blockIdx.x * blockDim.x + threadIdx.x, gridDim.x * blockDim.x);
+  if (k >= c) return;
   const int nJ = min(B, b - j);
   constexpr int MAXI = kMaxBlock / 32;
   float w[MAXI], e[MAXI];
@@ -440,14 +442,14 @@ __global__ void __launch_bounds__(256) sparsegpt_solve_kernel(const float* __res
 
 template <bool NM>
 void launch_thanos_variant(const float* W, int c, int b, int j, int B, const float* Kt, const float* xnorm,
-                           Ctl* ctl, uint8_t* mask, float* Zs, int nm_n, int nm_m, float* gscratch,
+                           Ctl* ctl, Level2 l2, uint8_t* mask, float* Zs, int nm_n, int nm_m, float* gscratch,
                            pwp_stats* st, cudaStream_t s) {
   const int smem = kSolveWarps * kPerWarp * 4;
   static std::atomic<unsigned long long> attr_done{0};
   if (first_on_device(attr_done))
     cudaFuncSetAttribute(thanos_solve_kernel<NM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   const int grid = min((c + kSolveWarps - 1) / kSolveWarps, kSolveCtas);
-  launch_pdl(thanos_solve_kernel<NM>, dim3(grid), dim3(kSolveWarps * 32), smem, s, W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m,
+  launch_pdl(thanos_solve_kernel<NM>, dim3(grid), dim3(kSolveWarps * 32), smem, s, W, c, b, j, B, Kt, xnorm, ctl, l2, mask, Zs, nm_n, nm_m,
                                                                gscratch, st);
 }
 
@@ -467,23 +469,23 @@ size_t solve_scratch_bytes(int c, int B, bool nm, int nm_n, int nm_m) {
 // shared memory; rows past them (rows with larger sets) go to the warp's slot of global
 // scratch.
 int launch_thanos_solve(bool nm, const float* W, int c, int b, int j, int B, const float* Kt,
-                        const float* xnorm, Ctl* ctl, uint8_t* mask, float* Zs, int nm_n, int nm_m,
+                        const float* xnorm, Ctl* ctl, Level2 l2, uint8_t* mask, float* Zs, int nm_n, int nm_m,
                         float* gscratch, pwp_stats* st, cudaStream_t s) {
   if (nm)
-    launch_thanos_variant<true>(W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, gscratch, st, s);
+    launch_thanos_variant<true>(W, c, b, j, B, Kt, xnorm, ctl, l2, mask, Zs, nm_n, nm_m, gscratch, st, s);
   else
-    launch_thanos_variant<false>(W, c, b, j, B, Kt, xnorm, ctl, mask, Zs, nm_n, nm_m, gscratch, st, s);
+    launch_thanos_variant<false>(W, c, b, j, B, Kt, xnorm, ctl, l2, mask, Zs, nm_n, nm_m, gscratch, st, s);
   return 1;
 }
 
 int launch_sparsegpt_solve(bool nm, const float* W, int c, int b, int j, int B, const float* H,
-                           const float* udiag, Ctl* ctl, uint8_t* mask, float* Zs, int nm_n, int nm_m,
+                           const float* udiag, Ctl* ctl, Level2 l2, uint8_t* mask, float* Zs, int nm_n, int nm_m,
                            pwp_stats* st, cudaStream_t s) {
   const int grid = (c + 7) / 8;
   if (nm)
-    launch_pdl(sparsegpt_solve_kernel<true>, dim3(grid), dim3(256), 0, s, W, c, b, j, B, H, udiag, ctl, mask, Zs, nm_n, nm_m, st);
+    launch_pdl(sparsegpt_solve_kernel<true>, dim3(grid), dim3(256), 0, s, W, c, b, j, B, H, udiag, ctl, l2, mask, Zs, nm_n, nm_m, st);
   else
-    launch_pdl(sparsegpt_solve_kernel<false>, dim3(grid), dim3(256), 0, s, W, c, b, j, B, H, udiag, ctl, mask, Zs, nm_n, nm_m, st);
+    launch_pdl(sparsegpt_solve_kernel<false>, dim3(grid), dim3(256), 0, s, W, c, b, j, B, H, udiag, ctl, l2, mask, Zs, nm_n, nm_m, st);
   return 1;
 }
 
