@@ -635,7 +635,7 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
       prof_begin(kKSelect, s);
       launch_select_finish(R.score, R.pb.ctl, R.pb.l2, Wout, c, b, j, j1, R.thanos ? b : j1, R.sc, st, s);
       prof_end(kKSelect, s);
-      ++nl;
+      nl += 2;
     }
     prune_solve(R, t, &nl);
   }

@@ -248,8 +248,9 @@ struct PickArgs {
   int enabled;
 };
 
-// The rest of the exact selection of a block (select.cu): the re-read when the level-1 bin
-// was not predicted, the cut-off among tied entries, and clearing the level-2 histograms.
+// The rest of the exact selection of a block (select.cu), two launches: the re-read when
+// the level-1 bin was not predicted, then the cut-off among tied entries (each a no-op
+// when not needed).
 void launch_select_finish(int score, Ctl* ctl, Level2 l2, const float* W, int c, int b, int j, int j1, int q1,
                           const float* sc, pwp_stats* st, cudaStream_t s);
 void launch_sweep_select(int step, int score, Ctl* ctl, unsigned int* hist1, Level2 l2, PickArgs pk, const float* W,

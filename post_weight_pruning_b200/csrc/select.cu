@@ -1,13 +1,13 @@
 // The part of a block's exact selection that follows the scoring pass (pick.cuh has the
 // selection itself and its page citations).  The scoring pass's last CTA has already taken
 // the level-1 bin of the r-th smallest key and, when the pass predicted that bin, the
-// exact threshold T.  One grid-wide kernel does the rest, when there is any:
-//   - when the bin was not predicted (rare): re-read the region for the level-2 histogram
-//     of the chosen bin; the last CTA to finish takes T, and, if only some entries tied at
-//     T are taken, counts the block's ties per column and finds the cut-off itself;
-//   - otherwise, when only some tied entries are taken: count the block's ties per column
-//     over the grid; the last CTA finds the (column, row) cut-off;
-//   - otherwise it has nothing to do.
+// exact threshold T.  Two grid-wide kernels do the rest, each returning at once when it
+// has nothing to do:
+//   - select_finish: when the bin was not predicted (rare; always for the first block),
+//     re-read the region for the level-2 histogram of the chosen bin; the last CTA to
+//     finish takes T;
+//   - select_ties: when only some entries tied at T are taken, count the block's ties per
+//     column over the grid; the last CTA finds the (column, row) cut-off.
 // The level-2 histograms the block used are cleared by the row solve that follows.
 #include "pick.cuh"
 
@@ -19,44 +19,41 @@ namespace {
 template <int SCORE>
 __global__ void __launch_bounds__(pick::kThreads) select_finish_kernel(Ctl* ctl, Level2 l2,
                                                                       const float* __restrict__ W, int c, int b,
-                                                                      int j, int j1, int q1,
+                                                                      int j, int q1,
                                                                       const float* __restrict__ sc, pwp_stats* st) {
   pdl_enter();
   __shared__ pick::Shared sh;
   if (cta_failed(st)) return;
-  const int tid = threadIdx.x;
-  const int gtid = blockIdx.x * blockDim.x + tid, stride = gridDim.x * blockDim.x;
   // the outcome of the scoring pass's last CTA (an earlier kernel)
-  const int mode = ctl->mode, ready = ctl->l2_ready, tie_scan = ctl->tie_scan;
-  if (mode == 0 || (ready && !tie_scan)) return;
-  if (!ready) {
-    // the level-2 histogram of bin b1 over the region: rows over CTAs, columns over threads
-    const unsigned int b1 = ctl->b1;
-    const long long r1 = ctl->r1;
-    for (int r = blockIdx.x; r < c; r += gridDim.x) {
-      const float* wr = W + (long long)r * b;
-      for (int q = j + tid; q < q1; q += blockDim.x)
-        count_level2(key_of<SCORE>(wr[q], __ldg(sc + q)), b1, l2.reread, l2.reread_sum);
-    }
-    if (!pick::last_cta(&ctl->ticket, sh)) return;
-    pick::level2(ctl, l2, r1, 0, st, sh, 1, tid);
-    if (sh.mode != 0 && sh.tie_scan) {
-      const unsigned int T = sh.T;
-      const long long m = sh.m;
-      pick::count_ties<SCORE>(T, l2, W, b, j, j1, sc, tid >> 5, c, pick::kWarps);
-      __threadfence_block();
-      pick::sync(1);
-      pick::tie_cutoff<SCORE>(ctl, T, m, l2, W, c, b, j, j1, sc, sh, 1, tid);
-    }
-    return;
+  if (ctl->mode == 0 || ctl->l2_ready) return;
+  const int tid = threadIdx.x;
+  // the level-2 histogram of bin b1 over the region: rows over CTAs, columns over threads
+  const unsigned int b1 = ctl->b1;
+  const long long r1 = ctl->r1;
+  for (int r = blockIdx.x; r < c; r += gridDim.x) {
+    const float* wr = W + (long long)r * b;
+    for (int q = j + tid; q < q1; q += blockDim.x)
+      count_level2(key_of<SCORE>(wr[q], __ldg(sc + q)), b1, l2.reread, l2.reread_sum);
   }
-  // predicted, with a partial tie group at T
+  if (!pick::last_cta(&ctl->ticket, sh)) return;
+  pick::level2(ctl, l2, r1, 0, st, sh, 1, tid);
+}
+
+template <int SCORE>
+__global__ void __launch_bounds__(pick::kThreads) select_ties_kernel(Ctl* ctl, Level2 l2,
+                                                                    const float* __restrict__ W, int c, int b,
+                                                                    int j, int j1, const float* __restrict__ sc,
+                                                                    pwp_stats* st) {
+  pdl_enter();
+  __shared__ pick::Shared sh;
+  if (cta_failed(st)) return;
+  if (ctl->mode == 0 || !ctl->tie_scan) return;
   const unsigned int T = ctl->T;
   const long long m = ctl->m;
-  const int gwarp = gtid >> 5, nwarps = stride >> 5;
-  pick::count_ties<SCORE>(T, l2, W, b, j, j1, sc, gwarp, c, nwarps);
+  const int gtid = blockIdx.x * blockDim.x + threadIdx.x, stride = gridDim.x * blockDim.x;
+  pick::count_ties<SCORE>(T, l2, W, b, j, j1, sc, gtid >> 5, c, stride >> 5);
   if (!pick::last_cta(&ctl->ticket, sh)) return;
-  pick::tie_cutoff<SCORE>(ctl, T, m, l2, W, c, b, j, j1, sc, sh, 1, tid);
+  pick::tie_cutoff<SCORE>(ctl, T, m, l2, W, c, b, j, j1, sc, sh, 1, threadIdx.x);
 }
 
 // ---------------------------------------------------------------- the stepwise sweep
@@ -202,12 +199,14 @@ __global__ void __launch_bounds__(pick::kThreads) cut_ties_kernel(Ctl* ctl, Leve
 
 void launch_select_finish(int score, Ctl* ctl, Level2 l2, const float* W, int c, int b, int j, int j1, int q1,
                           const float* sc, pwp_stats* st, cudaStream_t s) {
-  if (score == kWanda)
-    launch_pdl(select_finish_kernel<kWanda>, dim3(kNumSM), dim3(pick::kThreads), 0, s, ctl, l2, W, c, b, j, j1, q1,
-               sc, st);
-  else
-    launch_pdl(select_finish_kernel<kObs>, dim3(kNumSM), dim3(pick::kThreads), 0, s, ctl, l2, W, c, b, j, j1, q1,
-               sc, st);
+  if (score == kWanda) {
+    launch_pdl(select_finish_kernel<kWanda>, dim3(kNumSM), dim3(pick::kThreads), 0, s, ctl, l2, W, c, b, j, q1, sc,
+               st);
+    launch_pdl(select_ties_kernel<kWanda>, dim3(kNumSM), dim3(pick::kThreads), 0, s, ctl, l2, W, c, b, j, j1, sc, st);
+  } else {
+    launch_pdl(select_finish_kernel<kObs>, dim3(kNumSM), dim3(pick::kThreads), 0, s, ctl, l2, W, c, b, j, q1, sc, st);
+    launch_pdl(select_ties_kernel<kObs>, dim3(kNumSM), dim3(pick::kThreads), 0, s, ctl, l2, W, c, b, j, j1, sc, st);
+  }
 }
 
 }  // namespace pwp
