@@ -46,6 +46,8 @@ __global__ void init_ctl_kernel(Ctl* ctl, long long zstar, pwp_stats* st, long l
   ctl->dirty_reread = 0;
   ctl->tie_scan = 0;
   ctl->ticket = 0u;
+  ctl->row_next = 0u;
+  ctl->warps_done = 0u;
   st->target = target;
 }
 

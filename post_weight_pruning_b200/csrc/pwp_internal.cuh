@@ -100,6 +100,8 @@ struct Ctl {
   int dirty_reread;       // the re-read level-2 histogram holds counts to clear
   int tie_scan;           // some but not all entries tied at T are taken: locate the cut-off
   unsigned int ticket;    // arrivals of a grid's CTAs; the last one finishes the selection
+  unsigned int row_next;  // the row solve's next row to hand out (reset by its last warp)
+  unsigned int warps_done;  // the row solve's warps that have run out of rows
 };
 
 // Where device-side failures are recorded (pwp_stats::status_site).

@@ -28,21 +28,17 @@ __host__ __device__ constexpr int poff(int i) {
 }
 
 // Per warp: rows 0..kNS-1 of the packed factor, the u/y/z vector, the selected indices
-// (reused for the pivots' reciprocals) and the panel buffer (4 rows of kPbStride: the
-// current 4-column panel, transposed; the general path stages its 8x8 diagonal block
-// there), in shared memory; rows kNS..kCap-1 (only rows with more than kNS selections
-// reach them) in a per-warp slot of global scratch, which stays in L2.  Seven warps per
-// CTA, two CTAs per SM.
+// (reused for the pivots' reciprocals) and the staged 8x8 diagonal block, in shared
+// memory; rows kNS..kCap-1 (only rows with more than kNS selections reach them) in a
+// per-warp slot of global scratch, which stays in L2.
 constexpr int kCap = kMaxBlock;      // largest selected set of a row
 constexpr int kNS = kSolveNS;        // factor rows kept in shared memory
 constexpr int kL = poff(kNS);
 constexpr int kY = kCap + 8;
-constexpr int kPbStride = (kNS + 4 + 3) & ~3;   // panel rows 0..kNS (the u row) and a tile's overhang
-constexpr int kPerWarp = kL + kY + kCap + 4 * kPbStride;   // floats: L, y, Qidx, Pb
+constexpr int kPerWarp = kL + kY + kCap + 64;        // floats: L, y, Qidx, D
 constexpr int kGlobalPerWarp = poff(kCap) - poff(kNS);
-constexpr int kSolveWarps = 7;
-static_assert(kL % 4 == 0 && kY % 4 == 0 && kCap % 4 == 0 && kPbStride % 4 == 0, "16-byte aligned regions");
-static_assert(4 * kPbStride >= 64, "the general path's 8x8 block fits the panel buffer");
+constexpr int kSolveWarps = 8;
+static_assert(kL % 4 == 0 && kY % 4 == 0 && kCap % 4 == 0, "16-byte aligned regions");
 
 // Rows of the packed factor.  SMALL: every row lives in shared memory (s <= kNS), so all
 // pointers stay shared-memory pointers; otherwise rows from kNS on are in global scratch.
@@ -234,150 +230,6 @@ __device__ bool chol_solve(const Rows<SMALL> R, float* __restrict__ y, float* __
   return true;
 }
 
-// Component a (a compile-time index) of a float4.
-template <int A>
-__device__ __forceinline__ float comp(const float4& v) {
-  return A == 0 ? v.x : A == 1 ? v.y : A == 2 ? v.z : v.w;
-}
-
-// One row of a 4 x 4 trailing tile: acc[b] -= sum_c pi[c].a * pj[c].b (a = A).
-template <int A>
-__device__ __forceinline__ void tile_row(float* __restrict__ p, const float4 (&pi)[4], const float4 (&pj)[4]) {
-  float4 acc = *reinterpret_cast<const float4*>(p);
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    const float x = comp<A>(pi[c]);
-    acc.x = fmaf(-x, pj[c].x, acc.x);
-    acc.y = fmaf(-x, pj[c].y, acc.y);
-    acc.z = fmaf(-x, pj[c].z, acc.z);
-    acc.w = fmaf(-x, pj[c].w, acc.w);
-  }
-  *reinterpret_cast<float4*>(p) = acc;
-}
-
-// Cholesky R-hat = L L^T of the s x s gathered matrix for s <= kNS (its lower triangle in
-// the packed rows L on entry, L on return), right-looking in 4-column panels, with u
-// carried as an extra row s (in y) so that the same sweep gives y = L^-1 u; then the back
-// substitution L^T z = y.  On return y[0..s) = z.  Per panel [k0, k0+4):
-//   every lane factors the 4 x 4 diagonal block alike (rows past s are an identity pad;
-//   the pivots' reciprocals go to idg, and lane r writes back row k0+r of the block);
-//   the rows below it, the u row included, go over the lanes and finish their four
-//   panel entries by forward substitution, into the packed rows and, transposed, into
-//   Pb (row c of Pb holds column k0+c of L by row index);
-//   the trailing lower triangle of rows and columns k0+4..s (the u row only as a row)
-//   drops the panel's rank-4 product in 4 x 4 tiles spread over the lanes: each tile
-//   reads its eight panel vectors as float4 and each of its rows once as a float4.
-// A packed row i holds columns up to 4*(i/4)+3, so every float4 of a tile lies inside its
-// row's storage; entries past a row's diagonal in that padding are written but never read.
-// Returns false on a non-positive pivot (uniform: every lane sees the same pivots).
-__device__ bool chol_solve_small(float* __restrict__ L, float* __restrict__ y, float* __restrict__ idg,
-                                 float* __restrict__ Pb, int s, int lane) {
-  auto row = [&](int i) -> float* { return i < s ? L + poff(i) : y; };
-  for (int k0 = 0; k0 < s; k0 += 4) {
-    const int pw = min(4, s - k0);
-    float d[4][4], il[4];
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (r < pw) v = *reinterpret_cast<const float4*>(row(k0 + r) + k0);
-      const float e[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int c = 0; c < 4; ++c) d[r][c] = c <= r ? (r < pw ? e[c] : (c == r ? 1.f : 0.f)) : 0.f;
-    }
-    bool ok = true;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const float piv = d[c][c];
-      ok = ok && (piv > 0.f) && isfinite(piv);
-      il[c] = rsqrtf(piv);
-      d[c][c] = piv * il[c];
-#pragma unroll
-      for (int r = c + 1; r < 4; ++r) d[r][c] *= il[c];
-#pragma unroll
-      for (int r = c + 1; r < 4; ++r)
-#pragma unroll
-        for (int c2 = c + 1; c2 <= r; ++c2) d[r][c2] = fmaf(-d[r][c], d[c2][c], d[r][c2]);
-    }
-    if (!ok) return false;
-#pragma unroll
-    for (int r = 0; r < 4; ++r)
-      if (lane == r && r < pw) {
-        *reinterpret_cast<float4*>(row(k0 + r) + k0) = make_float4(d[r][0], d[r][1], d[r][2], d[r][3]);
-        idg[k0 + r] = il[r];
-      }
-    // panel rows below the block (the u row is row s)
-    for (int i = k0 + pw + lane; i <= s; i += 32) {
-      float* ri = row(i) + k0;
-      const float4 a4 = *reinterpret_cast<const float4*>(ri);
-      float v[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        float t = v[a];
-#pragma unroll
-        for (int c = 0; c < a; ++c) t = fmaf(-v[c], d[a][c], t);
-        v[a] = a < pw ? t * il[a] : 0.f;
-      }
-      *reinterpret_cast<float4*>(ri) = make_float4(v[0], v[1], v[2], v[3]);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) Pb[c * kPbStride + i] = v[c];
-    }
-    __syncwarp();
-    // trailing update of rows/columns [r0, s] in 4 x 4 tiles (tile row ti >= tile column tj)
-    const int r0 = k0 + 4;
-    if (r0 <= s) {
-      const int nt = (s - r0 + 4) >> 2, ntiles = nt * (nt + 1) / 2;
-      for (int e = lane; e < ntiles; e += 32) {
-        int ti = (int)((sqrtf(8.f * (float)e + 1.f) - 1.f) * 0.5f);
-        if ((ti + 1) * (ti + 2) / 2 <= e) ++ti;
-        if (ti * (ti + 1) / 2 > e) --ti;
-        const int i0 = r0 + 4 * ti, j0 = r0 + 4 * (e - ti * (ti + 1) / 2);
-        float4 pi[4], pj[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          pi[c] = *reinterpret_cast<const float4*>(Pb + c * kPbStride + i0);
-          pj[c] = *reinterpret_cast<const float4*>(Pb + c * kPbStride + j0);
-        }
-        tile_row<0>(row(i0) + j0, pi, pj);
-        if (i0 + 1 <= s) tile_row<1>(row(i0 + 1) + j0, pi, pj);
-        if (i0 + 2 <= s) tile_row<2>(row(i0 + 2) + j0, pi, pj);
-        if (i0 + 3 <= s) tile_row<3>(row(i0 + 3) + j0, pi, pj);
-      }
-    }
-    __syncwarp();
-  }
-  // back substitution L^T z = y, four rows at a time from the bottom: the 4x4 corner
-  // is solved redundantly by every lane, then the rows above drop its contribution
-  for (int a0 = (s - 1) & ~3; a0 >= 0; a0 -= 4) {
-    const int pw = min(4, s - a0);
-    const float* rr[4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) rr[c] = L + poff(a0 + (c < pw ? c : pw - 1));
-    float z[4];
-#pragma unroll
-    for (int c = 3; c >= 0; --c) {
-      z[c] = 0.f;
-      if (c < pw) {
-        float v = y[a0 + c];
-#pragma unroll
-        for (int c2 = c + 1; c2 < 4; ++c2)
-          if (c2 < pw) v = fmaf(-rr[c2][a0 + c], z[c2], v);
-        z[c] = v * idg[a0 + c];
-      }
-    }
-    __syncwarp();
-    for (int t = lane; t < a0; t += 32) {
-      float v = y[t];
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        if (c < pw) v = fmaf(-rr[c][t], z[c], v);
-      y[t] = v;
-    }
-    if (lane < pw) y[a0 + lane] = z[lane];
-    __syncwarp();
-  }
-  return true;
-}
-
 // R-hat = K[Q, Q], lower triangle, into the packed rows: row a is K row q_a, loaded whole
 // (lane l holds columns 4l..4l+3), and entry (a, cc) is picked from lane q_cc / 4 by
 // shuffles.
@@ -450,13 +302,30 @@ __global__ void __launch_bounds__(kSolveWarps * 32, 2) thanos_solve_kernel(const
   float* L = smem + warp * kPerWarp;
   float* y = L + kL;
   int* Qidx = reinterpret_cast<int*>(y + kY);
-  float* Pb = reinterpret_cast<float*>(Qidx + kCap);   // also the general path's 8x8 block
+  float* D = reinterpret_cast<float*>(Qidx + kCap);
   float* G = gscratch ? gscratch + (size_t)slot * kGlobalPerWarp : nullptr;
   const Ctl ctl = *ctlp;
   clear_used_level2(ctl, l2, blockIdx.x * blockDim.x + threadIdx.x, gridDim.x * blockDim.x);
   const int nJ = min(B, b - j);
   constexpr int MAXI = kMaxBlock / 32;
-  for (int k = slot; k < c; k += gridDim.x * nwarps) {
+  // the size of row k's selected set (nothing written)
+  auto count_selected = [&](int k) -> int {
+    const float* wrow = W + (long long)k * b + j;
+    int s = 0;
+#pragma unroll
+    for (int i = 0; i < MAXI; ++i) {
+      const int qq = lane + 32 * i;
+      const bool valid = qq < nJ;
+      const float w = valid ? wrow[qq] : 0.f;
+      const unsigned int key = valid ? key_of<kWanda>(w, __ldg(xnorm + j + qq)) : 0xffffffffu;
+      const bool sel = (32 * i < nJ) ? selected<NM>(key, valid, qq, k, c, ctl, nm_n, nm_m) : false;
+      s += __popc(__ballot_sync(0xffffffffu, sel));
+    }
+    return s;
+  };
+  // row k's whole work; with small_only a row whose set exceeds kNS is left (after its mask
+  // bytes, which its slice's warp writes identically) to that warp
+  auto solve_row = [&](int k, bool small_only) {
     const float* wrow = W + (long long)k * b + j;
     uint8_t* mrow = mask + (long long)k * b + j;
     // the selection: mask bytes, the selected indices and u = W[k, Q]; the warp keeps only
@@ -478,9 +347,10 @@ __global__ void __launch_bounds__(kSolveWarps * 32, 2) thanos_solve_kernel(const
         y[pos] = w;
       }
     }
+    if (small_only && s > kNS) return;
     if (s > kNS && !G) {   // excluded by the launcher's choice of scratch
       if (lane == 0) set_error(st, PWP_EINVAL, kSiteSolve);
-      continue;
+      return;
     }
     __syncwarp();
     bool ok = true;
@@ -489,11 +359,11 @@ __global__ void __launch_bounds__(kSolveWarps * 32, 2) thanos_solve_kernel(const
       if (s <= kNS) {
         const Rows<true> R{L, nullptr};
         gather_rhat<true>(R, Kt, Qidx, s, B, nJ, lane);
-        ok = chol_solve_small(L, y, reinterpret_cast<float*>(Qidx), Pb, s, lane);
+        ok = chol_solve<true>(R, y, reinterpret_cast<float*>(Qidx), D, s, lane);
       } else {
         const Rows<false> R{L, G};
         gather_rhat<false>(R, Kt, Qidx, s, B, nJ, lane);
-        ok = chol_solve<false>(R, y, reinterpret_cast<float*>(Qidx), Pb, s, lane);
+        ok = chol_solve<false>(R, y, reinterpret_cast<float*>(Qidx), D, s, lane);
       }
       if (!ok && lane == 0) set_error(st, PWP_ENOTSPD, kSiteSolve);
       if (lane == 0) atomicAdd((unsigned long long*)&ctlp->pruned, (unsigned long long)s);
@@ -516,6 +386,26 @@ __global__ void __launch_bounds__(kSolveWarps * 32, 2) thanos_solve_kernel(const
       }
     }
     __syncwarp();
+  };
+  // First the rows of this warp's slice whose sets exceed the shared rows (the slow
+  // general path starts at once, under the other warps' work); then every other row,
+  // handed out one at a time, so that a warp held up by a large row takes fewer.
+  for (int k = slot; k < c; k += gridDim.x * nwarps)
+    if (count_selected(k) > kNS) solve_row(k, false);
+  for (;;) {
+    unsigned int k = 0;
+    if (lane == 0) k = atomicAdd(&ctlp->row_next, 1u);
+    k = __shfl_sync(0xffffffffu, k, 0);
+    if (k >= (unsigned int)c) break;
+    solve_row((int)k, true);
+  }
+  // the last warp to run out of rows resets the counters for the next launch
+  if (lane == 0) {
+    __threadfence();
+    if (atomicAdd(&ctlp->warps_done, 1u) == gridDim.x * nwarps - 1) {
+      ctlp->row_next = 0u;
+      ctlp->warps_done = 0u;
+    }
   }
 }
 
