@@ -231,23 +231,29 @@ __device__ bool chol_solve(const Rows<SMALL> R, float* __restrict__ y, float* __
 }
 
 // R-hat = K[Q, Q], lower triangle, into the packed rows: row a is K row q_a, loaded whole
-// (lane l holds columns 4l..4l+3), and entry (a, cc) is picked from lane q_cc / 4 by
-// shuffles.
+// (lane l holds columns 4l..4l+3) and staged in the warp's index slots (the indices are
+// held in registers by then), from which entry (a, cc) is read at column q_cc.
 template <bool SMALL>
-__device__ void gather_rhat(const Rows<SMALL> R, const float* __restrict__ Kt, const int* __restrict__ Qidx, int s,
+__device__ void gather_rhat(const Rows<SMALL> R, const float* __restrict__ Kt, int* __restrict__ Qidx, int s,
                             int B, int nJ, int lane) {
   constexpr int CH = (kCap + 31) / 32;
   int qv[CH];
 #pragma unroll
   for (int ch = 0; ch < CH; ++ch) qv[ch] = (lane + 32 * ch < s) ? Qidx[lane + 32 * ch] : 0;
+  __syncwarp();   // the index slots become the staging row
+  float* stage = reinterpret_cast<float*>(Qidx);
   const bool vec = (B & 3) == 0;
   const int c4 = 4 * lane;
   for (int a0 = 0; a0 < s; a0 += 4) {
     float4 kv[4];
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-      const int a = a0 + r;
-      const float* krow = Kt + (size_t)(a < s ? Qidx[a] : Qidx[0]) * B;
+      const int a = a0 + r < s ? a0 + r : 0;
+      int qa = 0;
+#pragma unroll
+      for (int ch = 0; ch < CH; ++ch)
+        if ((a >> 5) == ch) qa = __shfl_sync(0xffffffffu, qv[ch], a & 31);
+      const float* krow = Kt + (size_t)qa * B;
       if (vec && c4 + 3 < nJ) {
         kv[r] = __ldg(reinterpret_cast<const float4*>(krow + c4));
       } else {
@@ -261,19 +267,17 @@ __device__ void gather_rhat(const Rows<SMALL> R, const float* __restrict__ Kt, c
     for (int r = 0; r < 4; ++r) {
       const int a = a0 + r;
       if (a >= s) break;
+      *reinterpret_cast<float4*>(stage + c4) = kv[r];
+      __syncwarp();
       float* row = R.row(a);
 #pragma unroll
       for (int ch = 0; ch < CH; ++ch) {
         if (32 * ch > a) break;
-        const int src = qv[ch] >> 2, comp = qv[ch] & 3;
-        const float vx = __shfl_sync(0xffffffffu, kv[r].x, src);
-        const float vy = __shfl_sync(0xffffffffu, kv[r].y, src);
-        const float vz = __shfl_sync(0xffffffffu, kv[r].z, src);
-        const float vw = __shfl_sync(0xffffffffu, kv[r].w, src);
-        const float v = comp == 0 ? vx : comp == 1 ? vy : comp == 2 ? vz : vw;
         const int cc = lane + 32 * ch;
+        const float v = stage[qv[ch]];
         if (cc <= a) row[cc] = v;
       }
+      __syncwarp();   // the staging row is rewritten next
     }
   }
   __syncwarp();
