@@ -45,12 +45,12 @@ constexpr int TM = 128, TN = 128, TK = 32, STAGES = 2;
 constexpr int A_BYTES = TM * TK * 4;                     // 16 KB: 128 rows x 128 bytes
 constexpr int B_BYTES = TN * TK * 4;                     // 16 KB: 128 rows x 128 bytes
 constexpr int STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;   // heads and remainders of both
-constexpr int W_BOX = TM * 32 * 4;                       // 16 KB: 128 rows x 32 columns of W
-constexpr int W_HALF = 2 * W_BOX;                        // 64 columns
+constexpr int W_BOX = TM * 32 * 4;                       // 16 KB: 128 rows x 32 columns of W (a quarter)
+constexpr int kWBufs = 4;                                // the ring of W quarters
 constexpr int W_OFF = STAGES * STAGE_BYTES;
-constexpr int HIST_OFF = W_OFF + 2 * W_HALF;
+constexpr int HIST_OFF = W_OFF + kWBufs * W_BOX;
 constexpr int BAR_OFF = HIST_OFF + kHist1Bins * 4;
-constexpr int SMEM_BYTES = 1024 + BAR_OFF + 128;
+constexpr int SMEM_BYTES = 1024 + BAR_OFF + 256;
 constexpr int kAccCols = 2 * TN;
 constexpr int kEpiWarps = 8, kProducerWarp = 8, kMmaWarp = 9, kWLoadWarp = 10, kThreads = 352;
 constexpr int kEpiBarrier = 1;
@@ -107,9 +107,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;   // accumulator a holds a finished tile
   uint64_t* tempty = tfull + 2;       // accumulator a has been read out
-  uint64_t* wfull = tempty + 2;       // W half h is in shared memory
-  uint64_t* wfree = wfull + 2;        // W half h has been stored back
-  uint64_t* drain = wfree + 2;
+  uint64_t* wfull = tempty + 2;       // W quarter buffer in shared memory
+  uint64_t* wdone = wfull + kWBufs;   // W quarter buffer computed, to be stored
+  uint64_t* drain = wdone + kWBufs;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   volatile int* abortp = &abort_flag;
@@ -132,8 +132,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], kEpiWarps);
-      mbar_init(&wfull[a], 1);
-      mbar_init(&wfree[a], 1);
+    }
+    for (int q = 0; q < kWBufs; ++q) {
+      mbar_init(&wfull[q], 1);
+      mbar_init(&wdone[q], 1);
     }
     mbar_init(drain, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -223,87 +225,117 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == kWLoadWarp) {
     if (lane == 0) {
+      // quarters g = 0, 1, .. of this CTA's walk (tile g/4, columns n0 + 32(g%4)..) in a
+      // ring of kWBufs buffers: quarter g loads into the buffer of quarter g - kWBufs once
+      // that one has been computed (wdone), stored, and read out of shared memory by its store
       prefetch_map(&mw);
-      int tc = 0, issued = 0;
+      int issued = 0, stored = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tc) {
+      auto store_quarter = [&](int gs) -> bool {
+        const int buf = gs % kWBufs;
+        if (!mbar_wait(&wdone[buf], (gs / kWBufs) & 1, abortp, spin)) return false;
+        int m0, n0;
+        tile_origin(blockIdx.x + (gs >> 2) * gridDim.x, mt, u0, upper, m0, n0);
+        // rows and columns outside W are not written
+        tma_store_2d(&mw, wbuf + buf * W_BOX, n0 + 32 * (gs & 3), m0);
+        bulk_commit();
+        return true;
+      };
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
         int m0, n0;
         tile_origin(tile, mt, u0, upper, m0, n0);
-        for (int h = 0; h < 2; ++h) {
-          if (tc >= 1 && !mbar_wait(&wfree[h], (tc - 1) & 1, abortp, spin)) {
-            ok = false;
-            break;
+        for (int qt = 0; qt < 4; ++qt) {
+          const int buf = issued % kWBufs;
+          if (issued >= kWBufs) {
+            if (!store_quarter(issued - kWBufs)) {
+              ok = false;
+              break;
+            }
+            ++stored;
+            bulk_wait_read0();   // that store has read the buffer
           }
-          uint8_t* dst = wbuf + h * W_HALF;
-          mbar_expect_tx(&wfull[h], W_HALF);
-          tma_load_2d(dst, &mw, &wfull[h], n0 + 64 * h, m0);
-          tma_load_2d(dst + W_BOX, &mw, &wfull[h], n0 + 64 * h + 32, m0);
+          mbar_expect_tx(&wfull[buf], W_BOX);
+          tma_load_2d(wbuf + buf * W_BOX, &mw, &wfull[buf], n0 + 32 * qt, m0);
           ++issued;
         }
       }
+      // the last quarters go back once computed (unless a role gave up)
+      while (ok && stored < issued) {
+        if (!store_quarter(stored)) {
+          ok = false;
+          break;
+        }
+        ++stored;
+      }
       if (!ok) *abortp = 1;
+      bulk_wait0();   // every store issued has completed
       // the last loads of W land before the CTA leaves, whether or not they were used
-      for (int k = issued - 2 > 0 ? issued - 2 : 0; k < issued; ++k)
-        mbar_wait(&wfull[k & 1], (k >> 1) & 1, kDrainLimit);
+      for (int k = issued - kWBufs > 0 ? issued - kWBufs : 0; k < issued; ++k)
+        mbar_wait(&wfull[k % kWBufs], (k / kWBufs) & 1, kDrainLimit);
     }
     __syncwarp();
   } else {
-    // epilogue: warp w reads accumulator lanes 32(w%4).. (tile rows) and, in each half,
-    // the 32 columns 32(w/4)..
+    // epilogue: warp w reads accumulator lanes 32(w%4).. (tile rows) and, in each W
+    // quarter, the 16 columns 16(w/4)..; quarter g of the walk sits in buffer g % kWBufs
     const int quarter = warp & 3, colsel = warp >> 2;
     const int rl = quarter * 32 + lane;  // tile row of this thread
-    int tc = 0;
-    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tc) {
+    int tc = 0, g = 0;
+    bool stop = false;
+    for (int tile = blockIdx.x; tile < ntiles && !stop; tile += gridDim.x, ++tc) {
       const int acc = tc & 1;
       int m0, n0;
-        tile_origin(tile, mt, u0, upper, m0, n0);
+      tile_origin(tile, mt, u0, upper, m0, n0);
       const int r = m0 + rl;
       const bool row_ok = r < c;
       bool ok = mbar_wait(&tfull[acc], (tc >> 1) & 1, abortp, spin);
-      bool stop = false;
-      for (int h = 0; h < 2; ++h) {
-        ok = ok && mbar_wait(&wfull[h], tc & 1, abortp, spin);
+      for (int qt = 0; qt < 4; ++qt, ++g) {
+        const int buf = g % kWBufs;
+        ok = ok && mbar_wait(&wfull[buf], (g / kWBufs) & 1, abortp, spin);
         ok = __all_sync(0xffffffffu, ok);
         if (ok) {
           fence_after();
-          float v[32];
-          tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * TN + h * 64 + colsel * 32), v);
-          if (h == 1) {  // this warp is done with the accumulator
+          float v[16];
+          tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * TN + qt * 32 + colsel * 16), v);
+          if (qt == 3) {  // this warp is done with the accumulator
             fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[acc]);
           }
-          const int q0 = n0 + h * 64 + colsel * 32;
-          uint8_t* box = wbuf + h * W_HALF + colsel * W_BOX;
-          if (q0 + 32 <= j) {
+          const int q0 = n0 + qt * 32 + colsel * 16;
+          uint8_t* box = wbuf + buf * W_BOX;
+          if (q0 + 16 <= j) {
             // previous block: apply, and zero the removed weights
             const uint32_t* mr = reinterpret_cast<const uint32_t*>(mask + (long long)r * b + q0);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              float4* p4 = reinterpret_cast<float4*>(box + sw_off(rl, u));
+            for (int uu = 0; uu < 4; ++uu) {
+              float4* p4 = reinterpret_cast<float4*>(box + sw_off(rl, 4 * colsel + uu));
               float4 w4 = *p4;
-              const uint32_t mb = row_ok ? mr[u] : 0u;
-              w4.x = (mb & 0xffu) ? 0.f : w4.x - v[4 * u];
-              w4.y = (mb & 0xff00u) ? 0.f : w4.y - v[4 * u + 1];
-              w4.z = (mb & 0xff0000u) ? 0.f : w4.z - v[4 * u + 2];
-              w4.w = (mb & 0xff000000u) ? 0.f : w4.w - v[4 * u + 3];
+              const uint32_t mb = row_ok ? mr[uu] : 0u;
+              w4.x = (mb & 0xffu) ? 0.f : w4.x - v[4 * uu];
+              w4.y = (mb & 0xff00u) ? 0.f : w4.y - v[4 * uu + 1];
+              w4.z = (mb & 0xff0000u) ? 0.f : w4.z - v[4 * uu + 2];
+              w4.w = (mb & 0xff000000u) ? 0.f : w4.w - v[4 * uu + 3];
               *p4 = w4;
             }
-          } else if (q0 >= j && q0 + 32 <= hist_end && q0 + 32 <= b) {
+          } else if (q0 >= j && q0 + 16 <= hist_end && q0 + 16 <= b) {
             // active columns, all scored
+            float4 s4[4];
+            if (SCORE != kNoScore) {
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              float4* p4 = reinterpret_cast<float4*>(box + sw_off(rl, u));
+              for (int uu = 0; uu < 4; ++uu) s4[uu] = __ldg(reinterpret_cast<const float4*>(sc + q0 + 4 * uu));
+            }
+#pragma unroll
+            for (int uu = 0; uu < 4; ++uu) {
+              float4* p4 = reinterpret_cast<float4*>(box + sw_off(rl, 4 * colsel + uu));
               float4 w4 = *p4;
-              w4.x -= v[4 * u];
-              w4.y -= v[4 * u + 1];
-              w4.z -= v[4 * u + 2];
-              w4.w -= v[4 * u + 3];
+              w4.x -= v[4 * uu];
+              w4.y -= v[4 * uu + 1];
+              w4.z -= v[4 * uu + 2];
+              w4.w -= v[4 * uu + 3];
               *p4 = w4;
               if (SCORE != kNoScore && row_ok) {
-                const float4 s4 = __ldg(reinterpret_cast<const float4*>(sc + q0 + 4 * u));
-                const unsigned int k0 = key_of<SCORE>(w4.x, s4.x), k1 = key_of<SCORE>(w4.y, s4.y);
-                const unsigned int k2 = key_of<SCORE>(w4.z, s4.z), k3 = key_of<SCORE>(w4.w, s4.w);
+                const unsigned int k0 = key_of<SCORE>(w4.x, s4[uu].x), k1 = key_of<SCORE>(w4.y, s4[uu].y);
+                const unsigned int k2 = key_of<SCORE>(w4.z, s4[uu].z), k3 = key_of<SCORE>(w4.w, s4[uu].w);
                 atomicAdd(&shist[k0 >> kKeyLoBits], 1u);
                 atomicAdd(&shist[k1 >> kKeyLoBits], 1u);
                 atomicAdd(&shist[k2 >> kKeyLoBits], 1u);
@@ -317,19 +349,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else if (q0 < b) {
             // mixed chunk (block edge, scored-range edge or the layer's last columns)
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              float4* p4 = reinterpret_cast<float4*>(box + sw_off(rl, u));
+            for (int uu = 0; uu < 4; ++uu) {
+              float4* p4 = reinterpret_cast<float4*>(box + sw_off(rl, 4 * colsel + uu));
               float o[4];
               {
                 const float4 w4 = *p4;
-                o[0] = w4.x - v[4 * u];
-                o[1] = w4.y - v[4 * u + 1];
-                o[2] = w4.z - v[4 * u + 2];
-                o[3] = w4.w - v[4 * u + 3];
+                o[0] = w4.x - v[4 * uu];
+                o[1] = w4.y - v[4 * uu + 1];
+                o[2] = w4.z - v[4 * uu + 2];
+                o[3] = w4.w - v[4 * uu + 3];
               }
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
-                const int q = q0 + 4 * u + e;
+                const int q = q0 + 4 * uu + e;
                 if (!row_ok || q >= b) continue;
                 if (q < j) {
                   if (mask[(long long)r * b + q]) o[e] = 0.f;
@@ -346,22 +378,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         stop = barrier_or(kEpiBarrier, kEpiWarps * 32, !ok || *abortp);
         if (stop) break;
-        if (tid == 0) {
-          // the whole half goes back; rows and columns outside W are not written
-          const uint8_t* src = wbuf + h * W_HALF;
-          tma_store_2d(&mw, src, n0 + 64 * h, m0);
-          tma_store_2d(&mw, src + W_BOX, n0 + 64 * h + 32, m0);
-          bulk_commit();
-          bulk_wait_read0();
-          mbar_arrive(&wfree[h]);
-        }
+        if (tid == 0) mbar_arrive(&wdone[buf]);   // the quarter is computed: the W thread stores it
       }
-      if (stop) {
-        if (lane == 0) *abortp = 1;
-        break;
-      }
+      if (stop && lane == 0) *abortp = 1;
     }
-    if (tid == 0) bulk_wait0();
   }
 
   fence_before();
