@@ -27,6 +27,7 @@ namespace pwp {
 namespace {
 
 constexpr int NB = kFactorNB;  // 64
+constexpr int kDiagThreads = 512;
 
 __global__ void __launch_bounds__(1024) damp_kernel(float* __restrict__ H, int b, float damp,
                                                     float* __restrict__ g_diag, pwp_stats* st) {
@@ -90,7 +91,8 @@ __device__ __forceinline__ bool chol_inv8(float (&L)[8][8], float (&X)[8][8]) {
 }
 
 // Factor the nb x nb diagonal block (nb <= 64) held in A (symmetric; the upper triangle
-// is read) as A = V V^T with V upper triangular, and invert V.  256 threads.
+// is read) as A = V V^T with V upper triangular, and invert V.  At least 64 threads (the
+// first 64 take each step's 8x8 block; every other loop is strided by the block size).
 // Working on the reversed matrix P = J A J (J the reversal; P[r][s] = A[63-r][63-s], so
 // P's lower triangle is A's upper one and the work happens in place), this is the
 // ordinary Cholesky P = L L^T from the top-left, with V = J L J and V^-1 = J X J for
@@ -198,8 +200,11 @@ __device__ bool factor_diag_block(float (*A)[NB + 1], float (*Wi)[NB + 1], int n
   return true;
 }
 
-// Stand-alone factorisation of the diagonal block at p0 (used for the last panel).
-__global__ void __launch_bounds__(256) chol_diag_kernel(float* __restrict__ H, int b, int p0, int nb,
+// Stand-alone factorisation of the diagonal block at p0 (used for the last panel, and for
+// every panel when the trailing update runs on the tensor cores): 512 threads, so that the
+// trailing updates of its 8-column steps spread thin (the step's 8x8 factor stays on the
+// first 64 threads).
+__global__ void __launch_bounds__(kDiagThreads) chol_diag_kernel(float* __restrict__ H, int b, int p0, int nb,
                                                         float* __restrict__ Vinv, pwp_stats* st) {
   pdl_enter();
   extern __shared__ __align__(16) float dsm[];   // A and Wi, 2 x NB x (NB + 1) floats
@@ -690,7 +695,7 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
   // factor, panels from the last; the last panel's diagonal block stands alone
   {
     const int p = np - 1, p0 = p * NB, nb = b - p0;
-    launch_pdl(chol_diag_kernel, dim3(1), dim3(256), 2 * NB * (NB + 1) * 4, s, H, b, p0, nb, Vall + (size_t)p * NB * NB, st);
+    launch_pdl(chol_diag_kernel, dim3(1), dim3(kDiagThreads), 2 * NB * (NB + 1) * 4, s, H, b, p0, nb, Vall + (size_t)p * NB * NB, st);
     ++nl;
   }
   for (int p = np - 1; p >= 1; --p) {
@@ -706,7 +711,7 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
                                      nullptr, p0, nullptr, nullptr, Level2{}, st, s, &e2, true);
     if (e2 != cudaSuccess) return e2;
     if (tc) {
-      launch_pdl(chol_diag_kernel, dim3(1), dim3(256), 2 * NB * (NB + 1) * 4, s, H, b, p0 - NB, NB, Vall + (size_t)(p - 1) * NB * NB, st);
+      launch_pdl(chol_diag_kernel, dim3(1), dim3(kDiagThreads), 2 * NB * (NB + 1) * 4, s, H, b, p0 - NB, NB, Vall + (size_t)(p - 1) * NB * NB, st);
     } else {
       const int nT = (p0 + 127) / 128;
       launch_pdl(chol_update_kernel, dim3(nT * (nT + 1) / 2), dim3(256), 2 * NB * 132 * 4, s, H, b, p0, nb,
