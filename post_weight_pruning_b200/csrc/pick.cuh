@@ -250,7 +250,7 @@ __device__ inline void count_ties(unsigned int T, Level2 l2, const float* W, int
   }
 #pragma unroll
   for (int e = 0; e < E; ++e)
-    if (cnt[e]) atomicAdd(&l2.tie_count[lane + 32 * e], cnt[e]);
+    if (cnt[e]) red_add_global(&l2.tie_count[lane + 32 * e], cnt[e]);
 }
 
 // The cut-off among the tied entries: with m of them taken in (column, row) order, the

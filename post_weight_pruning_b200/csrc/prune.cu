@@ -274,7 +274,7 @@ __global__ void __launch_bounds__(256) stream_kernel(float* __restrict__ W, int 
           if (Bp > 0) W[(long long)r * b + q] = v;
           if (SCORE != kNoScore && q < hist_end) {
             unsigned int key = key_of<SCORE>(v, __ldg(sc + q));
-            atomicAdd(&shist[key >> kKeyLoBits], 1u);
+            red_add_shared(&shist[key >> kKeyLoBits], 1u);
             count_level2(key, pred, h2, h2s);
           }
         }
@@ -285,7 +285,7 @@ __global__ void __launch_bounds__(256) stream_kernel(float* __restrict__ W, int 
     __syncthreads();
     for (int i = tid; i < kHist1Bins; i += blockDim.x) {
       unsigned int v = shist[i];
-      if (v) atomicAdd(&hist1[i], v);
+      if (v) red_add_global(&hist1[i], v);
     }
     // the last CTA to finish takes the block's level-1 bin (and threshold, when predicted)
     if (pk.enabled) pick::after_scoring(ctl, hist1, l2, pk.region_n, pk.global_budget, pk.quota, st, psh);

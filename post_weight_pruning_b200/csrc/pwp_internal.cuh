@@ -165,14 +165,23 @@ __device__ __forceinline__ unsigned int key_of(float w, float p) {
   return SCORE == kWanda ? score_key(wanda_score(w, p)) : score_key(obs_score(w, p));
 }
 
+// Counter increments whose old value nobody reads: reductions (red), which the issuing
+// thread does not wait for, unlike an atomic that returns the old value.
+__device__ __forceinline__ void red_add_shared(unsigned int* p, unsigned int v) {
+  asm volatile("red.shared.add.u32 [%0], %1;" ::"r"((unsigned int)__cvta_generic_to_shared(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ void red_add_global(unsigned int* p, unsigned int v) {
+  asm volatile("red.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // Level-2 histogram entry of a key whose level-1 bin is the predicted one (pred is
 // 0xffffffff when there is no prediction): the exact count plus its 512-bin summary.
 __device__ __forceinline__ void count_level2(unsigned int key, unsigned int pred, unsigned int* __restrict__ h2,
                                              unsigned int* __restrict__ h2s) {
   if ((key >> kKeyLoBits) == pred) {
     const unsigned int lo = key & (unsigned int)(kHist2Bins - 1);
-    atomicAdd(&h2[lo], 1u);
-    atomicAdd(&h2s[lo >> kHist2SumShift], 1u);
+    red_add_global(&h2[lo], 1u);
+    red_add_global(&h2s[lo >> kHist2SumShift], 1u);
   }
 }
 

@@ -336,10 +336,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (SCORE != kNoScore && row_ok) {
                 const unsigned int k0 = key_of<SCORE>(w4.x, s4[uu].x), k1 = key_of<SCORE>(w4.y, s4[uu].y);
                 const unsigned int k2 = key_of<SCORE>(w4.z, s4[uu].z), k3 = key_of<SCORE>(w4.w, s4[uu].w);
-                atomicAdd(&shist[k0 >> kKeyLoBits], 1u);
-                atomicAdd(&shist[k1 >> kKeyLoBits], 1u);
-                atomicAdd(&shist[k2 >> kKeyLoBits], 1u);
-                atomicAdd(&shist[k3 >> kKeyLoBits], 1u);
+                red_add_shared(&shist[k0 >> kKeyLoBits], 1u);
+                red_add_shared(&shist[k1 >> kKeyLoBits], 1u);
+                red_add_shared(&shist[k2 >> kKeyLoBits], 1u);
+                red_add_shared(&shist[k3 >> kKeyLoBits], 1u);
                 count_level2(k0, pred, h2, h2s);
                 count_level2(k1, pred, h2, h2s);
                 count_level2(k2, pred, h2, h2s);
@@ -367,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   if (mask[(long long)r * b + q]) o[e] = 0.f;
                 } else if (SCORE != kNoScore && q < hist_end) {
                   const unsigned int key = key_of<SCORE>(o[e], __ldg(sc + q));
-                  atomicAdd(&shist[key >> kKeyLoBits], 1u);
+                  red_add_shared(&shist[key >> kKeyLoBits], 1u);
                   count_level2(key, pred, h2, h2s);
                 }
               }
@@ -392,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (SCORE != kNoScore) {
     for (int i = tid; i < kHist1Bins; i += kThreads) {
       const unsigned int v = shist[i];
-      if (v) atomicAdd(&hist1[i], v);
+      if (v) red_add_global(&hist1[i], v);
     }
     // the last CTA to finish takes the block's level-1 bin (and threshold, when predicted)
     if (pk.enabled) pick::after_scoring(ctl, hist1, l2, pk.region_n, pk.global_budget, pk.quota, st, psh);
