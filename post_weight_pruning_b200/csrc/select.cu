@@ -27,13 +27,25 @@ __global__ void __launch_bounds__(pick::kThreads) select_finish_kernel(Ctl* ctl,
   // the outcome of the scoring pass's last CTA (an earlier kernel)
   if (ctl->mode == 0 || ctl->l2_ready) return;
   const int tid = threadIdx.x;
-  // the level-2 histogram of bin b1 over the region: rows over CTAs, columns over threads
+  // the level-2 histogram of bin b1 over the region: rows over CTAs, columns over threads,
+  // eight loads in flight per thread before their counts
   const unsigned int b1 = ctl->b1;
   const long long r1 = ctl->r1;
+  constexpr int kU = 8;
   for (int r = blockIdx.x; r < c; r += gridDim.x) {
     const float* wr = W + (long long)r * b;
-    for (int q = j + tid; q < q1; q += blockDim.x)
-      count_level2(key_of<SCORE>(wr[q], __ldg(sc + q)), b1, l2.reread, l2.reread_sum);
+    for (int q0 = j + tid; q0 < q1; q0 += kU * blockDim.x) {
+      float w[kU], p[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int q = q0 + u * blockDim.x;
+        w[u] = q < q1 ? wr[q] : 0.f;
+        p[u] = q < q1 ? __ldg(sc + q) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u)
+        if (q0 + u * blockDim.x < q1) count_level2(key_of<SCORE>(w[u], p[u]), b1, l2.reread, l2.reread_sum);
+    }
   }
   if (!pick::last_cta(&ctl->ticket, sh)) return;
   pick::level2(ctl, l2, r1, 0, st, sh, 1, tid);
