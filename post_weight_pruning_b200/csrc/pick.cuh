@@ -73,7 +73,8 @@ __device__ void find_rank(const unsigned int* __restrict__ hist, long long rank,
     const int per = size / kWarps;
     const unsigned int* h = hist + base + warp * per;
     long long sum = 0;
-    for (int i = lane; i < per; i += 32) sum += h[i];
+#pragma unroll 8
+    for (int i = lane; i < per; i += 32) sum += h[i];   // eight loads in flight
     sum = warp_sum_ll(sum);
     if (lane == 0) sh.warp[warp] = sum;
     sync(bar);
