@@ -21,7 +21,6 @@
 //   inverse, recursive doubling: with the diagonal blocks inverted, neighbouring
 //     blocks [A B; 0 D] are merged as [A^-1, -A^-1 B D^-1; 0, D^-1] level by level,
 //     each level two batched triangular-times-dense products.
-#include "diag_factor.cuh"
 #include "tc_common.cuh"
 
 namespace pwp {
@@ -29,7 +28,6 @@ namespace {
 
 constexpr int NB = kFactorNB;  // 64
 constexpr int kDiagThreads = 512;
-using diagf::factor_diag_block;
 
 __global__ void __launch_bounds__(1024) damp_kernel(float* __restrict__ H, int b, float damp,
                                                     float* __restrict__ g_diag, pwp_stats* st) {
@@ -58,6 +56,148 @@ __global__ void __launch_bounds__(1024) damp_kernel(float* __restrict__ H, int b
   __syncthreads();
   const float lam = lam_s;
   for (int q = threadIdx.x; q < b; q += blockDim.x) H[(long long)q * b + q] += lam;
+}
+
+// Cholesky and inverse of an 8 x 8 SPD block in registers (lower triangles; compile-time
+// indices throughout): L L^T = D, X = L^-1.  False on a non-positive pivot.
+__device__ __forceinline__ bool chol_inv8(float (&L)[8][8], float (&X)[8][8]) {
+  bool ok = true;
+  float il[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const float piv = L[c][c];
+    ok = ok && (piv > 0.f) && isfinite(piv);
+    il[c] = rsqrtf(piv);
+    L[c][c] = piv * il[c];
+#pragma unroll
+    for (int r = c + 1; r < 8; ++r) L[r][c] *= il[c];
+#pragma unroll
+    for (int r = c + 1; r < 8; ++r)
+#pragma unroll
+      for (int c2 = c + 1; c2 <= r; ++c2) L[r][c2] = fmaf(-L[r][c], L[c2][c], L[r][c2]);
+  }
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    X[r][r] = il[r];
+#pragma unroll
+    for (int c = 0; c < r; ++c) {
+      float acc = 0.f;
+#pragma unroll
+      for (int t = c; t < r; ++t) acc = fmaf(L[r][t], X[t][c], acc);
+      X[r][c] = -il[r] * acc;
+    }
+  }
+  return ok;
+}
+
+// Factor the nb x nb diagonal block (nb <= 64) held in A (symmetric; the upper triangle
+// is read) as A = V V^T with V upper triangular, and invert V.  At least 64 threads (the
+// first 64 take each step's 8x8 block; every other loop is strided by the block size).
+// Working on the reversed matrix P = J A J (J the reversal; P[r][s] = A[63-r][63-s], so
+// P's lower triangle is A's upper one and the work happens in place), this is the
+// ordinary Cholesky P = L L^T from the top-left, with V = J L J and V^-1 = J X J for
+// X = L^-1.  Right-looking in 8-column steps, every step two barriers apart:
+//   the step's 8 x 8 diagonal block is factored and inverted in registers (Ld, Xd) by
+//   each of the first 64 threads alike; thread r < 56 - k0 forms row k0+8+r of the panel,
+//   L[i, blk] = P[i, blk] Xd^T; thread t < k0 brings column t of the block's rows of X up
+//   to date, X[blk, t] := Xd X[blk, t] (those rows already carry the earlier steps'
+//   eliminations; their own columns become Xd);
+//   then all threads update the trailing part, P[i][j] -= L[i, blk] L[j, blk], and
+//   eliminate the block's rows from X's rows below it, X[i][t] -= L[i, blk] X[blk, t].
+// Rows and columns beyond nb (A indices >= nb) are an identity pad.  On return A's upper
+// triangle holds V and Wi holds V^-1 (upper, zero below).  Returns false on a
+// non-positive pivot (recorded in st).
+__device__ bool factor_diag_block(float (*A)[NB + 1], float (*Wi)[NB + 1], int nb, int* bad, pwp_stats* st) {
+  constexpr int BS = 8, NBK = NB / BS;
+  const int tid = threadIdx.x;
+  auto P = [&](int r, int c) -> float& { return A[NB - 1 - r][NB - 1 - c]; };
+  auto X = [&](int r, int c) -> float& { return Wi[NB - 1 - r][NB - 1 - c]; };
+  // identity pad beyond nb (A indices >= nb) and X = 0
+  for (int idx = tid; idx < NB * NB; idx += blockDim.x) {
+    const int i = idx / NB, jc = idx % NB;
+    if (i <= jc && jc >= nb) A[i][jc] = (i == jc) ? 1.f : 0.f;
+    Wi[i][jc] = 0.f;
+  }
+  if (tid == 0) *bad = 0;
+  __syncthreads();
+#pragma unroll 1
+  for (int kb = 0; kb < NBK; ++kb) {
+    const int k0 = BS * kb, r0 = k0 + BS, rest = NB - r0;
+    if (tid < 64) {
+      float Ld[8][8], Xd[8][8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          Ld[r][c] = c <= r ? P(k0 + r, k0 + c) : 0.f;
+          Xd[r][c] = 0.f;
+        }
+      const bool ok = chol_inv8(Ld, Xd);
+      if (!ok && tid == 0) *bad = 1;
+      if (tid < rest) {                      // panel row k0 + 8 + tid
+        const int i = r0 + tid;
+        float pr[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) pr[c] = P(i, k0 + c);
+#pragma unroll
+        for (int a = 0; a < 8; ++a) {
+          float acc = 0.f;
+#pragma unroll
+          for (int c = 0; c <= a; ++c) acc = fmaf(pr[c], Xd[a][c], acc);
+          P(i, k0 + a) = acc;
+        }
+      }
+      if (tid < k0) {                        // column tid of the block's rows of X
+        float xo[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) xo[c] = X(k0 + c, tid);
+#pragma unroll
+        for (int a = 0; a < 8; ++a) {
+          float acc = 0.f;
+#pragma unroll
+          for (int c = 0; c <= a; ++c) acc = fmaf(Xd[a][c], xo[c], acc);
+          X(k0 + a, tid) = acc;
+        }
+      }
+      if (tid == 63) {                       // the block itself
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+#pragma unroll
+          for (int c = 0; c <= r; ++c) {
+            P(k0 + r, k0 + c) = Ld[r][c];
+            X(k0 + r, k0 + c) = Xd[r][c];
+          }
+      }
+    }
+    __syncthreads();
+    if (*bad) {
+      if (tid == 0) set_error(st, PWP_ENOTSPD, kSiteCholDiag);
+      return false;
+    }
+    // trailing update of P (lower triangle of the rest x rest part) and elimination of
+    // the block's rows from the rows of X below it (columns < k0 + 8)
+    const int nP = rest * (rest + 1) / 2, nX = rest * r0;
+    for (int e = tid; e < nP + nX; e += blockDim.x) {
+      if (e < nP) {
+        int ii = (int)((sqrtf(8.f * (float)e + 1.f) - 1.f) * 0.5f);
+        if ((ii + 1) * (ii + 2) / 2 <= e) ++ii;
+        if (ii * (ii + 1) / 2 > e) --ii;
+        const int i = r0 + ii, j = r0 + (e - ii * (ii + 1) / 2);
+        float acc = P(i, j);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc = fmaf(-P(i, k0 + c), P(j, k0 + c), acc);
+        P(i, j) = acc;
+      } else {
+        const int e2 = e - nP, i = r0 + e2 / r0, t = e2 % r0;
+        float acc = X(i, t);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc = fmaf(-P(i, k0 + c), X(k0 + c, t), acc);
+        X(i, t) = acc;
+      }
+    }
+    __syncthreads();
+  }
+  return true;
 }
 
 // Stand-alone factorisation of the diagonal block at p0 (used for the last panel, and for
@@ -90,25 +230,15 @@ __global__ void __launch_bounds__(kDiagThreads) chol_diag_kernel(float* __restri
 // per row over a grid of one CTA per SM (the 64x64 inverse is staged once per CTA);
 // lane l produces columns l and l + 32.  With vs_hi set, the rows also go to vs_hi /
 // vs_lo (row stride NB) as TF32 head and fp32 remainder: the operand of the tensor-core
-// trailing update.  With dsnap set, CTA 0 also copies the next panel's diagonal block
-// (before this panel's update) there, for the update's look-ahead CTA.
+// trailing update.
 __global__ void __launch_bounds__(256) chol_panel_kernel(float* __restrict__ H, int b, int p0, int nb,
                                                          const float* __restrict__ Vinv,
                                                          float* __restrict__ vs_hi, float* __restrict__ vs_lo,
-                                                         float* __restrict__ dsnap, const pwp_stats* st) {
+                                                         const pwp_stats* st) {
   pdl_enter();
   __shared__ float WiT[NB][NB + 1];  // WiT[t][c] = Wi[c][t]
   __shared__ float rowbuf[8][NB];
   if (cta_failed(st)) return;
-  if (dsnap && blockIdx.x == 0) {
-    // the next panel's diagonal block [p0-NB, p0) as it stands before this panel's update
-    // (this kernel writes only columns >= p0), for the update's look-ahead CTA
-    const int q0 = p0 - NB;
-    for (int idx = threadIdx.x; idx < NB * NB; idx += blockDim.x) {
-      const int r = idx / NB, c = idx % NB;
-      if (r <= c) dsnap[idx] = H[(long long)(q0 + r) * b + q0 + c];
-    }
-  }
   for (int idx = threadIdx.x; idx < NB * NB; idx += blockDim.x) WiT[idx % NB][idx / NB] = Vinv[idx];
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -486,8 +616,7 @@ static size_t tc_levels_floats(int b) {
 // and remainder (2 x b x NB), the last 256-byte aligned, then the tensor-core levels' scratch.
 size_t factor_ws_bytes(int b) {
   const size_t np = (size_t)(b + NB - 1) / NB;
-  return (np * NB * NB + doubling_tmp_floats(b) + 2 * (size_t)b * NB + tc_levels_floats(b) + NB * NB) * sizeof(float) +
-         1024;
+  return (np * NB * NB + doubling_tmp_floats(b) + 2 * (size_t)b * NB + tc_levels_floats(b)) * sizeof(float) + 1024;
 }
 
 // One pair [A B; 0 D] of a doubling level on the tensor cores: T = A^-1 B, then
@@ -554,7 +683,6 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
       (reinterpret_cast<uintptr_t>(T + doubling_tmp_floats(b)) + 255) & ~(uintptr_t)255);
   float* vs_lo = vs_hi + (size_t)b * NB;
   float* tcw = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(vs_lo + (size_t)b * NB) + 255) & ~(uintptr_t)255);
-  float* dsnap = tcw + tc_levels_floats(b);   // the look-ahead's snapshot of the next diagonal block
   static std::atomic<unsigned long long> attr_done{0};
   if (first_on_device(attr_done)) {
     cudaFuncSetAttribute(chol_update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * NB * 132 * 4);
@@ -574,22 +702,22 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
     const int p0 = p * NB, nb = min(NB, b - p0);
     float* V = Vall + (size_t)p * NB * NB;
     const int pgrid = min((p0 + 7) / 8, kNumSM);
-    launch_pdl(chol_panel_kernel, dim3(pgrid), dim3(256), 0, s, H, b, p0, nb, V, vs_hi, vs_lo, dsnap, st);
+    launch_pdl(chol_panel_kernel, dim3(pgrid), dim3(256), 0, s, H, b, p0, nb, V, vs_hi, vs_lo, st);
     // H[0:p0, 0:p0] -= V[0:p0, P] V[0:p0, P]^T on the tensor cores (tiles on or above the
-    // diagonal) while one more CTA of the same launch forms and factors the next panel's
-    // diagonal block from the snapshot (look-ahead); the CUDA-core kernel (which also
-    // factors that block) when the tensor-core path is not available
+    // diagonal), then the next panel's diagonal block on its own; the CUDA-core kernel
+    // (which also factors that block) when the tensor-core path is not available
     cudaError_t e2 = cudaSuccess;
-    const DiagAhead da{H, b, p0 - NB, p0, nb, dsnap, Vall + (size_t)(p - 1) * NB * NB, 1};
     const bool tc = launch_stream_tc(kNoScore, H, p0, p0, b, 0, 0, vs_hi, vs_lo, nb, NB, vs_hi, vs_lo, nullptr,
-                                     nullptr, p0, nullptr, nullptr, Level2{}, st, s, &e2, true, PickArgs{}, da);
+                                     nullptr, p0, nullptr, nullptr, Level2{}, st, s, &e2, true);
     if (e2 != cudaSuccess) return e2;
-    if (!tc) {
+    if (tc) {
+      launch_pdl(chol_diag_kernel, dim3(1), dim3(kDiagThreads), 2 * NB * (NB + 1) * 4, s, H, b, p0 - NB, NB, Vall + (size_t)(p - 1) * NB * NB, st);
+    } else {
       const int nT = (p0 + 127) / 128;
       launch_pdl(chol_update_kernel, dim3(nT * (nT + 1) / 2), dim3(256), 2 * NB * 132 * 4, s, H, b, p0, nb,
                                                                         Vall + (size_t)(p - 1) * NB * NB, st);
     }
-    nl += tc ? 2 : 3;
+    nl += 3;
   }
   launch_pdl(put_diag_inverses_kernel, dim3(np), dim3(256), 0, s, H, b, Vall, st);
   ++nl;

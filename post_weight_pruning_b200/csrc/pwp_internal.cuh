@@ -268,20 +268,6 @@ void launch_sweep_select(int step, int score, Ctl* ctl, unsigned int* hist1, Lev
                          int c, int b, int j, int j1, int q1, const float* sc, const unsigned int* ties_all, int world,
                          int rank, pwp_stats* st, cudaStream_t s);
 
-// Look-ahead of the factor's tensor-core trailing update (stream_tc.cu): one extra CTA
-// forms the next diagonal block [q0, q0+64) from its snapshot taken before this panel's
-// update, dsnap - V V^T with V = H[q0:q0+64, p0:p0+nb] (the panel's rows, already in H),
-// and factors and inverts it into vinv (64 x 64, upper) while the other CTAs update the
-// rest.  Its entries of H are left to the update (nothing reads them before the inverse
-// blocks replace them).
-struct DiagAhead {
-  const float* H;
-  int b, q0, p0, nb;
-  const float* dsnap;   // 64 x 64, row stride 64, upper triangle
-  float* vinv;
-  int enabled;
-};
-
 // W[:, u0:b] -= Z R on the tensor cores (stream_tc.cu), fused with zeroing the previous
 // block's removals and the level-1 histogram of the scores of columns [j, hist_end).
 // W is c x b with row stride ldw (mask: row stride b); with `upper` (c == b, u0 == 0)
@@ -292,8 +278,7 @@ struct DiagAhead {
 bool launch_stream_tc(int score, float* W, int c, int b, int ldw, int u0, int j, const float* Zhi, const float* Zlo,
                       int Bp, int ldz, const float* Rhi, const float* Rlo, const uint8_t* mask, const float* sc,
                       int hist_end, unsigned int* hist1, Ctl* ctl, Level2 l2, pwp_stats* st,
-                      cudaStream_t s, cudaError_t* err, bool upper = false, PickArgs pick = PickArgs{},
-                      DiagAhead diag = DiagAhead{});
+                      cudaStream_t s, cudaError_t* err, bool upper = false, PickArgs pick = PickArgs{});
 
 // Wanda / magnitude: per-row quota or N:M groups, no weight update (rowprune.cu).  H
 // (its diagonal) or X ([n, b]) gives ||X_q|| for Wanda.

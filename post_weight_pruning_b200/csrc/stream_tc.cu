@@ -33,7 +33,6 @@
 // at their next wait, and the epilogue warps take each stop decision together through a
 // reducing barrier.  Copies and MMAs already in flight are always waited for before the
 // CTA leaves.
-#include "diag_factor.cuh"
 #include "pick.cuh"
 #include "tc_common.cuh"
 
@@ -88,42 +87,13 @@ __device__ __forceinline__ void tile_origin(int tile, int mt, int u0, int upper,
 // Byte offset of the 16-byte unit u (columns 4u..4u+3) of row r in a 128-byte-swizzled box.
 __device__ __forceinline__ uint32_t sw_off(int r, int u) { return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4)); }
 
-// The factor's look-ahead (DiagAhead): the next diagonal block from its snapshot minus the
-// panel's rank-nb product, V staged in shared memory, then factored and inverted into
-// vinv.  All threads of the CTA; smem holds A, Wi and V (64 x 65 floats each).
-__device__ void diag_ahead(const DiagAhead& da, float* smem, int* bad, pwp_stats* st) {
-  constexpr int NB = kFactorNB;
-  float (*A)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(smem);
-  float (*Wi)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(smem + NB * (NB + 1));
-  float (*Vd)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(smem + 2 * NB * (NB + 1));
-  for (int idx = threadIdx.x; idx < NB * NB; idx += blockDim.x) {
-    const int r = idx / NB, t = idx % NB;
-    Vd[r][t] = t < da.nb ? da.H[(long long)(da.q0 + r) * da.b + da.p0 + t] : 0.f;
-  }
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < NB * NB; idx += blockDim.x) {
-    const int r = idx / NB, c = idx % NB;
-    if (r > c) continue;
-    float acc = da.dsnap[idx];
-#pragma unroll 8
-    for (int t = 0; t < NB; ++t) acc = fmaf(-Vd[r][t], Vd[c][t], acc);
-    A[r][c] = acc;
-  }
-  __syncthreads();
-  if (!diagf::factor_diag_block(A, Wi, NB, bad, st)) return;
-  for (int idx = threadIdx.x; idx < NB * NB; idx += blockDim.x) {
-    const int r = idx / NB, c = idx % NB;
-    da.vinv[idx] = r <= c ? Wi[r][c] : 0.f;
-  }
-}
-
 template <int SCORE>
 __global__ void __launch_bounds__(kThreads, 1)
     stream_tc_kernel(const __grid_constant__ CUtensorMap mzh, const __grid_constant__ CUtensorMap mzl,
                      const __grid_constant__ CUtensorMap mrh, const __grid_constant__ CUtensorMap mrl,
                      const __grid_constant__ CUtensorMap mw, int c, int b, int u0, int j, int Bp, int upper,
                      const uint8_t* __restrict__ mask, const float* __restrict__ sc, int hist_end,
-                     unsigned int* hist1, Ctl* ctl, Level2 l2, PickArgs pk, DiagAhead da,
+                     unsigned int* hist1, Ctl* ctl, Level2 l2, PickArgs pk,
                      pwp_stats* st, long long spin) {
   unsigned int* h2 = l2.pred;
   unsigned int* h2s = l2.pred_sum;
@@ -144,14 +114,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int abort_flag;
   volatile int* abortp = &abort_flag;
 
-  __shared__ int diag_bad;
   if (cta_failed(st)) return;
-  if (da.enabled && blockIdx.x == 0) {   // the factor's look-ahead CTA (no tiles)
-    diag_ahead(da, reinterpret_cast<float*>(smem), &diag_bad, st);
-    return;
-  }
-  // the tile walk over the CTAs other than the look-ahead one
-  const int cta = blockIdx.x - (da.enabled ? 1 : 0), nctas = gridDim.x - (da.enabled ? 1 : 0);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int mt = (c + TM - 1) / TM;
   const int ntiles = upper ? mt * (mt + 1) / 2 : mt * ((b - u0 + TN - 1) / TN);
@@ -192,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_map(&mrl);
       int it = 0;
       bool ok = true;
-      for (int tile = cta; tile < ntiles && ok; tile += nctas) {
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
         int m0, n0;
         tile_origin(tile, mt, u0, upper, m0, n0);
         for (int kc = 0; kc < nkc; ++kc) {
@@ -221,7 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sbase = smem_u32(smem);
       int it = 0, tc = 0;
       bool ok = true;
-      for (int tile = cta; tile < ntiles && ok; tile += nctas, ++tc) {
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tc) {
         const int acc = tc & 1;
         if (tc >= 2 && !mbar_wait(&tempty[acc], ((tc >> 1) - 1) & 1, abortp, spin)) {
           ok = false;
@@ -272,13 +235,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int buf = gs % kWBufs;
         if (!mbar_wait(&wdone[buf], (gs / kWBufs) & 1, abortp, spin)) return false;
         int m0, n0;
-        tile_origin(cta + (gs >> 2) * nctas, mt, u0, upper, m0, n0);
+        tile_origin(blockIdx.x + (gs >> 2) * gridDim.x, mt, u0, upper, m0, n0);
         // rows and columns outside W are not written
         tma_store_2d(&mw, wbuf + buf * W_BOX, n0 + 32 * (gs & 3), m0);
         bulk_commit();
         return true;
       };
-      for (int tile = cta; tile < ntiles && ok; tile += nctas) {
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
         int m0, n0;
         tile_origin(tile, mt, u0, upper, m0, n0);
         for (int qt = 0; qt < 4; ++qt) {
@@ -318,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int rl = quarter * 32 + lane;  // tile row of this thread
     int tc = 0, g = 0;
     bool stop = false;
-    for (int tile = cta; tile < ntiles && !stop; tile += nctas, ++tc) {
+    for (int tile = blockIdx.x; tile < ntiles && !stop; tile += gridDim.x, ++tc) {
       const int acc = tc & 1;
       int m0, n0;
       tile_origin(tile, mt, u0, upper, m0, n0);
@@ -439,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int SCORE>
 cudaError_t launch_variant(const CUtensorMap* maps, int c, int b, int u0, int j, int Bp, int upper,
                            const uint8_t* mask, const float* sc, int hist_end, unsigned int* hist1, Ctl* ctl,
-                           Level2 l2, PickArgs pk, DiagAhead da, pwp_stats* st, cudaStream_t s) {
+                           Level2 l2, PickArgs pk, pwp_stats* st, cudaStream_t s) {
   static std::atomic<unsigned long long> attr_done{0};
   if (first_on_device(attr_done)) {
     cudaError_t e = cudaFuncSetAttribute(stream_tc_kernel<SCORE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -451,11 +414,9 @@ cudaError_t launch_variant(const CUtensorMap* maps, int c, int b, int u0, int j,
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   const int mt = (c + TM - 1) / TM;
   const int ntiles = upper ? mt * (mt + 1) / 2 : mt * ((b - u0 + TN - 1) / TN);
-  // one CTA per SM; with the look-ahead, one SM goes to it (block 0, scheduled first)
-  const int tile_ctas = da.enabled ? (ntiles < nsm - 1 ? ntiles : nsm - 1) : (ntiles < nsm ? ntiles : nsm);
-  const int grid = tile_ctas + (da.enabled ? 1 : 0);
+  const int grid = ntiles < nsm ? ntiles : nsm;
   launch_pdl(stream_tc_kernel<SCORE>, dim3(grid), dim3(kThreads), SMEM_BYTES, s, maps[0], maps[1], maps[2], maps[3],
-             maps[4], c, b, u0, j, Bp, upper, mask, sc, hist_end, hist1, ctl, l2, pk, da, st, wait_limit());
+             maps[4], c, b, u0, j, Bp, upper, mask, sc, hist_end, hist1, ctl, l2, pk, st, wait_limit());
   return cudaGetLastError();
 }
 
@@ -478,10 +439,9 @@ bool encode_f32(CUtensorMap* map, const float* base, int inner, int rows, int ld
 bool launch_stream_tc(int score, float* W, int c, int b, int ldw, int u0, int j, const float* Zhi, const float* Zlo,
                       int Bp, int ldz, const float* Rhi, const float* Rlo, const uint8_t* mask, const float* sc,
                       int hist_end, unsigned int* hist1, Ctl* ctl, Level2 l2, pwp_stats* st, cudaStream_t s,
-                      cudaError_t* err, bool upper, PickArgs pk, DiagAhead da) {
+                      cudaError_t* err, bool upper, PickArgs pk) {
   *err = cudaSuccess;
   if (upper && (c != b || u0 != 0)) return false;
-  if (da.enabled && (score != kNoScore || pk.enabled)) return false;   // the look-ahead goes with the factor's update only
   // b, u0 multiples of 4: the epilogue moves whole float4s of W and 4-byte words of mask
   if (c < 1 || Bp < 1 || Bp > ldz || u0 >= b || (b % 4) != 0 || (ldw % 4) != 0 || ldw < b || (ldz % 4) != 0 ||
       (u0 % 4) != 0)
@@ -495,11 +455,11 @@ bool launch_stream_tc(int score, float* W, int c, int b, int ldw, int u0, int j,
       !encode_f32(&maps[4], W, b, c, ldw, 32, TM))
     return false;
   if (score == kWanda)
-    *err = launch_variant<kWanda>(maps, c, b, u0, j, Bp, upper ? 1 : 0, mask, sc, hist_end, hist1, ctl, l2, pk, da, st, s);
+    *err = launch_variant<kWanda>(maps, c, b, u0, j, Bp, upper ? 1 : 0, mask, sc, hist_end, hist1, ctl, l2, pk, st, s);
   else if (score == kObs)
-    *err = launch_variant<kObs>(maps, c, b, u0, j, Bp, upper ? 1 : 0, mask, sc, hist_end, hist1, ctl, l2, pk, da, st, s);
+    *err = launch_variant<kObs>(maps, c, b, u0, j, Bp, upper ? 1 : 0, mask, sc, hist_end, hist1, ctl, l2, pk, st, s);
   else
-    *err = launch_variant<kNoScore>(maps, c, b, u0, j, Bp, upper ? 1 : 0, mask, sc, hist_end, hist1, ctl, l2, pk, da, st, s);
+    *err = launch_variant<kNoScore>(maps, c, b, u0, j, Bp, upper ? 1 : 0, mask, sc, hist_end, hist1, ctl, l2, pk, st, s);
   return true;
 }
 
