@@ -160,6 +160,28 @@ pwp_status pwp_prune_layer_x(const pwp_config* cfg, const void* W_dev, int32_t w
                              int64_t n, float* H_dev, float* W_out_dev, uint8_t* mask_dev,
                              void* ws, size_t ws_bytes, pwp_stats* stats_dev, void* stream);
 
+/* One layer end to end from host memory, the transfers overlapping the work.
+ *   W_host, X_host  : pinned host copies of W (c x b, wtype) and X ([n, b], xtype).
+ *   W_dev, X_dev    : device buffers of the same sizes (overwritten with the copies).
+ *   H_dev           : b x b fp32 device scratch (as pwp_prune_layer_x; may be NULL for
+ *                     PWP_WANDA and PWP_MAGNITUDE).
+ *   W_out_dev, mask_dev : device results, as pwp_prune_layer.
+ *   W_out_host, mask_out_host : pinned host buffers (c x b fp32, c x b bytes) receiving
+ *                     copies of the results.
+ * X goes in in row chunks on a copy stream of the call's own, each chunk folded into H as
+ * soon as it lands (the fp32 sum over chunks rounds like any other split of the tokens);
+ * W follows while H is factored; with PWP_THANOS and PWP_SPARSEGPT (alpha 0) every column
+ * block of W-hat and of the mask goes back as soon as the sweep has finished it (its update
+ * and its removals applied), the rest at the end.  The work is enqueued on `stream`, which
+ * waits for the last copy: once it is synchronised, the host outputs are complete.  Errors
+ * as pwp_prune_layer_x. */
+pwp_status pwp_prune_layer_host(const pwp_config* cfg, const void* W_host, int32_t wtype,
+                                int32_t c, int32_t b, const void* X_host, int32_t xtype,
+                                int64_t n, void* W_dev, void* X_dev, float* H_dev,
+                                float* W_out_dev, uint8_t* mask_dev, float* W_out_host,
+                                uint8_t* mask_out_host, void* ws, size_t ws_bytes,
+                                pwp_stats* stats_dev, void* stream);
+
 /* Stepwise sweep: one layer's rows sharded over ranks (one process per GPU), pruned with the
  * unstructured budget counted over all ranks' rows ("Pruning LLMs with Thanos", section
  * "Contribution two: keep the budget global and the execution local": the budget couples

@@ -69,6 +69,8 @@ _SIGS = {
                                _vp, _vp]),
     "pwp_prune_layer_x": (_i32, [ctypes.POINTER(Config), _vp, _i32, _i32, _i32, _vp, _i32, _i64, _vp,
                                  _vp, _vp, _vp, _sz, _vp, _vp]),
+    "pwp_prune_layer_host": (_i32, [ctypes.POINTER(Config), _vp, _i32, _i32, _i32, _vp, _i32, _i64, _vp, _vp,
+                                    _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
     "pwp_pack_24": (_i32, [_vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp]),
     "pwp_status_string": (ctypes.c_char_p, [_i32]),
     "pwp_sweep_step": (_i32, [ctypes.POINTER(SweepArgs), _i32, _i32]),
@@ -418,20 +420,51 @@ def pack_24(W_hat, mask, *, stream=None, check=True):
     return values, meta, s
 
 
-def prune_layer_host(W_host, X_host, *, out_W=None, out_mask=None, device="cuda", **kw):
-    """End-to-end call from host memory: copies W and X (pinned torch CPU tensors) to the
-    device, prunes, and copies W_hat and the mask back into (pinned) host tensors."""
+def prune_layer_host(W_host, X_host, *, out_W=None, out_mask=None, device="cuda", stream=None, **kw):
+    """End-to-end call from host memory (pwp_prune_layer_host): W ([c, b]) and X ([n, b]),
+    bf16/fp32 pinned torch CPU tensors, go to the device on a copy stream of the call's own
+    -- X in chunks folded into H as they land, W while H is factored -- and the finished
+    column blocks of W_hat and the mask come back into pinned host tensors during the sweep.
+    Keyword arguments as prune_layer (method, sparsity, pattern, nm, block, damp, alpha).
+    Returns (W_hat, mask, stats tensor); nothing syncs: synchronise the stream (the current
+    one by default) before reading them."""
     torch = _torch()
+    if W_host.dim() != 2 or X_host.dim() != 2 or X_host.shape[1] != W_host.shape[1]:
+        raise ValueError(f"W [c, b] and X [n, b] expected, got {tuple(W_host.shape)} and {tuple(X_host.shape)}")
     c, b = W_host.shape
-    Wd = W_host.to(device, non_blocking=True)
-    Xd = X_host.to(device, non_blocking=True)
-    Wo, mk, stats = prune_layer(Wd, X=Xd, check=False, **kw)
+    n = X_host.shape[0]
+    for name, t in (("W_host", W_host), ("X_host", X_host)):
+        if t.device.type != "cpu" or not t.is_pinned() or not t.is_contiguous():
+            raise ValueError(f"{name}: a contiguous pinned CPU tensor is required")
+        if t.dtype not in (torch.bfloat16, torch.float32):
+            raise ValueError(f"{name}: bf16 or fp32 expected, got {t.dtype}")
     if out_W is None:
         out_W = torch.empty((c, b), dtype=torch.float32, pin_memory=True)
     if out_mask is None:
         out_mask = torch.empty((c, b), dtype=torch.uint8, pin_memory=True)
-    out_W.copy_(Wo, non_blocking=True)
-    out_mask.copy_(mk, non_blocking=True)
+    for name, t, dt in (("out_W", out_W, torch.float32), ("out_mask", out_mask, torch.uint8)):
+        if t.shape != (c, b) or t.dtype != dt or not t.is_pinned() or not t.is_contiguous():
+            raise ValueError(f"{name}: a contiguous pinned CPU tensor [{c}, {b}] of {dt} is required")
+    cfg = config(kw.pop("method", "thanos"), kw.pop("pattern", "unstructured"), kw.pop("nm", (2, 4)),
+                 kw.pop("sparsity", 0.5), kw.pop("block", 128), kw.pop("damp", 0.01), kw.pop("alpha", 0.0))
+    if kw:
+        raise TypeError(f"unexpected arguments {sorted(kw)}")
+    dev = torch.device(device)
+    W_dev = torch.empty((c, b), dtype=W_host.dtype, device=dev)
+    X_dev = torch.empty((n, b), dtype=X_host.dtype, device=dev)
+    no_update = cfg.method in (WANDA, MAGNITUDE)
+    H_dev = None if no_update else torch.empty((b, b), dtype=torch.float32, device=dev)
+    W_out = torch.empty((c, b), dtype=torch.float32, device=dev)
+    mask = torch.empty((c, b), dtype=torch.uint8, device=dev)
+    workspace = make_workspace(cfg, c, b, dev)
+    stats = new_stats(dev)
+    st = lib().pwp_prune_layer_host(ctypes.byref(cfg), _vp(W_host.data_ptr()), _dtype_code(W_host), int(c), int(b),
+                                    _vp(X_host.data_ptr()), _dtype_code(X_host), int(n), _vp(W_dev.data_ptr()),
+                                    _vp(X_dev.data_ptr()), _vp(H_dev.data_ptr() if H_dev is not None else 0),
+                                    _vp(W_out.data_ptr()), _vp(mask.data_ptr()), _vp(out_W.data_ptr()),
+                                    _vp(out_mask.data_ptr()), _vp(workspace.ws.data_ptr()), workspace.nbytes,
+                                    _vp(stats.data_ptr()), _stream_ptr(stream))
+    _check(st, "pwp_prune_layer_host")
     return out_W, out_mask, stats
 
 

@@ -143,6 +143,95 @@ pwp_status pwp_prune_layer_x(const pwp_config* cfg, const void* W, int32_t wtype
   return e == cudaSuccess ? PWP_OK : PWP_ECUDA;
 }
 
+static size_t dtype_bytes(int32_t t) { return t == PWP_BF16 ? 2 : 4; }
+
+pwp_status pwp_prune_layer_host(const pwp_config* cfg, const void* W_host, int32_t wtype, int32_t c, int32_t b,
+                                const void* X_host, int32_t xtype, int64_t n, void* W_dev, void* X_dev,
+                                float* H_dev, float* W_out_dev, uint8_t* mask_dev, float* W_out_host,
+                                uint8_t* mask_out_host, void* ws, size_t ws_bytes, pwp_stats* st, void* stream) {
+  const bool no_update = valid_cfg(cfg, c, b) && (cfg->method == PWP_WANDA || cfg->method == PWP_MAGNITUDE);
+  if (!valid_cfg(cfg, c, b) || !valid_dtype(wtype) || !valid_dtype(xtype) || !W_host || !W_dev ||
+      (!H_dev && !no_update) || !W_out_dev || !mask_dev || !W_out_host || !mask_out_host || !st || n < 0 ||
+      (n > 0 && (!X_host || !X_dev)))
+    return PWP_EINVAL;
+  if (!ws || !aligned(ws, 256) || ws_bytes < prune_ws_layout(cfg, c, b, nullptr, nullptr))
+    return PWP_EWORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  // a copy stream and two events of this call's own (released once their work is done)
+  cudaStream_t cp = nullptr;
+  cudaEvent_t ev = nullptr, ev_w = nullptr;
+  if (cudaStreamCreateWithFlags(&cp, cudaStreamNonBlocking) != cudaSuccess) return PWP_ECUDA;
+  cudaError_t e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_w, cudaEventDisableTiming);
+  // the copies start after the caller's earlier work on `stream`
+  if (e == cudaSuccess) e = cudaEventRecord(ev, s);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(cp, ev, 0);
+  if (e == cudaSuccess) e = launch_stats_init(st, s);
+  pwp_status ps = e == cudaSuccess ? PWP_OK : PWP_ECUDA;
+  const size_t xrow = (size_t)b * dtype_bytes(xtype);
+  if (ps == PWP_OK && no_update) {
+    // Wanda and magnitude: no Hessian; X (Wanda's column norms) and W, then the prune
+    if (n > 0) e = cudaMemcpyAsync(X_dev, X_host, (size_t)n * xrow, cudaMemcpyHostToDevice, cp);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(W_dev, W_host, (size_t)c * b * dtype_bytes(wtype), cudaMemcpyHostToDevice, cp);
+    if (e == cudaSuccess) e = cudaEventRecord(ev, cp);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev, 0);
+    if (e == cudaSuccess)
+      e = launch_no_update(cfg, W_dev, wtype, c, b, nullptr, cfg->method == PWP_WANDA ? X_dev : nullptr, xtype,
+                           cfg->method == PWP_WANDA ? n : 0, W_out_dev, mask_dev, ws, st, true, s);
+    if (e != cudaSuccess) ps = PWP_ECUDA;
+  } else if (ps == PWP_OK) {
+    // X in row chunks, each folded into H as soon as it lands; then W, which the prune first
+    // needs after the factor
+    const int64_t nch = n >= 8 * 1024 ? 8 : 1;
+    const int64_t rows = (n + nch - 1) / nch;
+    for (int64_t r0 = 0; r0 < n && ps == PWP_OK; r0 += rows) {
+      const int64_t nr = n - r0 < rows ? n - r0 : rows;
+      e = cudaMemcpyAsync((char*)X_dev + (size_t)r0 * xrow, (const char*)X_host + (size_t)r0 * xrow,
+                          (size_t)nr * xrow, cudaMemcpyHostToDevice, cp);
+      if (e == cudaSuccess) e = cudaEventRecord(ev, cp);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev, 0);
+      if (e != cudaSuccess) {
+        ps = PWP_ECUDA;
+        break;
+      }
+      ps = hessian_impl((const char*)X_dev + (size_t)r0 * xrow, xtype, nr, b, H_dev, r0 > 0 ? 1 : 0, st, s);
+    }
+    if (ps == PWP_OK && n == 0) e = cudaMemsetAsync(H_dev, 0, (size_t)b * b * sizeof(float), s);
+    if (ps == PWP_OK && e == cudaSuccess)
+      e = cudaMemcpyAsync(W_dev, W_host, (size_t)c * b * dtype_bytes(wtype), cudaMemcpyHostToDevice, cp);
+    if (ps == PWP_OK && e == cudaSuccess) e = cudaEventRecord(ev_w, cp);
+    if (ps == PWP_OK && e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_w, 0);
+    // finished column blocks go back during the sweep (not for outlier rows, whose compact
+    // prune is scattered back at the end)
+    const HostOut ho{W_out_host, mask_out_host, cp, ev};
+    const bool blockwise = cfg->alpha == 0.f;
+    if (ps == PWP_OK && e == cudaSuccess)
+      e = launch_prune_out(cfg, W_dev, wtype, c, b, H_dev, W_out_dev, mask_dev, ws, st, s, true,
+                           blockwise ? &ho : nullptr);
+    if (e != cudaSuccess) ps = PWP_ECUDA;
+    if (ps == PWP_OK && blockwise) {
+      // the outputs are on their way; `stream` waits for the last copies
+      e = cudaEventRecord(ev, cp);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev, 0);
+      if (e != cudaSuccess) ps = PWP_ECUDA;
+      cudaEventDestroy(ev);
+      cudaEventDestroy(ev_w);
+      cudaStreamDestroy(cp);
+      return ps;
+    }
+  }
+  if (ps == PWP_OK) {
+    e = cudaMemcpyAsync(W_out_host, W_out_dev, (size_t)c * b * sizeof(float), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(mask_out_host, mask_dev, (size_t)c * b, cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) ps = PWP_ECUDA;
+  }
+  if (ev) cudaEventDestroy(ev);
+  if (ev_w) cudaEventDestroy(ev_w);
+  cudaStreamDestroy(cp);
+  return ps;
+}
+
 pwp_status pwp_pack_24(const float* W_hat, const uint8_t* mask, int32_t c, int32_t b, uint16_t* values,
                        uint32_t* meta, pwp_stats* st, void* stream) {
   if (!W_hat || !mask || !values || !meta || !st || c < 1 || b < 4 || b > 16384 || (b % 4) != 0 ||

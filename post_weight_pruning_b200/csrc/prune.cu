@@ -609,6 +609,26 @@ static void prune_solve(PruneRun& R, int t, long long* nl) {
 cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c, int b, float* H,
                          float* Wout, uint8_t* mask, void* ws, pwp_stats* st, cudaStream_t s,
                          bool stats_ready) {
+  return launch_prune_out(cfg, W, wtype, c, b, H, Wout, mask, ws, st, s, stats_ready, nullptr);
+}
+
+// Block t-1's columns of W-hat and of the mask are final once pass t has run (it applies
+// that block's update to columns >= jp and zeroes its removals; later passes start at
+// column j_t): with `ho`, they go back to the host on its copy stream right then.
+static void copy_block_out(const PruneRun& R, int tb, const HostOut* ho) {
+  if (!ho || tb < 0 || tb >= R.nblk) return;
+  const int jq = tb * R.B, w = min(R.B, R.b - jq);
+  cudaEventRecord(ho->ev, R.s);
+  cudaStreamWaitEvent(ho->copy, ho->ev, 0);
+  cudaMemcpy2DAsync(ho->W_host + jq, (size_t)R.b * sizeof(float), R.Wout + jq, (size_t)R.b * sizeof(float),
+                    (size_t)w * sizeof(float), (size_t)R.c, cudaMemcpyDeviceToHost, ho->copy);
+  cudaMemcpy2DAsync(ho->mask_host + jq, (size_t)R.b, R.mask + jq, (size_t)R.b, (size_t)w, (size_t)R.c,
+                    cudaMemcpyDeviceToHost, ho->copy);
+}
+
+cudaError_t launch_prune_out(const pwp_config* cfg, const void* W, int wtype, int c, int b, float* H,
+                             float* Wout, uint8_t* mask, void* ws, pwp_stats* st, cudaStream_t s,
+                             bool stats_ready, const HostOut* ho) {
   if (cfg->method == PWP_WANDA || cfg->method == PWP_MAGNITUDE)
     return launch_no_update(cfg, W, wtype, c, b, cfg->method == PWP_WANDA ? H : nullptr, nullptr, 0, 0, Wout,
                             mask, ws, st, stats_ready, s);
@@ -631,6 +651,7 @@ cudaError_t launch_prune(const pwp_config* cfg, const void* W, int wtype, int c,
     // threshold, when predicted); select_finish does the rest
     e = prune_pass(R, t, pick_args(R, t, true), &nl);
     if (e != cudaSuccess) return e;
+    copy_block_out(R, t - 1, ho);
     if (t == R.nblk) break;
     if (R.score != kNoScore) {
       const int j = t * R.B, j1 = min(b, j + R.B);

@@ -300,6 +300,19 @@ cudaError_t launch_prune_alpha(const pwp_config* cfg, const void* W, int wtype, 
 cudaError_t launch_pack24(const float* What, const uint8_t* mask, int c, int b, uint16_t* values, uint32_t* meta,
                           pwp_stats* st, cudaStream_t s);
 
+// The prune's block loop with its finished column blocks of W-hat and the mask copied to
+// pinned host memory as it goes (prune.cu; the host entry point in api.cu): each block's
+// copies wait for an event recorded on the prune's stream and run on `copy`.
+struct HostOut {
+  float* W_host;
+  uint8_t* mask_host;
+  cudaStream_t copy;
+  cudaEvent_t ev;
+};
+cudaError_t launch_prune_out(const pwp_config* cfg, const void* W, int wtype, int c, int b, float* H,
+                             float* Wout, uint8_t* mask, void* ws, pwp_stats* st, cudaStream_t s,
+                             bool stats_ready, const HostOut* ho);
+
 // per-row work of one block (solve.cu); returns the number of kernels launched
 // (both also clear the level-2 histograms the block's selection used)
 int launch_thanos_solve(bool nm, const float* W, int c, int b, int j, int B, const float* Kt,

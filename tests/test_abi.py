@@ -75,6 +75,14 @@ def test_argument_errors_return_before_any_launch():
     assert L.pwp_damp_factor(fake, 16, 0.01, fake, None, 0, fake, None) == 3
     assert L.pwp_prune_layer_x(ctypes.byref(cfg), fake, 0, 16, 16, fake, 0, -1, fake, fake, fake, fake, n,
                                fake, None) == 1
+    # the host entry point: null host buffers, a negative n, then a short workspace
+    a = [fake] * 8
+    assert L.pwp_prune_layer_host(ctypes.byref(cfg), None, 0, 16, 16, fake, 0, 10, *a[:7], fake, n, fake,
+                                  None) == 1
+    assert L.pwp_prune_layer_host(ctypes.byref(cfg), fake, 0, 16, 16, fake, 0, -1, *a[:7], fake, n, fake,
+                                  None) == 1
+    assert L.pwp_prune_layer_host(ctypes.byref(cfg), fake, 0, 16, 16, fake, 0, 10, *a[:7], fake, 10, fake,
+                                  None) == 3
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
