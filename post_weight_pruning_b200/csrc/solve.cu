@@ -84,11 +84,12 @@ __device__ __forceinline__ void panel_gemm(float (&acc)[2][8], const float* cons
 // lane and pass (lane l: rows jp+l+64p and jp+l+64p+32): each takes the contributions of
 // the columns before jp (float4 dot products with the eight panel rows, which every lane
 // reads as broadcasts), the panel's 8x8 diagonal block is staged in D and factored by every
-// lane alike (no shuffles; the pivots are uniform across the warp), and each row finishes
-// its eight panel entries by forward substitution.  A packed row i holds columns up to
-// 4*(i/4)+3, so rows jp..jp+3 of a panel store only its first four columns; columns beyond
-// i inside a row's padding are never read.  Reciprocal pivots go to idg for the back
-// substitution.  Returns false on a non-positive pivot (uniform).
+// lane alike into registers (no shuffles; the pivots are uniform across the warp), and each
+// row finishes its eight panel entries by forward substitution against those registers.  A
+// packed row i holds columns up to 4*(i/4)+3, so rows jp..jp+3 of a panel store only its
+// first four columns; columns beyond i inside a row's padding are never read.  Reciprocal
+// pivots go to idg for the back substitution.  Returns false on a non-positive pivot
+// (uniform).
 template <bool SMALL>
 __device__ bool chol_solve(const Rows<SMALL> R, float* __restrict__ y, float* __restrict__ idg,
                            float* __restrict__ D, int s, int lane) {
@@ -125,52 +126,41 @@ __device__ bool chol_solve(const Rows<SMALL> R, float* __restrict__ y, float* __
           *reinterpret_cast<float4*>(D + 8 * lane + 4) = make_float4(acc[0][4], acc[0][5], acc[0][6], acc[0][7]);
         }
         __syncwarp();
-        // factored in place: Ld's lower triangle becomes the block's L (its diagonal is
-        // not used: the reciprocal pivots il stand in for it)
-        float Ld[8][8];
-        float il[8];
+      }
+      // factored by every lane (a later pass of the panel factors it again): Ld's strict
+      // lower triangle becomes the block's L, il its reciprocal pivots (rows past pw are
+      // padding and feed only padding columns)
+      float Ld[8][8];
+      float il[8];
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-          const float4 lo = *reinterpret_cast<const float4*>(D + 8 * r);
-          const float4 hi = *reinterpret_cast<const float4*>(D + 8 * r + 4);
-          const float v[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+      for (int r = 0; r < 8; ++r) {
+        const float4 lo = *reinterpret_cast<const float4*>(D + 8 * r);
+        const float4 hi = *reinterpret_cast<const float4*>(D + 8 * r + 4);
+        const float v[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
 #pragma unroll
-          for (int c = 0; c <= r; ++c) Ld[r][c] = v[c];
+        for (int c = 0; c <= r; ++c) Ld[r][c] = v[c];
+      }
+      bool ok = true;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        il[c] = 1.f;
+        if (c < pw) {
+          const float d = Ld[c][c];
+          ok = ok && (d > 0.f);
+          il[c] = rsqrtf(d);
+#pragma unroll
+          for (int r = c + 1; r < 8; ++r) Ld[r][c] *= il[c];
+#pragma unroll
+          for (int r = c + 1; r < 8; ++r)
+#pragma unroll
+            for (int c2 = c + 1; c2 <= r; ++c2) Ld[r][c2] = fmaf(-Ld[r][c], Ld[c2][c], Ld[r][c2]);
         }
-        bool ok = true;
+      }
+      if (!ok) return false;   // the same pivots in every lane
+      if (pass == 0 && lane == 0) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          il[c] = 1.f;
-          if (c < pw) {
-            const float d = Ld[c][c];
-            ok = ok && (d > 0.f);
-            il[c] = rsqrtf(d);
-#pragma unroll
-            for (int r = c + 1; r < 8; ++r) Ld[r][c] *= il[c];
-#pragma unroll
-            for (int r = c + 1; r < 8; ++r)
-#pragma unroll
-              for (int c2 = c + 1; c2 <= r; ++c2) Ld[r][c2] = fmaf(-Ld[r][c], Ld[c2][c], Ld[r][c2]);
-          }
-        }
-        if (!ok) return false;   // the same pivots in every lane
-        // back to D for the forward substitutions: L's strict lower triangle, and the
-        // reciprocal pivots on the diagonal (every lane holds the same values)
-        __syncwarp();
-        if (lane == 0) {
-#pragma unroll
-          for (int r = 0; r < 8; ++r) {
-            float v[8];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) v[c] = c < r ? Ld[r][c] : (c == r ? il[r] : 0.f);
-            *reinterpret_cast<float4*>(D + 8 * r) = make_float4(v[0], v[1], v[2], v[3]);
-            *reinterpret_cast<float4*>(D + 8 * r + 4) = make_float4(v[4], v[5], v[6], v[7]);
-          }
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            if (c < pw) idg[jp + c] = il[c];
-        }
-        __syncwarp();
+        for (int c = 0; c < 8; ++c)
+          if (c < pw) idg[jp + c] = il[c];
       }
       // forward substitution of each row's panel entries; for a diagonal row i = jp + r
       // this gives L[i][jp..i] with the pivot's square root at column i
@@ -182,13 +172,10 @@ __device__ bool chol_solve(const Rows<SMALL> R, float* __restrict__ y, float* __
         float x[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          const float4 lo = *reinterpret_cast<const float4*>(D + 8 * c);
-          const float4 hi = *reinterpret_cast<const float4*>(D + 8 * c + 4);
-          const float l[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
           float v = acc[q][c];
 #pragma unroll
-          for (int c2 = 0; c2 < c; ++c2) v = fmaf(-x[c2], l[c2], v);
-          x[c] = v * l[c];
+          for (int c2 = 0; c2 < c; ++c2) v = fmaf(-x[c2], Ld[c][c2], v);
+          x[c] = v * il[c];
         }
         float* r = const_cast<float*>(rp[q]);
         *reinterpret_cast<float4*>(r + jp) = make_float4(x[0], x[1], x[2], x[3]);
@@ -197,87 +184,81 @@ __device__ bool chol_solve(const Rows<SMALL> R, float* __restrict__ y, float* __
     }
     __syncwarp();
   }
-  // back substitution L^T z = y, four rows at a time from the bottom: the 4x4 corner
-  // is solved redundantly by every lane, then the rows above drop its contribution
-  for (int a0 = (s - 1) & ~3; a0 >= 0; a0 -= 4) {
-    const int pw = min(4, s - a0);
-    const float* rr[4];
+  // back substitution L^T z = y from the bottom, one unknown at a time with y held in
+  // registers (lane l: y[l + 32q]): the owner of unknown i forms z_i = y_i / L_ii and
+  // broadcasts it, and every lane drops z_i L[i][t] from its y_t, t < i (row i of the
+  // packed factor, read along its length)
+  constexpr int CH = SMALL ? (kNS + 31) / 32 : (kCap + 31) / 32;
+  float yv[CH], dv[CH];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) rr[c] = R.row(a0 + (c < pw ? c : pw - 1));
-    float z[4];
-#pragma unroll
-    for (int c = 3; c >= 0; --c) {
-      z[c] = 0.f;
-      if (c < pw) {
-        float v = y[a0 + c];
-#pragma unroll
-        for (int c2 = c + 1; c2 < 4; ++c2)
-          if (c2 < pw) v = fmaf(-rr[c2][a0 + c], z[c2], v);
-        z[c] = v * idg[a0 + c];
-      }
-    }
-    __syncwarp();
-    for (int t = lane; t < a0; t += 32) {
-      float v = y[t];
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        if (c < pw) v = fmaf(-rr[c][t], z[c], v);
-      y[t] = v;
-    }
-    if (lane < pw) y[a0 + lane] = z[lane];
-    __syncwarp();
+  for (int q = 0; q < CH; ++q) {
+    const int t = lane + 32 * q;
+    yv[q] = t < s ? y[t] : 0.f;
+    dv[q] = t < s ? idg[t] : 0.f;
   }
+#pragma unroll
+  for (int qc = CH - 1; qc >= 0; --qc) {
+    if (32 * qc >= s) continue;
+#pragma unroll 4
+    for (int i = min(s, 32 * qc + 32) - 1; i >= 32 * qc; --i) {
+      const int src = i & 31;
+      const float zi = __shfl_sync(0xffffffffu, yv[qc] * dv[qc], src);
+      const float* Li = R.row(i);
+#pragma unroll
+      for (int q = 0; q <= qc; ++q) {
+        const int t = lane + 32 * q;
+        if (q < qc || t < i) yv[q] = fmaf(-Li[t], zi, yv[q]);
+      }
+      if (lane == src) yv[qc] = zi;
+    }
+  }
+  __syncwarp();
+#pragma unroll
+  for (int q = 0; q < CH; ++q) {
+    const int t = lane + 32 * q;
+    if (t < s) y[t] = yv[q];
+  }
+  __syncwarp();
   return true;
 }
 
-// R-hat = K[Q, Q], lower triangle, into the packed rows: row a is K row q_a, loaded whole
-// (lane l holds columns 4l..4l+3) and staged in the warp's index slots (the indices are
-// held in registers by then), from which entry (a, cc) is read at column q_cc.
+// R-hat = K[Q, Q], lower triangle, into the packed rows: entry (a, cc), cc <= a, is
+// K[q_a, q_cc], loaded straight from K's row q_a (lane l takes columns q_l, q_{l+32}, ...;
+// one load instruction stays inside one 512-byte row), eight rows' loads in flight before
+// their stores.
 template <bool SMALL>
-__device__ void gather_rhat(const Rows<SMALL> R, const float* __restrict__ Kt, int* __restrict__ Qidx, int s,
-                            int B, int nJ, int lane) {
-  constexpr int CH = (kCap + 31) / 32;
+__device__ void gather_rhat(const Rows<SMALL> R, const float* __restrict__ Kt, const int* __restrict__ Qidx, int s,
+                            int B, int lane) {
+  constexpr int CH = SMALL ? (kNS + 31) / 32 : (kCap + 31) / 32;
+  constexpr int G = 8;
   int qv[CH];
 #pragma unroll
   for (int ch = 0; ch < CH; ++ch) qv[ch] = (lane + 32 * ch < s) ? Qidx[lane + 32 * ch] : 0;
-  __syncwarp();   // the index slots become the staging row
-  float* stage = reinterpret_cast<float*>(Qidx);
-  const bool vec = (B & 3) == 0;
-  const int c4 = 4 * lane;
-  for (int a0 = 0; a0 < s; a0 += 4) {
-    float4 kv[4];
+  for (int a0 = 0; a0 < s; a0 += G) {
+    const int hc = a0 >> 5;   // the chunk of q that holds q_a for every row of the group
+    float v[G][CH];
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int a = a0 + r < s ? a0 + r : 0;
+    for (int r = 0; r < G; ++r) {
+      const int a = a0 + r;
       int qa = 0;
 #pragma unroll
       for (int ch = 0; ch < CH; ++ch)
-        if ((a >> 5) == ch) qa = __shfl_sync(0xffffffffu, qv[ch], a & 31);
+        if (hc == ch) qa = __shfl_sync(0xffffffffu, qv[ch], a & 31);
       const float* krow = Kt + (size_t)qa * B;
-      if (vec && c4 + 3 < nJ) {
-        kv[r] = __ldg(reinterpret_cast<const float4*>(krow + c4));
-      } else {
-        kv[r].x = c4 < nJ ? __ldg(krow + c4) : 0.f;
-        kv[r].y = c4 + 1 < nJ ? __ldg(krow + c4 + 1) : 0.f;
-        kv[r].z = c4 + 2 < nJ ? __ldg(krow + c4 + 2) : 0.f;
-        kv[r].w = c4 + 3 < nJ ? __ldg(krow + c4 + 3) : 0.f;
+#pragma unroll
+      for (int ch = 0; ch < CH; ++ch) {
+        v[r][ch] = 0.f;
+        if (ch <= hc && a < s && lane + 32 * ch <= a) v[r][ch] = __ldg(krow + qv[ch]);
       }
     }
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
+    for (int r = 0; r < G; ++r) {
       const int a = a0 + r;
       if (a >= s) break;
-      *reinterpret_cast<float4*>(stage + c4) = kv[r];
-      __syncwarp();
       float* row = R.row(a);
 #pragma unroll
-      for (int ch = 0; ch < CH; ++ch) {
-        if (32 * ch > a) break;
-        const int cc = lane + 32 * ch;
-        const float v = stage[qv[ch]];
-        if (cc <= a) row[cc] = v;
-      }
-      __syncwarp();   // the staging row is rewritten next
+      for (int ch = 0; ch < CH; ++ch)
+        if (ch <= hc && lane + 32 * ch <= a) row[lane + 32 * ch] = v[r][ch];
     }
   }
   __syncwarp();
@@ -362,11 +343,11 @@ __global__ void __launch_bounds__(kSolveWarps * 32, 2) thanos_solve_kernel(const
       // after the gather the selected indices are spent: their slots hold 1 / L_ii
       if (s <= kNS) {
         const Rows<true> R{L, nullptr};
-        gather_rhat<true>(R, Kt, Qidx, s, B, nJ, lane);
+        gather_rhat<true>(R, Kt, Qidx, s, B, lane);
         ok = chol_solve<true>(R, y, reinterpret_cast<float*>(Qidx), D, s, lane);
       } else {
         const Rows<false> R{L, G};
-        gather_rhat<false>(R, Kt, Qidx, s, B, nJ, lane);
+        gather_rhat<false>(R, Kt, Qidx, s, B, lane);
         ok = chol_solve<false>(R, y, reinterpret_cast<float*>(Qidx), D, s, lane);
       }
       if (!ok && lane == 0) set_error(st, PWP_ENOTSPD, kSiteSolve);
