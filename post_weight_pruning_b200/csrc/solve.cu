@@ -46,11 +46,21 @@ template <bool SMALL>
 struct Rows {
   float* L;   // shared, rows < kNS
   float* G;   // global, rows >= kNS
-  __device__ __forceinline__ float* row(int i) const {
-    if (SMALL) return L + poff(i);
-    return i < kNS ? L + poff(i) : G + (poff(i) - poff(kNS));
+  __device__ __forceinline__ float* row(int i) const { return at(poff(i)); }
+  // the row at packed offset off (row i + 1 starts 4 * (i / 4 + 1) floats after row i)
+  __device__ __forceinline__ float* at(int off) const {
+    if (SMALL) return L + off;
+    return off < kL ? L + off : G + (off - kL);
   }
 };
+
+// Four bytes global -> shared without a register stop (completion: cp_async_wait_all)
+__device__ __forceinline__ void cp_async4(float* sdst, const float* gsrc) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"((unsigned int)__cvta_generic_to_shared(sdst)),
+               "l"(gsrc)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ float dot4(float4 a, float4 b, float acc) {
   acc = fmaf(-a.x, b.x, acc);
@@ -196,6 +206,7 @@ __device__ bool chol_solve(const Rows<SMALL> R, float* __restrict__ y, float* __
     yv[q] = t < s ? y[t] : 0.f;
     dv[q] = t < s ? idg[t] : 0.f;
   }
+  int off = poff(s - 1);
 #pragma unroll
   for (int qc = CH - 1; qc >= 0; --qc) {
     if (32 * qc >= s) continue;
@@ -203,7 +214,8 @@ __device__ bool chol_solve(const Rows<SMALL> R, float* __restrict__ y, float* __
     for (int i = min(s, 32 * qc + 32) - 1; i >= 32 * qc; --i) {
       const int src = i & 31;
       const float zi = __shfl_sync(0xffffffffu, yv[qc] * dv[qc], src);
-      const float* Li = R.row(i);
+      const float* Li = R.at(off);
+      off -= 4 * ((i - 1) >> 2) + 4;   // row i - 1 (unused past row 0)
 #pragma unroll
       for (int q = 0; q <= qc; ++q) {
         const int t = lane + 32 * q;
@@ -223,44 +235,39 @@ __device__ bool chol_solve(const Rows<SMALL> R, float* __restrict__ y, float* __
 }
 
 // R-hat = K[Q, Q], lower triangle, into the packed rows: entry (a, cc), cc <= a, is
-// K[q_a, q_cc], loaded straight from K's row q_a (lane l takes columns q_l, q_{l+32}, ...;
-// one load instruction stays inside one 512-byte row), eight rows' loads in flight before
-// their stores.
+// K[q_a, q_cc], copied straight from K's row q_a (lane l takes columns q_l, q_{l+32}, ...;
+// one copy instruction stays inside one 512-byte row) by asynchronous copies into shared
+// memory, all of them in flight before one wait (rows past the shared ones, on the
+// general path, go through registers).
 template <bool SMALL>
 __device__ void gather_rhat(const Rows<SMALL> R, const float* __restrict__ Kt, const int* __restrict__ Qidx, int s,
                             int B, int lane) {
   constexpr int CH = SMALL ? (kNS + 31) / 32 : (kCap + 31) / 32;
-  constexpr int G = 8;
   int qv[CH];
 #pragma unroll
   for (int ch = 0; ch < CH; ++ch) qv[ch] = (lane + 32 * ch < s) ? Qidx[lane + 32 * ch] : 0;
-  for (int a0 = 0; a0 < s; a0 += G) {
-    const int hc = a0 >> 5;   // the chunk of q that holds q_a for every row of the group
-    float v[G][CH];
+  int off = 0;
+#pragma unroll 4
+  for (int a = 0; a < s; ++a) {
+    const int hc = a >> 5;   // uniform
+    int qsrc = qv[0];
 #pragma unroll
-    for (int r = 0; r < G; ++r) {
-      const int a = a0 + r;
-      int qa = 0;
+    for (int ch = 1; ch < CH; ++ch)
+      if (hc == ch) qsrc = qv[ch];
+    const int qa = __shfl_sync(0xffffffffu, qsrc, a & 31);
+    const float* krow = Kt + (size_t)qa * B;
+    float* row = R.at(off);
+    const bool shared_row = SMALL || off < kL;
 #pragma unroll
-      for (int ch = 0; ch < CH; ++ch)
-        if (hc == ch) qa = __shfl_sync(0xffffffffu, qv[ch], a & 31);
-      const float* krow = Kt + (size_t)qa * B;
-#pragma unroll
-      for (int ch = 0; ch < CH; ++ch) {
-        v[r][ch] = 0.f;
-        if (ch <= hc && a < s && lane + 32 * ch <= a) v[r][ch] = __ldg(krow + qv[ch]);
+    for (int ch = 0; ch < CH; ++ch) {
+      if (ch <= hc && lane + 32 * ch <= a) {
+        if (shared_row) cp_async4(row + lane + 32 * ch, krow + qv[ch]);
+        else row[lane + 32 * ch] = __ldg(krow + qv[ch]);
       }
     }
-#pragma unroll
-    for (int r = 0; r < G; ++r) {
-      const int a = a0 + r;
-      if (a >= s) break;
-      float* row = R.row(a);
-#pragma unroll
-      for (int ch = 0; ch < CH; ++ch)
-        if (ch <= hc && lane + 32 * ch <= a) row[lane + 32 * ch] = v[r][ch];
-    }
+    off += 4 * ((a >> 2) + 1);
   }
+  cp_async_wait_all();
   __syncwarp();
 }
 
