@@ -93,21 +93,25 @@ __device__ __forceinline__ void panel_gemm(float (&acc)[2][8], const float* cons
 // y[0..s) = z.  Per panel [jp, jp+8) the rows i in [jp, s] go over the lanes, two rows per
 // lane and pass (lane l: rows jp+l+64p and jp+l+64p+32): each takes the contributions of
 // the columns before jp (float4 dot products with the eight panel rows, which every lane
-// reads as broadcasts), the panel's 8x8 diagonal block is staged in D and factored by every
-// lane alike into registers (no shuffles; the pivots are uniform across the warp), and each
-// row finishes its eight panel entries by forward substitution against those registers.  A
-// packed row i holds columns up to 4*(i/4)+3, so rows jp..jp+3 of a panel store only its
-// first four columns; columns beyond i inside a row's padding are never read.  Reciprocal
-// pivots go to idg for the back substitution.  Returns false on a non-positive pivot
-// (uniform).
+// reads as broadcasts), then finishes its eight panel entries column by column.  In the
+// first pass the panel's diagonal rows are slot 0 of lanes 0..7: at column c lane c's
+// entries so far and its pivot reach every lane by shuffles, so the diagonal block is
+// factored and every row's panel entries solved in one sweep; a later pass reads the
+// stored diagonal rows and reciprocal pivots instead.  A packed row i holds columns up to
+// 4*(i/4)+3, so rows jp..jp+3 of a panel store only its first four columns; columns
+// beyond i inside a row's padding are never read.  Reciprocal pivots go to idg for the
+// back substitution.  Returns false on a non-positive pivot (uniform).
 template <bool SMALL>
 __device__ bool chol_solve(const Rows<SMALL> R, float* __restrict__ y, float* __restrict__ idg,
                            float* __restrict__ D, int s, int lane) {
+  (void)D;
+  int pan = 0;   // packed offset of row jp
   for (int jp = 0; jp < s; jp += 8) {
     const int pw = min(8, s - jp);
+    // row jp + c starts c * (jp + 4) + 4 * max(c - 4, 0) floats after row jp
     const float* pr[8];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) pr[c] = R.row(jp + (c < pw ? c : 0));   // padding columns: any valid row
+    for (int c = 0; c < 8; ++c) pr[c] = R.at(pan + (c < pw ? c * (jp + 4) + (c > 4 ? 4 * (c - 4) : 0) : 0));
     for (int pass = 0; jp + 64 * pass <= s; ++pass) {
       const bool two = jp + 64 * pass + 32 <= s;   // uniform: some lane has a second row
       int ii[2];
@@ -128,71 +132,63 @@ __device__ bool chol_solve(const Rows<SMALL> R, float* __restrict__ y, float* __
       }
       if (two) panel_gemm<2>(acc, rp, pr, jp);
       else panel_gemm<1>(acc, rp, pr, jp);
+      float x[2][8];
       if (pass == 0) {
-        // the diagonal block: rows jp..jp+pw-1 are slot 0 of lanes 0..pw-1
-        __syncwarp();
-        if (lane < pw) {
-          *reinterpret_cast<float4*>(D + 8 * lane) = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
-          *reinterpret_cast<float4*>(D + 8 * lane + 4) = make_float4(acc[0][4], acc[0][5], acc[0][6], acc[0][7]);
+        bool ok = true;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          if (c < pw) {   // uniform
+            float lc[8];
+#pragma unroll
+            for (int c2 = 0; c2 < c; ++c2) lc[c2] = __shfl_sync(0xffffffffu, x[0][c2], c);
+            float v[2];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              v[q] = acc[q][c];
+#pragma unroll
+              for (int c2 = 0; c2 < c; ++c2) v[q] = fmaf(-x[q][c2], lc[c2], v[q]);
+            }
+            const float d = __shfl_sync(0xffffffffu, v[0], c);
+            ok = ok && (d > 0.f);
+            const float il = rsqrtf(d);
+            if (lane == 0) idg[jp + c] = il;
+#pragma unroll
+            for (int q = 0; q < 2; ++q) x[q][c] = v[q] * il;
+          } else {
+            x[0][c] = 0.f;
+            x[1][c] = 0.f;
+          }
         }
-        __syncwarp();
-      }
-      // factored by every lane (a later pass of the panel factors it again): Ld's strict
-      // lower triangle becomes the block's L, il its reciprocal pivots (rows past pw are
-      // padding and feed only padding columns)
-      float Ld[8][8];
-      float il[8];
+        if (!ok) return false;   // the same pivots in every lane
+      } else {
+        // the diagonal rows were stored by the first pass
+        float il[8];
 #pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        const float4 lo = *reinterpret_cast<const float4*>(D + 8 * r);
-        const float4 hi = *reinterpret_cast<const float4*>(D + 8 * r + 4);
-        const float v[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+        for (int c = 0; c < 8; ++c) il[c] = c < pw ? idg[jp + c] : 1.f;
 #pragma unroll
-        for (int c = 0; c <= r; ++c) Ld[r][c] = v[c];
-      }
-      bool ok = true;
+        for (int q = 0; q < 2; ++q) {
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        il[c] = 1.f;
-        if (c < pw) {
-          const float d = Ld[c][c];
-          ok = ok && (d > 0.f);
-          il[c] = rsqrtf(d);
+          for (int c = 0; c < 8; ++c) {
+            float v = acc[q][c];
 #pragma unroll
-          for (int r = c + 1; r < 8; ++r) Ld[r][c] *= il[c];
-#pragma unroll
-          for (int r = c + 1; r < 8; ++r)
-#pragma unroll
-            for (int c2 = c + 1; c2 <= r; ++c2) Ld[r][c2] = fmaf(-Ld[r][c], Ld[c2][c], Ld[r][c2]);
+            for (int c2 = 0; c2 < c; ++c2) v = fmaf(-x[q][c2], pr[c][jp + c2], v);
+            x[q][c] = v * il[c];
+          }
         }
       }
-      if (!ok) return false;   // the same pivots in every lane
-      if (pass == 0 && lane == 0) {
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          if (c < pw) idg[jp + c] = il[c];
-      }
-      // forward substitution of each row's panel entries; for a diagonal row i = jp + r
-      // this gives L[i][jp..i] with the pivot's square root at column i
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
         if (q == 1 && !two) break;
         const int i = ii[q];
         if (i > s) continue;
-        float x[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          float v = acc[q][c];
-#pragma unroll
-          for (int c2 = 0; c2 < c; ++c2) v = fmaf(-x[c2], Ld[c][c2], v);
-          x[c] = v * il[c];
-        }
         float* r = const_cast<float*>(rp[q]);
-        *reinterpret_cast<float4*>(r + jp) = make_float4(x[0], x[1], x[2], x[3]);
-        if (i >= jp + 4 || i >= s) *reinterpret_cast<float4*>(r + jp + 4) = make_float4(x[4], x[5], x[6], x[7]);
+        *reinterpret_cast<float4*>(r + jp) = make_float4(x[q][0], x[q][1], x[q][2], x[q][3]);
+        if (i >= jp + 4 || i >= s)
+          *reinterpret_cast<float4*>(r + jp + 4) = make_float4(x[q][4], x[q][5], x[q][6], x[q][7]);
       }
+      __syncwarp();   // a later pass reads the stored diagonal rows
     }
-    __syncwarp();
+    pan += 8 * jp + 48;   // rows jp .. jp+7: 4 * (jp/4 + 1) floats each, +4 for the second four
   }
   // back substitution L^T z = y from the bottom, one unknown at a time with y held in
   // registers (lane l: y[l + 32q]): the owner of unknown i forms z_i = y_i / L_ii and
