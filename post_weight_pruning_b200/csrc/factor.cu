@@ -27,7 +27,7 @@ namespace pwp {
 namespace {
 
 constexpr int NB = kFactorNB;  // 64
-constexpr int kDiagThreads = 512;
+constexpr int kDiagThreads = 256;
 
 __global__ void __launch_bounds__(1024) damp_kernel(float* __restrict__ H, int b, float damp,
                                                     float* __restrict__ g_diag, pwp_stats* st) {
@@ -58,11 +58,11 @@ __global__ void __launch_bounds__(1024) damp_kernel(float* __restrict__ H, int b
   for (int q = threadIdx.x; q < b; q += blockDim.x) H[(long long)q * b + q] += lam;
 }
 
-// Cholesky and inverse of an 8 x 8 SPD block in registers (lower triangles; compile-time
-// indices throughout): L L^T = D, X = L^-1.  False on a non-positive pivot.
-__device__ __forceinline__ bool chol_inv8(float (&L)[8][8], float (&X)[8][8]) {
+// Cholesky of an 8 x 8 SPD block in registers (lower triangle; compile-time indices
+// throughout): L L^T = D, with L's diagonal the pivots' square roots and il their
+// reciprocals.  False on a non-positive or non-finite pivot.
+__device__ __forceinline__ bool chol8(float (&L)[8][8], float (&il)[8]) {
   bool ok = true;
-  float il[8];
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
     const float piv = L[c][c];
@@ -76,123 +76,149 @@ __device__ __forceinline__ bool chol_inv8(float (&L)[8][8], float (&X)[8][8]) {
 #pragma unroll
       for (int c2 = c + 1; c2 <= r; ++c2) L[r][c2] = fmaf(-L[r][c], L[c2][c], L[r][c2]);
   }
-#pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    X[r][r] = il[r];
-#pragma unroll
-    for (int c = 0; c < r; ++c) {
-      float acc = 0.f;
-#pragma unroll
-      for (int t = c; t < r; ++t) acc = fmaf(L[r][t], X[t][c], acc);
-      X[r][c] = -il[r] * acc;
-    }
-  }
   return ok;
 }
 
 // Factor the nb x nb diagonal block (nb <= 64) held in A (symmetric; the upper triangle
-// is read) as A = V V^T with V upper triangular, and invert V.  At least 64 threads (the
-// first 64 take each step's 8x8 block; every other loop is strided by the block size).
-// Working on the reversed matrix P = J A J (J the reversal; P[r][s] = A[63-r][63-s], so
-// P's lower triangle is A's upper one and the work happens in place), this is the
-// ordinary Cholesky P = L L^T from the top-left, with V = J L J and V^-1 = J X J for
-// X = L^-1.  Right-looking in 8-column steps, every step two barriers apart:
-//   the step's 8 x 8 diagonal block is factored and inverted in registers (Ld, Xd) by
-//   each of the first 64 threads alike; thread r < 56 - k0 forms row k0+8+r of the panel,
-//   L[i, blk] = P[i, blk] Xd^T; thread t < k0 brings column t of the block's rows of X up
-//   to date, X[blk, t] := Xd X[blk, t] (those rows already carry the earlier steps'
-//   eliminations; their own columns become Xd);
-//   then all threads update the trailing part, P[i][j] -= L[i, blk] L[j, blk], and
-//   eliminate the block's rows from X's rows below it, X[i][t] -= L[i, blk] X[blk, t].
-// Rows and columns beyond nb (A indices >= nb) are an identity pad.  On return A's upper
-// triangle holds V and Wi holds V^-1 (upper, zero below).  Returns false on a
-// non-positive pivot (recorded in st).
+// is read) as A = V V^T with V upper triangular, and invert V.  256 threads.  Working on
+// the reversed matrix P = J A J (J the reversal; P[r][c] = A[63-r][63-c], so P's lower
+// triangle is A's upper one and the work happens in place), this is the ordinary
+// Cholesky P = L L^T from the top-left, with V = J L J and V^-1 = J X J for X = L^-1.
+// Right-looking in 8-column steps, with X built alongside by forward elimination from
+// X = I.  Per step k (columns blk = [8k, 8k+8), rows below from r0 = 8k+8):
+//   (b) threads 0..63: thread r < 56-8k forms row r0+r of the panel, L[i, blk] =
+//       P[i, blk] L_kk^-T (forward substitution with the factored diagonal block), the
+//       others bring column t < r0 of the block's rows of X up to date, X[blk, t] :=
+//       L_kk^-1 X[blk, t] (the block's own columns start as I and become L_kk^-1);
+//   (c) warp 0 applies the step to the next diagonal block and factors it (look-ahead:
+//       step k+1's 8x8 Cholesky runs under the rest of step k), while warps 1..7 update
+//       the rest of the trailing part, P[i][j] -= L[i, blk] L[j, blk], and eliminate the
+//       block's rows from X's rows below it, X[i][t] -= L[i, blk] X[blk, t], t < r0, in
+//       2x2 register tiles.
+// Two barriers per step.  On entry A's upper triangle holds the block with rows and
+// columns beyond nb (A indices >= nb) an identity pad, Wi = I and *bad = 0, visible to
+// every thread (load_diag_block).  On return A's upper triangle holds V and Wi holds V^-1
+// (upper, zero below).  Returns false on a non-positive pivot (recorded in st).
 __device__ bool factor_diag_block(float (*A)[NB + 1], float (*Wi)[NB + 1], int nb, int* bad, pwp_stats* st) {
-  constexpr int BS = 8, NBK = NB / BS;
-  const int tid = threadIdx.x;
-  auto P = [&](int r, int c) -> float& { return A[NB - 1 - r][NB - 1 - c]; };
-  auto X = [&](int r, int c) -> float& { return Wi[NB - 1 - r][NB - 1 - c]; };
-  // identity pad beyond nb (A indices >= nb) and X = 0
-  for (int idx = tid; idx < NB * NB; idx += blockDim.x) {
-    const int i = idx / NB, jc = idx % NB;
-    if (i <= jc && jc >= nb) A[i][jc] = (i == jc) ? 1.f : 0.f;
-    Wi[i][jc] = 0.f;
-  }
-  if (tid == 0) *bad = 0;
+  constexpr int BS = 8, NBK = NB / BS, LD = NB + 1;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  __shared__ float il_s[NB];
+  float* const Pe = &A[NB - 1][NB - 1];   // P(r, c) = Pe[-(r * LD + c)]
+  float* const Xe = &Wi[NB - 1][NB - 1];
+  auto P = [&](int r, int c) -> float& { return Pe[-(r * LD + c)]; };
+  auto X = [&](int r, int c) -> float& { return Xe[-(r * LD + c)]; };
+  (void)nb;
+  // warp 0: factor the diagonal block at k0 in place (every lane alike; lane 0 stores)
+  auto diag = [&](int k0) {
+    float Ld[8][8], il[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) Ld[r][c] = c <= r ? P(k0 + r, k0 + c) : 0.f;
+    const bool ok = chol8(Ld, il);
+    if (lane == 0) {
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        il_s[k0 + r] = il[r];
+#pragma unroll
+        for (int c = 0; c <= r; ++c) P(k0 + r, k0 + c) = Ld[r][c];
+      }
+      if (!ok) *bad = 1;
+    }
+  };
+  // one 2x2 tile of the trailing update of P (rows i0, i0+1; columns j0, j0+1)
+  auto ptile = [&](int i0, int j0, int k0) {
+    float c00 = P(i0, j0), c01 = P(i0, j0 + 1), c10 = P(i0 + 1, j0), c11 = P(i0 + 1, j0 + 1);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const float a0 = P(i0, k0 + c), a1 = P(i0 + 1, k0 + c), b0 = P(j0, k0 + c), b1 = P(j0 + 1, k0 + c);
+      c00 = fmaf(-a0, b0, c00);
+      c01 = fmaf(-a0, b1, c01);
+      c10 = fmaf(-a1, b0, c10);
+      c11 = fmaf(-a1, b1, c11);
+    }
+    P(i0, j0) = c00;
+    P(i0, j0 + 1) = c01;   // above the diagonal on a diagonal tile: never read
+    P(i0 + 1, j0) = c10;
+    P(i0 + 1, j0 + 1) = c11;
+  };
+  if (warp == 0) diag(0);
   __syncthreads();
 #pragma unroll 1
   for (int kb = 0; kb < NBK; ++kb) {
     const int k0 = BS * kb, r0 = k0 + BS, rest = NB - r0;
-    if (tid < 64) {
-      float Ld[8][8], Xd[8][8];
-#pragma unroll
-      for (int r = 0; r < 8; ++r)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          Ld[r][c] = c <= r ? P(k0 + r, k0 + c) : 0.f;
-          Xd[r][c] = 0.f;
-        }
-      const bool ok = chol_inv8(Ld, Xd);
-      if (!ok && tid == 0) *bad = 1;
-      if (tid < rest) {                      // panel row k0 + 8 + tid
-        const int i = r0 + tid;
-        float pr[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) pr[c] = P(i, k0 + c);
-#pragma unroll
-        for (int a = 0; a < 8; ++a) {
-          float acc = 0.f;
-#pragma unroll
-          for (int c = 0; c <= a; ++c) acc = fmaf(pr[c], Xd[a][c], acc);
-          P(i, k0 + a) = acc;
-        }
-      }
-      if (tid < k0) {                        // column tid of the block's rows of X
-        float xo[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) xo[c] = X(k0 + c, tid);
-#pragma unroll
-        for (int a = 0; a < 8; ++a) {
-          float acc = 0.f;
-#pragma unroll
-          for (int c = 0; c <= a; ++c) acc = fmaf(Xd[a][c], xo[c], acc);
-          X(k0 + a, tid) = acc;
-        }
-      }
-      if (tid == 63) {                       // the block itself
-#pragma unroll
-        for (int r = 0; r < 8; ++r)
-#pragma unroll
-          for (int c = 0; c <= r; ++c) {
-            P(k0 + r, k0 + c) = Ld[r][c];
-            X(k0 + r, k0 + c) = Xd[r][c];
-          }
-      }
-    }
-    __syncthreads();
-    if (*bad) {
+    if (*reinterpret_cast<volatile int*>(bad)) {
       if (tid == 0) set_error(st, PWP_ENOTSPD, kSiteCholDiag);
       return false;
     }
-    // trailing update of P (lower triangle of the rest x rest part) and elimination of
-    // the block's rows from the rows of X below it (columns < k0 + 8)
-    const int nP = rest * (rest + 1) / 2, nX = rest * r0;
-    for (int e = tid; e < nP + nX; e += blockDim.x) {
-      if (e < nP) {
-        int ii = (int)((sqrtf(8.f * (float)e + 1.f) - 1.f) * 0.5f);
-        if ((ii + 1) * (ii + 2) / 2 <= e) ++ii;
-        if (ii * (ii + 1) / 2 > e) --ii;
-        const int i = r0 + ii, j = r0 + (e - ii * (ii + 1) / 2);
-        float acc = P(i, j);
+    if (tid < NB) {
+      float Ld[8][8], il[8];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) acc = fmaf(-P(i, k0 + c), P(j, k0 + c), acc);
-        P(i, j) = acc;
+      for (int r = 0; r < 8; ++r) {
+        il[r] = il_s[k0 + r];
+#pragma unroll
+        for (int c = 0; c < r; ++c) Ld[r][c] = P(k0 + r, k0 + c);
+      }
+      float x[8];
+      if (tid < rest) {                      // panel row r0 + tid
+        const int i = r0 + tid;
+#pragma unroll
+        for (int a2 = 0; a2 < 8; ++a2) {
+          float v = P(i, k0 + a2);
+#pragma unroll
+          for (int c = 0; c < a2; ++c) v = fmaf(-x[c], Ld[a2][c], v);
+          x[a2] = v * il[a2];
+        }
+#pragma unroll
+        for (int a2 = 0; a2 < 8; ++a2) P(i, k0 + a2) = x[a2];
+      } else {                               // column t of the block's rows of X
+        const int t = tid - rest;
+#pragma unroll
+        for (int a2 = 0; a2 < 8; ++a2) {
+          float v = X(k0 + a2, t);
+#pragma unroll
+          for (int c = 0; c < a2; ++c) v = fmaf(-Ld[a2][c], x[c], v);
+          x[a2] = v * il[a2];
+        }
+#pragma unroll
+        for (int a2 = 0; a2 < 8; ++a2) X(k0 + a2, t) = x[a2];
+      }
+    }
+    __syncthreads();
+    if (rest > 0) {
+      const int th = r0 >> 1;   // first tile row of the trailing part
+      if (warp == 0) {
+        // the next diagonal block's ten lower 2x2 tiles, then its factorisation
+        if (lane < 10) {
+          const int ta = lane < 1 ? 0 : lane < 3 ? 1 : lane < 6 ? 2 : 3;
+          const int tb = lane - ta * (ta + 1) / 2;
+          ptile(r0 + 2 * ta, r0 + 2 * tb, k0);
+        }
+        __syncwarp();
+        diag(r0);
       } else {
-        const int e2 = e - nP, i = r0 + e2 / r0, t = e2 % r0;
-        float acc = X(i, t);
+        for (int id = tid - 32; id < 32 * 32; id += blockDim.x - 32) {
+          const int ti = id >> 5, tj = id & 31;
+          if (ti < th || (ti < th + 4 && tj >= th) || tj > ti) continue;
+          if (tj >= th) {
+            ptile(2 * ti, 2 * tj, k0);
+          } else {                           // X rows 2ti, 2ti+1 at columns 2tj, 2tj+1 < r0
+            const int i0 = 2 * ti, t0 = 2 * tj;
+            float c00 = X(i0, t0), c01 = X(i0, t0 + 1), c10 = X(i0 + 1, t0), c11 = X(i0 + 1, t0 + 1);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) acc = fmaf(-P(i, k0 + c), X(k0 + c, t), acc);
-        X(i, t) = acc;
+            for (int c = 0; c < 8; ++c) {
+              const float a0 = P(i0, k0 + c), a1 = P(i0 + 1, k0 + c), b0 = X(k0 + c, t0), b1 = X(k0 + c, t0 + 1);
+              c00 = fmaf(-a0, b0, c00);
+              c01 = fmaf(-a0, b1, c01);
+              c10 = fmaf(-a1, b0, c10);
+              c11 = fmaf(-a1, b1, c11);
+            }
+            X(i0, t0) = c00;
+            X(i0, t0 + 1) = c01;
+            X(i0 + 1, t0) = c10;
+            X(i0 + 1, t0 + 1) = c11;
+          }
+        }
       }
     }
     __syncthreads();
@@ -200,10 +226,45 @@ __device__ bool factor_diag_block(float (*A)[NB + 1], float (*Wi)[NB + 1], int n
   return true;
 }
 
+// The block at (q0, q0) of H into A (upper triangle; identity pad beyond nb), Wi = I and
+// *bad = 0, then a barrier.  256 threads: thread t owns column t % 64 and rows t / 64 + 4m,
+// its sixteen loads all in flight at once.
+__device__ __forceinline__ void load_diag_block(const float* H, int b, int q0, int nb, float (*A)[NB + 1],
+                                                float (*Wi)[NB + 1], int* bad) {
+  const int tid = threadIdx.x, sc = tid & (NB - 1), r0 = tid >> 6;
+  float v[NB * NB / 256];
+#pragma unroll
+  for (int m = 0; m < NB * NB / 256; ++m) {
+    const int r = r0 + 4 * m;
+    v[m] = (r == sc) ? 1.f : 0.f;
+    if (r <= sc && sc < nb) v[m] = H[(long long)(q0 + r) * b + q0 + sc];
+  }
+#pragma unroll
+  for (int m = 0; m < NB * NB / 256; ++m) {
+    const int r = r0 + 4 * m;
+    if (r <= sc) A[r][sc] = v[m];
+    Wi[r][sc] = (r == sc) ? 1.f : 0.f;
+  }
+  if (tid == 0) *bad = 0;
+  __syncthreads();
+}
+
+// V (A's upper triangle) back into H's block and V^-1 (upper, zero below) into Vinv,
+// 64 x 64 row-major (zero outside nb x nb).
+__device__ __forceinline__ void store_diag_block(float* H, int b, int q0, int nb, float (*A)[NB + 1],
+                                                 float (*Wi)[NB + 1], float* __restrict__ Vinv) {
+  const int tid = threadIdx.x, sc = tid & (NB - 1), r0 = tid >> 6;
+#pragma unroll
+  for (int m = 0; m < NB * NB / 256; ++m) {
+    const int r = r0 + 4 * m;
+    const bool in = r <= sc && sc < nb;
+    Vinv[r * NB + sc] = in ? Wi[r][sc] : 0.f;
+    if (in) H[(long long)(q0 + r) * b + q0 + sc] = A[r][sc];
+  }
+}
+
 // Stand-alone factorisation of the diagonal block at p0 (used for the last panel, and for
-// every panel when the trailing update runs on the tensor cores): 512 threads, so that the
-// trailing updates of its 8-column steps spread thin (the step's 8x8 factor stays on the
-// first 64 threads).
+// every panel when the trailing update runs on the tensor cores): one CTA of 256 threads.
 __global__ void __launch_bounds__(kDiagThreads) chol_diag_kernel(float* __restrict__ H, int b, int p0, int nb,
                                                         float* __restrict__ Vinv, pwp_stats* st) {
   pdl_enter();
@@ -212,17 +273,85 @@ __global__ void __launch_bounds__(kDiagThreads) chol_diag_kernel(float* __restri
   float (*Wi)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(dsm + NB * (NB + 1));
   __shared__ int bad;
   if (cta_failed(st)) return;
-  if (threadIdx.x == 0) bad = 0;
-  for (int idx = threadIdx.x; idx < nb * nb; idx += blockDim.x) {
-    int r = idx / nb, s = idx % nb;
-    if (r <= s) A[r][s] = H[(long long)(p0 + r) * b + p0 + s];
+  load_diag_block(H, b, p0, nb, A, Wi, &bad);
+  if (!factor_diag_block(A, Wi, nb, &bad, st)) return;
+  store_diag_block(H, b, p0, nb, A, Wi, Vinv);
+}
+
+// The next panel's diagonal block ahead of the trailing update that would produce it,
+// so that its factorisation runs beside that update: A = S - Vr Vr^T, with S the block
+// [q0, q0+64)^2 as it stood before this step (the panel kernel's snapshot, left in the
+// block's slot of Vinv) and Vr the panel rows q0..q0+63 that the panel kernel just formed
+// (H[q0 + r][p0 + t], t < nb); then factored and inverted as in chol_diag_kernel, V^-1
+// into the same slot.  V itself is not stored: nothing reads H's diagonal blocks before
+// they receive their inverses (put_diag_inverses_kernel), and the trailing update still
+// writes the unfactored block there.
+__global__ void __launch_bounds__(kDiagThreads) chol_diag_ahead_kernel(const float* __restrict__ H, int b,
+                                                                       int p0, int nb, float* __restrict__ Vinv,
+                                                                       pwp_stats* st) {
+  pdl_enter();
+  extern __shared__ __align__(16) float dsm[];
+  float (*A)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(dsm);
+  float (*Wi)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(dsm + NB * (NB + 1));
+  __shared__ int bad;
+  if (cta_failed(st)) return;
+  const int q0 = p0 - NB, tid = threadIdx.x, sc = tid & (NB - 1), r0 = tid >> 6;
+  {
+    // S into A's upper triangle, Vr into Wi (Wi[r][t] = Vr[r][t]): all loads in flight
+    float v[NB * NB / 256], w[NB * NB / 256];
+#pragma unroll
+    for (int m = 0; m < NB * NB / 256; ++m) {
+      const int r = r0 + 4 * m;
+      v[m] = r <= sc ? Vinv[r * NB + sc] : 0.f;
+      w[m] = sc < nb ? H[(long long)(q0 + r) * b + p0 + sc] : 0.f;
+    }
+#pragma unroll
+    for (int m = 0; m < NB * NB / 256; ++m) {
+      const int r = r0 + 4 * m;
+      if (r <= sc) A[r][sc] = v[m];
+      Wi[r][sc] = w[m];
+    }
   }
   __syncthreads();
-  if (!factor_diag_block(A, Wi, nb, &bad, st)) return;
-  for (int idx = threadIdx.x; idx < NB * NB; idx += blockDim.x) {
-    int r = idx / NB, s = idx % NB;
-    Vinv[idx] = (r < nb && s < nb && r <= s) ? Wi[r][s] : 0.f;
-    if (r < nb && s < nb && r <= s) H[(long long)(p0 + r) * b + p0 + s] = A[r][s];
+  {
+    // A[r][c] -= sum_t Vr[r][t] Vr[c][t] for r <= c: one 4 x 4 tile per thread (tiles on
+    // or above the diagonal of a 16 x 16 tile grid)
+    const int tr = tid >> 4, tc = tid & 15;
+    if (tr <= tc) {
+      float acc[4][4] = {};
+#pragma unroll 4
+      for (int t = 0; t < NB; ++t) {
+        float a[4], c4[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          a[i] = Wi[4 * tr + i][t];
+          c4[i] = Wi[4 * tc + i][t];
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], c4[j], acc[i][j]);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (4 * tr + i <= 4 * tc + j) A[4 * tr + i][4 * tc + j] -= acc[i][j];
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int m = 0; m < NB * NB / 256; ++m) {
+    const int r = r0 + 4 * m;
+    Wi[r][sc] = (r == sc) ? 1.f : 0.f;
+  }
+  if (tid == 0) bad = 0;
+  __syncthreads();
+  if (!factor_diag_block(A, Wi, NB, &bad, st)) return;
+#pragma unroll
+  for (int m = 0; m < NB * NB / 256; ++m) {
+    const int r = r0 + 4 * m;
+    Vinv[r * NB + sc] = r <= sc ? Wi[r][sc] : 0.f;
   }
 }
 
@@ -234,12 +363,35 @@ __global__ void __launch_bounds__(kDiagThreads) chol_diag_kernel(float* __restri
 __global__ void __launch_bounds__(256) chol_panel_kernel(float* __restrict__ H, int b, int p0, int nb,
                                                          const float* __restrict__ Vinv,
                                                          float* __restrict__ vs_hi, float* __restrict__ vs_lo,
-                                                         const pwp_stats* st) {
+                                                         float* __restrict__ snap, const pwp_stats* st) {
   pdl_enter();
   __shared__ float WiT[NB][NB + 1];  // WiT[t][c] = Wi[c][t]
   __shared__ float rowbuf[8][NB];
   if (cta_failed(st)) return;
-  for (int idx = threadIdx.x; idx < NB * NB; idx += blockDim.x) WiT[idx % NB][idx / NB] = Vinv[idx];
+  {
+    // WiT[t][c] = Vinv[c][t]: sixteen loads per thread in flight at once
+    float v[NB * NB / 256];
+#pragma unroll
+    for (int m = 0; m < NB * NB / 256; ++m) v[m] = Vinv[threadIdx.x + 256 * m];
+#pragma unroll
+    for (int m = 0; m < NB * NB / 256; ++m) {
+      const int idx = threadIdx.x + 256 * m;
+      WiT[idx % NB][idx / NB] = v[m];
+    }
+  }
+  if (snap != nullptr && blockIdx.x == gridDim.x - 1) {
+    // the next diagonal block [p0-64, p0)^2 as it stands before this step's trailing
+    // update (its upper triangle, 64 x 64 row-major), for chol_diag_ahead_kernel
+    const int q0 = p0 - NB, sc = threadIdx.x & (NB - 1), r0 = threadIdx.x >> 6;
+    float v[NB * NB / 256];
+#pragma unroll
+    for (int m = 0; m < NB * NB / 256; ++m) {
+      const int r = r0 + 4 * m;
+      v[m] = r <= sc ? H[(long long)(q0 + r) * b + q0 + sc] : 0.f;
+    }
+#pragma unroll
+    for (int m = 0; m < NB * NB / 256; ++m) snap[(r0 + 4 * m) * NB + sc] = v[m];
+  }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int r = blockIdx.x * 8 + warp; r < p0; r += gridDim.x * 8) {
@@ -268,36 +420,18 @@ __global__ void __launch_bounds__(256) chol_panel_kernel(float* __restrict__ H, 
   }
 }
 
-// Symmetric update of the top-left part: A[r][s] -= sum_t V[r][p0+t] V[s][p0+t] for
-// r <= s < p0, 128x128 tiles on or above the diagonal, 8x8 outputs per thread.  The CTA
-// whose tile holds the next panel's diagonal block [p0-NB, p0) then factors it (reading
-// back entries of H its other threads wrote: H is not __restrict__).
-__global__ void __launch_bounds__(256) chol_update_kernel(float* H, int b, int p0, int nb,
-                                                          float* __restrict__ Vinv_next,
-                                                          pwp_stats* st) {
+// Symmetric update of the top-left part on the CUDA cores (when the tensor-core update
+// cannot take the shape): A[r][s] -= sum_t V[r][p0+t] V[s][p0+t] for r <= s < p0,
+// 128x128 tiles on or above the diagonal, 8x8 outputs per thread.
+__global__ void __launch_bounds__(256) chol_update_kernel(float* __restrict__ H, int b, int p0, int nb,
+                                                          const pwp_stats* st) {
   pdl_enter();
   extern __shared__ __align__(16) float fsm[];
   float (*As)[128 + 4] = reinterpret_cast<float (*)[132]>(fsm);               // [NB][132], k-major
   float (*Bs)[128 + 4] = reinterpret_cast<float (*)[132]>(fsm + NB * 132);
-  __shared__ int bad;
   if (cta_failed(st)) return;
   const int nT = (p0 + 127) / 128;
-  // blockIdx 0 takes the tile holding the next panel's diagonal block, so its serial
-  // factorisation starts first and overlaps the other tiles; that tile's own slot in
-  // the upper-triangle enumeration goes to blockIdx 0's original tile.
-  const int q0 = p0 - NB;
-  int look = -1;
-  if (q0 >= 0) {
-    const int Id = q0 / 128;  // diagonal tile (Id, Id)
-    look = 0;
-    for (int i = 0; i < Id; ++i) look += nT - i;
-  }
-  int slot = blockIdx.x;
-  if (look >= 0) {
-    if (slot == 0) slot = look;
-    else if (slot == look) slot = 0;
-  }
-  int I = 0, rem = slot;
+  int I = 0, rem = blockIdx.x;
   while (rem >= nT - I) { rem -= nT - I; ++I; }
   const int J = I + rem;
   const int i0 = I * 128, j0 = J * 128;
@@ -336,23 +470,6 @@ __global__ void __launch_bounds__(256) chol_update_kernel(float* H, int b, int p
       const int s = j0 + (y < 4 ? tx * 4 + y : 64 + tx * 4 + y - 4);
       if (s < p0 && r <= s) H[(long long)r * b + s] -= acc[x][y];
     }
-  }
-  // look-ahead: factor the next panel's diagonal block if this tile holds it
-  if (q0 < 0 || I != J || q0 < i0 || q0 >= i0 + 128) return;
-  __syncthreads();  // this CTA's own writes to H are visible to its threads
-  float (*A)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(fsm);
-  float (*Wi)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(fsm + NB * (NB + 1));
-  if (threadIdx.x == 0) bad = 0;
-  for (int idx = threadIdx.x; idx < NB * NB; idx += blockDim.x) {
-    int r = idx / NB, s = idx % NB;
-    if (r <= s) A[r][s] = H[(long long)(q0 + r) * b + q0 + s];
-  }
-  __syncthreads();
-  if (!factor_diag_block(A, Wi, NB, &bad, st)) return;
-  for (int idx = threadIdx.x; idx < NB * NB; idx += blockDim.x) {
-    int r = idx / NB, s = idx % NB;
-    Vinv_next[idx] = (r <= s) ? Wi[r][s] : 0.f;
-    if (r <= s) H[(long long)(q0 + r) * b + q0 + s] = A[r][s];
   }
 }
 
@@ -686,8 +803,6 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
   static std::atomic<unsigned long long> attr_done{0};
   if (first_on_device(attr_done)) {
     cudaFuncSetAttribute(chol_update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * NB * 132 * 4);
-    // 33 KB dynamic on top of 17 KB static shared memory: above the 48 KB default
-    cudaFuncSetAttribute(chol_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * NB * (NB + 1) * 4);
   }
   long long nl = 0;
   launch_pdl(damp_kernel, dim3(1), dim3(1024), 0, s, H, b, damp, g_diag, st);
@@ -698,27 +813,65 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
     launch_pdl(chol_diag_kernel, dim3(1), dim3(kDiagThreads), 2 * NB * (NB + 1) * 4, s, H, b, p0, nb, Vall + (size_t)p * NB * NB, st);
     ++nl;
   }
-  for (int p = np - 1; p >= 1; --p) {
+  // Each step: the panel (which also snapshots the next diagonal block), then on a side
+  // stream the next diagonal block ahead of its trailing update (factored and inverted
+  // while the update runs on the other SMs), the trailing update, and a join before the
+  // next panel, which needs that block's inverse.  While the stream is being captured the
+  // side kernel goes on the stream itself, in the same order.
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(s, &cap);
+  cudaStream_t s2 = s;
+  cudaEvent_t ev_panel = nullptr, ev_diag = nullptr;
+  if (cap == cudaStreamCaptureStatusNone && np > 1) {
+    int lo = 0, hi = 0;
+    cudaDeviceGetStreamPriorityRange(&lo, &hi);
+    if (cudaStreamCreateWithPriority(&s2, cudaStreamNonBlocking, hi) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ev_panel, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ev_diag, cudaEventDisableTiming) != cudaSuccess) {
+      if (s2 != s && s2 != nullptr) cudaStreamDestroy(s2);
+      if (ev_panel) cudaEventDestroy(ev_panel);
+      s2 = s;
+      ev_panel = nullptr;
+    }
+  }
+  const bool side = s2 != s;
+  cudaError_t e = cudaSuccess;
+  for (int p = np - 1; p >= 1 && e == cudaSuccess; --p) {
     const int p0 = p * NB, nb = min(NB, b - p0);
     float* V = Vall + (size_t)p * NB * NB;
+    float* Vnext = Vall + (size_t)(p - 1) * NB * NB;
     const int pgrid = min((p0 + 7) / 8, kNumSM);
-    launch_pdl(chol_panel_kernel, dim3(pgrid), dim3(256), 0, s, H, b, p0, nb, V, vs_hi, vs_lo, st);
+    launch_pdl(chol_panel_kernel, dim3(pgrid), dim3(256), 0, s, H, b, p0, nb, (const float*)V, vs_hi, vs_lo, Vnext,
+               (const pwp_stats*)st);
+    if (side) {
+      e = cudaEventRecord(ev_panel, s);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(s2, ev_panel, 0);
+      if (e != cudaSuccess) break;
+    }
+    launch_pdl(chol_diag_ahead_kernel, dim3(1), dim3(kDiagThreads), 2 * NB * (NB + 1) * 4, s2, (const float*)H, b,
+               p0, nb, Vnext, st);
+    if (side) e = cudaEventRecord(ev_diag, s2);
     // H[0:p0, 0:p0] -= V[0:p0, P] V[0:p0, P]^T on the tensor cores (tiles on or above the
-    // diagonal), then the next panel's diagonal block on its own; the CUDA-core kernel
-    // (which also factors that block) when the tensor-core path is not available
+    // diagonal; one SM left to the side kernel), else on the CUDA cores
     cudaError_t e2 = cudaSuccess;
     const bool tc = launch_stream_tc(kNoScore, H, p0, p0, b, 0, 0, vs_hi, vs_lo, nb, NB, vs_hi, vs_lo, nullptr,
-                                     nullptr, p0, nullptr, nullptr, Level2{}, st, s, &e2, true);
-    if (e2 != cudaSuccess) return e2;
-    if (tc) {
-      launch_pdl(chol_diag_kernel, dim3(1), dim3(kDiagThreads), 2 * NB * (NB + 1) * 4, s, H, b, p0 - NB, NB, Vall + (size_t)(p - 1) * NB * NB, st);
-    } else {
+                                     nullptr, p0, nullptr, nullptr, Level2{}, st, s, &e2, true, PickArgs{},
+                                     side ? 1 : 0);
+    if (e2 != cudaSuccess && e == cudaSuccess) e = e2;
+    if (!tc) {
       const int nT = (p0 + 127) / 128;
       launch_pdl(chol_update_kernel, dim3(nT * (nT + 1) / 2), dim3(256), 2 * NB * 132 * 4, s, H, b, p0, nb,
-                                                                        Vall + (size_t)(p - 1) * NB * NB, st);
+                 (const pwp_stats*)st);
     }
+    if (side && e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_diag, 0);
     nl += 3;
   }
+  if (side) {
+    cudaEventDestroy(ev_panel);
+    cudaEventDestroy(ev_diag);
+    cudaStreamDestroy(s2);
+  }
+  if (e != cudaSuccess) return e;
   launch_pdl(put_diag_inverses_kernel, dim3(np), dim3(256), 0, s, H, b, Vall, st);
   ++nl;
   // inverse by recursive doubling: merge [A B; 0 D] pairs of width m

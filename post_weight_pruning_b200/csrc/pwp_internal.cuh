@@ -274,11 +274,13 @@ void launch_sweep_select(int step, int score, Ctl* ctl, unsigned int* hist1, Lev
 // only the 128x128 tiles on or above the diagonal are visited.  Z (c x Bp, row stride ldz) and R,
 // stored transposed (b x Bp, row stride ldz), come as TF32 head and fp32 remainder
 // arrays.  Returns false, launching nothing, when the shape or alignment does not allow
-// the tensor-core path.
+// the tensor-core path.  spare_sms > 0 keeps that many SMs out of the persistent grid (for
+// a kernel that runs beside it on another stream).
 bool launch_stream_tc(int score, float* W, int c, int b, int ldw, int u0, int j, const float* Zhi, const float* Zlo,
                       int Bp, int ldz, const float* Rhi, const float* Rlo, const uint8_t* mask, const float* sc,
                       int hist_end, unsigned int* hist1, Ctl* ctl, Level2 l2, pwp_stats* st,
-                      cudaStream_t s, cudaError_t* err, bool upper = false, PickArgs pick = PickArgs{});
+                      cudaStream_t s, cudaError_t* err, bool upper = false, PickArgs pick = PickArgs{},
+                      int spare_sms = 0);
 
 // Wanda / magnitude: per-row quota or N:M groups, no weight update (rowprune.cu).  H
 // (its diagonal) or X ([n, b]) gives ||X_q|| for Wanda.

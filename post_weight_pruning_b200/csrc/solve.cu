@@ -95,7 +95,7 @@ __device__ __forceinline__ void panel_gemm(float (&acc)[2][8], const float* cons
 // the columns before jp (float4 dot products with the eight panel rows, which every lane
 // reads as broadcasts), then finishes its eight panel entries column by column.  In the
 // first pass the panel's diagonal rows are slot 0 of lanes 0..7: at column c lane c's
-// entries so far and its pivot reach every lane by shuffles, so the diagonal block is
+// entries so far reach every lane by shuffles (each lane forms the pivot), so the diagonal block is
 // factored and every row's panel entries solved in one sweep; a later pass reads the
 // stored diagonal rows and reciprocal pivots instead.  A packed row i holds columns up to
 // 4*(i/4)+3, so rows jp..jp+3 of a panel store only its first four columns; columns
@@ -141,6 +141,11 @@ __device__ bool chol_solve(const Rows<SMALL> R, float* __restrict__ y, float* __
             float lc[8];
 #pragma unroll
             for (int c2 = 0; c2 < c; ++c2) lc[c2] = __shfl_sync(0xffffffffu, x[0][c2], c);
+            // the pivot, formed in every lane from lane c's entries (the same operations
+            // in the same order as lane c's own v[0], so the same value)
+            float d = __shfl_sync(0xffffffffu, acc[0][c], c);
+#pragma unroll
+            for (int c2 = 0; c2 < c; ++c2) d = fmaf(-lc[c2], lc[c2], d);
             float v[2];
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
@@ -148,7 +153,6 @@ __device__ bool chol_solve(const Rows<SMALL> R, float* __restrict__ y, float* __
 #pragma unroll
               for (int c2 = 0; c2 < c; ++c2) v[q] = fmaf(-x[q][c2], lc[c2], v[q]);
             }
-            const float d = __shfl_sync(0xffffffffu, v[0], c);
             ok = ok && (d > 0.f);
             const float il = rsqrtf(d);
             if (lane == 0) idg[jp + c] = il;

@@ -402,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int SCORE>
 cudaError_t launch_variant(const CUtensorMap* maps, int c, int b, int u0, int j, int Bp, int upper,
                            const uint8_t* mask, const float* sc, int hist_end, unsigned int* hist1, Ctl* ctl,
-                           Level2 l2, PickArgs pk, pwp_stats* st, cudaStream_t s) {
+                           Level2 l2, PickArgs pk, pwp_stats* st, cudaStream_t s, int spare_sms) {
   static std::atomic<unsigned long long> attr_done{0};
   if (first_on_device(attr_done)) {
     cudaError_t e = cudaFuncSetAttribute(stream_tc_kernel<SCORE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -414,6 +414,7 @@ cudaError_t launch_variant(const CUtensorMap* maps, int c, int b, int u0, int j,
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   const int mt = (c + TM - 1) / TM;
   const int ntiles = upper ? mt * (mt + 1) / 2 : mt * ((b - u0 + TN - 1) / TN);
+  nsm = nsm - spare_sms > 1 ? nsm - spare_sms : 1;
   const int grid = ntiles < nsm ? ntiles : nsm;
   launch_pdl(stream_tc_kernel<SCORE>, dim3(grid), dim3(kThreads), SMEM_BYTES, s, maps[0], maps[1], maps[2], maps[3],
              maps[4], c, b, u0, j, Bp, upper, mask, sc, hist_end, hist1, ctl, l2, pk, st, wait_limit());
@@ -439,7 +440,7 @@ bool encode_f32(CUtensorMap* map, const float* base, int inner, int rows, int ld
 bool launch_stream_tc(int score, float* W, int c, int b, int ldw, int u0, int j, const float* Zhi, const float* Zlo,
                       int Bp, int ldz, const float* Rhi, const float* Rlo, const uint8_t* mask, const float* sc,
                       int hist_end, unsigned int* hist1, Ctl* ctl, Level2 l2, pwp_stats* st, cudaStream_t s,
-                      cudaError_t* err, bool upper, PickArgs pk) {
+                      cudaError_t* err, bool upper, PickArgs pk, int spare_sms) {
   *err = cudaSuccess;
   if (upper && (c != b || u0 != 0)) return false;
   // b, u0 multiples of 4: the epilogue moves whole float4s of W and 4-byte words of mask
@@ -455,11 +456,14 @@ bool launch_stream_tc(int score, float* W, int c, int b, int ldw, int u0, int j,
       !encode_f32(&maps[4], W, b, c, ldw, 32, TM))
     return false;
   if (score == kWanda)
-    *err = launch_variant<kWanda>(maps, c, b, u0, j, Bp, upper ? 1 : 0, mask, sc, hist_end, hist1, ctl, l2, pk, st, s);
+    *err = launch_variant<kWanda>(maps, c, b, u0, j, Bp, upper ? 1 : 0, mask, sc, hist_end, hist1, ctl, l2, pk, st, s,
+                                  spare_sms);
   else if (score == kObs)
-    *err = launch_variant<kObs>(maps, c, b, u0, j, Bp, upper ? 1 : 0, mask, sc, hist_end, hist1, ctl, l2, pk, st, s);
+    *err = launch_variant<kObs>(maps, c, b, u0, j, Bp, upper ? 1 : 0, mask, sc, hist_end, hist1, ctl, l2, pk, st, s,
+                                spare_sms);
   else
-    *err = launch_variant<kNoScore>(maps, c, b, u0, j, Bp, upper ? 1 : 0, mask, sc, hist_end, hist1, ctl, l2, pk, st, s);
+    *err = launch_variant<kNoScore>(maps, c, b, u0, j, Bp, upper ? 1 : 0, mask, sc, hist_end, hist1, ctl, l2, pk, st, s,
+                                    spare_sms);
   return true;
 }
 
