@@ -147,10 +147,6 @@ __device__ bool factor_diag_block(float (*A)[NB + 1], float (*Wi)[NB + 1], int n
 #pragma unroll 1
   for (int kb = 0; kb < NBK; ++kb) {
     const int k0 = BS * kb, r0 = k0 + BS, rest = NB - r0;
-    if (*reinterpret_cast<volatile int*>(bad)) {
-      if (tid == 0) set_error(st, PWP_ENOTSPD, kSiteCholDiag);
-      return false;
-    }
     if (tid < NB) {
       float Ld[8][8], il[8];
 #pragma unroll
@@ -222,6 +218,11 @@ __device__ bool factor_diag_block(float (*A)[NB + 1], float (*Wi)[NB + 1], int n
       }
     }
     __syncthreads();
+  }
+  // a non-positive pivot anywhere (the steps after it ran on garbage, harmlessly)
+  if (*bad) {
+    if (tid == 0) set_error(st, PWP_ENOTSPD, kSiteCholDiag);
+    return false;
   }
   return true;
 }
@@ -368,6 +369,15 @@ __global__ void __launch_bounds__(256) chol_panel_kernel(float* __restrict__ H, 
   __shared__ float WiT[NB][NB + 1];  // WiT[t][c] = Wi[c][t]
   __shared__ float rowbuf[8][NB];
   if (cta_failed(st)) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, stride = gridDim.x * 8;
+  // each warp's rows go software-pipelined: the next row's two values are loaded before
+  // the current row is computed (the first ones before the staging below)
+  int r = blockIdx.x * 8 + warp;
+  float n0 = 0.f, n1 = 0.f;
+  if (r < p0) {
+    n0 = lane < nb ? H[(long long)r * b + p0 + lane] : 0.f;
+    n1 = lane + 32 < nb ? H[(long long)r * b + p0 + lane + 32] : 0.f;
+  }
   {
     // WiT[t][c] = Vinv[c][t]: sixteen loads per thread in flight at once
     float v[NB * NB / 256];
@@ -393,11 +403,15 @@ __global__ void __launch_bounds__(256) chol_panel_kernel(float* __restrict__ H, 
     for (int m = 0; m < NB * NB / 256; ++m) snap[(r0 + 4 * m) * NB + sc] = v[m];
   }
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int r = blockIdx.x * 8 + warp; r < p0; r += gridDim.x * 8) {
+  for (; r < p0; r += stride) {
     float* hr = H + (long long)r * b + p0;
-    rowbuf[warp][lane] = lane < nb ? hr[lane] : 0.f;
-    rowbuf[warp][lane + 32] = lane + 32 < nb ? hr[lane + 32] : 0.f;
+    rowbuf[warp][lane] = n0;
+    rowbuf[warp][lane + 32] = n1;
+    const int rn = r + stride;
+    if (rn < p0) {
+      n0 = lane < nb ? H[(long long)rn * b + p0 + lane] : 0.f;
+      n1 = lane + 32 < nb ? H[(long long)rn * b + p0 + lane + 32] : 0.f;
+    }
     __syncwarp();
     // Wi is upper triangular: Wi[c][t] = 0 for t < c
     float s0 = 0.f, s1 = 0.f;
