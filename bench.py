@@ -626,7 +626,7 @@ def time_other_workloads(dev, args):
 
         def call():
             pwp.prune_layer(Wt, X=Xt, H=H, W_out=W_out, mask=mask, workspace=ws, stats=stats, check=False, **kw)
-        ms = _time_calls(call, steps=3)
+        ms = _time_calls(call, steps=5)
         nblk = (wl.b + wl.block - 1) // wl.block
         per_class = {K_HESSIAN: 1, K_FACTOR: 1, K_STREAM: nblk, K_SELECT: nblk, K_SOLVE: nblk}
         phases = {}
@@ -642,6 +642,7 @@ def time_other_workloads(dev, args):
             raise RuntimeError(f"{name}: status {st.status}")
         t = statistics.median(ms)
         out[name] = {"ms": t, "weights_per_s": wl.c * wl.b / (t / 1e3), "steps": len(ms),
+                     "ms_calls": [round(x, 3) for x in ms],
                      "config": f"W {wl.c}x{wl.b} bf16, X {wl.n}x{wl.b} bf16 ({wl.x_dist}), Thanos "
                                f"{wl.nm[0]}:{wl.nm[1]}, B={wl.block}, damp={wl.damp}",
                      "phases_ms": phases}
@@ -654,7 +655,7 @@ def time_other_workloads(dev, args):
     def block():
         res.update(pwp.prune_block(weights, acts, feeds, method="thanos", pattern="unstructured", sparsity=0.5,
                                    block=128, damp=0.01, check=False))
-    ms = _time_calls(block, steps=2)
+    ms = _time_calls(block, steps=3)
     for layer, (_, _, st_t) in res.items():
         st = pwp.read_stats(st_t)
         if st.status != 0 or st.pruned != st.target:
@@ -662,6 +663,7 @@ def time_other_workloads(dev, args):
     total = sum(int(w.numel()) for w in weights.values())
     t = statistics.median(ms)
     out["decoder_block"] = {"ms": t, "weights_per_s": total / (t / 1e3), "steps": len(ms),
+                            "ms_calls": [round(x, 3) for x in ms],
                             "config": ("q,k,v,o 4096x4096; gate,up 11008x4096; down 4096x11008 bf16; 128x2048 "
                                        "tokens per input drawn on the device; Thanos 50% unstructured global budget "
                                        "per layer, B=128; one H per input (4 builds), 7 prunes")}
