@@ -279,39 +279,84 @@ __global__ void __launch_bounds__(kDiagThreads) chol_diag_kernel(float* __restri
   store_diag_block(H, b, p0, nb, A, Wi, Vinv);
 }
 
-// The next panel's diagonal block ahead of the trailing update that would produce it,
-// so that its factorisation runs beside that update: A = S - Vr Vr^T, with S the block
-// [q0, q0+64)^2 as it stood before this step (the panel kernel's snapshot, left in the
-// block's slot of Vinv) and Vr the panel rows q0..q0+63 that the panel kernel just formed
-// (H[q0 + r][p0 + t], t < nb); then factored and inverted as in chol_diag_kernel, V^-1
-// into the same slot.  V itself is not stored: nothing reads H's diagonal blocks before
-// they receive their inverses (put_diag_inverses_kernel), and the trailing update still
-// writes the unfactored block there.
-__global__ void __launch_bounds__(kDiagThreads) chol_diag_ahead_kernel(const float* __restrict__ H, int b,
-                                                                       int p0, int nb, float* __restrict__ Vinv,
-                                                                       pwp_stats* st) {
+// Before panel p (panel columns [p0, p0+nb)) and after the trailing update of panel p+1:
+// the next diagonal block [q0, q0+64)^2, q0 = p0 - 64, as it stands (its upper triangle,
+// 64 x 64 row-major, into that block's slot of Vinv), and the rows q0..q0+63 of the panel
+// columns before the panel kernel turns them into V (64 x 64, zero beyond nb).
+__global__ void __launch_bounds__(256) chol_snap_kernel(const float* __restrict__ H, int b, int p0, int nb,
+                                                        float* __restrict__ snap, float* __restrict__ arows,
+                                                        const pwp_stats* st) {
   pdl_enter();
-  extern __shared__ __align__(16) float dsm[];
+  if (cta_failed(st)) return;
+  const int q0 = p0 - NB, sc = threadIdx.x & (NB - 1), r0 = threadIdx.x >> 6;
+  float v[NB * NB / 256], w[NB * NB / 256];
+#pragma unroll
+  for (int m = 0; m < NB * NB / 256; ++m) {
+    const int r = r0 + 4 * m;
+    v[m] = r <= sc ? H[(long long)(q0 + r) * b + q0 + sc] : 0.f;
+    w[m] = sc < nb ? H[(long long)(q0 + r) * b + p0 + sc] : 0.f;
+  }
+#pragma unroll
+  for (int m = 0; m < NB * NB / 256; ++m) {
+    snap[(r0 + 4 * m) * NB + sc] = v[m];
+    arows[(r0 + 4 * m) * NB + sc] = w[m];
+  }
+}
+
+// The next panel's diagonal block, off the factor's critical path: it needs only what the
+// snapshot kernel staged and the current panel's diagonal inverse, so it runs on a side
+// stream beside the panel kernel and the trailing update.  A = S - Vr Vr^T, with S the
+// staged block and Vr = Ar V_PP^-T the panel rows q0..q0+63 formed here from their staged
+// pre-panel values Ar (the same products, in the same order, as the panel kernel's); then
+// factored and inverted as in chol_diag_kernel, V^-1 into the block's slot (which held S).
+// V itself is not stored: nothing reads H's diagonal blocks before they receive their
+// inverses (put_diag_inverses_kernel), and the trailing update writes the unfactored block.
+__global__ void __launch_bounds__(kDiagThreads) chol_diag_ahead_kernel(const float* __restrict__ arows,
+                                                                       const float* __restrict__ Vinv_p,
+                                                                       float* __restrict__ Vinv, pwp_stats* st) {
+  pdl_enter();
+  extern __shared__ __align__(16) float dsm[];   // three 64 x 65 arrays
   float (*A)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(dsm);
   float (*Wi)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(dsm + NB * (NB + 1));
+  float (*WpT)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(dsm + 2 * NB * (NB + 1));
   __shared__ int bad;
   if (cta_failed(st)) return;
-  const int q0 = p0 - NB, tid = threadIdx.x, sc = tid & (NB - 1), r0 = tid >> 6;
+  const int tid = threadIdx.x, sc = tid & (NB - 1), r0 = tid >> 6;
   {
-    // S into A's upper triangle, Vr into Wi (Wi[r][t] = Vr[r][t]): all loads in flight
-    float v[NB * NB / 256], w[NB * NB / 256];
+    // S into A's upper triangle, Ar into Wi, V_PP^-1 transposed into WpT: loads in flight
+    float v[NB * NB / 256], w[NB * NB / 256], x[NB * NB / 256];
 #pragma unroll
     for (int m = 0; m < NB * NB / 256; ++m) {
       const int r = r0 + 4 * m;
       v[m] = r <= sc ? Vinv[r * NB + sc] : 0.f;
-      w[m] = sc < nb ? H[(long long)(q0 + r) * b + p0 + sc] : 0.f;
+      w[m] = arows[r * NB + sc];
+      x[m] = Vinv_p[r * NB + sc];
     }
 #pragma unroll
     for (int m = 0; m < NB * NB / 256; ++m) {
       const int r = r0 + 4 * m;
       if (r <= sc) A[r][sc] = v[m];
       Wi[r][sc] = w[m];
+      WpT[sc][r] = x[m];
     }
+  }
+  __syncthreads();
+  {
+    // Vr[r][c] = sum_t Ar[r][t] V_PP^-1[c][t], t ascending (the panel kernel's order): row
+    // r = tid / 4, columns c = tid % 4 + 4k; results to WpT's place once every thread is done
+    const int r = tid >> 2, c0 = tid & 3;
+    float acc[NB / 4];
+#pragma unroll
+    for (int k = 0; k < NB / 4; ++k) acc[k] = 0.f;
+#pragma unroll 4
+    for (int t = 0; t < NB; ++t) {
+      const float a = Wi[r][t];
+#pragma unroll
+      for (int k = 0; k < NB / 4; ++k) acc[k] = fmaf(a, WpT[t][c0 + 4 * k], acc[k]);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < NB / 4; ++k) WpT[r][c0 + 4 * k] = acc[k];   // WpT now holds Vr
   }
   __syncthreads();
   {
@@ -325,8 +370,8 @@ __global__ void __launch_bounds__(kDiagThreads) chol_diag_ahead_kernel(const flo
         float a[4], c4[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          a[i] = Wi[4 * tr + i][t];
-          c4[i] = Wi[4 * tc + i][t];
+          a[i] = WpT[4 * tr + i][t];
+          c4[i] = WpT[4 * tc + i][t];
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i)
@@ -340,7 +385,6 @@ __global__ void __launch_bounds__(kDiagThreads) chol_diag_ahead_kernel(const flo
           if (4 * tr + i <= 4 * tc + j) A[4 * tr + i][4 * tc + j] -= acc[i][j];
     }
   }
-  __syncthreads();
 #pragma unroll
   for (int m = 0; m < NB * NB / 256; ++m) {
     const int r = r0 + 4 * m;
@@ -364,7 +408,7 @@ __global__ void __launch_bounds__(kDiagThreads) chol_diag_ahead_kernel(const flo
 __global__ void __launch_bounds__(256) chol_panel_kernel(float* __restrict__ H, int b, int p0, int nb,
                                                          const float* __restrict__ Vinv,
                                                          float* __restrict__ vs_hi, float* __restrict__ vs_lo,
-                                                         float* __restrict__ snap, const pwp_stats* st) {
+                                                         const pwp_stats* st) {
   pdl_enter();
   __shared__ float WiT[NB][NB + 1];  // WiT[t][c] = Wi[c][t]
   __shared__ float rowbuf[8][NB];
@@ -388,19 +432,6 @@ __global__ void __launch_bounds__(256) chol_panel_kernel(float* __restrict__ H, 
       const int idx = threadIdx.x + 256 * m;
       WiT[idx % NB][idx / NB] = v[m];
     }
-  }
-  if (snap != nullptr && blockIdx.x == gridDim.x - 1) {
-    // the next diagonal block [p0-64, p0)^2 as it stands before this step's trailing
-    // update (its upper triangle, 64 x 64 row-major), for chol_diag_ahead_kernel
-    const int q0 = p0 - NB, sc = threadIdx.x & (NB - 1), r0 = threadIdx.x >> 6;
-    float v[NB * NB / 256];
-#pragma unroll
-    for (int m = 0; m < NB * NB / 256; ++m) {
-      const int r = r0 + 4 * m;
-      v[m] = r <= sc ? H[(long long)(q0 + r) * b + q0 + sc] : 0.f;
-    }
-#pragma unroll
-    for (int m = 0; m < NB * NB / 256; ++m) snap[(r0 + 4 * m) * NB + sc] = v[m];
   }
   __syncthreads();
   for (; r < p0; r += stride) {
@@ -743,11 +774,15 @@ static size_t tc_levels_floats(int b) {
   return need;
 }
 
-// Diagonal-block inverses, the doubling temporary, the current panel's rows as TF32 head
-// and remainder (2 x b x NB), the last 256-byte aligned, then the tensor-core levels' scratch.
+// Diagonal-block inverses, two 64 x 64 staging slots of the next panel rows (pre-panel
+// values, for chol_diag_ahead_kernel), the doubling temporary, the current panel's rows as
+// TF32 head and remainder (2 x b x NB), the last 256-byte aligned, then the tensor-core
+// levels' scratch.
 size_t factor_ws_bytes(int b) {
   const size_t np = (size_t)(b + NB - 1) / NB;
-  return (np * NB * NB + doubling_tmp_floats(b) + 2 * (size_t)b * NB + tc_levels_floats(b)) * sizeof(float) + 1024;
+  return (np * NB * NB + 2 * NB * NB + doubling_tmp_floats(b) + 2 * (size_t)b * NB + tc_levels_floats(b)) *
+             sizeof(float) +
+         1024;
 }
 
 // One pair [A B; 0 D] of a doubling level on the tensor cores: T = A^-1 B, then
@@ -809,7 +844,8 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
                                pwp_stats* st, cudaStream_t s) {
   const int np = (b + NB - 1) / NB;
   float* Vall = (float*)ws;
-  float* T = Vall + (size_t)np * NB * NB;
+  float* arows = Vall + (size_t)np * NB * NB;   // two slots, by the parity of the panel
+  float* T = arows + 2 * NB * NB;
   float* vs_hi = reinterpret_cast<float*>(
       (reinterpret_cast<uintptr_t>(T + doubling_tmp_floats(b)) + 255) & ~(uintptr_t)255);
   float* vs_lo = vs_hi + (size_t)b * NB;
@@ -817,6 +853,8 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
   static std::atomic<unsigned long long> attr_done{0};
   if (first_on_device(attr_done)) {
     cudaFuncSetAttribute(chol_update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * NB * 132 * 4);
+    cudaFuncSetAttribute(chol_diag_ahead_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         3 * NB * (NB + 1) * 4);
   }
   long long nl = 0;
   launch_pdl(damp_kernel, dim3(1), dim3(1024), 0, s, H, b, damp, g_diag, st);
@@ -827,25 +865,29 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
     launch_pdl(chol_diag_kernel, dim3(1), dim3(kDiagThreads), 2 * NB * (NB + 1) * 4, s, H, b, p0, nb, Vall + (size_t)p * NB * NB, st);
     ++nl;
   }
-  // Each step: the panel (which also snapshots the next diagonal block), then on a side
-  // stream the next diagonal block ahead of its trailing update (factored and inverted
-  // while the update runs on the other SMs), the trailing update, and a join before the
-  // next panel, which needs that block's inverse.  While the stream is being captured the
-  // side kernel goes on the stream itself, in the same order.
+  // Each step: the snapshot of the next diagonal block and of the panel rows that form it,
+  // then on a side stream that block's kernel (it needs nothing else of this step, so it
+  // runs beside the panel kernel and the trailing update), the panel, and the trailing
+  // update.  The next panel waits for the block's inverse through an event (one of two,
+  // by parity, so that waiting for one step's block never waits for the next one's).  While
+  // the stream is being captured into a graph everything goes on the stream itself, in the
+  // same order.
   cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
   cudaStreamIsCapturing(s, &cap);
   cudaStream_t s2 = s;
-  cudaEvent_t ev_panel = nullptr, ev_diag = nullptr;
+  cudaEvent_t ev_snap = nullptr, ev_diag[2] = {nullptr, nullptr};
   if (cap == cudaStreamCaptureStatusNone && np > 1) {
     int lo = 0, hi = 0;
     cudaDeviceGetStreamPriorityRange(&lo, &hi);
-    if (cudaStreamCreateWithPriority(&s2, cudaStreamNonBlocking, hi) != cudaSuccess ||
-        cudaEventCreateWithFlags(&ev_panel, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&ev_diag, cudaEventDisableTiming) != cudaSuccess) {
+    bool ok = cudaStreamCreateWithPriority(&s2, cudaStreamNonBlocking, hi) == cudaSuccess;
+    for (cudaEvent_t* ev : {&ev_snap, &ev_diag[0], &ev_diag[1]})
+      ok = ok && cudaEventCreateWithFlags(ev, cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) {
       if (s2 != s && s2 != nullptr) cudaStreamDestroy(s2);
-      if (ev_panel) cudaEventDestroy(ev_panel);
+      for (cudaEvent_t ev : {ev_snap, ev_diag[0], ev_diag[1]})
+        if (ev) cudaEventDestroy(ev);
       s2 = s;
-      ev_panel = nullptr;
+      ev_snap = ev_diag[0] = ev_diag[1] = nullptr;
     }
   }
   const bool side = s2 != s;
@@ -854,17 +896,25 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
     const int p0 = p * NB, nb = min(NB, b - p0);
     float* V = Vall + (size_t)p * NB * NB;
     float* Vnext = Vall + (size_t)(p - 1) * NB * NB;
-    const int pgrid = min((p0 + 7) / 8, kNumSM);
-    launch_pdl(chol_panel_kernel, dim3(pgrid), dim3(256), 0, s, H, b, p0, nb, (const float*)V, vs_hi, vs_lo, Vnext,
+    float* ar = arows + (size_t)(p & 1) * NB * NB;
+    launch_pdl(chol_snap_kernel, dim3(1), dim3(256), 0, s, (const float*)H, b, p0, nb, Vnext, ar,
                (const pwp_stats*)st);
     if (side) {
-      e = cudaEventRecord(ev_panel, s);
-      if (e == cudaSuccess) e = cudaStreamWaitEvent(s2, ev_panel, 0);
+      e = cudaEventRecord(ev_snap, s);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(s2, ev_snap, 0);
       if (e != cudaSuccess) break;
     }
-    launch_pdl(chol_diag_ahead_kernel, dim3(1), dim3(kDiagThreads), 2 * NB * (NB + 1) * 4, s2, (const float*)H, b,
-               p0, nb, Vnext, st);
-    if (side) e = cudaEventRecord(ev_diag, s2);
+    launch_pdl(chol_diag_ahead_kernel, dim3(1), dim3(kDiagThreads), 3 * NB * (NB + 1) * 4, s2, (const float*)ar,
+               (const float*)V, Vnext, st);
+    if (side) {
+      e = cudaEventRecord(ev_diag[(p - 1) & 1], s2);
+      // this panel needs its own block's inverse (the previous step's side kernel)
+      if (e == cudaSuccess && p < np - 1) e = cudaStreamWaitEvent(s, ev_diag[p & 1], 0);
+      if (e != cudaSuccess) break;
+    }
+    const int pgrid = min((p0 + 7) / 8, kNumSM);
+    launch_pdl(chol_panel_kernel, dim3(pgrid), dim3(256), 0, s, H, b, p0, nb, (const float*)V, vs_hi, vs_lo,
+               (const pwp_stats*)st);
     // H[0:p0, 0:p0] -= V[0:p0, P] V[0:p0, P]^T on the tensor cores (tiles on or above the
     // diagonal; one SM left to the side kernel), else on the CUDA cores
     cudaError_t e2 = cudaSuccess;
@@ -877,12 +927,12 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
       launch_pdl(chol_update_kernel, dim3(nT * (nT + 1) / 2), dim3(256), 2 * NB * 132 * 4, s, H, b, p0, nb,
                  (const pwp_stats*)st);
     }
-    if (side && e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_diag, 0);
-    nl += 3;
+    nl += 4;
   }
+  // the last block's inverse before the inverses go in place
+  if (side && e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_diag[0], 0);
   if (side) {
-    cudaEventDestroy(ev_panel);
-    cudaEventDestroy(ev_diag);
+    for (cudaEvent_t ev : {ev_snap, ev_diag[0], ev_diag[1]}) cudaEventDestroy(ev);
     cudaStreamDestroy(s2);
   }
   if (e != cudaSuccess) return e;
