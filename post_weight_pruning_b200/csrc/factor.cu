@@ -279,39 +279,17 @@ __global__ void __launch_bounds__(kDiagThreads) chol_diag_kernel(float* __restri
   store_diag_block(H, b, p0, nb, A, Wi, Vinv);
 }
 
-// Before panel p (panel columns [p0, p0+nb)) and after the trailing update of panel p+1:
-// the next diagonal block [q0, q0+64)^2, q0 = p0 - 64, as it stands (its upper triangle,
-// 64 x 64 row-major, into that block's slot of Vinv), and the rows q0..q0+63 of the panel
-// columns before the panel kernel turns them into V (64 x 64, zero beyond nb).
-__global__ void __launch_bounds__(256) chol_snap_kernel(const float* __restrict__ H, int b, int p0, int nb,
-                                                        float* __restrict__ snap, float* __restrict__ arows,
-                                                        const pwp_stats* st) {
-  pdl_enter();
-  if (cta_failed(st)) return;
-  const int q0 = p0 - NB, sc = threadIdx.x & (NB - 1), r0 = threadIdx.x >> 6;
-  float v[NB * NB / 256], w[NB * NB / 256];
-#pragma unroll
-  for (int m = 0; m < NB * NB / 256; ++m) {
-    const int r = r0 + 4 * m;
-    v[m] = r <= sc ? H[(long long)(q0 + r) * b + q0 + sc] : 0.f;
-    w[m] = sc < nb ? H[(long long)(q0 + r) * b + p0 + sc] : 0.f;
-  }
-#pragma unroll
-  for (int m = 0; m < NB * NB / 256; ++m) {
-    snap[(r0 + 4 * m) * NB + sc] = v[m];
-    arows[(r0 + 4 * m) * NB + sc] = w[m];
-  }
-}
-
-// The next panel's diagonal block, off the factor's critical path: it needs only what the
-// snapshot kernel staged and the current panel's diagonal inverse, so it runs on a side
-// stream beside the panel kernel and the trailing update.  A = S - Vr Vr^T, with S the
-// staged block and Vr = Ar V_PP^-T the panel rows q0..q0+63 formed here from their staged
-// pre-panel values Ar (the same products, in the same order, as the panel kernel's); then
-// factored and inverted as in chol_diag_kernel, V^-1 into the block's slot (which held S).
-// V itself is not stored: nothing reads H's diagonal blocks before they receive their
-// inverses (put_diag_inverses_kernel), and the trailing update writes the unfactored block.
-__global__ void __launch_bounds__(kDiagThreads) chol_diag_ahead_kernel(const float* __restrict__ arows,
+// The next panel's diagonal block, off the factor's critical path.  Between the trailing
+// update of panel p+1 and the end of the factor nothing changes the block [q0, q0+64)^2,
+// q0 = p0 - 64 (panel p's update leaves it as it was), nor the pre-panel values Ar of rows
+// q0..q0+63 in panel p's columns (panel p parks their V in a slot, the next panel puts it in
+// place), so this kernel runs on a side stream beside panel p and its update: A = S - Vr Vr^T
+// with S the block and Vr = Ar V_PP^-T (the same products, in the same order, as the panel
+// kernel's), then factored and inverted as in chol_diag_kernel, V^-1 into the block's slot
+// of Vinv.  V itself is not stored: nothing reads H's diagonal blocks before they receive
+// their inverses (put_diag_inverses_kernel).
+__global__ void __launch_bounds__(kDiagThreads) chol_diag_ahead_kernel(const float* __restrict__ H, int b,
+                                                                       int p0, int nb,
                                                                        const float* __restrict__ Vinv_p,
                                                                        float* __restrict__ Vinv, pwp_stats* st) {
   pdl_enter();
@@ -321,15 +299,15 @@ __global__ void __launch_bounds__(kDiagThreads) chol_diag_ahead_kernel(const flo
   float (*WpT)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(dsm + 2 * NB * (NB + 1));
   __shared__ int bad;
   if (cta_failed(st)) return;
-  const int tid = threadIdx.x, sc = tid & (NB - 1), r0 = tid >> 6;
+  const int q0 = p0 - NB, tid = threadIdx.x, sc = tid & (NB - 1), r0 = tid >> 6;
   {
     // S into A's upper triangle, Ar into Wi, V_PP^-1 transposed into WpT: loads in flight
     float v[NB * NB / 256], w[NB * NB / 256], x[NB * NB / 256];
 #pragma unroll
     for (int m = 0; m < NB * NB / 256; ++m) {
       const int r = r0 + 4 * m;
-      v[m] = r <= sc ? Vinv[r * NB + sc] : 0.f;
-      w[m] = arows[r * NB + sc];
+      v[m] = r <= sc ? H[(long long)(q0 + r) * b + q0 + sc] : 0.f;
+      w[m] = sc < nb ? H[(long long)(q0 + r) * b + p0 + sc] : 0.f;
       x[m] = Vinv_p[r * NB + sc];
     }
 #pragma unroll
@@ -408,7 +386,8 @@ __global__ void __launch_bounds__(kDiagThreads) chol_diag_ahead_kernel(const flo
 __global__ void __launch_bounds__(256) chol_panel_kernel(float* __restrict__ H, int b, int p0, int nb,
                                                          const float* __restrict__ Vinv,
                                                          float* __restrict__ vs_hi, float* __restrict__ vs_lo,
-                                                         const pwp_stats* st) {
+                                                         float* __restrict__ vr_out, const float* __restrict__ vr_in,
+                                                         int in_nb, const pwp_stats* st) {
   pdl_enter();
   __shared__ float WiT[NB][NB + 1];  // WiT[t][c] = Wi[c][t]
   __shared__ float rowbuf[8][NB];
@@ -433,7 +412,20 @@ __global__ void __launch_bounds__(256) chol_panel_kernel(float* __restrict__ H, 
       WiT[idx % NB][idx / NB] = v[m];
     }
   }
+  if (vr_in != nullptr && blockIdx.x == gridDim.x - 1) {
+    // the previous panel's rows [p0, p0 + 64), parked in vr_in while this step's diagonal
+    // block kernel read their pre-panel values, go into place
+    const int sc = threadIdx.x & (NB - 1), r0 = threadIdx.x >> 6;
+    float v[NB * NB / 256];
+#pragma unroll
+    for (int m = 0; m < NB * NB / 256; ++m) v[m] = vr_in[(r0 + 4 * m) * NB + sc];
+    if (sc < in_nb) {
+#pragma unroll
+      for (int m = 0; m < NB * NB / 256; ++m) H[(long long)(p0 + r0 + 4 * m) * b + p0 + NB + sc] = v[m];
+    }
+  }
   __syncthreads();
+  const int q0 = vr_out != nullptr ? p0 - NB : p0;   // rows from q0 on are parked in vr_out
   for (; r < p0; r += stride) {
     float* hr = H + (long long)r * b + p0;
     rowbuf[warp][lane] = n0;
@@ -452,8 +444,9 @@ __global__ void __launch_bounds__(256) chol_panel_kernel(float* __restrict__ H, 
       s0 = fmaf(x, WiT[t][lane], s0);
       s1 = fmaf(x, WiT[t][lane + 32], s1);
     }
-    if (lane < nb) hr[lane] = s0;
-    if (lane + 32 < nb) hr[lane + 32] = s1;
+    float* dst = r < q0 ? hr : vr_out + (r - q0) * NB;
+    if (lane < nb) dst[lane] = s0;
+    if (lane + 32 < nb) dst[lane + 32] = s1;
     if (vs_hi) {
       const float h0 = tf32_head(s0), h1 = tf32_head(s1);
       vs_hi[(size_t)r * NB + lane] = h0;
@@ -467,9 +460,11 @@ __global__ void __launch_bounds__(256) chol_panel_kernel(float* __restrict__ H, 
 
 // Symmetric update of the top-left part on the CUDA cores (when the tensor-core update
 // cannot take the shape): A[r][s] -= sum_t V[r][p0+t] V[s][p0+t] for r <= s < p0,
-// 128x128 tiles on or above the diagonal, 8x8 outputs per thread.
-__global__ void __launch_bounds__(256) chol_update_kernel(float* __restrict__ H, int b, int p0, int nb,
-                                                          const pwp_stats* st) {
+// 128x128 tiles on or above the diagonal, 8x8 outputs per thread; with keep >= 0 the block
+// [keep, p0)^2 is left as it was and the panel's rows from keep on are read from vr, where
+// the panel kernel parked them.
+__global__ void __launch_bounds__(256) chol_update_kernel(float* __restrict__ H, int b, int p0, int nb, int keep,
+                                                          const float* __restrict__ vr, const pwp_stats* st) {
   pdl_enter();
   extern __shared__ __align__(16) float fsm[];
   float (*As)[128 + 4] = reinterpret_cast<float (*)[132]>(fsm);               // [NB][132], k-major
@@ -484,8 +479,10 @@ __global__ void __launch_bounds__(256) chol_update_kernel(float* __restrict__ H,
     const int rr = idx / NB, t = idx % NB;
     float a = 0.f, c = 0.f;
     if (t < nb) {
-      if (i0 + rr < p0) a = H[(long long)(i0 + rr) * b + p0 + t];
-      if (j0 + rr < p0) c = H[(long long)(j0 + rr) * b + p0 + t];
+      // the panel rows from keep on are parked in vr (64 x 64), the others are in place
+      const int ri = i0 + rr, rj = j0 + rr;
+      if (ri < p0) a = (keep >= 0 && ri >= keep) ? vr[(ri - keep) * NB + t] : H[(long long)ri * b + p0 + t];
+      if (rj < p0) c = (keep >= 0 && rj >= keep) ? vr[(rj - keep) * NB + t] : H[(long long)rj * b + p0 + t];
     }
     As[t][rr] = a;
     Bs[t][rr] = c;
@@ -513,7 +510,7 @@ __global__ void __launch_bounds__(256) chol_update_kernel(float* __restrict__ H,
 #pragma unroll
     for (int y = 0; y < 8; ++y) {
       const int s = j0 + (y < 4 ? tx * 4 + y : 64 + tx * 4 + y - 4);
-      if (s < p0 && r <= s) H[(long long)r * b + s] -= acc[x][y];
+      if (s < p0 && r <= s && !(r >= keep && keep >= 0)) H[(long long)r * b + s] -= acc[x][y];
     }
   }
 }
@@ -521,9 +518,16 @@ __global__ void __launch_bounds__(256) chol_update_kernel(float* __restrict__ H,
 // Put every diagonal block's inverse in place (the inverse of an upper-triangular
 // matrix has the inverses of its diagonal blocks on its block diagonal).
 __global__ void put_diag_inverses_kernel(float* __restrict__ H, int b, const float* __restrict__ Vall,
-                                         const pwp_stats* st) {
+                                         const float* __restrict__ vr_last, int last_nb, const pwp_stats* st) {
   pdl_enter();
   if (cta_failed(st)) return;
+  if (vr_last != nullptr && blockIdx.x == 0) {
+    // the first panel's rows [0, 64), parked by its panel kernel, into place (columns 64..)
+    for (int idx = threadIdx.x; idx < NB * NB; idx += blockDim.x) {
+      const int rr = idx / NB, cc = idx % NB;
+      if (cc < last_nb) H[(long long)rr * b + NB + cc] = vr_last[idx];
+    }
+  }
   const int p = blockIdx.x;
   const int p0 = p * NB, nb = min(NB, b - p0);
   const float* V = Vall + (size_t)p * NB * NB;
@@ -774,8 +778,8 @@ static size_t tc_levels_floats(int b) {
   return need;
 }
 
-// Diagonal-block inverses, two 64 x 64 staging slots of the next panel rows (pre-panel
-// values, for chol_diag_ahead_kernel), the doubling temporary, the current panel's rows as
+// Diagonal-block inverses, two 64 x 64 slots of parked panel rows (the V of the rows that
+// form the next diagonal block, held back one step), the doubling temporary, the current panel's rows as
 // TF32 head and remainder (2 x b x NB), the last 256-byte aligned, then the tensor-core
 // levels' scratch.
 size_t factor_ws_bytes(int b) {
@@ -844,8 +848,8 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
                                pwp_stats* st, cudaStream_t s) {
   const int np = (b + NB - 1) / NB;
   float* Vall = (float*)ws;
-  float* arows = Vall + (size_t)np * NB * NB;   // two slots, by the parity of the panel
-  float* T = arows + 2 * NB * NB;
+  float* vrows = Vall + (size_t)np * NB * NB;   // two slots of parked panel rows, by parity
+  float* T = vrows + 2 * NB * NB;
   float* vs_hi = reinterpret_cast<float*>(
       (reinterpret_cast<uintptr_t>(T + doubling_tmp_floats(b)) + 255) & ~(uintptr_t)255);
   float* vs_lo = vs_hi + (size_t)b * NB;
@@ -865,29 +869,30 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
     launch_pdl(chol_diag_kernel, dim3(1), dim3(kDiagThreads), 2 * NB * (NB + 1) * 4, s, H, b, p0, nb, Vall + (size_t)p * NB * NB, st);
     ++nl;
   }
-  // Each step: the snapshot of the next diagonal block and of the panel rows that form it,
-  // then on a side stream that block's kernel (it needs nothing else of this step, so it
-  // runs beside the panel kernel and the trailing update), the panel, and the trailing
-  // update.  The next panel waits for the block's inverse through an event (one of two,
-  // by parity, so that waiting for one step's block never waits for the next one's).  While
-  // the stream is being captured into a graph everything goes on the stream itself, in the
-  // same order.
+  // Each step: on a side stream the next diagonal block's kernel, which reads only what the
+  // trailing update of the previous panel left in H (after an event recorded behind it) and
+  // the current block's inverse, so it runs beside the panel kernel and this step's update
+  // (which leaves that block as it was); the panel, which parks the V of the rows that form
+  // the next block and puts the previous step's parked rows in place; the trailing update.
+  // The next panel waits for the block's inverse through an event (one of two, by parity,
+  // so that waiting for one step's block never waits for the next one's).  While the stream
+  // is being captured into a graph everything goes on the stream itself, in the same order.
   cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
   cudaStreamIsCapturing(s, &cap);
   cudaStream_t s2 = s;
-  cudaEvent_t ev_snap = nullptr, ev_diag[2] = {nullptr, nullptr};
+  cudaEvent_t ev_upd = nullptr, ev_diag[2] = {nullptr, nullptr};
   if (cap == cudaStreamCaptureStatusNone && np > 1) {
     int lo = 0, hi = 0;
     cudaDeviceGetStreamPriorityRange(&lo, &hi);
     bool ok = cudaStreamCreateWithPriority(&s2, cudaStreamNonBlocking, hi) == cudaSuccess;
-    for (cudaEvent_t* ev : {&ev_snap, &ev_diag[0], &ev_diag[1]})
+    for (cudaEvent_t* ev : {&ev_upd, &ev_diag[0], &ev_diag[1]})
       ok = ok && cudaEventCreateWithFlags(ev, cudaEventDisableTiming) == cudaSuccess;
     if (!ok) {
       if (s2 != s && s2 != nullptr) cudaStreamDestroy(s2);
-      for (cudaEvent_t ev : {ev_snap, ev_diag[0], ev_diag[1]})
+      for (cudaEvent_t ev : {ev_upd, ev_diag[0], ev_diag[1]})
         if (ev) cudaEventDestroy(ev);
       s2 = s;
-      ev_snap = ev_diag[0] = ev_diag[1] = nullptr;
+      ev_upd = ev_diag[0] = ev_diag[1] = nullptr;
     }
   }
   const bool side = s2 != s;
@@ -896,16 +901,13 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
     const int p0 = p * NB, nb = min(NB, b - p0);
     float* V = Vall + (size_t)p * NB * NB;
     float* Vnext = Vall + (size_t)(p - 1) * NB * NB;
-    float* ar = arows + (size_t)(p & 1) * NB * NB;
-    launch_pdl(chol_snap_kernel, dim3(1), dim3(256), 0, s, (const float*)H, b, p0, nb, Vnext, ar,
-               (const pwp_stats*)st);
     if (side) {
-      e = cudaEventRecord(ev_snap, s);
-      if (e == cudaSuccess) e = cudaStreamWaitEvent(s2, ev_snap, 0);
+      e = cudaEventRecord(ev_upd, s);   // behind the previous update (or the last block's factor)
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(s2, ev_upd, 0);
       if (e != cudaSuccess) break;
     }
-    launch_pdl(chol_diag_ahead_kernel, dim3(1), dim3(kDiagThreads), 3 * NB * (NB + 1) * 4, s2, (const float*)ar,
-               (const float*)V, Vnext, st);
+    launch_pdl(chol_diag_ahead_kernel, dim3(1), dim3(kDiagThreads), 3 * NB * (NB + 1) * 4, s2, (const float*)H, b,
+               p0, nb, (const float*)V, Vnext, st);
     if (side) {
       e = cudaEventRecord(ev_diag[(p - 1) & 1], s2);
       // this panel needs its own block's inverse (the previous step's side kernel)
@@ -913,30 +915,34 @@ cudaError_t launch_damp_factor(float* H, int b, float damp, float* g_diag, void*
       if (e != cudaSuccess) break;
     }
     const int pgrid = min((p0 + 7) / 8, kNumSM);
+    const float* vr_in = p < np - 1 ? vrows + (size_t)((p + 1) & 1) * NB * NB : nullptr;
+    const int in_nb = min(NB, b - (p0 + NB));
     launch_pdl(chol_panel_kernel, dim3(pgrid), dim3(256), 0, s, H, b, p0, nb, (const float*)V, vs_hi, vs_lo,
-               (const pwp_stats*)st);
+               vrows + (size_t)(p & 1) * NB * NB, vr_in, in_nb, (const pwp_stats*)st);
     // H[0:p0, 0:p0] -= V[0:p0, P] V[0:p0, P]^T on the tensor cores (tiles on or above the
-    // diagonal; one SM left to the side kernel), else on the CUDA cores
+    // diagonal, the next diagonal block left as it is; one SM left to the side kernel), else
+    // on the CUDA cores
     cudaError_t e2 = cudaSuccess;
     const bool tc = launch_stream_tc(kNoScore, H, p0, p0, b, 0, 0, vs_hi, vs_lo, nb, NB, vs_hi, vs_lo, nullptr,
                                      nullptr, p0, nullptr, nullptr, Level2{}, st, s, &e2, true, PickArgs{},
-                                     side ? 1 : 0);
+                                     side ? 1 : 0, p0 - NB);
     if (e2 != cudaSuccess && e == cudaSuccess) e = e2;
     if (!tc) {
       const int nT = (p0 + 127) / 128;
       launch_pdl(chol_update_kernel, dim3(nT * (nT + 1) / 2), dim3(256), 2 * NB * 132 * 4, s, H, b, p0, nb,
-                 (const pwp_stats*)st);
+                 p0 - NB, (const float*)(vrows + (size_t)(p & 1) * NB * NB), (const pwp_stats*)st);
     }
-    nl += 4;
+    nl += 3;
   }
   // the last block's inverse before the inverses go in place
   if (side && e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_diag[0], 0);
   if (side) {
-    for (cudaEvent_t ev : {ev_snap, ev_diag[0], ev_diag[1]}) cudaEventDestroy(ev);
+    for (cudaEvent_t ev : {ev_upd, ev_diag[0], ev_diag[1]}) cudaEventDestroy(ev);
     cudaStreamDestroy(s2);
   }
   if (e != cudaSuccess) return e;
-  launch_pdl(put_diag_inverses_kernel, dim3(np), dim3(256), 0, s, H, b, Vall, st);
+  launch_pdl(put_diag_inverses_kernel, dim3(np), dim3(256), 0, s, H, b, (const float*)Vall,
+             np > 1 ? (const float*)(vrows + NB * NB) : nullptr, min(NB, b - NB), (const pwp_stats*)st);
   ++nl;
   // inverse by recursive doubling: merge [A B; 0 D] pairs of width m
   const bool tc_levels = (b % 4) == 0 && tensor_map_encoder() != nullptr;

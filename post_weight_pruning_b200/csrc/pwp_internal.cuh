@@ -275,12 +275,13 @@ void launch_sweep_select(int step, int score, Ctl* ctl, unsigned int* hist1, Lev
 // stored transposed (b x Bp, row stride ldz), come as TF32 head and fp32 remainder
 // arrays.  Returns false, launching nothing, when the shape or alignment does not allow
 // the tensor-core path.  spare_sms > 0 keeps that many SMs out of the persistent grid (for
-// a kernel that runs beside it on another stream).
+// a kernel that runs beside it on another stream); keep >= 0 (score kNoScore; a multiple of
+// 16) leaves the block [keep, keep + 64)^2 of W as it was.
 bool launch_stream_tc(int score, float* W, int c, int b, int ldw, int u0, int j, const float* Zhi, const float* Zlo,
                       int Bp, int ldz, const float* Rhi, const float* Rlo, const uint8_t* mask, const float* sc,
                       int hist_end, unsigned int* hist1, Ctl* ctl, Level2 l2, pwp_stats* st,
                       cudaStream_t s, cudaError_t* err, bool upper = false, PickArgs pick = PickArgs{},
-                      int spare_sms = 0);
+                      int spare_sms = 0, int keep = -1);
 
 // Wanda / magnitude: per-row quota or N:M groups, no weight update (rowprune.cu).  H
 // (its diagonal) or X ([n, b]) gives ||X_q|| for Wanda.

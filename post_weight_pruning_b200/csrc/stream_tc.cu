@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __grid_constant__ CUtensorMap mw, int c, int b, int u0, int j, int Bp, int upper,
                      const uint8_t* __restrict__ mask, const float* __restrict__ sc, int hist_end,
                      unsigned int* hist1, Ctl* ctl, Level2 l2, PickArgs pk,
-                     pwp_stats* st, long long spin) {
+                     pwp_stats* st, long long spin, int keep) {
   unsigned int* h2 = l2.pred;
   unsigned int* h2s = l2.pred_sum;
   __shared__ pick::Shared psh;
@@ -303,6 +303,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const int q0 = n0 + qt * 32 + colsel * 16;
           uint8_t* box = wbuf + buf * W_BOX;
+          if (SCORE == kNoScore && keep >= 0 && r >= keep && r < keep + 64 && q0 >= keep && q0 < keep + 64) {
+            // the block [keep, keep + 64)^2 keeps its values (its 16-column groups lie wholly
+            // inside or outside it: keep and q0 are multiples of 16)
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] = 0.f;
+          }
           if (q0 + 16 <= j) {
             // previous block: apply, and zero the removed weights
             const uint32_t* mr = reinterpret_cast<const uint32_t*>(mask + (long long)r * b + q0);
@@ -402,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int SCORE>
 cudaError_t launch_variant(const CUtensorMap* maps, int c, int b, int u0, int j, int Bp, int upper,
                            const uint8_t* mask, const float* sc, int hist_end, unsigned int* hist1, Ctl* ctl,
-                           Level2 l2, PickArgs pk, pwp_stats* st, cudaStream_t s, int spare_sms) {
+                           Level2 l2, PickArgs pk, pwp_stats* st, cudaStream_t s, int spare_sms, int keep) {
   static std::atomic<unsigned long long> attr_done{0};
   if (first_on_device(attr_done)) {
     cudaError_t e = cudaFuncSetAttribute(stream_tc_kernel<SCORE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -417,7 +423,7 @@ cudaError_t launch_variant(const CUtensorMap* maps, int c, int b, int u0, int j,
   nsm = nsm - spare_sms > 1 ? nsm - spare_sms : 1;
   const int grid = ntiles < nsm ? ntiles : nsm;
   launch_pdl(stream_tc_kernel<SCORE>, dim3(grid), dim3(kThreads), SMEM_BYTES, s, maps[0], maps[1], maps[2], maps[3],
-             maps[4], c, b, u0, j, Bp, upper, mask, sc, hist_end, hist1, ctl, l2, pk, st, wait_limit());
+             maps[4], c, b, u0, j, Bp, upper, mask, sc, hist_end, hist1, ctl, l2, pk, st, wait_limit(), keep);
   return cudaGetLastError();
 }
 
@@ -440,7 +446,7 @@ bool encode_f32(CUtensorMap* map, const float* base, int inner, int rows, int ld
 bool launch_stream_tc(int score, float* W, int c, int b, int ldw, int u0, int j, const float* Zhi, const float* Zlo,
                       int Bp, int ldz, const float* Rhi, const float* Rlo, const uint8_t* mask, const float* sc,
                       int hist_end, unsigned int* hist1, Ctl* ctl, Level2 l2, pwp_stats* st, cudaStream_t s,
-                      cudaError_t* err, bool upper, PickArgs pk, int spare_sms) {
+                      cudaError_t* err, bool upper, PickArgs pk, int spare_sms, int keep) {
   *err = cudaSuccess;
   if (upper && (c != b || u0 != 0)) return false;
   // b, u0 multiples of 4: the epilogue moves whole float4s of W and 4-byte words of mask
@@ -457,13 +463,13 @@ bool launch_stream_tc(int score, float* W, int c, int b, int ldw, int u0, int j,
     return false;
   if (score == kWanda)
     *err = launch_variant<kWanda>(maps, c, b, u0, j, Bp, upper ? 1 : 0, mask, sc, hist_end, hist1, ctl, l2, pk, st, s,
-                                  spare_sms);
+                                  spare_sms, -1);
   else if (score == kObs)
     *err = launch_variant<kObs>(maps, c, b, u0, j, Bp, upper ? 1 : 0, mask, sc, hist_end, hist1, ctl, l2, pk, st, s,
-                                spare_sms);
+                                spare_sms, -1);
   else
     *err = launch_variant<kNoScore>(maps, c, b, u0, j, Bp, upper ? 1 : 0, mask, sc, hist_end, hist1, ctl, l2, pk, st, s,
-                                    spare_sms);
+                                    spare_sms, keep);
   return true;
 }
 
