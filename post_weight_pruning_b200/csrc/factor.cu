@@ -552,19 +552,24 @@ struct TriGemm {
 };
 
 // Operand chunk of one 16-deep K step, held in registers between the global loads and the
-// shared-memory stores: A rows m0 + (tid >> 2) + 64 h, columns k0 + 4 (tid & 3) ..;
-// B rows k0 + (tid >> 5) + 8 h, columns n0 + 4 (tid & 31) ...
+// shared-memory stores.  TILE = 128: A rows m0 + (tid >> 2) + 64 h, columns k0 + 4 (tid & 3)
+// ..; B rows k0 + (tid >> 5) + 8 h, columns n0 + 4 (tid & 31) ...  TILE = 64: one float4 of
+// each (A rows m0 + (tid >> 2); B rows k0 + (tid >> 4), columns n0 + 4 (tid & 15)).
+template <int TILE>
 struct TriChunk {
-  float4 a[2], b[2];
+  static constexpr int H = TILE / 64;
+  float4 a[H], b[H];
 };
 
 // vec: every row start and column origin is 16-byte aligned, so whole float4s are read
 // and the masks applied afterwards; otherwise element by element.
+template <int TILE>
 __device__ __forceinline__ void trigemm_load(const TriGemm& g, const float* A, const float* B, int m0, int n0,
-                                             int k0, int kend, bool vec, TriChunk& ch) {
+                                             int k0, int kend, bool vec, TriChunk<TILE>& ch) {
+  constexpr int H = TILE / 64;
   const int tid = threadIdx.x;
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
+  for (int h = 0; h < H; ++h) {
     const int m = m0 + (tid >> 2) + 64 * h, k = k0 + 4 * (tid & 3);
     float v[4] = {0.f, 0.f, 0.f, 0.f};
     if (m < g.M) {
@@ -583,9 +588,10 @@ __device__ __forceinline__ void trigemm_load(const TriGemm& g, const float* A, c
     }
     ch.a[h] = make_float4(v[0], v[1], v[2], v[3]);
   }
+  constexpr int BR = TILE / 4;   // threads per B row
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int k = k0 + (tid >> 5) + 8 * h, n = n0 + 4 * (tid & 31);
+  for (int h = 0; h < H; ++h) {
+    const int k = k0 + tid / BR + (256 / BR) * h, n = n0 + 4 * (tid % BR);
     float v[4] = {0.f, 0.f, 0.f, 0.f};
     if (k < kend) {
       const float* src = B + (long long)k * g.ldb + n;
@@ -605,75 +611,77 @@ __device__ __forceinline__ void trigemm_load(const TriGemm& g, const float* A, c
   }
 }
 
+// One TILE x TILE tile of C per CTA of 256 threads, (TILE/16) x (TILE/16) outputs per
+// thread (8 x 8 at TILE = 128, 4 x 4 at TILE = 64: four times the CTAs for the narrow
+// levels, which would otherwise leave most SMs idle).
+template <int TILE>
 __global__ void __launch_bounds__(256) trigemm_kernel(TriGemm g, int vec, const pwp_stats* st) {
+  constexpr int R = TILE / 16, HALF = TILE / 2;
   pdl_enter();
-  __shared__ __align__(16) float As[2][16][128 + 4];
-  __shared__ __align__(16) float Bs[2][16][128 + 4];
+  __shared__ __align__(16) float As[2][16][TILE + 4];
+  __shared__ __align__(16) float Bs[2][16][TILE + 4];
   if (cta_failed(st)) return;
   const float* A = g.A + blockIdx.z * g.batch_a;
   const float* B = g.B + blockIdx.z * g.batch_b;
   float* C = g.C + blockIdx.z * g.batch_c;
-  const int m0 = blockIdx.y * 128, n0 = blockIdx.x * 128;
+  const int m0 = blockIdx.y * TILE, n0 = blockIdx.x * TILE;
   if (m0 >= g.M || n0 >= g.N) return;
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   // the triangular operand bounds the useful k range of this tile
   int kbeg = 0, kend = g.K;
-  if (g.a_upper) kbeg = m0;                       // k >= m
-  if (g.b_upper) kend = min(kend, n0 + 128);      // k <= n
-  float acc[8][8] = {};
-  TriChunk ch;
+  if (g.a_upper) kbeg = m0;                        // k >= m
+  if (g.b_upper) kend = min(kend, n0 + TILE);      // k <= n
+  float acc[R][R] = {};
+  TriChunk<TILE> ch;
   int buf = 0;
-  if (kbeg < kend) trigemm_load(g, A, B, m0, n0, kbeg, kend, vec != 0, ch);
+  if (kbeg < kend) trigemm_load<TILE>(g, A, B, m0, n0, kbeg, kend, vec != 0, ch);
   for (int k0 = kbeg; k0 < kend; k0 += 16) {
     // stage the chunk in registers, fetch the next one, then compute on the stage
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
+    for (int h = 0; h < TILE / 64; ++h) {
       const int mm = (tid >> 2) + 64 * h, kk = 4 * (tid & 3);
       As[buf][kk][mm] = ch.a[h].x;
       As[buf][kk + 1][mm] = ch.a[h].y;
       As[buf][kk + 2][mm] = ch.a[h].z;
       As[buf][kk + 3][mm] = ch.a[h].w;
-      const int kb = (tid >> 5) + 8 * h, nn = 4 * (tid & 31);
+      const int kb = tid / (TILE / 4) + (1024 / TILE) * h, nn = 4 * (tid % (TILE / 4));
       *reinterpret_cast<float4*>(&Bs[buf][kb][nn]) = ch.b[h];
     }
     __syncthreads();
-    if (k0 + 16 < kend) trigemm_load(g, A, B, m0, n0, k0 + 16, kend, vec != 0, ch);
+    if (k0 + 16 < kend) trigemm_load<TILE>(g, A, B, m0, n0, k0 + 16, kend, vec != 0, ch);
 #pragma unroll
     for (int kk = 0; kk < 16; ++kk) {
-      const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
-      const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][64 + ty * 4]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][kk][64 + tx * 4]);
-      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+      float av[R], bv[R];
 #pragma unroll
-      for (int x = 0; x < 8; ++x)
+      for (int hh = 0; hh < R / 4; ++hh) {
+        const float4 a4 = *reinterpret_cast<const float4*>(&As[buf][kk][HALF * hh + ty * 4]);
+        const float4 b4 = *reinterpret_cast<const float4*>(&Bs[buf][kk][HALF * hh + tx * 4]);
+        av[4 * hh] = a4.x; av[4 * hh + 1] = a4.y; av[4 * hh + 2] = a4.z; av[4 * hh + 3] = a4.w;
+        bv[4 * hh] = b4.x; bv[4 * hh + 1] = b4.y; bv[4 * hh + 2] = b4.z; bv[4 * hh + 3] = b4.w;
+      }
 #pragma unroll
-        for (int y = 0; y < 8; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
+      for (int x = 0; x < R; ++x)
+#pragma unroll
+        for (int y = 0; y < R; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
     }
     buf ^= 1;  // the next chunk goes to the other stage: one barrier per chunk suffices
   }
 #pragma unroll
-  for (int x = 0; x < 8; ++x) {
-    const int m = m0 + (x < 4 ? ty * 4 + x : 64 + ty * 4 + x - 4);
+  for (int x = 0; x < R; ++x) {
+    const int m = m0 + HALF * (x / 4) + ty * 4 + (x & 3);
     if (m >= g.M) continue;
     float* crow = C + (long long)m * g.ldc;
-    const int na = n0 + tx * 4, nb2 = n0 + 64 + tx * 4;
-    if (vec && na + 3 < g.N) {
-      *reinterpret_cast<float4*>(crow + na) =
-          make_float4(g.alpha * acc[x][0], g.alpha * acc[x][1], g.alpha * acc[x][2], g.alpha * acc[x][3]);
-    } else {
 #pragma unroll
-      for (int y = 0; y < 4; ++y)
-        if (na + y < g.N) crow[na + y] = g.alpha * acc[x][y];
-    }
-    if (vec && nb2 + 3 < g.N) {
-      *reinterpret_cast<float4*>(crow + nb2) =
-          make_float4(g.alpha * acc[x][4], g.alpha * acc[x][5], g.alpha * acc[x][6], g.alpha * acc[x][7]);
-    } else {
+    for (int hh = 0; hh < R / 4; ++hh) {
+      const int na = n0 + HALF * hh + tx * 4;
+      if (vec && na + 3 < g.N) {
+        *reinterpret_cast<float4*>(crow + na) = make_float4(g.alpha * acc[x][4 * hh], g.alpha * acc[x][4 * hh + 1],
+                                                            g.alpha * acc[x][4 * hh + 2], g.alpha * acc[x][4 * hh + 3]);
+      } else {
 #pragma unroll
-      for (int y = 4; y < 8; ++y)
-        if (nb2 + y - 4 < g.N) crow[nb2 + y - 4] = g.alpha * acc[x][y];
+        for (int yy = 0; yy < 4; ++yy)
+          if (na + yy < g.N) crow[na + yy] = g.alpha * acc[x][4 * hh + yy];
+      }
     }
   }
 }
@@ -729,12 +737,18 @@ __global__ void __launch_bounds__(256) tsplit_kernel(const float* __restrict__ s
 }
 
 void launch_trigemm(const TriGemm& g, int batch, const pwp_stats* st, cudaStream_t s) {
-  dim3 grid((g.N + 127) / 128, (g.M + 127) / 128, batch);
   // float4 access needs 16-byte aligned rows and batch entries
   const bool vec = ((uintptr_t)g.A % 16) == 0 && ((uintptr_t)g.B % 16) == 0 && ((uintptr_t)g.C % 16) == 0 &&
                    (g.lda % 4) == 0 && (g.ldb % 4) == 0 && (g.ldc % 4) == 0 && (g.batch_a % 4) == 0 &&
                    (g.batch_b % 4) == 0 && (g.batch_c % 4) == 0;
-  launch_pdl(trigemm_kernel, dim3(grid), dim3(256), 0, s, g, vec ? 1 : 0, st);
+  const long long tiles128 = (long long)((g.N + 127) / 128) * ((g.M + 127) / 128) * batch;
+  if (tiles128 < 2 * kNumSM) {   // too few 128-wide tiles to fill the GPU: 64-wide ones
+    dim3 grid((g.N + 63) / 64, (g.M + 63) / 64, batch);
+    launch_pdl(trigemm_kernel<64>, grid, dim3(256), 0, s, g, vec ? 1 : 0, st);
+  } else {
+    dim3 grid((g.N + 127) / 128, (g.M + 127) / 128, batch);
+    launch_pdl(trigemm_kernel<128>, grid, dim3(256), 0, s, g, vec ? 1 : 0, st);
+  }
 }
 
 }  // namespace
