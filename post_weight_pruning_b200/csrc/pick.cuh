@@ -126,6 +126,19 @@ __device__ void find_rank(const unsigned int* __restrict__ hist, long long rank,
   *before = sel < 0 ? 0 : bef;
 }
 
+// N words from global into shared memory by threads 0..kThreads-1, every load issued before
+// the first store, then the named barrier.
+template <int N>
+__device__ __forceinline__ void stage_words(unsigned int* dst, const unsigned int* src, int bar, int tid) {
+  static_assert(N % kThreads == 0, "whole rounds");
+  unsigned int v[N / kThreads];
+#pragma unroll
+  for (int k = 0; k < N / kThreads; ++k) v[k] = src[tid + kThreads * k];
+#pragma unroll
+  for (int k = 0; k < N / kThreads; ++k) dst[tid + kThreads * k] = v[k];
+  sync(bar);
+}
+
 // Step 1 of the budget loop and the level-1 bin: take = min(r, region) with r the residual
 // global count (Thanos) or the block quota (SparseGPT); the bin of the take-th key; whether
 // the scoring pass predicted it (then the level-2 histogram is ready).  Clears the level-1
@@ -133,7 +146,8 @@ __device__ void find_rank(const unsigned int* __restrict__ hist, long long rank,
 // (pruned: the removals so far over every row the budget counts; -1 for this call's own.)
 // On return sh.mode, sh.ready and sh.r1 hold the outcome for every thread.
 __device__ inline void level1(Ctl* ctl, unsigned int* hist1, long long region_n, int global_budget,
-                              long long quota, pwp_stats* st, Shared& sh, int bar, int tid, long long pruned = -1) {
+                              long long quota, pwp_stats* st, Shared& sh, int bar, int tid, long long pruned = -1,
+                              const unsigned int* staged = nullptr) {
   if (tid == 0) {
     const long long r = global_budget ? ctl->zstar - (pruned >= 0 ? pruned : ctl->pruned) : quota;
     long long take = r < region_n ? r : region_n;
@@ -156,7 +170,7 @@ __device__ inline void level1(Ctl* ctl, unsigned int* hist1, long long region_n,
   if (take > 0) {
     int bin;
     long long before;
-    find_rank<kHist1Bins>(hist1, take, &bin, &before, sh, bar, tid);
+    find_rank<kHist1Bins>(staged ? staged : hist1, take, &bin, &before, sh, bar, tid);
     if (tid == 0) {
       if (bin < 0) {
         set_error(st, PWP_EBUDGET, kSitePick);
@@ -186,17 +200,30 @@ __device__ inline void level1(Ctl* ctl, unsigned int* hist1, long long region_n,
 // (level1's sh.r1, or the control block's when level1 ran in an earlier kernel).  On
 // return sh.mode, sh.T, sh.m and sh.tie_scan hold the outcome for every thread.
 __device__ inline void level2(Ctl* ctl, Level2 l2, long long r1, int ready, pwp_stats* st, Shared& sh, int bar,
-                              int tid) {
+                              int tid, unsigned int* stage = nullptr) {
   const unsigned int* h2 = ready ? l2.pred : l2.reread;
   const unsigned int* h2s = ready ? l2.pred_sum : l2.reread_sum;
   int sb;
   long long before_s;
-  find_rank<kHist2SumBins>(h2s, r1, &sb, &before_s, sh, bar, tid);
+  if (stage) {
+    // the summary and then the chosen summary bin's counts go through shared memory, each
+    // with all its loads in flight (a rank search over global memory pays an L2 round trip
+    // per narrowing step)
+    stage_words<kHist2SumBins>(stage, h2s, bar, tid);
+    find_rank<kHist2SumBins>(stage, r1, &sb, &before_s, sh, bar, tid);
+  } else {
+    find_rank<kHist2SumBins>(h2s, r1, &sb, &before_s, sh, bar, tid);
+  }
   int sub = -1;
   long long before_sub = 0;
-  if (sb >= 0)
-    find_rank<(1 << kHist2SumShift)>(h2 + ((size_t)sb << kHist2SumShift), r1 - before_s, &sub, &before_sub, sh,
-                                     bar, tid);
+  if (sb >= 0) {
+    const unsigned int* hsub = h2 + ((size_t)sb << kHist2SumShift);
+    if (stage) {
+      stage_words<(1 << kHist2SumShift)>(stage + kHist2SumBins, hsub, bar, tid);
+      hsub = stage + kHist2SumBins;
+    }
+    find_rank<(1 << kHist2SumShift)>(hsub, r1 - before_s, &sub, &before_sub, sh, bar, tid);
+  }
   if (sb < 0 || sub < 0) {
     if (tid == 0) {
       set_error(st, PWP_EBUDGET, kSitePick);
@@ -340,8 +367,11 @@ __device__ inline bool last_cta(unsigned int* ticket, Shared& sh) {
 
 // After a scoring pass (all CTAs have added their level-1 counts): the last CTA takes the
 // level-1 bin and, when the predicted level-2 histogram holds, the exact threshold.
+// stage: kHist1Bins words of shared memory the CTA no longer needs, through which the rank
+// searches read their histograms (or nullptr: straight from global memory).
 __device__ inline void after_scoring(Ctl* ctl, unsigned int* hist1, Level2 l2, long long region_n,
-                                     int global_budget, long long quota, pwp_stats* st, Shared& sh) {
+                                     int global_budget, long long quota, pwp_stats* st, Shared& sh,
+                                     unsigned int* stage = nullptr) {
   if (!last_cta(&ctl->ticket, sh)) return;
   const int tid = threadIdx.x;
   if (tid >= kThreads) return;
@@ -349,8 +379,9 @@ __device__ inline void after_scoring(Ctl* ctl, unsigned int* hist1, Level2 l2, l
     for (int i = tid; i < kHist1Bins; i += kThreads) hist1[i] = 0u;
     return;
   }
-  level1(ctl, hist1, region_n, global_budget, quota, st, sh, 1, tid);
-  if (sh.mode != 0 && sh.ready) level2(ctl, l2, sh.r1, 1, st, sh, 1, tid);
+  if (stage) stage_words<kHist1Bins>(stage, hist1, 1, tid);
+  level1(ctl, hist1, region_n, global_budget, quota, st, sh, 1, tid, -1, stage);
+  if (sh.mode != 0 && sh.ready) level2(ctl, l2, sh.r1, 1, st, sh, 1, tid, stage);
 }
 
 }  // namespace pick

@@ -401,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (v) red_add_global(&hist1[i], v);
     }
     // the last CTA to finish takes the block's level-1 bin (and threshold, when predicted)
-    if (pk.enabled) pick::after_scoring(ctl, hist1, l2, pk.region_n, pk.global_budget, pk.quota, st, psh);
+    if (pk.enabled) pick::after_scoring(ctl, hist1, l2, pk.region_n, pk.global_budget, pk.quota, st, psh, shist);
   }
 }
 
