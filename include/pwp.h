@@ -182,6 +182,30 @@ pwp_status pwp_prune_layer_host(const pwp_config* cfg, const void* W_host, int32
                                 uint8_t* mask_out_host, void* ws, size_t ws_bytes,
                                 pwp_stats* stats_dev, void* stream);
 
+/* A sequence of same-shaped layers end to end from host memory (a model pruned layer by
+ * layer), each layer's transfers overlapping its neighbours' work: layer i+1's X and W go
+ * in on an input copy stream while layer i is pruned, and layer i's results come back on
+ * an output copy stream while layer i+1 is.  Per layer the steps and results are those of
+ * pwp_prune_layer_host (X in row chunks folded into H as they land, finished column blocks
+ * returned during the sweep), each layer against its own H.
+ *   nlayers         : number of layers (0: nothing to do).
+ *   W_host[i], X_host[i] : pinned host copies of layer i's W (c x b, wtype) and X ([n, b],
+ *                     xtype); every layer has the same c, b, n and types.
+ *   W_out_host[i], mask_out_host[i] : pinned host buffers (c x b fp32, c x b bytes).
+ *   dev, dev_bytes  : device scratch of at least pwp_layers_host_bytes(...) bytes, 256-byte
+ *                     aligned (two input and two output buffers, H and the prune workspace).
+ *   stats_dev       : nlayers pwp_stats records in device memory, one per layer.
+ * The work is enqueued on `stream`, which waits for the last copy: once it is synchronised
+ * every host output is complete.  Errors as pwp_prune_layer_x (PWP_EWORKSPACE when dev is
+ * missing, misaligned or too small); a layer's own failure is in its stats record. */
+size_t pwp_layers_host_bytes(const pwp_config* cfg, int32_t c, int32_t b, int64_t n, int32_t wtype,
+                             int32_t xtype);
+pwp_status pwp_prune_layers_host(const pwp_config* cfg, int32_t nlayers, const void* const* W_host,
+                                 int32_t wtype, int32_t c, int32_t b, const void* const* X_host,
+                                 int32_t xtype, int64_t n, float* const* W_out_host,
+                                 uint8_t* const* mask_out_host, void* dev, size_t dev_bytes,
+                                 pwp_stats* stats_dev, void* stream);
+
 /* Stepwise sweep: one layer's rows sharded over ranks (one process per GPU), pruned with the
  * unstructured budget counted over all ranks' rows ("Pruning LLMs with Thanos", section
  * "Contribution two: keep the budget global and the execution local": the budget couples

@@ -71,6 +71,9 @@ _SIGS = {
                                  _vp, _vp, _vp, _sz, _vp, _vp]),
     "pwp_prune_layer_host": (_i32, [ctypes.POINTER(Config), _vp, _i32, _i32, _i32, _vp, _i32, _i64, _vp, _vp,
                                     _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
+    "pwp_layers_host_bytes": (_sz, [ctypes.POINTER(Config), _i32, _i32, _i64, _i32, _i32]),
+    "pwp_prune_layers_host": (_i32, [ctypes.POINTER(Config), _i32, _vp, _i32, _i32, _i32, _vp, _i32, _i64, _vp,
+                                     _vp, _vp, _sz, _vp, _vp]),
     "pwp_pack_24": (_i32, [_vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp]),
     "pwp_status_string": (ctypes.c_char_p, [_i32]),
     "pwp_sweep_step": (_i32, [ctypes.POINTER(SweepArgs), _i32, _i32]),
@@ -466,6 +469,63 @@ def prune_layer_host(W_host, X_host, *, out_W=None, out_mask=None, device="cuda"
                                     _vp(stats.data_ptr()), _stream_ptr(stream))
     _check(st, "pwp_prune_layer_host")
     return out_W, out_mask, stats
+
+
+def prune_layers_host(Ws_host, Xs_host, *, out_Ws=None, out_masks=None, device="cuda", stream=None, **kw):
+    """A sequence of same-shaped layers from pinned host memory (pwp_prune_layers_host):
+    layer i+1's transfers overlap layer i's work and layer i's results come back while
+    layer i+1 is pruned.  Ws_host[i] ([c, b]) and Xs_host[i] ([n, b]) are pinned CPU tensors
+    of one dtype each (bf16 or fp32); keyword arguments as prune_layer.  Returns (W_hats,
+    masks, stats tensor of len(Ws_host) records); nothing syncs: synchronise the stream (the
+    current one by default) before reading them."""
+    torch = _torch()
+    nl = len(Ws_host)
+    if len(Xs_host) != nl:
+        raise ValueError("one X per W expected")
+    if nl == 0:
+        return [], [], new_stats(device)
+    c, b = Ws_host[0].shape
+    n = Xs_host[0].shape[0]
+    for name, ts, shape in (("W", Ws_host, (c, b)), ("X", Xs_host, (n, b))):
+        for t in ts:
+            if (tuple(t.shape) != shape or t.device.type != "cpu" or not t.is_pinned() or not t.is_contiguous()
+                    or t.dtype != ts[0].dtype or t.dtype not in (torch.bfloat16, torch.float32)):
+                raise ValueError(f"{name}: contiguous pinned CPU tensors of one shape {shape} and dtype "
+                                 f"(bf16 or fp32) expected")
+    if out_Ws is None:
+        out_Ws = [torch.empty((c, b), dtype=torch.float32, pin_memory=True) for _ in range(nl)]
+    if out_masks is None:
+        out_masks = [torch.empty((c, b), dtype=torch.uint8, pin_memory=True) for _ in range(nl)]
+    for name, ts, dt in (("out_Ws", out_Ws, torch.float32), ("out_masks", out_masks, torch.uint8)):
+        if len(ts) != nl or any(t.shape != (c, b) or t.dtype != dt or not t.is_pinned() or not t.is_contiguous()
+                                for t in ts):
+            raise ValueError(f"{name}: {nl} contiguous pinned CPU tensors [{c}, {b}] of {dt} expected")
+    cfg = config(kw.pop("method", "thanos"), kw.pop("pattern", "unstructured"), kw.pop("nm", (2, 4)),
+                 kw.pop("sparsity", 0.5), kw.pop("block", 128), kw.pop("damp", 0.01), kw.pop("alpha", 0.0))
+    if kw:
+        raise TypeError(f"unexpected arguments {sorted(kw)}")
+    L = lib()
+    wt, xt = _dtype_code(Ws_host[0]), _dtype_code(Xs_host[0])
+    nbytes = int(L.pwp_layers_host_bytes(ctypes.byref(cfg), int(c), int(b), int(n), wt, xt))
+    if nbytes == 0:
+        raise PwpError(1, "pwp_layers_host_bytes")
+    dev = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    stats = torch.zeros(nl * ctypes.sizeof(Stats), dtype=torch.uint8, device=device)
+    arr = lambda ts: (_vp * nl)(*[_vp(t.data_ptr()) for t in ts])
+    Wp, Xp, Op, Mp = arr(Ws_host), arr(Xs_host), arr(out_Ws), arr(out_masks)
+    st = L.pwp_prune_layers_host(ctypes.byref(cfg), nl, Wp, wt, int(c), int(b), Xp, xt, int(n), Op, Mp,
+                                 _vp(dev.data_ptr()), nbytes, _vp(stats.data_ptr()), _stream_ptr(stream))
+    _check(st, "pwp_prune_layers_host")
+    # the device scratch lives until the stream has passed the call
+    dev.record_stream(torch.cuda.current_stream() if stream is None else stream)
+    return out_Ws, out_masks, stats
+
+
+def read_stats_list(stats_t):
+    """The per-layer records of a stats tensor holding several (prune_layers_host)."""
+    raw = stats_t.cpu().numpy().tobytes()
+    sz = ctypes.sizeof(Stats)
+    return [Stats.from_buffer_copy(raw[i:i + sz]) for i in range(0, len(raw), sz)]
 
 
 def from_bf16_bits(u16: np.ndarray, device="cuda"):

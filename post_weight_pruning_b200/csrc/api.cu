@@ -232,6 +232,149 @@ pwp_status pwp_prune_layer_host(const pwp_config* cfg, const void* W_host, int32
   return ps;
 }
 
+// Device memory of pwp_prune_layers_host, in order (each piece 256-byte aligned): two W
+// buffers, two X buffers, H, two W-hat buffers, two masks, the prune workspace.
+static size_t layers_host_layout(const pwp_config* cfg, int32_t c, int32_t b, int64_t n, int32_t wtype,
+                                 int32_t xtype, size_t* off) {
+  auto up = [](size_t v) { return (v + 255) & ~(size_t)255; };
+  const size_t wb = up((size_t)c * b * dtype_bytes(wtype)), xb = up((size_t)n * b * dtype_bytes(xtype));
+  const size_t hb = up((size_t)b * b * sizeof(float)), ob = up((size_t)c * b * sizeof(float)), mb = up((size_t)c * b);
+  const size_t sizes[10] = {wb, wb, xb, xb, hb, ob, ob, mb, mb, prune_ws_layout(cfg, c, b, nullptr, nullptr)};
+  size_t at = 0;
+  for (int i = 0; i < 10; ++i) {
+    if (off) off[i] = at;
+    at += up(sizes[i]);
+  }
+  return at;
+}
+
+size_t pwp_layers_host_bytes(const pwp_config* cfg, int32_t c, int32_t b, int64_t n, int32_t wtype, int32_t xtype) {
+  if (!valid_cfg(cfg, c, b) || !valid_dtype(wtype) || !valid_dtype(xtype) || n < 0) return 0;
+  return layers_host_layout(cfg, c, b, n, wtype, xtype, nullptr);
+}
+
+pwp_status pwp_prune_layers_host(const pwp_config* cfg, int32_t nlayers, const void* const* W_host, int32_t wtype,
+                                 int32_t c, int32_t b, const void* const* X_host, int32_t xtype, int64_t n,
+                                 float* const* W_out_host, uint8_t* const* mask_out_host, void* dev,
+                                 size_t dev_bytes, pwp_stats* st, void* stream) {
+  if (!valid_cfg(cfg, c, b) || !valid_dtype(wtype) || !valid_dtype(xtype) || nlayers < 0 || n < 0 || !W_host ||
+      !W_out_host || !mask_out_host || !st || (n > 0 && !X_host))
+    return PWP_EINVAL;
+  for (int i = 0; i < nlayers; ++i)
+    if (!W_host[i] || !W_out_host[i] || !mask_out_host[i] || (n > 0 && !X_host[i])) return PWP_EINVAL;
+  size_t off[10];
+  if (!dev || !aligned(dev, 256) || dev_bytes < layers_host_layout(cfg, c, b, n, wtype, xtype, off))
+    return PWP_EWORKSPACE;
+  if (nlayers == 0) return PWP_OK;
+  const bool no_update = cfg->method == PWP_WANDA || cfg->method == PWP_MAGNITUDE;
+  char* base = (char*)dev;
+  void* W_dev[2] = {base + off[0], base + off[1]};
+  void* X_dev[2] = {base + off[2], base + off[3]};
+  float* H_dev = (float*)(base + off[4]);
+  float* Wo_dev[2] = {(float*)(base + off[5]), (float*)(base + off[6])};
+  uint8_t* mk_dev[2] = {(uint8_t*)(base + off[7]), (uint8_t*)(base + off[8])};
+  void* ws = base + off[9];
+  cudaStream_t s = (cudaStream_t)stream;
+  // an input and an output copy stream and the events of this call (released once their
+  // work is done): a layer's inputs go in while the previous layer is pruned, its results
+  // come back while the next one is
+  constexpr int kChunks = 8;
+  cudaStream_t cin = nullptr, cout = nullptr;
+  cudaEvent_t ev_start = nullptr, ev_chunk[kChunks] = {}, ev_w = nullptr, ev_blk = nullptr, ev_in_free[2] = {},
+              ev_out_done[2] = {};
+  cudaError_t e = cudaStreamCreateWithFlags(&cin, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&cout, cudaStreamNonBlocking);
+  for (cudaEvent_t* ev : {&ev_start, &ev_w, &ev_blk, &ev_in_free[0], &ev_in_free[1], &ev_out_done[0],
+                          &ev_out_done[1]})
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+  for (int i = 0; i < kChunks && e == cudaSuccess; ++i) e = cudaEventCreateWithFlags(&ev_chunk[i], cudaEventDisableTiming);
+  // the copies start after the caller's earlier work on `stream`
+  if (e == cudaSuccess) e = cudaEventRecord(ev_start, s);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(cin, ev_start, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(cout, ev_start, 0);
+  pwp_status ps = e == cudaSuccess ? PWP_OK : PWP_ECUDA;
+  const size_t xrow = (size_t)b * dtype_bytes(xtype), wbytes = (size_t)c * b * dtype_bytes(wtype);
+  const int64_t nch = (!no_update && n >= 8 * 1024) ? kChunks : 1;
+  const int64_t rows = n > 0 ? (n + nch - 1) / nch : 0;
+  for (int i = 0; i < nlayers && ps == PWP_OK; ++i) {
+    const int k = i & 1;
+    pwp_stats* sti = st + i;
+    // inputs of layer i into set k, once layer i-2 is done with it
+    if (i >= 2) e = cudaStreamWaitEvent(cin, ev_in_free[k], 0);
+    int nchunks = 0;
+    for (int64_t r0 = 0; r0 < n && e == cudaSuccess; r0 += rows, ++nchunks) {
+      const int64_t nr = n - r0 < rows ? n - r0 : rows;
+      e = cudaMemcpyAsync((char*)X_dev[k] + (size_t)r0 * xrow, (const char*)X_host[i] + (size_t)r0 * xrow,
+                          (size_t)nr * xrow, cudaMemcpyHostToDevice, cin);
+      if (e == cudaSuccess) e = cudaEventRecord(ev_chunk[nchunks], cin);
+    }
+    if (e == cudaSuccess) e = cudaMemcpyAsync(W_dev[k], W_host[i], wbytes, cudaMemcpyHostToDevice, cin);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_w, cin);
+    if (e == cudaSuccess) e = launch_stats_init(sti, s);
+    // W-hat and the mask of set k are free once layer i-2's results are back
+    if (e == cudaSuccess && i >= 2) e = cudaStreamWaitEvent(s, ev_out_done[k], 0);
+    if (e != cudaSuccess) {
+      ps = PWP_ECUDA;
+      break;
+    }
+    if (no_update) {
+      for (int ch = 0; ch < nchunks && e == cudaSuccess; ++ch) e = cudaStreamWaitEvent(s, ev_chunk[ch], 0);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_w, 0);
+      if (e == cudaSuccess)
+        e = launch_no_update(cfg, W_dev[k], wtype, c, b, nullptr, cfg->method == PWP_WANDA ? X_dev[k] : nullptr,
+                             xtype, cfg->method == PWP_WANDA ? n : 0, Wo_dev[k], mk_dev[k], ws, sti, true, s);
+      if (e == cudaSuccess) e = cudaEventRecord(ev_in_free[k], s);
+    } else {
+      // each chunk of X folded into H as soon as it lands
+      int ch = 0;
+      for (int64_t r0 = 0; r0 < n && ps == PWP_OK; r0 += rows, ++ch) {
+        const int64_t nr = n - r0 < rows ? n - r0 : rows;
+        e = cudaStreamWaitEvent(s, ev_chunk[ch], 0);
+        if (e != cudaSuccess) {
+          ps = PWP_ECUDA;
+          break;
+        }
+        ps = hessian_impl((const char*)X_dev[k] + (size_t)r0 * xrow, xtype, nr, b, H_dev, r0 > 0 ? 1 : 0, sti, s);
+      }
+      if (ps != PWP_OK) break;
+      if (n == 0) e = cudaMemsetAsync(H_dev, 0, (size_t)b * b * sizeof(float), s);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_w, 0);
+      const HostOut ho{W_out_host[i], mask_out_host[i], cout, ev_blk};
+      const bool blockwise = cfg->alpha == 0.f;
+      if (e == cudaSuccess)
+        e = launch_prune_out(cfg, W_dev[k], wtype, c, b, H_dev, Wo_dev[k], mk_dev[k], ws, sti, s, true,
+                             blockwise ? &ho : nullptr);
+      if (e == cudaSuccess) e = cudaEventRecord(ev_in_free[k], s);
+      if (e == cudaSuccess && !blockwise) {
+        // outlier rows: the whole result once the prune is done
+        e = cudaStreamWaitEvent(cout, ev_in_free[k], 0);
+        if (e == cudaSuccess)
+          e = cudaMemcpyAsync(W_out_host[i], Wo_dev[k], (size_t)c * b * sizeof(float), cudaMemcpyDeviceToHost, cout);
+        if (e == cudaSuccess)
+          e = cudaMemcpyAsync(mask_out_host[i], mk_dev[k], (size_t)c * b, cudaMemcpyDeviceToHost, cout);
+      }
+    }
+    if (e == cudaSuccess && no_update) {
+      e = cudaStreamWaitEvent(cout, ev_in_free[k], 0);
+      if (e == cudaSuccess)
+        e = cudaMemcpyAsync(W_out_host[i], Wo_dev[k], (size_t)c * b * sizeof(float), cudaMemcpyDeviceToHost, cout);
+      if (e == cudaSuccess) e = cudaMemcpyAsync(mask_out_host[i], mk_dev[k], (size_t)c * b, cudaMemcpyDeviceToHost, cout);
+    }
+    if (e == cudaSuccess) e = cudaEventRecord(ev_out_done[k], cout);
+    if (e != cudaSuccess) ps = PWP_ECUDA;
+  }
+  // `stream` waits for the last copies either way
+  if (cudaEventRecord(ev_start, cout) == cudaSuccess) cudaStreamWaitEvent(s, ev_start, 0);
+  if (cudaEventRecord(ev_w, cin) == cudaSuccess) cudaStreamWaitEvent(s, ev_w, 0);
+  for (cudaEvent_t ev : {ev_start, ev_w, ev_blk, ev_in_free[0], ev_in_free[1], ev_out_done[0], ev_out_done[1]})
+    if (ev) cudaEventDestroy(ev);
+  for (cudaEvent_t ev : ev_chunk)
+    if (ev) cudaEventDestroy(ev);
+  if (cin) cudaStreamDestroy(cin);
+  if (cout) cudaStreamDestroy(cout);
+  return ps;
+}
+
 pwp_status pwp_pack_24(const float* W_hat, const uint8_t* mask, int32_t c, int32_t b, uint16_t* values,
                        uint32_t* meta, pwp_stats* st, void* stream) {
   if (!W_hat || !mask || !values || !meta || !st || c < 1 || b < 4 || b > 16384 || (b % 4) != 0 ||

@@ -83,6 +83,17 @@ def test_argument_errors_return_before_any_launch():
                                   None) == 1
     assert L.pwp_prune_layer_host(ctypes.byref(cfg), fake, 0, 16, 16, fake, 0, 10, *a[:7], fake, 10, fake,
                                   None) == 3
+    # the multi-layer host entry point: null arrays, a negative count, then short device scratch
+    arr = (vp * 2)(fake, fake)
+    nb = L.pwp_layers_host_bytes(ctypes.byref(cfg), 16, 16, 10, 0, 0)
+    assert nb > 0 and nb % 256 == 0
+    assert L.pwp_prune_layers_host(ctypes.byref(cfg), 2, None, 0, 16, 16, arr, 0, 10, arr, arr, fake, nb, fake,
+                                   None) == 1
+    assert L.pwp_prune_layers_host(ctypes.byref(cfg), -1, arr, 0, 16, 16, arr, 0, 10, arr, arr, fake, nb, fake,
+                                   None) == 1
+    assert L.pwp_prune_layers_host(ctypes.byref(cfg), 2, arr, 0, 16, 16, arr, 0, 10, arr, arr, fake, nb - 256, fake,
+                                   None) == 3
+    assert L.pwp_layers_host_bytes(ctypes.byref(cfg), 16, 16, -1, 0, 0) == 0
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

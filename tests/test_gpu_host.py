@@ -85,3 +85,38 @@ def test_host_entry_rejects_pageable_buffers():
     X = torch.zeros(4, 16).pin_memory()
     with pytest.raises(ValueError):
         pwp.prune_layer_host(W, X)
+
+
+@pytest.mark.parametrize("kw", [dict(method="thanos"), dict(method="sparsegpt", pattern="nm", nm=(2, 4)),
+                                dict(method="wanda"), dict(method="thanos", alpha=0.1, block=64)])
+def test_layers_entry_equals_one_layer_calls(kw):
+    """pwp_prune_layers_host (double-buffered transfers across layers) gives every layer
+    what pwp_prune_layer_host gives it alone, bit for bit."""
+    torch = _torch()
+    import post_weight_pruning_b200 as pwp
+    Ws, Xs = [], []
+    for seed in range(3):
+        wl = synth.custom(128, 256, 9000, dtype="bf16", sparsity=0.5, seed=40 + seed)
+        W, X = synth.make_W(wl), synth.make_X_tokens(wl)
+        Wd, Xd = P.torch_inputs(W, X, "bf16")
+        Ws.append(_pinned(Wd))
+        Xs.append(_pinned(Xd))
+    W_l, m_l, st_l = pwp.prune_layers_host(Ws, Xs, **kw)
+    torch.cuda.synchronize()
+    recs = pwp.read_stats_list(st_l)
+    for i in range(3):
+        W_1, m_1, st_1 = pwp.prune_layer_host(Ws[i], Xs[i], **kw)
+        torch.cuda.synchronize()
+        s1 = pwp.read_stats(st_1)
+        assert recs[i].status == 0 and recs[i].pruned == recs[i].target == s1.target
+        assert torch.equal(m_l[i], m_1)
+        assert torch.equal(W_l[i], W_1)
+
+
+def test_layers_entry_rejects_mixed_shapes():
+    torch = _torch()
+    import post_weight_pruning_b200 as pwp
+    W = [torch.zeros(8, 16).pin_memory(), torch.zeros(8, 32).pin_memory()]
+    X = [torch.zeros(4, 16).pin_memory(), torch.zeros(4, 32).pin_memory()]
+    with pytest.raises(ValueError):
+        pwp.prune_layers_host(W, X)
