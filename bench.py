@@ -467,7 +467,7 @@ def run_mine(args):
     # the layers of a model one after another through the multi-layer host entry point: each
     # step's inputs go host -> device and its results device -> host inside the timed region,
     # overlapping the neighbouring steps' work
-    e2e_steps = max(2, min(args.steps, 5))
+    e2e_steps = max(2, min(args.steps, 10))   # as many layers as the timed device steps, at most 10
     out_Ws = [torch.empty((c, b), dtype=torch.float32).pin_memory() for _ in range(e2e_steps)]
     out_ms = [torch.empty((c, b), dtype=torch.uint8).pin_memory() for _ in range(e2e_steps)]
     pwp.prune_layers_host([W_host] * 2, [X_host] * 2, out_Ws=out_Ws[:2], out_masks=out_ms[:2], device=dev,

@@ -98,7 +98,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned int* h2 = l2.pred;
   unsigned int* h2s = l2.pred_sum;
   __shared__ pick::Shared psh;
-  pdl_enter();
+  // the set-up below touches only this CTA's shared and tensor memory, so it runs before the
+  // wait for the previous kernel (no kernel that can share an SM with this one holds tensor
+  // memory: this one's shared memory leaves no room for another tensor-core CTA)
+  pdl_release();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* wbuf = smem + W_OFF;
@@ -114,13 +117,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int abort_flag;
   volatile int* abortp = &abort_flag;
 
-  if (cta_failed(st)) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int mt = (c + TM - 1) / TM;
   const int ntiles = upper ? mt * (mt + 1) / 2 : mt * ((b - u0 + TN - 1) / TN);
   const int nkc = (Bp + TK - 1) / TK;
-  // level-1 bin of the previous block's threshold: its level-2 histogram is built here
-  const unsigned int pred = (SCORE != kNoScore && ctl->b1_valid) ? ctl->b1 : 0xffffffffu;
 
   if (SCORE != kNoScore)
     for (int i = tid; i < kHist1Bins; i += kThreads) shist[i] = 0u;
@@ -146,6 +146,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   fence_after();
   const uint32_t tmem = tmem_slot;
+  pdl_wait();   // the previous kernel has completed and its writes are visible
+  if (cta_failed(st)) {
+    // leave as a whole CTA, the tensor memory given back
+    if (warp == kMmaWarp) tmem_free(tmem, kAccCols);
+    return;
+  }
+  // level-1 bin of the previous block's threshold: its level-2 histogram is built here
+  const unsigned int pred = (SCORE != kNoScore && ctl->b1_valid) ? ctl->b1 : 0xffffffffu;
 
   if (warp == kProducerWarp) {
     if (lane == 0) {
