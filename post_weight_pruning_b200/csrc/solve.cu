@@ -382,8 +382,11 @@ __global__ void __launch_bounds__(kSolveWarps * 32, 2) thanos_solve_kernel(const
   // First the rows of this warp's slice whose sets exceed the shared rows (the slow
   // general path starts at once, under the other warps' work); then every other row,
   // handed out one at a time, so that a warp held up by a large row takes fewer.
-  for (int k = slot; k < c; k += gridDim.x * nwarps)
-    if (count_selected(k) > kNS) solve_row(k, false);
+  // (N:M: every row selects B (m - n) / m entries, so when that fits the slab no row can be large)
+  const bool any_large = !NM || (long long)B * (nm_m - nm_n) / nm_m > kNS;
+  if (any_large)
+    for (int k = slot; k < c; k += gridDim.x * nwarps)
+      if (count_selected(k) > kNS) solve_row(k, false);
   for (;;) {
     unsigned int k = 0;
     if (lane == 0) k = atomicAdd(&ctlp->row_next, 1u);
