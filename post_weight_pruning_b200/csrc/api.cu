@@ -226,6 +226,8 @@ pwp_status pwp_prune_layer_host(const pwp_config* cfg, const void* W_host, int32
     if (e == cudaSuccess) e = cudaMemcpyAsync(mask_out_host, mask_dev, (size_t)c * b, cudaMemcpyDeviceToHost, s);
     if (e != cudaSuccess) ps = PWP_ECUDA;
   }
+  // `stream` waits for whatever the copy stream still has, on the error paths too
+  if (ev && cudaEventRecord(ev, cp) == cudaSuccess) cudaStreamWaitEvent(s, ev, 0);
   if (ev) cudaEventDestroy(ev);
   if (ev_w) cudaEventDestroy(ev_w);
   cudaStreamDestroy(cp);
