@@ -195,5 +195,11 @@ def prune_rows_global(W_local, H, c_total=None, *, method="thanos", group=None, 
         c_total = int(t.item())
     from . import Sweep
     sw = Sweep(W_local, H, c_total, world, rank, method=method, stream=stream, **kw)
-    global_sweep([sw], TorchComm(group) if world > 1 else LocalComm())
+    comm = TorchComm(group) if world > 1 else LocalComm()
+    if stream is None:
+        global_sweep([sw], comm)
+    else:
+        import torch
+        with torch.cuda.stream(stream):   # the exchanges are ordered with the steps on this stream
+            global_sweep([sw], comm)
     return sw.result()
