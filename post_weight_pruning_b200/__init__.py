@@ -12,6 +12,8 @@ Names mirror the C entry points: ``hessian_accumulate``, ``damp_factor``,
 from __future__ import annotations
 
 import ctypes
+import functools
+import inspect
 import os
 from dataclasses import dataclass
 
@@ -143,6 +145,31 @@ def _stream_ptr(stream=None):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _stream_ctx(stream):
+    return _torch().cuda.stream(stream)
+
+
+def _on_stream(fn):
+    """Run a binding call with the caller's stream, when one is given, as torch's current
+    stream: the device memory the call allocates then belongs to that stream (the caching
+    allocator hands it out again only in that stream's order, after the call's kernels),
+    and the call's own copies and host reads of results are ordered after its kernels."""
+    params = list(inspect.signature(fn).parameters.values())
+    # where a positional stream argument would sit (None: keyword-only)
+    pos = next((i for i, p in enumerate(params) if p.name == "stream" and p.kind == p.POSITIONAL_OR_KEYWORD), None)
+
+    @functools.wraps(fn)
+    def wrapped(*a, **kw):
+        stream = kw.get("stream")
+        if stream is None and pos is not None and len(a) > pos:
+            stream = a[pos]
+        if stream is None:
+            return fn(*a, **kw)
+        with _stream_ctx(stream):
+            return fn(*a, **kw)
+    return wrapped
+
+
 def _dtype_code(t):
     torch = _torch()
     if t.dtype == torch.bfloat16:
@@ -186,6 +213,7 @@ def read_stats(stats_t) -> Stats:
     return Stats.from_buffer_copy(raw)
 
 
+@_on_stream
 def hessian_accumulate(X, H=None, beta=0, stream=None):
     """H := beta*H + 2 X X^T for token-major X ([n, b], bf16 or fp32 CUDA tensor)."""
     torch = _torch()
@@ -203,6 +231,7 @@ def hessian_accumulate(X, H=None, beta=0, stream=None):
     return H
 
 
+@_on_stream
 def damp_factor(H, damp=0.01, stream=None):
     """In place: upper triangle of H becomes U with (H + lambda I)^-1 = U^T U.
     Returns (g_diag, stats tensor)."""
@@ -234,6 +263,7 @@ def make_workspace(cfg: Config, c, b, device="cuda") -> Workspace:
     return Workspace(torch.empty(n, dtype=torch.uint8, device=device), n)
 
 
+@_on_stream
 def prune_layer(W, *, H=None, X=None, sparsity=0.5, pattern="unstructured", nm=(2, 4), block=128,
                 damp=0.01, method="thanos", alpha=0.0, W_out=None, mask=None, workspace=None, stats=None,
                 stream=None, check=True):
@@ -300,6 +330,7 @@ def prune_layer(W, *, H=None, X=None, sparsity=0.5, pattern="unstructured", nm=(
     return W_out, mask, s
 
 
+@_on_stream
 def prune_block(weights, activations, feeds, *, stream=None, check=True, **cfg):
     """Prune the linear layers of one transformer block.  Thanos / SparseGPT: one H per
     distinct input, built once on the tensor cores and shared by every layer that reads
@@ -348,6 +379,7 @@ class Sweep:
     STEPS = {"setup": 0, "score": 1, "pick_bin": 2, "reread": 3, "pick_key": 4, "count_ties": 5, "cut_ties": 6,
              "solve": 7, "finish": 8}
 
+    @_on_stream
     def __init__(self, W_local, H, c_total, world=1, rank=0, *, method="thanos", sparsity=0.5, block=128,
                  damp=0.01, stream=None):
         torch = _torch()
@@ -391,12 +423,17 @@ class Sweep:
         """(W_hat fp32 [c, b], mask uint8 [c, b], Stats of this rank: pruned = its removals)."""
         if not check:
             return self.W_out, self.mask, self.stats
-        s = read_stats(self.stats)
+        if self.stream is None:
+            s = read_stats(self.stats)
+        else:
+            with _stream_ctx(self.stream):   # the read follows the steps on their stream
+                s = read_stats(self.stats)
         if s.status != 0:
             raise PwpError(s.status, "pwp_sweep_step (device)")
         return self.W_out, self.mask, s
 
 
+@_on_stream
 def pack_24(W_hat, mask, *, stream=None, check=True):
     """Compressed 2:4 storage of a pruned layer (pwp_pack_24).  W_hat: fp32 [c, b] and
     mask: uint8 [c, b] CUDA tensors with exactly two kept entries in every aligned group
@@ -423,6 +460,7 @@ def pack_24(W_hat, mask, *, stream=None, check=True):
     return values, meta, s
 
 
+@_on_stream
 def prune_layer_host(W_host, X_host, *, out_W=None, out_mask=None, device="cuda", stream=None, **kw):
     """End-to-end call from host memory (pwp_prune_layer_host): W ([c, b]) and X ([n, b]),
     bf16/fp32 pinned torch CPU tensors, go to the device on a copy stream of the call's own
@@ -471,6 +509,7 @@ def prune_layer_host(W_host, X_host, *, out_W=None, out_mask=None, device="cuda"
     return out_W, out_mask, stats
 
 
+@_on_stream
 def prune_layers_host(Ws_host, Xs_host, *, out_Ws=None, out_masks=None, device="cuda", stream=None, **kw):
     """A sequence of same-shaped layers from pinned host memory (pwp_prune_layers_host):
     layer i+1's transfers overlap layer i's work and layer i's results come back while
@@ -516,8 +555,6 @@ def prune_layers_host(Ws_host, Xs_host, *, out_Ws=None, out_masks=None, device="
     st = L.pwp_prune_layers_host(ctypes.byref(cfg), nl, Wp, wt, int(c), int(b), Xp, xt, int(n), Op, Mp,
                                  _vp(dev.data_ptr()), nbytes, _vp(stats.data_ptr()), _stream_ptr(stream))
     _check(st, "pwp_prune_layers_host")
-    # the device scratch lives until the stream has passed the call
-    dev.record_stream(torch.cuda.current_stream() if stream is None else stream)
     return out_Ws, out_masks, stats
 
 

@@ -192,3 +192,50 @@ def test_prune_block_checks_its_wiring(fake):
         pwp.prune_block({"q": torch.zeros(4, 16)}, {"attn_in": torch.zeros(8, 16)}, {})
     with pytest.raises(ValueError, match="does not match"):
         pwp.prune_block({"q": torch.zeros(4, 16)}, {"a": torch.zeros(8, 12)}, {"q": "a"})
+
+
+class _StreamCtx:
+    """Stands in for torch.cuda.stream(s): records which stream is current."""
+    current = []
+
+    def __init__(self, s):
+        self.s = s
+
+    def __enter__(self):
+        _StreamCtx.current.append(self.s)
+
+    def __exit__(self, *exc):
+        _StreamCtx.current.pop()
+
+
+@pytest.fixture
+def fake_streams(fake, monkeypatch):
+    """The fake library, each entry point also noting the current stream at its call."""
+    monkeypatch.setattr(pwp, "_stream_ctx", _StreamCtx)
+    seen = []
+    for name in ("pwp_prune_layer", "pwp_prune_layer_x", "pwp_pack_24", "pwp_hessian_accumulate"):
+        inner = getattr(fake, name)
+
+        def f(*a, _inner=inner, _name=name):
+            seen.append((_name, _StreamCtx.current[-1] if _StreamCtx.current else None))
+            return _inner(*a)
+        monkeypatch.setattr(fake, name, f)
+    return seen
+
+
+def test_calls_given_a_stream_run_with_it_current(fake_streams):
+    """With a caller's stream, the call's allocations, copies and host reads happen with that
+    stream current (positional or keyword); without one, nothing changes torch's stream."""
+    s = object()
+    W = torch.zeros(4, 16)
+    X = torch.zeros(8, 16, dtype=torch.bfloat16)
+    pwp.prune_layer(W, X=X, stream=s)
+    pwp.hessian_accumulate(X, None, 0, s)
+    pwp.pack_24(torch.zeros(2, 8), torch.zeros(2, 8, dtype=torch.uint8), stream=s)
+    pwp.prune_block({"q": W}, {"a": X}, {"q": "a"}, stream=s, method="thanos")
+    assert [x[1] for x in fake_streams] == [s] * len(fake_streams) and len(fake_streams) == 5
+    fake_streams.clear()
+    pwp.prune_layer(W, X=X)
+    pwp.hessian_accumulate(X)
+    assert [x[1] for x in fake_streams] == [None, None]
+    assert not _StreamCtx.current
