@@ -19,8 +19,13 @@
  *   - All pointers named *_dev are device pointers; the caller owns every buffer.
  *     The library allocates no device memory: all scratch comes from the caller's
  *     workspace `ws` of `ws_bytes` bytes (at least 256-byte aligned), or, for
- *     pwp_prune_layer_noalloc, from one static array inside the library.  Only the
- *     optional event timing (pwp_profile_enable) creates CUDA events.
+ *     pwp_prune_layer_noalloc, from one static array inside the library.  A call may
+ *     create CUDA streams and events of its own and release them before it returns:
+ *     the factor puts its next diagonal block on a side stream (three events; not
+ *     while `stream` is being captured into a graph), the host entry points put their
+ *     copies on copy streams; `stream` waits for all of that work, so it stays ordered
+ *     as if it had been enqueued on `stream` itself.  The optional event timing
+ *     (pwp_profile_enable) keeps its events until it is switched off.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream)
  *     and the call returns without synchronising.
  *   - Argument errors are detected on the host before anything is enqueued and
