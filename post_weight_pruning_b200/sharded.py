@@ -26,6 +26,7 @@ Without an initialised process group every function acts as a single rank.
 from __future__ import annotations
 
 from . import MAGNITUDE, METHODS, NM, WANDA, hessian_accumulate, prune_layer
+from . import _stream_ctx
 
 __all__ = ["token_range", "row_range", "rows_independent", "allreduce_hessian", "hessian_sharded",
            "prune_rows", "gather_rows", "TorchComm", "LocalComm", "global_sweep", "prune_rows_global"]
@@ -84,8 +85,7 @@ def hessian_sharded(X_local, group=None, stream=None):
     H = hessian_accumulate(X_local, stream=stream)
     if stream is None:
         return allreduce_hessian(H, group)
-    import torch
-    with torch.cuda.stream(stream):            # the collective waits for the H build on this stream
+    with _stream_ctx(stream):                  # the collective waits for the H build on this stream
         return allreduce_hessian(H, group)
 
 
@@ -199,7 +199,6 @@ def prune_rows_global(W_local, H, c_total=None, *, method="thanos", group=None, 
     if stream is None:
         global_sweep([sw], comm)
     else:
-        import torch
-        with torch.cuda.stream(stream):   # the exchanges are ordered with the steps on this stream
+        with _stream_ctx(stream):   # the exchanges are ordered with the steps on this stream
             global_sweep([sw], comm)
     return sw.result()

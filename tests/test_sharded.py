@@ -294,3 +294,53 @@ def test_local_comm_emulates_ranks_in_one_process():
     want = oracle.prune_layer(W, H=H, sparsity=0.4, block=8)
     assert np.array_equal(np.concatenate([sw.mask for sw in sweeps]), want["mask"])
     assert np.allclose(np.concatenate([sw.W for sw in sweeps]), want["W"], rtol=1e-9, atol=1e-12)
+
+
+def test_global_budget_exchanges_run_on_the_callers_stream(monkeypatch):
+    """prune_rows_global given a stream: every step and every exchange between the steps
+    happens with that stream current (one rank, the in-process communicator)."""
+    import post_weight_pruning_b200 as pwp
+    from tests._sweep_standin import NumpySweep
+    current = []
+
+    class Ctx:
+        def __init__(self, s):
+            self.s = s
+
+        def __enter__(self):
+            current.append(self.s)
+
+        def __exit__(self, *exc):
+            current.pop()
+
+    seen = []
+
+    class Recording(NumpySweep):
+        def __init__(self, W_local, H, c_total, world, rank, *, method="thanos", stream=None, **kw):
+            super().__init__(W_local, H, c_total, world, rank, **kw)
+
+        def step(self, name, t=0):
+            seen.append(("step", current[-1] if current else None))
+            super().step(name, t)
+
+        def result(self):
+            return self.W, self.mask, None
+
+    orig_sum = sharded.LocalComm.sum
+
+    def rec_sum(self, tensors):
+        seen.append(("sum", current[-1] if current else None))
+        return orig_sum(self, tensors)
+
+    monkeypatch.setattr(sharded, "_stream_ctx", Ctx)
+    monkeypatch.setattr(pwp, "Sweep", Recording)
+    monkeypatch.setattr(sharded.LocalComm, "sum", rec_sum)
+    rng = np.random.default_rng(5)
+    W = rng.normal(0, 0.02, size=(6, 16))
+    H = oracle.hessian(rng.normal(size=(40, 16)))
+    s = object()
+    W_hat, mask, _ = sharded.prune_rows_global(W, H, 6, stream=s, sparsity=0.5, block=8)
+    assert seen and all(who is s for _, who in seen)
+    assert {kind for kind, _ in seen} == {"step", "sum"} and not current
+    want = oracle.prune_layer(W, H=H, sparsity=0.5, block=8)
+    assert np.array_equal(mask, want["mask"])
