@@ -223,6 +223,29 @@ def test_nm_ties_prune_lower_column_first():
     assert mask.astype(int).tolist() == [[1, 1, 0, 0, 0, 1, 0, 1]]
 
 
+@pytest.mark.parametrize("n,m", [(1, 4), (2, 4), (4, 8), (3, 8)])
+def test_nm_mask_by_exhaustive_subsets(n, m):
+    """Brute force over every removal set of size m - n in each group: exactly one set has
+    every removed (score, column) below every kept one, and nm_mask removes that set; the
+    reported gap is that of the boundary pair.  Small integer scores make ties common."""
+    rng = np.random.default_rng(100 + 10 * n + m)
+    S = rng.integers(0, 4, size=(5, 2 * m)).astype(float) + 1.0
+    mask, gaps = oracle.nm_mask(S, n, m)
+    for k in range(S.shape[0]):
+        for g in range(0, S.shape[1], m):
+            cols = range(g, g + m)
+            valid = []
+            for R in itertools.combinations(cols, m - n):
+                kept = [q for q in cols if q not in R]
+                if max((S[k, q], q) for q in R) < min((S[k, q], q) for q in kept):
+                    valid.append(set(R))
+            assert len(valid) == 1
+            assert {q for q in cols if mask[k, q]} == valid[0]
+            hi = min(S[k, q] for q in cols if q not in valid[0])
+            lo = max(S[k, q] for q in valid[0])
+            assert gaps[k, g // m] == pytest.approx((hi - lo) / abs(hi))
+
+
 def test_global_selection_tie_order():
     S = np.array([[1.0, 0.5, 1.0],
                   [1.0, 2.0, 1.0]])
@@ -382,6 +405,25 @@ def test_sparsegpt_uses_conditioned_diagonal():
     U = oracle.inverse_cholesky_upper(Hd)
     for q in range(8):
         assert U[q, q] ** 2 == pytest.approx(oracle.conditioned_diag(Hd, q), rel=1e-10)
+
+
+def test_obs_score_is_the_compensated_single_removal_loss():
+    """"Pruning LLMs with Thanos", "One deletion with compensation: the OBS view": removing
+    W_kq and letting the row's other weights compensate raises the loss by an amount
+    proportional to W_kq^2 / [H^-1]_qq.  Brute force: the best compensation is a least-squares
+    fit of W_kq X_q by the other feature rows; its residual is the loss.  With H = 2 X X^T
+    the score is exactly twice that loss, for every weight (so it ranks them the same)."""
+    W, Xt = _rand_problem(91, c=3, b=7, n=30)
+    X = Xt.T                                             # b x n, features as rows
+    H = oracle.hessian(Xt)
+    S = oracle.obs_scores(W, np.diag(np.linalg.inv(H)))
+    for k in range(W.shape[0]):
+        for q in range(W.shape[1]):
+            rest = [t for t in range(W.shape[1]) if t != q]
+            target = W[k, q] * X[q]
+            coef, *_ = np.linalg.lstsq(X[rest].T, target, rcond=None)
+            loss = float(np.sum((target - coef @ X[rest]) ** 2))
+            assert S[k, q] == pytest.approx(2.0 * loss, rel=1e-8)
 
 
 # ----------------------------------------------------------------------------- no-update baselines
