@@ -52,3 +52,28 @@ def test_threaded_and_subset_draws_match_the_serial_draw():
     assert np.array_equal(synth.make_X_tokens(wl, threads=4), X)
     cols = [0, 7, 64, 299]
     assert np.array_equal(synth.make_X_features(wl, cols), X[:, cols].T)
+
+
+def test_bf16_storage_rounds_fp64_once_to_nearest_even():
+    """Inputs are stored as bfloat16 rounded once from fp64 (no detour through fp32, whose
+    own rounding could move a value that sits just off a halfway point onto it)."""
+    rng = np.random.default_rng(7)
+    x = rng.normal(size=3000) * 10.0 ** rng.integers(-20, 20, size=3000)
+    # exact halfway points between neighbouring bfloat16 values (even and odd lower
+    # neighbour), and points one fp64 step either side of them
+    v = synth.bf16_bits_to_f64(np.arange(0x3F80, 0x3F80 + 64, dtype=np.uint16))
+    mid = 0.5 * (v[:-1] + v[1:])
+    x = np.concatenate([x, mid, -mid, np.nextafter(mid, np.inf), np.nextafter(mid, -np.inf)])
+    u = synth.f64_to_bf16_bits(x)
+    y = synth.bf16_bits_to_f64(u)
+    up = synth.bf16_bits_to_f64(u + np.uint16(1))       # the neighbours of y in magnitude
+    dn = synth.bf16_bits_to_f64(u - np.uint16(1))
+    d = np.abs(y - x)
+    assert np.all(d <= np.abs(up - x)) and np.all(d <= np.abs(dn - x))
+    tie = (d == np.abs(up - x)) | (d == np.abs(dn - x))
+    assert tie.sum() == 2 * len(mid)                     # only the exact halfway points tie
+    assert np.all((u[tie] & 1) == 0)                     # and they go to the even pattern
+    n = len(mid)
+    above, below = x[-2 * n:-n], x[-n:]
+    assert np.all(synth.bf16_bits_to_f64(synth.f64_to_bf16_bits(above)) == v[1:])
+    assert np.all(synth.bf16_bits_to_f64(synth.f64_to_bf16_bits(below)) == v[:-1])
